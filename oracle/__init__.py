@@ -1,0 +1,213 @@
+"""fp64 CPU oracle for attention with an additive bias (FlashBias, arXiv 2505.12044).
+
+TEST INFRASTRUCTURE ONLY: the test suite, the smoke check and the CPU-baseline
+leg of the benchmark are the only callers. The product path never imports this
+package, and this package imports nothing from the product.
+
+The arithmetic lives in ``fb_oracle.c`` (the definition of biased attention,
+the Sandwich and ALiBi biases and their exact factors). This module only
+marshals numpy arrays for it, plus the one step that is a library primitive:
+the truncated SVD of a static bias (FlashBias rebuttal, reply to Reviewer
+xU4x, Q6: SVD decomposition with a per-head rank), done with
+``numpy.linalg.svd``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+BIAS_NONE, BIAS_DENSE, BIAS_LOWRANK, BIAS_SANDWICH, BIAS_ALIBI = 0, 1, 2, 3, 4
+
+
+class _Bias(ctypes.Structure):
+    _fields_ = [
+        ("kind", ctypes.c_int),
+        ("dense", ctypes.c_void_p),
+        ("ld", ctypes.c_int64),
+        ("phi_q", ctypes.c_void_p),
+        ("phi_k", ctypes.c_void_p),
+        ("R", ctypes.c_int),
+        ("C", ctypes.c_int),
+        ("slope", ctypes.c_double),
+    ]
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        lib.fbo_attention_rows.argtypes = [ctypes.c_int64, ctypes.c_int, P, P, P,
+                                           ctypes.POINTER(_Bias), ctypes.c_double,
+                                           ctypes.c_int, P, ctypes.c_int64, P, P]
+        lib.fbo_attention_rows.restype = ctypes.c_int
+        lib.fbo_bias_dense.argtypes = [ctypes.c_int64, ctypes.POINTER(_Bias), P]
+        lib.fbo_bias_dense.restype = ctypes.c_int
+        lib.fbo_bias_value.argtypes = [ctypes.POINTER(_Bias), ctypes.c_int64, ctypes.c_int64]
+        lib.fbo_bias_value.restype = ctypes.c_double
+        lib.fbo_sandwich_factors.argtypes = [ctypes.c_int64, ctypes.c_int, P]
+        lib.fbo_sandwich_factors.restype = ctypes.c_int
+        lib.fbo_alibi_slope.argtypes = [ctypes.c_int, ctypes.c_int]
+        lib.fbo_alibi_slope.restype = ctypes.c_double
+        lib.fbo_alibi_factors.argtypes = [ctypes.c_int64, ctypes.c_double, P, P]
+        lib.fbo_alibi_factors.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+class HeadBias:
+    """The bias of one head, by kind. Keeps its arrays alive for the C call."""
+
+    def __init__(self, kind: int, dense=None, phi_q=None, phi_k=None, C: int = 0,
+                 slope: float = 0.0):
+        self.kind = kind
+        self._keep = []
+        self.s = _Bias()
+        self.s.kind = kind
+        if kind == BIAS_DENSE:
+            dense = _f64(dense)
+            self._keep.append(dense)
+            self.s.dense = dense.ctypes.data
+            self.s.ld = dense.shape[1]
+        elif kind == BIAS_LOWRANK:
+            phi_q, phi_k = _f64(phi_q), _f64(phi_k)
+            assert phi_q.shape[1] == phi_k.shape[1]
+            self._keep += [phi_q, phi_k]
+            self.s.phi_q = phi_q.ctypes.data
+            self.s.phi_k = phi_k.ctypes.data
+            self.s.R = phi_q.shape[1]
+        elif kind == BIAS_SANDWICH:
+            self.s.C = int(C)
+        elif kind == BIAS_ALIBI:
+            self.s.slope = float(slope)
+
+    @staticmethod
+    def none():
+        return HeadBias(BIAS_NONE)
+
+    @staticmethod
+    def dense(b):
+        return HeadBias(BIAS_DENSE, dense=b)
+
+    @staticmethod
+    def lowrank(phi_q, phi_k):
+        return HeadBias(BIAS_LOWRANK, phi_q=phi_q, phi_k=phi_k)
+
+    @staticmethod
+    def sandwich(C: int):
+        return HeadBias(BIAS_SANDWICH, C=C)
+
+    @staticmethod
+    def alibi(slope: float):
+        return HeadBias(BIAS_ALIBI, slope=slope)
+
+    def value(self, i: int, j: int) -> float:
+        return _load().fbo_bias_value(ctypes.byref(self.s), int(i), int(j))
+
+    def dense_matrix(self, N: int) -> np.ndarray:
+        out = np.empty((N, N), dtype=np.float64)
+        rc = _load().fbo_bias_dense(N, ctypes.byref(self.s), _ptr(out))
+        assert rc == 0
+        return out
+
+
+def attention_head(q, k, v, bias: HeadBias, scale: float, causal: bool, rows=None):
+    """One head: q, k, v [N, d]. Returns (o [len(rows), d], lse [len(rows)]) in fp64."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    N, d = q.shape
+    assert k.shape == (N, d) and v.shape == (N, d)
+    rows = np.arange(N, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    o = np.empty((rows.shape[0], d), dtype=np.float64)
+    lse = np.empty((rows.shape[0],), dtype=np.float64)
+    rc = _load().fbo_attention_rows(N, d, _ptr(q), _ptr(k), _ptr(v), ctypes.byref(bias.s),
+                                    float(scale), int(bool(causal)), _ptr(rows), rows.shape[0],
+                                    _ptr(o), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments")
+    return o, lse
+
+
+def attention(q, k, v, bias_of, scale: float, causal: bool, rows=None, heads=None):
+    """q, k, v [B, H, N, d]. ``bias_of(b, h)`` returns the HeadBias of head (b, h).
+
+    rows: optional query indices evaluated for every head (default: all).
+    heads: optional list of (b, h) pairs to evaluate (default: all).
+    Returns (o, lse) as dicts keyed by (b, h) when ``heads`` is given, else as
+    arrays [B, H, len(rows), d] and [B, H, len(rows)].
+    """
+    B, H, N, d = q.shape
+    pairs = heads if heads is not None else [(b, h) for b in range(B) for h in range(H)]
+    out_o, out_l = {}, {}
+    for (b, h) in pairs:
+        o, l = attention_head(q[b, h], k[b, h], v[b, h], bias_of(b, h), scale, causal, rows)
+        out_o[(b, h)], out_l[(b, h)] = o, l
+    if heads is not None:
+        return out_o, out_l
+    nr = N if rows is None else len(rows)
+    O = np.empty((B, H, nr, d))
+    L = np.empty((B, H, nr))
+    for (b, h) in pairs:
+        O[b, h], L[b, h] = out_o[(b, h)], out_l[(b, h)]
+    return O, L
+
+
+def sandwich_factors(N: int, C: int) -> np.ndarray:
+    """Exact Sandwich factors phi [N, C] (phi_q = phi_k = phi)."""
+    out = np.empty((N, C), dtype=np.float64)
+    assert _load().fbo_sandwich_factors(N, C, _ptr(out)) == 0
+    return out
+
+
+def alibi_slope(h: int, H: int) -> float:
+    return _load().fbo_alibi_slope(h, H)
+
+
+def alibi_factors(N: int, slope: float):
+    """Exact rank-2 ALiBi factors (phi_q [N, 2], phi_k [N, 2]) of one head."""
+    pq = np.empty((N, 2), dtype=np.float64)
+    pk = np.empty((N, 2), dtype=np.float64)
+    assert _load().fbo_alibi_factors(N, float(slope), _ptr(pq), _ptr(pk)) == 0
+    return pq, pk
+
+
+def truncated_svd_factors(bias, R: int):
+    """Rank-R truncation of one head's bias by SVD, split evenly between the sides.
+
+    phi_q = U_R sqrt(S_R), phi_k = V_R sqrt(S_R), so phi_q phi_k^T is the best
+    rank-R approximation (Eckart-Young). Returns (phi_q, phi_k, rel_fro_err,
+    energy) with rel_fro_err = ||B - phi_q phi_k^T||_F / ||B||_F and energy =
+    sum_{r<R} s_r^2 / sum_r s_r^2 (the "95% energy" criterion of the rebuttal,
+    reply to Reviewer Bp2x, Q2 (2), is reported, not enforced).
+    """
+    Bm = _f64(bias)
+    U, S, Vt = np.linalg.svd(Bm, full_matrices=False)
+    root = np.sqrt(S[:R])
+    phi_q = U[:, :R] * root[None, :]
+    phi_k = Vt[:R, :].T * root[None, :]
+    approx = phi_q @ phi_k.T
+    nrm = np.linalg.norm(Bm)
+    rel = float(np.linalg.norm(Bm - approx) / nrm) if nrm > 0 else 0.0
+    tot = float(np.sum(S * S))
+    energy = float(np.sum(S[:R] ** 2) / tot) if tot > 0 else 1.0
+    return phi_q, phi_k, rel, energy
+
+
+def lowrank_dense(phi_q, phi_k) -> np.ndarray:
+    """phi_q phi_k^T in fp64 (the dense bias a set of factors stands for)."""
+    return _f64(phi_q) @ _f64(phi_k).T

@@ -1,0 +1,263 @@
+"""Pins for the fp64 oracle: each check compares it with something other than itself.
+
+- a library attention routine (torch SDPA, fp64 CPU) and torch.logsumexp;
+- a 50-digit mpmath evaluation on tiny inputs;
+- invariants of the definition (row-constant bias, zero bias, rows of P sum to
+  one, key permutation, saturating scores, the first causal row);
+- the closed-form identities the pages state (Sandwich bias = product of its
+  exact factors; ALiBi = product of its rank-2 factors) and golden constants;
+- the truncated SVD against matrices with known singular values.
+"""
+import json
+import math
+import os
+
+import mpmath
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import HeadBias
+import seeded_inputs as si
+
+GOLDEN = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "closed_forms.json")))
+
+
+def _rand(shape, seed, std=1.0):
+    return np.random.Generator(np.random.PCG64(seed)).standard_normal(shape) * std
+
+
+def _sdpa(q, k, v, bias, scale, causal):
+    """Library attention with an additive float mask (fp64, CPU)."""
+    Q, K, V = (torch.from_numpy(np.ascontiguousarray(x))[None, None] for x in (q, k, v))
+    mask = torch.from_numpy(np.ascontiguousarray(bias)).clone()
+    if causal:
+        N = q.shape[0]
+        mask = mask.masked_fill(torch.triu(torch.ones(N, N, dtype=torch.bool), 1), float("-inf"))
+    o = torch.nn.functional.scaled_dot_product_attention(Q, K, V, attn_mask=mask[None, None], scale=scale)
+    scores = scale * (torch.from_numpy(q) @ torch.from_numpy(k).T) + mask
+    lse = torch.logsumexp(scores, dim=-1)
+    return o[0, 0].numpy(), lse.numpy()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N,d", [(1, 4), (37, 8), (64, 16), (130, 24)])
+def test_dense_bias_matches_library_attention(N, d, causal):
+    q, k, v = (_rand((N, d), s) for s in (1, 2, 3))
+    bias = _rand((N, N), 4, 2.0)  # asymmetric: a transposed bias would not match
+    scale = 1.0 / math.sqrt(d)
+    o, lse = oracle.attention_head(q, k, v, HeadBias.dense(bias), scale, causal)
+    o_ref, lse_ref = _sdpa(q, k, v, bias, scale, causal)
+    np.testing.assert_allclose(o, o_ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, lse_ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_lowrank_bias_matches_library_matmul(causal):
+    N, d, R = 50, 8, 5
+    q, k, v = (_rand((N, d), s) for s in (5, 6, 7))
+    pq, pk = _rand((N, R), 8, 0.7), _rand((N, R), 9, 0.7)
+    scale = 0.3
+    o, lse = oracle.attention_head(q, k, v, HeadBias.lowrank(pq, pk), scale, causal)
+    o_ref, lse_ref = _sdpa(q, k, v, torch.from_numpy(pq) @ torch.from_numpy(pk).T, scale, causal)
+    np.testing.assert_allclose(o, o_ref, atol=1e-12)
+    np.testing.assert_allclose(lse, lse_ref, atol=1e-12)
+    # the LOWRANK definition element by element against a library matmul
+    dense = HeadBias.lowrank(pq, pk).dense_matrix(N)
+    np.testing.assert_allclose(dense, pq @ pk.T, atol=1e-13)
+
+
+def test_zero_bias_is_plain_attention():
+    N, d = 40, 16
+    q, k, v = (_rand((N, d), s) for s in (11, 12, 13))
+    for causal in (False, True):
+        o0, l0 = oracle.attention_head(q, k, v, HeadBias.none(), 0.25, causal)
+        Q, K, V = (torch.from_numpy(x)[None, None] for x in (q, k, v))
+        o_ref = torch.nn.functional.scaled_dot_product_attention(Q, K, V, is_causal=causal, scale=0.25)[0, 0]
+        np.testing.assert_allclose(o0, o_ref.numpy(), atol=1e-12)
+        od, ld = oracle.attention_head(q, k, v, HeadBias.dense(np.zeros((N, N))), 0.25, causal)
+        np.testing.assert_array_equal(o0, od)
+        np.testing.assert_array_equal(l0, ld)
+
+
+def _mp_attention_row(q, k, v, bias, scale, i, causal):
+    jmax = i + 1 if causal else k.shape[0]
+    s = [mpmath.mpf(scale) * mpmath.fsum(mpmath.mpf(q[i, c]) * mpmath.mpf(k[j, c]) for c in range(q.shape[1]))
+         + mpmath.mpf(bias[i, j]) for j in range(jmax)]
+    e = [mpmath.exp(x) for x in s]
+    z = mpmath.fsum(e)
+    o = [mpmath.fsum(e[j] * mpmath.mpf(v[j, c]) for j in range(jmax)) / z for c in range(v.shape[1])]
+    return o, mpmath.log(z)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fifty_digit_bruteforce(causal):
+    mpmath.mp.dps = 50
+    N, d = 12, 4
+    q, k, v = (_rand((N, d), s) for s in (21, 22, 23))
+    bias = _rand((N, N), 24, 3.0)
+    o, lse = oracle.attention_head(q, k, v, HeadBias.dense(bias), 0.7, causal)
+    for i in range(N):
+        o_mp, l_mp = _mp_attention_row(q, k, v, bias, 0.7, i, causal)
+        for c in range(d):
+            assert abs(o[i, c] - float(o_mp[c])) < 1e-13
+        assert abs(lse[i] - float(l_mp)) < 1e-13 * max(1.0, abs(float(l_mp)))
+
+
+def test_row_constant_bias_leaves_output_and_shifts_lse():
+    N, d = 33, 8
+    q, k, v = (_rand((N, d), s) for s in (31, 32, 33))
+    c = _rand((N,), 34, 5.0)
+    for causal in (False, True):
+        o0, l0 = oracle.attention_head(q, k, v, HeadBias.none(), 0.5, causal)
+        o1, l1 = oracle.attention_head(q, k, v, HeadBias.dense(np.repeat(c[:, None], N, 1)), 0.5, causal)
+        np.testing.assert_allclose(o1, o0, atol=1e-14)
+        np.testing.assert_allclose(l1 - l0, c, atol=1e-12)
+
+
+def test_rows_of_p_sum_to_one_and_first_causal_row():
+    N, d = 29, 6
+    q, k = _rand((N, d), 41), _rand((N, d), 42)
+    v = np.ones((N, d))
+    bias = _rand((N, N), 43, 4.0)
+    o, _ = oracle.attention_head(q, k, v, HeadBias.dense(bias), 1.0, False)
+    np.testing.assert_allclose(o, 1.0, atol=1e-14 * N)
+    v = _rand((N, d), 44)
+    o, lse = oracle.attention_head(q, k, v, HeadBias.dense(bias), 1.0, True)
+    np.testing.assert_array_equal(o[0], v[0])  # causal row 0 sees key 0 only
+    assert abs(lse[0] - (q[0] @ k[0] + bias[0, 0])) < 1e-14
+
+
+def test_key_permutation_equivariance():
+    N, d = 31, 8
+    q, k, v = (_rand((N, d), s) for s in (51, 52, 53))
+    bias = _rand((N, N), 54)
+    perm = np.random.Generator(np.random.PCG64(55)).permutation(N)
+    o, l = oracle.attention_head(q, k, v, HeadBias.dense(bias), 0.4, False)
+    op, lp = oracle.attention_head(q, k[perm], v[perm], HeadBias.dense(bias[:, perm]), 0.4, False)
+    np.testing.assert_allclose(op, o, atol=1e-13)
+    np.testing.assert_allclose(lp, l, atol=1e-13)
+
+
+def test_saturating_scores_pick_one_key():
+    N, d = 20, 4
+    q, k, v = (_rand((N, d), s) for s in (61, 62, 63))
+    bias = np.zeros((N, N))
+    bias[:, 7] = 1.0e4  # exp would overflow without the max shift
+    o, lse = oracle.attention_head(q, k, v, HeadBias.dense(bias), 1.0, False)
+    np.testing.assert_allclose(o, np.repeat(v[7:8], N, 0), atol=1e-300)
+    np.testing.assert_allclose(lse, q @ k[7] + 1.0e4, rtol=1e-15)
+
+
+# --- Sandwich ---------------------------------------------------------------
+
+def test_sandwich_identity_bias_equals_factor_product():
+    """The pages state b = phi_q phi_k^T for the exact Sandwich factors."""
+    C, N = 64, 2048
+    phi = oracle.sandwich_factors(N, C)
+    bias = HeadBias.sandwich(C)
+    rng = np.random.Generator(np.random.PCG64(70))
+    pairs = [(0, 0), (N - 1, 0), (0, N - 1), (N - 1, N - 1)] + [tuple(x) for x in rng.integers(0, N, (300, 2))]
+    for i, j in pairs:
+        assert abs(bias.value(i, j) - float(phi[i] @ phi[j])) < 1e-11
+    # whole small block through the dense builder as well
+    Bd = HeadBias.sandwich(16).dense_matrix(300)
+    f16 = oracle.sandwich_factors(300, 16)
+    np.testing.assert_allclose(Bd, f16 @ f16.T, atol=1e-12)
+
+
+def test_sandwich_golden_values():
+    g = GOLDEN
+    b = HeadBias.sandwich(g["sandwich_diagonal"]["C"])
+    for i in (0, 5, 4095):
+        assert b.value(i, i) == g["sandwich_diagonal"]["value"]
+    for delta, val in g["sandwich_delta"]["points"]:
+        assert abs(b.value(delta + 3, 3) - val) < 1e-12
+        assert abs(b.value(3, delta + 3) - val) < 1e-12  # even in i - j
+    phi = oracle.sandwich_factors(2, 64)
+    assert abs(math.acos(phi[1, 0]) - g["sandwich_w1"]["value"]) < 1e-14
+    assert abs(math.atan2(phi[1, 63], phi[1, 62]) - g["sandwich_w_last"]["value"]) < 1e-16
+    np.testing.assert_array_equal(oracle.sandwich_factors(1, 8)[0], g["sandwich_phi_at_zero"]["value"])
+
+
+# --- ALiBi ------------------------------------------------------------------
+
+def test_alibi_slopes_golden():
+    for key in ("alibi_slopes_H8", "alibi_slopes_H16"):
+        H = GOLDEN[key]["H"]
+        got = [oracle.alibi_slope(h, H) for h in range(H)]
+        np.testing.assert_allclose(got, GOLDEN[key]["value"], rtol=1e-15)
+
+
+def test_alibi_factor_product_is_distance_bias():
+    N = 8192
+    for h, H in ((0, 16), (7, 16), (15, 16), (3, 8)):
+        m = oracle.alibi_slope(h, H)
+        pq, pk = oracle.alibi_factors(N, m)
+        bias = HeadBias.alibi(m)
+        rng = np.random.Generator(np.random.PCG64(80 + h))
+        for i, j in [(0, 0), (N - 1, 0), (N - 1, N - 1), (5, 9)] + [tuple(x) for x in rng.integers(0, N, (200, 2))]:
+            want = -m * (i - j)
+            assert abs(float(pq[i] @ pk[j]) - want) <= 1e-9 * max(1.0, abs(want))
+            assert bias.value(i, j) == want
+
+
+def test_multiplicative_example_rank2():
+    """cos(i-j) = [cos i, sin i].[cos j, sin j] (the pages' rank-2 example)."""
+    n = np.arange(64, dtype=np.float64)
+    f = np.stack([np.cos(n), np.sin(n)], 1)
+    np.testing.assert_allclose(f @ f.T, np.cos(n[:, None] - n[None, :]), atol=1e-13)
+    assert np.linalg.matrix_rank(np.cos(n[:, None] - n[None, :])) == GOLDEN["multiplicative_cos_rank2"]["R"]
+
+
+# --- truncated SVD ----------------------------------------------------------
+
+def _known_spectrum(N, sigma, seed):
+    rng = np.random.Generator(np.random.PCG64(seed))
+    U, _ = np.linalg.qr(rng.standard_normal((N, len(sigma))))
+    V, _ = np.linalg.qr(rng.standard_normal((N, len(sigma))))
+    return U @ np.diag(sigma) @ V.T
+
+
+def test_svd_truncation_against_known_spectrum():
+    sigma = np.array([50.0, 20.0, 9.0, 4.0, 2.0, 1.0, 0.5, 0.25])
+    Bm = _known_spectrum(200, sigma, 90)
+    for R in (1, 3, 8):
+        pq, pk, rel, energy = oracle.truncated_svd_factors(Bm, R)
+        want_rel = math.sqrt(np.sum(sigma[R:] ** 2) / np.sum(sigma ** 2))
+        want_energy = np.sum(sigma[:R] ** 2) / np.sum(sigma ** 2)
+        assert abs(rel - want_rel) < 1e-12
+        assert abs(energy - want_energy) < 1e-12
+        # balanced split: phi_q^T phi_q = phi_k^T phi_k = diag(sigma_R)
+        np.testing.assert_allclose(pq.T @ pq, np.diag(sigma[:R]), atol=1e-10)
+        np.testing.assert_allclose(pk.T @ pk, np.diag(sigma[:R]), atol=1e-10)
+    pq, pk, rel, _ = oracle.truncated_svd_factors(Bm, 8)
+    np.testing.assert_allclose(pq @ pk.T, Bm, atol=1e-11)
+    assert rel < 1e-12
+
+
+# --- seeded inputs (the workload definitions both sides receive) ------------
+
+def test_rbf_field_rank_and_gather():
+    grid, M = 12, 6
+    om, ph = si.rbf_params(2, M)
+    tab = si.rbf_offset_table(om, ph, grid)
+    dense = si.rbf_dense(tab, grid)
+    assert dense.shape == (2, grid * grid, grid * grid)
+    for h in range(2):
+        assert np.linalg.matrix_rank(dense[h], tol=1e-9 * np.abs(dense[h]).max()) <= 2 * M
+        for (i, j) in [(0, 0), (5, 77), (143, 3)]:
+            dx = i % grid - j % grid
+            dy = i // grid - j // grid
+            want = math.sqrt(2.0 / M) * sum(math.cos(om[h, m, 0] * dx + om[h, m, 1] * dy + ph[h, m]) for m in range(M))
+            assert abs(dense[h, i, j] - want) < 1e-12
+
+
+def test_bf16_rounding_is_round_to_nearest_even():
+    x = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -2.5, 1e-3, 65504.0], dtype=np.float32)
+    r = si.round_to_bf16(x)
+    t = torch.from_numpy(x).to(torch.bfloat16).to(torch.float32).numpy()
+    np.testing.assert_array_equal(r, t)
+    y = si.normal((4096,), 5)
+    np.testing.assert_array_equal(si.round_to_bf16(y), torch.from_numpy(y).to(torch.bfloat16).float().numpy())
