@@ -1,0 +1,254 @@
+"""attention_rank_additive_b200 -- attention with a low-rank additive bias on B200.
+
+Python binding of libflashbias (the C ABI in include/flashbias.h). The
+functions named ``fb_*`` mirror the C entry points one to one and take raw
+integers for pointers; the helpers below them (``attn``, ``attn_dense_bias``,
+``factors_sandwich``, ``factors_alibi``, ``svd_factors``) only marshal torch
+tensors: every step of the computation runs in the library's kernels.
+
+There is no fallback: importing works without a GPU, but the first call that
+needs the library raises if ``libflashbias.so`` has not been built
+(``python -m attention_rank_additive_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+__all__ = [
+    "FB_OK", "FB_ERR_INVALID_ARG", "FB_ERR_UNSUPPORTED", "FB_ERR_RANGE", "FB_ERR_WORKSPACE", "FB_ERR_CUDA",
+    "FB_ERR_TIMEOUT", "FB_F32", "FB_BF16", "FlashBiasError", "lib", "lib_path", "EXPORTED",
+    "fb_status_str", "fb_version", "fb_attn_workspace_bytes", "fb_attn_fwd", "fb_attn_dense_bias_fwd",
+    "fb_factors_sandwich", "fb_factors_alibi", "fb_svd_factors_host", "fb_check_device_error",
+    "fb_selftest_wait_timeout", "attn", "attn_dense_bias", "factors_sandwich", "factors_alibi", "svd_factors",
+    "attn_flops",
+]
+
+FB_OK, FB_ERR_INVALID_ARG, FB_ERR_UNSUPPORTED, FB_ERR_RANGE, FB_ERR_WORKSPACE, FB_ERR_CUDA, FB_ERR_TIMEOUT = range(7)
+FB_F32, FB_BF16 = 0, 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_HERE, "libflashbias.so")
+
+# Every symbol include/flashbias.h declares.
+EXPORTED = (
+    "fb_status_str", "fb_version", "fb_attn_workspace_bytes", "fb_attn_fwd", "fb_attn_dense_bias_fwd",
+    "fb_factors_sandwich", "fb_factors_alibi", "fb_svd_factors_host", "fb_check_device_error",
+    "fb_selftest_wait_timeout",
+)
+
+
+class FlashBiasError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {fb_status_str(status)} ({status})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libflashbias; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(lib_path):
+            raise RuntimeError(f"libflashbias.so is missing at {lib_path}; build it with "
+                               "`python -m attention_rank_additive_b200.build`")
+        L = ctypes.CDLL(lib_path)
+        i32, i64, sz, vp, f32 = ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_float
+        L.fb_status_str.argtypes, L.fb_status_str.restype = [i32], ctypes.c_char_p
+        L.fb_version.argtypes, L.fb_version.restype = [], i32
+        L.fb_attn_workspace_bytes.argtypes = [i32, i32, i32, i32, i64, i64]
+        L.fb_attn_workspace_bytes.restype = sz
+        L.fb_attn_fwd.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, i32, vp, vp, i64, i64, f32, i32, vp, vp, vp,
+                                  sz, vp]
+        L.fb_attn_fwd.restype = i32
+        L.fb_attn_dense_bias_fwd.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, i64, i64, f32, i32, vp, vp, vp]
+        L.fb_attn_dense_bias_fwd.restype = i32
+        L.fb_factors_sandwich.argtypes, L.fb_factors_sandwich.restype = [i32, i32, vp, vp, vp], i32
+        L.fb_factors_alibi.argtypes, L.fb_factors_alibi.restype = [i32, i32, vp, vp, vp], i32
+        L.fb_svd_factors_host.argtypes = [vp, i32, i32, i32, i32, ctypes.c_uint64, vp, vp, vp, vp]
+        L.fb_svd_factors_host.restype = i32
+        L.fb_check_device_error.argtypes, L.fb_check_device_error.restype = [vp], i32
+        L.fb_selftest_wait_timeout.argtypes, L.fb_selftest_wait_timeout.restype = [i32, vp], i32
+        _lib = L
+    return _lib
+
+
+# ---------------------------------------------------------------- raw C ABI
+
+def fb_status_str(status: int) -> str:
+    return lib().fb_status_str(int(status)).decode()
+
+
+def fb_version() -> int:
+    return lib().fb_version()
+
+
+def fb_attn_workspace_bytes(B, H, N, R, phi_bstride, phi_hstride) -> int:
+    return lib().fb_attn_workspace_bytes(B, H, N, R, phi_bstride, phi_hstride)
+
+
+def fb_attn_fwd(dt, B, H, N, d, Q, K, V, R, phi_q, phi_k, phi_bstride, phi_hstride, scale, causal, O, LSE,
+                workspace, workspace_bytes, stream) -> int:
+    return lib().fb_attn_fwd(dt, B, H, N, d, Q, K, V, R, phi_q, phi_k, phi_bstride, phi_hstride, scale, causal, O,
+                             LSE, workspace, workspace_bytes, stream)
+
+
+def fb_attn_dense_bias_fwd(dt, B, H, N, d, Q, K, V, Bias, bias_bstride, bias_hstride, scale, causal, O, LSE,
+                           stream) -> int:
+    return lib().fb_attn_dense_bias_fwd(dt, B, H, N, d, Q, K, V, Bias, bias_bstride, bias_hstride, scale, causal, O,
+                                        LSE, stream)
+
+
+def fb_factors_sandwich(N, C, phi_q, phi_k, stream) -> int:
+    return lib().fb_factors_sandwich(N, C, phi_q, phi_k, stream)
+
+
+def fb_factors_alibi(H, N, phi_q, phi_k, stream) -> int:
+    return lib().fb_factors_alibi(H, N, phi_q, phi_k, stream)
+
+
+def fb_svd_factors_host(bias_host, N, R, oversample, power_iters, seed, phi_q_host, phi_k_host, rel_fro_err,
+                        energy) -> int:
+    return lib().fb_svd_factors_host(bias_host, N, R, oversample, power_iters, seed, phi_q_host, phi_k_host,
+                                     rel_fro_err, energy)
+
+
+def fb_check_device_error(stream) -> int:
+    return lib().fb_check_device_error(stream)
+
+
+def fb_selftest_wait_timeout(limit_ms, stream) -> int:
+    return lib().fb_selftest_wait_timeout(limit_ms, stream)
+
+
+# ------------------------------------------------- torch-tensor marshalling
+
+def _check(status: int, where: str):
+    if status != FB_OK:
+        raise FlashBiasError(status, where)
+
+
+def _stream(device=None) -> int:
+    import torch
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return FB_BF16
+    if t.dtype == torch.float32:
+        return FB_F32
+    raise TypeError(f"unsupported dtype {t.dtype}; use bfloat16 or float32")
+
+
+def _factor_strides(phi, B, H, N, R):
+    """Element strides (b, h) of a factor tensor broadcastable to [B, H, N, R]."""
+    if phi.dim() == 2:  # [N, R]: shared by every head and batch
+        return 0, 0
+    if phi.dim() == 3:  # [H, N, R]: shared by the batch
+        return 0, (phi.stride(0) if phi.shape[0] == H and H > 1 else 0)
+    bs = phi.stride(0) if phi.shape[0] == B and B > 1 else 0
+    hs = phi.stride(1) if phi.shape[1] == H and H > 1 else 0
+    return bs, hs
+
+
+def attn(q, k, v, phi_q=None, phi_k=None, scale=None, causal=False, out=None, lse=None, workspace=None):
+    """O, LSE = softmax(scale q k^T + phi_q phi_k^T [+ causal]) v through fb_attn_fwd.
+
+    q, k, v: CUDA tensors [B, H, N, d] (bf16 or fp32, contiguous).
+    phi_q, phi_k: fp32 factors [N, R], [H, N, R] or [B, H, N, R] (last two dims
+    contiguous), or None for plain attention. Returns (O, LSE).
+    """
+    import torch
+    assert q.is_cuda and q.is_contiguous() and k.is_contiguous() and v.is_contiguous()
+    B, H, N, d = q.shape
+    dt = _dtype_code(q)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    R, bs, hs, pq, pk = 0, 0, 0, 0, 0
+    if phi_q is not None:
+        assert phi_q.dtype == torch.float32 and phi_k.dtype == torch.float32
+        assert phi_q.shape == phi_k.shape and phi_q.stride() == phi_k.stride()
+        assert phi_q.stride(-1) == 1 and phi_q.stride(-2) == phi_q.shape[-1]
+        R = phi_q.shape[-1]
+        bs, hs = _factor_strides(phi_q, B, H, N, R)
+        pq, pk = phi_q.data_ptr(), phi_k.data_ptr()
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if lse is None else lse
+    ws_bytes = fb_attn_workspace_bytes(B, H, N, R, bs, hs) if dt == FB_BF16 else 0
+    if ws_bytes and workspace is None:
+        workspace = torch.empty(ws_bytes, device=q.device, dtype=torch.uint8)
+    ws_ptr = workspace.data_ptr() if (workspace is not None and ws_bytes) else 0
+    _check(fb_attn_fwd(dt, B, H, N, d, q.data_ptr(), k.data_ptr(), v.data_ptr(), R, pq, pk, bs, hs, scale,
+                       int(bool(causal)), o.data_ptr(), l.data_ptr(), ws_ptr, ws_bytes, _stream(q.device)),
+           "fb_attn_fwd")
+    return o, l
+
+
+def attn_dense_bias(q, k, v, bias, scale=None, causal=False, out=None, lse=None):
+    """The dense-bias comparison path through fb_attn_dense_bias_fwd.
+
+    bias: [N, N], [H, N, N] or [B, H, N, N] tensor of q's dtype (last two dims
+    contiguous). Returns (O, LSE).
+    """
+    import torch
+    B, H, N, d = q.shape
+    dt = _dtype_code(q)
+    assert bias.dtype == q.dtype and bias.stride(-1) == 1 and bias.stride(-2) == N
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if bias.dim() == 2:
+        bs, hs = 0, 0
+    elif bias.dim() == 3:
+        bs, hs = 0, (bias.stride(0) if H > 1 else 0)
+    else:
+        bs = bias.stride(0) if (bias.shape[0] == B and B > 1) else 0
+        hs = bias.stride(1) if (bias.shape[1] == H and H > 1) else 0
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if lse is None else lse
+    _check(fb_attn_dense_bias_fwd(dt, B, H, N, d, q.data_ptr(), k.data_ptr(), v.data_ptr(), bias.data_ptr(), bs, hs,
+                                  scale, int(bool(causal)), o.data_ptr(), l.data_ptr(), _stream(q.device)),
+           "fb_attn_dense_bias_fwd")
+    return o, l
+
+
+def factors_sandwich(N: int, C: int, device="cuda"):
+    """Exact Sandwich factors phi [N, C] fp32 (phi_q = phi_k); one kernel."""
+    import torch
+    phi = torch.empty((N, C), device=device, dtype=torch.float32)
+    _check(fb_factors_sandwich(N, C, phi.data_ptr(), phi.data_ptr(), _stream(phi.device)), "fb_factors_sandwich")
+    return phi
+
+
+def factors_alibi(H: int, N: int, device="cuda"):
+    """Exact rank-2 ALiBi factors (phi_q, phi_k), each [H, N, 2] fp32; one kernel."""
+    import torch
+    pq = torch.empty((H, N, 2), device=device, dtype=torch.float32)
+    pk = torch.empty((H, N, 2), device=device, dtype=torch.float32)
+    _check(fb_factors_alibi(H, N, pq.data_ptr(), pk.data_ptr(), _stream(pq.device)), "fb_factors_alibi")
+    return pq, pk
+
+
+def svd_factors(bias, R: int, oversample: int = 16, power_iters: int = 2, seed: int = 0):
+    """Host truncated SVD of one head's bias (numpy float64 [N, N]).
+
+    Returns (phi_q [N, R] fp32, phi_k [N, R] fp32, rel_fro_err, energy) as numpy.
+    """
+    import numpy as np
+    b = np.ascontiguousarray(bias, dtype=np.float64)
+    N = b.shape[0]
+    assert b.shape == (N, N)
+    pq = np.empty((N, R), dtype=np.float32)
+    pk = np.empty((N, R), dtype=np.float32)
+    err, en = ctypes.c_double(), ctypes.c_double()
+    _check(fb_svd_factors_host(b.ctypes.data, N, R, oversample, power_iters, seed, pq.ctypes.data, pk.ctypes.data,
+                               ctypes.addressof(err), ctypes.addressof(en)), "fb_svd_factors_host")
+    return pq, pk, err.value, en.value
+
+
+def attn_flops(B: int, H: int, N: int, d: int, R: int, causal: bool) -> float:
+    """Counted FLOPs: 4 N^2 d + 2 N^2 R per head, halved when causal."""
+    f = float(B) * H * (4.0 * N * N * d + 2.0 * N * N * R)
+    return f / 2.0 if causal else f

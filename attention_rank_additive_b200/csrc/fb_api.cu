@@ -1,0 +1,360 @@
+// fb_api.cu -- the extern "C" entry points of libflashbias: argument
+// validation, the launch plan, TMA tensor maps and the launches. Every check
+// that can fail does so before anything is launched.
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "fb_internal.h"
+
+namespace fb {
+
+__device__ int g_device_flags;  // one word per device; see fb_check_device_error
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int *g_flag_ptr[kMaxDevices] = {nullptr};
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, []() {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int pad_dim(int d) { return d <= 16 ? 16 : (d <= 32 ? 32 : (d <= 64 ? 64 : 128)); }
+int pad_rank(int r) { return r <= 16 ? 16 : (r <= 32 ? 32 : (r <= 64 ? 64 : 128)); }
+
+CUtensorMapSwizzle swizzle_for(int row_bytes) {
+  return row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                          : (row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                             : (row_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                                                : CU_TENSOR_MAP_SWIZZLE_NONE));
+}
+
+// Tiled map over a tensor of `rank` dims (innermost first), strides in bytes
+// for dims 1..rank-1.
+bool encode(CUtensorMap *m, CUtensorMapDataType dt, int rank, const void *ptr, const uint64_t *dims,
+            const uint64_t *strides, const uint32_t *box, CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gd[5], gs[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i < rank - 1; ++i) gs[i] = strides[i];
+  CUresult r = fn(m, dt, cuuint32_t(rank), const_cast<void *>(ptr), gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Q/K/V: bf16 [BH, N, d] with a box of (min(DP, 64), 128, 1).
+bool encode_qkv(CUtensorMap *m, const void *ptr, int BH, int N, int d, int DP) {
+  const int ch = DP > 64 ? 64 : DP;
+  const uint64_t dims[3] = {uint64_t(d), uint64_t(N), uint64_t(BH)};
+  const uint64_t strides[2] = {uint64_t(d) * 2, uint64_t(N) * d * 2};
+  const uint32_t box[3] = {uint32_t(ch), 128u, 1u};
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, ptr, dims, strides, box, swizzle_for(ch * 2));
+}
+
+int *flags_for_current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_flag_ptr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_flags) != cudaSuccess) return nullptr;
+    g_flag_ptr[dev] = static_cast<int *>(p);
+  }
+  return g_flag_ptr[dev];
+}
+
+struct WsLayout {
+  size_t q_off, k_off, total;
+};
+
+WsLayout workspace_layout(int B, int H, int N, int R, int64_t bs, int64_t hs) {
+  WsLayout w{0, 0, 0};
+  if (R <= 0) return w;
+  const size_t fb = size_t(bs == 0 ? 1 : B) * size_t(hs == 0 ? 1 : H);
+  const size_t per = R <= 4 ? fb * size_t(N) * 16 : fb * size_t(N) * size_t(pad_rank(R)) * 2;
+  const size_t per_al = (per + 255) & ~size_t(255);
+  w.q_off = 0;
+  w.k_off = per_al;
+  w.total = 2 * per_al;
+  return w;
+}
+
+bool valid_shape_bf16(int B, int H, int N, int d) {
+  return B >= 1 && H >= 1 && N >= 1 && d >= 8 && d <= 128 && d % 8 == 0 && (long long)B * H <= (1ll << 31) - 1 &&
+         (long long)N <= (1ll << 31) - 256 && ((long long)N + 255) / 256 <= 65535;
+}
+
+bool valid_scale(float s) { return std::isfinite(s) && s > 0.f; }
+
+// Pick query tiles per CTA: two (the K/V tiles serve 256 rows) when there are
+// enough CTAs to fill the GPU at one CTA per SM and the ring keeps >= 2 stages.
+// FLASHBIAS_QUERY_TILES=1|2 pins the choice (a tuning and test knob).
+int forced_query_tiles() {
+  const char *e = std::getenv("FLASHBIAS_QUERY_TILES");
+  if (!e) return 0;
+  const int v = std::atoi(e);
+  return (v == 1 || v == 2) ? v : 0;
+}
+
+FwdPlan choose_plan(int DP, int RP, int mode, int BH, int N, int num_sms) {
+  const FwdPlan p2{DP, RP, mode, 2}, p1{DP, RP, mode, 1};
+  const int forced = forced_query_tiles();
+  if (forced == 2 && sm100_smem_bytes(p2) > 0) return p2;
+  if (forced == 1 && sm100_smem_bytes(p1) > 0) return p1;
+  const long long ctas2 = (long long)BH * ((N + 255) / 256);
+  if (sm100_smem_bytes(p2) > 0 && ctas2 >= 2ll * num_sms) return p2;
+  if (sm100_smem_bytes(p1) > 0) return p1;
+  return p2;
+}
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+}  // namespace
+
+int *device_flags() { return flags_for_current_device(); }
+
+}  // namespace fb
+
+using namespace fb;
+
+extern "C" {
+
+const char *fb_status_str(int s) {
+  switch (s) {
+    case FB_OK: return "FB_OK";
+    case FB_ERR_INVALID_ARG: return "FB_ERR_INVALID_ARG";
+    case FB_ERR_UNSUPPORTED: return "FB_ERR_UNSUPPORTED";
+    case FB_ERR_RANGE: return "FB_ERR_RANGE";
+    case FB_ERR_WORKSPACE: return "FB_ERR_WORKSPACE";
+    case FB_ERR_CUDA: return "FB_ERR_CUDA";
+    case FB_ERR_TIMEOUT: return "FB_ERR_TIMEOUT";
+    default: return "FB_ERR_UNKNOWN";
+  }
+}
+
+int fb_version(void) { return 100; }
+
+size_t fb_attn_workspace_bytes(int B, int H, int N, int R, int64_t phi_bstride, int64_t phi_hstride) {
+  if (B < 1 || H < 1 || N < 1 || R < 0 || R > 128) return 0;
+  return workspace_layout(B, H, N, R, phi_bstride, phi_hstride).total;
+}
+
+int fb_attn_fwd(int dt, int B, int H, int N, int d, const void *Q, const void *K, const void *V, int R,
+                const float *phi_q, const float *phi_k, int64_t phi_bstride, int64_t phi_hstride, float scale,
+                int causal, void *O, float *LSE, void *workspace, size_t workspace_bytes, void *stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!Q || !K || !V || !O || !LSE) return FB_ERR_INVALID_ARG;
+  if (R < 0 || R > 128) return FB_ERR_UNSUPPORTED;
+  if (R > 0 && (!phi_q || !phi_k || phi_bstride < 0 || phi_hstride < 0)) return FB_ERR_INVALID_ARG;
+  if (!valid_scale(scale)) return FB_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE)) return FB_ERR_INVALID_ARG;
+  if (R > 0 && (((reinterpret_cast<uintptr_t>(phi_q) | reinterpret_cast<uintptr_t>(phi_k)) & 3u) != 0))
+    return FB_ERR_INVALID_ARG;
+
+  if (dt == FB_F32) {
+    if (B < 1 || H < 1 || N < 1 || d < 4 || d > 128 || d % 4 != 0 || (N + 31) / 32 > (1 << 30) || B * H > 65535)
+      return FB_ERR_UNSUPPORTED;
+    int *flags = device_flags();
+    if (!flags) return FB_ERR_CUDA;
+    cudaError_t e = f32_launch(B, H, N, d, static_cast<const float *>(Q), static_cast<const float *>(K),
+                               static_cast<const float *>(V), R, phi_q, phi_k, phi_bstride, phi_hstride, nullptr, 0, 0,
+                               scale, causal, static_cast<float *>(O), LSE, st);
+    return e == cudaSuccess ? FB_OK : FB_ERR_CUDA;
+  }
+  if (dt != FB_BF16) return FB_ERR_UNSUPPORTED;
+  if (!valid_shape_bf16(B, H, N, d)) return FB_ERR_UNSUPPORTED;
+
+  const WsLayout ws = workspace_layout(B, H, N, R, phi_bstride, phi_hstride);
+  if (ws.total > 0) {
+    if (!workspace || workspace_bytes < ws.total) return FB_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FB_ERR_WORKSPACE;
+  }
+  const int DP = pad_dim(d);
+  const int mode = R == 0 ? kBiasNone : (R <= 4 ? kBiasReg : kBiasMma);
+  const int RP = mode == kBiasMma ? pad_rank(R) : (mode == kBiasReg ? (R <= 2 ? 2 : 4) : 0);
+  const int fac_B = phi_bstride == 0 ? 1 : B, fac_H = phi_hstride == 0 ? 1 : H;
+  const FwdPlan plan = choose_plan(DP, RP, mode, B * H, N, sm_count());
+  if (sm100_smem_bytes(plan) == 0) return FB_ERR_UNSUPPORTED;
+
+  int *flags = device_flags();
+  if (!flags) return FB_ERR_CUDA;
+
+  FwdMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  const int BH = B * H;
+  if (!encode_qkv(&maps.q, Q, BH, N, d, DP) || !encode_qkv(&maps.k, K, BH, N, d, DP) ||
+      !encode_qkv(&maps.v, V, BH, N, d, DP))
+    return FB_ERR_CUDA;
+  uint8_t *wsb = static_cast<uint8_t *>(workspace);
+  void *wq = ws.total ? wsb + ws.q_off : nullptr;
+  void *wk = ws.total ? wsb + ws.k_off : nullptr;
+  const int FB = fac_B * fac_H;
+  if (mode == kBiasMma) {
+    const int ch = RP > 64 ? 64 : RP;
+    const uint64_t dims[3] = {uint64_t(RP), uint64_t(N), uint64_t(FB)};
+    const uint64_t strides[2] = {uint64_t(RP) * 2, uint64_t(N) * RP * 2};
+    const uint32_t box[3] = {uint32_t(ch), 128u, 1u};
+    if (!encode(&maps.fq, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, wq, dims, strides, box, swizzle_for(ch * 2)) ||
+        !encode(&maps.fk, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, wk, dims, strides, box, swizzle_for(ch * 2)))
+      return FB_ERR_CUDA;
+  } else if (mode == kBiasReg) {
+    const uint64_t dims[3] = {4, uint64_t(N), uint64_t(FB)};
+    const uint64_t strides[2] = {16, uint64_t(N) * 16};
+    const uint32_t box[3] = {4u, 128u, 1u};
+    if (!encode(&maps.fk, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, wk, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return FB_ERR_CUDA;
+  }
+
+  cudaError_t e = cudaSuccess;
+  if (mode != kBiasNone) {
+    e = launch_prep_factors(mode, B, H, N, R, RP, phi_q, phi_k, phi_bstride, phi_hstride, fac_B, fac_H, scale, wq, wk,
+                            flags, st);
+    if (e != cudaSuccess) return FB_ERR_CUDA;
+  }
+  FwdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.B = B, a.H = H, a.N = N, a.d = d;
+  a.n_kv = (N + 127) / 128;
+  a.n_cta_q = (a.n_kv + plan.QT - 1) / plan.QT;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.causal = causal ? 1 : 0;
+  a.O = O;
+  a.LSE = LSE;
+  a.phiq_reg = mode == kBiasReg ? static_cast<const float *>(wq) : nullptr;
+  a.fac_B = fac_B, a.fac_H = fac_H;
+  a.bias_B = 1, a.bias_H = 1;
+  a.flags = flags;
+  e = sm100_launch(plan, maps, a, st);
+  return e == cudaSuccess ? FB_OK : FB_ERR_CUDA;
+}
+
+int fb_attn_dense_bias_fwd(int dt, int B, int H, int N, int d, const void *Q, const void *K, const void *V,
+                           const void *Bias, int64_t bias_bstride, int64_t bias_hstride, float scale, int causal,
+                           void *O, float *LSE, void *stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!Q || !K || !V || !O || !LSE || !Bias) return FB_ERR_INVALID_ARG;
+  if (bias_bstride < 0 || bias_hstride < 0) return FB_ERR_INVALID_ARG;
+  if (!valid_scale(scale)) return FB_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE) || !aligned16(Bias))
+    return FB_ERR_INVALID_ARG;
+  if (dt == FB_F32) {
+    if (B < 1 || H < 1 || N < 1 || d < 4 || d > 128 || d % 4 != 0 || B * H > 65535) return FB_ERR_UNSUPPORTED;
+    if (!device_flags()) return FB_ERR_CUDA;
+    cudaError_t e = f32_launch(B, H, N, d, static_cast<const float *>(Q), static_cast<const float *>(K),
+                               static_cast<const float *>(V), 0, nullptr, nullptr, 0, 0,
+                               static_cast<const float *>(Bias), bias_bstride, bias_hstride, scale, causal,
+                               static_cast<float *>(O), LSE, st);
+    return e == cudaSuccess ? FB_OK : FB_ERR_CUDA;
+  }
+  if (dt != FB_BF16) return FB_ERR_UNSUPPORTED;
+  if (!valid_shape_bf16(B, H, N, d)) return FB_ERR_UNSUPPORTED;
+  if (N % 8 != 0 || bias_bstride % 8 != 0 || bias_hstride % 8 != 0) return FB_ERR_UNSUPPORTED;
+  const int DP = pad_dim(d);
+  // The dense path keeps a two-deep ring: one query tile per CTA when two do not leave room for it.
+  FwdPlan plan{DP, 0, kBiasDense, 2};
+  {
+    const long long ctas2 = (long long)B * H * ((N + 255) / 256);
+    const size_t s2 = sm100_smem_bytes(plan);
+    FwdPlan p1{DP, 0, kBiasDense, 1};
+    const bool deep2 = s2 > 0 && DP <= 64;
+    const int forced = forced_query_tiles();
+    if (forced == 1 || (forced != 2 && !(deep2 && ctas2 >= 2ll * sm_count()))) plan = p1;
+    if (forced == 2 && s2 == 0) plan = p1;
+    if (sm100_smem_bytes(plan) == 0) return FB_ERR_UNSUPPORTED;
+  }
+  int *flags = device_flags();
+  if (!flags) return FB_ERR_CUDA;
+  FwdMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  const int BH = B * H;
+  if (!encode_qkv(&maps.q, Q, BH, N, d, DP) || !encode_qkv(&maps.k, K, BH, N, d, DP) ||
+      !encode_qkv(&maps.v, V, BH, N, d, DP))
+    return FB_ERR_CUDA;
+  const int bias_B = bias_bstride == 0 ? 1 : B, bias_H = bias_hstride == 0 ? 1 : H;
+  {
+    const uint64_t nn2 = uint64_t(N) * uint64_t(N) * 2;
+    const uint64_t dims[4] = {uint64_t(N), uint64_t(N), uint64_t(bias_H), uint64_t(bias_B)};
+    const uint64_t strides[3] = {uint64_t(N) * 2, bias_H > 1 ? uint64_t(bias_hstride) * 2 : nn2,
+                                 bias_B > 1 ? uint64_t(bias_bstride) * 2 : nn2};
+    const uint32_t box[4] = {64u, 128u, 1u, 1u};
+    if (!encode(&maps.bias, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, Bias, dims, strides, box,
+                CU_TENSOR_MAP_SWIZZLE_128B))
+      return FB_ERR_CUDA;
+  }
+  FwdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.B = B, a.H = H, a.N = N, a.d = d;
+  a.n_kv = (N + 127) / 128;
+  a.n_cta_q = (a.n_kv + plan.QT - 1) / plan.QT;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.causal = causal ? 1 : 0;
+  a.O = O;
+  a.LSE = LSE;
+  a.fac_B = 1, a.fac_H = 1;
+  a.bias_B = bias_B, a.bias_H = bias_H;
+  a.flags = flags;
+  cudaError_t e = sm100_launch(plan, maps, a, st);
+  return e == cudaSuccess ? FB_OK : FB_ERR_CUDA;
+}
+
+int fb_factors_sandwich(int N, int C, float *phi_q, float *phi_k, void *stream) {
+  if (N < 1 || C < 2 || C > 128 || C % 2 != 0 || !phi_q) return FB_ERR_INVALID_ARG;
+  return launch_sandwich(N, C, phi_q, phi_k, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FB_OK : FB_ERR_CUDA;
+}
+
+int fb_factors_alibi(int H, int N, float *phi_q, float *phi_k, void *stream) {
+  if (H < 1 || N < 1 || !phi_q || !phi_k) return FB_ERR_INVALID_ARG;
+  return launch_alibi(H, N, phi_q, phi_k, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FB_OK : FB_ERR_CUDA;
+}
+
+int fb_check_device_error(void *stream) {
+  int *flags = device_flags();
+  if (!flags) return FB_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return FB_ERR_CUDA;
+  int host = 0;
+  if (cudaMemcpyFromSymbol(&host, g_device_flags, sizeof(int)) != cudaSuccess) return FB_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_device_flags, &zero, sizeof(int)) != cudaSuccess) return FB_ERR_CUDA;
+  if (host & kFlagTimeout) return FB_ERR_TIMEOUT;
+  if (host & kFlagRange) return FB_ERR_RANGE;
+  return FB_OK;
+}
+
+int fb_selftest_wait_timeout(int limit_ms, void *stream) {
+  if (limit_ms < 1 || limit_ms > 2000) return FB_ERR_INVALID_ARG;
+  int *flags = device_flags();
+  if (!flags) return FB_ERR_CUDA;
+  return launch_wait_selftest(limit_ms, flags, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FB_OK
+                                                                                                 : FB_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,562 @@
+// fb_attn_sm100.cu -- fused forward of attention with an additive bias on
+// B200 (sm_100a): TMA -> shared memory -> tcgen05 MMA -> TMEM -> softmax on
+// the CUDA cores -> tcgen05 MMA -> TMEM -> HBM.
+//
+// Method: FlashBias (arXiv 2505.12044). The bias b = phi_q phi_k^T joins the
+// QK^T tile product: q' = [q, phi_q], k' = [k, phi_k] gives q'k'^T = qk^T +
+// phi_q phi_k^T (rebuttal, reply to Reviewer UJUf, Q2, "Eq. (3) of main
+// text"). Here the concatenation is never formed: the Q tile and the phi_q
+// tile sit in two shared-memory tiles and the two MMAs (bf16 QK^T, then fp16
+// phi_q' phi_k^T with phi_q' = phi_q / scale) accumulate into one fp32 TMEM
+// accumulator, so the N x N bias is never read or written (Figure 2). For
+// rank <= 4 (the ALiBi factors, Example 3.4) the factor tile is created next
+// to the scores on the CUDA cores in fp32 instead, as the rebuttal describes
+// for ALiBi (reply to Reviewer BRmd, Q2 (2): Block x 2 factor tiles made "in
+// JIT"). The dense mode streams a materialised bias tile per tile pair: the
+// "FlashAttention w/ Bias" comparison path of Figure 1(c).
+//
+// CTA organisation (QT = 1 or 2 query tiles of 128 rows per CTA):
+//   warps 0..4QT-1  softmax warpgroups; warpgroup t owns query tile t, one
+//                   thread per row (TMEM lane), so row max and row sum are
+//                   thread-local; it also rescales O in TMEM when the running
+//                   max grows by more than 2^8 and writes the epilogue.
+//   warp 4QT        TMA producer (one thread): Q|phi_q once, then K|phi_k and
+//                   V per 128-key step into a KS-deep ring, plus the
+//                   softmax-side tiles (dense bias / rank<=4 factors).
+//   warp 4QT+1      TMEM allocator and MMA issuer (one thread).
+// TMEM columns: S_t at 128 t, O_t at 128 QT + 128 t; P_t (bf16) overwrites
+// the first 64 columns of S_t and feeds the PV MMA as the TMEM A operand.
+// MMA issue order per key step i: S_0(i), PV_1(i-1), S_1(i), PV_0(i). With
+// that order the commit that publishes S_t(i) also covers PV_t(i-1), so the
+// softmax may rescale O_t right after seeing S_t(i), and S_t(i+1) is issued
+// after PV_t(i) has been issued (tcgen05 MMAs of one thread run in order).
+#include <algorithm>
+
+#include "fb_internal.h"
+#include "fb_ptx.cuh"
+
+namespace fb {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows by > 2^8
+constexpr uint32_t kSmemLimit = 227u * 1024u;
+
+template <int DP, int RP, int MODE, int QT>
+struct Sm100Cfg {
+  static constexpr int BM = 128;
+  static constexpr int BN = 128;
+  static constexpr int DCH = DP > 64 ? 64 : DP;  // columns per TMA box / swizzle atom
+  static constexpr int NDCH = DP / DCH;
+  static constexpr int RCH = (MODE == kBiasMma) ? (RP > 64 ? 64 : RP) : 16;
+  static constexpr int NRCH = (MODE == kBiasMma) ? RP / RCH : 0;
+  static constexpr uint32_t Q_TILE = BM * DP * 2;
+  static constexpr uint32_t KV_TILE = BN * DP * 2;
+  static constexpr uint32_t FQ_TILE = MODE == kBiasMma ? BM * RP * 2 : 0;
+  static constexpr uint32_t FK_TILE = MODE == kBiasMma ? BN * RP * 2 : 0;
+  static constexpr uint32_t AUX_TILE = MODE == kBiasReg ? BN * 16 : (MODE == kBiasDense ? BM * BN * 2 : 0);
+  static constexpr bool HAS_AUX = AUX_TILE > 0;
+  static constexpr uint32_t FIXED = QT * (Q_TILE + FQ_TILE);
+  static constexpr uint32_t STAGE = 2 * KV_TILE + FK_TILE + QT * AUX_TILE;
+  static constexpr uint32_t CTRL = 1024;  // barriers + TMEM address + abort flag
+  static constexpr uint32_t ALIGN_SLACK = 1024;
+  static constexpr int KS_FIT = (kSmemLimit > FIXED + CTRL + ALIGN_SLACK)
+                                    ? int((kSmemLimit - FIXED - CTRL - ALIGN_SLACK) / STAGE)
+                                    : 0;
+  static constexpr int KS = KS_FIT > 3 ? 3 : KS_FIT;
+  static constexpr uint32_t SMEM = FIXED + uint32_t(KS) * STAGE + CTRL + ALIGN_SLACK;
+  static constexpr int THREADS = QT * 128 + 64;
+  static constexpr int PRODUCER_WARP = QT * 4;
+  static constexpr int MMA_WARP = QT * 4 + 1;
+  static constexpr uint32_t TMEM_COLS = QT == 2 ? 512 : 256;
+  static constexpr uint32_t IDESC_QK = make_idesc_f16(true, true, 128, 128, false);
+  static constexpr uint32_t IDESC_F = make_idesc_f16(false, false, 128, 128, false);
+  static constexpr uint32_t IDESC_PV = make_idesc_f16(true, true, 128, DP, true);
+};
+
+struct SmemCtrl {
+  uint64_t q_full;
+  uint64_t o_final;
+  uint64_t drain;
+  uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
+  uint64_t s_full[2], p_full[2];
+  uint64_t aux_full[2][3], aux_empty[2][3];
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(SmemCtrl) <= 1024, "control block too large");
+
+// K-major tile of `rows` x (NCH * CH) 16-bit elements as NCH swizzled column
+// chunks of CH elements; descriptor for the 16-column MMA step kk.
+template <int CH>
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, int rows, int kk) {
+  constexpr int row_bytes = CH * 2;
+  constexpr int steps_per_chunk = CH / 16;
+  const int chunk = kk / steps_per_chunk;
+  const uint32_t off = uint32_t(chunk) * uint32_t(rows * row_bytes) + uint32_t(kk % steps_per_chunk) * 32u;
+  return make_smem_desc(base + off, 16, 8 * row_bytes, swizzle_code(row_bytes));
+}
+
+// V tile, [128 keys] x (NCH * CH) values, as the MN-major B operand of the PV
+// MMA; descriptor for the 16-key step kk.
+template <int CH>
+__device__ __forceinline__ uint64_t desc_v(uint32_t base, int kk) {
+  constexpr int row_bytes = CH * 2;
+  return make_smem_desc(base + uint32_t(kk) * 16u * row_bytes, 128 * row_bytes, 8 * row_bytes,
+                        swizzle_code(row_bytes));
+}
+
+template <int DP, int RP, int MODE, int QT>
+__global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, QT == 1 ? 2 : 1)
+    attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_fq,
+                   const __grid_constant__ CUtensorMap tm_fk, const __grid_constant__ CUtensorMap tm_bias,
+                   const FwdArgs args) {
+  using C = Sm100Cfg<DP, RP, MODE, QT>;
+  constexpr int KS = C::KS;
+  static_assert(KS >= 1, "configuration does not fit in shared memory");
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sQ = smem;                                     // QT x Q_TILE
+  uint8_t *sFQ = sQ + QT * C::Q_TILE;                     // QT x FQ_TILE
+  uint8_t *sK = sFQ + QT * C::FQ_TILE;                    // KS x KV_TILE
+  uint8_t *sFK = sK + KS * C::KV_TILE;                    // KS x FK_TILE
+  uint8_t *sV = sFK + KS * C::FK_TILE;                    // KS x KV_TILE
+  uint8_t *sAux = sV + KS * C::KV_TILE;                   // QT x KS x AUX_TILE
+  SmemCtrl *ctrl = reinterpret_cast<SmemCtrl *>(sAux + QT * KS * C::AUX_TILE);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int bh = blockIdx.x;
+  const int b = bh / args.H;
+  const int h = bh - b * args.H;
+  const int qg = args.n_cta_q - 1 - int(blockIdx.y);  // heaviest causal row groups first
+  const int N = args.N;
+  const int fb_slice = (args.fac_B > 1 ? b : 0) * args.fac_H + (args.fac_H > 1 ? h : 0);
+
+  // Per query tile: first row and number of key steps.
+  int q0[2], nk[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int qt = qg * QT + t;
+    q0[t] = qt * 128;
+    const bool active = (t < QT) && (q0[t] < N);
+    nk[t] = active ? (args.causal ? min(qt + 1, args.n_kv) : args.n_kv) : 0;
+  }
+  const int n_steps = max(nk[0], nk[1]);
+
+  if (threadIdx.x == 0) {
+    mbar_init(&ctrl->q_full, 1);
+    mbar_init(&ctrl->o_final, 1);
+    mbar_init(&ctrl->drain, 1);
+    for (int s = 0; s < KS; ++s) {
+      mbar_init(&ctrl->k_full[s], 1);
+      mbar_init(&ctrl->k_empty[s], 1);
+      mbar_init(&ctrl->v_full[s], 1);
+      mbar_init(&ctrl->v_empty[s], 1);
+      for (int t = 0; t < QT; ++t) {
+        mbar_init(&ctrl->aux_full[t][s], 1);
+        mbar_init(&ctrl->aux_empty[t][s], 128);
+      }
+    }
+    for (int t = 0; t < QT; ++t) {
+      mbar_init(&ctrl->s_full[t], 1);
+      mbar_init(&ctrl->p_full[t], 128);
+    }
+    ctrl->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(&ctrl->tmem_base, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctrl->tmem_base;
+  volatile int *abort = &ctrl->abort;
+
+  if (warp == C::PRODUCER_WARP) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_map(&tm_q);
+      tma_prefetch_map(&tm_k);
+      tma_prefetch_map(&tm_v);
+      if (MODE == kBiasMma) {
+        tma_prefetch_map(&tm_fq);
+        tma_prefetch_map(&tm_fk);
+      }
+      if (MODE == kBiasReg) tma_prefetch_map(&tm_fk);
+      if (MODE == kBiasDense) tma_prefetch_map(&tm_bias);
+      uint32_t qbytes = 0;
+      for (int t = 0; t < QT; ++t)
+        if (nk[t] > 0) qbytes += C::Q_TILE + C::FQ_TILE;
+      mbar_arrive_expect_tx(&ctrl->q_full, qbytes);
+      for (int t = 0; t < QT; ++t) {
+        if (nk[t] == 0) continue;
+        for (int ch = 0; ch < C::NDCH; ++ch)
+          tma_load_3d(sQ + t * C::Q_TILE + ch * (128 * C::DCH * 2), &tm_q, &ctrl->q_full, ch * C::DCH, q0[t], bh);
+        if (MODE == kBiasMma)
+          for (int ch = 0; ch < C::NRCH; ++ch)
+            tma_load_3d(sFQ + t * C::FQ_TILE + ch * (128 * C::RCH * 2), &tm_fq, &ctrl->q_full, ch * C::RCH, q0[t],
+                        fb_slice);
+      }
+      int hb = 0, bb = 0;
+      if (MODE == kBiasDense) {
+        hb = args.bias_H > 1 ? h : 0;
+        bb = args.bias_B > 1 ? b : 0;
+      }
+      bool ok = true;
+      for (int i = 0; i < n_steps && ok; ++i) {
+        const int s = i % KS;
+        const uint32_t ph = uint32_t(i / KS) & 1u;
+        if (!(ok = mbar_wait(&ctrl->k_empty[s], ph ^ 1u, abort))) break;
+        mbar_arrive_expect_tx(&ctrl->k_full[s], C::KV_TILE + C::FK_TILE);
+        for (int ch = 0; ch < C::NDCH; ++ch)
+          tma_load_3d(sK + s * C::KV_TILE + ch * (128 * C::DCH * 2), &tm_k, &ctrl->k_full[s], ch * C::DCH, i * 128,
+                      bh);
+        if (MODE == kBiasMma)
+          for (int ch = 0; ch < C::NRCH; ++ch)
+            tma_load_3d(sFK + s * C::FK_TILE + ch * (128 * C::RCH * 2), &tm_fk, &ctrl->k_full[s], ch * C::RCH,
+                        i * 128, fb_slice);
+        if (C::HAS_AUX) {
+          for (int t = 0; t < QT; ++t) {
+            if (i >= nk[t]) continue;
+            if (!(ok = mbar_wait(&ctrl->aux_empty[t][s], ph ^ 1u, abort))) break;
+            uint8_t *dst = sAux + (t * KS + s) * C::AUX_TILE;
+            mbar_arrive_expect_tx(&ctrl->aux_full[t][s], C::AUX_TILE);
+            if (MODE == kBiasReg) {
+              tma_load_3d(dst, &tm_fk, &ctrl->aux_full[t][s], 0, i * 128, fb_slice);
+            } else {
+              tma_load_4d(dst, &tm_bias, &ctrl->aux_full[t][s], i * 128, q0[t], hb, bb);
+              tma_load_4d(dst + 128 * 128, &tm_bias, &ctrl->aux_full[t][s], i * 128 + 64, q0[t], hb, bb);
+            }
+          }
+          if (!ok) break;
+        }
+        if (!(ok = mbar_wait(&ctrl->v_empty[s], ph ^ 1u, abort))) break;
+        mbar_arrive_expect_tx(&ctrl->v_full[s], C::KV_TILE);
+        for (int ch = 0; ch < C::NDCH; ++ch)
+          tma_load_3d(sV + s * C::KV_TILE + ch * (128 * C::DCH * 2), &tm_v, &ctrl->v_full[s], ch * C::DCH, i * 128,
+                      bh);
+      }
+      if (!ok) {
+        // Aborted: let the copies already issued land before the CTA exits.
+        for (int s = 0; s < KS; ++s) {
+          mbar_wait_for(&ctrl->k_full[s], 0, 100000000ull);
+          mbar_wait_for(&ctrl->k_full[s], 1, 100000000ull);
+          mbar_wait_for(&ctrl->v_full[s], 0, 100000000ull);
+          mbar_wait_for(&ctrl->v_full[s], 1, 100000000ull);
+        }
+        atomicOr(args.flags, kFlagTimeout);
+      }
+    }
+  } else if (warp == C::MMA_WARP) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t sQa = smem_u32(sQ), sFQa = smem_u32(sFQ), sKa = smem_u32(sK), sFKa = smem_u32(sFK),
+                     sVa = smem_u32(sV);
+      auto issue_s = [&](int t, int s) {
+        const uint32_t d_tm = tmem + uint32_t(128 * t);
+#pragma unroll
+        for (int kk = 0; kk < DP / 16; ++kk)
+          mma_ss(d_tm, desc_kmajor<C::DCH>(sQa + t * C::Q_TILE, 128, kk),
+                 desc_kmajor<C::DCH>(sKa + s * C::KV_TILE, 128, kk), C::IDESC_QK, kk > 0 ? 1u : 0u);
+        if (MODE == kBiasMma) {
+#pragma unroll
+          for (int kk = 0; kk < (MODE == kBiasMma ? RP / 16 : 0); ++kk)
+            mma_ss(d_tm, desc_kmajor<C::RCH>(sFQa + t * C::FQ_TILE, 128, kk),
+                   desc_kmajor<C::RCH>(sFKa + s * C::FK_TILE, 128, kk), C::IDESC_F, 1u);
+        }
+      };
+      auto issue_pv = [&](int t, int s, bool acc) {
+        const uint32_t d_tm = tmem + uint32_t(128 * QT + 128 * t);
+        const uint32_t p_tm = tmem + uint32_t(128 * t);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(d_tm, p_tm + uint32_t(kk * 8), desc_v<C::DCH>(sVa + s * C::KV_TILE, kk), C::IDESC_PV,
+                 (acc || kk > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(&ctrl->q_full, 0, abort);
+      tc_fence_after();
+      for (int i = 0; i < n_steps && ok; ++i) {
+        const int s = i % KS;
+        const uint32_t ph = uint32_t(i / KS) & 1u;
+        if (!(ok = mbar_wait(&ctrl->k_full[s], ph, abort))) break;
+        tc_fence_after();
+        if (i < nk[0]) {
+          issue_s(0, s);
+          tc_commit(&ctrl->s_full[0]);
+        }
+        if (QT == 2) {
+          const int j = i - 1;  // PV of tile 1 for the previous step
+          if (j >= 0 && j < nk[1]) {
+            const int sj = j % KS;
+            const uint32_t phj = uint32_t(j / KS) & 1u;
+            if (j >= nk[0] && !(ok = mbar_wait(&ctrl->v_full[sj], phj, abort))) break;
+            if (!(ok = mbar_wait(&ctrl->p_full[1], uint32_t(j) & 1u, abort))) break;
+            tc_fence_after();
+            issue_pv(1, sj, j > 0);
+            tc_commit(&ctrl->v_empty[sj]);
+          }
+          if (i < nk[1]) {
+            issue_s(1, s);
+            tc_commit(&ctrl->s_full[1]);
+          }
+        }
+        tc_commit(&ctrl->k_empty[s]);
+        if (i < nk[0]) {
+          if (!(ok = mbar_wait(&ctrl->v_full[s], ph, abort))) break;
+          if (!(ok = mbar_wait(&ctrl->p_full[0], uint32_t(i) & 1u, abort))) break;
+          tc_fence_after();
+          issue_pv(0, s, i > 0);
+          if (QT == 1 || i >= nk[1]) tc_commit(&ctrl->v_empty[s]);
+        }
+      }
+      if (ok && QT == 2 && nk[1] == n_steps && n_steps > 0) {
+        const int j = n_steps - 1;
+        const int sj = j % KS;
+        const uint32_t phj = uint32_t(j / KS) & 1u;
+        ok = (j < nk[0]) || mbar_wait(&ctrl->v_full[sj], phj, abort);
+        ok = ok && mbar_wait(&ctrl->p_full[1], uint32_t(j) & 1u, abort);
+        if (ok) {
+          tc_fence_after();
+          issue_pv(1, sj, j > 0);
+          tc_commit(&ctrl->v_empty[sj]);
+        }
+      }
+      tc_commit(&ctrl->o_final);
+      if (!ok) {
+        // Aborted: wait (bounded) for the MMAs already issued to finish.
+        tc_commit(&ctrl->drain);
+        mbar_wait_for(&ctrl->drain, 0, 100000000ull);
+        atomicOr(args.flags, kFlagTimeout);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------- softmax
+    const int t = warp >> 2;  // query tile of this warpgroup
+    const int wq = warp & 3;  // TMEM lane quarter
+    const int r_loc = wq * 32 + lane;
+    const int row = q0[t] + r_loc;
+    const uint32_t lane_base = tmem + (uint32_t(wq * 32) << 16);
+    const uint32_t s_tm = lane_base + uint32_t(128 * t);
+    const uint32_t o_tm = lane_base + uint32_t(128 * QT + 128 * t);
+    const float sl2 = args.scale_log2;
+
+    float aq0 = 0.f, aq1 = 0.f, aq2 = 0.f, aq3 = 0.f;
+    if (MODE == kBiasReg && row < N) {
+      const float4 v = *reinterpret_cast<const float4 *>(args.phiq_reg + (size_t(fb_slice) * N + row) * 4);
+      aq0 = v.x, aq1 = v.y, aq2 = v.z, aq3 = v.w;
+    }
+
+    float m_use = -INFINITY, l_sum = 0.f;
+    bool ok = true;
+    for (int i = 0; i < nk[t]; ++i) {
+      const int s = i % KS;
+      const uint32_t ph = uint32_t(i / KS) & 1u;
+      if (C::HAS_AUX && !(ok = mbar_wait(&ctrl->aux_full[t][s], ph, abort))) break;
+      if (!(ok = mbar_wait(&ctrl->s_full[t], uint32_t(i) & 1u, abort))) break;
+      tc_fence_after();
+
+      // Raw scores of this thread's row; with a softmax-side bias they are
+      // turned into log2-domain logits in place, otherwise the scale is
+      // folded into the exponent below.
+      uint32_t x[128];
+      tmem_ld32(s_tm + 0, x + 0);
+      tmem_ld32(s_tm + 32, x + 32);
+      tmem_ld32(s_tm + 64, x + 64);
+      tmem_ld32(s_tm + 96, x + 96);
+      tmem_ld_wait32(x + 0);
+      tmem_ld_wait32(x + 32);
+      tmem_ld_wait32(x + 64);
+      tmem_ld_wait32(x + 96);
+      float mul = sl2;  // logit = raw * mul
+      if (MODE == kBiasReg) {
+        const uint8_t *fk = sAux + (t * KS + s) * C::AUX_TILE;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          float v;
+          if (RP <= 2) {
+            const float2 f = *reinterpret_cast<const float2 *>(fk + c * 16);
+            v = fmaf(aq0, f.x, fmaf(aq1, f.y, __uint_as_float(x[c]) * sl2));
+          } else {
+            const float4 f = *reinterpret_cast<const float4 *>(fk + c * 16);
+            v = fmaf(aq0, f.x, fmaf(aq1, f.y, fmaf(aq2, f.z, fmaf(aq3, f.w, __uint_as_float(x[c]) * sl2))));
+          }
+          x[c] = __float_as_uint(v);
+        }
+        mbar_arrive(&ctrl->aux_empty[t][s]);
+        mul = 1.f;
+      } else if (MODE == kBiasDense) {
+        const uint8_t *tile = sAux + (t * KS + s) * C::AUX_TILE;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+          for (int ck = 0; ck < 8; ++ck) {
+            const uint4 u =
+                *reinterpret_cast<const uint4 *>(tile + hh * 16384 + r_loc * 128 + ((ck ^ (r_loc & 7)) * 16));
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c = hh * 64 + ck * 8 + 2 * e;
+              x[c] = __float_as_uint(fmaf(__uint_as_float(w[e] << 16), kLog2e, __uint_as_float(x[c]) * sl2));
+              x[c + 1] =
+                  __float_as_uint(fmaf(__uint_as_float(w[e] & 0xFFFF0000u), kLog2e, __uint_as_float(x[c + 1]) * sl2));
+            }
+          }
+        }
+        mbar_arrive(&ctrl->aux_empty[t][s]);
+        mul = 1.f;
+      }
+      // Causal diagonal tile and the ragged last key tile.
+      const int key0 = i * 128;
+      if ((args.causal && key0 + 127 > q0[t]) || key0 + 128 > N) {
+        const int lim = args.causal ? min(row + 1, N) : N;  // keys [0, lim) are visible
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (key0 + c >= lim) x[c] = __float_as_uint(-INFINITY);
+      }
+      float mx = __uint_as_float(x[0]);
+#pragma unroll
+      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(x[c]));
+      const float m_new = fmaxf(m_use, mx * mul);
+      float alpha = 1.f;
+      bool resc = false;
+      if (m_use == -INFINITY || m_new > m_use + kRescaleThreshold) {
+        alpha = (m_use == -INFINITY) ? 0.f : ex2_approx(m_use - m_new);
+        resc = (i > 0) && (m_use != -INFINITY);
+        m_use = m_new;
+      }
+      l_sum *= alpha;
+      if (__any_sync(0xffffffffu, resc)) {
+        // PV_t(i-1) has completed: the commit that published S_t(i) covers it.
+#pragma unroll
+        for (int c0 = 0; c0 < DP; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld16(o_tm + c0, r);
+          tmem_ld_wait16(r);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+          tmem_st16(o_tm + c0, r);
+        }
+      }
+      const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(x[q4 * 32 + 2 * e]), mul, neg_m));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(x[q4 * 32 + 2 * e + 1]), mul, neg_m));
+          l_sum += p0 + p1;
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(s_tm + uint32_t(q4 * 16), pk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&ctrl->p_full[t]);
+    }
+
+    // ------------------------------------------------------------ epilogue
+    if (ok && nk[t] > 0) ok = mbar_wait(&ctrl->o_final, 0, abort);
+    if (ok && nk[t] > 0) {
+      tc_fence_after();
+      const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
+      __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(args.O) + (size_t(bh) * N + row) * args.d;
+#pragma unroll
+      for (int c0 = 0; c0 < DP; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld16(o_tm + c0, r);
+        tmem_ld_wait16(r);
+        if (row < N) {
+#pragma unroll
+          for (int v8 = 0; v8 < 2; ++v8) {
+            const int col = c0 + v8 * 8;
+            if (col < args.d) {
+              uint4 u;
+              u.x = pack_bf16x2(__uint_as_float(r[v8 * 8 + 0]) * inv_l, __uint_as_float(r[v8 * 8 + 1]) * inv_l);
+              u.y = pack_bf16x2(__uint_as_float(r[v8 * 8 + 2]) * inv_l, __uint_as_float(r[v8 * 8 + 3]) * inv_l);
+              u.z = pack_bf16x2(__uint_as_float(r[v8 * 8 + 4]) * inv_l, __uint_as_float(r[v8 * 8 + 5]) * inv_l);
+              u.w = pack_bf16x2(__uint_as_float(r[v8 * 8 + 6]) * inv_l, __uint_as_float(r[v8 * 8 + 7]) * inv_l);
+              *reinterpret_cast<uint4 *>(orow + col) = u;
+            }
+          }
+        }
+      }
+      if (row < N)
+        args.LSE[size_t(bh) * N + row] = l_sum > 0.f ? (m_use + __log2f(l_sum)) * kLn2 : -INFINITY;
+    }
+    if (!ok) atomicOr(args.flags, kFlagTimeout);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == C::MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <int DP, int RP, int MODE, int QT>
+static cudaError_t launch_one(const FwdMaps &m, const FwdArgs &a, cudaStream_t stream) {
+  using C = Sm100Cfg<DP, RP, MODE, QT>;
+  if constexpr (C::KS < 1) {
+    return cudaErrorInvalidConfiguration;
+  } else {
+    auto kern = attn_fwd_sm100<DP, RP, MODE, QT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::SMEM));
+    if (e != cudaSuccess) return e;
+    dim3 grid(a.B * a.H, a.n_cta_q);
+    kern<<<grid, C::THREADS, C::SMEM, stream>>>(m.q, m.k, m.v, m.fq, m.fk, m.bias, a);
+    return cudaGetLastError();
+  }
+}
+
+template <int DP, int RP, int MODE, int QT>
+static constexpr size_t smem_of() {
+  using C = Sm100Cfg<DP, RP, MODE, QT>;
+  return C::KS >= 1 ? size_t(C::SMEM) : 0;
+}
+
+#define FB_DISPATCH_QT(DPv, RPv, MODEv)                                          \
+  if (p.QT == 1) return FB_ACTION(DPv, RPv, MODEv, 1);                           \
+  if (p.QT == 2) return FB_ACTION(DPv, RPv, MODEv, 2);
+
+#define FB_DISPATCH_MODE(DPv)                                                    \
+  if (p.mode == kBiasNone) { FB_DISPATCH_QT(DPv, 0, kBiasNone) }                 \
+  if (p.mode == kBiasReg) {                                                      \
+    if (p.RP == 2) { FB_DISPATCH_QT(DPv, 2, kBiasReg) }                          \
+    if (p.RP == 4) { FB_DISPATCH_QT(DPv, 4, kBiasReg) }                          \
+  }                                                                              \
+  if (p.mode == kBiasDense) { FB_DISPATCH_QT(DPv, 0, kBiasDense) }               \
+  if (p.mode == kBiasMma) {                                                      \
+    if (p.RP == 16) { FB_DISPATCH_QT(DPv, 16, kBiasMma) }                        \
+    if (p.RP == 32) { FB_DISPATCH_QT(DPv, 32, kBiasMma) }                        \
+    if (p.RP == 64) { FB_DISPATCH_QT(DPv, 64, kBiasMma) }                        \
+    if (p.RP == 128) { FB_DISPATCH_QT(DPv, 128, kBiasMma) }                      \
+  }
+
+#define FB_DISPATCH_ALL                                                          \
+  if (p.DP == 16) { FB_DISPATCH_MODE(16) }                                       \
+  if (p.DP == 32) { FB_DISPATCH_MODE(32) }                                       \
+  if (p.DP == 64) { FB_DISPATCH_MODE(64) }                                       \
+  if (p.DP == 128) { FB_DISPATCH_MODE(128) }
+
+size_t sm100_smem_bytes(const FwdPlan &p) {
+#define FB_ACTION(DPv, RPv, MODEv, QTv) smem_of<DPv, RPv, MODEv, QTv>()
+  FB_DISPATCH_ALL
+#undef FB_ACTION
+  return 0;
+}
+
+cudaError_t sm100_launch(const FwdPlan &p, const FwdMaps &maps, const FwdArgs &a, cudaStream_t stream) {
+#define FB_ACTION(DPv, RPv, MODEv, QTv) launch_one<DPv, RPv, MODEv, QTv>(maps, a, stream)
+  FB_DISPATCH_ALL
+#undef FB_ACTION
+  return cudaErrorInvalidConfiguration;
+}
+
+}  // namespace fb

@@ -1,0 +1,77 @@
+// fb_internal.h -- declarations shared by the translation units of
+// libflashbias (host side). Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/flashbias.h"
+
+namespace fb {
+
+// Bits of the library's device flag word.
+constexpr int kFlagTimeout = 1;
+constexpr int kFlagRange = 2;
+
+// Bias handling inside the tensor-core kernel.
+enum BiasMode : int {
+  kBiasNone = 0,   // plain attention (R == 0)
+  kBiasMma = 1,    // fp16 factors, second tcgen05 MMA into the score accumulator
+  kBiasReg = 2,    // R <= 4 fp32 factors, added on the CUDA cores
+  kBiasDense = 3,  // materialised bf16 bias tile streamed by TMA (comparison path)
+};
+
+// Runtime arguments of the tensor-core forward kernel.
+struct FwdArgs {
+  int B, H, N, d;
+  int n_kv;          // number of 128-key tiles
+  int n_cta_q;       // number of CTA row groups along N
+  float scale_log2;  // scale * log2(e)
+  int causal;
+  void *O;
+  float *LSE;
+  const float *phiq_reg;  // kBiasReg: [FB, N, 4] fp32, phi_q * log2(e)
+  int fac_B, fac_H;       // factor slices: B or 1, H or 1 (1 = broadcast)
+  int bias_B, bias_H;     // dense bias slices, same convention
+  int *flags;             // device flag word
+};
+
+// Launch description chosen by the host for one call.
+struct FwdPlan {
+  int DP;    // padded head dim: 16, 32, 64, 128
+  int RP;    // kBiasMma: padded factor rank (16..128); kBiasReg: 2 or 4 live factor columns; else 0
+  int mode;  // BiasMode
+  int QT;    // 128-row query tiles per CTA: 1 or 2
+};
+
+struct FwdMaps {
+  CUtensorMap q, k, v;  // bf16 [BH, N, d] with box (min(DP,64), 128, 1)
+  CUtensorMap fq, fk;   // factors: fp16 [FB, N, RP] (mma) or fp32 [FB, N, 4] (reg, fk only)
+  CUtensorMap bias;     // dense bias bf16 [B', H', N, N] with box (64, 128, 1, 1)
+};
+
+// Shared-memory bytes the kernel needs for a plan, or 0 if it does not fit.
+size_t sm100_smem_bytes(const FwdPlan &p);
+// Launches the tcgen05 kernel; returns a cudaError_t.
+cudaError_t sm100_launch(const FwdPlan &p, const FwdMaps &maps, const FwdArgs &a, cudaStream_t stream);
+
+// CUDA-core fp32 path (also the oracle-precision path of the bf16-free workload).
+cudaError_t f32_launch(int B, int H, int N, int d, const float *Q, const float *K, const float *V, int R,
+                       const float *phi_q, const float *phi_k, int64_t phi_bs, int64_t phi_hs, const float *bias,
+                       int64_t bias_bs, int64_t bias_hs, float scale, int causal, float *O, float *LSE,
+                       cudaStream_t stream);
+
+// Factor generators and preparation.
+cudaError_t launch_sandwich(int N, int C, float *phi_q, float *phi_k, cudaStream_t s);
+cudaError_t launch_alibi(int H, int N, float *phi_q, float *phi_k, cudaStream_t s);
+// kBiasMma: fp16 [FB, N, RP], phi_q / scale. kBiasReg: fp32 [FB, N, 4], phi_q * log2 e.
+cudaError_t launch_prep_factors(int mode, int B, int H, int N, int R, int RP, const float *phi_q, const float *phi_k,
+                                int64_t bs, int64_t hs, int fac_B, int fac_H, float scale, void *out_q, void *out_k,
+                                int *flags, cudaStream_t s);
+cudaError_t launch_wait_selftest(int limit_ms, int *flags, cudaStream_t s);
+
+// Per-device flag word (allocated once per device as a module global).
+int *device_flags();
+
+}  // namespace fb

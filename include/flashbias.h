@@ -1,0 +1,188 @@
+/*
+ * flashbias.h -- C ABI of libflashbias: attention with a low-rank additive
+ * bias on NVIDIA B200 (sm_100a).
+ *
+ * The method is "FlashBias: Fast Computation of Attention with Bias" (Wu et
+ * al., arXiv 2505.12044). Attention with bias adds an N x N matrix b to the
+ * query-key scores (FlashBias abstract; Figure 1). FlashBias replaces b by
+ * per-token factors phi_q, phi_k of rank R, b = phi_q phi_k^T (Figure 2), and
+ * joins them to the QK^T tile product by concatenating them with the queries
+ * and keys (rebuttal, reply to Reviewer UJUf, Q2: "Eq. (3) of main text").
+ * The N x N bias is never materialised; only heads x N x R factor values are
+ * read (reply to Reviewer BRmd, Q3).
+ *
+ * Conventions shared by every entry point:
+ *  - Tensor pointers are DEVICE pointers unless the name ends in _host.
+ *  - Q, K, V, O are [B, H, N, d] row-major (d innermost, contiguous).
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL = the legacy default stream).
+ *  - The caller owns all memory. Besides caller-provided workspace the
+ *    library allocates no device memory.
+ *  - Argument, shape, alignment and range errors are reported synchronously,
+ *    before anything is launched. A launch failure returns FB_ERR_CUDA.
+ *  - Kernel-side conditions (a pipeline wait that ran out, a factor that
+ *    overflowed fp16) set a library-wide device flag that
+ *    fb_check_device_error() reads back; the kernels never trap.
+ *  - No C++ exception crosses this interface. Entry points may be called
+ *    from several host threads.
+ */
+#ifndef FLASHBIAS_H_
+#define FLASHBIAS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FB_OK = 0,
+  FB_ERR_INVALID_ARG = 1, /* null pointer, bad shape, bad stride, bad scale   */
+  FB_ERR_UNSUPPORTED = 2, /* valid but outside what this build implements     */
+  FB_ERR_RANGE = 3,       /* a factor value does not fit the kernel's type    */
+  FB_ERR_WORKSPACE = 4,   /* workspace missing, too small or misaligned       */
+  FB_ERR_CUDA = 5,        /* CUDA runtime/driver call or launch failed        */
+  FB_ERR_TIMEOUT = 6      /* a kernel's bounded pipeline wait ran out         */
+} fb_status;
+
+typedef enum { FB_F32 = 0, FB_BF16 = 1 } fb_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *fb_status_str(int status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int fb_version(void);
+
+/*
+ * Workspace for fb_attn_fwd with the bf16 path: the factor tensors after the
+ * preparation step (scaled, converted and padded so the tensor cores can read
+ * them). Depends on which factor dimensions are broadcast (stride 0).
+ * Returns 0 when R == 0. The fp32 path needs no workspace.
+ */
+size_t fb_attn_workspace_bytes(int B, int H, int N, int R,
+                               int64_t phi_bstride, int64_t phi_hstride);
+
+/*
+ * Fused forward of attention with a low-rank additive bias:
+ *
+ *   O = softmax(scale * Q K^T + phi_q phi_k^T [+ causal mask]) V
+ *   LSE[b,h,i] = ln sum_j exp(scale * q_i.k_j + b_ij)   (over visible j)
+ *
+ * (FlashBias abstract and Figure 2; rebuttal, reply to Reviewer UJUf, Q2, the
+ * concatenation q' = [q, phi_q], k' = [k, phi_k]. The bias is not scaled:
+ * scale multiplies QK^T only.)
+ *
+ *  dt          FB_BF16: Q, K, V, O are bf16, tensor-core path (tcgen05).
+ *              FB_F32 : Q, K, V, O are fp32, CUDA-core path, fp32 throughout.
+ *  B, H, N, d  batch, heads, sequence length, head dim. bf16: d % 8 == 0,
+ *              8 <= d <= 128. fp32: d % 4 == 0, 4 <= d <= 128. N >= 1.
+ *  Q, K, V     [B, H, N, d] device, 16-byte aligned.
+ *  R           bias rank, 0 <= R <= 128. R == 0 is plain attention.
+ *  phi_q/phi_k fp32 device factors; element (b, h, n, r) sits at
+ *              b*phi_bstride + h*phi_hstride + n*R + r. A stride of 0
+ *              broadcasts that dimension (the Sandwich and ALiBi factors do
+ *              not depend on the batch). May be NULL when R == 0.
+ *  scale       multiplies QK^T; finite and > 0 (usually 1/sqrt(d)).
+ *  causal      nonzero: key j is visible to query i iff j <= i.
+ *  O           [B, H, N, d] device output (dtype dt).
+ *  LSE         [B, H, N] fp32 device output, natural log.
+ *  workspace   device scratch of at least fb_attn_workspace_bytes(...) bytes,
+ *              256-byte aligned; may be NULL when that is 0 or dt == FB_F32.
+ *              It must not be shared by calls that can run concurrently.
+ *  stream      cudaStream_t.
+ *
+ * bf16 path numerics: QK^T in bf16 x bf16 -> fp32; the factors enter the same
+ * fp32 accumulator as a second MMA in fp16 (phi_q pre-divided by scale) when
+ * R > 4, or are added in fp32 on the CUDA cores when R <= 4; softmax in fp32;
+ * P rounded to bf16 for the PV MMA; O rounded to bf16. A factor that does not
+ * fit fp16 is saturated and flags FB_ERR_RANGE for fb_check_device_error().
+ */
+int fb_attn_fwd(int dt, int B, int H, int N, int d,
+                const void *Q, const void *K, const void *V,
+                int R, const float *phi_q, const float *phi_k,
+                int64_t phi_bstride, int64_t phi_hstride,
+                float scale, int causal,
+                void *O, float *LSE,
+                void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Comparison path, "FlashAttention w/ Bias" (FlashBias Figure 1(c)): the same
+ * attention with a materialised dense bias that is streamed from HBM tile by
+ * tile (the quadratic bias IO that FlashBias avoids, Figure 2).
+ *
+ *  Bias        [., ., N, N] device, dtype dt; element (b, h, i, j) sits at
+ *              b*bias_bstride + h*bias_hstride + i*N + j (strides in
+ *              elements, 0 = broadcast, otherwise multiples of 8).
+ *              bf16 path: N % 8 == 0 (TMA row pitch) and 16-byte alignment.
+ *  Other arguments as fb_attn_fwd. No workspace.
+ */
+int fb_attn_dense_bias_fwd(int dt, int B, int H, int N, int d,
+                           const void *Q, const void *K, const void *V,
+                           const void *Bias, int64_t bias_bstride,
+                           int64_t bias_hstride, float scale, int causal,
+                           void *O, float *LSE, void *stream);
+
+/*
+ * Exact Sandwich factors (rebuttal, reply to Reviewer UJUf, Q1 (1)-(2)):
+ *   b_ij = sum_{k=1}^{C/2} cos((i-j) / 10000^{2k/C}) = phi(i) . phi(j),
+ *   phi(i) = [cos(i w_1), sin(i w_1), ..., cos(i w_{C/2}), sin(i w_{C/2})],
+ *   w_k = 10000^{-2k/C}.
+ * Writes phi_q and phi_k, each [N, C] fp32 device (rank R = C), computed in
+ * fp64. phi_k may be NULL or equal phi_q (the two factors are identical).
+ * C even, 2 <= C <= 128.
+ */
+int fb_factors_sandwich(int N, int C, float *phi_q, float *phi_k, void *stream);
+
+/*
+ * Exact rank-2 ALiBi factors (FlashBias Example 3.4; rebuttal, reply to
+ * Reviewer BRmd, Q2 (2): Block x 2 factor tiles in place of the
+ * Block x Block bias): for head h of H, m_h = 2^{-8(h+1)/H},
+ *   phi_q(i) = [-m_h i, 1],  phi_k(j) = [1, m_h j],  phi_q(i).phi_k(j) = -m_h (i-j).
+ * Writes phi_q, phi_k as [H, N, 2] fp32 device (use phi_bstride = 0,
+ * phi_hstride = 2N). Products are formed in fp64 and rounded once.
+ */
+int fb_factors_alibi(int H, int N, float *phi_q, float *phi_k, void *stream);
+
+/*
+ * Truncated SVD of one head's static dense bias on the host (rebuttal, reply
+ * to Reviewer xU4x, Q6: SVD decomposition, rank chosen per head; computed
+ * once, not per inference). Randomized range finder with `oversample` extra
+ * columns and `power_iters` subspace iterations, then a one-sided Jacobi SVD
+ * of the projected matrix. Balanced split: phi_q = U_R sqrt(S_R),
+ * phi_k = V_R sqrt(S_R).
+ *
+ *  bias_host     [N, N] fp64 host, row-major.
+ *  R             rank, 1 <= R <= min(N, 128); R + oversample <= N is clamped.
+ *  seed          seeds the Gaussian test matrix.
+ *  phi_q_host, phi_k_host   [N, R] fp32 host outputs.
+ *  rel_fro_err   optional: ||B - phi_q phi_k^T||_F / ||B||_F (exact, fp64).
+ *  energy        optional: sum_{r<R} s_r^2 / ||B||_F^2.
+ * Synchronous; uses the host's cores. Allocates host memory internally.
+ */
+int fb_svd_factors_host(const double *bias_host, int N, int R, int oversample,
+                        int power_iters, uint64_t seed, float *phi_q_host,
+                        float *phi_k_host, double *rel_fro_err, double *energy);
+
+/*
+ * Synchronises `stream`, then reads and clears the library's device flag:
+ * FB_ERR_TIMEOUT if a kernel's bounded wait ran out, FB_ERR_RANGE if a factor
+ * overflowed fp16 in the preparation step, FB_OK otherwise (FB_ERR_CUDA if
+ * the synchronisation itself failed). The flag is per device and shared by
+ * all calls on that device.
+ */
+int fb_check_device_error(void *stream);
+
+/*
+ * Self-test of the failure path: launches one CTA whose pipeline wait is on
+ * a barrier that nothing completes, with a limit of `limit_ms` milliseconds
+ * (1 <= limit_ms <= 2000). The kernel gives up, records FB_ERR_TIMEOUT in
+ * the device flag and exits normally; the context stays usable. Returns the
+ * launch status; read the outcome with fb_check_device_error().
+ */
+int fb_selftest_wait_timeout(int limit_ms, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FLASHBIAS_H_ */

@@ -20,7 +20,7 @@ import numpy as np
 
 from . import build as _build
 
-BIAS_NONE, BIAS_DENSE, BIAS_LOWRANK, BIAS_SANDWICH, BIAS_ALIBI = 0, 1, 2, 3, 4
+BIAS_NONE, BIAS_DENSE, BIAS_LOWRANK, BIAS_SANDWICH, BIAS_ALIBI, BIAS_TOEPLITZ, BIAS_GRID = range(7)
 
 
 class _Bias(ctypes.Structure):
@@ -33,6 +33,8 @@ class _Bias(ctypes.Structure):
         ("R", ctypes.c_int),
         ("C", ctypes.c_int),
         ("slope", ctypes.c_double),
+        ("table", ctypes.c_void_p),
+        ("n", ctypes.c_int64),
     ]
 
 
@@ -59,6 +61,8 @@ def _load():
         lib.fbo_alibi_slope.restype = ctypes.c_double
         lib.fbo_alibi_factors.argtypes = [ctypes.c_int64, ctypes.c_double, P, P]
         lib.fbo_alibi_factors.restype = ctypes.c_int
+        lib.fbo_num_threads.argtypes = []
+        lib.fbo_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -75,7 +79,7 @@ class HeadBias:
     """The bias of one head, by kind. Keeps its arrays alive for the C call."""
 
     def __init__(self, kind: int, dense=None, phi_q=None, phi_k=None, C: int = 0,
-                 slope: float = 0.0):
+                 slope: float = 0.0, table=None, n: int = 0):
         self.kind = kind
         self._keep = []
         self.s = _Bias()
@@ -96,6 +100,13 @@ class HeadBias:
             self.s.C = int(C)
         elif kind == BIAS_ALIBI:
             self.s.slope = float(slope)
+        elif kind in (BIAS_TOEPLITZ, BIAS_GRID):
+            table = _f64(table).ravel()
+            want = 2 * n - 1 if kind == BIAS_TOEPLITZ else (2 * n - 1) ** 2
+            assert table.size == want
+            self._keep.append(table)
+            self.s.table = table.ctypes.data
+            self.s.n = int(n)
 
     @staticmethod
     def none():
@@ -116,6 +127,16 @@ class HeadBias:
     @staticmethod
     def alibi(slope: float):
         return HeadBias(BIAS_ALIBI, slope=slope)
+
+    @staticmethod
+    def toeplitz(table, N: int):
+        """b_ij = table[i - j + N - 1] (table over the 2N-1 offsets)."""
+        return HeadBias(BIAS_TOEPLITZ, table=table, n=N)
+
+    @staticmethod
+    def grid(table, g: int):
+        """b_ij = table[dx + g - 1, dy + g - 1] for tokens on a g x g grid (n = g*y + x)."""
+        return HeadBias(BIAS_GRID, table=table, n=g)
 
     def value(self, i: int, j: int) -> float:
         return _load().fbo_bias_value(ctypes.byref(self.s), int(i), int(j))
@@ -165,6 +186,11 @@ def attention(q, k, v, bias_of, scale: float, causal: bool, rows=None, heads=Non
     for (b, h) in pairs:
         O[b, h], L[b, h] = out_o[(b, h)], out_l[(b, h)]
     return O, L
+
+
+def num_threads() -> int:
+    """Host threads the oracle's parallel loops use."""
+    return _load().fbo_num_threads()
 
 
 def sandwich_factors(N: int, C: int) -> np.ndarray:

@@ -32,12 +32,22 @@
  *   SANDWICH  b_ij = sum_{k=1}^{C/2} cos((i-j) / 10000^{2k/C}) (rebuttal,
  *             reply to Reviewer UJUf, Q1 (1)).
  *   ALIBI     b_ij = -m (i - j) (FlashBias Example 3.4, ALiBi; slope m given).
+ *   TOEPLITZ  b_ij = table[i - j + N - 1]: a bias given by its values on the
+ *             2N-1 offsets (how a materialised Sandwich or ALiBi bias is
+ *             stored), for the dense comparison path.
+ *   GRID      tokens on a g x g grid, token n = g*y + x; b_ij =
+ *             table[(x_i - x_j + g - 1) * (2g - 1) + (y_i - y_j + g - 1)]: a
+ *             bias given by its values on the 2-D offsets (Example 3.5,
+ *             spatial distance), for the dense comparison path.
  *
  * Parity of every function here is pinned by the tests in tests/ against
  * closed forms, invariants, a library attention routine and a 50-digit
  * evaluation; none of those pins reuses this code.
  */
 #include <math.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -47,6 +57,8 @@
 #define FBO_BIAS_LOWRANK 2
 #define FBO_BIAS_SANDWICH 3
 #define FBO_BIAS_ALIBI 4
+#define FBO_BIAS_TOEPLITZ 5
+#define FBO_BIAS_GRID 6
 
 /* Per-head bias description. Pointers refer to fp64 host arrays. */
 typedef struct {
@@ -58,6 +70,8 @@ typedef struct {
   int R;
   int C;        /* SANDWICH: channel count C (even) */
   double slope; /* ALIBI: m */
+  const double *table; /* TOEPLITZ: [2N-1]; GRID: [(2g-1) * (2g-1)] */
+  int64_t n;           /* TOEPLITZ: N; GRID: g */
 } fbo_bias;
 
 /* b_ij straight from the definition of its kind. */
@@ -83,6 +97,13 @@ static double fbo_bias_at(const fbo_bias *b, int64_t i, int64_t j) {
   }
   case FBO_BIAS_ALIBI:
     return -b->slope * (double)(i - j);
+  case FBO_BIAS_TOEPLITZ:
+    return b->table[i - j + b->n - 1];
+  case FBO_BIAS_GRID: {
+    const int64_t g = b->n;
+    const int64_t dx = i % g - j % g, dy = i / g - j / g;
+    return b->table[(dx + g - 1) * (2 * g - 1) + (dy + g - 1)];
+  }
   default:
     return NAN;
   }
@@ -203,4 +224,13 @@ int fbo_alibi_factors(int64_t N, double m, double *phi_q, double *phi_k) {
     phi_k[2 * i + 1] = m * (double)i;
   }
   return 0;
+}
+
+/* Number of host threads the oracle's parallel loops use. */
+int fbo_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
 }

@@ -142,3 +142,53 @@ def sample_rows(N: int, count: int, seed: int) -> np.ndarray:
     if count > 2:
         rows.update(g.choice(N, size=count - 2, replace=False).tolist())
     return np.array(sorted(rows), dtype=np.int64)
+
+
+# --- dense biases for the comparison path -----------------------------------
+#
+# The dense-bias path reads a materialised bias. For biases that depend only
+# on i - j (Sandwich, ALiBi) the workload builds a table over the 2N-1
+# offsets, rounds it to bf16 once, and lays the N x N matrix out on the device
+# by pure data movement (a strided view and a copy), so host and device hold
+# bit-identical values.
+
+def sandwich_offset_table(N: int, C: int) -> np.ndarray:
+    """f(delta) = sum_{k=1}^{C/2} cos(delta / 10000^{2k/C}) for delta = -(N-1)..N-1 (fp64)."""
+    delta = np.arange(-(N - 1), N, dtype=np.float64)
+    k = np.arange(1, C // 2 + 1, dtype=np.float64)
+    w = np.power(10000.0, -2.0 * k / C)
+    return np.cos(delta[:, None] * w[None, :]).sum(axis=1)
+
+
+def alibi_offset_table(N: int, slope: float) -> np.ndarray:
+    """f(delta) = -m * delta for delta = -(N-1)..N-1 (fp64)."""
+    return -slope * np.arange(-(N - 1), N, dtype=np.float64)
+
+
+def toeplitz_rows(table: np.ndarray, N: int, rows) -> np.ndarray:
+    """Rows of the N x N matrix M[i, j] = table[i - j + N - 1] (host)."""
+    rows = np.asarray(rows)
+    j = np.arange(N)
+    return table[rows[:, None] - j[None, :] + N - 1]
+
+
+def toeplitz_device(table_bf16: np.ndarray, N: int, device):
+    """N x N bf16 device matrix M[i, j] = table[i - j + N - 1] by data movement only."""
+    import torch
+    bits = torch.from_numpy(bf16_bits(table_bf16).view(np.int16)).to(device)
+    t = bits.view(torch.bfloat16)
+    w = torch.flip(t, dims=[0])  # w[k] = table[2N-2-k]
+    # row i' = N-1-i of the strided view reads w[i' + j] = table[i - j + N - 1]
+    v = torch.as_strided(w, size=(N, N), stride=(1, 1))
+    return torch.flip(v, dims=[0]).contiguous()
+
+
+def bf16_tensor(x: np.ndarray, device):
+    """Device bf16 tensor holding the bf16-representable fp32 values x exactly."""
+    import torch
+    return torch.from_numpy(bf16_bits(x).view(np.int16)).to(device).view(torch.bfloat16)
+
+
+def alibi_slope(h: int, H: int) -> float:
+    """Slope of head h (0-based) of H in the ALiBi workload: 2^(-8(h+1)/H)."""
+    return 2.0 ** (-8.0 * (h + 1) / H)

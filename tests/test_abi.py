@@ -1,0 +1,159 @@
+"""Host-side checks of libflashbias (no GPU): the library loads, exports every
+symbol the header declares, rejects bad arguments before any launch, and its
+host truncated SVD matches the oracle's library SVD."""
+import ctypes
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+
+import attention_rank_additive_b200 as fb
+import oracle
+import seeded_inputs as si
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from attention_rank_additive_b200 import build
+    build.build()
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "flashbias.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fb_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_symbols_exported():
+    declared = _declared()
+    assert set(declared) == set(fb.EXPORTED)
+    L = ctypes.CDLL(fb.lib_path)
+    for name in declared:
+        assert hasattr(L, name), name
+
+
+def test_status_strings_and_version():
+    assert fb.fb_status_str(fb.FB_OK) == "FB_OK"
+    assert fb.fb_status_str(fb.FB_ERR_TIMEOUT) == "FB_ERR_TIMEOUT"
+    assert fb.fb_status_str(99) == "FB_ERR_UNKNOWN"
+    assert fb.fb_version() >= 100
+
+
+def test_workspace_bytes():
+    assert fb.fb_attn_workspace_bytes(8, 12, 2048, 0, 0, 0) == 0
+    # broadcast Sandwich factors: one [N, 64] fp16 slice per side
+    assert fb.fb_attn_workspace_bytes(8, 12, 2048, 64, 0, 0) == 2 * 2048 * 64 * 2
+    # rank 8 pads to 16 columns; per-head factors
+    assert fb.fb_attn_workspace_bytes(4, 8, 4096, 8, 0, 4096 * 8) == 2 * 8 * 4096 * 16 * 2
+    # rank <= 4 keeps fp32 in 16-byte rows
+    assert fb.fb_attn_workspace_bytes(4, 16, 8192, 2, 0, 8192 * 2) == 2 * 16 * 8192 * 16
+    assert fb.fb_attn_workspace_bytes(1, 1, 17, 3, 0, 0) == 2 * 512  # rounded to 256 B
+    assert fb.fb_attn_workspace_bytes(1, 1, 16, 129, 0, 0) == 0  # out of range -> 0
+
+
+FAKE = 1 << 20  # a 16-byte aligned address; never dereferenced by the checks below
+
+
+def _fwd(**kw):
+    a = dict(dt=fb.FB_BF16, B=1, H=1, N=128, d=64, Q=FAKE, K=FAKE, V=FAKE, R=0, phi_q=0, phi_k=0, phi_bstride=0,
+             phi_hstride=0, scale=0.125, causal=0, O=FAKE, LSE=FAKE, workspace=0, workspace_bytes=0, stream=None)
+    a.update(kw)
+    return fb.fb_attn_fwd(**a)
+
+
+def test_forward_rejects_bad_arguments_before_launch():
+    assert _fwd(Q=0) == fb.FB_ERR_INVALID_ARG
+    assert _fwd(LSE=0) == fb.FB_ERR_INVALID_ARG
+    assert _fwd(Q=FAKE + 8) == fb.FB_ERR_INVALID_ARG  # misaligned
+    assert _fwd(scale=0.0) == fb.FB_ERR_INVALID_ARG
+    assert _fwd(scale=-1.0) == fb.FB_ERR_INVALID_ARG
+    assert _fwd(scale=float("nan")) == fb.FB_ERR_INVALID_ARG
+    assert _fwd(R=129) == fb.FB_ERR_UNSUPPORTED
+    assert _fwd(R=-1) == fb.FB_ERR_UNSUPPORTED
+    assert _fwd(R=8) == fb.FB_ERR_INVALID_ARG  # factors missing
+    assert _fwd(R=8, phi_q=FAKE, phi_k=FAKE, phi_bstride=-1) == fb.FB_ERR_INVALID_ARG
+    assert _fwd(d=12) == fb.FB_ERR_UNSUPPORTED
+    assert _fwd(d=136) == fb.FB_ERR_UNSUPPORTED
+    assert _fwd(N=0) == fb.FB_ERR_UNSUPPORTED
+    assert _fwd(B=0) == fb.FB_ERR_UNSUPPORTED
+    assert _fwd(dt=7) == fb.FB_ERR_UNSUPPORTED
+    assert _fwd(dt=fb.FB_F32, d=6) == fb.FB_ERR_UNSUPPORTED
+    # workspace missing / too small / misaligned
+    assert _fwd(R=8, phi_q=FAKE, phi_k=FAKE) == fb.FB_ERR_WORKSPACE
+    need = fb.fb_attn_workspace_bytes(1, 1, 128, 8, 0, 0)
+    assert _fwd(R=8, phi_q=FAKE, phi_k=FAKE, workspace=FAKE, workspace_bytes=need - 1) == fb.FB_ERR_WORKSPACE
+    assert _fwd(R=8, phi_q=FAKE, phi_k=FAKE, workspace=FAKE + 16, workspace_bytes=need) == fb.FB_ERR_WORKSPACE
+
+
+def _dense(**kw):
+    a = dict(dt=fb.FB_BF16, B=1, H=1, N=128, d=64, Q=FAKE, K=FAKE, V=FAKE, Bias=FAKE, bias_bstride=0, bias_hstride=0,
+             scale=0.125, causal=0, O=FAKE, LSE=FAKE, stream=None)
+    a.update(kw)
+    return fb.fb_attn_dense_bias_fwd(**a)
+
+
+def test_dense_rejects_bad_arguments_before_launch():
+    assert _dense(Bias=0) == fb.FB_ERR_INVALID_ARG
+    assert _dense(Bias=FAKE + 2) == fb.FB_ERR_INVALID_ARG
+    assert _dense(bias_hstride=-8) == fb.FB_ERR_INVALID_ARG
+    assert _dense(N=130) == fb.FB_ERR_UNSUPPORTED  # bias row pitch must be 16-byte aligned
+    assert _dense(bias_hstride=12, H=2) == fb.FB_ERR_UNSUPPORTED
+    assert _dense(scale=0.0) == fb.FB_ERR_INVALID_ARG
+
+
+def test_factor_generators_reject_bad_arguments():
+    assert fb.fb_factors_sandwich(16, 7, FAKE, FAKE, None) == fb.FB_ERR_INVALID_ARG
+    assert fb.fb_factors_sandwich(0, 8, FAKE, FAKE, None) == fb.FB_ERR_INVALID_ARG
+    assert fb.fb_factors_sandwich(16, 130, FAKE, FAKE, None) == fb.FB_ERR_INVALID_ARG
+    assert fb.fb_factors_alibi(0, 16, FAKE, FAKE, None) == fb.FB_ERR_INVALID_ARG
+    assert fb.fb_factors_alibi(4, 16, 0, FAKE, None) == fb.FB_ERR_INVALID_ARG
+    assert fb.fb_selftest_wait_timeout(0, None) == fb.FB_ERR_INVALID_ARG
+    assert fb.fb_selftest_wait_timeout(5000, None) == fb.FB_ERR_INVALID_ARG
+
+
+# --- host truncated SVD (product) against the oracle's library SVD ----------
+
+def _known_spectrum(N, sigma, seed):
+    rng = np.random.Generator(np.random.PCG64(seed))
+    U, _ = np.linalg.qr(rng.standard_normal((N, len(sigma))))
+    V, _ = np.linalg.qr(rng.standard_normal((N, len(sigma))))
+    return U @ np.diag(sigma) @ V.T
+
+
+def test_svd_host_known_spectrum():
+    sigma = np.array([40.0, 15.0, 7.0, 3.0, 1.0, 0.3, 0.1, 0.03, 0.01, 0.003])
+    Bm = _known_spectrum(257, sigma, 5)
+    for R in (1, 4, 8):
+        pq, pk, rel, energy = fb.svd_factors(Bm, R, oversample=16, power_iters=2, seed=3)
+        want_rel = math.sqrt(np.sum(sigma[R:] ** 2) / np.sum(sigma ** 2))
+        assert abs(rel - want_rel) < 1e-6
+        assert abs(energy - np.sum(sigma[:R] ** 2) / np.sum(sigma ** 2)) < 1e-6
+        opq, opk, orel, _ = oracle.truncated_svd_factors(Bm, R)
+        np.testing.assert_allclose(pq.astype(np.float64) @ pk.T.astype(np.float64), opq @ opk.T, atol=2e-5)
+
+
+def test_svd_host_rbf_field_matches_oracle():
+    grid, M, R = 24, 32, 8
+    om, ph = si.rbf_params(2, M)
+    dense = si.rbf_dense(si.rbf_offset_table(om, ph, grid), grid)
+    for h in range(2):
+        pq, pk, rel, energy = fb.svd_factors(dense[h], R, oversample=64, power_iters=1, seed=11)
+        opq, opk, orel, oen = oracle.truncated_svd_factors(dense[h], R)
+        assert abs(rel - orel) < 1e-6 and abs(energy - oen) < 1e-6
+        np.testing.assert_allclose(pq.astype(np.float64) @ pk.T.astype(np.float64), opq @ opk.T,
+                                   atol=1e-5 * np.abs(dense[h]).max())
+
+
+def test_svd_host_rejects_bad_arguments():
+    b = np.zeros((4, 4))
+    out = np.zeros((4, 8), dtype=np.float32)
+    assert fb.fb_svd_factors_host(b.ctypes.data, 4, 0, 4, 1, 0, out.ctypes.data, out.ctypes.data, None, None) \
+        == fb.FB_ERR_INVALID_ARG
+    assert fb.fb_svd_factors_host(b.ctypes.data, 4, 5, 4, 1, 0, out.ctypes.data, out.ctypes.data, None, None) \
+        == fb.FB_ERR_INVALID_ARG
+    assert fb.fb_svd_factors_host(None, 4, 2, 4, 1, 0, out.ctypes.data, out.ctypes.data, None, None) \
+        == fb.FB_ERR_INVALID_ARG

@@ -1,0 +1,203 @@
+"""GPU parity of every kernel against the fp64 oracle on small seeded inputs
+that still span several 128-row tiles and a ragged tail, plus the edge cases
+(one row, d not a multiple of 16, every factor path, broadcast layouts) and
+the failure-path checks (fp16 range flag, bounded-wait timeout)."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import HeadBias
+import seeded_inputs as si
+from gpu_util import compare, dev, host
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+import attention_rank_additive_b200 as fb  # noqa: E402
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from attention_rank_additive_b200 import build
+    build.build()
+    fb.lib()
+    yield
+    torch.cuda.synchronize()
+
+
+def _no_device_error():
+    assert fb.fb_check_device_error(torch.cuda.current_stream().cuda_stream) == fb.FB_OK
+
+
+# ---------------------------------------------------------------- factors
+
+@pytest.mark.parametrize("N,C", [(2048, 64), (5, 8), (300, 2), (1, 128)])
+def test_sandwich_factors_match_oracle(N, C):
+    phi = fb.factors_sandwich(N, C)
+    torch.cuda.synchronize()
+    ref = oracle.sandwich_factors(N, C)
+    np.testing.assert_allclose(host(phi), ref, rtol=0, atol=1e-6)
+
+
+@pytest.mark.parametrize("H,N", [(16, 8192), (3, 100)])
+def test_alibi_factors_match_oracle(H, N):
+    pq, pk = fb.factors_alibi(H, N)
+    torch.cuda.synchronize()
+    pq, pk = host(pq), host(pk)
+    for h in range(H):
+        rq, rk = oracle.alibi_factors(N, oracle.alibi_slope(h, H))
+        np.testing.assert_allclose(pq[h], rq, rtol=1e-7, atol=0)
+        np.testing.assert_allclose(pk[h], rk, rtol=1e-7, atol=0)
+
+
+# ------------------------------------------------------- fused bf16 sweeps
+
+def _run_fused(B, H, N, d, R, causal, seed, std=None, layout="bhnr", dtype="bf16"):
+    q, k, v = si.qkv(B, H, N, d, seed, dtype)
+    scale = 1.0 / math.sqrt(d)
+    pq = pk = None
+    if R > 0:
+        std = std if std is not None else math.sqrt(1.0 / R)
+        shape = {"nr": (N, R), "hnr": (H, N, R), "bhnr": (B, H, N, R)}[layout]
+        pq, pk = si.random_factors(shape, std, seed + 7)
+    o, l = fb.attn(dev(q, dtype), dev(k, dtype), dev(v, dtype),
+                   None if pq is None else dev(pq, "f32"), None if pk is None else dev(pk, "f32"),
+                   scale=scale, causal=causal)
+    torch.cuda.synchronize()
+    _no_device_error()
+
+    def bias_of(b, h):
+        if R == 0:
+            return HeadBias.none()
+        if layout == "nr":
+            return HeadBias.lowrank(pq, pk)
+        if layout == "hnr":
+            return HeadBias.lowrank(pq[h], pk[h])
+        return HeadBias.lowrank(pq[b, h], pk[b, h])
+
+    heads = [(0, 0), (B - 1, H - 1)] if B * H > 2 else [(b, h) for b in range(B) for h in range(H)]
+    ro, rl = oracle.attention(q, k, v, bias_of, scale, causal, heads=heads)
+    og, lg = host(o), host(l)
+    for (b, h) in heads:
+        compare(og[b, h], lg[b, h], ro[(b, h)], rl[(b, h)], dtype, f"B{B} H{H} N{N} d{d} R{R} c{causal} ({b},{h})")
+
+
+SWEEP = [
+    # B, H, N, d, R, causal
+    (1, 1, 1, 64, 0, False),
+    (1, 1, 1, 64, 8, True),
+    (1, 2, 17, 16, 8, False),
+    (1, 2, 128, 64, 64, True),
+    (2, 1, 129, 64, 64, True),
+    (1, 2, 255, 24, 32, False),
+    (1, 1, 256, 128, 2, True),
+    (1, 2, 300, 128, 2, False),
+    (1, 1, 300, 8, 3, True),
+    (1, 1, 384, 32, 1, True),
+    (1, 2, 513, 40, 4, False),
+    (1, 1, 513, 72, 5, True),
+    (1, 1, 400, 96, 100, False),
+    (1, 1, 260, 120, 128, True),
+    (1, 1, 640, 128, 16, True),
+    (1, 2, 700, 64, 0, True),
+    (2, 2, 1000, 16, 8, False),
+]
+
+
+@pytest.mark.parametrize("qt", ["1", "2"])
+@pytest.mark.parametrize("B,H,N,d,R,causal", SWEEP)
+def test_fused_bf16_matches_oracle(monkeypatch, qt, B, H, N, d, R, causal):
+    monkeypatch.setenv("FLASHBIAS_QUERY_TILES", qt)
+    _run_fused(B, H, N, d, R, causal, seed=100 + N + d + R)
+
+
+@pytest.mark.parametrize("layout", ["nr", "hnr", "bhnr"])
+@pytest.mark.parametrize("R", [2, 16])
+def test_fused_factor_layouts(layout, R):
+    _run_fused(2, 3, 200, 64, R, True, seed=7, layout=layout)
+
+
+def test_fused_default_plan_many_heads():
+    # enough (batch, head) pairs for the two-tile plan on its own
+    _run_fused(4, 40, 512, 64, 32, True, seed=11)
+
+
+def test_fused_f32_matches_oracle_tight():
+    for (B, H, N, d, R, causal) in [(1, 2, 256, 64, 8, False), (1, 1, 1, 4, 0, True), (2, 1, 300, 128, 5, True),
+                                    (1, 3, 33, 12, 128, False)]:
+        _run_fused(B, H, N, d, R, causal, seed=5, dtype="f32")
+
+
+# ------------------------------------------------------------ dense path
+
+def _run_dense(B, H, N, d, causal, layout, dtype, seed):
+    q, k, v = si.qkv(B, H, N, d, seed, dtype)
+    scale = 1.0 / math.sqrt(d)
+    rng = si.generator(seed + 3)
+    shape = {"nn": (N, N), "hnn": (H, N, N), "bhnn": (B, H, N, N)}[layout]
+    bias = (rng.standard_normal(size=shape) * 2.0).astype(np.float32)
+    if dtype == "bf16":
+        bias = si.round_to_bf16(bias)
+    o, l = fb.attn_dense_bias(dev(q, dtype), dev(k, dtype), dev(v, dtype), dev(bias, dtype), scale=scale,
+                              causal=causal)
+    torch.cuda.synchronize()
+    _no_device_error()
+
+    def bias_of(b, h):
+        return HeadBias.dense({"nn": bias, "hnn": bias[h] if layout == "hnn" else None,
+                               "bhnn": bias[b, h] if layout == "bhnn" else None}[layout])
+
+    heads = [(0, 0), (B - 1, H - 1)] if B * H > 2 else [(b, h) for b in range(B) for h in range(H)]
+    ro, rl = oracle.attention(q, k, v, bias_of, scale, causal, heads=heads)
+    og, lg = host(o), host(l)
+    for (b, h) in heads:
+        compare(og[b, h], lg[b, h], ro[(b, h)], rl[(b, h)], dtype, f"dense N{N} d{d} c{causal} {layout} ({b},{h})")
+
+
+@pytest.mark.parametrize("qt", ["1", "2"])
+@pytest.mark.parametrize("B,H,N,d,causal,layout", [
+    (1, 1, 8, 64, False, "nn"),
+    (1, 2, 136, 16, True, "hnn"),
+    (2, 2, 256, 24, False, "bhnn"),
+    (1, 1, 264, 128, True, "nn"),
+    (1, 2, 520, 64, True, "bhnn"),
+    (1, 1, 384, 40, False, "hnn"),
+])
+def test_dense_bf16_matches_oracle(monkeypatch, qt, B, H, N, d, causal, layout):
+    monkeypatch.setenv("FLASHBIAS_QUERY_TILES", qt)
+    _run_dense(B, H, N, d, causal, layout, "bf16", seed=200 + N)
+
+
+@pytest.mark.parametrize("B,H,N,d,causal,layout", [(1, 2, 256, 64, False, "hnn"), (2, 1, 77, 8, True, "bhnn")])
+def test_dense_f32_matches_oracle(B, H, N, d, causal, layout):
+    _run_dense(B, H, N, d, causal, layout, "f32", seed=300 + N)
+
+
+# ------------------------------------------------------ failure paths
+
+def test_fp16_range_flag():
+    N, d, R = 128, 64, 8
+    q, k, v = si.qkv(1, 1, N, d, 9, "bf16")
+    pq = np.full((N, R), 1.0e6, dtype=np.float32)  # / scale overflows fp16
+    fb.attn(dev(q, "bf16"), dev(k, "bf16"), dev(v, "bf16"), dev(pq, "f32"), dev(pq, "f32"), causal=False)
+    assert fb.fb_check_device_error(torch.cuda.current_stream().cuda_stream) == fb.FB_ERR_RANGE
+    _no_device_error()  # the flag was cleared by the read
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    s = torch.cuda.current_stream().cuda_stream
+    assert fb.fb_selftest_wait_timeout(20, s) == fb.FB_OK
+    assert fb.fb_check_device_error(s) == fb.FB_ERR_TIMEOUT
+    _no_device_error()
+    _run_fused(1, 1, 200, 64, 8, True, seed=3)  # the context is still usable
+
+
+def test_unsupported_dense_pitch_returns_before_launch():
+    x = torch.zeros((1, 1, 130, 64), device="cuda", dtype=torch.bfloat16)
+    b = torch.zeros((130, 130), device="cuda", dtype=torch.bfloat16)
+    with pytest.raises(fb.FlashBiasError) as e:
+        fb.attn_dense_bias(x, x, x, b)
+    assert e.value.status == fb.FB_ERR_UNSUPPORTED

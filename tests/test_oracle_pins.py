@@ -261,3 +261,22 @@ def test_bf16_rounding_is_round_to_nearest_even():
     np.testing.assert_array_equal(r, t)
     y = si.normal((4096,), 5)
     np.testing.assert_array_equal(si.round_to_bf16(y), torch.from_numpy(y).to(torch.bfloat16).float().numpy())
+
+
+def test_offset_table_kinds():
+    """TOEPLITZ and GRID biases: the offset-table forms of the dense inputs."""
+    N, C = 200, 16
+    tab = si.sandwich_offset_table(N, C)
+    tb = HeadBias.toeplitz(tab, N)
+    sw = HeadBias.sandwich(C)
+    for i, j in [(0, 0), (199, 0), (0, 199), (57, 123)]:
+        assert abs(tb.value(i, j) - sw.value(i, j)) < 1e-12
+    np.testing.assert_array_equal(tb.dense_matrix(N), si.toeplitz_rows(tab, N, np.arange(N)))
+    m = oracle.alibi_slope(2, 8)
+    ta = HeadBias.toeplitz(si.alibi_offset_table(N, m), N)
+    for i, j in [(0, 0), (199, 0), (5, 9)]:
+        assert ta.value(i, j) == HeadBias.alibi(m).value(i, j)
+    g = 9
+    om, ph = si.rbf_params(1, 4)
+    t2 = si.rbf_offset_table(om, ph, g)
+    np.testing.assert_array_equal(HeadBias.grid(t2[0], g).dense_matrix(g * g), si.rbf_dense(t2, g)[0])
