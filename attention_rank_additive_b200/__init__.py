@@ -21,7 +21,7 @@ __all__ = [
     "FB_ERR_TIMEOUT", "FB_F32", "FB_BF16", "FlashBiasError", "lib", "lib_path", "EXPORTED",
     "fb_status_str", "fb_version", "fb_attn_workspace_bytes", "fb_attn_fwd", "fb_attn_dense_bias_fwd",
     "fb_factors_sandwich", "fb_factors_alibi", "fb_svd_factors_host", "fb_check_device_error",
-    "fb_selftest_wait_timeout", "attn", "attn_dense_bias", "factors_sandwich", "factors_alibi", "svd_factors",
+    "fb_selftest_wait_timeout", "fb_attn_fwd_noalloc", "attn", "attn_dense_bias", "factors_sandwich", "factors_alibi", "svd_factors",
     "attn_flops",
 ]
 
@@ -35,7 +35,7 @@ lib_path = os.path.join(_HERE, "libflashbias.so")
 EXPORTED = (
     "fb_status_str", "fb_version", "fb_attn_workspace_bytes", "fb_attn_fwd", "fb_attn_dense_bias_fwd",
     "fb_factors_sandwich", "fb_factors_alibi", "fb_svd_factors_host", "fb_check_device_error",
-    "fb_selftest_wait_timeout",
+    "fb_selftest_wait_timeout", "fb_attn_fwd_noalloc",
 )
 
 
@@ -64,6 +64,9 @@ def lib() -> ctypes.CDLL:
         L.fb_attn_fwd.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, i32, vp, vp, i64, i64, f32, i32, vp, vp, vp,
                                   sz, vp]
         L.fb_attn_fwd.restype = i32
+        L.fb_attn_fwd_noalloc.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, i32, vp, vp, i64, i64, f32, i32, vp,
+                                          vp, vp]
+        L.fb_attn_fwd_noalloc.restype = i32
         L.fb_attn_dense_bias_fwd.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, i64, i64, f32, i32, vp, vp, vp]
         L.fb_attn_dense_bias_fwd.restype = i32
         L.fb_factors_sandwich.argtypes, L.fb_factors_sandwich.restype = [i32, i32, vp, vp, vp], i32
@@ -94,6 +97,16 @@ def fb_attn_fwd(dt, B, H, N, d, Q, K, V, R, phi_q, phi_k, phi_bstride, phi_hstri
                 workspace, workspace_bytes, stream) -> int:
     return lib().fb_attn_fwd(dt, B, H, N, d, Q, K, V, R, phi_q, phi_k, phi_bstride, phi_hstride, scale, causal, O,
                              LSE, workspace, workspace_bytes, stream)
+
+
+def fb_attn_fwd_noalloc(dt, B, H, N, d, Q, K, V, R, phi_q, phi_k, phi_bstride, phi_hstride, scale, causal, O, LSE,
+                        stream) -> int:
+    """fb_attn_fwd without a caller workspace, for callers that cannot allocate
+    device memory: the prepared factors go to the library's fixed 8 MiB device
+    array (larger needs return FB_ERR_WORKSPACE). Calls that overlap on the GPU
+    share that array and must be serialised by the caller."""
+    return lib().fb_attn_fwd_noalloc(dt, B, H, N, d, Q, K, V, R, phi_q, phi_k, phi_bstride, phi_hstride, scale,
+                                     causal, O, LSE, stream)
 
 
 def fb_attn_dense_bias_fwd(dt, B, H, N, d, Q, K, V, Bias, bias_bstride, bias_hstride, scale, causal, O, LSE,

@@ -17,7 +17,10 @@
  *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
  *    NULL = the legacy default stream).
  *  - The caller owns all memory. Besides caller-provided workspace the
- *    library allocates no device memory.
+ *    library allocates no device memory at run time; its only device
+ *    storage is module globals (a flag word per device and the fixed 8 MiB
+ *    scratch array of fb_attn_fwd_noalloc), reserved when the library's
+ *    module is loaded on a device.
  *  - Argument, shape, alignment and range errors are reported synchronously,
  *    before anything is launched. A launch failure returns FB_ERR_CUDA.
  *  - Kernel-side conditions (a pipeline wait that ran out, a factor that
@@ -105,6 +108,40 @@ int fb_attn_fwd(int dt, int B, int H, int N, int d,
                 float scale, int causal,
                 void *O, float *LSE,
                 void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * fb_attn_fwd for callers that cannot allocate device memory. (The FlashBias
+ * paper has no counterpart: this is an interface convenience.)
+ *
+ * Who needs it: code that only receives the tensors it works on and has no
+ * allocator of its own to call (a plugin or operator interface whose
+ * signature carries inputs and outputs only, a host framework that owns every
+ * device buffer through its own pool), and code that must not call
+ * cudaMalloc on its path (it synchronises the device and can fail under
+ * memory pressure). Such callers cannot supply fb_attn_fwd's workspace.
+ *
+ * Same arguments and results as fb_attn_fwd, without workspace and
+ * workspace_bytes. The prepared factors live instead in a fixed 8 MiB array
+ * in the library's device memory, reserved on every device that loads the
+ * library until the process exits. A call whose prepared factors need more
+ * than 8 MiB (fb_attn_workspace_bytes(...) > 8 MiB) returns FB_ERR_WORKSPACE
+ * before anything is launched; fb_attn_fwd with a caller workspace has no
+ * such limit. The function allocates nothing.
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it; make that first call before capturing the
+ * stream into a graph. All calls on a device share the one array and it
+ * keeps the last call's contents; the preparation step rewrites every byte a
+ * call reads, so nothing needs clearing, but calls that can overlap on the
+ * GPU (on different streams, or from different host threads) race on it and
+ * must be serialised by the caller.
+ */
+int fb_attn_fwd_noalloc(int dt, int B, int H, int N, int d,
+                        const void *Q, const void *K, const void *V,
+                        int R, const float *phi_q, const float *phi_k,
+                        int64_t phi_bstride, int64_t phi_hstride,
+                        float scale, int causal,
+                        void *O, float *LSE, void *stream);
 
 /*
  * Comparison path, "FlashAttention w/ Bias" (FlashBias Figure 1(c)): the same
