@@ -23,13 +23,15 @@
 //   warp 4QT        TMA producer (one thread): Q|phi_q once, then K|phi_k and
 //                   V per 128-key step into a KS-deep ring, plus the
 //                   softmax-side tiles (dense bias / rank<=4 factors).
-//   warp 4QT+1      TMEM allocator and MMA issuer (one thread).
+//   warp 4QT+1      TMEM allocator and MMA issuer (one elected lane).
 // TMEM columns: S_t at 128 t, O_t at 128 QT + 128 t; P_t (bf16) overwrites
 // the first 64 columns of S_t and feeds the PV MMA as the TMEM A operand.
-// MMA issue order per key step i: S_0(i), PV_1(i-1), S_1(i), PV_0(i). With
+// MMA issue order per key step i: S_0(i), PV_1(i-1), S_1(i), PV_0(i), so the
+// tensor core works on one tile while the softmax of the other runs. With
 // that order the commit that publishes S_t(i) also covers PV_t(i-1), so the
-// softmax may rescale O_t right after seeing S_t(i), and S_t(i+1) is issued
-// after PV_t(i) has been issued (tcgen05 MMAs of one thread run in order).
+// softmax may rescale O_t right after seeing S_t(i), and S_t(i+1) (which
+// overwrites P_t(i)) is issued after PV_t(i) (tcgen05 MMAs of one thread run
+// in order).
 #include <algorithm>
 
 #include "fb_internal.h"
@@ -40,6 +42,10 @@ namespace fb {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows by > 2^8
+// Of every 16 element pairs of P, this many get exp2 from the packed FMA-pipe
+// polynomial (ex2_fma_pair) and the rest from the MUFU unit, which balances
+// the MUFU against the issue slots of the two softmax warps per scheduler.
+constexpr int kEmuPairs = 4;
 constexpr uint32_t kSmemLimit = 227u * 1024u;
 
 template <int DP, int RP, int MODE, int QT>
@@ -65,10 +71,29 @@ struct Sm100Cfg {
                                     : 0;
   static constexpr int KS = KS_FIT > 3 ? 3 : KS_FIT;
   static constexpr uint32_t SMEM = FIXED + uint32_t(KS) * STAGE + CTRL + ALIGN_SLACK;
-  static constexpr int THREADS = QT * 128 + 64;
+  // QT softmax warpgroups + one warpgroup holding the producer warp, the MMA
+  // warp and two idle warps. Registers are moved from that warpgroup to the
+  // softmax warpgroups with setmaxnreg: the launch allocation is
+  // THREADS * LAUNCH_REGS and the shares below add up to exactly that.
+  static constexpr int THREADS = QT * 128 + 128;
+  static constexpr int MIN_BLOCKS = QT == 1 ? 2 : 1;
+  static constexpr int LAUNCH_REGS = QT == 1 ? 128 : 168;
+  static constexpr int REG_SOFTMAX = QT == 1 ? 208 : 216;
+  static constexpr int REG_OTHER = QT == 1 ? 48 : 72;
+  static_assert(QT * 128 * REG_SOFTMAX + 128 * REG_OTHER == THREADS * LAUNCH_REGS, "register split");
   static constexpr int PRODUCER_WARP = QT * 4;
   static constexpr int MMA_WARP = QT * 4 + 1;
   static constexpr uint32_t TMEM_COLS = QT == 2 ? 512 : 256;
+  // With DP <= 64 the bf16 P tile gets its own 64 TMEM columns, so S(i+1)
+  // can be computed while the softmax of S(i) is still running; with DP = 128
+  // P overwrites the first 64 columns of S.
+  static constexpr bool SEP_P = DP <= 64;
+  static constexpr uint32_t S_COL0 = 0;                                // + 128 t
+  static constexpr uint32_t P_COL0 = SEP_P ? 128 * QT : 0;             // + (SEP_P ? 64 : 128) t
+  static constexpr uint32_t P_STRIDE = SEP_P ? 64 : 128;
+  static constexpr uint32_t O_COL0 = SEP_P ? 128 * QT + 64 * QT : 128 * QT;  // + O_STRIDE t
+  static constexpr uint32_t O_STRIDE = SEP_P ? DP : 128;
+  static_assert(O_COL0 + O_STRIDE * QT <= TMEM_COLS, "TMEM layout");
   static constexpr uint32_t IDESC_QK = make_idesc_f16(true, true, 128, 128, false);
   static constexpr uint32_t IDESC_F = make_idesc_f16(false, false, 128, 128, false);
   static constexpr uint32_t IDESC_PV = make_idesc_f16(true, true, 128, DP, true);
@@ -76,9 +101,11 @@ struct Sm100Cfg {
 
 struct SmemCtrl {
   uint64_t q_full;
-  uint64_t o_final;
-  uint64_t drain;
-  uint64_t k_full[3], k_empty[3], v_full[3], v_empty[3];
+  uint64_t o_final[2];
+  uint64_t drain[2];
+  uint64_t s_free[2], pv_done[2];  // separate-P schedule only
+  uint64_t k_full[3], v_full[3];
+  uint64_t k_empty[2][3], v_empty[2][3];  // released by the MMA issuer of each query tile
   uint64_t s_full[2], p_full[2];
   uint64_t aux_full[2][3], aux_empty[2][3];
   uint32_t tmem_base;
@@ -86,28 +113,31 @@ struct SmemCtrl {
 };
 static_assert(sizeof(SmemCtrl) <= 1024, "control block too large");
 
-// K-major tile of `rows` x (NCH * CH) 16-bit elements as NCH swizzled column
-// chunks of CH elements; descriptor for the 16-column MMA step kk.
+// K-major tile of 128 rows x (NCH * CH) 16-bit elements, stored as NCH
+// swizzled column chunks of CH elements: descriptor of the chunk base, and
+// the start-address offset (in 16-byte units) of the 16-column MMA step kk.
 template <int CH>
-__device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, int rows, int kk) {
-  constexpr int row_bytes = CH * 2;
-  constexpr int steps_per_chunk = CH / 16;
-  const int chunk = kk / steps_per_chunk;
-  const uint32_t off = uint32_t(chunk) * uint32_t(rows * row_bytes) + uint32_t(kk % steps_per_chunk) * 32u;
-  return make_smem_desc(base + off, 16, 8 * row_bytes, swizzle_code(row_bytes));
+__device__ __forceinline__ uint64_t desc_kmajor_base(uint32_t base) {
+  return make_smem_desc(base, 16, 8 * CH * 2, swizzle_code(CH * 2));
+}
+template <int CH>
+__host__ __device__ constexpr uint32_t kmajor_step(int kk) {
+  return uint32_t((kk / (CH / 16)) * (128 * CH * 2) + (kk % (CH / 16)) * 32) >> 4;
 }
 
 // V tile, [128 keys] x (NCH * CH) values, as the MN-major B operand of the PV
-// MMA; descriptor for the 16-key step kk.
+// MMA: descriptor of the tile base and the offset of the 16-key step kk.
 template <int CH>
-__device__ __forceinline__ uint64_t desc_v(uint32_t base, int kk) {
-  constexpr int row_bytes = CH * 2;
-  return make_smem_desc(base + uint32_t(kk) * 16u * row_bytes, 128 * row_bytes, 8 * row_bytes,
-                        swizzle_code(row_bytes));
+__device__ __forceinline__ uint64_t desc_v_base(uint32_t base) {
+  return make_smem_desc(base, 128 * CH * 2, 8 * CH * 2, swizzle_code(CH * 2));
+}
+template <int CH>
+__host__ __device__ constexpr uint32_t v_step(int kk) {
+  return uint32_t(kk * 16 * CH * 2) >> 4;
 }
 
 template <int DP, int RP, int MODE, int QT>
-__global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, QT == 1 ? 2 : 1)
+__global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<DP, RP, MODE, QT>::MIN_BLOCKS)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_fq,
                    const __grid_constant__ CUtensorMap tm_fk, const __grid_constant__ CUtensorMap tm_bias,
@@ -148,14 +178,12 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, QT == 1 ?
 
   if (threadIdx.x == 0) {
     mbar_init(&ctrl->q_full, 1);
-    mbar_init(&ctrl->o_final, 1);
-    mbar_init(&ctrl->drain, 1);
     for (int s = 0; s < KS; ++s) {
       mbar_init(&ctrl->k_full[s], 1);
-      mbar_init(&ctrl->k_empty[s], 1);
       mbar_init(&ctrl->v_full[s], 1);
-      mbar_init(&ctrl->v_empty[s], 1);
       for (int t = 0; t < QT; ++t) {
+        mbar_init(&ctrl->k_empty[t][s], 1);
+        mbar_init(&ctrl->v_empty[t][s], 1);
         mbar_init(&ctrl->aux_full[t][s], 1);
         mbar_init(&ctrl->aux_empty[t][s], 128);
       }
@@ -163,6 +191,10 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, QT == 1 ?
     for (int t = 0; t < QT; ++t) {
       mbar_init(&ctrl->s_full[t], 1);
       mbar_init(&ctrl->p_full[t], 128);
+      mbar_init(&ctrl->o_final[t], 1);
+      mbar_init(&ctrl->drain[t], 1);
+      mbar_init(&ctrl->s_free[t], 128);
+      mbar_init(&ctrl->pv_done[t], 1);
     }
     ctrl->abort = 0;
     fence_mbar_init();
@@ -177,9 +209,15 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, QT == 1 ?
   const uint32_t tmem = ctrl->tmem_base;
   volatile int *abort = &ctrl->abort;
 
+  if (warp >= QT * 4) {
+  setmaxnreg_dec<C::REG_OTHER>();
+  // The producer and MMA warps run their loops with all 32 lanes so that
+  // coordinates and descriptors stay warp-uniform; lane 0 alone issues each
+  // TMA copy, expect-tx arrival, MMA and commit (predicated inside the asm).
+  const uint32_t leader = lane == 0 ? 1u : 0u;
   if (warp == C::PRODUCER_WARP) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    if (leader) {
       tma_prefetch_map(&tm_q);
       tma_prefetch_map(&tm_k);
       tma_prefetch_map(&tm_v);
@@ -189,97 +227,150 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, QT == 1 ?
       }
       if (MODE == kBiasReg) tma_prefetch_map(&tm_fk);
       if (MODE == kBiasDense) tma_prefetch_map(&tm_bias);
-      uint32_t qbytes = 0;
-      for (int t = 0; t < QT; ++t)
-        if (nk[t] > 0) qbytes += C::Q_TILE + C::FQ_TILE;
-      mbar_arrive_expect_tx(&ctrl->q_full, qbytes);
-      for (int t = 0; t < QT; ++t) {
-        if (nk[t] == 0) continue;
-        for (int ch = 0; ch < C::NDCH; ++ch)
-          tma_load_3d(sQ + t * C::Q_TILE + ch * (128 * C::DCH * 2), &tm_q, &ctrl->q_full, ch * C::DCH, q0[t], bh);
-        if (MODE == kBiasMma)
-          for (int ch = 0; ch < C::NRCH; ++ch)
-            tma_load_3d(sFQ + t * C::FQ_TILE + ch * (128 * C::RCH * 2), &tm_fq, &ctrl->q_full, ch * C::RCH, q0[t],
-                        fb_slice);
+    }
+    uint32_t qbytes = 0;
+    for (int t = 0; t < QT; ++t)
+      if (nk[t] > 0) qbytes += C::Q_TILE + C::FQ_TILE;
+    mbar_arrive_expect_tx_leader(&ctrl->q_full, qbytes, leader);
+    for (int t = 0; t < QT; ++t) {
+      if (nk[t] == 0) continue;
+      for (int ch = 0; ch < C::NDCH; ++ch)
+        tma_load_3d_leader(sQ + t * C::Q_TILE + ch * (128 * C::DCH * 2), &tm_q, &ctrl->q_full, ch * C::DCH, q0[t], bh,
+                           leader);
+      if (MODE == kBiasMma)
+        for (int ch = 0; ch < C::NRCH; ++ch)
+          tma_load_3d_leader(sFQ + t * C::FQ_TILE + ch * (128 * C::RCH * 2), &tm_fq, &ctrl->q_full, ch * C::RCH,
+                             q0[t], fb_slice, leader);
+    }
+    int hb = 0, bb = 0;
+    if (MODE == kBiasDense) {
+      hb = args.bias_H > 1 ? h : 0;
+      bb = args.bias_B > 1 ? b : 0;
+    }
+    bool ok = true;
+    for (int i = 0; i < n_steps && ok; ++i) {
+      const int s = i % KS;
+      const uint32_t ph = uint32_t(i / KS) & 1u;
+      // stage s last held step i - KS: wait until every tile that used it released it
+      if (i >= KS)
+        for (int t = 0; t < QT && ok; ++t)
+          if (i - KS < nk[t]) ok = mbar_wait(&ctrl->k_empty[t][s], ph ^ 1u, abort);
+      if (!ok) break;
+      mbar_arrive_expect_tx_leader(&ctrl->k_full[s], C::KV_TILE + C::FK_TILE, leader);
+      for (int ch = 0; ch < C::NDCH; ++ch)
+        tma_load_3d_leader(sK + s * C::KV_TILE + ch * (128 * C::DCH * 2), &tm_k, &ctrl->k_full[s], ch * C::DCH,
+                           i * 128, bh, leader);
+      if (MODE == kBiasMma)
+        for (int ch = 0; ch < C::NRCH; ++ch)
+          tma_load_3d_leader(sFK + s * C::FK_TILE + ch * (128 * C::RCH * 2), &tm_fk, &ctrl->k_full[s], ch * C::RCH,
+                             i * 128, fb_slice, leader);
+      if (C::HAS_AUX) {
+        for (int t = 0; t < QT; ++t) {
+          if (i >= nk[t]) continue;
+          if (!(ok = mbar_wait(&ctrl->aux_empty[t][s], ph ^ 1u, abort))) break;
+          uint8_t *dst = sAux + (t * KS + s) * C::AUX_TILE;
+          mbar_arrive_expect_tx_leader(&ctrl->aux_full[t][s], C::AUX_TILE, leader);
+          if (MODE == kBiasReg) {
+            tma_load_3d_leader(dst, &tm_fk, &ctrl->aux_full[t][s], 0, i * 128, fb_slice, leader);
+          } else {
+            tma_load_4d_leader(dst, &tm_bias, &ctrl->aux_full[t][s], i * 128, q0[t], hb, bb, leader);
+            tma_load_4d_leader(dst + 128 * 128, &tm_bias, &ctrl->aux_full[t][s], i * 128 + 64, q0[t], hb, bb,
+                               leader);
+          }
+        }
+        if (!ok) break;
       }
-      int hb = 0, bb = 0;
-      if (MODE == kBiasDense) {
-        hb = args.bias_H > 1 ? h : 0;
-        bb = args.bias_B > 1 ? b : 0;
+      if (i >= KS)
+        for (int t = 0; t < QT && ok; ++t)
+          if (i - KS < nk[t]) ok = mbar_wait(&ctrl->v_empty[t][s], ph ^ 1u, abort);
+      if (!ok) break;
+      mbar_arrive_expect_tx_leader(&ctrl->v_full[s], C::KV_TILE, leader);
+      for (int ch = 0; ch < C::NDCH; ++ch)
+        tma_load_3d_leader(sV + s * C::KV_TILE + ch * (128 * C::DCH * 2), &tm_v, &ctrl->v_full[s], ch * C::DCH,
+                           i * 128, bh, leader);
+    }
+    if (!ok) {
+      // Aborted: let the copies already issued land before the CTA exits.
+      for (int s = 0; s < KS; ++s) {
+        mbar_wait_for(&ctrl->k_full[s], 0, 100000000ull);
+        mbar_wait_for(&ctrl->k_full[s], 1, 100000000ull);
+        mbar_wait_for(&ctrl->v_full[s], 0, 100000000ull);
+        mbar_wait_for(&ctrl->v_full[s], 1, 100000000ull);
       }
-      bool ok = true;
-      for (int i = 0; i < n_steps && ok; ++i) {
+      if (leader) atomicOr(args.flags, kFlagTimeout);
+    }
+  } else if (warp == C::MMA_WARP || (C::SEP_P && QT == 2 && warp == C::MMA_WARP + 1)) {
+    // ---------------------------------------------------------- MMA issuer
+    // Descriptors of every tile base, computed once; each MMA adds a
+    // compile-time step offset (the start address is the low field, and
+    // shared addresses >> 4 stay below 2^14, so plain adds cannot carry).
+    const uint32_t tm_u = __shfl_sync(0xffffffffu, tmem, 0);
+    const uint64_t dk0 = desc_kmajor_base<C::DCH>(smem_u32(sK));
+    const uint64_t dfk0 = desc_kmajor_base<C::RCH>(smem_u32(sFK));
+    const uint64_t dv0 = desc_v_base<C::DCH>(smem_u32(sV));
+    auto issue_s = [&](int t, int s) {  // S_t = Q_t K_s^T (+ phi_q' phi_k^T)
+      const uint32_t d_tm = tm_u + C::S_COL0 + uint32_t(128 * t);
+      const uint64_t dq = desc_kmajor_base<C::DCH>(smem_u32(sQ + t * C::Q_TILE));
+      const uint64_t dk = dk0 + uint64_t((uint32_t(s) * C::KV_TILE) >> 4);
+#pragma unroll
+      for (int kk = 0; kk < DP / 16; ++kk)
+        mma_ss_elect(d_tm, dq + kmajor_step<C::DCH>(kk), dk + kmajor_step<C::DCH>(kk), C::IDESC_QK,
+                     kk > 0 ? 1u : 0u);
+      if (MODE == kBiasMma) {
+        const uint64_t dfq = desc_kmajor_base<C::RCH>(smem_u32(sFQ + t * C::FQ_TILE));
+        const uint64_t dfk = dfk0 + uint64_t((uint32_t(s) * C::FK_TILE) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < (MODE == kBiasMma ? RP / 16 : 0); ++kk)
+          mma_ss_elect(d_tm, dfq + kmajor_step<C::RCH>(kk), dfk + kmajor_step<C::RCH>(kk), C::IDESC_F, 1u);
+      }
+    };
+    auto issue_pv = [&](int t, int s, bool acc) {  // O_t += P_t V_s, P_t read from TMEM
+      const uint32_t d_tm = tm_u + C::O_COL0 + C::O_STRIDE * uint32_t(t);
+      const uint32_t p_tm = tm_u + C::P_COL0 + C::P_STRIDE * uint32_t(t);
+      const uint64_t dv = dv0 + uint64_t((uint32_t(s) * C::KV_TILE) >> 4);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_ts_elect(d_tm, p_tm + uint32_t(kk * 8), dv + v_step<C::DCH>(kk), C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+    };
+    bool ok = mbar_wait(&ctrl->q_full, 0, abort);
+    tc_fence_after();
+    if constexpr (C::SEP_P) {
+      // One issuer warp per query tile t: S_t(i+1) as soon as the softmax has
+      // read S_t(i) into registers, PV_t(i) once P_t(i) is written. The two
+      // tiles' chains are independent and share the tensor core.
+      const int t = warp - C::MMA_WARP;
+      if (ok && nk[t] > 0 && (ok = mbar_wait(&ctrl->k_full[0], 0, abort))) {
+        tc_fence_after();
+        issue_s(t, 0);
+        tc_commit_elect(&ctrl->s_full[t]);
+        tc_commit_elect(&ctrl->k_empty[t][0]);
+      }
+      for (int i = 0; i < nk[t] && ok; ++i) {
         const int s = i % KS;
         const uint32_t ph = uint32_t(i / KS) & 1u;
-        if (!(ok = mbar_wait(&ctrl->k_empty[s], ph ^ 1u, abort))) break;
-        mbar_arrive_expect_tx(&ctrl->k_full[s], C::KV_TILE + C::FK_TILE);
-        for (int ch = 0; ch < C::NDCH; ++ch)
-          tma_load_3d(sK + s * C::KV_TILE + ch * (128 * C::DCH * 2), &tm_k, &ctrl->k_full[s], ch * C::DCH, i * 128,
-                      bh);
-        if (MODE == kBiasMma)
-          for (int ch = 0; ch < C::NRCH; ++ch)
-            tma_load_3d(sFK + s * C::FK_TILE + ch * (128 * C::RCH * 2), &tm_fk, &ctrl->k_full[s], ch * C::RCH,
-                        i * 128, fb_slice);
-        if (C::HAS_AUX) {
-          for (int t = 0; t < QT; ++t) {
-            if (i >= nk[t]) continue;
-            if (!(ok = mbar_wait(&ctrl->aux_empty[t][s], ph ^ 1u, abort))) break;
-            uint8_t *dst = sAux + (t * KS + s) * C::AUX_TILE;
-            mbar_arrive_expect_tx(&ctrl->aux_full[t][s], C::AUX_TILE);
-            if (MODE == kBiasReg) {
-              tma_load_3d(dst, &tm_fk, &ctrl->aux_full[t][s], 0, i * 128, fb_slice);
-            } else {
-              tma_load_4d(dst, &tm_bias, &ctrl->aux_full[t][s], i * 128, q0[t], hb, bb);
-              tma_load_4d(dst + 128 * 128, &tm_bias, &ctrl->aux_full[t][s], i * 128 + 64, q0[t], hb, bb);
-            }
-          }
-          if (!ok) break;
+        if (i + 1 < nk[t]) {
+          const int s1 = (i + 1) % KS;
+          if (!(ok = mbar_wait(&ctrl->k_full[s1], uint32_t((i + 1) / KS) & 1u, abort))) break;
+          if (!(ok = mbar_wait(&ctrl->s_free[t], uint32_t(i) & 1u, abort))) break;
+          tc_fence_after();
+          issue_s(t, s1);
+          tc_commit_elect(&ctrl->s_full[t]);
+          tc_commit_elect(&ctrl->k_empty[t][s1]);
         }
-        if (!(ok = mbar_wait(&ctrl->v_empty[s], ph ^ 1u, abort))) break;
-        mbar_arrive_expect_tx(&ctrl->v_full[s], C::KV_TILE);
-        for (int ch = 0; ch < C::NDCH; ++ch)
-          tma_load_3d(sV + s * C::KV_TILE + ch * (128 * C::DCH * 2), &tm_v, &ctrl->v_full[s], ch * C::DCH, i * 128,
-                      bh);
+        if (!(ok = mbar_wait(&ctrl->v_full[s], ph, abort))) break;
+        if (!(ok = mbar_wait(&ctrl->p_full[t], uint32_t(i) & 1u, abort))) break;
+        tc_fence_after();
+        issue_pv(t, s, i > 0);
+        tc_commit_elect(&ctrl->pv_done[t]);
+        tc_commit_elect(&ctrl->v_empty[t][s]);
       }
+      tc_commit_elect(&ctrl->o_final[t]);
       if (!ok) {
-        // Aborted: let the copies already issued land before the CTA exits.
-        for (int s = 0; s < KS; ++s) {
-          mbar_wait_for(&ctrl->k_full[s], 0, 100000000ull);
-          mbar_wait_for(&ctrl->k_full[s], 1, 100000000ull);
-          mbar_wait_for(&ctrl->v_full[s], 0, 100000000ull);
-          mbar_wait_for(&ctrl->v_full[s], 1, 100000000ull);
-        }
-        atomicOr(args.flags, kFlagTimeout);
+        tc_commit_elect(&ctrl->drain[t]);
+        mbar_wait_for(&ctrl->drain[t], 0, 100000000ull);
+        if (leader) atomicOr(args.flags, kFlagTimeout);
       }
-    }
-  } else if (warp == C::MMA_WARP) {
-    // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      const uint32_t sQa = smem_u32(sQ), sFQa = smem_u32(sFQ), sKa = smem_u32(sK), sFKa = smem_u32(sFK),
-                     sVa = smem_u32(sV);
-      auto issue_s = [&](int t, int s) {
-        const uint32_t d_tm = tmem + uint32_t(128 * t);
-#pragma unroll
-        for (int kk = 0; kk < DP / 16; ++kk)
-          mma_ss(d_tm, desc_kmajor<C::DCH>(sQa + t * C::Q_TILE, 128, kk),
-                 desc_kmajor<C::DCH>(sKa + s * C::KV_TILE, 128, kk), C::IDESC_QK, kk > 0 ? 1u : 0u);
-        if (MODE == kBiasMma) {
-#pragma unroll
-          for (int kk = 0; kk < (MODE == kBiasMma ? RP / 16 : 0); ++kk)
-            mma_ss(d_tm, desc_kmajor<C::RCH>(sFQa + t * C::FQ_TILE, 128, kk),
-                   desc_kmajor<C::RCH>(sFKa + s * C::FK_TILE, 128, kk), C::IDESC_F, 1u);
-        }
-      };
-      auto issue_pv = [&](int t, int s, bool acc) {
-        const uint32_t d_tm = tmem + uint32_t(128 * QT + 128 * t);
-        const uint32_t p_tm = tmem + uint32_t(128 * t);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(d_tm, p_tm + uint32_t(kk * 8), desc_v<C::DCH>(sVa + s * C::KV_TILE, kk), C::IDESC_PV,
-                 (acc || kk > 0) ? 1u : 0u);
-      };
-      bool ok = mbar_wait(&ctrl->q_full, 0, abort);
-      tc_fence_after();
+    } else {
       for (int i = 0; i < n_steps && ok; ++i) {
         const int s = i % KS;
         const uint32_t ph = uint32_t(i / KS) & 1u;
@@ -287,7 +378,8 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, QT == 1 ?
         tc_fence_after();
         if (i < nk[0]) {
           issue_s(0, s);
-          tc_commit(&ctrl->s_full[0]);
+          tc_commit_elect(&ctrl->s_full[0]);
+          tc_commit_elect(&ctrl->k_empty[0][s]);
         }
         if (QT == 2) {
           const int j = i - 1;  // PV of tile 1 for the previous step
@@ -298,20 +390,20 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, QT == 1 ?
             if (!(ok = mbar_wait(&ctrl->p_full[1], uint32_t(j) & 1u, abort))) break;
             tc_fence_after();
             issue_pv(1, sj, j > 0);
-            tc_commit(&ctrl->v_empty[sj]);
+            tc_commit_elect(&ctrl->v_empty[1][sj]);
           }
           if (i < nk[1]) {
             issue_s(1, s);
-            tc_commit(&ctrl->s_full[1]);
+            tc_commit_elect(&ctrl->s_full[1]);
+            tc_commit_elect(&ctrl->k_empty[1][s]);
           }
         }
-        tc_commit(&ctrl->k_empty[s]);
         if (i < nk[0]) {
           if (!(ok = mbar_wait(&ctrl->v_full[s], ph, abort))) break;
           if (!(ok = mbar_wait(&ctrl->p_full[0], uint32_t(i) & 1u, abort))) break;
           tc_fence_after();
           issue_pv(0, s, i > 0);
-          if (QT == 1 || i >= nk[1]) tc_commit(&ctrl->v_empty[s]);
+          tc_commit_elect(&ctrl->v_empty[0][s]);
         }
       }
       if (ok && QT == 2 && nk[1] == n_steps && n_steps > 0) {
@@ -323,26 +415,29 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, QT == 1 ?
         if (ok) {
           tc_fence_after();
           issue_pv(1, sj, j > 0);
-          tc_commit(&ctrl->v_empty[sj]);
+          tc_commit_elect(&ctrl->v_empty[1][sj]);
         }
       }
-      tc_commit(&ctrl->o_final);
+      for (int t = 0; t < QT; ++t) tc_commit_elect(&ctrl->o_final[t]);
       if (!ok) {
         // Aborted: wait (bounded) for the MMAs already issued to finish.
-        tc_commit(&ctrl->drain);
-        mbar_wait_for(&ctrl->drain, 0, 100000000ull);
-        atomicOr(args.flags, kFlagTimeout);
+        tc_commit_elect(&ctrl->drain[0]);
+        mbar_wait_for(&ctrl->drain[0], 0, 100000000ull);
+        if (leader) atomicOr(args.flags, kFlagTimeout);
       }
     }
+  }
   } else {
+    setmaxnreg_inc<C::REG_SOFTMAX>();
     // ------------------------------------------------------------- softmax
     const int t = warp >> 2;  // query tile of this warpgroup
     const int wq = warp & 3;  // TMEM lane quarter
     const int r_loc = wq * 32 + lane;
     const int row = q0[t] + r_loc;
     const uint32_t lane_base = tmem + (uint32_t(wq * 32) << 16);
-    const uint32_t s_tm = lane_base + uint32_t(128 * t);
-    const uint32_t o_tm = lane_base + uint32_t(128 * QT + 128 * t);
+    const uint32_t s_tm = lane_base + C::S_COL0 + uint32_t(128 * t);
+    const uint32_t p_tm = lane_base + C::P_COL0 + C::P_STRIDE * uint32_t(t);
+    const uint32_t o_tm = lane_base + C::O_COL0 + C::O_STRIDE * uint32_t(t);
     const float sl2 = args.scale_log2;
 
     float aq0 = 0.f, aq1 = 0.f, aq2 = 0.f, aq3 = 0.f;
@@ -372,6 +467,10 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, QT == 1 ?
       tmem_ld_wait32(x + 32);
       tmem_ld_wait32(x + 64);
       tmem_ld_wait32(x + 96);
+      if (C::SEP_P) {  // S_t(i) is in registers: the tensor core may overwrite it
+        tc_fence_before();
+        mbar_arrive(&ctrl->s_free[t]);
+      }
       float mul = sl2;  // logit = raw * mul
       if (MODE == kBiasReg) {
         const uint8_t *fk = sAux + (t * KS + s) * C::AUX_TILE;
@@ -418,9 +517,17 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, QT == 1 ?
         for (int c = 0; c < 128; ++c)
           if (key0 + c >= lim) x[c] = __float_as_uint(-INFINITY);
       }
-      float mx = __uint_as_float(x[0]);
+      float mx;
+      {
+        float mp[8];
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(x[c]));
+        for (int e = 0; e < 8; ++e) mp[e] = __uint_as_float(x[e]);
+#pragma unroll
+        for (int c = 8; c < 128; c += 8)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) mp[e] = fmaxf(mp[e], __uint_as_float(x[c + e]));
+        mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])), fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+      }
       const float m_new = fmaxf(m_use, mx * mul);
       float alpha = 1.f;
       bool resc = false;
@@ -430,8 +537,14 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, QT == 1 ?
         m_use = m_new;
       }
       l_sum *= alpha;
+      if (C::SEP_P && i > 0) {
+        // O_t and P_t are still read by PV_t(i-1); wait until it has completed.
+        if (!(ok = mbar_wait(&ctrl->pv_done[t], uint32_t(i - 1) & 1u, abort))) break;
+        tc_fence_after();
+      }
       if (__any_sync(0xffffffffu, resc)) {
-        // PV_t(i-1) has completed: the commit that published S_t(i) covers it.
+        // PV_t(i-1) has completed (pv_done, or, when P aliases S, the commit
+        // that published S_t(i) covers it).
 #pragma unroll
         for (int c0 = 0; c0 < DP; c0 += 16) {
           uint32_t r[16];
@@ -443,17 +556,35 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, QT == 1 ?
         }
       }
       const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;
+      const uint64_t mul2 = f2_pack(mul, mul), negm2 = f2_pack(neg_m, neg_m);
+      uint64_t ls[4] = {0, 0, 0, 0};  // packed partial row sums
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(x[q4 * 32 + 2 * e]), mul, neg_m));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(x[q4 * 32 + 2 * e + 1]), mul, neg_m));
-          l_sum += p0 + p1;
+          const uint64_t a = f2_fma(f2_pack(__uint_as_float(x[q4 * 32 + 2 * e]), __uint_as_float(x[q4 * 32 + 2 * e + 1])),
+                                    mul2, negm2);
+          float a0, a1, p0, p1;
+          f2_unpack(a, a0, a1);
+          if (e < kEmuPairs) {
+            ex2_fma_pair(a0, a1, p0, p1);
+          } else {
+            p0 = ex2_approx(a0);
+            p1 = ex2_approx(a1);
+          }
+          ls[e & 3] = f2_add(ls[e & 3], f2_pack(p0, p1));
           pk[e] = pack_bf16x2(p0, p1);
         }
-        tmem_st16(s_tm + uint32_t(q4 * 16), pk);
+        tmem_st16(p_tm + uint32_t(q4 * 16), pk);
+      }
+      {
+        float s0, s1, s2, s3, s4, s5, s6, s7;
+        f2_unpack(ls[0], s0, s1);
+        f2_unpack(ls[1], s2, s3);
+        f2_unpack(ls[2], s4, s5);
+        f2_unpack(ls[3], s6, s7);
+        l_sum += ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
       }
       tmem_st_wait();
       tc_fence_before();
@@ -461,7 +592,7 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, QT == 1 ?
     }
 
     // ------------------------------------------------------------ epilogue
-    if (ok && nk[t] > 0) ok = mbar_wait(&ctrl->o_final, 0, abort);
+    if (ok && nk[t] > 0) ok = mbar_wait(&ctrl->o_final[t], 0, abort);
     if (ok && nk[t] > 0) {
       tc_fence_after();
       const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
@@ -507,7 +638,13 @@ static cudaError_t launch_one(const FwdMaps &m, const FwdArgs &a, cudaStream_t s
     return cudaErrorInvalidConfiguration;
   } else {
     auto kern = attn_fwd_sm100<DP, RP, MODE, QT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::SMEM));
+    // setmaxnreg.inc waits until the block's pool has the registers, so the
+    // launch allocation must be exactly what the split assumes.
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != C::LAUNCH_REGS) return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::SMEM));
     if (e != cudaSuccess) return e;
     dim3 grid(a.B * a.H, a.n_cta_q);
     kern<<<grid, C::THREADS, C::SMEM, stream>>>(m.q, m.k, m.v, m.fq, m.fk, m.bias, a);

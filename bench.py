@@ -494,7 +494,7 @@ def cpu_baseline(c: dict, budget_s: float):
     """The oracle, as it stands, on the host cores over ~budget_s of a bounded sample."""
     import oracle
     total_fl, total_s, step, parts = 0.0, 0.0, 0, []
-    while total_s < budget_s and step < 64:
+    while total_s < budget_s and step < 1024:
         run, fl, desc = oracle_sample(c, step, rows_per_head=256)
         t0 = time.perf_counter()
         run()

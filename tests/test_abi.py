@@ -157,3 +157,27 @@ def test_svd_host_rejects_bad_arguments():
         == fb.FB_ERR_INVALID_ARG
     assert fb.fb_svd_factors_host(None, 4, 2, 4, 1, 0, out.ctypes.data, out.ctypes.data, None, None) \
         == fb.FB_ERR_INVALID_ARG
+
+
+def test_fma_pipe_exp2_polynomial_error_bound():
+    """The FMA-pipe exp2 of the softmax (range reduction + fitted cubic),
+    restated in numpy float32 and checked against fp64 exp2: relative error
+    below 1e-4 on the range the softmax uses, so it is invisible after P is
+    rounded to bf16 (relative step 2^-8)."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "fit", os.path.join(ROOT, "attention_rank_additive_b200", "csrc", "fit_exp2_poly.py"))
+    fit = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(fit)
+    c, err = fit.fit(samples=4001, iters=150)
+    assert err < 1e-4
+    want = [0.9999252, 0.6958336, 0.22606726, 0.078024276]  # the constants in fb_ptx.cuh
+    np.testing.assert_allclose(np.float32(c), np.float32(want), rtol=2e-4)
+    x = np.concatenate([np.linspace(-126.0, 8.0, 200001), -np.arange(0, 127, dtype=np.float64)]).astype(np.float32)
+    n = np.floor(x)
+    f = (x - n).astype(np.float32)
+    w = np.float32(want)
+    p = ((w[3] * f + w[2]) * f + w[1]) * f + w[0]
+    got = p.astype(np.float64) * np.exp2(n.astype(np.float64))
+    rel = np.abs(got / np.exp2(x.astype(np.float64)) - 1.0)
+    assert rel.max() < 1e-4
