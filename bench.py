@@ -101,6 +101,11 @@ def reduce_max(value: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def weak_scaling_value(flops_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job TFLOP/s: every rank ran its own batch; time is the max over ranks."""
+    return flops_per_rank * world / (ms_max * 1e-3) / 1e12
+
+
 def barrier(world: int):
     if world > 1:
         import torch.distributed as dist
@@ -372,7 +377,7 @@ def run_ours(args, rank: int, world: int, local: int):
     ms_local = statistics.mean(step_ms)
     ms = reduce_max(ms_local, world, device)
     kern_ms = reduce_max(kern_ms, world, device)
-    value = c["flops"] * world / (ms * 1e-3) / 1e12
+    value = weak_scaling_value(c["flops"], world, ms)
 
     # end to end through the C ABI with host buffers: H2D of Q, K, V from
     # pinned memory, the step, D2H of O and LSE, every step.
