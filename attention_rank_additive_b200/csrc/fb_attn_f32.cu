@@ -5,8 +5,10 @@
 // bias), online softmax over 32-key tiles, O / l and the log-sum-exp.
 //
 // A CTA of 128 threads owns 32 query rows; four threads share a row, each
-// holding every fourth head-dim element and every fourth factor rank, and the
-// row's partial dot products meet through two xor-shuffles.
+// holding every fourth float4 column of q and o and every fourth factor
+// rank, and the row's partial dot products meet through two xor-shuffles.
+// Key, value and factor tiles are staged in shared memory with all of a
+// tile's global loads in flight before the first store.
 #include <cfloat>
 
 #include "fb_internal.h"
@@ -15,9 +17,10 @@ namespace fb {
 
 constexpr int kF32Rows = 32;
 constexpr int kF32Keys = 32;
-constexpr int kF32MaxD = 128;
 constexpr int kF32MaxR = 128;
 
+// DQ: float4 columns per row after padding (4, 8, 16 or 32; d <= 4 DQ).
+template <int DQ>
 __global__ void __launch_bounds__(128) attn_fwd_f32_kernel(int B, int H, int N, int d, const float *__restrict__ Q,
                                                            const float *__restrict__ K, const float *__restrict__ V,
                                                            int R, const float *__restrict__ phi_q,
@@ -25,27 +28,35 @@ __global__ void __launch_bounds__(128) attn_fwd_f32_kernel(int B, int H, int N, 
                                                            long long phi_hs, const float *__restrict__ bias,
                                                            long long bias_bs, long long bias_hs, float scale,
                                                            int causal, float *__restrict__ O, float *__restrict__ LSE) {
-  __shared__ float sK[kF32Keys][kF32MaxD];
-  __shared__ float sV[kF32Keys][kF32MaxD];
+  constexpr int U = DQ / 4;  // float4 columns per thread
+  __shared__ float4 sK[kF32Keys][DQ];
+  __shared__ float4 sV[kF32Keys][DQ];
   __shared__ float sF[kF32Keys][kF32MaxR];
 
   const int bh = blockIdx.y;
   const int b = bh / H, h = bh - (bh / H) * H;
-  const int sub = threadIdx.x & 3;
-  const int row = blockIdx.x * kF32Rows + (threadIdx.x >> 2);
+  const int tid = threadIdx.x;
+  const int sub = tid & 3;
+  const int row = blockIdx.x * kF32Rows + (tid >> 2);
   const bool row_ok = row < N;
+  const int d4 = d >> 2;
   const size_t head = size_t(bh) * N * d;
+  const float4 *Q4 = reinterpret_cast<const float4 *>(Q + head);
+  const float4 *K4 = reinterpret_cast<const float4 *>(K + head);
+  const float4 *V4 = reinterpret_cast<const float4 *>(V + head);
   const float *phq = phi_q ? phi_q + b * phi_bs + h * phi_hs : nullptr;
   const float *phk = phi_k ? phi_k + b * phi_bs + h * phi_hs : nullptr;
   const float *brow = bias ? bias + b * bias_bs + h * bias_hs + (size_t)(row_ok ? row : 0) * N : nullptr;
+  const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
 
-  float q[kF32MaxD / 4], o[kF32MaxD / 4], fq[kF32MaxR / 4];
+  float4 q[U], o[U];
 #pragma unroll
-  for (int u = 0; u < kF32MaxD / 4; ++u) {
-    const int c = sub + 4 * u;
-    q[u] = (row_ok && c < d) ? Q[head + size_t(row) * d + c] : 0.f;
-    o[u] = 0.f;
+  for (int u = 0; u < U; ++u) {
+    const int c4 = sub + 4 * u;
+    q[u] = (row_ok && c4 < d4) ? Q4[size_t(row) * d4 + c4] : zero4;
+    o[u] = zero4;
   }
+  float fq[kF32MaxR / 4];
 #pragma unroll
   for (int u = 0; u < kF32MaxR / 4; ++u) {
     const int r = sub + 4 * u;
@@ -56,17 +67,30 @@ __global__ void __launch_bounds__(128) attn_fwd_f32_kernel(int B, int H, int N, 
   const int kmax = causal ? min(N, (blockIdx.x + 1) * kF32Rows) : N;  // keys any row of this CTA can see
   for (int k0 = 0; k0 < kmax; k0 += kF32Keys) {
     __syncthreads();
-    for (int e = threadIdx.x; e < kF32Keys * d; e += blockDim.x) {
-      const int j = e / d, c = e - (e / d) * d;
-      const bool ok = k0 + j < N;
-      sK[j][c] = ok ? K[head + size_t(k0 + j) * d + c] : 0.f;
-      sV[j][c] = ok ? V[head + size_t(k0 + j) * d + c] : 0.f;
+    {
+      constexpr int PER = kF32Keys * DQ / 128;  // float4 per thread per tensor
+      float4 kr[PER], vr[PER];
+#pragma unroll
+      for (int it = 0; it < PER; ++it) {
+        const int e = tid + 128 * it;
+        const int j = e / DQ, c4 = e % DQ;
+        const bool ok = (k0 + j < N) && (c4 < d4);
+        kr[it] = ok ? K4[size_t(k0 + j) * d4 + c4] : zero4;
+        vr[it] = ok ? V4[size_t(k0 + j) * d4 + c4] : zero4;
+      }
+#pragma unroll
+      for (int it = 0; it < PER; ++it) {
+        const int e = tid + 128 * it;
+        sK[e / DQ][e % DQ] = kr[it];
+        sV[e / DQ][e % DQ] = vr[it];
+      }
     }
-    if (phk)
-      for (int e = threadIdx.x; e < kF32Keys * R; e += blockDim.x) {
+    if (phk) {
+      for (int e = tid; e < kF32Keys * R; e += 128) {
         const int j = e / R, r = e - (e / R) * R;
         sF[j][r] = (k0 + j < N) ? phk[size_t(k0 + j) * R + r] : 0.f;
       }
+    }
     __syncthreads();
 
     float s[kF32Keys];
@@ -75,9 +99,9 @@ __global__ void __launch_bounds__(128) attn_fwd_f32_kernel(int B, int H, int N, 
     for (int j = 0; j < kF32Keys; ++j) {
       float dot = 0.f, fb = 0.f;
 #pragma unroll
-      for (int u = 0; u < kF32MaxD / 4; ++u) {
-        const int c = sub + 4 * u;
-        if (c < d) dot = fmaf(q[u], sK[j][c], dot);
+      for (int u = 0; u < U; ++u) {
+        const float4 kv = sK[j][sub + 4 * u];
+        dot = fmaf(q[u].x, kv.x, fmaf(q[u].y, kv.y, fmaf(q[u].z, kv.z, fmaf(q[u].w, kv.w, dot))));
       }
       if (phk) {
 #pragma unroll
@@ -102,15 +126,23 @@ __global__ void __launch_bounds__(128) attn_fwd_f32_kernel(int B, int H, int N, 
     const float alpha = expf(m - m_new);
     l *= alpha;
 #pragma unroll
-    for (int u = 0; u < kF32MaxD / 4; ++u) o[u] *= alpha;
+    for (int u = 0; u < U; ++u) {
+      o[u].x *= alpha;
+      o[u].y *= alpha;
+      o[u].z *= alpha;
+      o[u].w *= alpha;
+    }
 #pragma unroll
     for (int j = 0; j < kF32Keys; ++j) {
       const float p = expf(s[j] - m_new);
       l += p;
 #pragma unroll
-      for (int u = 0; u < kF32MaxD / 4; ++u) {
-        const int c = sub + 4 * u;
-        if (c < d) o[u] = fmaf(p, sV[j][c], o[u]);
+      for (int u = 0; u < U; ++u) {
+        const float4 vv = sV[j][sub + 4 * u];
+        o[u].x = fmaf(p, vv.x, o[u].x);
+        o[u].y = fmaf(p, vv.y, o[u].y);
+        o[u].z = fmaf(p, vv.z, o[u].z);
+        o[u].w = fmaf(p, vv.w, o[u].w);
       }
     }
     m = m_new;
@@ -118,10 +150,11 @@ __global__ void __launch_bounds__(128) attn_fwd_f32_kernel(int B, int H, int N, 
 
   if (row_ok) {
     const float inv = l > 0.f ? 1.f / l : 0.f;
+    float4 *O4 = reinterpret_cast<float4 *>(O + head);
 #pragma unroll
-    for (int u = 0; u < kF32MaxD / 4; ++u) {
-      const int c = sub + 4 * u;
-      if (c < d) O[head + size_t(row) * d + c] = o[u] * inv;
+    for (int u = 0; u < U; ++u) {
+      const int c4 = sub + 4 * u;
+      if (c4 < d4) O4[size_t(row) * d4 + c4] = make_float4(o[u].x * inv, o[u].y * inv, o[u].z * inv, o[u].w * inv);
     }
     if (sub == 0) LSE[size_t(bh) * N + row] = l > 0.f ? m + logf(l) : -INFINITY;
   }
@@ -132,9 +165,20 @@ cudaError_t f32_launch(int B, int H, int N, int d, const float *Q, const float *
                        int64_t bias_bs, int64_t bias_hs, float scale, int causal, float *O, float *LSE,
                        cudaStream_t stream) {
   dim3 grid((N + kF32Rows - 1) / kF32Rows, B * H);
-  attn_fwd_f32_kernel<<<grid, 128, 0, stream>>>(B, H, N, d, Q, K, V, R, R > 0 ? phi_q : nullptr,
-                                                 R > 0 ? phi_k : nullptr, phi_bs, phi_hs, bias, bias_bs, bias_hs,
-                                                 scale, causal, O, LSE);
+  const float *pq = R > 0 ? phi_q : nullptr, *pk = R > 0 ? phi_k : nullptr;
+  const int d4 = d / 4;
+#define FB_F32_LAUNCH(DQv)                                                                                         \
+  attn_fwd_f32_kernel<DQv><<<grid, 128, 0, stream>>>(B, H, N, d, Q, K, V, R, pq, pk, phi_bs, phi_hs, bias, bias_bs, \
+                                                      bias_hs, scale, causal, O, LSE)
+  if (d4 <= 4)
+    FB_F32_LAUNCH(4);
+  else if (d4 <= 8)
+    FB_F32_LAUNCH(8);
+  else if (d4 <= 16)
+    FB_F32_LAUNCH(16);
+  else
+    FB_F32_LAUNCH(32);
+#undef FB_F32_LAUNCH
   return cudaGetLastError();
 }
 

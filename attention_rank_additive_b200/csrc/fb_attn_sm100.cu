@@ -94,6 +94,9 @@ struct Sm100Cfg {
   static constexpr uint32_t O_COL0 = SEP_P ? 128 * QT + 64 * QT : 128 * QT;  // + O_STRIDE t
   static constexpr uint32_t O_STRIDE = SEP_P ? DP : 128;
   static_assert(O_COL0 + O_STRIDE * QT <= TMEM_COLS, "TMEM layout");
+  // MMA issuer warps (one per query tile with separate P, else one), each of
+  // which releases every K/V stage once per key step.
+  static constexpr int RELEASERS = SEP_P ? QT : 1;
   static constexpr uint32_t IDESC_QK = make_idesc_f16(true, true, 128, 128, false);
   static constexpr uint32_t IDESC_F = make_idesc_f16(false, false, 128, 128, false);
   static constexpr uint32_t IDESC_PV = make_idesc_f16(true, true, 128, DP, true);
@@ -105,7 +108,7 @@ struct SmemCtrl {
   uint64_t drain[2];
   uint64_t s_free[2], pv_done[2];  // separate-P schedule only
   uint64_t k_full[3], v_full[3];
-  uint64_t k_empty[2][3], v_empty[2][3];  // released by the MMA issuer of each query tile
+  uint64_t k_empty[3], v_empty[3];  // one arrival per MMA issuer per key step
   uint64_t s_full[2], p_full[2];
   uint64_t aux_full[2][3], aux_empty[2][3];
   uint32_t tmem_base;
@@ -165,7 +168,12 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
   const int N = args.N;
   const int fb_slice = (args.fac_B > 1 ? b : 0) * args.fac_H + (args.fac_H > 1 ? h : 0);
 
-  // Per query tile: first row and number of key steps.
+  // Per query tile: first row and number of key tiles. Key tiles are visited
+  // from the last one down (step i reads key tile n_steps - 1 - i), so for a
+  // causal mask the diagonal comes first: biases that decay away from the
+  // diagonal then set the running max at once and O is rarely rescaled. Tile
+  // t is active for steps first[t] .. n_steps - 1 (its local step j = i -
+  // first[t]); in causal attention tile 0 skips the first step.
   int q0[2], nk[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
@@ -175,15 +183,16 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
     nk[t] = active ? (args.causal ? min(qt + 1, args.n_kv) : args.n_kv) : 0;
   }
   const int n_steps = max(nk[0], nk[1]);
+  const int first[2] = {n_steps - nk[0], n_steps - nk[1]};
 
   if (threadIdx.x == 0) {
     mbar_init(&ctrl->q_full, 1);
     for (int s = 0; s < KS; ++s) {
       mbar_init(&ctrl->k_full[s], 1);
       mbar_init(&ctrl->v_full[s], 1);
+      mbar_init(&ctrl->k_empty[s], C::RELEASERS);
+      mbar_init(&ctrl->v_empty[s], C::RELEASERS);
       for (int t = 0; t < QT; ++t) {
-        mbar_init(&ctrl->k_empty[t][s], 1);
-        mbar_init(&ctrl->v_empty[t][s], 1);
         mbar_init(&ctrl->aux_full[t][s], 1);
         mbar_init(&ctrl->aux_empty[t][s], 128);
       }
@@ -251,43 +260,39 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
     for (int i = 0; i < n_steps && ok; ++i) {
       const int s = i % KS;
       const uint32_t ph = uint32_t(i / KS) & 1u;
-      // stage s last held step i - KS: wait until every tile that used it released it
-      if (i >= KS)
-        for (int t = 0; t < QT && ok; ++t)
-          if (i - KS < nk[t]) ok = mbar_wait(&ctrl->k_empty[t][s], ph ^ 1u, abort);
-      if (!ok) break;
+      const int kv = (n_steps - 1 - i) * 128;  // first key of this step's tile
+      // stage s last held step i - KS: wait until every issuer released it
+      if (i >= KS && !(ok = mbar_wait(&ctrl->k_empty[s], ph ^ 1u, abort))) break;
       mbar_arrive_expect_tx_leader(&ctrl->k_full[s], C::KV_TILE + C::FK_TILE, leader);
       for (int ch = 0; ch < C::NDCH; ++ch)
-        tma_load_3d_leader(sK + s * C::KV_TILE + ch * (128 * C::DCH * 2), &tm_k, &ctrl->k_full[s], ch * C::DCH,
-                           i * 128, bh, leader);
+        tma_load_3d_leader(sK + s * C::KV_TILE + ch * (128 * C::DCH * 2), &tm_k, &ctrl->k_full[s], ch * C::DCH, kv,
+                           bh, leader);
       if (MODE == kBiasMma)
         for (int ch = 0; ch < C::NRCH; ++ch)
           tma_load_3d_leader(sFK + s * C::FK_TILE + ch * (128 * C::RCH * 2), &tm_fk, &ctrl->k_full[s], ch * C::RCH,
-                             i * 128, fb_slice, leader);
+                             kv, fb_slice, leader);
       if (C::HAS_AUX) {
         for (int t = 0; t < QT; ++t) {
-          if (i >= nk[t]) continue;
-          if (!(ok = mbar_wait(&ctrl->aux_empty[t][s], ph ^ 1u, abort))) break;
-          uint8_t *dst = sAux + (t * KS + s) * C::AUX_TILE;
-          mbar_arrive_expect_tx_leader(&ctrl->aux_full[t][s], C::AUX_TILE, leader);
+          const int j = i - first[t];  // the tile's local step; its own ring
+          if (j < 0) continue;
+          const int sa = j % KS;
+          if (j >= KS && !(ok = mbar_wait(&ctrl->aux_empty[t][sa], (uint32_t(j / KS) & 1u) ^ 1u, abort))) break;
+          uint8_t *dst = sAux + (t * KS + sa) * C::AUX_TILE;
+          mbar_arrive_expect_tx_leader(&ctrl->aux_full[t][sa], C::AUX_TILE, leader);
           if (MODE == kBiasReg) {
-            tma_load_3d_leader(dst, &tm_fk, &ctrl->aux_full[t][s], 0, i * 128, fb_slice, leader);
+            tma_load_3d_leader(dst, &tm_fk, &ctrl->aux_full[t][sa], 0, kv, fb_slice, leader);
           } else {
-            tma_load_4d_leader(dst, &tm_bias, &ctrl->aux_full[t][s], i * 128, q0[t], hb, bb, leader);
-            tma_load_4d_leader(dst + 128 * 128, &tm_bias, &ctrl->aux_full[t][s], i * 128 + 64, q0[t], hb, bb,
-                               leader);
+            tma_load_4d_leader(dst, &tm_bias, &ctrl->aux_full[t][sa], kv, q0[t], hb, bb, leader);
+            tma_load_4d_leader(dst + 128 * 128, &tm_bias, &ctrl->aux_full[t][sa], kv + 64, q0[t], hb, bb, leader);
           }
         }
         if (!ok) break;
       }
-      if (i >= KS)
-        for (int t = 0; t < QT && ok; ++t)
-          if (i - KS < nk[t]) ok = mbar_wait(&ctrl->v_empty[t][s], ph ^ 1u, abort);
-      if (!ok) break;
+      if (i >= KS && !(ok = mbar_wait(&ctrl->v_empty[s], ph ^ 1u, abort))) break;
       mbar_arrive_expect_tx_leader(&ctrl->v_full[s], C::KV_TILE, leader);
       for (int ch = 0; ch < C::NDCH; ++ch)
-        tma_load_3d_leader(sV + s * C::KV_TILE + ch * (128 * C::DCH * 2), &tm_v, &ctrl->v_full[s], ch * C::DCH,
-                           i * 128, bh, leader);
+        tma_load_3d_leader(sV + s * C::KV_TILE + ch * (128 * C::DCH * 2), &tm_v, &ctrl->v_full[s], ch * C::DCH, kv,
+                           bh, leader);
     }
     if (!ok) {
       // Aborted: let the copies already issued land before the CTA exits.
@@ -337,32 +342,43 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
     if constexpr (C::SEP_P) {
       // One issuer warp per query tile t: S_t(i+1) as soon as the softmax has
       // read S_t(i) into registers, PV_t(i) once P_t(i) is written. The two
-      // tiles' chains are independent and share the tensor core.
+      // tiles' chains are independent and share the tensor core. Every issuer
+      // walks all key steps and releases each K/V stage once per step, also
+      // for steps its tile does not use.
       const int t = warp - C::MMA_WARP;
-      if (ok && nk[t] > 0 && (ok = mbar_wait(&ctrl->k_full[0], 0, abort))) {
-        tc_fence_after();
-        issue_s(t, 0);
-        tc_commit_elect(&ctrl->s_full[t]);
-        tc_commit_elect(&ctrl->k_empty[t][0]);
-      }
-      for (int i = 0; i < nk[t] && ok; ++i) {
+      for (int i = 0; i < n_steps && ok; ++i) {
         const int s = i % KS;
         const uint32_t ph = uint32_t(i / KS) & 1u;
-        if (i + 1 < nk[t]) {
+        const int j = i - first[t];
+        if (j < 0) {
+          if (!(ok = mbar_wait(&ctrl->k_full[s], ph, abort))) break;
+          tc_commit_elect(&ctrl->k_empty[s]);
+          if (!(ok = mbar_wait(&ctrl->v_full[s], ph, abort))) break;
+          tc_commit_elect(&ctrl->v_empty[s]);
+          continue;
+        }
+        if (j == 0) {
+          if (!(ok = mbar_wait(&ctrl->k_full[s], ph, abort))) break;
+          tc_fence_after();
+          issue_s(t, s);
+          tc_commit_elect(&ctrl->s_full[t]);
+          tc_commit_elect(&ctrl->k_empty[s]);
+        }
+        if (i + 1 < n_steps) {
           const int s1 = (i + 1) % KS;
           if (!(ok = mbar_wait(&ctrl->k_full[s1], uint32_t((i + 1) / KS) & 1u, abort))) break;
-          if (!(ok = mbar_wait(&ctrl->s_free[t], uint32_t(i) & 1u, abort))) break;
+          if (!(ok = mbar_wait(&ctrl->s_free[t], uint32_t(j) & 1u, abort))) break;
           tc_fence_after();
           issue_s(t, s1);
           tc_commit_elect(&ctrl->s_full[t]);
-          tc_commit_elect(&ctrl->k_empty[t][s1]);
+          tc_commit_elect(&ctrl->k_empty[s1]);
         }
         if (!(ok = mbar_wait(&ctrl->v_full[s], ph, abort))) break;
-        if (!(ok = mbar_wait(&ctrl->p_full[t], uint32_t(i) & 1u, abort))) break;
+        if (!(ok = mbar_wait(&ctrl->p_full[t], uint32_t(j) & 1u, abort))) break;
         tc_fence_after();
-        issue_pv(t, s, i > 0);
+        issue_pv(t, s, j > 0);
         tc_commit_elect(&ctrl->pv_done[t]);
-        tc_commit_elect(&ctrl->v_empty[t][s]);
+        tc_commit_elect(&ctrl->v_empty[s]);
       }
       tc_commit_elect(&ctrl->o_final[t]);
       if (!ok) {
@@ -371,51 +387,55 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
         if (leader) atomicOr(args.flags, kFlagTimeout);
       }
     } else {
+      // One issuer for both tiles, in the order S_0(i), PV_1(i-1), S_1(i),
+      // PV_0(i) (P overwrites S, so S_t(i+1) must follow PV_t(i)).
+      auto act = [&](int t, int i) { return t < QT && i >= first[t] && i < n_steps; };
       for (int i = 0; i < n_steps && ok; ++i) {
         const int s = i % KS;
         const uint32_t ph = uint32_t(i / KS) & 1u;
         if (!(ok = mbar_wait(&ctrl->k_full[s], ph, abort))) break;
         tc_fence_after();
-        if (i < nk[0]) {
+        if (act(0, i)) {
           issue_s(0, s);
           tc_commit_elect(&ctrl->s_full[0]);
-          tc_commit_elect(&ctrl->k_empty[0][s]);
         }
         if (QT == 2) {
-          const int j = i - 1;  // PV of tile 1 for the previous step
-          if (j >= 0 && j < nk[1]) {
-            const int sj = j % KS;
-            const uint32_t phj = uint32_t(j / KS) & 1u;
-            if (j >= nk[0] && !(ok = mbar_wait(&ctrl->v_full[sj], phj, abort))) break;
-            if (!(ok = mbar_wait(&ctrl->p_full[1], uint32_t(j) & 1u, abort))) break;
+          const int ip = i - 1;  // PV of tile 1 for the previous step
+          if (act(1, ip)) {
+            const int sp = ip % KS;
+            const uint32_t php = uint32_t(ip / KS) & 1u;
+            if (!act(0, ip) && !(ok = mbar_wait(&ctrl->v_full[sp], php, abort))) break;
+            if (!(ok = mbar_wait(&ctrl->p_full[1], uint32_t(ip - first[1]) & 1u, abort))) break;
             tc_fence_after();
-            issue_pv(1, sj, j > 0);
-            tc_commit_elect(&ctrl->v_empty[1][sj]);
+            issue_pv(1, sp, ip > first[1]);
+            tc_commit_elect(&ctrl->v_empty[sp]);
           }
-          if (i < nk[1]) {
+          if (act(1, i)) {
             issue_s(1, s);
             tc_commit_elect(&ctrl->s_full[1]);
-            tc_commit_elect(&ctrl->k_empty[1][s]);
           }
         }
-        if (i < nk[0]) {
+        tc_commit_elect(&ctrl->k_empty[s]);
+        if (act(0, i)) {
           if (!(ok = mbar_wait(&ctrl->v_full[s], ph, abort))) break;
-          if (!(ok = mbar_wait(&ctrl->p_full[0], uint32_t(i) & 1u, abort))) break;
+          if (!(ok = mbar_wait(&ctrl->p_full[0], uint32_t(i - first[0]) & 1u, abort))) break;
           tc_fence_after();
-          issue_pv(0, s, i > 0);
-          tc_commit_elect(&ctrl->v_empty[0][s]);
+          issue_pv(0, s, i > first[0]);
+          if (!act(1, i)) tc_commit_elect(&ctrl->v_empty[s]);
+        } else if (!act(1, i)) {
+          tc_commit_elect(&ctrl->v_empty[s]);  // no tile used this step's V
         }
       }
-      if (ok && QT == 2 && nk[1] == n_steps && n_steps > 0) {
-        const int j = n_steps - 1;
-        const int sj = j % KS;
-        const uint32_t phj = uint32_t(j / KS) & 1u;
-        ok = (j < nk[0]) || mbar_wait(&ctrl->v_full[sj], phj, abort);
-        ok = ok && mbar_wait(&ctrl->p_full[1], uint32_t(j) & 1u, abort);
+      if (ok && act(1, n_steps - 1)) {
+        const int ip = n_steps - 1;
+        const int sp = ip % KS;
+        const uint32_t php = uint32_t(ip / KS) & 1u;
+        ok = act(0, ip) || mbar_wait(&ctrl->v_full[sp], php, abort);
+        ok = ok && mbar_wait(&ctrl->p_full[1], uint32_t(ip - first[1]) & 1u, abort);
         if (ok) {
           tc_fence_after();
-          issue_pv(1, sj, j > 0);
-          tc_commit_elect(&ctrl->v_empty[1][sj]);
+          issue_pv(1, sp, ip > first[1]);
+          tc_commit_elect(&ctrl->v_empty[sp]);
         }
       }
       for (int t = 0; t < QT; ++t) tc_commit_elect(&ctrl->o_final[t]);
@@ -448,8 +468,8 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
 
     float m_use = -INFINITY, l_sum = 0.f;
     bool ok = true;
-    for (int i = 0; i < nk[t]; ++i) {
-      const int s = i % KS;
+    for (int i = 0; i < nk[t]; ++i) {  // i: this tile's local step (key tile nk[t] - 1 - i)
+      const int s = i % KS;             // its own ring of softmax-side tiles
       const uint32_t ph = uint32_t(i / KS) & 1u;
       if (C::HAS_AUX && !(ok = mbar_wait(&ctrl->aux_full[t][s], ph, abort))) break;
       if (!(ok = mbar_wait(&ctrl->s_full[t], uint32_t(i) & 1u, abort))) break;
@@ -510,7 +530,7 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
         mul = 1.f;
       }
       // Causal diagonal tile and the ragged last key tile.
-      const int key0 = i * 128;
+      const int key0 = (nk[t] - 1 - i) * 128;
       if ((args.causal && key0 + 127 > q0[t]) || key0 + 128 > N) {
         const int lim = args.causal ? min(row + 1, N) : N;  // keys [0, lim) are visible
 #pragma unroll
