@@ -5,8 +5,8 @@
 // bias), online softmax over 32-key tiles, O / l and the log-sum-exp.
 //
 // A CTA of 128 threads owns 32 query rows; four threads share a row, each
-// holding every fourth float4 column of q and o and every fourth factor
-// rank, and the row's partial dot products meet through two xor-shuffles.
+// holding every fourth float4 column of q, o and the factors, and the row's
+// partial dot products meet through two xor-shuffles.
 // Key, value and factor tiles are staged in shared memory with all of a
 // tile's global loads in flight before the first store.
 #include <cfloat>
@@ -17,10 +17,10 @@ namespace fb {
 
 constexpr int kF32Rows = 32;
 constexpr int kF32Keys = 32;
-constexpr int kF32MaxR = 128;
 
-// DQ: float4 columns per row after padding (4, 8, 16 or 32; d <= 4 DQ).
-template <int DQ>
+// DQ: float4 columns of q/k/v per row after padding (4, 8, 16 or 32; d <= 4 DQ).
+// FR: float4 columns of the factors after padding (0, 4, 8 or 32; R <= 4 FR).
+template <int DQ, int FR>
 __global__ void __launch_bounds__(128) attn_fwd_f32_kernel(int B, int H, int N, int d, const float *__restrict__ Q,
                                                            const float *__restrict__ K, const float *__restrict__ V,
                                                            int R, const float *__restrict__ phi_q,
@@ -28,10 +28,12 @@ __global__ void __launch_bounds__(128) attn_fwd_f32_kernel(int B, int H, int N, 
                                                            long long phi_hs, const float *__restrict__ bias,
                                                            long long bias_bs, long long bias_hs, float scale,
                                                            int causal, float *__restrict__ O, float *__restrict__ LSE) {
-  constexpr int U = DQ / 4;  // float4 columns per thread
+  constexpr int U = DQ / 4;   // q/k/v float4 columns per thread
+  constexpr int UF = FR / 4;  // factor float4 columns per thread
+  constexpr int FRS = FR > 0 ? FR : 1;
   __shared__ float4 sK[kF32Keys][DQ];
   __shared__ float4 sV[kF32Keys][DQ];
-  __shared__ float sF[kF32Keys][kF32MaxR];
+  __shared__ float4 sF[kF32Keys][FRS];
 
   const int bh = blockIdx.y;
   const int b = bh / H, h = bh - (bh / H) * H;
@@ -56,11 +58,14 @@ __global__ void __launch_bounds__(128) attn_fwd_f32_kernel(int B, int H, int N, 
     q[u] = (row_ok && c4 < d4) ? Q4[size_t(row) * d4 + c4] : zero4;
     o[u] = zero4;
   }
-  float fq[kF32MaxR / 4];
+  float4 fq[UF > 0 ? UF : 1];
 #pragma unroll
-  for (int u = 0; u < kF32MaxR / 4; ++u) {
-    const int r = sub + 4 * u;
-    fq[u] = (row_ok && phq && r < R) ? phq[size_t(row) * R + r] : 0.f;
+  for (int u = 0; u < UF; ++u) {
+    const int r = 4 * (sub + 4 * u);
+    float v[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) v[e] = (row_ok && phq && r + e < R) ? phq[size_t(row) * R + r + e] : 0.f;
+    fq[u] = make_float4(v[0], v[1], v[2], v[3]);
   }
 
   float m = -INFINITY, l = 0.f;
@@ -85,10 +90,19 @@ __global__ void __launch_bounds__(128) attn_fwd_f32_kernel(int B, int H, int N, 
         sV[e / DQ][e % DQ] = vr[it];
       }
     }
-    if (phk) {
-      for (int e = tid; e < kF32Keys * R; e += 128) {
-        const int j = e / R, r = e - (e / R) * R;
-        sF[j][r] = (k0 + j < N) ? phk[size_t(k0 + j) * R + r] : 0.f;
+    if (FR > 0) {
+      constexpr int PERF = kF32Keys * FR * 4 / 128;  // floats per thread
+      float fr[PERF > 0 ? PERF : 1];
+#pragma unroll
+      for (int it = 0; it < PERF; ++it) {
+        const int e = tid + 128 * it;
+        const int j = e / (FRS * 4), r = e % (FRS * 4);
+        fr[it] = (k0 + j < N && r < R) ? phk[size_t(k0 + j) * R + r] : 0.f;
+      }
+#pragma unroll
+      for (int it = 0; it < PERF; ++it) {
+        const int e = tid + 128 * it;
+        reinterpret_cast<float *>(&sF[0][0])[e] = fr[it];
       }
     }
     __syncthreads();
@@ -103,12 +117,10 @@ __global__ void __launch_bounds__(128) attn_fwd_f32_kernel(int B, int H, int N, 
         const float4 kv = sK[j][sub + 4 * u];
         dot = fmaf(q[u].x, kv.x, fmaf(q[u].y, kv.y, fmaf(q[u].z, kv.z, fmaf(q[u].w, kv.w, dot))));
       }
-      if (phk) {
 #pragma unroll
-        for (int u = 0; u < kF32MaxR / 4; ++u) {
-          const int r = sub + 4 * u;
-          if (r < R) fb = fmaf(fq[u], sF[j][r], fb);
-        }
+      for (int u = 0; u < UF; ++u) {
+        const float4 f = sF[j][sub + 4 * u];
+        fb = fmaf(fq[u].x, f.x, fmaf(fq[u].y, f.y, fmaf(fq[u].z, f.z, fmaf(fq[u].w, f.w, fb))));
       }
       dot += __shfl_xor_sync(0xffffffffu, dot, 1);
       dot += __shfl_xor_sync(0xffffffffu, dot, 2);
@@ -167,17 +179,29 @@ cudaError_t f32_launch(int B, int H, int N, int d, const float *Q, const float *
   dim3 grid((N + kF32Rows - 1) / kF32Rows, B * H);
   const float *pq = R > 0 ? phi_q : nullptr, *pk = R > 0 ? phi_k : nullptr;
   const int d4 = d / 4;
-#define FB_F32_LAUNCH(DQv)                                                                                         \
-  attn_fwd_f32_kernel<DQv><<<grid, 128, 0, stream>>>(B, H, N, d, Q, K, V, R, pq, pk, phi_bs, phi_hs, bias, bias_bs, \
-                                                      bias_hs, scale, causal, O, LSE)
-  if (d4 <= 4)
-    FB_F32_LAUNCH(4);
-  else if (d4 <= 8)
-    FB_F32_LAUNCH(8);
-  else if (d4 <= 16)
-    FB_F32_LAUNCH(16);
-  else
-    FB_F32_LAUNCH(32);
+  const int rr = R > 0 ? R : 0;
+#define FB_F32_LAUNCH(DQv, FRv)                                                                                    \
+  attn_fwd_f32_kernel<DQv, FRv><<<grid, 128, 0, stream>>>(B, H, N, d, Q, K, V, R, pq, pk, phi_bs, phi_hs, bias,     \
+                                                           bias_bs, bias_hs, scale, causal, O, LSE)
+#define FB_F32_BY_R(DQv)            \
+  if (rr == 0)                      \
+    FB_F32_LAUNCH(DQv, 0);          \
+  else if (rr <= 16)                \
+    FB_F32_LAUNCH(DQv, 4);          \
+  else if (rr <= 32)                \
+    FB_F32_LAUNCH(DQv, 8);          \
+  else                              \
+    FB_F32_LAUNCH(DQv, 32);
+  if (d4 <= 4) {
+    FB_F32_BY_R(4)
+  } else if (d4 <= 8) {
+    FB_F32_BY_R(8)
+  } else if (d4 <= 16) {
+    FB_F32_BY_R(16)
+  } else {
+    FB_F32_BY_R(32)
+  }
+#undef FB_F32_BY_R
 #undef FB_F32_LAUNCH
   return cudaGetLastError();
 }
