@@ -15,24 +15,34 @@
 // JIT"). The dense mode streams a materialised bias tile per tile pair: the
 // "FlashAttention w/ Bias" comparison path of Figure 1(c).
 //
+// Work items: one (batch, head, group of QT query tiles of 128 rows) each.
+// The grid is persistent (at most as many CTAs as are resident at once); CTA
+// c takes items c, 2G-1-c, 2G+c, ... (G CTAs), heaviest causal groups first,
+// so the heavy and light items of successive passes even out. Barrier phases
+// run on counters that continue across items, so the next item's Q and K/V
+// stream in while the current one finishes, and O is handed back through an
+// o_free barrier once the epilogue has read it.
+//
 // CTA organisation (QT = 1 or 2 query tiles of 128 rows per CTA):
 //   warps 0..4QT-1  softmax warpgroups; warpgroup t owns query tile t, one
 //                   thread per row (TMEM lane), so row max and row sum are
 //                   thread-local; it also rescales O in TMEM when the running
 //                   max grows by more than 2^8 and writes the epilogue.
-//   warp 4QT        TMA producer (one thread): Q|phi_q once, then K|phi_k and
-//                   V per 128-key step into a KS-deep ring, plus the
+//   warp 4QT        TMA producer (one thread): Q|phi_q per item, then K|phi_k
+//                   and V per 128-key step into a KS-deep ring, plus the
 //                   softmax-side tiles (dense bias / rank<=4 factors).
-//   warp 4QT+1      TMEM allocator and MMA issuer (one elected lane).
-// TMEM columns: S_t at 128 t, O_t at 128 QT + 128 t; P_t (bf16) overwrites
-// the first 64 columns of S_t and feeds the PV MMA as the TMEM A operand.
-// MMA issue order per key step i: S_0(i), PV_1(i-1), S_1(i), PV_0(i), so the
-// tensor core works on one tile while the softmax of the other runs. With
-// that order the commit that publishes S_t(i) also covers PV_t(i-1), so the
-// softmax may rescale O_t right after seeing S_t(i), and S_t(i+1) (which
-// overwrites P_t(i)) is issued after PV_t(i) (tcgen05 MMAs of one thread run
-// in order).
+//   warp 4QT+1      TMEM allocator and MMA issuer (one elected lane); with
+//   (and 4QT+2)     a separate P tile (head dim <= 64) one issuer per tile.
+// Head dim <= 64: TMEM holds S_t (128 columns), P_t (64 columns of bf16
+// pairs) and O_t per tile, so S_t(i+1) is computed as soon as the softmax has
+// read S_t(i) into registers, while P_t(i) waits for PV_t(i).
+// Head dim 128: P_t overwrites the first 64 columns of S_t, and one issuer
+// runs S_0(i), PV_1(i-1), S_1(i), PV_0(i), so the tensor core works on one
+// tile while the softmax of the other runs; the commit that publishes S_t(i)
+// also covers PV_t(i-1), and S_t(i+1) (which overwrites P_t(i)) follows
+// PV_t(i) (tcgen05 MMAs of one thread run in order).
 #include <algorithm>
+#include <atomic>
 
 #include "fb_internal.h"
 #include "fb_ptx.cuh"
@@ -78,8 +88,8 @@ struct Sm100Cfg {
   static constexpr int THREADS = QT * 128 + 128;
   static constexpr int MIN_BLOCKS = QT == 1 ? 2 : 1;
   static constexpr int LAUNCH_REGS = QT == 1 ? 128 : 168;
-  static constexpr int REG_SOFTMAX = QT == 1 ? 208 : 216;
-  static constexpr int REG_OTHER = QT == 1 ? 48 : 72;
+  static constexpr int REG_SOFTMAX = QT == 1 ? 192 : 216;
+  static constexpr int REG_OTHER = QT == 1 ? 64 : 72;
   static_assert(QT * 128 * REG_SOFTMAX + 128 * REG_OTHER == THREADS * LAUNCH_REGS, "register split");
   static constexpr int PRODUCER_WARP = QT * 4;
   static constexpr int MMA_WARP = QT * 4 + 1;
@@ -103,8 +113,8 @@ struct Sm100Cfg {
 };
 
 struct SmemCtrl {
-  uint64_t q_full;
-  uint64_t o_final[2];
+  uint64_t q_full, q_empty;
+  uint64_t o_final[2], o_free[2];
   uint64_t drain[2];
   uint64_t s_free[2], pv_done[2];  // separate-P schedule only
   uint64_t k_full[3], v_full[3];
@@ -139,6 +149,52 @@ __host__ __device__ constexpr uint32_t v_step(int kk) {
   return uint32_t(kk * 16 * CH * 2) >> 4;
 }
 
+// One schedulable work item: a group of QT query tiles of one (b, h) head.
+struct WorkItem {
+  int bh, b, h, fb_slice;
+  int q0[2], nk[2], first[2], n_steps;
+};
+
+template <int QT>
+__device__ __forceinline__ WorkItem make_item(int k, const FwdArgs &a) {
+  // Heaviest query groups first (causal work grows with the query index).
+  const int BH = a.B * a.H;
+  WorkItem w;
+  w.bh = k % BH;
+  const int qg = a.n_cta_q - 1 - k / BH;
+  w.b = w.bh / a.H;
+  w.h = w.bh - w.b * a.H;
+  w.fb_slice = (a.fac_B > 1 ? w.b : 0) * a.fac_H + (a.fac_H > 1 ? w.h : 0);
+  // Key tiles are visited from the last one down (step i reads key tile
+  // n_steps - 1 - i), so for a causal mask the diagonal comes first: biases
+  // that decay away from the diagonal then set the running max at once and O
+  // is rarely rescaled. Tile t is active for steps first[t] .. n_steps - 1.
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int qt = qg * QT + t;
+    w.q0[t] = qt * 128;
+    const bool active = (t < QT) && (w.q0[t] < a.N);
+    w.nk[t] = active ? (a.causal ? min(qt + 1, a.n_kv) : a.n_kv) : 0;
+  }
+  w.n_steps = max(w.nk[0], w.nk[1]);
+  w.first[0] = w.n_steps - w.nk[0];
+  w.first[1] = w.n_steps - w.nk[1];
+  return w;
+}
+
+// Entry t of a per-tile pair, by select: t is warp-dependent, and indexing
+// the pair with it would put the work item in local memory.
+__device__ __forceinline__ int pick(const int (&v)[2], int t) { return t == 0 ? v[0] : v[1]; }
+
+// Work item of this CTA's p-th pass, or -1: items are dealt out in passes of
+// gridDim.x, alternating direction each pass so that the heavy items of one
+// pass and the light items of the next even out across CTAs.
+__device__ __forceinline__ int item_of_pass(int p, int n_items) {
+  const int G = int(gridDim.x), c = int(blockIdx.x);
+  const int k = p * G + ((p & 1) ? (G - 1 - c) : c);
+  return k < n_items ? k : -1;
+}
+
 template <int DP, int RP, int MODE, int QT>
 __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<DP, RP, MODE, QT>::MIN_BLOCKS)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -151,42 +207,22 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *sQ = smem;                                     // QT x Q_TILE
-  uint8_t *sFQ = sQ + QT * C::Q_TILE;                     // QT x FQ_TILE
-  uint8_t *sK = sFQ + QT * C::FQ_TILE;                    // KS x KV_TILE
-  uint8_t *sFK = sK + KS * C::KV_TILE;                    // KS x FK_TILE
-  uint8_t *sV = sFK + KS * C::FK_TILE;                    // KS x KV_TILE
-  uint8_t *sAux = sV + KS * C::KV_TILE;                   // QT x KS x AUX_TILE
+  uint8_t *sQ = smem;                    // QT x Q_TILE
+  uint8_t *sFQ = sQ + QT * C::Q_TILE;    // QT x FQ_TILE
+  uint8_t *sK = sFQ + QT * C::FQ_TILE;   // KS x KV_TILE
+  uint8_t *sFK = sK + KS * C::KV_TILE;   // KS x FK_TILE
+  uint8_t *sV = sFK + KS * C::FK_TILE;   // KS x KV_TILE
+  uint8_t *sAux = sV + KS * C::KV_TILE;  // QT x KS x AUX_TILE
   SmemCtrl *ctrl = reinterpret_cast<SmemCtrl *>(sAux + QT * KS * C::AUX_TILE);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.x;
-  const int b = bh / args.H;
-  const int h = bh - b * args.H;
-  const int qg = args.n_cta_q - 1 - int(blockIdx.y);  // heaviest causal row groups first
   const int N = args.N;
-  const int fb_slice = (args.fac_B > 1 ? b : 0) * args.fac_H + (args.fac_H > 1 ? h : 0);
-
-  // Per query tile: first row and number of key tiles. Key tiles are visited
-  // from the last one down (step i reads key tile n_steps - 1 - i), so for a
-  // causal mask the diagonal comes first: biases that decay away from the
-  // diagonal then set the running max at once and O is rarely rescaled. Tile
-  // t is active for steps first[t] .. n_steps - 1 (its local step j = i -
-  // first[t]); in causal attention tile 0 skips the first step.
-  int q0[2], nk[2];
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    const int qt = qg * QT + t;
-    q0[t] = qt * 128;
-    const bool active = (t < QT) && (q0[t] < N);
-    nk[t] = active ? (args.causal ? min(qt + 1, args.n_kv) : args.n_kv) : 0;
-  }
-  const int n_steps = max(nk[0], nk[1]);
-  const int first[2] = {n_steps - nk[0], n_steps - nk[1]};
+  const int n_items = args.n_cta_q * args.B * args.H;
 
   if (threadIdx.x == 0) {
     mbar_init(&ctrl->q_full, 1);
+    mbar_init(&ctrl->q_empty, C::RELEASERS);
     for (int s = 0; s < KS; ++s) {
       mbar_init(&ctrl->k_full[s], 1);
       mbar_init(&ctrl->v_full[s], 1);
@@ -201,6 +237,7 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
       mbar_init(&ctrl->s_full[t], 1);
       mbar_init(&ctrl->p_full[t], 128);
       mbar_init(&ctrl->o_final[t], 1);
+      mbar_init(&ctrl->o_free[t], 128);
       mbar_init(&ctrl->drain[t], 1);
       mbar_init(&ctrl->s_free[t], 128);
       mbar_init(&ctrl->pv_done[t], 1);
@@ -218,6 +255,9 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
   const uint32_t tmem = ctrl->tmem_base;
   volatile int *abort = &ctrl->abort;
 
+  // Barrier phases run on per-role counters that continue across work items:
+  // g counts key steps (K/V ring), it counts items (Q, O), L_t counts the
+  // key steps query tile t has processed (S, P, softmax-side ring).
   if (warp >= QT * 4) {
   setmaxnreg_dec<C::REG_OTHER>();
   // The producer and MMA warps run their loops with all 32 lanes so that
@@ -237,62 +277,70 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
       if (MODE == kBiasReg) tma_prefetch_map(&tm_fk);
       if (MODE == kBiasDense) tma_prefetch_map(&tm_bias);
     }
-    uint32_t qbytes = 0;
-    for (int t = 0; t < QT; ++t)
-      if (nk[t] > 0) qbytes += C::Q_TILE + C::FQ_TILE;
-    mbar_arrive_expect_tx_leader(&ctrl->q_full, qbytes, leader);
-    for (int t = 0; t < QT; ++t) {
-      if (nk[t] == 0) continue;
-      for (int ch = 0; ch < C::NDCH; ++ch)
-        tma_load_3d_leader(sQ + t * C::Q_TILE + ch * (128 * C::DCH * 2), &tm_q, &ctrl->q_full, ch * C::DCH, q0[t], bh,
-                           leader);
-      if (MODE == kBiasMma)
-        for (int ch = 0; ch < C::NRCH; ++ch)
-          tma_load_3d_leader(sFQ + t * C::FQ_TILE + ch * (128 * C::RCH * 2), &tm_fq, &ctrl->q_full, ch * C::RCH,
-                             q0[t], fb_slice, leader);
-    }
-    int hb = 0, bb = 0;
-    if (MODE == kBiasDense) {
-      hb = args.bias_H > 1 ? h : 0;
-      bb = args.bias_B > 1 ? b : 0;
-    }
     bool ok = true;
-    for (int i = 0; i < n_steps && ok; ++i) {
-      const int s = i % KS;
-      const uint32_t ph = uint32_t(i / KS) & 1u;
-      const int kv = (n_steps - 1 - i) * 128;  // first key of this step's tile
-      // stage s last held step i - KS: wait until every issuer released it
-      if (i >= KS && !(ok = mbar_wait(&ctrl->k_empty[s], ph ^ 1u, abort))) break;
-      mbar_arrive_expect_tx_leader(&ctrl->k_full[s], C::KV_TILE + C::FK_TILE, leader);
-      for (int ch = 0; ch < C::NDCH; ++ch)
-        tma_load_3d_leader(sK + s * C::KV_TILE + ch * (128 * C::DCH * 2), &tm_k, &ctrl->k_full[s], ch * C::DCH, kv,
-                           bh, leader);
-      if (MODE == kBiasMma)
-        for (int ch = 0; ch < C::NRCH; ++ch)
-          tma_load_3d_leader(sFK + s * C::FK_TILE + ch * (128 * C::RCH * 2), &tm_fk, &ctrl->k_full[s], ch * C::RCH,
-                             kv, fb_slice, leader);
-      if (C::HAS_AUX) {
-        for (int t = 0; t < QT; ++t) {
-          const int j = i - first[t];  // the tile's local step; its own ring
-          if (j < 0) continue;
-          const int sa = j % KS;
-          if (j >= KS && !(ok = mbar_wait(&ctrl->aux_empty[t][sa], (uint32_t(j / KS) & 1u) ^ 1u, abort))) break;
-          uint8_t *dst = sAux + (t * KS + sa) * C::AUX_TILE;
-          mbar_arrive_expect_tx_leader(&ctrl->aux_full[t][sa], C::AUX_TILE, leader);
-          if (MODE == kBiasReg) {
-            tma_load_3d_leader(dst, &tm_fk, &ctrl->aux_full[t][sa], 0, kv, fb_slice, leader);
-          } else {
-            tma_load_4d_leader(dst, &tm_bias, &ctrl->aux_full[t][sa], kv, q0[t], hb, bb, leader);
-            tma_load_4d_leader(dst + 128 * 128, &tm_bias, &ctrl->aux_full[t][sa], kv + 64, q0[t], hb, bb, leader);
-          }
-        }
-        if (!ok) break;
+    int g = 0, it = 0, la[2] = {0, 0};
+    for (int p = 0; ok; ++p) {
+      if (p * int(gridDim.x) >= n_items) break;
+      const int k = item_of_pass(p, n_items);
+      if (k < 0) continue;
+      const WorkItem w = make_item<QT>(k, args);
+      // Q and phi_q of the item, once the previous item's last S MMAs are done.
+      if (it > 0 && !(ok = mbar_wait(&ctrl->q_empty, uint32_t(it - 1) & 1u, abort))) break;
+      uint32_t qbytes = 0;
+      for (int t = 0; t < QT; ++t)
+        if (w.nk[t] > 0) qbytes += C::Q_TILE + C::FQ_TILE;
+      mbar_arrive_expect_tx_leader(&ctrl->q_full, qbytes, leader);
+      for (int t = 0; t < QT; ++t) {
+        if (w.nk[t] == 0) continue;
+        for (int ch = 0; ch < C::NDCH; ++ch)
+          tma_load_3d_leader(sQ + t * C::Q_TILE + ch * (128 * C::DCH * 2), &tm_q, &ctrl->q_full, ch * C::DCH,
+                             w.q0[t], w.bh, leader);
+        if (MODE == kBiasMma)
+          for (int ch = 0; ch < C::NRCH; ++ch)
+            tma_load_3d_leader(sFQ + t * C::FQ_TILE + ch * (128 * C::RCH * 2), &tm_fq, &ctrl->q_full,
+                               ch * C::RCH, w.q0[t], w.fb_slice, leader);
       }
-      if (i >= KS && !(ok = mbar_wait(&ctrl->v_empty[s], ph ^ 1u, abort))) break;
-      mbar_arrive_expect_tx_leader(&ctrl->v_full[s], C::KV_TILE, leader);
-      for (int ch = 0; ch < C::NDCH; ++ch)
-        tma_load_3d_leader(sV + s * C::KV_TILE + ch * (128 * C::DCH * 2), &tm_v, &ctrl->v_full[s], ch * C::DCH, kv,
-                           bh, leader);
+      const int hb = args.bias_H > 1 ? w.h : 0;
+      const int bb = args.bias_B > 1 ? w.b : 0;
+      for (int i = 0; i < w.n_steps && ok; ++i, ++g) {
+        const int s = g % KS;
+        const uint32_t ph = uint32_t(g / KS) & 1u;
+        const int kv = (w.n_steps - 1 - i) * 128;  // first key of this step's tile
+        // stage s last held step g - KS: wait until every issuer released it
+        if (g >= KS && !(ok = mbar_wait(&ctrl->k_empty[s], ph ^ 1u, abort))) break;
+        mbar_arrive_expect_tx_leader(&ctrl->k_full[s], C::KV_TILE + C::FK_TILE, leader);
+        for (int ch = 0; ch < C::NDCH; ++ch)
+          tma_load_3d_leader(sK + s * C::KV_TILE + ch * (128 * C::DCH * 2), &tm_k, &ctrl->k_full[s], ch * C::DCH,
+                             kv, w.bh, leader);
+        if (MODE == kBiasMma)
+          for (int ch = 0; ch < C::NRCH; ++ch)
+            tma_load_3d_leader(sFK + s * C::FK_TILE + ch * (128 * C::RCH * 2), &tm_fk, &ctrl->k_full[s],
+                               ch * C::RCH, kv, w.fb_slice, leader);
+        if (C::HAS_AUX) {
+          for (int t = 0; t < QT; ++t) {
+            if (i < w.first[t]) continue;
+            const int ja = la[t]++;  // this tile's running step: its own ring
+            const int sa = ja % KS;
+            if (ja >= KS && !(ok = mbar_wait(&ctrl->aux_empty[t][sa], (uint32_t(ja / KS) & 1u) ^ 1u, abort))) break;
+            uint8_t *dst = sAux + (t * KS + sa) * C::AUX_TILE;
+            mbar_arrive_expect_tx_leader(&ctrl->aux_full[t][sa], C::AUX_TILE, leader);
+            if (MODE == kBiasReg) {
+              tma_load_3d_leader(dst, &tm_fk, &ctrl->aux_full[t][sa], 0, kv, w.fb_slice, leader);
+            } else {
+              tma_load_4d_leader(dst, &tm_bias, &ctrl->aux_full[t][sa], kv, w.q0[t], hb, bb, leader);
+              tma_load_4d_leader(dst + 128 * 128, &tm_bias, &ctrl->aux_full[t][sa], kv + 64, w.q0[t], hb, bb,
+                                 leader);
+            }
+          }
+          if (!ok) break;
+        }
+        if (g >= KS && !(ok = mbar_wait(&ctrl->v_empty[s], ph ^ 1u, abort))) break;
+        mbar_arrive_expect_tx_leader(&ctrl->v_full[s], C::KV_TILE, leader);
+        for (int ch = 0; ch < C::NDCH; ++ch)
+          tma_load_3d_leader(sV + s * C::KV_TILE + ch * (128 * C::DCH * 2), &tm_v, &ctrl->v_full[s], ch * C::DCH,
+                             kv, w.bh, leader);
+      }
+      ++it;
     }
     if (!ok) {
       // Aborted: let the copies already issued land before the CTA exits.
@@ -337,50 +385,78 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
       for (int kk = 0; kk < 8; ++kk)
         mma_ts_elect(d_tm, p_tm + uint32_t(kk * 8), dv + v_step<C::DCH>(kk), C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
     };
-    bool ok = mbar_wait(&ctrl->q_full, 0, abort);
-    tc_fence_after();
+    bool ok = true;
+    int g = 0, it = 0;
     if constexpr (C::SEP_P) {
       // One issuer warp per query tile t: S_t(i+1) as soon as the softmax has
       // read S_t(i) into registers, PV_t(i) once P_t(i) is written. The two
       // tiles' chains are independent and share the tensor core. Every issuer
-      // walks all key steps and releases each K/V stage once per step, also
-      // for steps its tile does not use.
+      // walks all key steps and releases each K/V stage and the Q tiles once
+      // per step or item, also where its query tile does no work.
       const int t = warp - C::MMA_WARP;
-      for (int i = 0; i < n_steps && ok; ++i) {
-        const int s = i % KS;
-        const uint32_t ph = uint32_t(i / KS) & 1u;
-        const int j = i - first[t];
-        if (j < 0) {
-          if (!(ok = mbar_wait(&ctrl->k_full[s], ph, abort))) break;
-          tc_commit_elect(&ctrl->k_empty[s]);
-          if (!(ok = mbar_wait(&ctrl->v_full[s], ph, abort))) break;
-          tc_commit_elect(&ctrl->v_empty[s]);
-          continue;
-        }
-        if (j == 0) {
-          if (!(ok = mbar_wait(&ctrl->k_full[s], ph, abort))) break;
-          tc_fence_after();
-          issue_s(t, s);
-          tc_commit_elect(&ctrl->s_full[t]);
-          tc_commit_elect(&ctrl->k_empty[s]);
-        }
-        if (i + 1 < n_steps) {
-          const int s1 = (i + 1) % KS;
-          if (!(ok = mbar_wait(&ctrl->k_full[s1], uint32_t((i + 1) / KS) & 1u, abort))) break;
-          if (!(ok = mbar_wait(&ctrl->s_free[t], uint32_t(j) & 1u, abort))) break;
-          tc_fence_after();
-          issue_s(t, s1);
-          tc_commit_elect(&ctrl->s_full[t]);
-          tc_commit_elect(&ctrl->k_empty[s1]);
-        }
-        if (!(ok = mbar_wait(&ctrl->v_full[s], ph, abort))) break;
-        if (!(ok = mbar_wait(&ctrl->p_full[t], uint32_t(j) & 1u, abort))) break;
+      int L = 0;
+      for (int p = 0; ok; ++p) {
+        if (p * int(gridDim.x) >= n_items) break;
+        const int k = item_of_pass(p, n_items);
+        if (k < 0) continue;
+        const WorkItem w = make_item<QT>(k, args);
+        const int nk_t = pick(w.nk, t), first_t = pick(w.first, t);
+        if (!(ok = mbar_wait(&ctrl->q_full, uint32_t(it) & 1u, abort))) break;
         tc_fence_after();
-        issue_pv(t, s, j > 0);
-        tc_commit_elect(&ctrl->pv_done[t]);
-        tc_commit_elect(&ctrl->v_empty[s]);
+        bool q_released = false;
+        if (nk_t == 0) {
+          tc_commit_elect(&ctrl->q_empty);
+          q_released = true;
+        }
+        for (int i = 0; i < w.n_steps && ok; ++i) {
+          const int gi = g + i;
+          const int s = gi % KS;
+          const uint32_t ph = uint32_t(gi / KS) & 1u;
+          const int j = i - first_t;
+          if (j < 0) {
+            if (!(ok = mbar_wait(&ctrl->k_full[s], ph, abort))) break;
+            tc_commit_elect(&ctrl->k_empty[s]);
+            if (!(ok = mbar_wait(&ctrl->v_full[s], ph, abort))) break;
+            tc_commit_elect(&ctrl->v_empty[s]);
+            continue;
+          }
+          if (j == 0) {
+            if (!(ok = mbar_wait(&ctrl->k_full[s], ph, abort))) break;
+            // S_t overwrites the columns the softmax read at its last step
+            if (L > 0 && !(ok = mbar_wait(&ctrl->s_free[t], uint32_t(L - 1) & 1u, abort))) break;
+            tc_fence_after();
+            issue_s(t, s);
+            tc_commit_elect(&ctrl->s_full[t]);
+            tc_commit_elect(&ctrl->k_empty[s]);
+          }
+          if (i + 1 < w.n_steps) {
+            const int s1 = (gi + 1) % KS;
+            if (!(ok = mbar_wait(&ctrl->k_full[s1], uint32_t((gi + 1) / KS) & 1u, abort))) break;
+            if (!(ok = mbar_wait(&ctrl->s_free[t], uint32_t(L) & 1u, abort))) break;
+            tc_fence_after();
+            issue_s(t, s1);
+            tc_commit_elect(&ctrl->s_full[t]);
+            tc_commit_elect(&ctrl->k_empty[s1]);
+          }
+          if (i + 1 == w.n_steps && !q_released) {
+            tc_commit_elect(&ctrl->q_empty);  // last S of this item issued
+            q_released = true;
+          }
+          if (!(ok = mbar_wait(&ctrl->v_full[s], ph, abort))) break;
+          if (!(ok = mbar_wait(&ctrl->p_full[t], uint32_t(L) & 1u, abort))) break;
+          // the first PV of an item overwrites O_t: its epilogue must have read it
+          if (j == 0 && it > 0 && !(ok = mbar_wait(&ctrl->o_free[t], uint32_t(it - 1) & 1u, abort))) break;
+          tc_fence_after();
+          issue_pv(t, s, j > 0);
+          tc_commit_elect(&ctrl->pv_done[t]);
+          tc_commit_elect(&ctrl->v_empty[s]);
+          ++L;
+        }
+        if (!ok) break;
+        tc_commit_elect(&ctrl->o_final[t]);
+        g += w.n_steps;
+        ++it;
       }
-      tc_commit_elect(&ctrl->o_final[t]);
       if (!ok) {
         tc_commit_elect(&ctrl->drain[t]);
         mbar_wait_for(&ctrl->drain[t], 0, 100000000ull);
@@ -388,57 +464,81 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
       }
     } else {
       // One issuer for both tiles, in the order S_0(i), PV_1(i-1), S_1(i),
-      // PV_0(i) (P overwrites S, so S_t(i+1) must follow PV_t(i)).
-      auto act = [&](int t, int i) { return t < QT && i >= first[t] && i < n_steps; };
-      for (int i = 0; i < n_steps && ok; ++i) {
-        const int s = i % KS;
-        const uint32_t ph = uint32_t(i / KS) & 1u;
-        if (!(ok = mbar_wait(&ctrl->k_full[s], ph, abort))) break;
+      // PV_0(i) (P overwrites S, so S_t(i+1) must follow PV_t(i); tcgen05 MMAs
+      // of one thread run in order).
+      int L[2] = {0, 0};
+      for (int p = 0; ok; ++p) {
+        if (p * int(gridDim.x) >= n_items) break;
+        const int k = item_of_pass(p, n_items);
+        if (k < 0) continue;
+        const WorkItem w = make_item<QT>(k, args);
+        auto act = [&](int t, int i) { return t < QT && i >= w.first[t] && i < w.n_steps; };
+        if (!(ok = mbar_wait(&ctrl->q_full, uint32_t(it) & 1u, abort))) break;
         tc_fence_after();
-        if (act(0, i)) {
-          issue_s(0, s);
-          tc_commit_elect(&ctrl->s_full[0]);
-        }
-        if (QT == 2) {
-          const int ip = i - 1;  // PV of tile 1 for the previous step
-          if (act(1, ip)) {
-            const int sp = ip % KS;
-            const uint32_t php = uint32_t(ip / KS) & 1u;
-            if (!act(0, ip) && !(ok = mbar_wait(&ctrl->v_full[sp], php, abort))) break;
-            if (!(ok = mbar_wait(&ctrl->p_full[1], uint32_t(ip - first[1]) & 1u, abort))) break;
+        for (int i = 0; i < w.n_steps && ok; ++i) {
+          const int gi = g + i;
+          const int s = gi % KS;
+          const uint32_t ph = uint32_t(gi / KS) & 1u;
+          if (!(ok = mbar_wait(&ctrl->k_full[s], ph, abort))) break;
+          tc_fence_after();
+          if (act(0, i)) {
+            issue_s(0, s);
+            tc_commit_elect(&ctrl->s_full[0]);
+          }
+          if (QT == 2) {
+            const int ip = i - 1;  // PV of tile 1 for the previous step
+            if (act(1, ip)) {
+              const int sp = (gi - 1) % KS;
+              const uint32_t php = uint32_t((gi - 1) / KS) & 1u;
+              if (!act(0, ip) && !(ok = mbar_wait(&ctrl->v_full[sp], php, abort))) break;
+              if (!(ok = mbar_wait(&ctrl->p_full[1], uint32_t(L[1]) & 1u, abort))) break;
+              if (ip == w.first[1] && it > 0 && !(ok = mbar_wait(&ctrl->o_free[1], uint32_t(it - 1) & 1u, abort)))
+                break;
+              tc_fence_after();
+              issue_pv(1, sp, ip > w.first[1]);
+              tc_commit_elect(&ctrl->v_empty[sp]);
+              ++L[1];
+            }
+            if (act(1, i)) {
+              issue_s(1, s);
+              tc_commit_elect(&ctrl->s_full[1]);
+            }
+          }
+          tc_commit_elect(&ctrl->k_empty[s]);
+          if (i + 1 == w.n_steps) tc_commit_elect(&ctrl->q_empty);  // last S of this item issued
+          if (act(0, i)) {
+            if (!(ok = mbar_wait(&ctrl->v_full[s], ph, abort))) break;
+            if (!(ok = mbar_wait(&ctrl->p_full[0], uint32_t(L[0]) & 1u, abort))) break;
+            if (i == w.first[0] && it > 0 && !(ok = mbar_wait(&ctrl->o_free[0], uint32_t(it - 1) & 1u, abort)))
+              break;
             tc_fence_after();
-            issue_pv(1, sp, ip > first[1]);
+            issue_pv(0, s, i > w.first[0]);
+            ++L[0];
+            if (!act(1, i)) tc_commit_elect(&ctrl->v_empty[s]);
+          } else if (!act(1, i)) {
+            tc_commit_elect(&ctrl->v_empty[s]);  // no tile used this step's V
+          }
+        }
+        if (ok && act(1, w.n_steps - 1)) {
+          const int ip = w.n_steps - 1;
+          const int gp = g + ip;
+          const int sp = gp % KS;
+          const uint32_t php = uint32_t(gp / KS) & 1u;
+          ok = act(0, ip) || mbar_wait(&ctrl->v_full[sp], php, abort);
+          ok = ok && mbar_wait(&ctrl->p_full[1], uint32_t(L[1]) & 1u, abort);
+          ok = ok && (ip != w.first[1] || it == 0 || mbar_wait(&ctrl->o_free[1], uint32_t(it - 1) & 1u, abort));
+          if (ok) {
+            tc_fence_after();
+            issue_pv(1, sp, ip > w.first[1]);
             tc_commit_elect(&ctrl->v_empty[sp]);
-          }
-          if (act(1, i)) {
-            issue_s(1, s);
-            tc_commit_elect(&ctrl->s_full[1]);
+            ++L[1];
           }
         }
-        tc_commit_elect(&ctrl->k_empty[s]);
-        if (act(0, i)) {
-          if (!(ok = mbar_wait(&ctrl->v_full[s], ph, abort))) break;
-          if (!(ok = mbar_wait(&ctrl->p_full[0], uint32_t(i - first[0]) & 1u, abort))) break;
-          tc_fence_after();
-          issue_pv(0, s, i > first[0]);
-          if (!act(1, i)) tc_commit_elect(&ctrl->v_empty[s]);
-        } else if (!act(1, i)) {
-          tc_commit_elect(&ctrl->v_empty[s]);  // no tile used this step's V
-        }
+        if (!ok) break;
+        for (int t = 0; t < QT; ++t) tc_commit_elect(&ctrl->o_final[t]);
+        g += w.n_steps;
+        ++it;
       }
-      if (ok && act(1, n_steps - 1)) {
-        const int ip = n_steps - 1;
-        const int sp = ip % KS;
-        const uint32_t php = uint32_t(ip / KS) & 1u;
-        ok = act(0, ip) || mbar_wait(&ctrl->v_full[sp], php, abort);
-        ok = ok && mbar_wait(&ctrl->p_full[1], uint32_t(ip - first[1]) & 1u, abort);
-        if (ok) {
-          tc_fence_after();
-          issue_pv(1, sp, ip > first[1]);
-          tc_commit_elect(&ctrl->v_empty[sp]);
-        }
-      }
-      for (int t = 0; t < QT; ++t) tc_commit_elect(&ctrl->o_final[t]);
       if (!ok) {
         // Aborted: wait (bounded) for the MMAs already issued to finish.
         tc_commit_elect(&ctrl->drain[0]);
@@ -453,192 +553,212 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
     const int t = warp >> 2;  // query tile of this warpgroup
     const int wq = warp & 3;  // TMEM lane quarter
     const int r_loc = wq * 32 + lane;
-    const int row = q0[t] + r_loc;
     const uint32_t lane_base = tmem + (uint32_t(wq * 32) << 16);
     const uint32_t s_tm = lane_base + C::S_COL0 + uint32_t(128 * t);
     const uint32_t p_tm = lane_base + C::P_COL0 + C::P_STRIDE * uint32_t(t);
     const uint32_t o_tm = lane_base + C::O_COL0 + C::O_STRIDE * uint32_t(t);
     const float sl2 = args.scale_log2;
-
-    float aq0 = 0.f, aq1 = 0.f, aq2 = 0.f, aq3 = 0.f;
-    if (MODE == kBiasReg && row < N) {
-      const float4 v = *reinterpret_cast<const float4 *>(args.phiq_reg + (size_t(fb_slice) * N + row) * 4);
-      aq0 = v.x, aq1 = v.y, aq2 = v.z, aq3 = v.w;
-    }
-
-    float m_use = -INFINITY, l_sum = 0.f;
     bool ok = true;
-    for (int i = 0; i < nk[t]; ++i) {  // i: this tile's local step (key tile nk[t] - 1 - i)
-      const int s = i % KS;             // its own ring of softmax-side tiles
-      const uint32_t ph = uint32_t(i / KS) & 1u;
-      if (C::HAS_AUX && !(ok = mbar_wait(&ctrl->aux_full[t][s], ph, abort))) break;
-      if (!(ok = mbar_wait(&ctrl->s_full[t], uint32_t(i) & 1u, abort))) break;
-      tc_fence_after();
-
-      // Raw scores of this thread's row; with a softmax-side bias they are
-      // turned into log2-domain logits in place, otherwise the scale is
-      // folded into the exponent below.
-      uint32_t x[128];
-      tmem_ld32(s_tm + 0, x + 0);
-      tmem_ld32(s_tm + 32, x + 32);
-      tmem_ld32(s_tm + 64, x + 64);
-      tmem_ld32(s_tm + 96, x + 96);
-      tmem_ld_wait32(x + 0);
-      tmem_ld_wait32(x + 32);
-      tmem_ld_wait32(x + 64);
-      tmem_ld_wait32(x + 96);
-      if (C::SEP_P) {  // S_t(i) is in registers: the tensor core may overwrite it
-        tc_fence_before();
-        mbar_arrive(&ctrl->s_free[t]);
+    int L = 0, it = 0;
+    for (int p = 0; ok; ++p) {
+      if (p * int(gridDim.x) >= n_items) break;
+      const int k = item_of_pass(p, n_items);
+      if (k < 0) continue;
+      const WorkItem w = make_item<QT>(k, args);
+      const int q0_t = pick(w.q0, t), nk_t = pick(w.nk, t), first_t = pick(w.first, t);
+      const int row = q0_t + r_loc;
+      float aq0 = 0.f, aq1 = 0.f, aq2 = 0.f, aq3 = 0.f;
+      if (MODE == kBiasReg && row < N && nk_t > 0) {
+        const float4 v = *reinterpret_cast<const float4 *>(args.phiq_reg + (size_t(w.fb_slice) * N + row) * 4);
+        aq0 = v.x, aq1 = v.y, aq2 = v.z, aq3 = v.w;
       }
-      float mul = sl2;  // logit = raw * mul
-      if (MODE == kBiasReg) {
-        const uint8_t *fk = sAux + (t * KS + s) * C::AUX_TILE;
-#pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          float v;
-          if (RP <= 2) {
-            const float2 f = *reinterpret_cast<const float2 *>(fk + c * 16);
-            v = fmaf(aq0, f.x, fmaf(aq1, f.y, __uint_as_float(x[c]) * sl2));
-          } else {
-            const float4 f = *reinterpret_cast<const float4 *>(fk + c * 16);
-            v = fmaf(aq0, f.x, fmaf(aq1, f.y, fmaf(aq2, f.z, fmaf(aq3, f.w, __uint_as_float(x[c]) * sl2))));
-          }
-          x[c] = __float_as_uint(v);
+      float m_use = -INFINITY, l_sum = 0.f;
+      for (int i = first_t; i < w.n_steps; ++i) {  // key tile n_steps - 1 - i
+        const int s = L % KS;  // the softmax-side ring runs on L
+        const uint32_t ph = uint32_t(L / KS) & 1u;
+        if (C::HAS_AUX && !(ok = mbar_wait(&ctrl->aux_full[t][s], ph, abort))) break;
+        if (!(ok = mbar_wait(&ctrl->s_full[t], uint32_t(L) & 1u, abort))) break;
+        tc_fence_after();
+
+        // Raw scores of this thread's row; with a softmax-side bias they are
+        // turned into log2-domain logits in place, otherwise the scale is
+        // folded into the exponent below.
+        uint32_t x[128];
+        tmem_ld32(s_tm + 0, x + 0);
+        tmem_ld32(s_tm + 32, x + 32);
+        tmem_ld32(s_tm + 64, x + 64);
+        tmem_ld32(s_tm + 96, x + 96);
+        tmem_ld_wait32(x + 0);
+        tmem_ld_wait32(x + 32);
+        tmem_ld_wait32(x + 64);
+        tmem_ld_wait32(x + 96);
+        if (C::SEP_P) {  // S_t is in registers: the tensor core may overwrite it
+          tc_fence_before();
+          mbar_arrive(&ctrl->s_free[t]);
         }
-        mbar_arrive(&ctrl->aux_empty[t][s]);
-        mul = 1.f;
-      } else if (MODE == kBiasDense) {
-        const uint8_t *tile = sAux + (t * KS + s) * C::AUX_TILE;
+        float mul = sl2;  // logit = raw * mul
+        if (MODE == kBiasReg) {
+          const uint8_t *fk = sAux + (t * KS + s) * C::AUX_TILE;
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
+          for (int c = 0; c < 128; ++c) {
+            float v;
+            if (RP <= 2) {
+              const float2 f = *reinterpret_cast<const float2 *>(fk + c * 16);
+              v = fmaf(aq0, f.x, fmaf(aq1, f.y, __uint_as_float(x[c]) * sl2));
+            } else {
+              const float4 f = *reinterpret_cast<const float4 *>(fk + c * 16);
+              v = fmaf(aq0, f.x, fmaf(aq1, f.y, fmaf(aq2, f.z, fmaf(aq3, f.w, __uint_as_float(x[c]) * sl2))));
+            }
+            x[c] = __float_as_uint(v);
+          }
+          mbar_arrive(&ctrl->aux_empty[t][s]);
+          mul = 1.f;
+        } else if (MODE == kBiasDense) {
+          const uint8_t *tile = sAux + (t * KS + s) * C::AUX_TILE;
 #pragma unroll
-          for (int ck = 0; ck < 8; ++ck) {
-            const uint4 u =
-                *reinterpret_cast<const uint4 *>(tile + hh * 16384 + r_loc * 128 + ((ck ^ (r_loc & 7)) * 16));
-            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+          for (int hh = 0; hh < 2; ++hh) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c = hh * 64 + ck * 8 + 2 * e;
-              x[c] = __float_as_uint(fmaf(__uint_as_float(w[e] << 16), kLog2e, __uint_as_float(x[c]) * sl2));
-              x[c + 1] =
-                  __float_as_uint(fmaf(__uint_as_float(w[e] & 0xFFFF0000u), kLog2e, __uint_as_float(x[c + 1]) * sl2));
+            for (int ck = 0; ck < 8; ++ck) {
+              const uint4 u =
+                  *reinterpret_cast<const uint4 *>(tile + hh * 16384 + r_loc * 128 + ((ck ^ (r_loc & 7)) * 16));
+              const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int c = hh * 64 + ck * 8 + 2 * e;
+                x[c] = __float_as_uint(fmaf(__uint_as_float(wv[e] << 16), kLog2e, __uint_as_float(x[c]) * sl2));
+                x[c + 1] = __float_as_uint(
+                    fmaf(__uint_as_float(wv[e] & 0xFFFF0000u), kLog2e, __uint_as_float(x[c + 1]) * sl2));
+              }
             }
           }
+          mbar_arrive(&ctrl->aux_empty[t][s]);
+          mul = 1.f;
         }
-        mbar_arrive(&ctrl->aux_empty[t][s]);
-        mul = 1.f;
-      }
-      // Causal diagonal tile and the ragged last key tile.
-      const int key0 = (nk[t] - 1 - i) * 128;
-      if ((args.causal && key0 + 127 > q0[t]) || key0 + 128 > N) {
-        const int lim = args.causal ? min(row + 1, N) : N;  // keys [0, lim) are visible
+        // Causal diagonal tile and the ragged last key tile.
+        const int key0 = (w.n_steps - 1 - i) * 128;
+        if ((args.causal && key0 + 127 > q0_t) || key0 + 128 > N) {
+          const int lim = args.causal ? min(row + 1, N) : N;  // keys [0, lim) are visible
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (key0 + c >= lim) x[c] = __float_as_uint(-INFINITY);
-      }
-      float mx;
-      {
-        float mp[8];
+          for (int c = 0; c < 128; ++c)
+            if (key0 + c >= lim) x[c] = __float_as_uint(-INFINITY);
+        }
+        float mx;
+        {
+          // eight independent chains of three-input max (one instruction per
+          // two elements)
+          float mp[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) mp[e] = __uint_as_float(x[e]);
+          for (int e = 0; e < 8; ++e) mp[e] = fmax3(__uint_as_float(x[e]), __uint_as_float(x[8 + e]), __uint_as_float(x[16 + e]));
 #pragma unroll
-        for (int c = 8; c < 128; c += 8)
+          for (int c = 24; c < 120; c += 16)
 #pragma unroll
-          for (int e = 0; e < 8; ++e) mp[e] = fmaxf(mp[e], __uint_as_float(x[c + e]));
-        mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])), fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+            for (int e = 0; e < 8; ++e) mp[e] = fmax3(mp[e], __uint_as_float(x[c + e]), __uint_as_float(x[c + 8 + e]));
+#pragma unroll
+          for (int e = 0; e < 8; ++e) mp[e] = fmaxf(mp[e], __uint_as_float(x[120 + e]));
+          mx = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
+        }
+        const float m_new = fmaxf(m_use, mx * mul);
+        float alpha = 1.f;
+        bool resc = false;
+        if (m_use == -INFINITY || m_new > m_use + kRescaleThreshold) {
+          alpha = (m_use == -INFINITY) ? 0.f : ex2_approx(m_use - m_new);
+          resc = (i > first_t) && (m_use != -INFINITY);
+          m_use = m_new;
+        }
+        l_sum *= alpha;
+        // P of the whole row stays in registers (each 32-column group of x
+        // dies as its 16 bf16 pairs are made) and goes to TMEM at the end, so
+        // the wait for the previous PV_t overlaps the exponentials.
+        const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;
+        const uint64_t mul2 = f2_pack(mul, mul), negm2 = f2_pack(neg_m, neg_m);
+        uint64_t ls[4] = {0, 0, 0, 0};  // packed partial row sums
+        uint32_t pk[64];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const uint64_t a =
+                f2_fma(f2_pack(__uint_as_float(x[q4 * 32 + 2 * e]), __uint_as_float(x[q4 * 32 + 2 * e + 1])), mul2,
+                       negm2);
+            float a0, a1, p0, p1;
+            f2_unpack(a, a0, a1);
+            if (e < kEmuPairs) {
+              ex2_fma_pair(a0, a1, p0, p1);
+            } else {
+              p0 = ex2_approx(a0);
+              p1 = ex2_approx(a1);
+            }
+            ls[e & 3] = f2_add(ls[e & 3], f2_pack(p0, p1));
+            pk[q4 * 16 + e] = pack_bf16x2(p0, p1);
+          }
+        }
+        {
+          float s0, s1, s2, s3, s4, s5, s6, s7;
+          f2_unpack(ls[0], s0, s1);
+          f2_unpack(ls[1], s2, s3);
+          f2_unpack(ls[2], s4, s5);
+          f2_unpack(ls[3], s6, s7);
+          l_sum += ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
+        }
+        if (C::SEP_P && L > 0) {
+          // P_t (and O_t) are still read by the previous PV_t; wait for it.
+          if (!(ok = mbar_wait(&ctrl->pv_done[t], uint32_t(L - 1) & 1u, abort))) break;
+          tc_fence_after();
+        }
+        if (__any_sync(0xffffffffu, resc)) {
+          // PV_t(i-1) has completed (pv_done, or, when P aliases S, the commit
+          // that published S_t(i) covers it).
+#pragma unroll
+          for (int c0 = 0; c0 < DP; c0 += 16) {
+            uint32_t r[16];
+            tmem_ld16(o_tm + c0, r);
+            tmem_ld_wait16(r);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+            tmem_st16(o_tm + c0, r);
+          }
+        }
+        tmem_st32(p_tm, pk);
+        tmem_st32(p_tm + 32, pk + 32);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&ctrl->p_full[t]);
+        ++L;
       }
-      const float m_new = fmaxf(m_use, mx * mul);
-      float alpha = 1.f;
-      bool resc = false;
-      if (m_use == -INFINITY || m_new > m_use + kRescaleThreshold) {
-        alpha = (m_use == -INFINITY) ? 0.f : ex2_approx(m_use - m_new);
-        resc = (i > 0) && (m_use != -INFINITY);
-        m_use = m_new;
-      }
-      l_sum *= alpha;
-      if (C::SEP_P && i > 0) {
-        // O_t and P_t are still read by PV_t(i-1); wait until it has completed.
-        if (!(ok = mbar_wait(&ctrl->pv_done[t], uint32_t(i - 1) & 1u, abort))) break;
-        tc_fence_after();
-      }
-      if (__any_sync(0xffffffffu, resc)) {
-        // PV_t(i-1) has completed (pv_done, or, when P aliases S, the commit
-        // that published S_t(i) covers it).
+      if (!ok) break;
+
+      // ---------------------------------------------------------- epilogue
+      if (!(ok = mbar_wait(&ctrl->o_final[t], uint32_t(it) & 1u, abort))) break;
+      tc_fence_after();
+      if (nk_t > 0) {
+        const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
+        __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(args.O) + (size_t(w.bh) * N + row) * args.d;
 #pragma unroll
         for (int c0 = 0; c0 < DP; c0 += 16) {
           uint32_t r[16];
           tmem_ld16(o_tm + c0, r);
           tmem_ld_wait16(r);
+          if (row < N) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-          tmem_st16(o_tm + c0, r);
-        }
-      }
-      const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;
-      const uint64_t mul2 = f2_pack(mul, mul), negm2 = f2_pack(neg_m, neg_m);
-      uint64_t ls[4] = {0, 0, 0, 0};  // packed partial row sums
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const uint64_t a = f2_fma(f2_pack(__uint_as_float(x[q4 * 32 + 2 * e]), __uint_as_float(x[q4 * 32 + 2 * e + 1])),
-                                    mul2, negm2);
-          float a0, a1, p0, p1;
-          f2_unpack(a, a0, a1);
-          if (e < kEmuPairs) {
-            ex2_fma_pair(a0, a1, p0, p1);
-          } else {
-            p0 = ex2_approx(a0);
-            p1 = ex2_approx(a1);
-          }
-          ls[e & 3] = f2_add(ls[e & 3], f2_pack(p0, p1));
-          pk[e] = pack_bf16x2(p0, p1);
-        }
-        tmem_st16(p_tm + uint32_t(q4 * 16), pk);
-      }
-      {
-        float s0, s1, s2, s3, s4, s5, s6, s7;
-        f2_unpack(ls[0], s0, s1);
-        f2_unpack(ls[1], s2, s3);
-        f2_unpack(ls[2], s4, s5);
-        f2_unpack(ls[3], s6, s7);
-        l_sum += ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&ctrl->p_full[t]);
-    }
-
-    // ------------------------------------------------------------ epilogue
-    if (ok && nk[t] > 0) ok = mbar_wait(&ctrl->o_final[t], 0, abort);
-    if (ok && nk[t] > 0) {
-      tc_fence_after();
-      const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
-      __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(args.O) + (size_t(bh) * N + row) * args.d;
-#pragma unroll
-      for (int c0 = 0; c0 < DP; c0 += 16) {
-        uint32_t r[16];
-        tmem_ld16(o_tm + c0, r);
-        tmem_ld_wait16(r);
-        if (row < N) {
-#pragma unroll
-          for (int v8 = 0; v8 < 2; ++v8) {
-            const int col = c0 + v8 * 8;
-            if (col < args.d) {
-              uint4 u;
-              u.x = pack_bf16x2(__uint_as_float(r[v8 * 8 + 0]) * inv_l, __uint_as_float(r[v8 * 8 + 1]) * inv_l);
-              u.y = pack_bf16x2(__uint_as_float(r[v8 * 8 + 2]) * inv_l, __uint_as_float(r[v8 * 8 + 3]) * inv_l);
-              u.z = pack_bf16x2(__uint_as_float(r[v8 * 8 + 4]) * inv_l, __uint_as_float(r[v8 * 8 + 5]) * inv_l);
-              u.w = pack_bf16x2(__uint_as_float(r[v8 * 8 + 6]) * inv_l, __uint_as_float(r[v8 * 8 + 7]) * inv_l);
-              *reinterpret_cast<uint4 *>(orow + col) = u;
+            for (int v8 = 0; v8 < 2; ++v8) {
+              const int col = c0 + v8 * 8;
+              if (col < args.d) {
+                uint4 u;
+                u.x = pack_bf16x2(__uint_as_float(r[v8 * 8 + 0]) * inv_l, __uint_as_float(r[v8 * 8 + 1]) * inv_l);
+                u.y = pack_bf16x2(__uint_as_float(r[v8 * 8 + 2]) * inv_l, __uint_as_float(r[v8 * 8 + 3]) * inv_l);
+                u.z = pack_bf16x2(__uint_as_float(r[v8 * 8 + 4]) * inv_l, __uint_as_float(r[v8 * 8 + 5]) * inv_l);
+                u.w = pack_bf16x2(__uint_as_float(r[v8 * 8 + 6]) * inv_l, __uint_as_float(r[v8 * 8 + 7]) * inv_l);
+                *reinterpret_cast<uint4 *>(orow + col) = u;
+              }
             }
           }
         }
+        if (row < N)
+          args.LSE[size_t(w.bh) * N + row] = l_sum > 0.f ? (m_use + __log2f(l_sum)) * kLn2 : -INFINITY;
       }
-      if (row < N)
-        args.LSE[size_t(bh) * N + row] = l_sum > 0.f ? (m_use + __log2f(l_sum)) * kLn2 : -INFINITY;
+      tc_fence_before();
+      mbar_arrive(&ctrl->o_free[t]);  // O_t has been read
+      ++it;
     }
     if (!ok) atomicOr(args.flags, kFlagTimeout);
   }
@@ -651,6 +771,10 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
   }
 }
 
+// Per device: the resident CTA capacity of one kernel instantiation (SMs x
+// CTAs per SM), found once together with the attribute checks and settings.
+constexpr int kMaxDevices = 64;
+
 template <int DP, int RP, int MODE, int QT>
 static cudaError_t launch_one(const FwdMaps &m, const FwdArgs &a, cudaStream_t stream) {
   using C = Sm100Cfg<DP, RP, MODE, QT>;
@@ -658,16 +782,47 @@ static cudaError_t launch_one(const FwdMaps &m, const FwdArgs &a, cudaStream_t s
     return cudaErrorInvalidConfiguration;
   } else {
     auto kern = attn_fwd_sm100<DP, RP, MODE, QT>;
-    // setmaxnreg.inc waits until the block's pool has the registers, so the
-    // launch allocation must be exactly what the split assumes.
-    cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+    static std::atomic<int> capacity[kMaxDevices];  // 0: not set up on that device yet
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (fa.numRegs != C::LAUNCH_REGS) return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::SMEM));
-    if (e != cudaSuccess) return e;
-    dim3 grid(a.B * a.H, a.n_cta_q);
-    kern<<<grid, C::THREADS, C::SMEM, stream>>>(m.q, m.k, m.v, m.fq, m.fk, m.bias, a);
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    int cap = capacity[dev].load(std::memory_order_acquire);
+    if (cap == 0) {
+      // setmaxnreg.inc waits until the block's pool has the registers, so the
+      // launch allocation must be exactly what the split assumes.
+      cudaFuncAttributes fa;
+      if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return e;
+      if (fa.numRegs != C::LAUNCH_REGS) return cudaErrorInvalidConfiguration;
+      if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::SMEM))) != cudaSuccess)
+        return e;
+      // All of the SM's unified L1/shared storage as shared memory, so that
+      // MIN_BLOCKS CTAs fit side by side.
+      if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                    int(cudaSharedmemCarveoutMaxShared))) != cudaSuccess)
+        return e;
+      // CTAs per SM from the per-SM limits: shared memory, registers,
+      // threads and the 512 TMEM columns (which no occupancy query knows of).
+      int sms = 0, smem_sm = 0, smem_res = 0, regs_sm = 0, thr_sm = 0;
+      if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+          (e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) != cudaSuccess ||
+          (e = cudaDeviceGetAttribute(&smem_res, cudaDevAttrReservedSharedMemoryPerBlock, dev)) != cudaSuccess ||
+          (e = cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev)) != cudaSuccess ||
+          (e = cudaDeviceGetAttribute(&thr_sm, cudaDevAttrMaxThreadsPerMultiProcessor, dev)) != cudaSuccess)
+        return e;
+      int per_sm = int(512 / C::TMEM_COLS);
+      per_sm = std::min(per_sm, smem_sm / (int(C::SMEM) + smem_res));
+      per_sm = std::min(per_sm, regs_sm / (C::THREADS * C::LAUNCH_REGS));
+      per_sm = std::min(per_sm, thr_sm / C::THREADS);
+      if (per_sm < 1 || sms < 1) return cudaErrorInvalidConfiguration;
+      cap = sms * per_sm;
+      capacity[dev].store(cap, std::memory_order_release);
+    }
+    // Persistent grid: at most as many CTAs as are resident at once, each
+    // walking its share of the work items.
+    const long long items = (long long)a.n_cta_q * a.B * a.H;
+    const long long ctas = std::min<long long>(items, cap);
+    kern<<<dim3(unsigned(ctas)), C::THREADS, C::SMEM, stream>>>(m.q, m.k, m.v, m.fq, m.fk, m.bias, a);
     return cudaGetLastError();
   }
 }

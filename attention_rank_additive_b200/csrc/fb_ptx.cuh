@@ -323,6 +323,13 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// Maximum of three (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float y;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
+  return y;
+}
+
 // Packed fp32 pairs (two lanes of one 64-bit register pair): Blackwell's
 // f32x2 add/sub/fma do two fp32 operations per issued instruction.
 __device__ __forceinline__ uint64_t f2_pack(float a, float b) {
