@@ -95,7 +95,8 @@ WsLayout workspace_layout(int B, int H, int N, int R, int64_t bs, int64_t hs) {
   WsLayout w{0, 0, 0};
   if (R <= 0) return w;
   const size_t fb = size_t(bs == 0 ? 1 : B) * size_t(hs == 0 ? 1 : H);
-  const size_t per = R <= 4 ? fb * size_t(N) * 16 : fb * size_t(N) * size_t(pad_rank(R)) * 2;
+  // rank <= 4: 16 bytes per row (phi_q) and per key rounded up to a key pair (phi_k)
+  const size_t per = R <= 4 ? fb * size_t(N + (N & 1)) * 16 : fb * size_t(N) * size_t(pad_rank(R)) * 2;
   const size_t per_al = (per + 255) & ~size_t(255);
   w.q_off = 0;
   w.k_off = per_al;
@@ -226,9 +227,11 @@ int fb_attn_fwd(int dt, int B, int H, int N, int d, const void *Q, const void *K
         !encode(&maps.fk, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, wk, dims, strides, box, swizzle_for(ch * 2)))
       return FB_ERR_CUDA;
   } else if (mode == kBiasReg) {
-    const uint64_t dims[3] = {4, uint64_t(N), uint64_t(FB)};
-    const uint64_t strides[2] = {16, uint64_t(N) * 16};
-    const uint32_t box[3] = {4u, 128u, 1u};
+    // phi_k by key pairs: RP * 2 floats per pair, 64 pairs per key tile
+    const uint64_t NP = (uint64_t(N) + 1) / 2;
+    const uint64_t dims[3] = {uint64_t(RP) * 2, NP, uint64_t(FB)};
+    const uint64_t strides[2] = {uint64_t(RP) * 8, NP * RP * 8};
+    const uint32_t box[3] = {uint32_t(RP) * 2, 64u, 1u};
     if (!encode(&maps.fk, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, wk, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
       return FB_ERR_CUDA;
   }

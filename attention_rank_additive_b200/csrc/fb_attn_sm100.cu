@@ -70,7 +70,7 @@ struct Sm100Cfg {
   static constexpr uint32_t KV_TILE = BN * DP * 2;
   static constexpr uint32_t FQ_TILE = MODE == kBiasMma ? BM * RP * 2 : 0;
   static constexpr uint32_t FK_TILE = MODE == kBiasMma ? BN * RP * 2 : 0;
-  static constexpr uint32_t AUX_TILE = MODE == kBiasReg ? BN * 16 : (MODE == kBiasDense ? BM * BN * 2 : 0);
+  static constexpr uint32_t AUX_TILE = MODE == kBiasReg ? BN * RP * 4 : (MODE == kBiasDense ? BM * BN * 2 : 0);
   static constexpr bool HAS_AUX = AUX_TILE > 0;
   static constexpr uint32_t FIXED = QT * (Q_TILE + FQ_TILE);
   static constexpr uint32_t STAGE = 2 * KV_TILE + FK_TILE + QT * AUX_TILE;
@@ -325,7 +325,7 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
             uint8_t *dst = sAux + (t * KS + sa) * C::AUX_TILE;
             mbar_arrive_expect_tx_leader(&ctrl->aux_full[t][sa], C::AUX_TILE, leader);
             if (MODE == kBiasReg) {
-              tma_load_3d_leader(dst, &tm_fk, &ctrl->aux_full[t][sa], 0, kv, w.fb_slice, leader);
+              tma_load_3d_leader(dst, &tm_fk, &ctrl->aux_full[t][sa], 0, kv / 2, w.fb_slice, leader);
             } else {
               tma_load_4d_leader(dst, &tm_bias, &ctrl->aux_full[t][sa], kv, w.q0[t], hb, bb, leader);
               tma_load_4d_leader(dst + 128 * 128, &tm_bias, &ctrl->aux_full[t][sa], kv + 64, w.q0[t], hb, bb,
@@ -361,17 +361,22 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
     const uint64_t dk0 = desc_kmajor_base<C::DCH>(smem_u32(sK));
     const uint64_t dfk0 = desc_kmajor_base<C::RCH>(smem_u32(sFK));
     const uint64_t dv0 = desc_v_base<C::DCH>(smem_u32(sV));
+    // The descriptors are made opaque at each call, so that the compiler
+    // does not keep every per-step descriptor of the loop-invariant tiles
+    // live in registers across the issue loop (this warpgroup runs on few).
     auto issue_s = [&](int t, int s) {  // S_t = Q_t K_s^T (+ phi_q' phi_k^T)
       const uint32_t d_tm = tm_u + C::S_COL0 + uint32_t(128 * t);
-      const uint64_t dq = desc_kmajor_base<C::DCH>(smem_u32(sQ + t * C::Q_TILE));
-      const uint64_t dk = dk0 + uint64_t((uint32_t(s) * C::KV_TILE) >> 4);
+      uint64_t dq = desc_kmajor_base<C::DCH>(smem_u32(sQ + t * C::Q_TILE));
+      uint64_t dk = dk0 + uint64_t((uint32_t(s) * C::KV_TILE) >> 4);
+      asm volatile("" : "+l"(dq), "+l"(dk));
 #pragma unroll
       for (int kk = 0; kk < DP / 16; ++kk)
         mma_ss_elect(d_tm, dq + kmajor_step<C::DCH>(kk), dk + kmajor_step<C::DCH>(kk), C::IDESC_QK,
                      kk > 0 ? 1u : 0u);
       if (MODE == kBiasMma) {
-        const uint64_t dfq = desc_kmajor_base<C::RCH>(smem_u32(sFQ + t * C::FQ_TILE));
-        const uint64_t dfk = dfk0 + uint64_t((uint32_t(s) * C::FK_TILE) >> 4);
+        uint64_t dfq = desc_kmajor_base<C::RCH>(smem_u32(sFQ + t * C::FQ_TILE));
+        uint64_t dfk = dfk0 + uint64_t((uint32_t(s) * C::FK_TILE) >> 4);
+        asm volatile("" : "+l"(dfq), "+l"(dfk));
 #pragma unroll
         for (int kk = 0; kk < (MODE == kBiasMma ? RP / 16 : 0); ++kk)
           mma_ss_elect(d_tm, dfq + kmajor_step<C::RCH>(kk), dfk + kmajor_step<C::RCH>(kk), C::IDESC_F, 1u);
@@ -380,7 +385,8 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
     auto issue_pv = [&](int t, int s, bool acc) {  // O_t += P_t V_s, P_t read from TMEM
       const uint32_t d_tm = tm_u + C::O_COL0 + C::O_STRIDE * uint32_t(t);
       const uint32_t p_tm = tm_u + C::P_COL0 + C::P_STRIDE * uint32_t(t);
-      const uint64_t dv = dv0 + uint64_t((uint32_t(s) * C::KV_TILE) >> 4);
+      uint64_t dv = dv0 + uint64_t((uint32_t(s) * C::KV_TILE) >> 4);
+      asm volatile("" : "+l"(dv));
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
         mma_ts_elect(d_tm, p_tm + uint32_t(kk * 8), dv + v_step<C::DCH>(kk), C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
@@ -598,21 +604,29 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
         }
         float mul = sl2;  // logit = raw * mul
         if (MODE == kBiasReg) {
-          const uint8_t *fk = sAux + (t * KS + s) * C::AUX_TILE;
+          // Key pairs: one 16-byte load gives a factor column for two keys,
+          // and the raw scores take the bias in packed pairs; the factors on
+          // the query side carry 1 / scale, so the scale stays in mul.
+          const float4 *fk = reinterpret_cast<const float4 *>(sAux + (t * KS + s) * C::AUX_TILE);
+          const uint64_t a0 = f2_pack(aq0, aq0), a1 = f2_pack(aq1, aq1);
+          const uint64_t a2 = f2_pack(aq2, aq2), a3 = f2_pack(aq3, aq3);
 #pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            float v;
-            if (RP <= 2) {
-              const float2 f = *reinterpret_cast<const float2 *>(fk + c * 16);
-              v = fmaf(aq0, f.x, fmaf(aq1, f.y, __uint_as_float(x[c]) * sl2));
-            } else {
-              const float4 f = *reinterpret_cast<const float4 *>(fk + c * 16);
-              v = fmaf(aq0, f.x, fmaf(aq1, f.y, fmaf(aq2, f.z, fmaf(aq3, f.w, __uint_as_float(x[c]) * sl2))));
+          for (int j = 0; j < 64; ++j) {
+            uint64_t xp = f2_pack(__uint_as_float(x[2 * j]), __uint_as_float(x[2 * j + 1]));
+            const float4 f = fk[j * (RP / 2)];
+            xp = f2_fma(a0, f2_pack(f.x, f.y), xp);
+            xp = f2_fma(a1, f2_pack(f.z, f.w), xp);
+            if (RP > 2) {
+              const float4 g = fk[j * (RP / 2) + 1];
+              xp = f2_fma(a2, f2_pack(g.x, g.y), xp);
+              xp = f2_fma(a3, f2_pack(g.z, g.w), xp);
             }
-            x[c] = __float_as_uint(v);
+            float v0, v1;
+            f2_unpack(xp, v0, v1);
+            x[2 * j] = __float_as_uint(v0);
+            x[2 * j + 1] = __float_as_uint(v1);
           }
           mbar_arrive(&ctrl->aux_empty[t][s]);
-          mul = 1.f;
         } else if (MODE == kBiasDense) {
           const uint8_t *tile = sAux + (t * KS + s) * C::AUX_TILE;
 #pragma unroll

@@ -78,22 +78,35 @@ __global__ void prep_mma_kernel(int N, int R, int RP, int fac_H, const float *__
 
 // Preparation for the CUDA-core factor path (R <= 4, fp32):
 //   out_q[f, n, 0..3] = phi_q * log2(e) (zero padded), out_k[f, n, 0..3] = phi_k.
-__global__ void prep_reg_kernel(int N, int R, int fac_H, const float *__restrict__ pq, const float *__restrict__ pk,
-                                long long bs, long long hs, float4 *__restrict__ oq, float4 *__restrict__ ok,
-                                long long total) {
+// Rank <= 4 (factors applied on the CUDA cores, fp32): phi_q / scale per
+// row as [slice][N] float4, and phi_k by key pairs, so that one 16-byte load
+// gives a factor column for two adjacent keys: pair j (keys 2j, 2j+1) holds
+// (f0[2j], f0[2j+1], f1[2j], f1[2j+1]) and, for RP = 4, a second float4 with
+// f2, f3. A missing key 2j+1 (odd N) has zero factors.
+__global__ void prep_reg_kernel(int N, int R, int RP, int fac_H, const float *__restrict__ pq,
+                                const float *__restrict__ pk, long long bs, long long hs, float inv_scale,
+                                float4 *__restrict__ oq, float4 *__restrict__ ok, long long total) {
+  const long long NP = (N + 1) / 2;
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
        idx += (long long)gridDim.x * blockDim.x) {
-    const long long n = idx % N;
-    const long long f = idx / N;
+    const long long j = idx % NP;
+    const long long f = idx / NP;
     const long long fb = f / fac_H, fh = f - (f / fac_H) * fac_H;
-    const long long src = fb * bs + fh * hs + n * R;
-    float q[4] = {0.f, 0.f, 0.f, 0.f}, k[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int r = 0; r < R; ++r) {
-      q[r] = pq[src + r] * 1.4426950408889634f;
-      k[r] = pk[src + r];
+    float k[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    for (int e = 0; e < 2; ++e) {
+      const long long n = 2 * j + e;
+      if (n >= N) break;
+      const long long src = fb * bs + fh * hs + n * R;
+      float q[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int r = 0; r < R; ++r) {
+        q[r] = pq[src + r] * inv_scale;
+        k[e][r] = pk[src + r];
+      }
+      oq[f * N + n] = make_float4(q[0], q[1], q[2], q[3]);
     }
-    oq[idx] = make_float4(q[0], q[1], q[2], q[3]);
-    ok[idx] = make_float4(k[0], k[1], k[2], k[3]);
+    float4 *dst = ok + (f * NP + j) * (RP / 2);
+    dst[0] = make_float4(k[0][0], k[1][0], k[0][1], k[1][1]);
+    if (RP > 2) dst[1] = make_float4(k[0][2], k[1][2], k[0][3], k[1][3]);
   }
 }
 
@@ -143,8 +156,8 @@ cudaError_t launch_prep_factors(int mode, int B, int H, int N, int R, int RP, co
                                                          static_cast<__half *>(out_q), static_cast<__half *>(out_k),
                                                          flags, total);
   } else {
-    const long long total = (long long)fac_B * fac_H * N;
-    prep_reg_kernel<<<grid_for(total, 256), 256, 0, s>>>(N, R, fac_H, phi_q, phi_k, bs, hs,
+    const long long total = (long long)fac_B * fac_H * ((N + 1) / 2);
+    prep_reg_kernel<<<grid_for(total, 256), 256, 0, s>>>(N, R, RP, fac_H, phi_q, phi_k, bs, hs, 1.0f / scale,
                                                          static_cast<float4 *>(out_q), static_cast<float4 *>(out_k),
                                                          total);
   }
