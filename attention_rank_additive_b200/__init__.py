@@ -21,7 +21,8 @@ __all__ = [
     "FB_ERR_TIMEOUT", "FB_F32", "FB_BF16", "FlashBiasError", "lib", "lib_path", "EXPORTED",
     "fb_status_str", "fb_version", "fb_attn_workspace_bytes", "fb_attn_fwd", "fb_attn_dense_bias_fwd",
     "fb_factors_sandwich", "fb_factors_alibi", "fb_svd_factors_host", "fb_check_device_error",
-    "fb_selftest_wait_timeout", "fb_attn_fwd_noalloc", "attn", "attn_dense_bias", "factors_sandwich", "factors_alibi", "svd_factors",
+    "fb_selftest_wait_timeout", "fb_attn_fwd_noalloc", "fb_attn_prepare_factors", "fb_attn_fwd_prepared", "attn",
+    "PreparedBias", "attn_dense_bias", "factors_sandwich", "factors_alibi", "svd_factors",
     "attn_flops",
 ]
 
@@ -35,7 +36,7 @@ lib_path = os.path.join(_HERE, "libflashbias.so")
 EXPORTED = (
     "fb_status_str", "fb_version", "fb_attn_workspace_bytes", "fb_attn_fwd", "fb_attn_dense_bias_fwd",
     "fb_factors_sandwich", "fb_factors_alibi", "fb_svd_factors_host", "fb_check_device_error",
-    "fb_selftest_wait_timeout", "fb_attn_fwd_noalloc",
+    "fb_selftest_wait_timeout", "fb_attn_fwd_noalloc", "fb_attn_prepare_factors", "fb_attn_fwd_prepared",
 )
 
 
@@ -67,6 +68,11 @@ def lib() -> ctypes.CDLL:
         L.fb_attn_fwd_noalloc.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, i32, vp, vp, i64, i64, f32, i32, vp,
                                           vp, vp]
         L.fb_attn_fwd_noalloc.restype = i32
+        L.fb_attn_prepare_factors.argtypes = [i32, i32, i32, i32, vp, vp, i64, i64, f32, vp, sz, vp]
+        L.fb_attn_prepare_factors.restype = i32
+        L.fb_attn_fwd_prepared.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, i32, i64, i64, f32, i32, vp, vp, vp,
+                                           sz, vp]
+        L.fb_attn_fwd_prepared.restype = i32
         L.fb_attn_dense_bias_fwd.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, i64, i64, f32, i32, vp, vp, vp]
         L.fb_attn_dense_bias_fwd.restype = i32
         L.fb_factors_sandwich.argtypes, L.fb_factors_sandwich.restype = [i32, i32, vp, vp, vp], i32
@@ -97,6 +103,18 @@ def fb_attn_fwd(dt, B, H, N, d, Q, K, V, R, phi_q, phi_k, phi_bstride, phi_hstri
                 workspace, workspace_bytes, stream) -> int:
     return lib().fb_attn_fwd(dt, B, H, N, d, Q, K, V, R, phi_q, phi_k, phi_bstride, phi_hstride, scale, causal, O,
                              LSE, workspace, workspace_bytes, stream)
+
+
+def fb_attn_prepare_factors(B, H, N, R, phi_q, phi_k, phi_bstride, phi_hstride, scale, workspace, workspace_bytes,
+                            stream) -> int:
+    return lib().fb_attn_prepare_factors(B, H, N, R, phi_q, phi_k, phi_bstride, phi_hstride, scale, workspace,
+                                         workspace_bytes, stream)
+
+
+def fb_attn_fwd_prepared(dt, B, H, N, d, Q, K, V, R, phi_bstride, phi_hstride, scale, causal, O, LSE, workspace,
+                         workspace_bytes, stream) -> int:
+    return lib().fb_attn_fwd_prepared(dt, B, H, N, d, Q, K, V, R, phi_bstride, phi_hstride, scale, causal, O, LSE,
+                                      workspace, workspace_bytes, stream)
 
 
 def fb_attn_fwd_noalloc(dt, B, H, N, d, Q, K, V, R, phi_q, phi_k, phi_bstride, phi_hstride, scale, causal, O, LSE,
@@ -199,6 +217,43 @@ def attn(q, k, v, phi_q=None, phi_k=None, scale=None, causal=False, out=None, ls
                        int(bool(causal)), o.data_ptr(), l.data_ptr(), ws_ptr, ws_bytes, _stream(q.device)),
            "fb_attn_fwd")
     return o, l
+
+
+class PreparedBias:
+    """Factors prepared once (fb_attn_prepare_factors) for many bf16 calls.
+
+    phi_q, phi_k as for attn(); B, H, N the shape of the q tensors it will be
+    used with; scale the softmax scale (it is folded into the prepared
+    factors). Call it as attn(q, k, v, causal=...) -> (O, LSE)."""
+
+    def __init__(self, phi_q, phi_k, B: int, H: int, N: int, d: int, scale=None):
+        import torch
+        assert phi_q.dtype == torch.float32 and phi_k.dtype == torch.float32
+        assert phi_q.shape == phi_k.shape and phi_q.stride() == phi_k.stride()
+        assert phi_q.stride(-1) == 1 and phi_q.stride(-2) == phi_q.shape[-1]
+        self.B, self.H, self.N, self.d = B, H, N, d
+        self.R = phi_q.shape[-1]
+        self.scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+        self.bs, self.hs = _factor_strides(phi_q, B, H, N, self.R)
+        self.ws_bytes = fb_attn_workspace_bytes(B, H, N, self.R, self.bs, self.hs)
+        self.workspace = torch.empty(max(self.ws_bytes, 1), device=phi_q.device, dtype=torch.uint8)
+        _check(fb_attn_prepare_factors(B, H, N, self.R, phi_q.data_ptr(), phi_k.data_ptr(), self.bs, self.hs,
+                                       self.scale, self.workspace.data_ptr(), self.ws_bytes,
+                                       _stream(phi_q.device)), "fb_attn_prepare_factors")
+
+    def attn(self, q, k, v, causal=False, out=None, lse=None):
+        import torch
+        assert q.is_cuda and q.dtype == torch.bfloat16 and q.is_contiguous() and k.is_contiguous() \
+            and v.is_contiguous()
+        B, H, N, d = q.shape
+        assert (B, H, N, d) == (self.B, self.H, self.N, self.d)
+        o = torch.empty_like(q) if out is None else out
+        l = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if lse is None else lse
+        _check(fb_attn_fwd_prepared(FB_BF16, B, H, N, d, q.data_ptr(), k.data_ptr(), v.data_ptr(), self.R, self.bs,
+                                    self.hs, self.scale, int(bool(causal)), o.data_ptr(), l.data_ptr(),
+                                    self.workspace.data_ptr(), self.ws_bytes, _stream(q.device)),
+               "fb_attn_fwd_prepared")
+        return o, l
 
 
 def attn_dense_bias(q, k, v, bias, scale=None, causal=False, out=None, lse=None):

@@ -105,8 +105,10 @@ WsLayout workspace_layout(int B, int H, int N, int R, int64_t bs, int64_t hs) {
 }
 
 bool valid_shape_bf16(int B, int H, int N, int d) {
+  // the kernel numbers its work items (B * H * query-tile groups) in int
   return B >= 1 && H >= 1 && N >= 1 && d >= 8 && d <= 128 && d % 8 == 0 && (long long)B * H <= (1ll << 31) - 1 &&
-         (long long)N <= (1ll << 31) - 256 && ((long long)N + 255) / 256 <= 65535;
+         (long long)N <= (1ll << 31) - 256 && ((long long)N + 255) / 256 <= 65535 &&
+         (long long)B * H * (((long long)N + 127) / 128) <= (1ll << 30);
 }
 
 bool valid_scale(float s) { return std::isfinite(s) && s > 0.f; }
@@ -168,6 +170,101 @@ size_t fb_attn_workspace_bytes(int B, int H, int N, int R, int64_t phi_bstride, 
   return workspace_layout(B, H, N, R, phi_bstride, phi_hstride).total;
 }
 
+int fb_attn_prepare_factors(int B, int H, int N, int R, const float *phi_q, const float *phi_k, int64_t phi_bstride,
+                            int64_t phi_hstride, float scale, void *workspace, size_t workspace_bytes, void *stream) {
+  if (R < 0 || R > 128 || B < 1 || H < 1 || N < 1) return FB_ERR_UNSUPPORTED;
+  if (R == 0) return FB_OK;
+  if (!phi_q || !phi_k || phi_bstride < 0 || phi_hstride < 0) return FB_ERR_INVALID_ARG;
+  if (((reinterpret_cast<uintptr_t>(phi_q) | reinterpret_cast<uintptr_t>(phi_k)) & 3u) != 0) return FB_ERR_INVALID_ARG;
+  if (!valid_scale(scale)) return FB_ERR_INVALID_ARG;
+  if ((long long)N > (1ll << 31) - 256) return FB_ERR_UNSUPPORTED;
+  const WsLayout ws = workspace_layout(B, H, N, R, phi_bstride, phi_hstride);
+  if (!workspace || workspace_bytes < ws.total || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return FB_ERR_WORKSPACE;
+  int *flags = device_flags();
+  if (!flags) return FB_ERR_CUDA;
+  const int mode = R <= 4 ? kBiasReg : kBiasMma;
+  const int RP = mode == kBiasMma ? pad_rank(R) : (R <= 2 ? 2 : 4);
+  const int fac_B = phi_bstride == 0 ? 1 : B, fac_H = phi_hstride == 0 ? 1 : H;
+  uint8_t *wsb = static_cast<uint8_t *>(workspace);
+  const cudaError_t e = launch_prep_factors(mode, B, H, N, R, RP, phi_q, phi_k, phi_bstride, phi_hstride, fac_B,
+                                            fac_H, scale, wsb + ws.q_off, wsb + ws.k_off, flags,
+                                            static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FB_OK : FB_ERR_CUDA;
+}
+
+int fb_attn_fwd_prepared(int dt, int B, int H, int N, int d, const void *Q, const void *K, const void *V, int R,
+                         int64_t phi_bstride, int64_t phi_hstride, float scale, int causal, void *O, float *LSE,
+                         const void *workspace, size_t workspace_bytes, void *stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!Q || !K || !V || !O || !LSE) return FB_ERR_INVALID_ARG;
+  if (dt != FB_BF16) return FB_ERR_UNSUPPORTED;
+  if (R < 0 || R > 128) return FB_ERR_UNSUPPORTED;
+  if (R > 0 && (phi_bstride < 0 || phi_hstride < 0)) return FB_ERR_INVALID_ARG;
+  if (!valid_scale(scale)) return FB_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE)) return FB_ERR_INVALID_ARG;
+  if (!valid_shape_bf16(B, H, N, d)) return FB_ERR_UNSUPPORTED;
+
+  const WsLayout ws = workspace_layout(B, H, N, R, phi_bstride, phi_hstride);
+  if (ws.total > 0) {
+    if (!workspace || workspace_bytes < ws.total) return FB_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FB_ERR_WORKSPACE;
+  }
+  const int DP = pad_dim(d);
+  const int mode = R == 0 ? kBiasNone : (R <= 4 ? kBiasReg : kBiasMma);
+  const int RP = mode == kBiasMma ? pad_rank(R) : (mode == kBiasReg ? (R <= 2 ? 2 : 4) : 0);
+  const int fac_B = phi_bstride == 0 ? 1 : B, fac_H = phi_hstride == 0 ? 1 : H;
+  const FwdPlan plan = choose_plan(DP, RP, mode, B * H, N, sm_count());
+  if (sm100_smem_bytes(plan) == 0) return FB_ERR_UNSUPPORTED;
+
+  int *flags = device_flags();
+  if (!flags) return FB_ERR_CUDA;
+
+  FwdMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  const int BH = B * H;
+  if (!encode_qkv(&maps.q, Q, BH, N, d, DP) || !encode_qkv(&maps.k, K, BH, N, d, DP) ||
+      !encode_qkv(&maps.v, V, BH, N, d, DP))
+    return FB_ERR_CUDA;
+  const uint8_t *wsb = static_cast<const uint8_t *>(workspace);
+  void *wq = ws.total ? const_cast<uint8_t *>(wsb) + ws.q_off : nullptr;
+  void *wk = ws.total ? const_cast<uint8_t *>(wsb) + ws.k_off : nullptr;
+  const int FB = fac_B * fac_H;
+  if (mode == kBiasMma) {
+    const int ch = RP > 64 ? 64 : RP;
+    const uint64_t dims[3] = {uint64_t(RP), uint64_t(N), uint64_t(FB)};
+    const uint64_t strides[2] = {uint64_t(RP) * 2, uint64_t(N) * RP * 2};
+    const uint32_t box[3] = {uint32_t(ch), 128u, 1u};
+    if (!encode(&maps.fq, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, wq, dims, strides, box, swizzle_for(ch * 2)) ||
+        !encode(&maps.fk, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, wk, dims, strides, box, swizzle_for(ch * 2)))
+      return FB_ERR_CUDA;
+  } else if (mode == kBiasReg) {
+    // phi_k by key pairs: RP * 2 floats per pair, 64 pairs per key tile
+    const uint64_t NP = (uint64_t(N) + 1) / 2;
+    const uint64_t dims[3] = {uint64_t(RP) * 2, NP, uint64_t(FB)};
+    const uint64_t strides[2] = {uint64_t(RP) * 8, NP * RP * 8};
+    const uint32_t box[3] = {uint32_t(RP) * 2, 64u, 1u};
+    if (!encode(&maps.fk, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, wk, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return FB_ERR_CUDA;
+  }
+
+  FwdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.B = B, a.H = H, a.N = N, a.d = d;
+  a.n_kv = (N + 127) / 128;
+  a.n_cta_q = (a.n_kv + plan.QT - 1) / plan.QT;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.causal = causal ? 1 : 0;
+  a.O = O;
+  a.LSE = LSE;
+  a.phiq_reg = mode == kBiasReg ? static_cast<const float *>(wq) : nullptr;
+  a.fac_B = fac_B, a.fac_H = fac_H;
+  a.bias_B = 1, a.bias_H = 1;
+  a.flags = flags;
+  const cudaError_t e = sm100_launch(plan, maps, a, st);
+  return e == cudaSuccess ? FB_OK : FB_ERR_CUDA;
+}
+
 int fb_attn_fwd(int dt, int B, int H, int N, int d, const void *Q, const void *K, const void *V, int R,
                 const float *phi_q, const float *phi_k, int64_t phi_bstride, int64_t phi_hstride, float scale,
                 int causal, void *O, float *LSE, void *workspace, size_t workspace_bytes, void *stream) {
@@ -192,71 +289,17 @@ int fb_attn_fwd(int dt, int B, int H, int N, int d, const void *Q, const void *K
   }
   if (dt != FB_BF16) return FB_ERR_UNSUPPORTED;
   if (!valid_shape_bf16(B, H, N, d)) return FB_ERR_UNSUPPORTED;
-
   const WsLayout ws = workspace_layout(B, H, N, R, phi_bstride, phi_hstride);
   if (ws.total > 0) {
     if (!workspace || workspace_bytes < ws.total) return FB_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FB_ERR_WORKSPACE;
   }
-  const int DP = pad_dim(d);
-  const int mode = R == 0 ? kBiasNone : (R <= 4 ? kBiasReg : kBiasMma);
-  const int RP = mode == kBiasMma ? pad_rank(R) : (mode == kBiasReg ? (R <= 2 ? 2 : 4) : 0);
-  const int fac_B = phi_bstride == 0 ? 1 : B, fac_H = phi_hstride == 0 ? 1 : H;
-  const FwdPlan plan = choose_plan(DP, RP, mode, B * H, N, sm_count());
-  if (sm100_smem_bytes(plan) == 0) return FB_ERR_UNSUPPORTED;
-
-  int *flags = device_flags();
-  if (!flags) return FB_ERR_CUDA;
-
-  FwdMaps maps;
-  std::memset(&maps, 0, sizeof(maps));
-  const int BH = B * H;
-  if (!encode_qkv(&maps.q, Q, BH, N, d, DP) || !encode_qkv(&maps.k, K, BH, N, d, DP) ||
-      !encode_qkv(&maps.v, V, BH, N, d, DP))
-    return FB_ERR_CUDA;
-  uint8_t *wsb = static_cast<uint8_t *>(workspace);
-  void *wq = ws.total ? wsb + ws.q_off : nullptr;
-  void *wk = ws.total ? wsb + ws.k_off : nullptr;
-  const int FB = fac_B * fac_H;
-  if (mode == kBiasMma) {
-    const int ch = RP > 64 ? 64 : RP;
-    const uint64_t dims[3] = {uint64_t(RP), uint64_t(N), uint64_t(FB)};
-    const uint64_t strides[2] = {uint64_t(RP) * 2, uint64_t(N) * RP * 2};
-    const uint32_t box[3] = {uint32_t(ch), 128u, 1u};
-    if (!encode(&maps.fq, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, wq, dims, strides, box, swizzle_for(ch * 2)) ||
-        !encode(&maps.fk, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, wk, dims, strides, box, swizzle_for(ch * 2)))
-      return FB_ERR_CUDA;
-  } else if (mode == kBiasReg) {
-    // phi_k by key pairs: RP * 2 floats per pair, 64 pairs per key tile
-    const uint64_t NP = (uint64_t(N) + 1) / 2;
-    const uint64_t dims[3] = {uint64_t(RP) * 2, NP, uint64_t(FB)};
-    const uint64_t strides[2] = {uint64_t(RP) * 8, NP * RP * 8};
-    const uint32_t box[3] = {uint32_t(RP) * 2, 64u, 1u};
-    if (!encode(&maps.fk, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, wk, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
-      return FB_ERR_CUDA;
-  }
-
-  cudaError_t e = cudaSuccess;
-  if (mode != kBiasNone) {
-    e = launch_prep_factors(mode, B, H, N, R, RP, phi_q, phi_k, phi_bstride, phi_hstride, fac_B, fac_H, scale, wq, wk,
-                            flags, st);
-    if (e != cudaSuccess) return FB_ERR_CUDA;
-  }
-  FwdArgs a;
-  std::memset(&a, 0, sizeof(a));
-  a.B = B, a.H = H, a.N = N, a.d = d;
-  a.n_kv = (N + 127) / 128;
-  a.n_cta_q = (a.n_kv + plan.QT - 1) / plan.QT;
-  a.scale_log2 = scale * 1.4426950408889634f;
-  a.causal = causal ? 1 : 0;
-  a.O = O;
-  a.LSE = LSE;
-  a.phiq_reg = mode == kBiasReg ? static_cast<const float *>(wq) : nullptr;
-  a.fac_B = fac_B, a.fac_H = fac_H;
-  a.bias_B = 1, a.bias_H = 1;
-  a.flags = flags;
-  e = sm100_launch(plan, maps, a, st);
-  return e == cudaSuccess ? FB_OK : FB_ERR_CUDA;
+  // the preparation step, then the fused kernel, in stream order
+  int rc = fb_attn_prepare_factors(B, H, N, R, phi_q, phi_k, phi_bstride, phi_hstride, scale, workspace,
+                                   workspace_bytes, stream);
+  if (rc != FB_OK) return rc;
+  return fb_attn_fwd_prepared(dt, B, H, N, d, Q, K, V, R, phi_bstride, phi_hstride, scale, causal, O, LSE, workspace,
+                              workspace_bytes, stream);
 }
 
 int fb_attn_dense_bias_fwd(int dt, int B, int H, int N, int d, const void *Q, const void *K, const void *V,

@@ -110,6 +110,41 @@ int fb_attn_fwd(int dt, int B, int H, int N, int d,
                 void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * The two halves of fb_attn_fwd's bf16 path, for factors that are reused
+ * across calls (the Sandwich and ALiBi factors depend only on N, H and the
+ * bias parameters, not on the inputs): fb_attn_prepare_factors writes the
+ * prepared factors into the workspace once, and fb_attn_fwd_prepared runs
+ * the fused kernel alone, as often as needed. fb_attn_fwd is exactly
+ * prepare-then-run on one stream. (FlashBias rebuttal, reply to Reviewer
+ * xU4x, Q6: the decomposition of a static bias is done once, not at every
+ * inference; only dynamic biases need factors per call.)
+ *
+ * fb_attn_prepare_factors: B, H, N, R, phi_q, phi_k, the strides and scale
+ *   as for fb_attn_fwd (scale is folded into the prepared factors). R == 0
+ *   does nothing and returns FB_OK. The workspace (fb_attn_workspace_bytes,
+ *   256-byte aligned) is written on `stream`; the fp32 factors may be freed
+ *   or changed once that work has run.
+ * fb_attn_fwd_prepared: dt must be FB_BF16; every argument as for
+ *   fb_attn_fwd, and B, H, N, R, the strides and scale equal to those of
+ *   the fb_attn_prepare_factors call that filled `workspace` (the library
+ *   cannot check this: other values read the workspace under the wrong
+ *   layout). The workspace is only read, so concurrent calls may share it.
+ * Errors as fb_attn_fwd; both return before launching anything on an
+ * argument error.
+ */
+int fb_attn_prepare_factors(int B, int H, int N, int R,
+                            const float *phi_q, const float *phi_k,
+                            int64_t phi_bstride, int64_t phi_hstride, float scale,
+                            void *workspace, size_t workspace_bytes, void *stream);
+
+int fb_attn_fwd_prepared(int dt, int B, int H, int N, int d,
+                         const void *Q, const void *K, const void *V,
+                         int R, int64_t phi_bstride, int64_t phi_hstride,
+                         float scale, int causal,
+                         void *O, float *LSE,
+                         const void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * fb_attn_fwd for callers that cannot allocate device memory. (The FlashBias
  * paper has no counterpart: this is an interface convenience.)
  *

@@ -181,3 +181,47 @@ def test_fma_pipe_exp2_polynomial_error_bound():
     got = p.astype(np.float64) * np.exp2(n.astype(np.float64))
     rel = np.abs(got / np.exp2(x.astype(np.float64)) - 1.0)
     assert rel.max() < 1e-4
+
+
+def test_prepared_entry_points_reject_bad_arguments_before_launch():
+    need = fb.fb_attn_workspace_bytes(1, 1, 128, 8, 0, 0)
+    prep = dict(B=1, H=1, N=128, R=8, phi_q=FAKE, phi_k=FAKE, phi_bstride=0, phi_hstride=0, scale=0.125,
+                workspace=FAKE, workspace_bytes=need, stream=None)
+
+    def p(**kw):
+        a = dict(prep)
+        a.update(kw)
+        return fb.fb_attn_prepare_factors(**a)
+
+    assert p(R=0, phi_q=0, phi_k=0, workspace=0, workspace_bytes=0) == fb.FB_OK  # nothing to prepare
+    assert p(R=129) == fb.FB_ERR_UNSUPPORTED
+    assert p(N=0) == fb.FB_ERR_UNSUPPORTED
+    assert p(phi_q=0) == fb.FB_ERR_INVALID_ARG
+    assert p(phi_k=FAKE + 2) == fb.FB_ERR_INVALID_ARG
+    assert p(phi_hstride=-1) == fb.FB_ERR_INVALID_ARG
+    assert p(scale=0.0) == fb.FB_ERR_INVALID_ARG
+    assert p(workspace=0) == fb.FB_ERR_WORKSPACE
+    assert p(workspace_bytes=need - 1) == fb.FB_ERR_WORKSPACE
+    assert p(workspace=FAKE + 16) == fb.FB_ERR_WORKSPACE
+
+    run = dict(dt=fb.FB_BF16, B=1, H=1, N=128, d=64, Q=FAKE, K=FAKE, V=FAKE, R=8, phi_bstride=0, phi_hstride=0,
+               scale=0.125, causal=0, O=FAKE, LSE=FAKE, workspace=FAKE, workspace_bytes=need, stream=None)
+
+    def r(**kw):
+        a = dict(run)
+        a.update(kw)
+        return fb.fb_attn_fwd_prepared(**a)
+
+    assert r(dt=fb.FB_F32) == fb.FB_ERR_UNSUPPORTED  # the prepared form is the tensor-core path
+    assert r(Q=0) == fb.FB_ERR_INVALID_ARG
+    assert r(O=FAKE + 8) == fb.FB_ERR_INVALID_ARG
+    assert r(d=12) == fb.FB_ERR_UNSUPPORTED
+    assert r(R=129) == fb.FB_ERR_UNSUPPORTED
+    assert r(scale=-1.0) == fb.FB_ERR_INVALID_ARG
+    assert r(workspace=0) == fb.FB_ERR_WORKSPACE
+    assert r(workspace_bytes=need - 1) == fb.FB_ERR_WORKSPACE
+
+
+def test_shape_limit_on_work_items():
+    # B * H * ceil(N / 128) work items must stay below 2^30 (the kernel counts them in int)
+    assert _fwd(B=65536, H=128, N=16512) == fb.FB_ERR_UNSUPPORTED

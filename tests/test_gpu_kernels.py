@@ -125,6 +125,41 @@ def test_fused_default_plan_many_heads():
     _run_fused(4, 40, 512, 64, 32, True, seed=11)
 
 
+@pytest.mark.parametrize("qt", ["1", "2"])
+def test_fused_persistent_many_items(monkeypatch, qt):
+    # more work items than resident CTAs, ragged last tile: every CTA walks
+    # several items, so barrier phases carry across items
+    monkeypatch.setenv("FLASHBIAS_QUERY_TILES", qt)
+    _run_fused(3, 50, 300, 64, 16, True, seed=13)
+
+
+@pytest.mark.parametrize("R,layout", [(2, "hnr"), (3, "bhnr"), (32, "nr"), (64, "bhnr")])
+def test_prepared_factors_equal_fused_and_reuse(R, layout):
+    """fb_attn_prepare_factors once + fb_attn_fwd_prepared per call gives
+    bit-identical results to fb_attn_fwd, for several inputs, and does not
+    read the fp32 factors after the preparation."""
+    B, H, N, d = 2, 3, 300, 64
+    shape = {"nr": (N, R), "hnr": (H, N, R), "bhnr": (B, H, N, R)}[layout]
+    pq, pk = si.random_factors(shape, math.sqrt(1.0 / R), 31 + R)
+    pq_d, pk_d = dev(pq, "f32"), dev(pk, "f32")
+    prep = fb.PreparedBias(pq_d, pk_d, B, H, N, d)
+    ref = []
+    for seed in (3, 4):
+        q, k, v = (dev(x, "bf16") for x in si.qkv(B, H, N, d, seed, "bf16"))
+        o1, l1 = fb.attn(q, k, v, pq_d, pk_d, causal=True)
+        o2, l2 = prep.attn(q, k, v, causal=True)
+        torch.cuda.synchronize()
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+        ref.append((q, k, v, o1, l1))
+    pq_d.zero_()
+    pk_d.zero_()
+    for q, k, v, o1, l1 in ref:
+        o3, l3 = prep.attn(q, k, v, causal=True)
+        torch.cuda.synchronize()
+        assert torch.equal(o1, o3) and torch.equal(l1, l3)
+    _no_device_error()
+
+
 def test_fused_f32_matches_oracle_tight():
     for (B, H, N, d, R, causal) in [(1, 2, 256, 64, 8, False), (1, 1, 1, 4, 0, True), (2, 1, 300, 128, 5, True),
                                     (1, 3, 33, 12, 128, False)]:
