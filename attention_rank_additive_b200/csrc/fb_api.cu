@@ -91,12 +91,16 @@ struct WsLayout {
   size_t q_off, k_off, total;
 };
 
+// Rank <= 4 factors go to the tensor cores as tf32 hi/lo parts: q' = [qh, qh, ql],
+// k' = [kh, kl, kh] (3R columns, zero-padded to 8 or 16).
+int tf32_cols(int R) { return R <= 2 ? 8 : 16; }
+
 WsLayout workspace_layout(int B, int H, int N, int R, int64_t bs, int64_t hs) {
   WsLayout w{0, 0, 0};
   if (R <= 0) return w;
   const size_t fb = size_t(bs == 0 ? 1 : B) * size_t(hs == 0 ? 1 : H);
-  // rank <= 4: 16 bytes per row (phi_q) and per key rounded up to a key pair (phi_k)
-  const size_t per = R <= 4 ? fb * size_t(N + (N & 1)) * 16 : fb * size_t(N) * size_t(pad_rank(R)) * 2;
+  // rank <= 4: fp32 hi/lo split factors, 8 or 16 columns; else fp16 padded to 16..128
+  const size_t per = R <= 4 ? fb * size_t(N) * size_t(tf32_cols(R)) * 4 : fb * size_t(N) * size_t(pad_rank(R)) * 2;
   const size_t per_al = (per + 255) & ~size_t(255);
   w.q_off = 0;
   w.k_off = per_al;
@@ -183,8 +187,8 @@ int fb_attn_prepare_factors(int B, int H, int N, int R, const float *phi_q, cons
     return FB_ERR_WORKSPACE;
   int *flags = device_flags();
   if (!flags) return FB_ERR_CUDA;
-  const int mode = R <= 4 ? kBiasReg : kBiasMma;
-  const int RP = mode == kBiasMma ? pad_rank(R) : (R <= 2 ? 2 : 4);
+  const int mode = R <= 4 ? kBiasTf32 : kBiasMma;
+  const int RP = mode == kBiasMma ? pad_rank(R) : tf32_cols(R);
   const int fac_B = phi_bstride == 0 ? 1 : B, fac_H = phi_hstride == 0 ? 1 : H;
   uint8_t *wsb = static_cast<uint8_t *>(workspace);
   const cudaError_t e = launch_prep_factors(mode, B, H, N, R, RP, phi_q, phi_k, phi_bstride, phi_hstride, fac_B,
@@ -211,8 +215,8 @@ int fb_attn_fwd_prepared(int dt, int B, int H, int N, int d, const void *Q, cons
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FB_ERR_WORKSPACE;
   }
   const int DP = pad_dim(d);
-  const int mode = R == 0 ? kBiasNone : (R <= 4 ? kBiasReg : kBiasMma);
-  const int RP = mode == kBiasMma ? pad_rank(R) : (mode == kBiasReg ? (R <= 2 ? 2 : 4) : 0);
+  const int mode = R == 0 ? kBiasNone : (R <= 4 ? kBiasTf32 : kBiasMma);
+  const int RP = mode == kBiasMma ? pad_rank(R) : (mode == kBiasTf32 ? tf32_cols(R) : 0);
   const int fac_B = phi_bstride == 0 ? 1 : B, fac_H = phi_hstride == 0 ? 1 : H;
   const FwdPlan plan = choose_plan(DP, RP, mode, B * H, N, sm_count());
   if (sm100_smem_bytes(plan) == 0) return FB_ERR_UNSUPPORTED;
@@ -238,13 +242,12 @@ int fb_attn_fwd_prepared(int dt, int B, int H, int N, int d, const void *Q, cons
     if (!encode(&maps.fq, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, wq, dims, strides, box, swizzle_for(ch * 2)) ||
         !encode(&maps.fk, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, wk, dims, strides, box, swizzle_for(ch * 2)))
       return FB_ERR_CUDA;
-  } else if (mode == kBiasReg) {
-    // phi_k by key pairs: RP * 2 floats per pair, 64 pairs per key tile
-    const uint64_t NP = (uint64_t(N) + 1) / 2;
-    const uint64_t dims[3] = {uint64_t(RP) * 2, NP, uint64_t(FB)};
-    const uint64_t strides[2] = {uint64_t(RP) * 8, NP * RP * 8};
-    const uint32_t box[3] = {uint32_t(RP) * 2, 64u, 1u};
-    if (!encode(&maps.fk, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, wk, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
+  } else if (mode == kBiasTf32) {
+    const uint64_t dims[3] = {uint64_t(RP), uint64_t(N), uint64_t(FB)};
+    const uint64_t strides[2] = {uint64_t(RP) * 4, uint64_t(N) * RP * 4};
+    const uint32_t box[3] = {uint32_t(RP), 128u, 1u};
+    if (!encode(&maps.fq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, wq, dims, strides, box, swizzle_for(RP * 4)) ||
+        !encode(&maps.fk, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, wk, dims, strides, box, swizzle_for(RP * 4)))
       return FB_ERR_CUDA;
   }
 
@@ -257,7 +260,6 @@ int fb_attn_fwd_prepared(int dt, int B, int H, int N, int d, const void *Q, cons
   a.causal = causal ? 1 : 0;
   a.O = O;
   a.LSE = LSE;
-  a.phiq_reg = mode == kBiasReg ? static_cast<const float *>(wq) : nullptr;
   a.fac_B = fac_B, a.fac_H = fac_H;
   a.bias_B = 1, a.bias_H = 1;
   a.flags = flags;

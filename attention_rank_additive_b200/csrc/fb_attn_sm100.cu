@@ -64,17 +64,29 @@ struct Sm100Cfg {
   static constexpr int BN = 128;
   static constexpr int DCH = DP > 64 ? 64 : DP;  // columns per TMA box / swizzle atom
   static constexpr int NDCH = DP / DCH;
-  static constexpr int RCH = (MODE == kBiasMma) ? (RP > 64 ? 64 : RP) : 16;
-  static constexpr int NRCH = (MODE == kBiasMma) ? RP / RCH : 0;
+  // Factor tiles: fp16 [128 x RP] (mma) or fp32 [128 x RP] (tf32). RCH is a
+  // chunk's width in 16-bit units (the descriptors and swizzle are made from
+  // the chunk's byte width, so a tf32 row of RP floats is 2 RP such units).
+  static constexpr bool FAC_MMA = MODE == kBiasMma || MODE == kBiasTf32;
+  static constexpr int RCH = MODE == kBiasMma ? (RP > 64 ? 64 : RP) : (MODE == kBiasTf32 ? 2 * RP : 16);
+  static constexpr int NRCH = MODE == kBiasMma ? RP / RCH : (MODE == kBiasTf32 ? 1 : 0);
   static constexpr uint32_t Q_TILE = BM * DP * 2;
   static constexpr uint32_t KV_TILE = BN * DP * 2;
-  static constexpr uint32_t FQ_TILE = MODE == kBiasMma ? BM * RP * 2 : 0;
-  static constexpr uint32_t FK_TILE = MODE == kBiasMma ? BN * RP * 2 : 0;
-  static constexpr uint32_t AUX_TILE = MODE == kBiasReg ? BN * RP * 4 : (MODE == kBiasDense ? BM * BN * 2 : 0);
+  static constexpr uint32_t FQ_TILE = MODE == kBiasMma ? BM * RP * 2 : (MODE == kBiasTf32 ? BM * RP * 4 : 0);
+  static constexpr uint32_t FK_TILE = MODE == kBiasMma ? BN * RP * 2 : (MODE == kBiasTf32 ? BN * RP * 4 : 0);
+  static constexpr uint32_t AUX_TILE = MODE == kBiasDense ? BM * BN * 2 : 0;
   static constexpr bool HAS_AUX = AUX_TILE > 0;
   static constexpr uint32_t FIXED = QT * (Q_TILE + FQ_TILE);
   static constexpr uint32_t STAGE = 2 * KV_TILE + FK_TILE + QT * AUX_TILE;
-  static constexpr uint32_t CTRL = 1024;  // barriers + TMEM address + abort flag
+  // Key split (head dim 128, one query tile): two softmax warpgroups share
+  // the tile's rows, warpgroup h taking keys 64h .. 64h+63 of every key tile
+  // with its own running max, row sum and O accumulator; the two partial
+  // results are merged once per item in the epilogue. TMEM: S 128 + P 64 +
+  // 2 x O 128 = 448 columns, so S(i+1) never waits for PV(i).
+  static constexpr bool KSPLIT = DP == 128 && QT == 1;
+  static constexpr int NSWG = KSPLIT ? 2 : QT;  // softmax warpgroups
+  static constexpr uint32_t XCH = KSPLIT ? 4u * 2u * 2u * 2u * 32u * 4u : 0u;  // [quarter][half][slot][m,l][lane]
+  static constexpr uint32_t CTRL = 1024 + XCH;  // barriers, TMEM address, abort flag, exchange
   static constexpr uint32_t ALIGN_SLACK = 1024;
   static constexpr int KS_FIT = (kSmemLimit > FIXED + CTRL + ALIGN_SLACK)
                                     ? int((kSmemLimit - FIXED - CTRL - ALIGN_SLACK) / STAGE)
@@ -85,30 +97,33 @@ struct Sm100Cfg {
   // warp and two idle warps. Registers are moved from that warpgroup to the
   // softmax warpgroups with setmaxnreg: the launch allocation is
   // THREADS * LAUNCH_REGS and the shares below add up to exactly that.
-  static constexpr int THREADS = QT * 128 + 128;
-  static constexpr int MIN_BLOCKS = QT == 1 ? 2 : 1;
-  static constexpr int LAUNCH_REGS = QT == 1 ? 128 : 168;
-  static constexpr int REG_SOFTMAX = QT == 1 ? 192 : 216;
-  static constexpr int REG_OTHER = QT == 1 ? 64 : 72;
-  static_assert(QT * 128 * REG_SOFTMAX + 128 * REG_OTHER == THREADS * LAUNCH_REGS, "register split");
-  static constexpr int PRODUCER_WARP = QT * 4;
-  static constexpr int MMA_WARP = QT * 4 + 1;
-  static constexpr uint32_t TMEM_COLS = QT == 2 ? 512 : 256;
-  // With DP <= 64 the bf16 P tile gets its own 64 TMEM columns, so S(i+1)
-  // can be computed while the softmax of S(i) is still running; with DP = 128
-  // P overwrites the first 64 columns of S.
-  static constexpr bool SEP_P = DP <= 64;
+  static constexpr int THREADS = NSWG * 128 + 128;
+  static constexpr bool SMALL = QT == 1 && !KSPLIT;  // two CTAs per SM
+  static constexpr int MIN_BLOCKS = SMALL ? 2 : 1;
+  static constexpr int LAUNCH_REGS = SMALL ? 128 : 168;
+  static constexpr int REG_SOFTMAX = SMALL ? 192 : 216;
+  static constexpr int REG_OTHER = SMALL ? 64 : 72;
+  static_assert(NSWG * 128 * REG_SOFTMAX + 128 * REG_OTHER == THREADS * LAUNCH_REGS, "register split");
+  static constexpr int PRODUCER_WARP = NSWG * 4;
+  static constexpr int MMA_WARP = NSWG * 4 + 1;
+  static constexpr uint32_t TMEM_COLS = SMALL ? 256 : 512;
+  // With DP <= 64 (and with the key split) the bf16 P tile gets its own 64
+  // TMEM columns, so S(i+1) can be computed while the softmax of S(i) is
+  // still running; with DP = 128 and two query tiles P overwrites the first
+  // 64 columns of S.
+  static constexpr bool SEP_P = DP <= 64 || KSPLIT;
   static constexpr uint32_t S_COL0 = 0;                                // + 128 t
   static constexpr uint32_t P_COL0 = SEP_P ? 128 * QT : 0;             // + (SEP_P ? 64 : 128) t
   static constexpr uint32_t P_STRIDE = SEP_P ? 64 : 128;
-  static constexpr uint32_t O_COL0 = SEP_P ? 128 * QT + 64 * QT : 128 * QT;  // + O_STRIDE t
+  static constexpr uint32_t O_COL0 = SEP_P ? 128 * QT + 64 * QT : 128 * QT;  // + O_STRIDE t (or half h)
   static constexpr uint32_t O_STRIDE = SEP_P ? DP : 128;
-  static_assert(O_COL0 + O_STRIDE * QT <= TMEM_COLS, "TMEM layout");
-  // MMA issuer warps (one per query tile with separate P, else one), each of
-  // which releases every K/V stage once per key step.
-  static constexpr int RELEASERS = SEP_P ? QT : 1;
+  static_assert(O_COL0 + O_STRIDE * (KSPLIT ? 2 : QT) <= TMEM_COLS, "TMEM layout");
+  // MMA issuer warps (one per query tile or key half with separate P, else
+  // one), each of which releases every K/V stage once per key step.
+  static constexpr int RELEASERS = SEP_P ? NSWG : 1;
   static constexpr uint32_t IDESC_QK = make_idesc_f16(true, true, 128, 128, false);
-  static constexpr uint32_t IDESC_F = make_idesc_f16(false, false, 128, 128, false);
+  static constexpr uint32_t IDESC_F =
+      MODE == kBiasTf32 ? make_idesc_tf32(128, 128) : make_idesc_f16(false, false, 128, 128, false);
   static constexpr uint32_t IDESC_PV = make_idesc_f16(true, true, 128, DP, true);
 };
 
@@ -121,6 +136,7 @@ struct SmemCtrl {
   uint64_t k_empty[3], v_empty[3];  // one arrival per MMA issuer per key step
   uint64_t s_full[2], p_full[2];
   uint64_t aux_full[2][3], aux_empty[2][3];
+  uint64_t pair[4];  // key split: the two halves of a 32-row quarter exchange (m, l)
   uint32_t tmem_base;
   int abort;
 };
@@ -147,6 +163,25 @@ __device__ __forceinline__ uint64_t desc_v_base(uint32_t base) {
 template <int CH>
 __host__ __device__ constexpr uint32_t v_step(int kk) {
   return uint32_t(kk * 16 * CH * 2) >> 4;
+}
+
+// Maximum of the NC floats (bit patterns) in x: eight independent chains of
+// three-input max, one instruction per two elements.
+template <int NC>
+__device__ __forceinline__ float row_max(const uint32_t *x) {
+  static_assert(NC % 8 == 0 && NC >= 24, "row_max");
+  float mp[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) mp[e] = fmax3(__uint_as_float(x[e]), __uint_as_float(x[8 + e]), __uint_as_float(x[16 + e]));
+#pragma unroll
+  for (int c = 24; c + 16 <= NC; c += 16)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) mp[e] = fmax3(mp[e], __uint_as_float(x[c + e]), __uint_as_float(x[c + 8 + e]));
+  if constexpr ((NC - 24) % 16 == 8) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) mp[e] = fmaxf(mp[e], __uint_as_float(x[NC - 8 + e]));
+  }
+  return fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
 }
 
 // One schedulable work item: a group of QT query tiles of one (b, h) head.
@@ -230,17 +265,26 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
       mbar_init(&ctrl->v_empty[s], C::RELEASERS);
       for (int t = 0; t < QT; ++t) {
         mbar_init(&ctrl->aux_full[t][s], 1);
-        mbar_init(&ctrl->aux_empty[t][s], 128);
+        mbar_init(&ctrl->aux_empty[t][s], C::KSPLIT ? 256 : 128);
       }
     }
     for (int t = 0; t < QT; ++t) {
       mbar_init(&ctrl->s_full[t], 1);
       mbar_init(&ctrl->p_full[t], 128);
       mbar_init(&ctrl->o_final[t], 1);
-      mbar_init(&ctrl->o_free[t], 128);
+      mbar_init(&ctrl->o_free[t], C::KSPLIT ? 256 : 128);
       mbar_init(&ctrl->drain[t], 1);
-      mbar_init(&ctrl->s_free[t], 128);
+      mbar_init(&ctrl->s_free[t], C::KSPLIT ? 256 : 128);
       mbar_init(&ctrl->pv_done[t], 1);
+    }
+    if (C::KSPLIT) {
+      for (int t = 0; t < 2; ++t) {  // per key half: P hand-over, PV completion, final O
+        mbar_init(&ctrl->p_full[t], 128);
+        mbar_init(&ctrl->pv_done[t], 1);
+        mbar_init(&ctrl->o_final[t], 1);
+        mbar_init(&ctrl->drain[t], 1);
+      }
+      for (int q = 0; q < 4; ++q) mbar_init(&ctrl->pair[q], 64);
     }
     ctrl->abort = 0;
     fence_mbar_init();
@@ -258,7 +302,7 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
   // Barrier phases run on per-role counters that continue across work items:
   // g counts key steps (K/V ring), it counts items (Q, O), L_t counts the
   // key steps query tile t has processed (S, P, softmax-side ring).
-  if (warp >= QT * 4) {
+  if (warp >= C::PRODUCER_WARP) {
   setmaxnreg_dec<C::REG_OTHER>();
   // The producer and MMA warps run their loops with all 32 lanes so that
   // coordinates and descriptors stay warp-uniform; lane 0 alone issues each
@@ -270,11 +314,10 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
       tma_prefetch_map(&tm_q);
       tma_prefetch_map(&tm_k);
       tma_prefetch_map(&tm_v);
-      if (MODE == kBiasMma) {
+      if (C::FAC_MMA) {
         tma_prefetch_map(&tm_fq);
         tma_prefetch_map(&tm_fk);
       }
-      if (MODE == kBiasReg) tma_prefetch_map(&tm_fk);
       if (MODE == kBiasDense) tma_prefetch_map(&tm_bias);
     }
     bool ok = true;
@@ -295,7 +338,7 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
         for (int ch = 0; ch < C::NDCH; ++ch)
           tma_load_3d_leader(sQ + t * C::Q_TILE + ch * (128 * C::DCH * 2), &tm_q, &ctrl->q_full, ch * C::DCH,
                              w.q0[t], w.bh, leader);
-        if (MODE == kBiasMma)
+        if (C::FAC_MMA)
           for (int ch = 0; ch < C::NRCH; ++ch)
             tma_load_3d_leader(sFQ + t * C::FQ_TILE + ch * (128 * C::RCH * 2), &tm_fq, &ctrl->q_full,
                                ch * C::RCH, w.q0[t], w.fb_slice, leader);
@@ -312,7 +355,7 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
         for (int ch = 0; ch < C::NDCH; ++ch)
           tma_load_3d_leader(sK + s * C::KV_TILE + ch * (128 * C::DCH * 2), &tm_k, &ctrl->k_full[s], ch * C::DCH,
                              kv, w.bh, leader);
-        if (MODE == kBiasMma)
+        if (C::FAC_MMA)
           for (int ch = 0; ch < C::NRCH; ++ch)
             tma_load_3d_leader(sFK + s * C::FK_TILE + ch * (128 * C::RCH * 2), &tm_fk, &ctrl->k_full[s],
                                ch * C::RCH, kv, w.fb_slice, leader);
@@ -324,13 +367,8 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
             if (ja >= KS && !(ok = mbar_wait(&ctrl->aux_empty[t][sa], (uint32_t(ja / KS) & 1u) ^ 1u, abort))) break;
             uint8_t *dst = sAux + (t * KS + sa) * C::AUX_TILE;
             mbar_arrive_expect_tx_leader(&ctrl->aux_full[t][sa], C::AUX_TILE, leader);
-            if (MODE == kBiasReg) {
-              tma_load_3d_leader(dst, &tm_fk, &ctrl->aux_full[t][sa], 0, kv / 2, w.fb_slice, leader);
-            } else {
-              tma_load_4d_leader(dst, &tm_bias, &ctrl->aux_full[t][sa], kv, w.q0[t], hb, bb, leader);
-              tma_load_4d_leader(dst + 128 * 128, &tm_bias, &ctrl->aux_full[t][sa], kv + 64, w.q0[t], hb, bb,
-                                 leader);
-            }
+            tma_load_4d_leader(dst, &tm_bias, &ctrl->aux_full[t][sa], kv, w.q0[t], hb, bb, leader);
+            tma_load_4d_leader(dst + 128 * 128, &tm_bias, &ctrl->aux_full[t][sa], kv + 64, w.q0[t], hb, bb, leader);
           }
           if (!ok) break;
         }
@@ -352,7 +390,7 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
       }
       if (leader) atomicOr(args.flags, kFlagTimeout);
     }
-  } else if (warp == C::MMA_WARP || (C::SEP_P && QT == 2 && warp == C::MMA_WARP + 1)) {
+  } else if (warp == C::MMA_WARP || (C::SEP_P && C::NSWG == 2 && warp == C::MMA_WARP + 1)) {
     // ---------------------------------------------------------- MMA issuer
     // Descriptors of every tile base, computed once; each MMA adds a
     // compile-time step offset (the start address is the low field, and
@@ -373,13 +411,18 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
       for (int kk = 0; kk < DP / 16; ++kk)
         mma_ss_elect(d_tm, dq + kmajor_step<C::DCH>(kk), dk + kmajor_step<C::DCH>(kk), C::IDESC_QK,
                      kk > 0 ? 1u : 0u);
-      if (MODE == kBiasMma) {
+      if (C::FAC_MMA) {
         uint64_t dfq = desc_kmajor_base<C::RCH>(smem_u32(sFQ + t * C::FQ_TILE));
         uint64_t dfk = dfk0 + uint64_t((uint32_t(s) * C::FK_TILE) >> 4);
         asm volatile("" : "+l"(dfq), "+l"(dfk));
 #pragma unroll
-        for (int kk = 0; kk < (MODE == kBiasMma ? RP / 16 : 0); ++kk)
-          mma_ss_elect(d_tm, dfq + kmajor_step<C::RCH>(kk), dfk + kmajor_step<C::RCH>(kk), C::IDESC_F, 1u);
+        // one MMA step covers 32 bytes of a row: 16 fp16 or 8 tf32 factor columns
+        for (int kk = 0; kk < (C::FAC_MMA ? C::RCH * C::NRCH / 16 : 0); ++kk) {
+          if (MODE == kBiasTf32)
+            mma_ss_elect_tf32(d_tm, dfq + kmajor_step<C::RCH>(kk), dfk + kmajor_step<C::RCH>(kk), C::IDESC_F, 1u);
+          else
+            mma_ss_elect(d_tm, dfq + kmajor_step<C::RCH>(kk), dfk + kmajor_step<C::RCH>(kk), C::IDESC_F, 1u);
+        }
       }
     };
     auto issue_pv = [&](int t, int s, bool acc) {  // O_t += P_t V_s, P_t read from TMEM
@@ -391,9 +434,88 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
       for (int kk = 0; kk < 8; ++kk)
         mma_ts_elect(d_tm, p_tm + uint32_t(kk * 8), dv + v_step<C::DCH>(kk), C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
     };
+    // Key split: O_h += P[:, keys of half h] V_s[keys of half h] (MMA K-steps
+    // 4h .. 4h+3 of the 128 keys).
+    auto issue_pv_half = [&](int hh, int s, bool acc) {
+      const uint32_t d_tm = tm_u + C::O_COL0 + C::O_STRIDE * uint32_t(hh);
+      const uint32_t p_tm = tm_u + C::P_COL0;
+      uint64_t dv = dv0 + uint64_t((uint32_t(s) * C::KV_TILE) >> 4);
+      asm volatile("" : "+l"(dv));
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int kk = 4 * hh + q;
+        mma_ts_elect(d_tm, p_tm + uint32_t(kk * 8), dv + v_step<C::DCH>(kk), C::IDESC_PV, (acc || q > 0) ? 1u : 0u);
+      }
+    };
     bool ok = true;
     int g = 0, it = 0;
-    if constexpr (C::SEP_P) {
+    if constexpr (C::KSPLIT) {
+      // Issuer hh runs the PV MMAs of key half hh into O_hh; issuer 0 also
+      // issues every S, S(i+1) as soon as both halves have read S(i). Each
+      // issuer releases every K/V stage once per key step, and Q once per item.
+      const int hh = warp - C::MMA_WARP;
+      int L = 0;
+      for (int p = 0; ok; ++p) {
+        if (p * int(gridDim.x) >= n_items) break;
+        const int k = item_of_pass(p, n_items);
+        if (k < 0) continue;
+        const WorkItem w = make_item<QT>(k, args);
+        const int n = w.n_steps;
+        if (hh == 0) {
+          if (!(ok = mbar_wait(&ctrl->q_full, uint32_t(it) & 1u, abort))) break;
+          tc_fence_after();
+        }
+        for (int i = 0; i < n && ok; ++i) {
+          const int gi = g + i;
+          const int s = gi % KS;
+          const uint32_t ph = uint32_t(gi / KS) & 1u;
+          if (hh == 0) {
+            if (i == 0) {
+              if (!(ok = mbar_wait(&ctrl->k_full[s], ph, abort))) break;
+              // S overwrites the columns both halves read at their last step
+              if (L > 0 && !(ok = mbar_wait(&ctrl->s_free[0], uint32_t(L - 1) & 1u, abort))) break;
+              tc_fence_after();
+              issue_s(0, s);
+              tc_commit_elect(&ctrl->s_full[0]);
+              tc_commit_elect(&ctrl->k_empty[s]);
+            }
+            if (i + 1 < n) {
+              const int s1 = (gi + 1) % KS;
+              if (!(ok = mbar_wait(&ctrl->k_full[s1], uint32_t((gi + 1) / KS) & 1u, abort))) break;
+              if (!(ok = mbar_wait(&ctrl->s_free[0], uint32_t(L) & 1u, abort))) break;
+              tc_fence_after();
+              issue_s(0, s1);
+              tc_commit_elect(&ctrl->s_full[0]);
+              tc_commit_elect(&ctrl->k_empty[s1]);
+            } else {
+              tc_commit_elect(&ctrl->q_empty);  // last S of this item issued
+            }
+          } else {
+            if (!(ok = mbar_wait(&ctrl->k_full[s], ph, abort))) break;
+            tc_commit_elect(&ctrl->k_empty[s]);  // only issuer 0's MMAs read K
+          }
+          if (!(ok = mbar_wait(&ctrl->v_full[s], ph, abort))) break;
+          if (!(ok = mbar_wait(&ctrl->p_full[hh], uint32_t(L) & 1u, abort))) break;
+          // the first PV of an item overwrites O_hh: the epilogue must have read it
+          if (i == 0 && it > 0 && !(ok = mbar_wait(&ctrl->o_free[0], uint32_t(it - 1) & 1u, abort))) break;
+          tc_fence_after();
+          issue_pv_half(hh, s, i > 0);
+          tc_commit_elect(&ctrl->pv_done[hh]);
+          tc_commit_elect(&ctrl->v_empty[s]);
+          ++L;
+        }
+        if (!ok) break;
+        tc_commit_elect(&ctrl->o_final[hh]);
+        if (hh == 1) tc_commit_elect(&ctrl->q_empty);
+        g += n;
+        ++it;
+      }
+      if (!ok) {
+        tc_commit_elect(&ctrl->drain[hh]);
+        mbar_wait_for(&ctrl->drain[hh], 0, 100000000ull);
+        if (leader) atomicOr(args.flags, kFlagTimeout);
+      }
+    } else if constexpr (C::SEP_P) {
       // One issuer warp per query tile t: S_t(i+1) as soon as the softmax has
       // read S_t(i) into registers, PV_t(i) once P_t(i) is written. The two
       // tiles' chains are independent and share the tensor core. Every issuer
@@ -555,226 +677,382 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
   }
   } else {
     setmaxnreg_inc<C::REG_SOFTMAX>();
-    // ------------------------------------------------------------- softmax
-    const int t = warp >> 2;  // query tile of this warpgroup
-    const int wq = warp & 3;  // TMEM lane quarter
-    const int r_loc = wq * 32 + lane;
-    const uint32_t lane_base = tmem + (uint32_t(wq * 32) << 16);
-    const uint32_t s_tm = lane_base + C::S_COL0 + uint32_t(128 * t);
-    const uint32_t p_tm = lane_base + C::P_COL0 + C::P_STRIDE * uint32_t(t);
-    const uint32_t o_tm = lane_base + C::O_COL0 + C::O_STRIDE * uint32_t(t);
-    const float sl2 = args.scale_log2;
-    bool ok = true;
-    int L = 0, it = 0;
-    for (int p = 0; ok; ++p) {
-      if (p * int(gridDim.x) >= n_items) break;
-      const int k = item_of_pass(p, n_items);
-      if (k < 0) continue;
-      const WorkItem w = make_item<QT>(k, args);
-      const int q0_t = pick(w.q0, t), nk_t = pick(w.nk, t), first_t = pick(w.first, t);
-      const int row = q0_t + r_loc;
-      float aq0 = 0.f, aq1 = 0.f, aq2 = 0.f, aq3 = 0.f;
-      if (MODE == kBiasReg && row < N && nk_t > 0) {
-        const float4 v = *reinterpret_cast<const float4 *>(args.phiq_reg + (size_t(w.fb_slice) * N + row) * 4);
-        aq0 = v.x, aq1 = v.y, aq2 = v.z, aq3 = v.w;
-      }
-      float m_use = -INFINITY, l_sum = 0.f;
-      for (int i = first_t; i < w.n_steps; ++i) {  // key tile n_steps - 1 - i
-        const int s = L % KS;  // the softmax-side ring runs on L
-        const uint32_t ph = uint32_t(L / KS) & 1u;
-        if (C::HAS_AUX && !(ok = mbar_wait(&ctrl->aux_full[t][s], ph, abort))) break;
-        if (!(ok = mbar_wait(&ctrl->s_full[t], uint32_t(L) & 1u, abort))) break;
-        tc_fence_after();
-
-        // Raw scores of this thread's row; with a softmax-side bias they are
-        // turned into log2-domain logits in place, otherwise the scale is
-        // folded into the exponent below.
-        uint32_t x[128];
-        tmem_ld32(s_tm + 0, x + 0);
-        tmem_ld32(s_tm + 32, x + 32);
-        tmem_ld32(s_tm + 64, x + 64);
-        tmem_ld32(s_tm + 96, x + 96);
-        tmem_ld_wait32(x + 0);
-        tmem_ld_wait32(x + 32);
-        tmem_ld_wait32(x + 64);
-        tmem_ld_wait32(x + 96);
-        if (C::SEP_P) {  // S_t is in registers: the tensor core may overwrite it
+    if constexpr (C::KSPLIT) {
+      // Key split: warpgroup h takes keys 64h .. 64h+63 of every key tile of
+      // the item, with its own running max m_h, row sum l_h and O_h; the two
+      // are merged in the epilogue (O = sum_h 2^(m_h - M) O_h / sum_h 2^(m_h - M) l_h).
+      const int h = warp >> 2;
+      const int wq = warp & 3;  // TMEM lane quarter
+      const int r_loc = wq * 32 + lane;
+      const uint32_t lane_base = tmem + (uint32_t(wq * 32) << 16);
+      const uint32_t s_tm = lane_base + C::S_COL0 + uint32_t(64 * h);
+      const uint32_t p_tm = lane_base + C::P_COL0 + uint32_t(32 * h);
+      const uint32_t o0_tm = lane_base + C::O_COL0;
+      const uint32_t o1_tm = lane_base + C::O_COL0 + C::O_STRIDE;
+      const uint32_t own_tm = h ? o1_tm : o0_tm;
+      const float sl2 = args.scale_log2;
+      float *xch = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(ctrl) + 1024);
+      auto xslot = [&](int half, int slot, int v) { return xch + (((wq * 2 + half) * 2 + slot) * 2 + v) * 32 + lane; };
+      int n_ex = 0;
+      bool ok = true;
+      int L = 0, it = 0;
+      for (int p = 0; ok; ++p) {
+        if (p * int(gridDim.x) >= n_items) break;
+        const int k = item_of_pass(p, n_items);
+        if (k < 0) continue;
+        const WorkItem w = make_item<QT>(k, args);
+        const int q0 = w.q0[0], n = w.n_steps;
+        const int row = q0 + r_loc;
+        float m_use = -INFINITY, l_sum = 0.f;
+        for (int i = 0; i < n; ++i) {  // key tile n - 1 - i
+          const int s = L % KS;
+          const uint32_t ph = uint32_t(L / KS) & 1u;
+          if (C::HAS_AUX && !(ok = mbar_wait(&ctrl->aux_full[0][s], ph, abort))) break;
+          if (!(ok = mbar_wait(&ctrl->s_full[0], uint32_t(L) & 1u, abort))) break;
+          tc_fence_after();
+          uint32_t x[64];
+          tmem_ld32(s_tm, x);
+          tmem_ld32(s_tm + 32, x + 32);
+          tmem_ld_wait32(x);
+          tmem_ld_wait32(x + 32);
           tc_fence_before();
-          mbar_arrive(&ctrl->s_free[t]);
-        }
-        float mul = sl2;  // logit = raw * mul
-        if (MODE == kBiasReg) {
-          // Key pairs: one 16-byte load gives a factor column for two keys,
-          // and the raw scores take the bias in packed pairs; the factors on
-          // the query side carry 1 / scale, so the scale stays in mul.
-          const float4 *fk = reinterpret_cast<const float4 *>(sAux + (t * KS + s) * C::AUX_TILE);
-          const uint64_t a0 = f2_pack(aq0, aq0), a1 = f2_pack(aq1, aq1);
-          const uint64_t a2 = f2_pack(aq2, aq2), a3 = f2_pack(aq3, aq3);
-#pragma unroll
-          for (int j = 0; j < 64; ++j) {
-            uint64_t xp = f2_pack(__uint_as_float(x[2 * j]), __uint_as_float(x[2 * j + 1]));
-            const float4 f = fk[j * (RP / 2)];
-            xp = f2_fma(a0, f2_pack(f.x, f.y), xp);
-            xp = f2_fma(a1, f2_pack(f.z, f.w), xp);
-            if (RP > 2) {
-              const float4 g = fk[j * (RP / 2) + 1];
-              xp = f2_fma(a2, f2_pack(g.x, g.y), xp);
-              xp = f2_fma(a3, f2_pack(g.z, g.w), xp);
-            }
-            float v0, v1;
-            f2_unpack(xp, v0, v1);
-            x[2 * j] = __float_as_uint(v0);
-            x[2 * j + 1] = __float_as_uint(v1);
-          }
-          mbar_arrive(&ctrl->aux_empty[t][s]);
-        } else if (MODE == kBiasDense) {
-          const uint8_t *tile = sAux + (t * KS + s) * C::AUX_TILE;
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
+          mbar_arrive(&ctrl->s_free[0]);  // S is in registers: the tensor core may overwrite it
+          float mul = sl2;  // logit = raw * mul
+          if (MODE == kBiasDense) {
+            const uint8_t *tile = sAux + s * C::AUX_TILE + h * 16384;
 #pragma unroll
             for (int ck = 0; ck < 8; ++ck) {
-              const uint4 u =
-                  *reinterpret_cast<const uint4 *>(tile + hh * 16384 + r_loc * 128 + ((ck ^ (r_loc & 7)) * 16));
+              const uint4 u = *reinterpret_cast<const uint4 *>(tile + r_loc * 128 + ((ck ^ (r_loc & 7)) * 16));
               const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
-                const int c = hh * 64 + ck * 8 + 2 * e;
+                const int c = ck * 8 + 2 * e;
                 x[c] = __float_as_uint(fmaf(__uint_as_float(wv[e] << 16), kLog2e, __uint_as_float(x[c]) * sl2));
                 x[c + 1] = __float_as_uint(
                     fmaf(__uint_as_float(wv[e] & 0xFFFF0000u), kLog2e, __uint_as_float(x[c + 1]) * sl2));
               }
             }
+            mbar_arrive(&ctrl->aux_empty[0][s]);
+            mul = 1.f;
           }
-          mbar_arrive(&ctrl->aux_empty[t][s]);
-          mul = 1.f;
-        }
-        // Causal diagonal tile and the ragged last key tile.
-        const int key0 = (w.n_steps - 1 - i) * 128;
-        if ((args.causal && key0 + 127 > q0_t) || key0 + 128 > N) {
-          const int lim = args.causal ? min(row + 1, N) : N;  // keys [0, lim) are visible
+          // Causal diagonal tile and the ragged last key tile.
+          const int key0 = (n - 1 - i) * 128 + 64 * h;  // first key of this half
+          if ((args.causal && key0 + 63 > q0) || key0 + 64 > N) {
+            const int lim = args.causal ? min(row + 1, N) : N;  // keys [0, lim) are visible
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (key0 + c >= lim) x[c] = __float_as_uint(-INFINITY);
-        }
-        float mx;
-        {
-          // eight independent chains of three-input max (one instruction per
-          // two elements)
-          float mp[8];
+            for (int c = 0; c < 64; ++c)
+              if (key0 + c >= lim) x[c] = __float_as_uint(-INFINITY);
+          }
+          const float m_new = fmaxf(m_use, row_max<64>(x) * mul);
+          float alpha = 1.f;
+          bool resc = false;
+          if (m_use == -INFINITY || m_new > m_use + kRescaleThreshold) {
+            alpha = (m_use == -INFINITY) ? 0.f : ex2_approx(m_use - m_new);
+            resc = (i > 0) && (m_use != -INFINITY);
+            m_use = m_new;
+          }
+          l_sum *= alpha;
+          const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;
+          const uint64_t mul2 = f2_pack(mul, mul), negm2 = f2_pack(neg_m, neg_m);
+          uint64_t ls[4] = {0, 0, 0, 0};
+          uint32_t pk[32];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) mp[e] = fmax3(__uint_as_float(x[e]), __uint_as_float(x[8 + e]), __uint_as_float(x[16 + e]));
+          for (int q4 = 0; q4 < 2; ++q4) {
 #pragma unroll
-          for (int c = 24; c < 120; c += 16)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) mp[e] = fmax3(mp[e], __uint_as_float(x[c + e]), __uint_as_float(x[c + 8 + e]));
-#pragma unroll
-          for (int e = 0; e < 8; ++e) mp[e] = fmaxf(mp[e], __uint_as_float(x[120 + e]));
-          mx = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
-        }
-        const float m_new = fmaxf(m_use, mx * mul);
-        float alpha = 1.f;
-        bool resc = false;
-        if (m_use == -INFINITY || m_new > m_use + kRescaleThreshold) {
-          alpha = (m_use == -INFINITY) ? 0.f : ex2_approx(m_use - m_new);
-          resc = (i > first_t) && (m_use != -INFINITY);
-          m_use = m_new;
-        }
-        l_sum *= alpha;
-        // P of the whole row stays in registers (each 32-column group of x
-        // dies as its 16 bf16 pairs are made) and goes to TMEM at the end, so
-        // the wait for the previous PV_t overlaps the exponentials.
-        const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;
-        const uint64_t mul2 = f2_pack(mul, mul), negm2 = f2_pack(neg_m, neg_m);
-        uint64_t ls[4] = {0, 0, 0, 0};  // packed partial row sums
-        uint32_t pk[64];
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const uint64_t a =
-                f2_fma(f2_pack(__uint_as_float(x[q4 * 32 + 2 * e]), __uint_as_float(x[q4 * 32 + 2 * e + 1])), mul2,
-                       negm2);
-            float a0, a1, p0, p1;
-            f2_unpack(a, a0, a1);
-            if (e < kEmuPairs) {
-              ex2_fma_pair(a0, a1, p0, p1);
-            } else {
-              p0 = ex2_approx(a0);
-              p1 = ex2_approx(a1);
+            for (int e = 0; e < 16; ++e) {
+              const uint64_t a =
+                  f2_fma(f2_pack(__uint_as_float(x[q4 * 32 + 2 * e]), __uint_as_float(x[q4 * 32 + 2 * e + 1])),
+                         mul2, negm2);
+              float a0, a1, p0, p1;
+              f2_unpack(a, a0, a1);
+              if (e < kEmuPairs) {
+                ex2_fma_pair(a0, a1, p0, p1);
+              } else {
+                p0 = ex2_approx(a0);
+                p1 = ex2_approx(a1);
+              }
+              ls[e & 3] = f2_add(ls[e & 3], f2_pack(p0, p1));
+              pk[q4 * 16 + e] = pack_bf16x2(p0, p1);
             }
-            ls[e & 3] = f2_add(ls[e & 3], f2_pack(p0, p1));
-            pk[q4 * 16 + e] = pack_bf16x2(p0, p1);
           }
-        }
-        {
-          float s0, s1, s2, s3, s4, s5, s6, s7;
-          f2_unpack(ls[0], s0, s1);
-          f2_unpack(ls[1], s2, s3);
-          f2_unpack(ls[2], s4, s5);
-          f2_unpack(ls[3], s6, s7);
-          l_sum += ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
-        }
-        if (C::SEP_P && L > 0) {
-          // P_t (and O_t) are still read by the previous PV_t; wait for it.
-          if (!(ok = mbar_wait(&ctrl->pv_done[t], uint32_t(L - 1) & 1u, abort))) break;
-          tc_fence_after();
-        }
-        if (__any_sync(0xffffffffu, resc)) {
-          // PV_t(i-1) has completed (pv_done, or, when P aliases S, the commit
-          // that published S_t(i) covers it).
-#pragma unroll
-          for (int c0 = 0; c0 < DP; c0 += 16) {
-            uint32_t r[16];
-            tmem_ld16(o_tm + c0, r);
-            tmem_ld_wait16(r);
-#pragma unroll
-            for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-            tmem_st16(o_tm + c0, r);
+          {
+            float s0, s1, s2, s3, s4, s5, s6, s7;
+            f2_unpack(ls[0], s0, s1);
+            f2_unpack(ls[1], s2, s3);
+            f2_unpack(ls[2], s4, s5);
+            f2_unpack(ls[3], s6, s7);
+            l_sum += ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
           }
+          if (L > 0) {  // P_h and O_h are still read by the previous PV_h
+            if (!(ok = mbar_wait(&ctrl->pv_done[h], uint32_t(L - 1) & 1u, abort))) break;
+            tc_fence_after();
+          }
+          if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll
+            for (int c0 = 0; c0 < DP; c0 += 16) {
+              uint32_t r[16];
+              tmem_ld16(own_tm + c0, r);
+              tmem_ld_wait16(r);
+#pragma unroll
+              for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+              tmem_st16(own_tm + c0, r);
+            }
+          }
+          tmem_st32(p_tm, pk);
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&ctrl->p_full[h]);
+          ++L;
         }
-        tmem_st32(p_tm, pk);
-        tmem_st32(p_tm + 32, pk + 32);
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&ctrl->p_full[t]);
-        ++L;
-      }
-      if (!ok) break;
+        if (!ok) break;
 
-      // ---------------------------------------------------------- epilogue
-      if (!(ok = mbar_wait(&ctrl->o_final[t], uint32_t(it) & 1u, abort))) break;
-      tc_fence_after();
-      if (nk_t > 0) {
-        const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
+        // ---------------------------------------------------- epilogue (merge)
+        if (!(ok = mbar_wait(&ctrl->o_final[0], uint32_t(it) & 1u, abort))) break;
+        if (!(ok = mbar_wait(&ctrl->o_final[1], uint32_t(it) & 1u, abort))) break;
+        tc_fence_after();
+        const int slot = n_ex & 1;
+        *xslot(h, slot, 0) = m_use;
+        *xslot(h, slot, 1) = l_sum;
+        mbar_arrive(&ctrl->pair[wq]);
+        if (!(ok = mbar_wait(&ctrl->pair[wq], uint32_t(n_ex) & 1u, abort))) break;
+        const float m_o = *xslot(h ^ 1, slot, 0), l_o = *xslot(h ^ 1, slot, 1);
+        ++n_ex;
+        const float m0 = h ? m_o : m_use, l0 = h ? l_o : l_sum;
+        const float m1 = h ? m_use : m_o, l1 = h ? l_sum : l_o;
+        const float M = fmaxf(m0, m1);
+        const float w0 = m0 == -INFINITY ? 0.f : ex2_approx(m0 - M);
+        const float w1 = m1 == -INFINITY ? 0.f : ex2_approx(m1 - M);
+        const float l_tot = w0 * l0 + w1 * l1;
+        const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
+        const float c0s = w0 * inv_l, c1s = w1 * inv_l;
         __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(args.O) + (size_t(w.bh) * N + row) * args.d;
 #pragma unroll
-        for (int c0 = 0; c0 < DP; c0 += 16) {
-          uint32_t r[16];
-          tmem_ld16(o_tm + c0, r);
-          tmem_ld_wait16(r);
+        for (int cc = 0; cc < 64; cc += 16) {  // this half writes O columns 64h .. 64h+63
+          const int col0 = 64 * h + cc;
+          uint32_t r0[16], r1[16];
+          tmem_ld16(o0_tm + col0, r0);
+          tmem_ld16(o1_tm + col0, r1);
+          tmem_ld_wait16(r0);
+          tmem_ld_wait16(r1);
           if (row < N) {
 #pragma unroll
             for (int v8 = 0; v8 < 2; ++v8) {
-              const int col = c0 + v8 * 8;
+              const int col = col0 + v8 * 8;
               if (col < args.d) {
+                float o[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                  o[e] = fmaf(__uint_as_float(r0[v8 * 8 + e]), c0s, __uint_as_float(r1[v8 * 8 + e]) * c1s);
                 uint4 u;
-                u.x = pack_bf16x2(__uint_as_float(r[v8 * 8 + 0]) * inv_l, __uint_as_float(r[v8 * 8 + 1]) * inv_l);
-                u.y = pack_bf16x2(__uint_as_float(r[v8 * 8 + 2]) * inv_l, __uint_as_float(r[v8 * 8 + 3]) * inv_l);
-                u.z = pack_bf16x2(__uint_as_float(r[v8 * 8 + 4]) * inv_l, __uint_as_float(r[v8 * 8 + 5]) * inv_l);
-                u.w = pack_bf16x2(__uint_as_float(r[v8 * 8 + 6]) * inv_l, __uint_as_float(r[v8 * 8 + 7]) * inv_l);
+                u.x = pack_bf16x2(o[0], o[1]);
+                u.y = pack_bf16x2(o[2], o[3]);
+                u.z = pack_bf16x2(o[4], o[5]);
+                u.w = pack_bf16x2(o[6], o[7]);
                 *reinterpret_cast<uint4 *>(orow + col) = u;
               }
             }
           }
         }
-        if (row < N)
-          args.LSE[size_t(w.bh) * N + row] = l_sum > 0.f ? (m_use + __log2f(l_sum)) * kLn2 : -INFINITY;
+        if (h == 0 && row < N)
+          args.LSE[size_t(w.bh) * N + row] = l_tot > 0.f ? (M + __log2f(l_tot)) * kLn2 : -INFINITY;
+        tc_fence_before();
+        mbar_arrive(&ctrl->o_free[0]);  // both O accumulators have been read
+        ++it;
       }
-      tc_fence_before();
-      mbar_arrive(&ctrl->o_free[t]);  // O_t has been read
-      ++it;
+      if (!ok) atomicOr(args.flags, kFlagTimeout);
+    } else {
+      // ------------------------------------------------------------- softmax
+      const int t = warp >> 2;  // query tile of this warpgroup
+      const int wq = warp & 3;  // TMEM lane quarter
+      const int r_loc = wq * 32 + lane;
+      const uint32_t lane_base = tmem + (uint32_t(wq * 32) << 16);
+      const uint32_t s_tm = lane_base + C::S_COL0 + uint32_t(128 * t);
+      const uint32_t p_tm = lane_base + C::P_COL0 + C::P_STRIDE * uint32_t(t);
+      const uint32_t o_tm = lane_base + C::O_COL0 + C::O_STRIDE * uint32_t(t);
+      const float sl2 = args.scale_log2;
+      bool ok = true;
+      int L = 0, it = 0;
+      for (int p = 0; ok; ++p) {
+        if (p * int(gridDim.x) >= n_items) break;
+        const int k = item_of_pass(p, n_items);
+        if (k < 0) continue;
+        const WorkItem w = make_item<QT>(k, args);
+        const int q0_t = pick(w.q0, t), nk_t = pick(w.nk, t), first_t = pick(w.first, t);
+        const int row = q0_t + r_loc;
+        float m_use = -INFINITY, l_sum = 0.f;
+        for (int i = first_t; i < w.n_steps; ++i) {  // key tile n_steps - 1 - i
+          const int s = L % KS;  // the softmax-side ring runs on L
+          const uint32_t ph = uint32_t(L / KS) & 1u;
+          if (C::HAS_AUX && !(ok = mbar_wait(&ctrl->aux_full[t][s], ph, abort))) break;
+          if (!(ok = mbar_wait(&ctrl->s_full[t], uint32_t(L) & 1u, abort))) break;
+          tc_fence_after();
+
+          // Raw scores of this thread's row; with a softmax-side bias they are
+          // turned into log2-domain logits in place, otherwise the scale is
+          // folded into the exponent below.
+          uint32_t x[128];
+          tmem_ld32(s_tm + 0, x + 0);
+          tmem_ld32(s_tm + 32, x + 32);
+          tmem_ld32(s_tm + 64, x + 64);
+          tmem_ld32(s_tm + 96, x + 96);
+          tmem_ld_wait32(x + 0);
+          tmem_ld_wait32(x + 32);
+          tmem_ld_wait32(x + 64);
+          tmem_ld_wait32(x + 96);
+          if (C::SEP_P) {  // S_t is in registers: the tensor core may overwrite it
+            tc_fence_before();
+            mbar_arrive(&ctrl->s_free[t]);
+          }
+          float mul = sl2;  // logit = raw * mul
+          if (MODE == kBiasDense) {
+            const uint8_t *tile = sAux + (t * KS + s) * C::AUX_TILE;
+  #pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+  #pragma unroll
+              for (int ck = 0; ck < 8; ++ck) {
+                const uint4 u =
+                    *reinterpret_cast<const uint4 *>(tile + hh * 16384 + r_loc * 128 + ((ck ^ (r_loc & 7)) * 16));
+                const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+  #pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int c = hh * 64 + ck * 8 + 2 * e;
+                  x[c] = __float_as_uint(fmaf(__uint_as_float(wv[e] << 16), kLog2e, __uint_as_float(x[c]) * sl2));
+                  x[c + 1] = __float_as_uint(
+                      fmaf(__uint_as_float(wv[e] & 0xFFFF0000u), kLog2e, __uint_as_float(x[c + 1]) * sl2));
+                }
+              }
+            }
+            mbar_arrive(&ctrl->aux_empty[t][s]);
+            mul = 1.f;
+          }
+          // Causal diagonal tile and the ragged last key tile.
+          const int key0 = (w.n_steps - 1 - i) * 128;
+          if ((args.causal && key0 + 127 > q0_t) || key0 + 128 > N) {
+            const int lim = args.causal ? min(row + 1, N) : N;  // keys [0, lim) are visible
+  #pragma unroll
+            for (int c = 0; c < 128; ++c)
+              if (key0 + c >= lim) x[c] = __float_as_uint(-INFINITY);
+          }
+          float mx;
+          {
+            // eight independent chains of three-input max (one instruction per
+            // two elements)
+            float mp[8];
+  #pragma unroll
+            for (int e = 0; e < 8; ++e) mp[e] = fmax3(__uint_as_float(x[e]), __uint_as_float(x[8 + e]), __uint_as_float(x[16 + e]));
+  #pragma unroll
+            for (int c = 24; c < 120; c += 16)
+  #pragma unroll
+              for (int e = 0; e < 8; ++e) mp[e] = fmax3(mp[e], __uint_as_float(x[c + e]), __uint_as_float(x[c + 8 + e]));
+  #pragma unroll
+            for (int e = 0; e < 8; ++e) mp[e] = fmaxf(mp[e], __uint_as_float(x[120 + e]));
+            mx = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
+          }
+          const float m_new = fmaxf(m_use, mx * mul);
+          float alpha = 1.f;
+          bool resc = false;
+          if (m_use == -INFINITY || m_new > m_use + kRescaleThreshold) {
+            alpha = (m_use == -INFINITY) ? 0.f : ex2_approx(m_use - m_new);
+            resc = (i > first_t) && (m_use != -INFINITY);
+            m_use = m_new;
+          }
+          l_sum *= alpha;
+          // P of the whole row stays in registers (each 32-column group of x
+          // dies as its 16 bf16 pairs are made) and goes to TMEM at the end, so
+          // the wait for the previous PV_t overlaps the exponentials.
+          const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;
+          const uint64_t mul2 = f2_pack(mul, mul), negm2 = f2_pack(neg_m, neg_m);
+          uint64_t ls[4] = {0, 0, 0, 0};  // packed partial row sums
+          uint32_t pk[64];
+  #pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+  #pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const uint64_t a =
+                  f2_fma(f2_pack(__uint_as_float(x[q4 * 32 + 2 * e]), __uint_as_float(x[q4 * 32 + 2 * e + 1])), mul2,
+                         negm2);
+              float a0, a1, p0, p1;
+              f2_unpack(a, a0, a1);
+              if (e < kEmuPairs) {
+                ex2_fma_pair(a0, a1, p0, p1);
+              } else {
+                p0 = ex2_approx(a0);
+                p1 = ex2_approx(a1);
+              }
+              ls[e & 3] = f2_add(ls[e & 3], f2_pack(p0, p1));
+              pk[q4 * 16 + e] = pack_bf16x2(p0, p1);
+            }
+          }
+          {
+            float s0, s1, s2, s3, s4, s5, s6, s7;
+            f2_unpack(ls[0], s0, s1);
+            f2_unpack(ls[1], s2, s3);
+            f2_unpack(ls[2], s4, s5);
+            f2_unpack(ls[3], s6, s7);
+            l_sum += ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
+          }
+          if (C::SEP_P && L > 0) {
+            // P_t (and O_t) are still read by the previous PV_t; wait for it.
+            if (!(ok = mbar_wait(&ctrl->pv_done[t], uint32_t(L - 1) & 1u, abort))) break;
+            tc_fence_after();
+          }
+          if (__any_sync(0xffffffffu, resc)) {
+            // PV_t(i-1) has completed (pv_done, or, when P aliases S, the commit
+            // that published S_t(i) covers it).
+  #pragma unroll
+            for (int c0 = 0; c0 < DP; c0 += 16) {
+              uint32_t r[16];
+              tmem_ld16(o_tm + c0, r);
+              tmem_ld_wait16(r);
+  #pragma unroll
+              for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+              tmem_st16(o_tm + c0, r);
+            }
+          }
+          tmem_st32(p_tm, pk);
+          tmem_st32(p_tm + 32, pk + 32);
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&ctrl->p_full[t]);
+          ++L;
+        }
+        if (!ok) break;
+
+        // ---------------------------------------------------------- epilogue
+        if (!(ok = mbar_wait(&ctrl->o_final[t], uint32_t(it) & 1u, abort))) break;
+        tc_fence_after();
+        if (nk_t > 0) {
+          const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
+          __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(args.O) + (size_t(w.bh) * N + row) * args.d;
+  #pragma unroll
+          for (int c0 = 0; c0 < DP; c0 += 16) {
+            uint32_t r[16];
+            tmem_ld16(o_tm + c0, r);
+            tmem_ld_wait16(r);
+            if (row < N) {
+  #pragma unroll
+              for (int v8 = 0; v8 < 2; ++v8) {
+                const int col = c0 + v8 * 8;
+                if (col < args.d) {
+                  uint4 u;
+                  u.x = pack_bf16x2(__uint_as_float(r[v8 * 8 + 0]) * inv_l, __uint_as_float(r[v8 * 8 + 1]) * inv_l);
+                  u.y = pack_bf16x2(__uint_as_float(r[v8 * 8 + 2]) * inv_l, __uint_as_float(r[v8 * 8 + 3]) * inv_l);
+                  u.z = pack_bf16x2(__uint_as_float(r[v8 * 8 + 4]) * inv_l, __uint_as_float(r[v8 * 8 + 5]) * inv_l);
+                  u.w = pack_bf16x2(__uint_as_float(r[v8 * 8 + 6]) * inv_l, __uint_as_float(r[v8 * 8 + 7]) * inv_l);
+                  *reinterpret_cast<uint4 *>(orow + col) = u;
+                }
+              }
+            }
+          }
+          if (row < N)
+            args.LSE[size_t(w.bh) * N + row] = l_sum > 0.f ? (m_use + __log2f(l_sum)) * kLn2 : -INFINITY;
+        }
+        tc_fence_before();
+        mbar_arrive(&ctrl->o_free[t]);  // O_t has been read
+        ++it;
+      }
+      if (!ok) atomicOr(args.flags, kFlagTimeout);
     }
-    if (!ok) atomicOr(args.flags, kFlagTimeout);
   }
 
   tc_fence_before();
@@ -853,9 +1131,9 @@ static constexpr size_t smem_of() {
 
 #define FB_DISPATCH_MODE(DPv)                                                    \
   if (p.mode == kBiasNone) { FB_DISPATCH_QT(DPv, 0, kBiasNone) }                 \
-  if (p.mode == kBiasReg) {                                                      \
-    if (p.RP == 2) { FB_DISPATCH_QT(DPv, 2, kBiasReg) }                          \
-    if (p.RP == 4) { FB_DISPATCH_QT(DPv, 4, kBiasReg) }                          \
+  if (p.mode == kBiasTf32) {                                                     \
+    if (p.RP == 8) { FB_DISPATCH_QT(DPv, 8, kBiasTf32) }                         \
+    if (p.RP == 16) { FB_DISPATCH_QT(DPv, 16, kBiasTf32) }                       \
   }                                                                              \
   if (p.mode == kBiasDense) { FB_DISPATCH_QT(DPv, 0, kBiasDense) }               \
   if (p.mode == kBiasMma) {                                                      \

@@ -78,35 +78,47 @@ __global__ void prep_mma_kernel(int N, int R, int RP, int fac_H, const float *__
 
 // Preparation for the CUDA-core factor path (R <= 4, fp32):
 //   out_q[f, n, 0..3] = phi_q * log2(e) (zero padded), out_k[f, n, 0..3] = phi_k.
-// Rank <= 4 (factors applied on the CUDA cores, fp32): phi_q / scale per
-// row as [slice][N] float4, and phi_k by key pairs, so that one 16-byte load
-// gives a factor column for two adjacent keys: pair j (keys 2j, 2j+1) holds
-// (f0[2j], f0[2j+1], f1[2j], f1[2j+1]) and, for RP = 4, a second float4 with
-// f2, f3. A missing key 2j+1 (odd N) has zero factors.
-__global__ void prep_reg_kernel(int N, int R, int RP, int fac_H, const float *__restrict__ pq,
-                                const float *__restrict__ pk, long long bs, long long hs, float inv_scale,
-                                float4 *__restrict__ oq, float4 *__restrict__ ok, long long total) {
-  const long long NP = (N + 1) / 2;
+// Rank <= 4: the factors enter the tensor cores as tf32 (kind::tf32 MMA),
+// split so that the product keeps fp32 accuracy: x = hi + lo with hi = x with
+// its 13 low mantissa bits cleared (what a tf32 operand holds) and lo = x - hi
+// (exact). Row layouts, KT = 8 or 16 columns, zero-padded:
+//   q' = [qh_0..qh_{R-1}, qh_0..qh_{R-1}, ql_0..ql_{R-1}]   (phi_q / scale)
+//   k' = [kh_0..kh_{R-1}, kl_0..kl_{R-1}, kh_0..kh_{R-1}]
+// so q'.k' = qh.kh + qh.kl + ql.kh; the dropped ql.kl and the tf32 rounding
+// of the lo parts are about 2^-22 of each product.
+__device__ __forceinline__ float tf32_hi(float x) { return __uint_as_float(__float_as_uint(x) & 0xFFFFE000u); }
+
+__global__ void prep_tf32_kernel(int N, int R, int KT, int fac_H, const float *__restrict__ pq,
+                                 const float *__restrict__ pk, long long bs, long long hs, float inv_scale,
+                                 float *__restrict__ oq, float *__restrict__ ok, long long total) {
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
        idx += (long long)gridDim.x * blockDim.x) {
-    const long long j = idx % NP;
-    const long long f = idx / NP;
+    const long long n = idx % N;
+    const long long f = idx / N;
     const long long fb = f / fac_H, fh = f - (f / fac_H) * fac_H;
-    float k[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    for (int e = 0; e < 2; ++e) {
-      const long long n = 2 * j + e;
-      if (n >= N) break;
-      const long long src = fb * bs + fh * hs + n * R;
-      float q[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int r = 0; r < R; ++r) {
-        q[r] = pq[src + r] * inv_scale;
-        k[e][r] = pk[src + r];
-      }
-      oq[f * N + n] = make_float4(q[0], q[1], q[2], q[3]);
+    const long long src = fb * bs + fh * hs + n * R;
+    float q[16], k[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) q[c] = k[c] = 0.f;
+    for (int r = 0; r < R; ++r) {
+      const float x = pq[src + r] * inv_scale, y = pk[src + r];
+      const float xh = tf32_hi(x), yh = tf32_hi(y);
+      q[r] = xh;
+      q[R + r] = xh;
+      q[2 * R + r] = x - xh;
+      k[r] = yh;
+      k[R + r] = y - yh;
+      k[2 * R + r] = yh;
     }
-    float4 *dst = ok + (f * NP + j) * (RP / 2);
-    dst[0] = make_float4(k[0][0], k[1][0], k[0][1], k[1][1]);
-    if (RP > 2) dst[1] = make_float4(k[0][2], k[1][2], k[0][3], k[1][3]);
+    float4 *dq = reinterpret_cast<float4 *>(oq + idx * KT);
+    float4 *dk = reinterpret_cast<float4 *>(ok + idx * KT);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      if (4 * v < KT) {
+        dq[v] = make_float4(q[4 * v], q[4 * v + 1], q[4 * v + 2], q[4 * v + 3]);
+        dk[v] = make_float4(k[4 * v], k[4 * v + 1], k[4 * v + 2], k[4 * v + 3]);
+      }
+    }
   }
 }
 
@@ -156,10 +168,10 @@ cudaError_t launch_prep_factors(int mode, int B, int H, int N, int R, int RP, co
                                                          static_cast<__half *>(out_q), static_cast<__half *>(out_k),
                                                          flags, total);
   } else {
-    const long long total = (long long)fac_B * fac_H * ((N + 1) / 2);
-    prep_reg_kernel<<<grid_for(total, 256), 256, 0, s>>>(N, R, RP, fac_H, phi_q, phi_k, bs, hs, 1.0f / scale,
-                                                         static_cast<float4 *>(out_q), static_cast<float4 *>(out_k),
-                                                         total);
+    const long long total = (long long)fac_B * fac_H * N;
+    prep_tf32_kernel<<<grid_for(total, 256), 256, 0, s>>>(N, R, RP, fac_H, phi_q, phi_k, bs, hs, 1.0f / scale,
+                                                          static_cast<float *>(out_q), static_cast<float *>(out_k),
+                                                          total);
   }
   return cudaGetLastError();
 }

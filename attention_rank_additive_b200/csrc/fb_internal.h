@@ -18,7 +18,7 @@ constexpr int kFlagRange = 2;
 enum BiasMode : int {
   kBiasNone = 0,   // plain attention (R == 0)
   kBiasMma = 1,    // fp16 factors, second tcgen05 MMA into the score accumulator
-  kBiasReg = 2,    // R <= 4 fp32 factors, added on the CUDA cores
+  kBiasTf32 = 2,   // R <= 4: fp32 factors split hi/lo, second MMA (kind::tf32) into the score accumulator
   kBiasDense = 3,  // materialised bf16 bias tile streamed by TMA (comparison path)
 };
 
@@ -31,7 +31,6 @@ struct FwdArgs {
   int causal;
   void *O;
   float *LSE;
-  const float *phiq_reg;  // kBiasReg: [FB, N, 4] fp32, phi_q * log2(e)
   int fac_B, fac_H;       // factor slices: B or 1, H or 1 (1 = broadcast)
   int bias_B, bias_H;     // dense bias slices, same convention
   int *flags;             // device flag word
@@ -40,14 +39,14 @@ struct FwdArgs {
 // Launch description chosen by the host for one call.
 struct FwdPlan {
   int DP;    // padded head dim: 16, 32, 64, 128
-  int RP;    // kBiasMma: padded factor rank (16..128); kBiasReg: 2 or 4 live factor columns; else 0
+  int RP;    // kBiasMma: padded factor rank (16..128); kBiasTf32: split-factor columns 8 or 16; else 0
   int mode;  // BiasMode
   int QT;    // 128-row query tiles per CTA: 1 or 2
 };
 
 struct FwdMaps {
   CUtensorMap q, k, v;  // bf16 [BH, N, d] with box (min(DP,64), 128, 1)
-  CUtensorMap fq, fk;   // factors: fp16 [FB, N, RP] (mma) or fp32 [FB, N, 4] (reg, fk only)
+  CUtensorMap fq, fk;   // factors: fp16 [FB, N, RP] (mma) or fp32 [FB, N, RP] (tf32)
   CUtensorMap bias;     // dense bias bf16 [B', H', N, N] with box (64, 128, 1, 1)
 };
 
@@ -65,7 +64,7 @@ cudaError_t f32_launch(int B, int H, int N, int d, const float *Q, const float *
 // Factor generators and preparation.
 cudaError_t launch_sandwich(int N, int C, float *phi_q, float *phi_k, cudaStream_t s);
 cudaError_t launch_alibi(int H, int N, float *phi_q, float *phi_k, cudaStream_t s);
-// kBiasMma: fp16 [FB, N, RP], phi_q / scale. kBiasReg: fp32 [FB, N, 4], phi_q * log2 e.
+// kBiasMma: fp16 [FB, N, RP], phi_q / scale. kBiasTf32: fp32 [FB, N, RP] hi/lo split, phi_q / scale.
 cudaError_t launch_prep_factors(int mode, int B, int H, int N, int R, int RP, const float *phi_q, const float *phi_k,
                                 int64_t bs, int64_t hs, int fac_B, int fac_H, float scale, void *out_q, void *out_k,
                                 int *flags, cudaStream_t s);

@@ -49,9 +49,9 @@ def test_workspace_bytes():
     assert fb.fb_attn_workspace_bytes(8, 12, 2048, 64, 0, 0) == 2 * 2048 * 64 * 2
     # rank 8 pads to 16 columns; per-head factors
     assert fb.fb_attn_workspace_bytes(4, 8, 4096, 8, 0, 4096 * 8) == 2 * 8 * 4096 * 16 * 2
-    # rank <= 4 keeps fp32 in 16-byte rows
-    assert fb.fb_attn_workspace_bytes(4, 16, 8192, 2, 0, 8192 * 2) == 2 * 16 * 8192 * 16
-    assert fb.fb_attn_workspace_bytes(1, 1, 17, 3, 0, 0) == 2 * 512  # rounded to 256 B
+    # rank <= 4: fp32 hi/lo split factors, 3R columns padded to 8 (R <= 2) or 16
+    assert fb.fb_attn_workspace_bytes(4, 16, 8192, 2, 0, 8192 * 2) == 2 * 16 * 8192 * 8 * 4
+    assert fb.fb_attn_workspace_bytes(1, 1, 17, 3, 0, 0) == 2 * 1280  # 17 rows x 64 B, rounded to 256 B
     assert fb.fb_attn_workspace_bytes(1, 1, 16, 129, 0, 0) == 0  # out of range -> 0
 
 
