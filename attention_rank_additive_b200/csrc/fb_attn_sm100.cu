@@ -9,10 +9,11 @@
 // tile sit in two shared-memory tiles and the two MMAs (bf16 QK^T, then fp16
 // phi_q' phi_k^T with phi_q' = phi_q / scale) accumulate into one fp32 TMEM
 // accumulator, so the N x N bias is never read or written (Figure 2). For
-// rank <= 4 (the ALiBi factors, Example 3.4) the factor tile is created next
-// to the scores on the CUDA cores in fp32 instead, as the rebuttal describes
-// for ALiBi (reply to Reviewer BRmd, Q2 (2): Block x 2 factor tiles made "in
-// JIT"). The dense mode streams a materialised bias tile per tile pair: the
+// rank <= 4 (the ALiBi factors, Example 3.4; rebuttal, reply to Reviewer
+// BRmd, Q2 (2)) fp16 cannot hold the factors, and they enter as a tf32 MMA
+// of hi/lo split fp32 values instead (q' = [qh, qh, ql], k' = [kh, kl, kh]),
+// which keeps fp32-level accuracy at one extra K = 8 or 16 MMA per tile.
+// The dense mode streams a materialised bias tile per tile pair: the
 // "FlashAttention w/ Bias" comparison path of Figure 1(c).
 //
 // Work items: one (batch, head, group of QT query tiles of 128 rows) each.

@@ -97,7 +97,8 @@ size_t fb_attn_workspace_bytes(int B, int H, int N, int R,
  *
  * bf16 path numerics: QK^T in bf16 x bf16 -> fp32; the factors enter the same
  * fp32 accumulator as a second MMA in fp16 (phi_q pre-divided by scale) when
- * R > 4, or are added in fp32 on the CUDA cores when R <= 4; softmax in fp32;
+ * R > 4, or as a tf32 MMA of hi/lo split fp32 factors when R <= 4 (fp32-level
+ * accuracy: q'.k' = qh.kh + qh.kl + ql.kh); softmax in fp32;
  * P rounded to bf16 for the PV MMA; O rounded to bf16. A factor that does not
  * fit fp16 is saturated and flags FB_ERR_RANGE for fb_check_device_error().
  */
