@@ -202,12 +202,14 @@ def profiled_traffic(cfg_idx: int):
 
 
 def measured_peaks():
+    """(bf16 burst TF/s, bf16 sustained TF/s, HBM GB/s, 'measured' | 'fallback')."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         with open(path) as f:
             p = json.load(f)
-        return float(p["bf16_tflops"]), float(p["hbm_gbs"]), "measured"
-    return 1590.0, 6650.0, "fallback"
+        burst = float(p["bf16_tflops"])
+        return burst, float(p.get("bf16_tflops_sustained", burst)), float(p["hbm_gbs"]), "measured"
+    return 1590.0, 1400.0, 6650.0, "fallback"
 
 
 # ------------------------------------------------------------ GPU workload
@@ -444,7 +446,13 @@ def run_ours(args, rank: int, world: int, local: int):
                  "fused_speedup": round(d_ms / kern_ms, 3),
                  "layout": "[B,H,N,N] bf16 materialised, L2 flushed between steps"}
 
-    peak_tf, peak_hbm, peak_kind = measured_peaks()
+    clk_sum = clk.summary()
+    burst_tf, sustained_tf, peak_hbm, peak_src = measured_peaks()
+    # the burst peak for a kernel timed alone; the sustained one when the run
+    # itself was held at the power cap (the clock record says so)
+    capped = bool(clk_sum) and "sw_power_cap" in clk_sum.get("reasons", [])
+    peak_tf = sustained_tf if capped else burst_tf
+    peak_kind = f"{peak_src} bf16 {'sustained (run power-capped)' if capped else 'burst'}"
     achieved = c["flops"] / (kern_ms * 1e-3) / 1e12
     traffic = profiled_traffic(args.config)
     out = {
@@ -454,7 +462,7 @@ def run_ours(args, rank: int, world: int, local: int):
         "config": config_json(c, "flushed: 256 MiB memset between timed steps (untimed)"),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": round(achieved / peak_tf, 4), "traffic": traffic,
-                     "kernel": "attn_fwd_sm100", "peak_kind": f"{peak_kind} bf16 burst",
+                     "kernel": "attn_fwd_sm100", "peak_kind": peak_kind,
                      "kernel_ms": round(kern_ms, 5)},
         "e2e": {"value": round(c["flops"] * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -463,7 +471,6 @@ def run_ours(args, rank: int, world: int, local: int):
     }
     if hasattr(w, "svd_err"):
         out["svd_rank_error_energy_per_head"] = w.svd_err
-    clk_sum = clk.summary()
     if world > 1:
         # every rank sampled its own GPU; rank 0 reports its own
         pass
