@@ -5,11 +5,12 @@ leg of the benchmark are the only callers. The product path never imports this
 package, and this package imports nothing from the product.
 
 The arithmetic lives in ``fb_oracle.c`` (the definition of biased attention,
-the Sandwich and ALiBi biases and their exact factors). This module only
-marshals numpy arrays for it, plus the one step that is a library primitive:
-the truncated SVD of a static bias (FlashBias rebuttal, reply to Reviewer
-xU4x, Q6: SVD decomposition with a per-head rank), done with
-``numpy.linalg.svd``.
+the Sandwich and ALiBi biases and their exact factors). This module marshals
+numpy arrays for it, and adds two things in plain numpy fp64: the truncated
+SVD of a static bias (FlashBias rebuttal, reply to Reviewer xU4x, Q6: SVD
+decomposition with a per-head rank), done with ``numpy.linalg.svd``, and
+attention with a multiplicative bias (rebuttal, reply to Reviewer BRmd, Q1
+(2), its Eq. (1): the scaled scores are multiplied elementwise by b).
 """
 from __future__ import annotations
 
@@ -237,3 +238,29 @@ def truncated_svd_factors(bias, R: int):
 def lowrank_dense(phi_q, phi_k) -> np.ndarray:
     """phi_q phi_k^T in fp64 (the dense bias a set of factors stands for)."""
     return _f64(phi_q) @ _f64(phi_k).T
+
+
+def attention_mul_head(q, k, v, phi_q, phi_k, scale: float, causal: bool, rows=None):
+    """One head with a multiplicative bias b = phi_q phi_k^T (rebuttal, reply to
+    Reviewer BRmd, Q1 (2), Eq. (1)): s_ij = scale * (q_i . k_j) * b_ij, then the
+    softmax over the visible j (j <= i when causal) and O = P v; LSE = ln sum_j
+    exp(s_ij). q, k, v [N, d]; phi_q, phi_k [N, R]. The plain definition in
+    fp64, the whole score row at once. Returns (o [len(rows), d], lse)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    N = q.shape[0]
+    rows = np.arange(N, dtype=np.int64) if rows is None else np.asarray(rows, dtype=np.int64)
+    b = _f64(phi_q)[rows] @ _f64(phi_k).T                    # [rows, N]
+    s = float(scale) * (q[rows] @ k.T) * b
+    if causal:
+        s = np.where(np.arange(N)[None, :] <= rows[:, None], s, -np.inf)
+    m = np.max(s, axis=1, keepdims=True)
+    e = np.exp(s - m)
+    l = np.sum(e, axis=1, keepdims=True)
+    return (e @ v) / l, (m + np.log(l))[:, 0]
+
+
+def cos_factors(N: int) -> np.ndarray:
+    """The rebuttal's multiplicative example b_ij = cos(i - j): phi_q = phi_k =
+    [cos i, sin i] (reply to Reviewer BRmd, Q1 (2), Example), [N, 2] fp64."""
+    i = np.arange(N, dtype=np.float64)
+    return np.stack([np.cos(i), np.sin(i)], axis=1)

@@ -280,3 +280,60 @@ def test_offset_table_kinds():
     om, ph = si.rbf_params(1, 4)
     t2 = si.rbf_offset_table(om, ph, g)
     np.testing.assert_array_equal(HeadBias.grid(t2[0], g).dense_matrix(g * g), si.rbf_dense(t2, g)[0])
+
+
+# --- multiplicative bias (rebuttal, reply to Reviewer BRmd, Q1 (2)) ---------
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_multiplicative_unit_bias_is_plain_attention(causal):
+    """b = 1 (phi_q = phi_k = [1]): the multiplicative form is plain attention,
+    checked against torch SDPA; an additive reading would shift the LSE by 1."""
+    N, d = 40, 8
+    q, k, v = (_rand((N, d), s) for s in (31, 32, 33))
+    ones = np.ones((N, 1))
+    o, lse = oracle.attention_mul_head(q, k, v, ones, ones, 0.35, causal)
+    o_ref, lse_ref = _sdpa(q, k, v, np.zeros((N, N)), 0.35, causal)
+    np.testing.assert_allclose(o, o_ref, atol=1e-12)
+    np.testing.assert_allclose(lse, lse_ref, atol=1e-12)
+
+
+def _mp_mul_row(q, k, v, pq, pk, scale, i, causal):
+    jmax = i + 1 if causal else q.shape[0]
+    s = [mpmath.mpf(scale) * mpmath.fsum(mpmath.mpf(q[i, c]) * mpmath.mpf(k[j, c]) for c in range(q.shape[1]))
+         * mpmath.fsum(mpmath.mpf(pq[i, r]) * mpmath.mpf(pk[j, r]) for r in range(pq.shape[1])) for j in range(jmax)]
+    m = max(s)
+    e = [mpmath.exp(x - m) for x in s]
+    z = mpmath.fsum(e)
+    o = [mpmath.fsum(e[j] * mpmath.mpf(v[j, c]) for j in range(jmax)) / z for c in range(v.shape[1])]
+    return o, m + mpmath.log(z)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_multiplicative_fifty_digit_bruteforce(causal):
+    """Loops over i, j, c, r at 50 digits, with phi_q != phi_k so that b_ij and
+    b_ji differ (a transposed bias fails)."""
+    mpmath.mp.dps = 50
+    N, d, R = 10, 4, 3
+    q, k, v = (_rand((N, d), s) for s in (41, 42, 43))
+    pq, pk = _rand((N, R), 44), _rand((N, R), 45)
+    o, lse = oracle.attention_mul_head(q, k, v, pq, pk, 0.6, causal)
+    for i in range(N):
+        o_mp, l_mp = _mp_mul_row(q, k, v, pq, pk, 0.6, i, causal)
+        for c in range(d):
+            assert abs(o[i, c] - float(o_mp[c])) < 1e-13
+        assert abs(lse[i] - float(l_mp)) < 1e-13 * max(1.0, abs(float(l_mp)))
+
+
+def test_multiplicative_cos_example_closed_form():
+    """The pages' example b_ij = cos(i - j) from its rank-2 factors, against the
+    scores built from np.cos(i - j) directly and a library softmax."""
+    N, d = 50, 8
+    q, k, v = (_rand((N, d), s) for s in (51, 52, 53))
+    f = oracle.cos_factors(N)
+    o, lse = oracle.attention_mul_head(q, k, v, f, f, 0.5, True)
+    n = np.arange(N, dtype=np.float64)
+    s = 0.5 * (q @ k.T) * np.cos(n[:, None] - n[None, :])
+    s = np.where(n[None, :] <= n[:, None], s, -np.inf)
+    st = torch.from_numpy(s)
+    np.testing.assert_allclose(lse, torch.logsumexp(st, dim=-1).numpy(), atol=1e-12)
+    np.testing.assert_allclose(o, (torch.softmax(st, dim=-1) @ torch.from_numpy(v)).numpy(), atol=1e-12)
