@@ -21,7 +21,8 @@ __all__ = [
     "FB_ERR_TIMEOUT", "FB_F32", "FB_BF16", "FlashBiasError", "lib", "lib_path", "EXPORTED",
     "fb_status_str", "fb_version", "fb_attn_workspace_bytes", "fb_attn_fwd", "fb_attn_dense_bias_fwd",
     "fb_factors_sandwich", "fb_factors_alibi", "fb_svd_factors_host", "fb_check_device_error",
-    "fb_selftest_wait_timeout", "fb_attn_fwd_noalloc", "fb_attn_prepare_factors", "fb_attn_fwd_prepared", "attn",
+    "fb_selftest_wait_timeout", "fb_attn_fwd_noalloc", "fb_attn_prepare_factors", "fb_attn_fwd_prepared",
+    "fb_attn_mul_bias_workspace_bytes", "fb_attn_mul_bias_fwd", "attn_mul_bias", "attn",
     "PreparedBias", "attn_dense_bias", "factors_sandwich", "factors_alibi", "svd_factors",
     "attn_flops",
 ]
@@ -37,6 +38,7 @@ EXPORTED = (
     "fb_status_str", "fb_version", "fb_attn_workspace_bytes", "fb_attn_fwd", "fb_attn_dense_bias_fwd",
     "fb_factors_sandwich", "fb_factors_alibi", "fb_svd_factors_host", "fb_check_device_error",
     "fb_selftest_wait_timeout", "fb_attn_fwd_noalloc", "fb_attn_prepare_factors", "fb_attn_fwd_prepared",
+    "fb_attn_mul_bias_workspace_bytes", "fb_attn_mul_bias_fwd",
 )
 
 
@@ -73,6 +75,11 @@ def lib() -> ctypes.CDLL:
         L.fb_attn_fwd_prepared.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, i32, i64, i64, f32, i32, vp, vp, vp,
                                            sz, vp]
         L.fb_attn_fwd_prepared.restype = i32
+        L.fb_attn_mul_bias_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
+        L.fb_attn_mul_bias_workspace_bytes.restype = sz
+        L.fb_attn_mul_bias_fwd.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, i32, vp, vp, i64, i64, f32, i32, vp,
+                                           vp, vp, sz, vp]
+        L.fb_attn_mul_bias_fwd.restype = i32
         L.fb_attn_dense_bias_fwd.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, i64, i64, f32, i32, vp, vp, vp]
         L.fb_attn_dense_bias_fwd.restype = i32
         L.fb_factors_sandwich.argtypes, L.fb_factors_sandwich.restype = [i32, i32, vp, vp, vp], i32
@@ -115,6 +122,16 @@ def fb_attn_fwd_prepared(dt, B, H, N, d, Q, K, V, R, phi_bstride, phi_hstride, s
                          workspace_bytes, stream) -> int:
     return lib().fb_attn_fwd_prepared(dt, B, H, N, d, Q, K, V, R, phi_bstride, phi_hstride, scale, causal, O, LSE,
                                       workspace, workspace_bytes, stream)
+
+
+def fb_attn_mul_bias_workspace_bytes(B, H, N, d, R) -> int:
+    return lib().fb_attn_mul_bias_workspace_bytes(B, H, N, d, R)
+
+
+def fb_attn_mul_bias_fwd(dt, B, H, N, d, Q, K, V, R, phi_q, phi_k, phi_bstride, phi_hstride, scale, causal, O, LSE,
+                         workspace, workspace_bytes, stream) -> int:
+    return lib().fb_attn_mul_bias_fwd(dt, B, H, N, d, Q, K, V, R, phi_q, phi_k, phi_bstride, phi_hstride, scale,
+                                      causal, O, LSE, workspace, workspace_bytes, stream)
 
 
 def fb_attn_fwd_noalloc(dt, B, H, N, d, Q, K, V, R, phi_q, phi_k, phi_bstride, phi_hstride, scale, causal, O, LSE,
@@ -216,6 +233,33 @@ def attn(q, k, v, phi_q=None, phi_k=None, scale=None, causal=False, out=None, ls
     _check(fb_attn_fwd(dt, B, H, N, d, q.data_ptr(), k.data_ptr(), v.data_ptr(), R, pq, pk, bs, hs, scale,
                        int(bool(causal)), o.data_ptr(), l.data_ptr(), ws_ptr, ws_bytes, _stream(q.device)),
            "fb_attn_fwd")
+    return o, l
+
+
+def attn_mul_bias(q, k, v, phi_q, phi_k, scale=None, causal=False, out=None, lse=None, workspace=None):
+    """O, LSE = softmax(scale (q k^T) o (phi_q phi_k^T) [+ causal]) v through
+    fb_attn_mul_bias_fwd (multiplicative low-rank bias; bf16 q, k, v).
+
+    phi_q, phi_k: fp32 [N, R], [H, N, R] or [B, H, N, R] (last two dims
+    contiguous). Returns (O, LSE)."""
+    import torch
+    assert q.is_cuda and q.dtype == torch.bfloat16 and q.is_contiguous() and k.is_contiguous() \
+        and v.is_contiguous()
+    assert phi_q.dtype == torch.float32 and phi_k.dtype == torch.float32
+    assert phi_q.shape == phi_k.shape and phi_q.stride() == phi_k.stride()
+    assert phi_q.stride(-1) == 1 and phi_q.stride(-2) == phi_q.shape[-1]
+    B, H, N, d = q.shape
+    R = phi_q.shape[-1]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    bs, hs = _factor_strides(phi_q, B, H, N, R)
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if lse is None else lse
+    ws_bytes = fb_attn_mul_bias_workspace_bytes(B, H, N, d, R)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), device=q.device, dtype=torch.uint8)
+    _check(fb_attn_mul_bias_fwd(FB_BF16, B, H, N, d, q.data_ptr(), k.data_ptr(), v.data_ptr(), R, phi_q.data_ptr(),
+                                phi_k.data_ptr(), bs, hs, scale, int(bool(causal)), o.data_ptr(), l.data_ptr(),
+                                workspace.data_ptr(), ws_bytes, _stream(q.device)), "fb_attn_mul_bias_fwd")
     return o, l
 
 

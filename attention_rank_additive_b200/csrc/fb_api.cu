@@ -304,6 +304,61 @@ int fb_attn_fwd(int dt, int B, int H, int N, int d, const void *Q, const void *K
                               workspace_bytes, stream);
 }
 
+namespace {
+struct MulLayout {
+  size_t q1_off, k1_off, fac_off, fac_bytes, total;
+  int Rf;  // rank of the factor part: d (R - 1)
+};
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+MulLayout mul_layout(int B, int H, int N, int d, int R) {
+  MulLayout m{};
+  const size_t qk = size_t(B) * H * N * d * 2;
+  m.Rf = d * (R - 1);
+  m.q1_off = 0;
+  m.k1_off = align256(qk);
+  m.fac_off = m.k1_off + align256(qk);
+  const int64_t hs = int64_t(N) * m.Rf, bs = int64_t(H) * hs;
+  m.fac_bytes = m.Rf > 0 ? workspace_layout(B, H, N, m.Rf, bs, hs).total : 0;
+  m.total = m.fac_off + m.fac_bytes;
+  return m;
+}
+}  // namespace
+
+size_t fb_attn_mul_bias_workspace_bytes(int B, int H, int N, int d, int R) {
+  if (B < 1 || H < 1 || N < 1 || R < 1 || d < 8 || d * (R - 1) > 128) return 0;
+  return mul_layout(B, H, N, d, R).total;
+}
+
+int fb_attn_mul_bias_fwd(int dt, int B, int H, int N, int d, const void *Q, const void *K, const void *V, int R,
+                         const float *phi_q, const float *phi_k, int64_t phi_bstride, int64_t phi_hstride, float scale,
+                         int causal, void *O, float *LSE, void *workspace, size_t workspace_bytes, void *stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!Q || !K || !V || !O || !LSE || !phi_q || !phi_k) return FB_ERR_INVALID_ARG;
+  if (dt != FB_BF16) return FB_ERR_UNSUPPORTED;
+  if (R < 1 || d * (R - 1) > 128) return FB_ERR_UNSUPPORTED;
+  if (phi_bstride < 0 || phi_hstride < 0) return FB_ERR_INVALID_ARG;
+  if (!valid_scale(scale)) return FB_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE)) return FB_ERR_INVALID_ARG;
+  if (((reinterpret_cast<uintptr_t>(phi_q) | reinterpret_cast<uintptr_t>(phi_k)) & 3u) != 0) return FB_ERR_INVALID_ARG;
+  if (!valid_shape_bf16(B, H, N, d)) return FB_ERR_UNSUPPORTED;
+  const MulLayout m = mul_layout(B, H, N, d, R);
+  if (!workspace || workspace_bytes < m.total || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return FB_ERR_WORKSPACE;
+  int *flags = device_flags();
+  if (!flags) return FB_ERR_CUDA;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  const int64_t hs = int64_t(N) * m.Rf, bs = int64_t(H) * hs;
+  const WsLayout fl = workspace_layout(B, H, N, m.Rf, bs, hs);
+  const int RP = m.Rf > 0 ? pad_rank(m.Rf) : 0;
+  void *fq = m.Rf > 0 ? ws + m.fac_off + fl.q_off : nullptr;
+  void *fk = m.Rf > 0 ? ws + m.fac_off + fl.k_off : nullptr;
+  if (launch_prep_mul_bias(B, H, N, d, R, RP, Q, K, phi_q, phi_k, phi_bstride, phi_hstride, ws + m.q1_off,
+                           ws + m.k1_off, fq, fk, flags, st) != cudaSuccess)
+    return FB_ERR_CUDA;
+  return fb_attn_fwd_prepared(FB_BF16, B, H, N, d, ws + m.q1_off, ws + m.k1_off, V, m.Rf, bs, hs, scale, causal, O, LSE,
+                              m.Rf > 0 ? ws + m.fac_off : nullptr, m.fac_bytes, stream);
+}
+
 int fb_attn_dense_bias_fwd(int dt, int B, int H, int N, int d, const void *Q, const void *K, const void *V,
                            const void *Bias, int64_t bias_bstride, int64_t bias_hstride, float scale, int causal,
                            void *O, float *LSE, void *stream) {

@@ -76,8 +76,6 @@ __global__ void prep_mma_kernel(int N, int R, int RP, int fac_H, const float *__
   if (overflow) atomicOr(flags, kFlagRange);
 }
 
-// Preparation for the CUDA-core factor path (R <= 4, fp32):
-//   out_q[f, n, 0..3] = phi_q * log2(e) (zero padded), out_k[f, n, 0..3] = phi_k.
 // Rank <= 4: the factors enter the tensor cores as tf32 (kind::tf32 MMA),
 // split so that the product keeps fp32 accuracy: x = hi + lo with hi = x with
 // its 13 low mantissa bits cleared (what a tf32 operand holds) and lo = x - hi
@@ -120,6 +118,63 @@ __global__ void prep_tf32_kernel(int N, int R, int KT, int fac_H, const float *_
       }
     }
   }
+}
+
+// Multiplicative bias b = phi_q phi_k^T (rebuttal, reply to Reviewer BRmd,
+// Q1 (2), Eq. (3)): (q k^T) * b = sum_r (q phi_q,r)(k phi_k,r)^T. The first
+// term becomes the kernel's Q and K (bf16, [BH, N, d]); the others become its
+// factor tiles, fp16 [BH, N, RP] with column (r-1) d + c = q_c phi_q,r (not
+// divided by scale: the kernel's scale multiplies every term), zero-padded
+// from d (R-1) to RP. One thread per (row, column); values beyond the fp16
+// range are saturated and raise kFlagRange.
+__global__ void prep_mul_bias_kernel(int H, int N, int d, int R, int RP, const __nv_bfloat16 *__restrict__ Q,
+                                     const __nv_bfloat16 *__restrict__ K, const float *__restrict__ pq,
+                                     const float *__restrict__ pk, long long bs, long long hs,
+                                     __nv_bfloat16 *__restrict__ q1, __nv_bfloat16 *__restrict__ k1,
+                                     __half *__restrict__ fq, __half *__restrict__ fk, int *flags, int width,
+                                     long long total) {
+  bool overflow = false;
+  const int used = d * (R - 1);
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int c = int(idx % width);
+    const long long row = idx / width;  // bh * N + n
+    const long long n = row % N, bh = row / N;
+    const long long b = bh / H, h = bh - (bh / H) * H;
+    if (c < d) {
+      const float qc = __bfloat162float(Q[row * d + c]), kc = __bfloat162float(K[row * d + c]);
+      const long long src = b * bs + h * hs + n * R;
+      q1[row * d + c] = __float2bfloat16_rn(qc * pq[src]);
+      k1[row * d + c] = __float2bfloat16_rn(kc * pk[src]);
+      for (int r = 1; r < R; ++r) {
+        float vq = qc * pq[src + r], vk = kc * pk[src + r];
+        if (fabsf(vq) > 65504.f) { vq = copysignf(65504.f, vq); overflow = true; }
+        if (fabsf(vk) > 65504.f) { vk = copysignf(65504.f, vk); overflow = true; }
+        if (!(vq == vq) || !(vk == vk)) overflow = true;
+        fq[row * RP + (r - 1) * d + c] = __float2half_rn(vq);
+        fk[row * RP + (r - 1) * d + c] = __float2half_rn(vk);
+      }
+    }
+    if (RP > 0 && used + c < RP) {  // zero padding of the factor rows
+      fq[row * RP + used + c] = __float2half_rn(0.f);
+      fk[row * RP + used + c] = __float2half_rn(0.f);
+    }
+  }
+  if (overflow) atomicOr(flags, kFlagRange);
+}
+
+static int grid_for(long long total, int block);
+
+cudaError_t launch_prep_mul_bias(int B, int H, int N, int d, int R, int RP, const void *Q, const void *K,
+                                 const float *phi_q, const float *phi_k, int64_t bs, int64_t hs, void *q1, void *k1,
+                                 void *fq, void *fk, int *flags, cudaStream_t s) {
+  const int width = d > RP - d * (R - 1) ? d : RP - d * (R - 1);
+  const long long total = (long long)B * H * N * width;
+  prep_mul_bias_kernel<<<grid_for(total, 256), 256, 0, s>>>(
+      H, N, d, R, RP, static_cast<const __nv_bfloat16 *>(Q), static_cast<const __nv_bfloat16 *>(K), phi_q, phi_k,
+      bs, hs, static_cast<__nv_bfloat16 *>(q1), static_cast<__nv_bfloat16 *>(k1), static_cast<__half *>(fq),
+      static_cast<__half *>(fk), flags, width, total);
+  return cudaGetLastError();
 }
 
 // One CTA waits on an mbarrier that nothing completes, with a short limit,

@@ -69,6 +69,11 @@ cudaError_t launch_prep_factors(int mode, int B, int H, int N, int R, int RP, co
                                 int64_t bs, int64_t hs, int fac_B, int fac_H, float scale, void *out_q, void *out_k,
                                 int *flags, cudaStream_t s);
 cudaError_t launch_wait_selftest(int limit_ms, int *flags, cudaStream_t s);
+// Multiplicative bias: q1 = q phi_q,0 and k1 = k phi_k,0 (bf16 [BH, N, d]);
+// fp16 factor rows [BH, N, RP] with the terms r >= 1.
+cudaError_t launch_prep_mul_bias(int B, int H, int N, int d, int R, int RP, const void *Q, const void *K,
+                                 const float *phi_q, const float *phi_k, int64_t bs, int64_t hs, void *q1, void *k1,
+                                 void *fq, void *fk, int *flags, cudaStream_t s);
 
 // Per-device flag word (allocated once per device as a module global).
 int *device_flags();

@@ -146,6 +146,37 @@ int fb_attn_fwd_prepared(int dt, int B, int H, int N, int d,
                          const void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Attention with a multiplicative low-rank bias (FlashBias rebuttal, reply
+ * to Reviewer BRmd, Q1 (2), Eq. (1) and (3)):
+ *
+ *   O = softmax(scale * (Q K^T) o (phi_q phi_k^T) [+ causal mask]) V
+ *
+ * (o: elementwise product), computed as (Q K^T) o b = sum_r (Q phi_q,r)
+ * (K phi_k,r)^T: the repeated, reweighted q and k of the rebuttal's Eq. (3).
+ * The first term runs as the fused kernel's bf16 Q K^T, the other R - 1 as
+ * its fp16 factor MMA (a factor rank of d (R - 1) <= 128). Reading of Eq. (3):
+ * the printed sqrt(C) in q' would cancel the 1/sqrt(C) of Eq. (1), so it is
+ * taken as a typo and `scale` multiplies the whole product, as in Eq. (1).
+ *
+ *  dt          FB_BF16 only.
+ *  R           1 <= R and d (R - 1) <= 128 (R = 1 is a rank-1 bias).
+ *  phi_q/phi_k fp32 device factors, layout and strides as for fb_attn_fwd.
+ *  workspace   fb_attn_mul_bias_workspace_bytes(B, H, N, d, R) bytes,
+ *              256-byte aligned: the reweighted q, k and the fp16 factor rows.
+ *  Other arguments and errors as fb_attn_fwd. A product q_c phi_q,r beyond
+ *  the fp16 range is saturated and flags FB_ERR_RANGE.
+ */
+size_t fb_attn_mul_bias_workspace_bytes(int B, int H, int N, int d, int R);
+
+int fb_attn_mul_bias_fwd(int dt, int B, int H, int N, int d,
+                         const void *Q, const void *K, const void *V,
+                         int R, const float *phi_q, const float *phi_k,
+                         int64_t phi_bstride, int64_t phi_hstride,
+                         float scale, int causal,
+                         void *O, float *LSE,
+                         void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * fb_attn_fwd for callers that cannot allocate device memory. (The FlashBias
  * paper has no counterpart: this is an interface convenience.)
  *

@@ -225,3 +225,36 @@ def test_prepared_entry_points_reject_bad_arguments_before_launch():
 def test_shape_limit_on_work_items():
     # B * H * ceil(N / 128) work items must stay below 2^30 (the kernel counts them in int)
     assert _fwd(B=65536, H=128, N=16512) == fb.FB_ERR_UNSUPPORTED
+
+
+def test_mul_bias_workspace_and_argument_errors():
+    # q1, k1 bf16 [BH, N, d] each, then fp16 factor rows of rank d (R - 1) padded to 16..128
+    B, H, N, d, R = 2, 3, 130, 64, 2
+    qk = B * H * N * d * 2
+    al = lambda x: (x + 255) // 256 * 256
+    fac = fb.fb_attn_workspace_bytes(B, H, N, d * (R - 1), H * N * d, N * d)
+    assert fb.fb_attn_mul_bias_workspace_bytes(B, H, N, d, R) == 2 * al(qk) + fac
+    assert fb.fb_attn_mul_bias_workspace_bytes(B, H, N, d, 1) == 2 * al(qk)  # rank 1: no factor part
+    assert fb.fb_attn_mul_bias_workspace_bytes(B, H, N, 64, 4) == 0  # d (R - 1) > 128
+    need = fb.fb_attn_mul_bias_workspace_bytes(1, 1, 128, 64, 2)
+    run = dict(dt=fb.FB_BF16, B=1, H=1, N=128, d=64, Q=FAKE, K=FAKE, V=FAKE, R=2, phi_q=FAKE, phi_k=FAKE,
+               phi_bstride=0, phi_hstride=0, scale=0.125, causal=1, O=FAKE, LSE=FAKE, workspace=FAKE,
+               workspace_bytes=need, stream=None)
+
+    def m(**kw):
+        a = dict(run)
+        a.update(kw)
+        return fb.fb_attn_mul_bias_fwd(**a)
+
+    assert m(dt=fb.FB_F32) == fb.FB_ERR_UNSUPPORTED
+    assert m(R=0) == fb.FB_ERR_UNSUPPORTED
+    assert m(R=4) == fb.FB_ERR_UNSUPPORTED  # 64 * 3 > 128
+    assert m(phi_q=0) == fb.FB_ERR_INVALID_ARG
+    assert m(phi_k=FAKE + 2) == fb.FB_ERR_INVALID_ARG
+    assert m(phi_hstride=-1) == fb.FB_ERR_INVALID_ARG
+    assert m(Q=FAKE + 8) == fb.FB_ERR_INVALID_ARG
+    assert m(scale=0.0) == fb.FB_ERR_INVALID_ARG
+    assert m(d=12) == fb.FB_ERR_UNSUPPORTED
+    assert m(workspace=0) == fb.FB_ERR_WORKSPACE
+    assert m(workspace_bytes=need - 1) == fb.FB_ERR_WORKSPACE
+    assert m(workspace=FAKE + 16) == fb.FB_ERR_WORKSPACE

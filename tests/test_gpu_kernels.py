@@ -236,3 +236,40 @@ def test_unsupported_dense_pitch_returns_before_launch():
     with pytest.raises(fb.FlashBiasError) as e:
         fb.attn_dense_bias(x, x, x, b)
     assert e.value.status == fb.FB_ERR_UNSUPPORTED
+
+
+# ------------------------------------------------- multiplicative low-rank bias
+
+MUL_CASES = [
+    # B, H, N, d, R, causal, factors ("cos": the rebuttal's cos(i - j) example; else N(0, std) per layout)
+    (1, 2, 300, 64, 2, True, "cos"),
+    (2, 2, 257, 32, 3, False, "bhnr"),
+    (1, 2, 200, 128, 2, True, "hnr"),
+    (1, 1, 384, 16, 9, True, "nr"),
+    (1, 2, 130, 64, 1, False, "nr"),
+]
+
+
+@pytest.mark.parametrize("B,H,N,d,R,causal,kind", MUL_CASES)
+def test_mul_bias_matches_oracle(B, H, N, d, R, causal, kind):
+    """fb_attn_mul_bias_fwd against the oracle's multiplicative definition
+    (rebuttal, reply to Reviewer BRmd, Q1 (2)); ragged tails, every head."""
+    q, k, v = si.qkv(B, H, N, d, 400 + N + R, "bf16")
+    if kind == "cos":
+        i = np.arange(N, dtype=np.float64)
+        pq = pk = np.stack([np.cos(i), np.sin(i)], 1).astype(np.float32)
+    else:
+        shape = {"nr": (N, R), "hnr": (H, N, R), "bhnr": (B, H, N, R)}[kind]
+        pq, pk = si.random_factors(shape, 0.6, 500 + R)
+    scale = 1.0 / math.sqrt(d)
+    o, l = fb.attn_mul_bias(dev(q, "bf16"), dev(k, "bf16"), dev(v, "bf16"), dev(pq, "f32"), dev(pk, "f32"),
+                            scale=scale, causal=causal)
+    torch.cuda.synchronize()
+    _no_device_error()
+    og, lg = host(o), host(l)
+    for b in range(B):
+        for h in range(H):
+            fq = pq if pq.ndim == 2 else (pq[h] if pq.ndim == 3 else pq[b, h])
+            fk = pk if pk.ndim == 2 else (pk[h] if pk.ndim == 3 else pk[b, h])
+            ro, rl = oracle.attention_mul_head(q[b, h], k[b, h], v[b, h], fq, fk, scale, causal)
+            compare(og[b, h], lg[b, h], ro, rl, "bf16", f"mul B{B} H{H} N{N} d{d} R{R} {kind} ({b},{h})")
