@@ -47,7 +47,7 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--config", type=int, default=1, choices=[0, 1, 2, 3, 4])
+    ap.add_argument("--config", type=int, default=1, choices=[0, 1, 2, 3, 4, 5])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-bias comparison leg")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline leg")
@@ -56,13 +56,16 @@ def parse_args(argv=None):
 
 def workload(cfg_idx: int) -> dict:
     c = dict(si.CONFIGS[cfg_idx])
-    c["flops"] = flops(c["B"], c["H"], c["N"], c["d"], c["R"], c["causal"])
+    c["flops"] = flops(c["B"], c["H"], c["N"], c["d"], c["R"], c["causal"], c["bias"] == "mulcos")
     return c
 
 
-def flops(B, H, N, d, R, causal) -> float:
-    """Counted FLOPs: 4 N^2 d + 2 N^2 R per head, halved when causal."""
-    f = float(B) * H * (4.0 * N * N * d + 2.0 * N * N * R)
+def flops(B, H, N, d, R, causal, multiplicative=False) -> float:
+    """Counted FLOPs per head: additive 4 N^2 d + 2 N^2 R; multiplicative
+    2 N^2 d R (the scores over the R reweighted copies of q and k) + 2 N^2 d
+    (PV); halved when causal."""
+    per = 2.0 * N * N * d * R + 2.0 * N * N * d if multiplicative else 4.0 * N * N * d + 2.0 * N * N * R
+    f = float(B) * H * per
     return f / 2.0 if causal else f
 
 
@@ -244,6 +247,12 @@ class GpuWorkload:
         elif c["bias"] == "lowrank":
             pq, pk = si.random_factors((B, H, N, R), c["factor_std"], si.FACTOR_SEED_BASE + c["index"])
             self.pq, self.pk = torch.from_numpy(pq).to(device), torch.from_numpy(pk).to(device)
+        elif c["bias"] == "mulcos":
+            # the multiplicative example's exact rank-2 factors [cos i, sin i] (static input)
+            i = np.arange(N, dtype=np.float64)
+            f = np.stack([np.cos(i), np.sin(i)], 1).astype(np.float32)
+            self.pq = torch.from_numpy(f).to(device)
+            self.pk = self.pq
         elif c["bias"] == "rbf_svd":
             om, ph = si.rbf_params(H, c["rbf_terms"])
             table = si.rbf_offset_table(om, ph, c["grid"])
@@ -262,7 +271,11 @@ class GpuWorkload:
             self.bs = self.hs = 0
         Rk = self.pq.shape[-1] if self.pq is not None else 0
         self.R = Rk
-        self.ws_bytes = fb.fb_attn_workspace_bytes(B, H, N, Rk, self.bs, self.hs) if c["dtype"] == "bf16" else 0
+        self.mul = c["bias"] == "mulcos"
+        if self.mul:
+            self.ws_bytes = fb.fb_attn_mul_bias_workspace_bytes(B, H, N, d, Rk)
+        else:
+            self.ws_bytes = fb.fb_attn_workspace_bytes(B, H, N, Rk, self.bs, self.hs) if c["dtype"] == "bf16" else 0
         self.ws = torch.empty(max(self.ws_bytes, 256), device=device, dtype=torch.uint8)
         self.flush_buf = torch.empty(L2_FLUSH_BYTES, device=device, dtype=torch.uint8)
         self.dense = None
@@ -308,7 +321,7 @@ class GpuWorkload:
     def prepare(self):
         """The factor preparation launch (bf16 path with a bias); fb_attn_fwd's first half."""
         fb, c = self.fb, self.c
-        if c["dtype"] != "bf16" or self.R == 0:
+        if c["dtype"] != "bf16" or self.R == 0 or self.mul:
             return
         st = fb.fb_attn_prepare_factors(c["B"], c["H"], c["N"], self.R, self.pq.data_ptr(), self.pk.data_ptr(),
                                         self.bs, self.hs, self.scale, self.ws.data_ptr(), self.ws_bytes, self.stream)
@@ -317,7 +330,13 @@ class GpuWorkload:
     def run(self):
         """The fused kernel alone (bf16), or the whole fp32 call."""
         fb, c = self.fb, self.c
-        if c["dtype"] == "bf16":
+        if self.mul:  # reweighting launch + fused kernel (one C-ABI call)
+            st = fb.fb_attn_mul_bias_fwd(fb.FB_BF16, c["B"], c["H"], c["N"], c["d"], self.Q.data_ptr(),
+                                         self.K.data_ptr(), self.V.data_ptr(), self.R, self.pq.data_ptr(),
+                                         self.pk.data_ptr(), self.bs, self.hs, self.scale, int(c["causal"]),
+                                         self.O.data_ptr(), self.LSE.data_ptr(), self.ws.data_ptr(), self.ws_bytes,
+                                         self.stream)
+        elif c["dtype"] == "bf16":
             st = fb.fb_attn_fwd_prepared(fb.FB_BF16, c["B"], c["H"], c["N"], c["d"], self.Q.data_ptr(),
                                          self.K.data_ptr(), self.V.data_ptr(), self.R, self.bs, self.hs, self.scale,
                                          int(c["causal"]), self.O.data_ptr(), self.LSE.data_ptr(), self.ws.data_ptr(),
@@ -370,7 +389,8 @@ def run_ours(args, rank: int, world: int, local: int):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     fb.lib()
-    w = GpuWorkload(c, device, with_dense=not args.no_dense and c["dtype"] == "bf16")
+    # (no dense counterpart for the multiplicative bias: the comparison kernel adds its bias)
+    w = GpuWorkload(c, device, with_dense=not args.no_dense and c["dtype"] == "bf16" and c["bias"] != "mulcos")
     stream = torch.cuda.current_stream(device)
 
     attn_ms = []
@@ -462,7 +482,8 @@ def run_ours(args, rank: int, world: int, local: int):
         "config": config_json(c, "flushed: 256 MiB memset between timed steps (untimed)"),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": round(achieved / peak_tf, 4), "traffic": traffic,
-                     "kernel": "attn_fwd_sm100", "peak_kind": peak_kind,
+                     "kernel": "prep_mul_bias + attn_fwd_sm100" if w.mul else "attn_fwd_sm100",
+                     "peak_kind": peak_kind,
                      "kernel_ms": round(kern_ms, 5)},
         "e2e": {"value": round(c["flops"] * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -500,6 +521,14 @@ def oracle_sample(c: dict, step: int, rows_per_head: int):
     elif c["bias"] == "lowrank":
         pq, pk = si.random_factors((B, H, N, R), c["factor_std"], si.FACTOR_SEED_BASE + c["index"])
         bias = oracle.HeadBias.lowrank(pq[b, h], pk[b, h])
+    elif c["bias"] == "mulcos":
+        f = oracle.cos_factors(N)
+        keys = (rows + 1).astype(np.float64) if c["causal"] else np.full(rows.shape, float(N))
+
+        def run_mul():
+            oracle.attention_mul_head(q, k, v, f, f, scale, c["causal"], rows)
+
+        return run_mul, float(np.sum(keys * (2.0 * d * R + 2.0 * d))), f"{len(rows)} query rows of head (b={b}, h={h})"
     else:  # rbf_svd: the dense field truncated by the oracle's own SVD
         om, ph = si.rbf_params(H, c["rbf_terms"])
         dense = si.rbf_dense(si.rbf_offset_table(om, ph, c["grid"]), c["grid"], heads=[h])[0]

@@ -34,6 +34,9 @@ CONFIGS = [
          causal=False, bias="rbf_svd", grid=64, rbf_terms=32),
     dict(index=4, name="af3_pair_lowrank32_N1536_d24", dtype="bf16", B=1, H=16, N=1536, d=24,
          R=32, causal=False, bias="lowrank", factor_std=math.sqrt(1.0 / 32.0)),
+    # multiplicative bias b_ij = cos(i - j) (rank 2) on the GPT-2 shape: a widening case, not a headline
+    dict(index=5, name="gpt2_mulcos_N2048", dtype="bf16", B=8, H=12, N=2048, d=64, R=2,
+         causal=True, bias="mulcos"),
 ]
 
 QKV_SEED_BASE = 1000

@@ -159,3 +159,23 @@ def test_config4_pair_bias_fused_and_dense():
     torch.cuda.synchronize()
     _check_rows(od, ld, q, k, v, heads, rows, lambda b, h: HeadBias.dense(dense[h]), scale, False, "bf16",
                 "c4 dense")
+
+
+def test_config5_multiplicative_cos_full_size():
+    """The multiplicative cos(i - j) bias at the GPT-2 shape of the widening
+    case (bench.py --config 5), sampled rows of three heads against the oracle."""
+    c = si.CONFIGS[5]
+    B, H, N, d, R = c["B"], c["H"], c["N"], c["d"], c["R"]
+    q, k, v = si.qkv(B, H, N, d, si.QKV_SEED_BASE + 5, "bf16")
+    scale = 1.0 / math.sqrt(d)
+    i = np.arange(N, dtype=np.float64)
+    f = np.stack([np.cos(i), np.sin(i)], 1).astype(np.float32)
+    o, l = fb.attn_mul_bias(dev(q, "bf16"), dev(k, "bf16"), dev(v, "bf16"), dev(f, "f32"), dev(f, "f32"),
+                            scale=scale, causal=True)
+    torch.cuda.synchronize()
+    assert fb.fb_check_device_error(_stream()) == fb.FB_OK
+    og, lg = host(o), host(l)
+    rows = si.sample_rows(N, 40, 5)
+    for (b, h) in [(0, 0), (5, 6), (7, 11)]:
+        ro, rl = oracle.attention_mul_head(q[b, h], k[b, h], v[b, h], f, f, scale, True, rows)
+        compare(og[b, h][rows], lg[b, h][rows], ro, rl, "bf16", f"c5 ({b},{h})")
