@@ -125,8 +125,9 @@ __global__ void prep_tf32_kernel(int N, int R, int KT, int fac_H, const float *_
 // term becomes the kernel's Q and K (bf16, [BH, N, d]); the others become its
 // factor tiles, fp16 [BH, N, RP] with column (r-1) d + c = q_c phi_q,r (not
 // divided by scale: the kernel's scale multiplies every term), zero-padded
-// from d (R-1) to RP. One thread per (row, column); values beyond the fp16
-// range are saturated and raise kFlagRange.
+// from d (R-1) to RP. One thread per (row, group of 8 columns), 16-byte
+// loads and stores (d, d (R-1) and RP are multiples of 8); values beyond the
+// fp16 range are saturated and raise kFlagRange.
 __global__ void prep_mul_bias_kernel(int H, int N, int d, int R, int RP, const __nv_bfloat16 *__restrict__ Q,
                                      const __nv_bfloat16 *__restrict__ K, const float *__restrict__ pq,
                                      const float *__restrict__ pk, long long bs, long long hs,
@@ -137,27 +138,57 @@ __global__ void prep_mul_bias_kernel(int H, int N, int d, int R, int RP, const _
   const int used = d * (R - 1);
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
        idx += (long long)gridDim.x * blockDim.x) {
-    const int c = int(idx % width);
-    const long long row = idx / width;  // bh * N + n
+    const int c = int(idx % width) * 8;  // first of 8 columns
+    const long long row = idx / width;   // bh * N + n
     const long long n = row % N, bh = row / N;
     const long long b = bh / H, h = bh - (bh / H) * H;
     if (c < d) {
-      const float qc = __bfloat162float(Q[row * d + c]), kc = __bfloat162float(K[row * d + c]);
+      const uint4 uq = *reinterpret_cast<const uint4 *>(Q + row * d + c);
+      const uint4 uk = *reinterpret_cast<const uint4 *>(K + row * d + c);
+      const __nv_bfloat162 *hq = reinterpret_cast<const __nv_bfloat162 *>(&uq);
+      const __nv_bfloat162 *hk = reinterpret_cast<const __nv_bfloat162 *>(&uk);
+      float qv[8], kv[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 fqv = __bfloat1622float2(hq[e]), fkv = __bfloat1622float2(hk[e]);
+        qv[2 * e] = fqv.x, qv[2 * e + 1] = fqv.y, kv[2 * e] = fkv.x, kv[2 * e + 1] = fkv.y;
+      }
       const long long src = b * bs + h * hs + n * R;
-      q1[row * d + c] = __float2bfloat16_rn(qc * pq[src]);
-      k1[row * d + c] = __float2bfloat16_rn(kc * pk[src]);
-      for (int r = 1; r < R; ++r) {
-        float vq = qc * pq[src + r], vk = kc * pk[src + r];
-        if (fabsf(vq) > 65504.f) { vq = copysignf(65504.f, vq); overflow = true; }
-        if (fabsf(vk) > 65504.f) { vk = copysignf(65504.f, vk); overflow = true; }
-        if (!(vq == vq) || !(vk == vk)) overflow = true;
-        fq[row * RP + (r - 1) * d + c] = __float2half_rn(vq);
-        fk[row * RP + (r - 1) * d + c] = __float2half_rn(vk);
+      for (int r = 0; r < R; ++r) {
+        const float a = pq[src + r], g = pk[src + r];
+        if (r == 0) {
+          uint4 oq, ok;
+          __nv_bfloat162 *bq = reinterpret_cast<__nv_bfloat162 *>(&oq);
+          __nv_bfloat162 *bk = reinterpret_cast<__nv_bfloat162 *>(&ok);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            bq[e] = __floats2bfloat162_rn(qv[2 * e] * a, qv[2 * e + 1] * a);
+            bk[e] = __floats2bfloat162_rn(kv[2 * e] * g, kv[2 * e + 1] * g);
+          }
+          *reinterpret_cast<uint4 *>(q1 + row * d + c) = oq;
+          *reinterpret_cast<uint4 *>(k1 + row * d + c) = ok;
+        } else {
+          uint4 oq, ok;
+          __half2 *hq2 = reinterpret_cast<__half2 *>(&oq);
+          __half2 *hk2 = reinterpret_cast<__half2 *>(&ok);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float v0 = qv[2 * e] * a, v1 = qv[2 * e + 1] * a, w0 = kv[2 * e] * g, w1 = kv[2 * e + 1] * g;
+            overflow |= !(fabsf(v0) <= 65504.f) || !(fabsf(v1) <= 65504.f) || !(fabsf(w0) <= 65504.f) ||
+                        !(fabsf(w1) <= 65504.f);
+            v0 = fminf(fmaxf(v0, -65504.f), 65504.f), v1 = fminf(fmaxf(v1, -65504.f), 65504.f);
+            w0 = fminf(fmaxf(w0, -65504.f), 65504.f), w1 = fminf(fmaxf(w1, -65504.f), 65504.f);
+            hq2[e] = __floats2half2_rn(v0, v1);
+            hk2[e] = __floats2half2_rn(w0, w1);
+          }
+          *reinterpret_cast<uint4 *>(fq + row * RP + (r - 1) * d + c) = oq;
+          *reinterpret_cast<uint4 *>(fk + row * RP + (r - 1) * d + c) = ok;
+        }
       }
     }
     if (RP > 0 && used + c < RP) {  // zero padding of the factor rows
-      fq[row * RP + used + c] = __float2half_rn(0.f);
-      fk[row * RP + used + c] = __float2half_rn(0.f);
+      *reinterpret_cast<uint4 *>(fq + row * RP + used + c) = make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4 *>(fk + row * RP + used + c) = make_uint4(0u, 0u, 0u, 0u);
     }
   }
   if (overflow) atomicOr(flags, kFlagRange);
@@ -168,7 +199,7 @@ static int grid_for(long long total, int block);
 cudaError_t launch_prep_mul_bias(int B, int H, int N, int d, int R, int RP, const void *Q, const void *K,
                                  const float *phi_q, const float *phi_k, int64_t bs, int64_t hs, void *q1, void *k1,
                                  void *fq, void *fk, int *flags, cudaStream_t s) {
-  const int width = d > RP - d * (R - 1) ? d : RP - d * (R - 1);
+  const int width = (d > RP - d * (R - 1) ? d : RP - d * (R - 1)) / 8;  // groups of 8 columns
   const long long total = (long long)B * H * N * width;
   prep_mul_bias_kernel<<<grid_for(total, 256), 256, 0, s>>>(
       H, N, d, R, RP, static_cast<const __nv_bfloat16 *>(Q), static_cast<const __nv_bfloat16 *>(K), phi_q, phi_k,
