@@ -23,6 +23,7 @@ __all__ = [
     "fb_factors_sandwich", "fb_factors_alibi", "fb_svd_factors_host", "fb_check_device_error",
     "fb_selftest_wait_timeout", "fb_attn_fwd_noalloc", "fb_attn_prepare_factors", "fb_attn_fwd_prepared",
     "fb_attn_mul_bias_workspace_bytes", "fb_attn_mul_bias_fwd", "attn_mul_bias", "attn",
+    "fb_svd_device_workspace_bytes", "fb_svd_factors_device", "svd_factors_device",
     "PreparedBias", "attn_dense_bias", "factors_sandwich", "factors_alibi", "svd_factors",
     "attn_flops",
 ]
@@ -38,7 +39,8 @@ EXPORTED = (
     "fb_status_str", "fb_version", "fb_attn_workspace_bytes", "fb_attn_fwd", "fb_attn_dense_bias_fwd",
     "fb_factors_sandwich", "fb_factors_alibi", "fb_svd_factors_host", "fb_check_device_error",
     "fb_selftest_wait_timeout", "fb_attn_fwd_noalloc", "fb_attn_prepare_factors", "fb_attn_fwd_prepared",
-    "fb_attn_mul_bias_workspace_bytes", "fb_attn_mul_bias_fwd",
+    "fb_attn_mul_bias_workspace_bytes", "fb_attn_mul_bias_fwd", "fb_svd_device_workspace_bytes",
+    "fb_svd_factors_device",
 )
 
 
@@ -80,6 +82,10 @@ def lib() -> ctypes.CDLL:
         L.fb_attn_mul_bias_fwd.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, i32, vp, vp, i64, i64, f32, i32, vp,
                                            vp, vp, sz, vp]
         L.fb_attn_mul_bias_fwd.restype = i32
+        L.fb_svd_device_workspace_bytes.argtypes = [i32, i32, i32, i32]
+        L.fb_svd_device_workspace_bytes.restype = sz
+        L.fb_svd_factors_device.argtypes = [i32, i32, i32, i32, i32, ctypes.c_uint64, vp, vp, vp, vp, vp, sz, vp]
+        L.fb_svd_factors_device.restype = i32
         L.fb_attn_dense_bias_fwd.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, i64, i64, f32, i32, vp, vp, vp]
         L.fb_attn_dense_bias_fwd.restype = i32
         L.fb_factors_sandwich.argtypes, L.fb_factors_sandwich.restype = [i32, i32, vp, vp, vp], i32
@@ -132,6 +138,39 @@ def fb_attn_mul_bias_fwd(dt, B, H, N, d, Q, K, V, R, phi_q, phi_k, phi_bstride, 
                          workspace, workspace_bytes, stream) -> int:
     return lib().fb_attn_mul_bias_fwd(dt, B, H, N, d, Q, K, V, R, phi_q, phi_k, phi_bstride, phi_hstride, scale,
                                       causal, O, LSE, workspace, workspace_bytes, stream)
+
+
+def fb_svd_device_workspace_bytes(H, N, R, oversample) -> int:
+    return lib().fb_svd_device_workspace_bytes(H, N, R, oversample)
+
+
+def fb_svd_factors_device(H, N, R, oversample, power_iters, seed, bias, phi_q, phi_k, err_energy, workspace,
+                          workspace_bytes, stream) -> int:
+    return lib().fb_svd_factors_device(H, N, R, oversample, power_iters, seed, bias, phi_q, phi_k, err_energy,
+                                       workspace, workspace_bytes, stream)
+
+
+def svd_factors_device(bias, R: int, oversample: int = 16, power_iters: int = 2, seed: int = 0):
+    """Truncated SVD of dense biases on the GPU (fb_svd_factors_device).
+
+    bias: fp32 CUDA tensor [N, N] or [H, N, N]. Returns (phi_q, phi_k, err_energy)
+    with phi [.., N, R] fp32 on the device and err_energy a [H, 2] fp64 device
+    tensor (relative Frobenius error, captured energy per head)."""
+    import torch
+    squeeze = bias.dim() == 2
+    b = bias[None] if squeeze else bias
+    assert b.is_cuda and b.dtype == torch.float32 and b.is_contiguous()
+    H, N, _ = b.shape
+    pq = torch.empty((H, N, R), device=b.device, dtype=torch.float32)
+    pk = torch.empty_like(pq)
+    ee = torch.empty((H, 2), device=b.device, dtype=torch.float64)
+    nb = fb_svd_device_workspace_bytes(H, N, R, oversample)
+    ws = torch.empty(max(nb, 1), device=b.device, dtype=torch.uint8)
+    _check(fb_svd_factors_device(H, N, R, oversample, power_iters, seed, b.data_ptr(), pq.data_ptr(), pk.data_ptr(),
+                                 ee.data_ptr(), ws.data_ptr(), nb, _stream(b.device)), "fb_svd_factors_device")
+    if squeeze:
+        return pq[0], pk[0], ee
+    return pq, pk, ee
 
 
 def fb_attn_fwd_noalloc(dt, B, H, N, d, Q, K, V, R, phi_q, phi_k, phi_bstride, phi_hstride, scale, causal, O, LSE,

@@ -177,6 +177,33 @@ int fb_attn_mul_bias_fwd(int dt, int B, int H, int N, int d,
                          void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Truncated SVD of H dense biases on the GPU, for biases known only at call
+ * time (the SVD decomposition of the rebuttal, reply to Reviewer xU4x, Q6,
+ * done per call; the rebuttal calls this inefficient for dynamic biases,
+ * and this entry point makes it measurable). Randomized range finder with
+ * l = min(R + oversample, 32, N) columns and `power_iters` subspace
+ * iterations (orthonormalised by shifted CholeskyQR3 in fp64), then the
+ * eigen-decomposition of the l x l Gram matrix of the projected bias.
+ * Balanced split: phi_q = U_R sqrt(S_R), phi_k = V_R sqrt(S_R).
+ *
+ *  bias        [H, N, N] fp32 device, row-major, 4-byte aligned.
+ *  R           1 <= R <= min(N, 32).
+ *  phi_q/phi_k [H, N, R] fp32 device outputs.
+ *  err_energy  optional [H, 2] fp64 device output, 8-byte aligned:
+ *              ||B - phi_q phi_k^T||_F / ||B||_F (computed exactly) and
+ *              sum_{r<R} s_r^2 / ||B||_F^2.
+ *  workspace   fb_svd_device_workspace_bytes(H, N, R, oversample) bytes,
+ *              256-byte aligned.
+ * Asynchronous on `stream`; returns before any launch on an argument error.
+ */
+size_t fb_svd_device_workspace_bytes(int H, int N, int R, int oversample);
+
+int fb_svd_factors_device(int H, int N, int R, int oversample, int power_iters,
+                          uint64_t seed, const float *bias,
+                          float *phi_q, float *phi_k, double *err_energy,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * fb_attn_fwd for callers that cannot allocate device memory. (The FlashBias
  * paper has no counterpart: this is an interface convenience.)
  *

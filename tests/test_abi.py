@@ -258,3 +258,32 @@ def test_mul_bias_workspace_and_argument_errors():
     assert m(workspace=0) == fb.FB_ERR_WORKSPACE
     assert m(workspace_bytes=need - 1) == fb.FB_ERR_WORKSPACE
     assert m(workspace=FAKE + 16) == fb.FB_ERR_WORKSPACE
+
+
+def test_svd_device_workspace_and_argument_errors():
+    # three [H, l, N] fp32 buffers (l = min(R + oversample, 32, N)) + fp64 small matrices, each 256-aligned
+    al = lambda x: (x + 255) // 256 * 256
+    H, N, R, p = 3, 500, 8, 16
+    l = 24
+    assert fb.fb_svd_device_workspace_bytes(H, N, R, p) == 3 * al(H * l * N * 4) + al(H * (2 * l * l + 2 * l * R + 5) * 8)
+    assert fb.fb_svd_device_workspace_bytes(1, 10, 8, 40) == 3 * al(10 * 10 * 4) + al((2 * 100 + 2 * 10 * 8 + 5) * 8)
+    assert fb.fb_svd_device_workspace_bytes(1, 100, 33, 0) == 0  # R > 32
+    need = fb.fb_svd_device_workspace_bytes(2, 64, 4, 8)
+    a = dict(H=2, N=64, R=4, oversample=8, power_iters=1, seed=1, bias=FAKE, phi_q=FAKE, phi_k=FAKE, err_energy=0,
+             workspace=FAKE, workspace_bytes=need, stream=None)
+
+    def s(**kw):
+        b = dict(a)
+        b.update(kw)
+        return fb.fb_svd_factors_device(**b)
+
+    assert s(bias=0) == fb.FB_ERR_INVALID_ARG
+    assert s(phi_k=FAKE + 2) == fb.FB_ERR_INVALID_ARG
+    assert s(err_energy=FAKE + 4) == fb.FB_ERR_INVALID_ARG
+    assert s(R=0) == fb.FB_ERR_UNSUPPORTED
+    assert s(R=33) == fb.FB_ERR_UNSUPPORTED
+    assert s(R=65, N=64) == fb.FB_ERR_UNSUPPORTED
+    assert s(power_iters=-1) == fb.FB_ERR_UNSUPPORTED
+    assert s(workspace=0) == fb.FB_ERR_WORKSPACE
+    assert s(workspace_bytes=need - 1) == fb.FB_ERR_WORKSPACE
+    assert s(workspace=FAKE + 16) == fb.FB_ERR_WORKSPACE
