@@ -92,8 +92,10 @@ __global__ void __launch_bounds__(512) bx_kernel(int N, int l, const float *__re
   }
 }
 
-// Z[h] = B[h]^T X[h]: one thread per column of B (128 per CTA); X staged in
-// shared memory 64 rows at a time.
+// Z[h] += B[h]^T X[h] over one slice of 512 rows of B (Z zeroed beforehand):
+// one thread per column of B (128 per CTA), X staged in shared memory 64 rows
+// at a time; grid (column blocks, H, row slices), partial sums added with
+// atomics.
 __global__ void __launch_bounds__(128) btx_kernel(int N, int l, const float *__restrict__ B,
                                                   const float *__restrict__ X, float *__restrict__ Z) {
   __shared__ float xs[kMaxL][64];
@@ -104,14 +106,15 @@ __global__ void __launch_bounds__(128) btx_kernel(int N, int l, const float *__r
   float acc[kMaxL];
 #pragma unroll
   for (int j = 0; j < kMaxL; ++j) acc[j] = 0.f;
-  for (int i0 = 0; i0 < N; i0 += 64) {
+  const int i_end = min(N, int(blockIdx.z + 1) * 512);
+  for (int i0 = int(blockIdx.z) * 512; i0 < i_end; i0 += 64) {
     for (int e = threadIdx.x; e < l * 64; e += blockDim.x) {
       const int j = e / 64, r = e - j * 64;
       xs[j][r] = i0 + r < N ? Xh[(long long)j * N + i0 + r] : 0.f;
     }
     __syncthreads();
     if (c < N) {
-      const int rmax = min(64, N - i0);
+      const int rmax = min(64, i_end - i0);
       for (int r = 0; r < rmax; ++r) {
         const float bv = Bh[(long long)(i0 + r) * N + c];
 #pragma unroll
@@ -122,16 +125,24 @@ __global__ void __launch_bounds__(128) btx_kernel(int N, int l, const float *__r
     __syncthreads();
   }
   if (c < N) {
-    for (int j = 0; j < l; ++j) Z[(long long)h * l * N + (long long)j * N + c] = acc[j];
+    for (int j = 0; j < l; ++j) atomicAdd(&Z[(long long)h * l * N + (long long)j * N + c], acc[j]);
   }
 }
 
-// G[h] = A[h]^T A[h] in fp64 (A [l][N]); one CTA per head, one thread per
-// (a, b) pair with a <= b.
-__global__ void __launch_bounds__(1024) gram_kernel(int N, int l, const float *__restrict__ A,
-                                                    double *__restrict__ G) {
-  const int h = blockIdx.x;
+// G[h] += A[h]^T A[h] over one chunk of 256 rows (A [l][N]); fp64 sums of
+// exact fp64 products, added into G (zeroed beforehand) with atomics. Grid
+// (row chunks, H); one thread per (a, b) pair with a <= b.
+__global__ void __launch_bounds__(512) gram_kernel(int N, int l, const float *__restrict__ A,
+                                                   double *__restrict__ G) {
+  __shared__ float as[kMaxL][256];
+  const int h = blockIdx.y;
+  const long long i0 = (long long)blockIdx.x * 256;
   const float *Ah = A + (long long)h * l * N;
+  for (int e = threadIdx.x; e < l * 256; e += blockDim.x) {
+    const int j = e / 256, t = e - j * 256;
+    as[j][t] = i0 + t < N ? Ah[(long long)j * N + i0 + t] : 0.f;
+  }
+  __syncthreads();
   const int npairs = l * (l + 1) / 2;
   for (int p = threadIdx.x; p < npairs; p += blockDim.x) {
     int a = 0, rem = p;
@@ -141,44 +152,52 @@ __global__ void __launch_bounds__(1024) gram_kernel(int N, int l, const float *_
     }
     const int b = a + rem;
     double s = 0.0;
-    for (int i = 0; i < N; ++i) s += double(Ah[(long long)a * N + i]) * double(Ah[(long long)b * N + i]);
-    G[(long long)h * l * l + a * l + b] = s;
-    G[(long long)h * l * l + b * l + a] = s;
+    for (int t = 0; t < 256; ++t) s += double(as[a][t]) * double(as[b][t]);
+    atomicAdd(&G[(long long)h * l * l + a * l + b], s);
+    if (a != b) atomicAdd(&G[(long long)h * l * l + b * l + a], s);
   }
 }
 
 // T[h] = R^{-1} with R^T R = G + shift I (R upper triangular, Cholesky in
 // fp64), so that A T has orthonormal columns. A pivot that is not positive
 // (a column dependent on the previous ones) zeroes that column of T.
-// One CTA per head; its first thread does the l x l work in shared memory.
+// One warp per head: lane i updates entry i of the current row of R, and
+// lane j solves column j of the inverse.
 __global__ void chol_kernel(int H, int N, int l, double shift_coef, const double *__restrict__ G,
                             double *__restrict__ T) {
   __shared__ double Rm[kMaxL][kMaxL];
   __shared__ bool dead[kMaxL];
-  const int h = blockIdx.x;
-  if (h >= H || threadIdx.x != 0) return;
+  const int h = blockIdx.x, lane = threadIdx.x;
+  if (h >= H) return;
   const double *g = G + (long long)h * l * l;
   double *t = T + (long long)h * l * l;
   double tr = 0.0;
   for (int a = 0; a < l; ++a) tr += g[a * l + a];
   const double shift = shift_coef * tr;
-  for (int j = 0; j < l; ++j) {
-    for (int i = 0; i < l; ++i) Rm[i][j] = 0.0;
-  }
+  for (int i = 0; i < l; ++i) Rm[i][lane] = 0.0;
+  __syncwarp();
   for (int j = 0; j < l; ++j) {
     double dj = g[j * l + j] + shift;
     for (int k = 0; k < j; ++k) dj -= Rm[k][j] * Rm[k][j];
-    dead[j] = !(dj > 1e-300 && dj > 1e-14 * (g[j * l + j] + shift));
-    const double rjj = dead[j] ? 0.0 : sqrt(dj);
-    Rm[j][j] = rjj;
-    for (int i = j + 1; i < l; ++i) {
-      double v = g[j * l + i];
+    const bool dj_dead = !(dj > 1e-300 && dj > 1e-14 * (g[j * l + j] + shift));
+    const double rjj = dj_dead ? 0.0 : sqrt(dj);
+    const int i = lane;  // row j of R, entry i > j
+    double v = 0.0;
+    if (i > j && i < l) {
+      v = g[j * l + i];
       for (int k = 0; k < j; ++k) v -= Rm[k][j] * Rm[k][i];
-      Rm[j][i] = dead[j] ? 0.0 : v / rjj;
     }
+    __syncwarp();
+    if (lane == 0) {
+      dead[j] = dj_dead;
+      Rm[j][j] = rjj;
+    }
+    if (i > j && i < l) Rm[j][i] = dj_dead ? 0.0 : v / rjj;
+    __syncwarp();
   }
-  // inverse of the upper triangular Rm, column by column (back substitution)
-  for (int j = 0; j < l; ++j) {
+  // inverse of the upper triangular Rm: lane j back-substitutes column j
+  const int j = lane;
+  if (j < l) {
     for (int i = l - 1; i >= 0; --i) {
       if (i > j || dead[i]) {
         t[i * l + j] = 0.0;
@@ -212,29 +231,36 @@ __global__ void apply_kernel(int N, int l, const float *__restrict__ A, const do
   }
 }
 
-// Symmetric eigen-decomposition of M = Z^T Z (fp64 cyclic Jacobi, one thread
-// per head), then the coefficient matrices of the balanced factors:
-// Cq = W_R diag(sqrt sigma), Ck = W_R diag(1 / sqrt sigma), sigma^2 the R
-// largest eigenvalues; sig2[h] = sum of those sigma^2. One CTA per head;
-// its first thread works in shared memory.
+// Symmetric eigen-decomposition of M = Z^T Z (fp64 cyclic Jacobi), then the
+// coefficient matrices of the balanced factors: Cq = W_R diag(sqrt sigma),
+// Ck = W_R diag(1 / sqrt sigma), sigma^2 the R largest eigenvalues;
+// sig2[h] = sum of those sigma^2. One warp per head: every lane forms the
+// rotation, lane k updates entry k of the two columns, rows and V columns.
 __global__ void eig_kernel(int H, int l, int R, const double *__restrict__ Mg, double *__restrict__ Cq,
                            double *__restrict__ Ck, double *__restrict__ sig2) {
   __shared__ double A[kMaxL][kMaxL], V[kMaxL][kMaxL];
-  __shared__ bool used[kMaxL];
-  const int h = blockIdx.x;
-  if (h >= H || threadIdx.x != 0) return;
-  for (int i = 0; i < l; ++i)
-    for (int j = 0; j < l; ++j) {
-      A[i][j] = Mg[(long long)h * l * l + i * l + j];
-      V[i][j] = i == j ? 1.0 : 0.0;
+  __shared__ int order[kMaxL];
+  const int h = blockIdx.x, k = threadIdx.x;
+  if (h >= H) return;
+  for (int i = 0; i < l; ++i) {
+    if (k < l) {
+      A[i][k] = Mg[(long long)h * l * l + i * l + k];
+      V[i][k] = i == k ? 1.0 : 0.0;
     }
+  }
+  __syncwarp();
   for (int sweep = 0; sweep < 60; ++sweep) {
     double off = 0.0, diag = 0.0;
-    for (int i = 0; i < l; ++i) {
-      diag += A[i][i] * A[i][i];
-      for (int j = i + 1; j < l; ++j) off += A[i][j] * A[i][j];
+    if (k < l) {
+      diag = A[k][k] * A[k][k];
+      for (int j = k + 1; j < l; ++j) off += A[k][j] * A[k][j];
     }
-    if (off <= 1e-30 * diag || off == 0.0) break;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      off += __shfl_xor_sync(0xffffffffu, off, o);
+      diag += __shfl_xor_sync(0xffffffffu, diag, o);
+    }
+    if (off <= 1e-26 * diag || off == 0.0) break;
     for (int p = 0; p < l - 1; ++p) {
       for (int q = p + 1; q < l; ++q) {
         const double apq = A[p][q];
@@ -242,46 +268,54 @@ __global__ void eig_kernel(int H, int l, int R, const double *__restrict__ Mg, d
         const double theta = (A[q][q] - A[p][p]) / (2.0 * apq);
         const double tt = (theta >= 0 ? 1.0 : -1.0) / (fabs(theta) + sqrt(theta * theta + 1.0));
         const double cs = 1.0 / sqrt(tt * tt + 1.0), sn = tt * cs;
-        for (int k = 0; k < l; ++k) {  // columns p, q
+        __syncwarp();
+        if (k < l) {  // columns p, q
           const double akp = A[k][p], akq = A[k][q];
           A[k][p] = cs * akp - sn * akq;
           A[k][q] = sn * akp + cs * akq;
         }
-        for (int k = 0; k < l; ++k) {  // rows p, q
+        __syncwarp();
+        if (k < l) {  // rows p, q
           const double apk = A[p][k], aqk = A[q][k];
           A[p][k] = cs * apk - sn * aqk;
           A[q][k] = sn * apk + cs * aqk;
-        }
-        for (int k = 0; k < l; ++k) {
           const double vkp = V[k][p], vkq = V[k][q];
           V[k][p] = cs * vkp - sn * vkq;
           V[k][q] = sn * vkp + cs * vkq;
         }
+        __syncwarp();
       }
     }
   }
-  // the R largest eigenvalues, in decreasing order
-  for (int i = 0; i < l; ++i) used[i] = false;
-  double s2 = 0.0;
-  for (int r = 0; r < R; ++r) {
-    int best = -1;
-    for (int i = 0; i < l; ++i)
-      if (!used[i] && (best < 0 || A[i][i] > A[best][best])) best = i;
-    double lam = 0.0;
-    if (best >= 0) {
-      used[best] = true;
-      lam = fmax(A[best][best], 0.0);
+  // the R largest eigenvalues, in decreasing order (lane 0 picks them)
+  if (k == 0) {
+    bool used[kMaxL];
+    for (int i = 0; i < l; ++i) used[i] = false;
+    double s2 = 0.0;
+    for (int r = 0; r < R; ++r) {
+      int best = -1;
+      for (int i = 0; i < l; ++i)
+        if (!used[i] && (best < 0 || A[i][i] > A[best][best])) best = i;
+      order[r] = best;
+      if (best >= 0) {
+        used[best] = true;
+        s2 += fmax(A[best][best], 0.0);
+      }
     }
-    const double sigma = sqrt(lam);
-    s2 += lam;
-    const double sq = sqrt(sigma), isq = sigma > 0.0 ? 1.0 / sqrt(sigma) : 0.0;
-    for (int k = 0; k < l; ++k) {
+    sig2[h] = s2;
+  }
+  __syncwarp();
+  if (k < l) {
+    for (int r = 0; r < R; ++r) {
+      const int best = order[r];
+      const double lam = best >= 0 ? fmax(A[best][best], 0.0) : 0.0;
+      const double sigma = sqrt(lam);
+      const double sq = sqrt(sigma), isq = sigma > 0.0 ? 1.0 / sqrt(sigma) : 0.0;
       const double w = best >= 0 ? V[k][best] : 0.0;
       Cq[((long long)h * l + k) * R + r] = w * sq;
       Ck[((long long)h * l + k) * R + r] = w * isq;
     }
   }
-  sig2[h] = s2;
 }
 
 // phi[h, i, r] = sum_k A[h][k][i] C[h][k][r] (A [l][N], C [l][R] fp64,
@@ -420,19 +454,24 @@ extern "C" int fb_svd_factors_device(int H, int N, int R, int oversample, int po
   double *sums = sig2 + H;
   double *out = sums + 2 * H;
 
-  const dim3 rows16((N + 15) / 16, H), cols128((N + 127) / 128, H), rows256((N + 255) / 256, H);
+  const dim3 rows16((N + 15) / 16, H), cols128((N + 127) / 128, H, (N + 511) / 512), rows256((N + 255) / 256, H);
   const double u = 1.1102230246251565e-16;  // 2^-53: unit roundoff of the fp64 Gram matrices
   const double shift_coef = 11.0 * (double(N) * l + double(l) * (l + 1)) * u;
   const int hb = (H + 31) / 32;
   // orth(A) -> out via shifted CholeskyQR3; A and tmp are clobbered
+  const dim3 chunks256((N + 255) / 256, H);
+  auto gram = [&](const float *A) {
+    cudaMemsetAsync(G, 0, size_t(H) * l * l * sizeof(double), st);
+    gram_kernel<<<chunks256, 512, 0, st>>>(N, l, A, G);
+  };
   auto orth = [&](float *A, float *tmp, float *outp) {
-    gram_kernel<<<H, 1024, 0, st>>>(N, l, A, G);
+    gram(A);
     chol_kernel<<<H, 32, 0, st>>>(H, N, l, shift_coef, G, T);
     apply_kernel<<<rows256, 256, 0, st>>>(N, l, A, T, tmp);
-    gram_kernel<<<H, 1024, 0, st>>>(N, l, tmp, G);
+    gram(tmp);
     chol_kernel<<<H, 32, 0, st>>>(H, N, l, 0.0, G, T);
     apply_kernel<<<rows256, 256, 0, st>>>(N, l, tmp, T, A);
-    gram_kernel<<<H, 1024, 0, st>>>(N, l, A, G);
+    gram(A);
     chol_kernel<<<H, 32, 0, st>>>(H, N, l, 0.0, G, T);
     apply_kernel<<<rows256, 256, 0, st>>>(N, l, A, T, outp);
   };
@@ -441,13 +480,15 @@ extern "C" int fb_svd_factors_device(int H, int N, int R, int oversample, int po
   bx_kernel<<<rows16, 512, 0, st>>>(N, l, bias, P1, P0);  // Y = B Omega
   orth(P0, P1, P2);                                         // Q in P2
   for (int it = 0; it < power_iters; ++it) {
+    cudaMemsetAsync(P0, 0, size_t(H) * l * N * sizeof(float), st);
     btx_kernel<<<cols128, 128, 0, st>>>(N, l, bias, P2, P0);  // Z = B^T Q
     orth(P0, P2, P1);                                         // Z orthonormal in P1
     bx_kernel<<<rows16, 512, 0, st>>>(N, l, bias, P1, P0);   // Y = B Z
     orth(P0, P1, P2);                                         // Q in P2
   }
+  cudaMemsetAsync(P0, 0, size_t(H) * l * N * sizeof(float), st);
   btx_kernel<<<cols128, 128, 0, st>>>(N, l, bias, P2, P0);  // M = B^T Q
-  gram_kernel<<<H, 1024, 0, st>>>(N, l, P0, G);             // M^T M
+  gram(P0);                                                 // M^T M
   eig_kernel<<<H, 32, 0, st>>>(H, l, R, G, Cq, Ck, sig2);
   rows_kernel<<<rows256, 256, 0, st>>>(N, l, R, P2, Cq, phi_q);
   rows_kernel<<<rows256, 256, 0, st>>>(N, l, R, P0, Ck, phi_k);

@@ -259,10 +259,12 @@ class GpuWorkload:
             pq = np.empty((H, N, R), np.float32)
             pk = np.empty((H, N, R), np.float32)
             self.svd_err = []
+            t0 = time.perf_counter()
             for h in range(H):
                 pq[h], pk[h], err, en = fb.svd_factors(si.rbf_dense(table, c["grid"], heads=[h])[0], R,
                                                        oversample=64, power_iters=1, seed=h)
                 self.svd_err.append((round(err, 4), round(en, 4)))
+            self.svd_host_s = time.perf_counter() - t0  # includes building each dense field on the host
             self.pq, self.pk = torch.from_numpy(pq).to(device), torch.from_numpy(pk).to(device)
             self.rbf_table = table
         if self.pq is not None:
@@ -363,6 +365,32 @@ class GpuWorkload:
 
     def flush_l2(self):
         self.flush_buf.zero_()
+
+
+def svd_device_leg(torch, fb, w, c, stream):
+    """The same truncation on the GPU (fb_svd_factors_device) from the fp32
+    dense fields, timed with CUDA events; its per-head error and energy."""
+    H, N, R = c["H"], c["N"], c["R"]
+    dense = torch.from_numpy(si.rbf_dense(w.rbf_table, c["grid"]).astype(np.float32)).to(w.device)
+    pq = torch.empty((H, N, R), device=w.device, dtype=torch.float32)
+    pk = torch.empty_like(pq)
+    ee = torch.empty((H, 2), device=w.device, dtype=torch.float64)
+    nb = fb.fb_svd_device_workspace_bytes(H, N, R, 24)
+    ws = torch.empty(nb, device=w.device, dtype=torch.uint8)
+
+    def run():
+        st = fb.fb_svd_factors_device(H, N, R, 24, 2, 7, dense.data_ptr(), pq.data_ptr(), pk.data_ptr(),
+                                      ee.data_ptr(), ws.data_ptr(), nb, stream.cuda_stream)
+        assert st == fb.FB_OK, fb.fb_status_str(st)
+
+    run()
+    torch.cuda.synchronize()
+    ms = statistics.median(time_steps(torch, run, None, 5, stream))
+    e = ee.cpu().numpy()
+    return {"ms": round(ms, 3), "heads": H, "N": N, "R": R, "oversample": 24, "power_iters": 2,
+            "rank_error_energy_per_head": [(round(float(a), 4), round(float(b), 4)) for a, b in e],
+            "host_s_same_heads": round(w.svd_host_s, 2),
+            "host_settings": "fb_svd_factors_host, oversample 64, power_iters 1, fp64"}
 
 
 # ------------------------------------------------------------------ timing
@@ -492,6 +520,7 @@ def run_ours(args, rank: int, world: int, local: int):
     }
     if hasattr(w, "svd_err"):
         out["svd_rank_error_energy_per_head"] = w.svd_err
+        out["svd_device"] = svd_device_leg(torch, fb, w, c, stream)
     if world > 1:
         # every rank sampled its own GPU; rank 0 reports its own
         pass
