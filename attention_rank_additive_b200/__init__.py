@@ -24,6 +24,7 @@ __all__ = [
     "fb_selftest_wait_timeout", "fb_attn_fwd_noalloc", "fb_attn_prepare_factors", "fb_attn_fwd_prepared",
     "fb_attn_mul_bias_workspace_bytes", "fb_attn_mul_bias_fwd", "attn_mul_bias", "attn",
     "fb_svd_device_workspace_bytes", "fb_svd_factors_device", "svd_factors_device",
+    "fb_attn_neural_workspace_bytes", "fb_attn_neural_fwd", "attn_neural",
     "PreparedBias", "attn_dense_bias", "factors_sandwich", "factors_alibi", "svd_factors",
     "attn_flops",
 ]
@@ -40,7 +41,7 @@ EXPORTED = (
     "fb_factors_sandwich", "fb_factors_alibi", "fb_svd_factors_host", "fb_check_device_error",
     "fb_selftest_wait_timeout", "fb_attn_fwd_noalloc", "fb_attn_prepare_factors", "fb_attn_fwd_prepared",
     "fb_attn_mul_bias_workspace_bytes", "fb_attn_mul_bias_fwd", "fb_svd_device_workspace_bytes",
-    "fb_svd_factors_device",
+    "fb_svd_factors_device", "fb_attn_neural_workspace_bytes", "fb_attn_neural_fwd",
 )
 
 
@@ -86,6 +87,11 @@ def lib() -> ctypes.CDLL:
         L.fb_svd_device_workspace_bytes.restype = sz
         L.fb_svd_factors_device.argtypes = [i32, i32, i32, i32, i32, ctypes.c_uint64, vp, vp, vp, vp, vp, sz, vp]
         L.fb_svd_factors_device.restype = i32
+        L.fb_attn_neural_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
+        L.fb_attn_neural_workspace_bytes.restype = sz
+        L.fb_attn_neural_fwd.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, i32, i32, vp, vp, vp, vp, f32, i32, vp,
+                                         vp, vp, sz, vp]
+        L.fb_attn_neural_fwd.restype = i32
         L.fb_attn_dense_bias_fwd.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, i64, i64, f32, i32, vp, vp, vp]
         L.fb_attn_dense_bias_fwd.restype = i32
         L.fb_factors_sandwich.argtypes, L.fb_factors_sandwich.restype = [i32, i32, vp, vp, vp], i32
@@ -171,6 +177,41 @@ def svd_factors_device(bias, R: int, oversample: int = 16, power_iters: int = 2,
     if squeeze:
         return pq[0], pk[0], ee
     return pq, pk, ee
+
+
+def fb_attn_neural_workspace_bytes(B, H, N, F, R) -> int:
+    return lib().fb_attn_neural_workspace_bytes(B, H, N, F, R)
+
+
+def fb_attn_neural_fwd(dt, B, H, N, d, Q, K, V, F, R, X_q, X_k, W_q, W_k, scale, causal, O, LSE, workspace,
+                       workspace_bytes, stream) -> int:
+    return lib().fb_attn_neural_fwd(dt, B, H, N, d, Q, K, V, F, R, X_q, X_k, W_q, W_k, scale, causal, O, LSE,
+                                    workspace, workspace_bytes, stream)
+
+
+def attn_neural(q, k, v, x_q, x_k, w_q, w_k, scale=None, causal=False, out=None, lse=None):
+    """Attention whose bias factors come from linear layers on token features
+    (fb_attn_neural_fwd): phi_q[b, h] = x_q[b] w_q[h], phi_k[b, h] = x_k[b] w_k[h].
+
+    q, k, v: bf16 CUDA [B, H, N, d]; x_q, x_k: fp32 [B, N, F]; w_q, w_k: fp32
+    [H, F, R]. Returns (O, LSE)."""
+    import torch
+    assert q.is_cuda and q.dtype == torch.bfloat16 and q.is_contiguous() and k.is_contiguous() \
+        and v.is_contiguous()
+    for t in (x_q, x_k, w_q, w_k):
+        assert t.is_cuda and t.dtype == torch.float32 and t.is_contiguous()
+    B, H, N, d = q.shape
+    F, R = w_q.shape[1], w_q.shape[2]
+    assert x_q.shape == (B, N, F) and x_k.shape == (B, N, F) and w_k.shape == (H, F, R)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, H, N), device=q.device, dtype=torch.float32) if lse is None else lse
+    nb = fb_attn_neural_workspace_bytes(B, H, N, F, R)
+    ws = torch.empty(max(nb, 1), device=q.device, dtype=torch.uint8)
+    _check(fb_attn_neural_fwd(FB_BF16, B, H, N, d, q.data_ptr(), k.data_ptr(), v.data_ptr(), F, R, x_q.data_ptr(),
+                              x_k.data_ptr(), w_q.data_ptr(), w_k.data_ptr(), scale, int(bool(causal)), o.data_ptr(),
+                              l.data_ptr(), ws.data_ptr(), nb, _stream(q.device)), "fb_attn_neural_fwd")
+    return o, l
 
 
 def fb_attn_fwd_noalloc(dt, B, H, N, d, Q, K, V, R, phi_q, phi_k, phi_bstride, phi_hstride, scale, causal, O, LSE,

@@ -366,6 +366,54 @@ int fb_attn_mul_bias_fwd(int dt, int B, int H, int N, int d, const void *Q, cons
                               m.Rf > 0 ? ws + m.fac_off : nullptr, m.fac_bytes, stream);
 }
 
+namespace {
+struct NeuralLayout {
+  size_t q_off, k_off, prep_off, prep_bytes, total;
+};
+NeuralLayout neural_layout(int B, int H, int N, int R) {
+  NeuralLayout m{};
+  const size_t phi = align256(size_t(B) * H * N * R * 4);
+  m.q_off = 0;
+  m.k_off = phi;
+  m.prep_off = 2 * phi;
+  const int64_t hs = int64_t(N) * R, bs = int64_t(H) * hs;
+  m.prep_bytes = workspace_layout(B, H, N, R, bs, hs).total;
+  m.total = m.prep_off + m.prep_bytes;
+  return m;
+}
+bool neural_ok(int F, int R) { return F >= 1 && F <= 256 && R >= 1 && R <= 128 && F * R <= 8192; }
+}  // namespace
+
+size_t fb_attn_neural_workspace_bytes(int B, int H, int N, int F, int R) {
+  if (B < 1 || H < 1 || N < 1 || !neural_ok(F, R)) return 0;
+  return neural_layout(B, H, N, R).total;
+}
+
+int fb_attn_neural_fwd(int dt, int B, int H, int N, int d, const void *Q, const void *K, const void *V, int F,
+                       int R, const float *X_q, const float *X_k, const float *W_q, const float *W_k, float scale,
+                       int causal, void *O, float *LSE, void *workspace, size_t workspace_bytes, void *stream) {
+  if (!Q || !K || !V || !O || !LSE || !X_q || !X_k || !W_q || !W_k) return FB_ERR_INVALID_ARG;
+  if (dt != FB_BF16) return FB_ERR_UNSUPPORTED;
+  if (!neural_ok(F, R)) return FB_ERR_UNSUPPORTED;
+  if (!valid_scale(scale)) return FB_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE)) return FB_ERR_INVALID_ARG;
+  if (((reinterpret_cast<uintptr_t>(X_q) | reinterpret_cast<uintptr_t>(X_k) | reinterpret_cast<uintptr_t>(W_q) |
+        reinterpret_cast<uintptr_t>(W_k)) & 3u) != 0)
+    return FB_ERR_INVALID_ARG;
+  if (!valid_shape_bf16(B, H, N, d)) return FB_ERR_UNSUPPORTED;
+  const NeuralLayout m = neural_layout(B, H, N, R);
+  if (!workspace || workspace_bytes < m.total || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return FB_ERR_WORKSPACE;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  float *pq = reinterpret_cast<float *>(ws + m.q_off), *pk = reinterpret_cast<float *>(ws + m.k_off);
+  if (launch_neural_factors(B, H, N, F, R, X_q, X_k, W_q, W_k, pq, pk, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
+    return FB_ERR_CUDA;
+  const int64_t hs = int64_t(N) * R, bs = int64_t(H) * hs;
+  return fb_attn_fwd(FB_BF16, B, H, N, d, Q, K, V, R, pq, pk, bs, hs, scale, causal, O, LSE, ws + m.prep_off,
+                     m.prep_bytes, stream);
+}
+
 int fb_attn_dense_bias_fwd(int dt, int B, int H, int N, int d, const void *Q, const void *K, const void *V,
                            const void *Bias, int64_t bias_bstride, int64_t bias_hstride, float scale, int causal,
                            void *O, float *LSE, void *stream) {

@@ -194,6 +194,52 @@ __global__ void prep_mul_bias_kernel(int H, int N, int d, int R, int RP, const _
   if (overflow) atomicOr(flags, kFlagRange);
 }
 
+// Neural decomposition (rebuttal, reply to Reviewer xU4x, Q4: the factors
+// of a dynamic bias come from lightweight networks, "simple linear layers"):
+// phi_q[b, h] = X_q[b] W_q[h], phi_k[b, h] = X_k[b] W_k[h]; X [B, N, F],
+// W [H, F, R], phi [B, H, N, R], all fp32 (fp32 products and sums). Grid
+// (row blocks of 64, B H); the CTA holds W_q[h] and W_k[h] in shared memory
+// (F R <= 8192 each) and one thread computes one (row, column) pair of both.
+__global__ void __launch_bounds__(256) neural_factor_kernel(int H, int N, int F, int R,
+                                                            const float *__restrict__ Xq,
+                                                            const float *__restrict__ Xk,
+                                                            const float *__restrict__ Wq,
+                                                            const float *__restrict__ Wk, float *__restrict__ pq,
+                                                            float *__restrict__ pk) {
+  extern __shared__ float wsm[];  // [2][F][R]
+  const int bh = blockIdx.y, b = bh / H, h = bh - (bh / H) * H;
+  for (int e = threadIdx.x; e < F * R; e += blockDim.x) {
+    wsm[e] = Wq[(long long)h * F * R + e];
+    wsm[F * R + e] = Wk[(long long)h * F * R + e];
+  }
+  __syncthreads();
+  const long long n0 = (long long)blockIdx.x * 64;
+  for (int e = threadIdx.x; e < 64 * R; e += blockDim.x) {
+    const int rr = e / R, r = e - rr * R;
+    const long long n = n0 + rr;
+    if (n >= N) break;
+    const float *xq = Xq + ((long long)b * N + n) * F;
+    const float *xk = Xk + ((long long)b * N + n) * F;
+    float sq = 0.f, sk = 0.f;
+    for (int f = 0; f < F; ++f) {
+      sq = fmaf(xq[f], wsm[f * R + r], sq);
+      sk = fmaf(xk[f], wsm[F * R + f * R + r], sk);
+    }
+    pq[((long long)bh * N + n) * R + r] = sq;
+    pk[((long long)bh * N + n) * R + r] = sk;
+  }
+}
+
+cudaError_t launch_neural_factors(int B, int H, int N, int F, int R, const float *Xq, const float *Xk,
+                                  const float *Wq, const float *Wk, float *pq, float *pk, cudaStream_t s) {
+  const size_t smem = size_t(2) * F * R * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(neural_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  const dim3 grid((N + 63) / 64, B * H);
+  neural_factor_kernel<<<grid, 256, smem, s>>>(H, N, F, R, Xq, Xk, Wq, Wk, pq, pk);
+  return cudaGetLastError();
+}
+
 static int grid_for(long long total, int block);
 
 cudaError_t launch_prep_mul_bias(int B, int H, int N, int d, int R, int RP, const void *Q, const void *K,

@@ -71,6 +71,9 @@ cudaError_t launch_prep_factors(int mode, int B, int H, int N, int R, int RP, co
 cudaError_t launch_wait_selftest(int limit_ms, int *flags, cudaStream_t s);
 // Multiplicative bias: q1 = q phi_q,0 and k1 = k phi_k,0 (bf16 [BH, N, d]);
 // fp16 factor rows [BH, N, RP] with the terms r >= 1.
+// Neural decomposition: phi_q[b, h] = X_q[b] W_q[h], phi_k[b, h] = X_k[b] W_k[h] (fp32).
+cudaError_t launch_neural_factors(int B, int H, int N, int F, int R, const float *Xq, const float *Xk,
+                                  const float *Wq, const float *Wk, float *pq, float *pk, cudaStream_t s);
 cudaError_t launch_prep_mul_bias(int B, int H, int N, int d, int R, int RP, const void *Q, const void *K,
                                  const float *phi_q, const float *phi_k, int64_t bs, int64_t hs, void *q1, void *k1,
                                  void *fq, void *fk, int *flags, cudaStream_t s);

@@ -177,6 +177,32 @@ int fb_attn_mul_bias_fwd(int dt, int B, int H, int N, int d,
                          void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Attention with a bias from the neural decomposition (FlashBias rebuttal,
+ * reply to Reviewer xU4x, Q4: the factors of a dynamic bias come from
+ * "lightweight networks", simple linear layers added to the block):
+ *
+ *   phi_q[b, h] = X_q[b] W_q[h],  phi_k[b, h] = X_k[b] W_k[h],
+ *   O = softmax(scale Q K^T + phi_q phi_k^T [+ causal]) V
+ *
+ *  X_q, X_k    [B, N, F] fp32 device token features.
+ *  W_q, W_k    [H, F, R] fp32 device weights of the two linear layers.
+ *              1 <= F <= 256, 1 <= R <= 128, F R <= 8192.
+ *  workspace   fb_attn_neural_workspace_bytes(B, H, N, F, R) bytes, 256-byte
+ *              aligned: the fp32 factors and their prepared form.
+ *  Other arguments and errors as fb_attn_fwd (dt = FB_BF16 only). The linear
+ *  layers run in fp32 in one launch, then fb_attn_fwd's two launches.
+ */
+size_t fb_attn_neural_workspace_bytes(int B, int H, int N, int F, int R);
+
+int fb_attn_neural_fwd(int dt, int B, int H, int N, int d,
+                       const void *Q, const void *K, const void *V,
+                       int F, int R, const float *X_q, const float *X_k,
+                       const float *W_q, const float *W_k,
+                       float scale, int causal,
+                       void *O, float *LSE,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Truncated SVD of H dense biases on the GPU, for biases known only at call
  * time (the SVD decomposition of the rebuttal, reply to Reviewer xU4x, Q6,
  * done per call; the rebuttal calls this inefficient for dynamic biases,

@@ -8,9 +8,11 @@ The arithmetic lives in ``fb_oracle.c`` (the definition of biased attention,
 the Sandwich and ALiBi biases and their exact factors). This module marshals
 numpy arrays for it, and adds two things in plain numpy fp64: the truncated
 SVD of a static bias (FlashBias rebuttal, reply to Reviewer xU4x, Q6: SVD
-decomposition with a per-head rank), done with ``numpy.linalg.svd``, and
+decomposition with a per-head rank), done with ``numpy.linalg.svd``;
 attention with a multiplicative bias (rebuttal, reply to Reviewer BRmd, Q1
-(2), its Eq. (1): the scaled scores are multiplied elementwise by b).
+(2), its Eq. (1): the scaled scores are multiplied elementwise by b); and the
+factors of the neural decomposition (rebuttal, reply to Reviewer xU4x, Q4:
+linear layers on token features), a library matmul.
 """
 from __future__ import annotations
 
@@ -264,3 +266,11 @@ def cos_factors(N: int) -> np.ndarray:
     [cos i, sin i] (reply to Reviewer BRmd, Q1 (2), Example), [N, 2] fp64."""
     i = np.arange(N, dtype=np.float64)
     return np.stack([np.cos(i), np.sin(i)], axis=1)
+
+
+def neural_factors(x_q, x_k, w_q, w_k):
+    """Factors of the neural decomposition (rebuttal, reply to Reviewer xU4x,
+    Q4: "simple linear layers"): phi_q[b, h] = x_q[b] w_q[h] and phi_k[b, h] =
+    x_k[b] w_k[h] in fp64. x [B, N, F], w [H, F, R] -> phi [B, H, N, R]."""
+    xq, xk, wq, wk = _f64(x_q), _f64(x_k), _f64(w_q), _f64(w_k)
+    return np.einsum("bnf,hfr->bhnr", xq, wq), np.einsum("bnf,hfr->bhnr", xk, wk)

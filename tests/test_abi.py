@@ -287,3 +287,31 @@ def test_svd_device_workspace_and_argument_errors():
     assert s(workspace=0) == fb.FB_ERR_WORKSPACE
     assert s(workspace_bytes=need - 1) == fb.FB_ERR_WORKSPACE
     assert s(workspace=FAKE + 16) == fb.FB_ERR_WORKSPACE
+
+
+def test_neural_workspace_and_argument_errors():
+    al = lambda x: (x + 255) // 256 * 256
+    B, H, N, F, R = 2, 4, 100, 16, 8
+    prep = fb.fb_attn_workspace_bytes(B, H, N, R, H * N * R, N * R)
+    assert fb.fb_attn_neural_workspace_bytes(B, H, N, F, R) == 2 * al(B * H * N * R * 4) + prep
+    assert fb.fb_attn_neural_workspace_bytes(B, H, N, 128, 128) == 0  # F R > 8192
+    need = fb.fb_attn_neural_workspace_bytes(1, 2, 128, F, R)
+    run = dict(dt=fb.FB_BF16, B=1, H=2, N=128, d=64, Q=FAKE, K=FAKE, V=FAKE, F=F, R=R, X_q=FAKE, X_k=FAKE,
+               W_q=FAKE, W_k=FAKE, scale=0.125, causal=0, O=FAKE, LSE=FAKE, workspace=FAKE, workspace_bytes=need,
+               stream=None)
+
+    def n(**kw):
+        a = dict(run)
+        a.update(kw)
+        return fb.fb_attn_neural_fwd(**a)
+
+    assert n(dt=fb.FB_F32) == fb.FB_ERR_UNSUPPORTED
+    assert n(F=0) == fb.FB_ERR_UNSUPPORTED
+    assert n(R=129) == fb.FB_ERR_UNSUPPORTED
+    assert n(F=257) == fb.FB_ERR_UNSUPPORTED
+    assert n(W_k=0) == fb.FB_ERR_INVALID_ARG
+    assert n(X_q=FAKE + 2) == fb.FB_ERR_INVALID_ARG
+    assert n(scale=-1.0) == fb.FB_ERR_INVALID_ARG
+    assert n(d=20) == fb.FB_ERR_UNSUPPORTED
+    assert n(workspace=0) == fb.FB_ERR_WORKSPACE
+    assert n(workspace_bytes=need - 1) == fb.FB_ERR_WORKSPACE

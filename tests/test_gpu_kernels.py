@@ -338,3 +338,28 @@ def test_svd_device_exact_low_rank():
     pq, pk = host(pq), host(pk)
     assert np.linalg.norm(pq[0] @ pk[0].T - Bm[0]) <= 2e-6 * np.linalg.norm(Bm[0]) + 1e-6
     _no_device_error()
+
+
+# ------------------------------------------------------- neural decomposition
+
+@pytest.mark.parametrize("B,H,N,d,F,R,causal", [(2, 3, 200, 64, 32, 16, True), (1, 4, 300, 24, 64, 32, False),
+                                                (1, 2, 257, 128, 16, 2, True), (1, 1, 129, 32, 8, 128, False)])
+def test_neural_bias_matches_oracle(B, H, N, d, F, R, causal):
+    """fb_attn_neural_fwd against the oracle: factors x w in fp64, then the
+    low-rank biased attention."""
+    rng = np.random.Generator(np.random.PCG64(900 + F + R))
+    xq, xk = rng.standard_normal((B, N, F)).astype(np.float32), rng.standard_normal((B, N, F)).astype(np.float32)
+    wq = (rng.standard_normal((H, F, R)) / math.sqrt(F * R)).astype(np.float32)
+    wk = (rng.standard_normal((H, F, R)) / math.sqrt(F)).astype(np.float32)
+    q, k, v = si.qkv(B, H, N, d, 950 + N, "bf16")
+    scale = 1.0 / math.sqrt(d)
+    o, l = fb.attn_neural(dev(q, "bf16"), dev(k, "bf16"), dev(v, "bf16"), dev(xq, "f32"), dev(xk, "f32"),
+                          dev(wq, "f32"), dev(wk, "f32"), scale=scale, causal=causal)
+    torch.cuda.synchronize()
+    _no_device_error()
+    pq, pk = oracle.neural_factors(xq, xk, wq, wk)
+    ro, rl = oracle.attention(q, k, v, lambda b, h: HeadBias.lowrank(pq[b, h], pk[b, h]), scale, causal)
+    og, lg = host(o), host(l)
+    for b in range(B):
+        for h in range(H):
+            compare(og[b, h], lg[b, h], ro[b, h], rl[b, h], "bf16", f"neural F{F} R{R} ({b},{h})")

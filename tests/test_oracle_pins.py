@@ -337,3 +337,18 @@ def test_multiplicative_cos_example_closed_form():
     st = torch.from_numpy(s)
     np.testing.assert_allclose(lse, torch.logsumexp(st, dim=-1).numpy(), atol=1e-12)
     np.testing.assert_allclose(o, (torch.softmax(st, dim=-1) @ torch.from_numpy(v)).numpy(), atol=1e-12)
+
+
+def test_neural_factors_are_the_linear_layers():
+    """phi = x w per (batch, head), against explicit loops over n, f, r."""
+    rng = np.random.Generator(np.random.PCG64(81))
+    B, H, N, F, R = 2, 3, 5, 4, 2
+    xq, xk = rng.standard_normal((B, N, F)), rng.standard_normal((B, N, F))
+    wq, wk = rng.standard_normal((H, F, R)), rng.standard_normal((H, F, R))
+    pq, pk = oracle.neural_factors(xq, xk, wq, wk)
+    for b in range(B):
+        for h in range(H):
+            for n in range(N):
+                for r in range(R):
+                    assert abs(pq[b, h, n, r] - sum(xq[b, n, f] * wq[h, f, r] for f in range(F))) < 1e-12
+                    assert abs(pk[b, h, n, r] - sum(xk[b, n, f] * wk[h, f, r] for f in range(F))) < 1e-12
