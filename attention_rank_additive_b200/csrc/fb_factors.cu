@@ -1,5 +1,6 @@
 // fb_factors.cu -- exact factor generators (Sandwich, ALiBi), the factor
 // preparation step that feeds the tensor-core kernel, and the wait self-test.
+#include <atomic>
 #include <cmath>
 
 #include "fb_internal.h"
@@ -233,8 +234,18 @@ __global__ void __launch_bounds__(256) neural_factor_kernel(int H, int N, int F,
 cudaError_t launch_neural_factors(int B, int H, int N, int F, int R, const float *Xq, const float *Xk,
                                   const float *Wq, const float *Wk, float *pq, float *pk, cudaStream_t s) {
   const size_t smem = size_t(2) * F * R * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(neural_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  if (e != cudaSuccess) return e;
+  if (smem > 48 * 1024) {  // the opt-in above the default, once per device (64 KB covers F R <= 8192)
+    static std::atomic<int> done[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!done[dev].load(std::memory_order_acquire)) {
+      e = cudaFuncSetAttribute(neural_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+      if (e != cudaSuccess) return e;
+      done[dev].store(1, std::memory_order_release);
+    }
+  }
   const dim3 grid((N + 63) / 64, B * H);
   neural_factor_kernel<<<grid, 256, smem, s>>>(H, N, F, R, Xq, Xk, Wq, Wk, pq, pk);
   return cudaGetLastError();

@@ -47,7 +47,7 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--config", type=int, default=1, choices=[0, 1, 2, 3, 4, 5])
+    ap.add_argument("--config", type=int, default=1, choices=[0, 1, 2, 3, 4, 5, 6])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-bias comparison leg")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline leg")
@@ -57,6 +57,8 @@ def parse_args(argv=None):
 def workload(cfg_idx: int) -> dict:
     c = dict(si.CONFIGS[cfg_idx])
     c["flops"] = flops(c["B"], c["H"], c["N"], c["d"], c["R"], c["causal"], c["bias"] == "mulcos")
+    if c["bias"] == "neural":  # plus the two linear layers, per (batch, head)
+        c["flops"] += 2.0 * 2.0 * c["B"] * c["H"] * c["N"] * c["F"] * c["R"]
     return c
 
 
@@ -253,6 +255,10 @@ class GpuWorkload:
             f = np.stack([np.cos(i), np.sin(i)], 1).astype(np.float32)
             self.pq = torch.from_numpy(f).to(device)
             self.pk = self.pq
+        elif c["bias"] == "neural":
+            xq, xk, wq, wk = si.neural_inputs(B, H, N, c["F"], R, si.FACTOR_SEED_BASE + c["index"])
+            self.nx = [torch.from_numpy(a).to(device) for a in (xq, xk, wq, wk)]
+            self.pq = self.pk = None
         elif c["bias"] == "rbf_svd":
             om, ph = si.rbf_params(H, c["rbf_terms"])
             table = si.rbf_offset_table(om, ph, c["grid"])
@@ -271,10 +277,13 @@ class GpuWorkload:
             self.bs, self.hs = fb._factor_strides(self.pq, B, H, N, R)
         else:
             self.bs = self.hs = 0
-        Rk = self.pq.shape[-1] if self.pq is not None else 0
+        Rk = self.pq.shape[-1] if self.pq is not None else (R if c["bias"] == "neural" else 0)
         self.R = Rk
         self.mul = c["bias"] == "mulcos"
-        if self.mul:
+        self.neural = c["bias"] == "neural"
+        if self.neural:
+            self.ws_bytes = fb.fb_attn_neural_workspace_bytes(B, H, N, c["F"], Rk)
+        elif self.mul:
             self.ws_bytes = fb.fb_attn_mul_bias_workspace_bytes(B, H, N, d, Rk)
         else:
             self.ws_bytes = fb.fb_attn_workspace_bytes(B, H, N, Rk, self.bs, self.hs) if c["dtype"] == "bf16" else 0
@@ -283,7 +292,10 @@ class GpuWorkload:
         self.dense = None
         if with_dense and c["dtype"] == "bf16":
             self.dense = self._dense_bias()
-        self.launches_per_step = (1 if Rk > 0 and c["dtype"] == "bf16" else 0) + 1  # prep + fused kernel
+        # fused kernel, plus the preparation launch (bf16 with a bias); the multiplicative case has its
+        # reweighting launch instead, the neural case its linear-layer launch in addition
+        self.launches_per_step = (3 if self.neural else
+                                  (2 if self.mul or (Rk > 0 and c["dtype"] == "bf16") else 1))
 
     def _dense_bias(self):
         """The same bias materialised as [B, H, N, N] bf16 (the comparison path's input)."""
@@ -323,7 +335,7 @@ class GpuWorkload:
     def prepare(self):
         """The factor preparation launch (bf16 path with a bias); fb_attn_fwd's first half."""
         fb, c = self.fb, self.c
-        if c["dtype"] != "bf16" or self.R == 0 or self.mul:
+        if c["dtype"] != "bf16" or self.R == 0 or self.mul or self.neural:
             return
         st = fb.fb_attn_prepare_factors(c["B"], c["H"], c["N"], self.R, self.pq.data_ptr(), self.pk.data_ptr(),
                                         self.bs, self.hs, self.scale, self.ws.data_ptr(), self.ws_bytes, self.stream)
@@ -332,7 +344,14 @@ class GpuWorkload:
     def run(self):
         """The fused kernel alone (bf16), or the whole fp32 call."""
         fb, c = self.fb, self.c
-        if self.mul:  # reweighting launch + fused kernel (one C-ABI call)
+        if self.neural:  # linear layers + preparation + fused kernel (one C-ABI call)
+            xq, xk, wq, wk = self.nx
+            st = fb.fb_attn_neural_fwd(fb.FB_BF16, c["B"], c["H"], c["N"], c["d"], self.Q.data_ptr(),
+                                       self.K.data_ptr(), self.V.data_ptr(), c["F"], self.R, xq.data_ptr(),
+                                       xk.data_ptr(), wq.data_ptr(), wk.data_ptr(), self.scale, int(c["causal"]),
+                                       self.O.data_ptr(), self.LSE.data_ptr(), self.ws.data_ptr(), self.ws_bytes,
+                                       self.stream)
+        elif self.mul:  # reweighting launch + fused kernel (one C-ABI call)
             st = fb.fb_attn_mul_bias_fwd(fb.FB_BF16, c["B"], c["H"], c["N"], c["d"], self.Q.data_ptr(),
                                          self.K.data_ptr(), self.V.data_ptr(), self.R, self.pq.data_ptr(),
                                          self.pk.data_ptr(), self.bs, self.hs, self.scale, int(c["causal"]),
@@ -418,7 +437,8 @@ def run_ours(args, rank: int, world: int, local: int):
     torch.cuda.set_device(device)
     fb.lib()
     # (no dense counterpart for the multiplicative bias: the comparison kernel adds its bias)
-    w = GpuWorkload(c, device, with_dense=not args.no_dense and c["dtype"] == "bf16" and c["bias"] != "mulcos")
+    w = GpuWorkload(c, device, with_dense=not args.no_dense and c["dtype"] == "bf16"
+                    and c["bias"] not in ("mulcos", "neural"))
     stream = torch.cuda.current_stream(device)
 
     attn_ms = []
@@ -510,7 +530,8 @@ def run_ours(args, rank: int, world: int, local: int):
         "config": config_json(c, "flushed: 256 MiB memset between timed steps (untimed)"),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": round(achieved / peak_tf, 4), "traffic": traffic,
-                     "kernel": "prep_mul_bias + attn_fwd_sm100" if w.mul else "attn_fwd_sm100",
+                     "kernel": ("prep_mul_bias + attn_fwd_sm100" if w.mul else
+                                ("neural_factor + prep + attn_fwd_sm100" if w.neural else "attn_fwd_sm100")),
                      "peak_kind": peak_kind,
                      "kernel_ms": round(kern_ms, 5)},
         "e2e": {"value": round(c["flops"] * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
@@ -550,6 +571,10 @@ def oracle_sample(c: dict, step: int, rows_per_head: int):
     elif c["bias"] == "lowrank":
         pq, pk = si.random_factors((B, H, N, R), c["factor_std"], si.FACTOR_SEED_BASE + c["index"])
         bias = oracle.HeadBias.lowrank(pq[b, h], pk[b, h])
+    elif c["bias"] == "neural":
+        xq, xk, wq, wk = si.neural_inputs(B, H, N, c["F"], R, si.FACTOR_SEED_BASE + c["index"])
+        pq, pk = oracle.neural_factors(xq[b:b + 1], xk[b:b + 1], wq[h:h + 1], wk[h:h + 1])
+        bias = oracle.HeadBias.lowrank(pq[0, 0], pk[0, 0])
     elif c["bias"] == "mulcos":
         f = oracle.cos_factors(N)
         keys = (rows + 1).astype(np.float64) if c["causal"] else np.full(rows.shape, float(N))

@@ -37,6 +37,10 @@ CONFIGS = [
     # multiplicative bias b_ij = cos(i - j) (rank 2) on the GPT-2 shape: a widening case, not a headline
     dict(index=5, name="gpt2_mulcos_N2048", dtype="bf16", B=8, H=12, N=2048, d=64, R=2,
          causal=True, bias="mulcos"),
+    # neural decomposition: factors from per-head linear layers on token features (F = 64) on the
+    # pair-bias shape: a widening case, not a headline
+    dict(index=6, name="af3_neural_F64_R32_N1536_d24", dtype="bf16", B=1, H=16, N=1536, d=24, R=32,
+         causal=False, bias="neural", F=64),
 ]
 
 QKV_SEED_BASE = 1000
@@ -87,6 +91,18 @@ def random_factors(shape, std: float, seed: int):
     pq = g.standard_normal(size=shape, dtype=np.float32) * np.float32(std)
     pk = g.standard_normal(size=shape, dtype=np.float32) * np.float32(std)
     return pq, pk
+
+
+def neural_inputs(B: int, H: int, N: int, F: int, R: int, seed: int):
+    """Token features x_q, x_k ~ N(0, 1) [B, N, F] and linear-layer weights
+    w_q ~ N(0, 1/(F R)), w_k ~ N(0, 1/F) [H, F, R], fp32 (synthetic weights;
+    the bias phi_q phi_k^T then has entries of order 1)."""
+    g = generator(seed)
+    xq = g.standard_normal(size=(B, N, F), dtype=np.float32)
+    xk = g.standard_normal(size=(B, N, F), dtype=np.float32)
+    wq = g.standard_normal(size=(H, F, R), dtype=np.float32) * np.float32(1.0 / math.sqrt(F * R))
+    wk = g.standard_normal(size=(H, F, R), dtype=np.float32) * np.float32(1.0 / math.sqrt(F))
+    return xq, xk, wq, wk
 
 
 # --- vision-style smooth spatial bias (workload 3) -------------------------

@@ -179,3 +179,21 @@ def test_config5_multiplicative_cos_full_size():
     for (b, h) in [(0, 0), (5, 6), (7, 11)]:
         ro, rl = oracle.attention_mul_head(q[b, h], k[b, h], v[b, h], f, f, scale, True, rows)
         compare(og[b, h][rows], lg[b, h][rows], ro, rl, "bf16", f"c5 ({b},{h})")
+
+
+def test_config6_neural_full_size():
+    """The neural-decomposition widening case (bench.py --config 6) at full
+    size: sampled rows of three heads against the oracle."""
+    c = si.CONFIGS[6]
+    B, H, N, d, R, F = c["B"], c["H"], c["N"], c["d"], c["R"], c["F"]
+    q, k, v = si.qkv(B, H, N, d, si.QKV_SEED_BASE + 6, "bf16")
+    xq, xk, wq, wk = si.neural_inputs(B, H, N, F, R, si.FACTOR_SEED_BASE + 6)
+    scale = 1.0 / math.sqrt(d)
+    o, l = fb.attn_neural(dev(q, "bf16"), dev(k, "bf16"), dev(v, "bf16"), dev(xq, "f32"), dev(xk, "f32"),
+                          dev(wq, "f32"), dev(wk, "f32"), scale=scale, causal=False)
+    torch.cuda.synchronize()
+    assert fb.fb_check_device_error(_stream()) == fb.FB_OK
+    pq, pk = oracle.neural_factors(xq, xk, wq, wk)
+    rows = si.sample_rows(N, 40, 6)
+    _check_rows(o, l, q, k, v, [(0, 0), (0, 7), (0, 15)], rows, lambda b, h: HeadBias.lowrank(pq[b, h], pk[b, h]),
+                scale, False, "bf16", "c6")
