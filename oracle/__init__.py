@@ -12,7 +12,10 @@ decomposition with a per-head rank), done with ``numpy.linalg.svd``;
 attention with a multiplicative bias (rebuttal, reply to Reviewer BRmd, Q1
 (2), its Eq. (1): the scaled scores are multiplied elementwise by b); and the
 factors of the neural decomposition (rebuttal, reply to Reviewer xU4x, Q4:
-linear layers on token features), a library matmul.
+linear layers on token features), a library matmul; and the gradients of
+attention with a low-rank bias (the backward of the concatenated form
+q' = [q, phi_q], k' = [k, phi_k], rebuttal, reply to Reviewer UJUf, Q2, used
+for training in Q1 (3) and in the reply to Reviewer Bp2x, Q3).
 """
 from __future__ import annotations
 
@@ -274,3 +277,39 @@ def neural_factors(x_q, x_k, w_q, w_k):
     x_k[b] w_k[h] in fp64. x [B, N, F], w [H, F, R] -> phi [B, H, N, R]."""
     xq, xk, wq, wk = _f64(x_q), _f64(x_k), _f64(w_q), _f64(w_k)
     return np.einsum("bnf,hfr->bhnr", xq, wq), np.einsum("bnf,hfr->bhnr", xk, wk)
+
+
+def attention_lowrank_bwd_head(q, k, v, phi_q, phi_k, do, scale: float, causal: bool):
+    """Gradients of one head of O = softmax(scale q k^T + phi_q phi_k^T [causal]) v
+    for an upstream gradient dO, in fp64 (the chain rule through the softmax,
+    whole rows at once; library matmuls).
+
+    The pages train with the factorised bias by concatenating the factors to
+    the queries and keys (rebuttal, reply to Reviewer UJUf, Q2 and Q1 (3);
+    reply to Reviewer Bp2x, Q3), so the factor gradients are the extra columns
+    of the concatenated query and key gradients:
+        P = softmax(s) row-wise over the visible keys, O = P v
+        dV = P^T dO,  dP = dO v^T,  dS = P * (dP - rowsum(P * dP))
+        dq = scale dS k,  dk = scale dS^T q,  dphi_q = dS phi_k,  dphi_k = dS^T phi_q.
+    q, k, v, do [N, d]; phi_q, phi_k [N, R]. Returns a dict with dq, dk, dv,
+    dphi_q, dphi_k and the intermediate rowsum(P * dP) as ``delta``."""
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    pq, pk = _f64(phi_q), _f64(phi_k)
+    N = q.shape[0]
+    s = float(scale) * (q @ k.T) + pq @ pk.T
+    if causal:
+        s = np.where(np.arange(N)[None, :] <= np.arange(N)[:, None], s, -np.inf)
+    m = np.max(s, axis=1, keepdims=True)
+    e = np.exp(s - m)
+    p = e / np.sum(e, axis=1, keepdims=True)
+    dp = do @ v.T
+    delta = np.sum(p * dp, axis=1, keepdims=True)
+    ds = p * (dp - delta)
+    return {
+        "dq": float(scale) * (ds @ k),
+        "dk": float(scale) * (ds.T @ q),
+        "dv": p.T @ do,
+        "dphi_q": ds @ pk,
+        "dphi_k": ds.T @ pq,
+        "delta": delta[:, 0],
+    }

@@ -6,7 +6,10 @@
   one, key permutation, saturating scores, the first causal row);
 - the closed-form identities the pages state (Sandwich bias = product of its
   exact factors; ALiBi = product of its rank-2 factors) and golden constants;
-- the truncated SVD against matrices with known singular values.
+- the truncated SVD against matrices with known singular values;
+- the backward against central finite differences of the forward (the C
+  definition), and the invariants that rows of dS sum to zero and rows of P
+  to one.
 """
 import json
 import math
@@ -352,3 +355,56 @@ def test_neural_factors_are_the_linear_layers():
                 for r in range(R):
                     assert abs(pq[b, h, n, r] - sum(xq[b, n, f] * wq[h, f, r] for f in range(F))) < 1e-12
                     assert abs(pk[b, h, n, r] - sum(xk[b, n, f] * wk[h, f, r] for f in range(F))) < 1e-12
+
+
+def _fd_loss(q, k, v, pq, pk, g, scale, causal):
+    o, _ = oracle.attention_head(q, k, v, HeadBias.lowrank(pq, pk), scale, causal)
+    return float(np.sum(o * g))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_matches_finite_differences(causal):
+    """Every gradient against a central difference of the forward definition
+    (the C oracle, not the numpy backward): a dropped term, a transposed
+    operand or a wrong scale in any of the five gradients fails here."""
+    N, d, R = 6, 3, 2
+    q, k, v = (_rand((N, d), s) for s in (41, 42, 43))
+    pq, pk = _rand((N, R), 44, 0.8), _rand((N, R), 45, 0.8)
+    g = _rand((N, d), 46)
+    scale = 0.7
+    grads = oracle.attention_lowrank_bwd_head(q, k, v, pq, pk, g, scale, causal)
+    args = {"dq": q, "dk": k, "dv": v, "dphi_q": pq, "dphi_k": pk}
+    h = 1e-6
+    for name, x in args.items():
+        fd = np.empty_like(x)
+        for idx in np.ndindex(x.shape):
+            x0 = x[idx]
+            x[idx] = x0 + h
+            up = _fd_loss(q, k, v, pq, pk, g, scale, causal)
+            x[idx] = x0 - h
+            dn = _fd_loss(q, k, v, pq, pk, g, scale, causal)
+            x[idx] = x0
+            fd[idx] = (up - dn) / (2 * h)
+        np.testing.assert_allclose(grads[name], fd, rtol=0, atol=2e-8, err_msg=name)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_invariants(causal):
+    """Rows of dS sum to zero (the softmax is invariant to a per-row shift),
+    so the key and phi_k gradients sum to zero over the keys and a constant
+    phi_k column gets a zero phi_q gradient; rows of P sum to one, so the
+    value gradients sum to the sum of dO."""
+    N, d, R = 40, 8, 4
+    q, k, v = (_rand((N, d), s) for s in (51, 52, 53))
+    pq, pk = _rand((N, R), 54), _rand((N, R), 55)
+    pk[:, 2] = 1.5
+    g = _rand((N, d), 56)
+    out = oracle.attention_lowrank_bwd_head(q, k, v, pq, pk, g, 0.35, causal)
+    np.testing.assert_allclose(out["dk"].sum(axis=0), 0.0, atol=1e-12)
+    np.testing.assert_allclose(out["dphi_k"].sum(axis=0), 0.0, atol=1e-12)
+    np.testing.assert_allclose(out["dphi_q"][:, 2], 0.0, atol=1e-12)
+    np.testing.assert_allclose(out["dv"].sum(axis=0), g.sum(axis=0), atol=1e-12)
+    o, _ = oracle.attention_head(q, k, v, HeadBias.lowrank(pq, pk), 0.35, causal)
+    np.testing.assert_allclose(out["delta"], np.sum(o * g, axis=1), atol=1e-12)
+    if causal:  # the first query sees only key 0: its dS row is zero
+        np.testing.assert_allclose(out["dq"][0], 0.0, atol=1e-15)
