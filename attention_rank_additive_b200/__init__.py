@@ -41,7 +41,8 @@ EXPORTED = (
     "fb_factors_sandwich", "fb_factors_alibi", "fb_svd_factors_host", "fb_check_device_error",
     "fb_selftest_wait_timeout", "fb_attn_fwd_noalloc", "fb_attn_prepare_factors", "fb_attn_fwd_prepared",
     "fb_attn_mul_bias_workspace_bytes", "fb_attn_mul_bias_fwd", "fb_svd_device_workspace_bytes",
-    "fb_svd_factors_device", "fb_attn_neural_workspace_bytes", "fb_attn_neural_fwd",
+    "fb_svd_factors_device", "fb_attn_neural_workspace_bytes", "fb_attn_neural_fwd", "fb_attn_bwd_workspace_bytes",
+    "fb_attn_bwd",
 )
 
 
@@ -92,6 +93,11 @@ def lib() -> ctypes.CDLL:
         L.fb_attn_neural_fwd.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, i32, i32, vp, vp, vp, vp, f32, i32, vp,
                                          vp, vp, sz, vp]
         L.fb_attn_neural_fwd.restype = i32
+        L.fb_attn_bwd_workspace_bytes.argtypes = [i32, i32, i32, i32, i64, i64]
+        L.fb_attn_bwd_workspace_bytes.restype = sz
+        L.fb_attn_bwd.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, i32, vp, vp, i64, i64, f32, i32, vp, vp, vp,
+                                  vp, vp, vp, vp, vp, vp, sz, vp]
+        L.fb_attn_bwd.restype = i32
         L.fb_attn_dense_bias_fwd.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, i64, i64, f32, i32, vp, vp, vp]
         L.fb_attn_dense_bias_fwd.restype = i32
         L.fb_factors_sandwich.argtypes, L.fb_factors_sandwich.restype = [i32, i32, vp, vp, vp], i32
@@ -212,6 +218,48 @@ def attn_neural(q, k, v, x_q, x_k, w_q, w_k, scale=None, causal=False, out=None,
                               x_k.data_ptr(), w_q.data_ptr(), w_k.data_ptr(), scale, int(bool(causal)), o.data_ptr(),
                               l.data_ptr(), ws.data_ptr(), nb, _stream(q.device)), "fb_attn_neural_fwd")
     return o, l
+
+
+def fb_attn_bwd_workspace_bytes(B, H, N, R, phi_bstride, phi_hstride) -> int:
+    return lib().fb_attn_bwd_workspace_bytes(B, H, N, R, phi_bstride, phi_hstride)
+
+
+def fb_attn_bwd(dt, B, H, N, d, Q, K, V, R, phi_q, phi_k, phi_bstride, phi_hstride, scale, causal, O, LSE, dO,
+                dQ, dK, dV, dphi_q, dphi_k, workspace, workspace_bytes, stream) -> int:
+    return lib().fb_attn_bwd(dt, B, H, N, d, Q, K, V, R, phi_q, phi_k, phi_bstride, phi_hstride, scale, causal, O,
+                             LSE, dO, dQ, dK, dV, dphi_q, dphi_k, workspace, workspace_bytes, stream)
+
+
+def attn_bwd(q, k, v, phi_q, phi_k, o, lse, do, scale=None, causal=False, workspace=None):
+    """Gradients of attn's O for an upstream gradient do (fb_attn_bwd).
+
+    q, k, v, o, do: bf16 CUDA [B, H, N, d] contiguous; lse: fp32 [B, H, N]
+    from the forward; phi_q, phi_k as for attn (or None). Returns
+    (dq, dk, dv, dphi_q, dphi_k): bf16 [B, H, N, d] and fp32 gradients shaped
+    like phi_q, phi_k (None without factors)."""
+    import torch
+    for t in (q, k, v, o, do):
+        assert t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()
+    B, H, N, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    R, bs, hs, pq, pk, gq, gk = 0, 0, 0, 0, 0, 0, 0
+    dpq = dpk = None
+    if phi_q is not None:
+        assert phi_q.dtype == torch.float32 and phi_k.dtype == torch.float32
+        assert phi_q.shape == phi_k.shape and phi_q.stride() == phi_k.stride() and phi_q.is_contiguous()
+        R = phi_q.shape[-1]
+        bs, hs = _factor_strides(phi_q, B, H, N, R)
+        pq, pk = phi_q.data_ptr(), phi_k.data_ptr()
+        dpq, dpk = torch.empty_like(phi_q), torch.empty_like(phi_k)
+        gq, gk = dpq.data_ptr(), dpk.data_ptr()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    nb = fb_attn_bwd_workspace_bytes(B, H, N, R, bs, hs)
+    if workspace is None:
+        workspace = torch.empty(max(nb, 1), device=q.device, dtype=torch.uint8)
+    _check(fb_attn_bwd(FB_BF16, B, H, N, d, q.data_ptr(), k.data_ptr(), v.data_ptr(), R, pq, pk, bs, hs, scale,
+                       int(bool(causal)), o.data_ptr(), lse.data_ptr(), do.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                       dv.data_ptr(), gq, gk, workspace.data_ptr(), nb, _stream(q.device)), "fb_attn_bwd")
+    return dq, dk, dv, dpq, dpk
 
 
 def fb_attn_fwd_noalloc(dt, B, H, N, d, Q, K, V, R, phi_q, phi_k, phi_bstride, phi_hstride, scale, causal, O, LSE,

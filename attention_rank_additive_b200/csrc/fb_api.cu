@@ -493,6 +493,141 @@ int fb_factors_alibi(int H, int N, float *phi_q, float *phi_k, void *stream) {
   return launch_alibi(H, N, phi_q, phi_k, static_cast<cudaStream_t>(stream)) == cudaSuccess ? FB_OK : FB_ERR_CUDA;
 }
 
+namespace {
+struct BwdLayout {
+  WsLayout f;  // the S-side factor tiles (as the forward's workspace)
+  size_t gq_off, gk_off, l_off, d_off, total;
+  int RG, Npad;
+};
+size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
+BwdLayout bwd_layout(int B, int H, int N, int R, int64_t bs, int64_t hs) {
+  BwdLayout w{};
+  w.f = workspace_layout(B, H, N, R, bs, hs);
+  w.RG = R == 0 ? 0 : (R <= 4 ? 16 : pad_rank(R));
+  w.Npad = int(((long long)N + 127) / 128 * 128);
+  const size_t fb = size_t(bs == 0 ? 1 : B) * size_t(hs == 0 ? 1 : H);
+  const size_t g = al256(fb * size_t(N) * size_t(w.RG) * 2);
+  const size_t rows = al256(size_t(B) * H * size_t(w.Npad) * 4);
+  w.gq_off = w.f.total;
+  w.gk_off = w.gq_off + g;
+  w.l_off = w.gk_off + g;
+  w.d_off = w.l_off + rows;
+  w.total = w.d_off + rows;
+  return w;
+}
+bool encode_rows_bf16(CUtensorMap *m, const void *ptr, int slices, int N, int cols, int width, int rows) {
+  const int ch = width > 64 ? 64 : width;
+  const uint64_t dims[3] = {uint64_t(cols), uint64_t(N), uint64_t(slices)};
+  const uint64_t strides[2] = {uint64_t(cols) * 2, uint64_t(N) * cols * 2};
+  const uint32_t box[3] = {uint32_t(ch), uint32_t(rows), 1u};
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, ptr, dims, strides, box, swizzle_for(ch * 2));
+}
+bool encode_fac(CUtensorMap *m, int mode, const void *ptr, int FB, int N, int RP, int rows) {
+  const uint64_t dims[3] = {uint64_t(RP), uint64_t(N), uint64_t(FB)};
+  if (mode == kBiasMma) {
+    const int ch = RP > 64 ? 64 : RP;
+    const uint64_t strides[2] = {uint64_t(RP) * 2, uint64_t(N) * RP * 2};
+    const uint32_t box[3] = {uint32_t(ch), uint32_t(rows), 1u};
+    return encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, ptr, dims, strides, box, swizzle_for(ch * 2));
+  }
+  const uint64_t strides[2] = {uint64_t(RP) * 4, uint64_t(N) * RP * 4};
+  const uint32_t box[3] = {uint32_t(RP), uint32_t(rows), 1u};
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box, swizzle_for(RP * 4));
+}
+}  // namespace
+
+size_t fb_attn_bwd_workspace_bytes(int B, int H, int N, int R, int64_t phi_bstride, int64_t phi_hstride) {
+  if (B < 1 || H < 1 || N < 1 || R < 0 || R > 128 || phi_bstride < 0 || phi_hstride < 0) return 0;
+  if (!valid_shape_bf16(B, H, N, 16)) return 0;
+  return bwd_layout(B, H, N, R, phi_bstride, phi_hstride).total;
+}
+
+int fb_attn_bwd(int dt, int B, int H, int N, int d, const void *Q, const void *K, const void *V, int R,
+                const float *phi_q, const float *phi_k, int64_t phi_bstride, int64_t phi_hstride, float scale,
+                int causal, const void *O, const float *LSE, const void *dO, void *dQ, void *dK, void *dV,
+                float *dphi_q, float *dphi_k, void *workspace, size_t workspace_bytes, void *stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!Q || !K || !V || !O || !LSE || !dO || !dQ || !dK || !dV) return FB_ERR_INVALID_ARG;
+  if (dt != FB_BF16) return FB_ERR_UNSUPPORTED;
+  if (R < 0 || R > 128) return FB_ERR_UNSUPPORTED;
+  if (R > 0 && (!phi_q || !phi_k || !dphi_q || !dphi_k || phi_bstride < 0 || phi_hstride < 0))
+    return FB_ERR_INVALID_ARG;
+  if (R > 0 && (((reinterpret_cast<uintptr_t>(phi_q) | reinterpret_cast<uintptr_t>(phi_k) |
+                  reinterpret_cast<uintptr_t>(dphi_q) | reinterpret_cast<uintptr_t>(dphi_k)) &
+                 3u) != 0))
+    return FB_ERR_INVALID_ARG;
+  if (!valid_scale(scale)) return FB_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) || !aligned16(dQ) ||
+      !aligned16(dK) || !aligned16(dV) || !aligned16(LSE))
+    return FB_ERR_INVALID_ARG;
+  if (!valid_shape_bf16(B, H, N, d)) return FB_ERR_UNSUPPORTED;
+  const BwdLayout L = bwd_layout(B, H, N, R, phi_bstride, phi_hstride);
+  if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return FB_ERR_WORKSPACE;
+  BwdPlan plan;
+  plan.DP = pad_dim(d);
+  plan.mode = R == 0 ? kBiasNone : (R <= 4 ? kBiasTf32 : kBiasMma);
+  plan.RP = plan.mode == kBiasMma ? pad_rank(R) : (plan.mode == kBiasTf32 ? tf32_cols(R) : 0);
+  plan.RG = L.RG;
+  const int BQ = bwd_query_block_rows(plan);
+  if (BQ == 0) return FB_ERR_UNSUPPORTED;
+  int *flags = device_flags();
+  if (!flags) return FB_ERR_CUDA;
+
+  uint8_t *wsb = static_cast<uint8_t *>(workspace);
+  const int fac_B = phi_bstride == 0 ? 1 : B, fac_H = phi_hstride == 0 ? 1 : H;
+  const int FB = fac_B * fac_H;
+  const int BH = B * H;
+  // 1. the forward's factor tiles (S is recomputed as the forward computed it)
+  if (R > 0) {
+    const int rc = fb_attn_prepare_factors(B, H, N, R, phi_q, phi_k, phi_bstride, phi_hstride, scale, workspace,
+                                           workspace_bytes, stream);
+    if (rc != FB_OK) return rc;
+    // 2. bf16 factor copies for the gradient products; zeroed factor gradients
+    if (launch_prep_grad_factors(N, R, L.RG, phi_q, phi_k, phi_bstride, phi_hstride, fac_B, fac_H, wsb + L.gq_off,
+                                 wsb + L.gk_off, dphi_q, dphi_k, st) != cudaSuccess)
+      return FB_ERR_CUDA;
+  }
+  // 3. per-row LSE in log2 units and rowsum(dO * O)
+  float *lse2 = reinterpret_cast<float *>(wsb + L.l_off);
+  float *delta = reinterpret_cast<float *>(wsb + L.d_off);
+  if (launch_bwd_rows(BH, N, L.Npad, d, O, dO, LSE, lse2, delta, st) != cudaSuccess) return FB_ERR_CUDA;
+
+  // 4. the two gradient kernels
+  BwdMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  const int DP = plan.DP;
+  if (!encode_rows_bf16(&maps.q, Q, BH, N, d, DP, 128) || !encode_rows_bf16(&maps.k, K, BH, N, d, DP, 128) ||
+      !encode_rows_bf16(&maps.v, V, BH, N, d, DP, 128) || !encode_rows_bf16(&maps.dO, dO, BH, N, d, DP, 128) ||
+      !encode_rows_bf16(&maps.q_blk, Q, BH, N, d, DP, BQ) || !encode_rows_bf16(&maps.do_blk, dO, BH, N, d, DP, BQ))
+    return FB_ERR_CUDA;
+  if (R > 0) {
+    void *wq = wsb + L.f.q_off, *wk = wsb + L.f.k_off;
+    if (!encode_fac(&maps.fq, plan.mode, wq, FB, N, plan.RP, 128) ||
+        !encode_fac(&maps.fk, plan.mode, wk, FB, N, plan.RP, 128) ||
+        !encode_fac(&maps.fq_blk, plan.mode, wq, FB, N, plan.RP, BQ) ||
+        !encode_rows_bf16(&maps.gq_blk, wsb + L.gq_off, FB, N, L.RG, L.RG, BQ) ||
+        !encode_rows_bf16(&maps.gk, wsb + L.gk_off, FB, N, L.RG, L.RG, 128))
+      return FB_ERR_CUDA;
+  }
+  BwdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.B = B, a.H = H, a.N = N, a.d = d, a.R = R;
+  a.n_kv = (N + 127) / 128;
+  a.Npad = L.Npad;
+  a.scale = scale;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.causal = causal ? 1 : 0;
+  a.lse2 = lse2;
+  a.delta = delta;
+  a.dQ = dQ, a.dK = dK, a.dV = dV;
+  a.dphi_q = dphi_q, a.dphi_k = dphi_k;
+  a.phi_bs = phi_bstride, a.phi_hs = phi_hstride;
+  a.fac_B = fac_B, a.fac_H = fac_H;
+  a.flags = flags;
+  return bwd_launch(plan, maps, a, st) == cudaSuccess ? FB_OK : FB_ERR_CUDA;
+}
+
 int fb_check_device_error(void *stream) {
   int *flags = device_flags();
   if (!flags) return FB_ERR_CUDA;

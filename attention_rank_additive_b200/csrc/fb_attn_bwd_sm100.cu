@@ -1,0 +1,770 @@
+// fb_attn_bwd_sm100.cu -- backward of attention with a low-rank additive bias
+// on B200 (sm_100a): TMA -> shared memory -> tcgen05 MMA -> TMEM -> CUDA cores
+// -> tcgen05 MMA (A operand from TMEM) -> TMEM -> HBM.
+//
+// Method: FlashBias (arXiv 2505.12044) trains by concatenating the factors to
+// the queries and keys, q' = [q, phi_q], k' = [k, phi_k] (rebuttal, reply to
+// Reviewer UJUf, Q2 and the training speedup of Q1 (3); reply to Reviewer
+// Bp2x, Q3), so the backward is the attention backward of the concatenated
+// operands and the factor gradients are the extra columns of dq' and dk':
+//   P = exp(s - LSE), dP = dO V^T, dS = P * (dP - D) with D = rowsum(dO * O),
+//   dV = P^T dO, dK = scale dS^T Q, dphi_k = dS^T phi_q,
+//   dQ = scale dS K, dphi_q = dS phi_k.
+// S is recomputed exactly as the forward computes it (bf16 QK^T plus the
+// fp16 or tf32 factor MMA into one fp32 accumulator), so P matches the
+// forward's P; the gradient products run in bf16 with fp32 accumulation, the
+// factors entering them as bf16 copies.
+//
+// Two kernels, neither with atomics on the bf16 outputs:
+//   attn_bwd_dkdv_sm100  one CTA per (b, h, 128-key tile). The key tile K|phi_k
+//       and V stay in shared memory; query blocks of BQ rows (128, or 64 at
+//       head dim 128 so that TMEM holds everything) stream through a ring.
+//       Per block: S^T = K Q^T (+ phi_k' phi_q'^T), dP^T = V dO^T; the CUDA
+//       cores turn them into P^T and dS^T (bf16, written back over S^T and
+//       dP^T in TMEM); then dV += P^T dO, dK += dS^T Q, dphi_k += dS^T phi_q
+//       with the A operand read from TMEM and dO, Q, phi_q as MN-major B.
+//   attn_bwd_dq_sm100    one CTA per (b, h, 128-query tile): S = Q K^T (+ ...),
+//       dP = dO V^T, dS over S in TMEM, dQ += dS K, dphi_q += dS phi_k.
+// The factor gradients of a broadcast factor (stride 0) sum over the heads
+// and batches sharing it, so they are accumulated with fp32 reductions into
+// a buffer zeroed by the preparation step.
+//
+// CTA: warps 0-3 compute (one thread per TMEM lane = tile row), warp 4 TMA
+// producer, warp 5 TMEM allocator and MMA issuer. Every wait is bounded (the
+// abort flag and the device flag word report a timeout).
+#include <algorithm>
+#include <atomic>
+
+#include "fb_internal.h"
+#include "fb_ptx.cuh"
+
+namespace fb {
+namespace {
+
+constexpr uint32_t kSmemLimitB = 227u * 1024u;
+
+// Bulk copy (no tensor map) of `bytes` (multiple of 16, both addresses
+// 16-byte aligned) into shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_load_leader(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
+                                                 uint32_t leader) {
+  asm volatile(
+      "{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %3, 0;\n\t"
+      "@q cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%4];\n\t}" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(leader), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// K-major tile of ROWS rows x (NCH * CH) 16-bit units stored as NCH swizzled
+// chunks of CH units: descriptor of the base and offset (>> 4) of K-step kk
+// (32 bytes of a row).
+template <int CH>
+__device__ __forceinline__ uint64_t kdesc(uint32_t base) {
+  return make_smem_desc(base, 16, 8 * CH * 2, swizzle_code(CH * 2));
+}
+template <int CH, int ROWS>
+__host__ __device__ constexpr uint32_t kstep(int kk) {
+  return uint32_t((kk / (CH / 16)) * (ROWS * CH * 2) + (kk % (CH / 16)) * 32) >> 4;
+}
+// The same tile read as an MN-major B operand (rows = the MMA's K dimension,
+// columns = N): chunk stride as leading offset, 8 rows as stride offset;
+// offset of the 16-row step kk.
+template <int CH, int ROWS>
+__device__ __forceinline__ uint64_t mndesc(uint32_t base) {
+  return make_smem_desc(base, ROWS * CH * 2, 8 * CH * 2, swizzle_code(CH * 2));
+}
+template <int CH>
+__host__ __device__ constexpr uint32_t mnstep(int kk) {
+  return uint32_t(kk * 16 * CH * 2) >> 4;
+}
+
+}  // namespace
+
+template <int DP, int RP, int MODE, int RG>
+struct BwdCfg {
+  // Streamed block of the dK/dV kernel: 128 queries, or 64 at head dim 128
+  // (TMEM: S^T and dP^T BQ columns each, dV and dK DP each, dphi_k RG).
+  static constexpr int BQ = DP == 128 ? 64 : 128;
+  static constexpr int DCH = DP > 64 ? 64 : DP;
+  static constexpr int NDCH = DP / DCH;
+  static constexpr bool FAC = MODE == kBiasMma || MODE == kBiasTf32;
+  // S-side factor tile: fp16 [rows x RP] or fp32 [rows x RP] (tf32); width in
+  // 16-bit units of one chunk (tf32 rows are one chunk of RP floats).
+  static constexpr int FCH = MODE == kBiasMma ? (RP > 64 ? 64 : RP) : (MODE == kBiasTf32 ? 2 * RP : 16);
+  static constexpr int NFCH = MODE == kBiasMma ? RP / FCH : (MODE == kBiasTf32 ? 1 : 0);
+  static constexpr int FESZ = MODE == kBiasTf32 ? 4 : 2;
+  // bf16 gradient factor tile [rows x RG].
+  static constexpr int GCH = RG > 64 ? 64 : (RG > 0 ? RG : 16);
+  static constexpr int NGCH = RG > 0 ? RG / GCH : 0;
+  static constexpr uint32_t align1k(uint32_t x) { return (x + 1023u) & ~1023u; }
+  // dK/dV kernel
+  static constexpr uint32_t KV_FIXED = 2u * 128u * DP * 2u + (FAC ? 128u * RP * FESZ : 0u);
+  static constexpr uint32_t KV_STAGE =
+      align1k(2u * BQ * DP * 2u + (FAC ? BQ * RP * FESZ : 0u) + BQ * RG * 2u + 2u * BQ * 4u);
+  static constexpr uint32_t CTRL = 1024;
+  static constexpr uint32_t SLACK = 1024;
+  static constexpr int KV_KS_FIT =
+      kSmemLimitB > KV_FIXED + CTRL + SLACK ? int((kSmemLimitB - KV_FIXED - CTRL - SLACK) / KV_STAGE) : 0;
+  static constexpr int KV_KS = KV_KS_FIT > 2 ? 2 : KV_KS_FIT;
+  static constexpr uint32_t KV_SMEM = KV_FIXED + uint32_t(KV_KS) * KV_STAGE + CTRL + SLACK;
+  // dQ kernel
+  static constexpr uint32_t DQ_FIXED = 2u * 128u * DP * 2u + (FAC ? 128u * RP * FESZ : 0u);
+  static constexpr uint32_t DQ_STAGE_BYTES = 2u * 128u * DP * 2u + (FAC ? 128u * RP * FESZ : 0u) + 128u * RG * 2u;
+  static constexpr uint32_t DQ_STAGE = align1k(DQ_STAGE_BYTES);
+  static constexpr int DQ_KS_FIT =
+      kSmemLimitB > DQ_FIXED + CTRL + SLACK ? int((kSmemLimitB - DQ_FIXED - CTRL - SLACK) / DQ_STAGE) : 0;
+  static constexpr int DQ_KS = DQ_KS_FIT > 2 ? 2 : DQ_KS_FIT;
+  static constexpr uint32_t DQ_SMEM = DQ_FIXED + uint32_t(DQ_KS) * DQ_STAGE + CTRL + SLACK;
+  static constexpr int THREADS = 192;
+  static constexpr int PRODUCER_WARP = 4;
+  static constexpr int MMA_WARP = 5;
+  static constexpr uint32_t TMEM_COLS = 512;
+  // TMEM columns, dK/dV kernel
+  static constexpr uint32_t KV_S = 0, KV_DP = BQ, KV_DV = 2 * BQ, KV_DK = 2 * BQ + DP, KV_DF = 2 * BQ + 2 * DP;
+  static_assert(KV_DF + RG <= TMEM_COLS, "dK/dV TMEM layout");
+  // TMEM columns, dQ kernel
+  static constexpr uint32_t DQ_S = 0, DQ_DP = 128, DQ_DQ = 256, DQ_DF = 256 + DP;
+  static_assert(DQ_DF + RG <= TMEM_COLS, "dQ TMEM layout");
+  static constexpr uint32_t IDESC_KV_S = make_idesc_f16(true, true, 128, BQ, false);
+  static constexpr uint32_t IDESC_KV_F =
+      MODE == kBiasTf32 ? make_idesc_tf32(128, BQ) : make_idesc_f16(false, false, 128, BQ, false);
+  static constexpr uint32_t IDESC_DQ_S = make_idesc_f16(true, true, 128, 128, false);
+  static constexpr uint32_t IDESC_DQ_F =
+      MODE == kBiasTf32 ? make_idesc_tf32(128, 128) : make_idesc_f16(false, false, 128, 128, false);
+  static constexpr uint32_t IDESC_GD = make_idesc_f16(true, true, 128, DP, true);
+  static constexpr uint32_t IDESC_GR = make_idesc_f16(true, true, 128, RG > 0 ? RG : 16, true);
+};
+
+namespace {
+
+struct BwdCtrl {
+  uint64_t fixed_full;
+  uint64_t full[2], empty[2];
+  uint64_t s_full, p_full, acc_done;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(BwdCtrl) <= 1024, "control block too large");
+
+// fp32 -> bf16 pairs of a TMEM row segment, scaled, stored to a global row
+// (columns [c0, c0 + 16) of which those below d are written).
+__device__ __forceinline__ void store_row16_bf16(const uint32_t *r, float mul, uint16_t *row, int c0, int d) {
+  uint32_t w[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * mul, __uint_as_float(r[2 * e + 1]) * mul);
+  if (c0 + 8 <= d) *reinterpret_cast<uint4 *>(row + c0) = make_uint4(w[0], w[1], w[2], w[3]);
+  if (c0 + 16 <= d) *reinterpret_cast<uint4 *>(row + c0 + 8) = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
+}  // namespace
+
+// ------------------------------------------------------------ dK, dV, dphi_k
+template <int DP, int RP, int MODE, int RG>
+__global__ void __launch_bounds__(192, 1)
+    attn_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                        const __grid_constant__ CUtensorMap tm_fk, const __grid_constant__ CUtensorMap tm_q,
+                        const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_fq,
+                        const __grid_constant__ CUtensorMap tm_gq, const BwdArgs args) {
+  using C = BwdCfg<DP, RP, MODE, RG>;
+  constexpr int KS = C::KV_KS;
+  constexpr int BQ = C::BQ;
+  static_assert(KS >= 1, "configuration does not fit in shared memory");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sK = smem;                                  // 128 x DP bf16
+  uint8_t *sV = sK + 128 * DP * 2;                     // 128 x DP bf16
+  uint8_t *sFK = sV + 128 * DP * 2;                    // 128 x RP (fp16 / fp32)
+  uint8_t *sStage = smem + C::KV_FIXED;                // KS x KV_STAGE
+  BwdCtrl *ctrl = reinterpret_cast<BwdCtrl *>(sStage + KS * C::KV_STAGE);
+  // offsets inside a stage
+  constexpr uint32_t O_Q = 0, O_DO = BQ * DP * 2, O_FQ = 2 * BQ * DP * 2;
+  constexpr uint32_t O_GQ = O_FQ + (C::FAC ? BQ * RP * C::FESZ : 0);
+  constexpr uint32_t O_L = O_GQ + BQ * RG * 2, O_D = O_L + BQ * 4;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int BH = args.B * args.H;
+  const int kb = int(blockIdx.x) / BH;  // key tile; the heaviest causal tiles come first
+  const int bh = int(blockIdx.x) % BH;
+  const int b = bh / args.H, h = bh % args.H;
+  const int k0 = kb * 128;
+  const int fslice = (args.fac_B > 1 ? b : 0) * args.fac_H + (args.fac_H > 1 ? h : 0);
+  const int n_blk = (args.N + BQ - 1) / BQ;
+  const int j0 = args.causal ? k0 / BQ : 0;  // query blocks before the diagonal see none of these keys
+
+  if (threadIdx.x == 0) {
+    mbar_init(&ctrl->fixed_full, 1);
+    for (int s = 0; s < KS; ++s) {
+      mbar_init(&ctrl->full[s], 1);
+      mbar_init(&ctrl->empty[s], 1);
+    }
+    mbar_init(&ctrl->s_full, 1);
+    mbar_init(&ctrl->p_full, 128);
+    mbar_init(&ctrl->acc_done, 1);
+    ctrl->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(&ctrl->tmem_base, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctrl->tmem_base;
+  volatile int *abort = &ctrl->abort;
+  const uint32_t leader = lane == 0 ? 1u : 0u;
+
+  if (warp == C::PRODUCER_WARP) {
+    // ------------------------------------------------------------ producer
+    if (leader) {
+      tma_prefetch_map(&tm_k);
+      tma_prefetch_map(&tm_v);
+      tma_prefetch_map(&tm_q);
+      tma_prefetch_map(&tm_do);
+      if (C::FAC) {
+        tma_prefetch_map(&tm_fk);
+        tma_prefetch_map(&tm_fq);
+      }
+      if (RG > 0) tma_prefetch_map(&tm_gq);
+    }
+    mbar_arrive_expect_tx_leader(&ctrl->fixed_full, C::KV_FIXED, leader);
+    for (int ch = 0; ch < C::NDCH; ++ch) {
+      tma_load_3d_leader(sK + ch * (128 * C::DCH * 2), &tm_k, &ctrl->fixed_full, ch * C::DCH, k0, bh, leader);
+      tma_load_3d_leader(sV + ch * (128 * C::DCH * 2), &tm_v, &ctrl->fixed_full, ch * C::DCH, k0, bh, leader);
+    }
+    if (C::FAC)
+      for (int ch = 0; ch < C::NFCH; ++ch)
+        tma_load_3d_leader(sFK + ch * (128 * C::FCH * 2), &tm_fk, &ctrl->fixed_full, ch * C::FCH, k0, fslice,
+                           leader);
+    bool ok = true;
+    int it = 0;
+    for (int j = j0; j < n_blk; ++j, ++it) {
+      const int s = it % KS;
+      const uint32_t ph = uint32_t(it / KS) & 1u;
+      if (it >= KS && !(ok = mbar_wait(&ctrl->empty[s], ph ^ 1u, abort))) break;
+      uint8_t *st = sStage + s * C::KV_STAGE;
+      const int q0 = j * BQ;
+      mbar_arrive_expect_tx_leader(&ctrl->full[s], O_D + BQ * 4, leader);
+      for (int ch = 0; ch < C::NDCH; ++ch) {
+        tma_load_3d_leader(st + O_Q + ch * (BQ * C::DCH * 2), &tm_q, &ctrl->full[s], ch * C::DCH, q0, bh, leader);
+        tma_load_3d_leader(st + O_DO + ch * (BQ * C::DCH * 2), &tm_do, &ctrl->full[s], ch * C::DCH, q0, bh, leader);
+      }
+      if (C::FAC)
+        for (int ch = 0; ch < C::NFCH; ++ch)
+          tma_load_3d_leader(st + O_FQ + ch * (BQ * C::FCH * 2), &tm_fq, &ctrl->full[s], ch * C::FCH, q0, fslice,
+                             leader);
+      for (int ch = 0; ch < C::NGCH; ++ch)
+        tma_load_3d_leader(st + O_GQ + ch * (BQ * C::GCH * 2), &tm_gq, &ctrl->full[s], ch * C::GCH, q0, fslice,
+                           leader);
+      const size_t roff = size_t(bh) * args.Npad + q0;
+      bulk_load_leader(st + O_L, args.lse2 + roff, BQ * 4, &ctrl->full[s], leader);
+      bulk_load_leader(st + O_D, args.delta + roff, BQ * 4, &ctrl->full[s], leader);
+    }
+    if (!ok) {
+      // Aborted: let the copies already issued land before the CTA exits.
+      mbar_wait_for(&ctrl->fixed_full, 0, 100000000ull);
+      for (int s = 0; s < KS; ++s) {
+        mbar_wait_for(&ctrl->full[s], 0, 100000000ull);
+        mbar_wait_for(&ctrl->full[s], 1, 100000000ull);
+      }
+      if (leader) atomicOr(args.flags, kFlagTimeout);
+    }
+  } else if (warp == C::MMA_WARP) {
+    // ---------------------------------------------------------- MMA issuer
+    const uint32_t tm_u = __shfl_sync(0xffffffffu, tmem, 0);
+    bool ok = __all_sync(0xffffffffu, mbar_wait(&ctrl->fixed_full, 0, abort));  // warp-uniform for elect.sync
+    tc_fence_after();
+    const uint64_t dK = kdesc<C::DCH>(smem_u32(sK));
+    const uint64_t dV = kdesc<C::DCH>(smem_u32(sV));
+    const uint64_t dFK = kdesc<C::FCH>(smem_u32(sFK));
+    int it = 0;
+    for (int j = j0; j < n_blk && ok; ++j, ++it) {
+      const int s = it % KS;
+      const uint32_t ph = uint32_t(it / KS) & 1u;
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&ctrl->full[s], ph, abort)))) break;
+      tc_fence_after();
+      const uint32_t st = smem_u32(sStage + s * C::KV_STAGE);
+      // S^T = K Q^T (+ phi_k' phi_q'^T), dP^T = V dO^T
+      {
+        uint64_t dq = kdesc<C::DCH>(st + O_Q), ddo = kdesc<C::DCH>(st + O_DO);
+        asm volatile("" : "+l"(dq), "+l"(ddo));
+#pragma unroll
+        for (int kk = 0; kk < DP / 16; ++kk)
+          mma_ss_elect(tm_u + C::KV_S, dK + kstep<C::DCH, 128>(kk), dq + kstep<C::DCH, BQ>(kk), C::IDESC_KV_S,
+                       kk > 0 ? 1u : 0u);
+        if constexpr (C::FAC) {
+          uint64_t dfq = kdesc<C::FCH>(st + O_FQ);
+          asm volatile("" : "+l"(dfq));
+#pragma unroll
+          for (int kk = 0; kk < C::FCH * C::NFCH / 16; ++kk) {
+            if (MODE == kBiasTf32)
+              mma_ss_elect_tf32(tm_u + C::KV_S, dFK + kstep<C::FCH, 128>(kk), dfq + kstep<C::FCH, BQ>(kk),
+                                C::IDESC_KV_F, 1u);
+            else
+              mma_ss_elect(tm_u + C::KV_S, dFK + kstep<C::FCH, 128>(kk), dfq + kstep<C::FCH, BQ>(kk),
+                           C::IDESC_KV_F, 1u);
+          }
+        }
+#pragma unroll
+        for (int kk = 0; kk < DP / 16; ++kk)
+          mma_ss_elect(tm_u + C::KV_DP, dV + kstep<C::DCH, 128>(kk), ddo + kstep<C::DCH, BQ>(kk), C::IDESC_KV_S,
+                       kk > 0 ? 1u : 0u);
+      }
+      tc_commit_elect(&ctrl->s_full);
+      __syncwarp();
+      // P^T and dS^T are in TMEM (bf16 over the first BQ/2 columns of S^T and dP^T)
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&ctrl->p_full, uint32_t(it) & 1u, abort)))) break;
+      tc_fence_after();
+      {
+        uint64_t bdo = mndesc<C::DCH, BQ>(st + O_DO), bq = mndesc<C::DCH, BQ>(st + O_Q);
+        asm volatile("" : "+l"(bdo), "+l"(bq));
+#pragma unroll
+        for (int kk = 0; kk < BQ / 16; ++kk) {
+          const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+          mma_ts_elect(tm_u + C::KV_DV, tm_u + C::KV_S + uint32_t(kk * 8), bdo + mnstep<C::DCH>(kk), C::IDESC_GD, acc);
+          mma_ts_elect(tm_u + C::KV_DK, tm_u + C::KV_DP + uint32_t(kk * 8), bq + mnstep<C::DCH>(kk), C::IDESC_GD,
+                       acc);
+        }
+        if constexpr (RG > 0) {
+          uint64_t bg = mndesc<C::GCH, BQ>(st + O_GQ);
+          asm volatile("" : "+l"(bg));
+#pragma unroll
+          for (int kk = 0; kk < BQ / 16; ++kk)
+            mma_ts_elect(tm_u + C::KV_DF, tm_u + C::KV_DP + uint32_t(kk * 8), bg + mnstep<C::GCH>(kk), C::IDESC_GR,
+                         (it > 0 || kk > 0) ? 1u : 0u);
+        }
+      }
+      tc_commit_elect(&ctrl->empty[s]);
+      __syncwarp();
+    }
+    if (ok) {
+      tc_commit_elect(&ctrl->acc_done);
+      __syncwarp();
+    }
+    if (!ok && leader) atomicOr(args.flags, kFlagTimeout);
+  } else {
+    // ------------------------------------------------ compute (warps 0-3)
+    const int r_loc = warp * 32 + lane;
+    const int krow = k0 + r_loc;  // this thread's key
+    const uint32_t lane_base = tmem + (uint32_t(warp * 32) << 16);
+    const float sl2 = args.scale_log2;
+    bool ok = true;
+    int it = 0;
+    for (int j = j0; j < n_blk; ++j, ++it) {
+      const int s = it % KS;
+      // the whole warp leaves together: the TMEM accesses below are warp-collective
+      ok = mbar_wait(&ctrl->full[s], uint32_t(it / KS) & 1u, abort) && mbar_wait(&ctrl->s_full, uint32_t(it) & 1u, abort);
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint8_t *st = sStage + s * C::KV_STAGE;
+      const float *sL = reinterpret_cast<const float *>(st + O_L);
+      const float *sD = reinterpret_cast<const float *>(st + O_D);
+      const int q0 = j * BQ;
+      const bool diag = args.causal && q0 < k0 + 127;  // some query of the block precedes some key
+#pragma unroll 1
+      for (int c = 0; c < BQ / 32; ++c) {
+        uint32_t sx[32], dx[32];
+        tmem_ld32(lane_base + C::KV_S + uint32_t(32 * c), sx);
+        tmem_ld32(lane_base + C::KV_DP + uint32_t(32 * c), dx);
+        tmem_ld_wait32(sx);
+        tmem_ld_wait32(dx);
+        uint32_t pp[16], dd[16];
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 l4 = *reinterpret_cast<const float4 *>(sL + 32 * c + 4 * e4);
+          const float4 d4 = *reinterpret_cast<const float4 *>(sD + 32 * c + 4 * e4);
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
+          float p[4], g[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int col = 32 * c + 4 * e4 + e;
+            p[e] = ex2_approx(fmaf(__uint_as_float(sx[4 * e4 + e]), sl2, -lv[e]));
+            if (diag && q0 + col < krow) p[e] = 0.f;
+            g[e] = p[e] * (__uint_as_float(dx[4 * e4 + e]) - dv[e]);
+          }
+          pp[2 * e4] = pack_bf16x2(p[0], p[1]);
+          pp[2 * e4 + 1] = pack_bf16x2(p[2], p[3]);
+          dd[2 * e4] = pack_bf16x2(g[0], g[1]);
+          dd[2 * e4 + 1] = pack_bf16x2(g[2], g[3]);
+        }
+        tmem_st16(lane_base + C::KV_S + uint32_t(16 * c), pp);
+        tmem_st16(lane_base + C::KV_DP + uint32_t(16 * c), dd);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&ctrl->p_full);
+    }
+    if (ok) ok = mbar_wait(&ctrl->acc_done, 0, abort);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      tc_fence_after();
+      // TMEM loads are warp-collective: every lane loads, rows past N store nothing
+      const bool valid = krow < args.N;
+      const int d_st = valid ? args.d : 0;
+      uint16_t *dv_row = static_cast<uint16_t *>(args.dV) + (size_t(bh) * args.N + (valid ? krow : 0)) * args.d;
+      uint16_t *dk_row = static_cast<uint16_t *>(args.dK) + (size_t(bh) * args.N + (valid ? krow : 0)) * args.d;
+#pragma unroll 1
+      for (int c0 = 0; c0 < DP; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld16(lane_base + C::KV_DV + uint32_t(c0), r);
+        tmem_ld_wait16(r);
+        store_row16_bf16(r, 1.f, dv_row, c0, d_st);
+        tmem_ld16(lane_base + C::KV_DK + uint32_t(c0), r);
+        tmem_ld_wait16(r);
+        store_row16_bf16(r, args.scale, dk_row, c0, d_st);
+      }
+      if constexpr (RG > 0) {
+        const int r_st = valid ? args.R : 0;
+        float *df = args.dphi_k + (args.fac_B > 1 ? int64_t(b) * args.phi_bs : 0) +
+                    (args.fac_H > 1 ? int64_t(h) * args.phi_hs : 0) + int64_t(valid ? krow : 0) * args.R;
+#pragma unroll 1
+        for (int c0 = 0; c0 < RG; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld16(lane_base + C::KV_DF + uint32_t(c0), r);
+          tmem_ld_wait16(r);
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            if (c0 + e < r_st) atomicAdd(df + c0 + e, __uint_as_float(r[e]));
+        }
+      }
+    }
+    if (!ok && lane == 0) atomicOr(args.flags, kFlagTimeout);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == C::MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ dQ, dphi_q
+template <int DP, int RP, int MODE, int RG>
+__global__ void __launch_bounds__(192, 1)
+    attn_bwd_dq_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                      const __grid_constant__ CUtensorMap tm_fq, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_fk,
+                      const __grid_constant__ CUtensorMap tm_gk, const BwdArgs args) {
+  using C = BwdCfg<DP, RP, MODE, RG>;
+  constexpr int KS = C::DQ_KS;
+  static_assert(KS >= 1, "configuration does not fit in shared memory");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sQ = smem;                    // 128 x DP bf16
+  uint8_t *sDO = sQ + 128 * DP * 2;      // 128 x DP bf16
+  uint8_t *sFQ = sDO + 128 * DP * 2;     // 128 x RP (fp16 / fp32)
+  uint8_t *sStage = smem + C::DQ_FIXED;  // KS x DQ_STAGE
+  BwdCtrl *ctrl = reinterpret_cast<BwdCtrl *>(sStage + KS * C::DQ_STAGE);
+  constexpr uint32_t O_K = 0, O_V = 128 * DP * 2, O_FK = 2 * 128 * DP * 2;
+  constexpr uint32_t O_GK = O_FK + (C::FAC ? 128 * RP * C::FESZ : 0);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int BH = args.B * args.H;
+  const int qb = args.n_kv - 1 - int(blockIdx.x) / BH;  // the heaviest causal tiles come first
+  const int bh = int(blockIdx.x) % BH;
+  const int b = bh / args.H, h = bh % args.H;
+  const int q0 = qb * 128;
+  const int fslice = (args.fac_B > 1 ? b : 0) * args.fac_H + (args.fac_H > 1 ? h : 0);
+  const int nk = args.causal ? qb + 1 : args.n_kv;  // key tiles this query tile sees
+
+  if (threadIdx.x == 0) {
+    mbar_init(&ctrl->fixed_full, 1);
+    for (int s = 0; s < KS; ++s) {
+      mbar_init(&ctrl->full[s], 1);
+      mbar_init(&ctrl->empty[s], 1);
+    }
+    mbar_init(&ctrl->s_full, 1);
+    mbar_init(&ctrl->p_full, 128);
+    mbar_init(&ctrl->acc_done, 1);
+    ctrl->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == C::MMA_WARP) {
+    tmem_alloc(&ctrl->tmem_base, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctrl->tmem_base;
+  volatile int *abort = &ctrl->abort;
+  const uint32_t leader = lane == 0 ? 1u : 0u;
+
+  if (warp == C::PRODUCER_WARP) {
+    // ------------------------------------------------------------ producer
+    if (leader) {
+      tma_prefetch_map(&tm_q);
+      tma_prefetch_map(&tm_do);
+      tma_prefetch_map(&tm_k);
+      tma_prefetch_map(&tm_v);
+      if (C::FAC) {
+        tma_prefetch_map(&tm_fq);
+        tma_prefetch_map(&tm_fk);
+      }
+      if (RG > 0) tma_prefetch_map(&tm_gk);
+    }
+    mbar_arrive_expect_tx_leader(&ctrl->fixed_full, C::DQ_FIXED, leader);
+    for (int ch = 0; ch < C::NDCH; ++ch) {
+      tma_load_3d_leader(sQ + ch * (128 * C::DCH * 2), &tm_q, &ctrl->fixed_full, ch * C::DCH, q0, bh, leader);
+      tma_load_3d_leader(sDO + ch * (128 * C::DCH * 2), &tm_do, &ctrl->fixed_full, ch * C::DCH, q0, bh, leader);
+    }
+    if (C::FAC)
+      for (int ch = 0; ch < C::NFCH; ++ch)
+        tma_load_3d_leader(sFQ + ch * (128 * C::FCH * 2), &tm_fq, &ctrl->fixed_full, ch * C::FCH, q0, fslice,
+                           leader);
+    bool ok = true;
+    for (int i = 0; i < nk; ++i) {
+      const int s = i % KS;
+      const uint32_t ph = uint32_t(i / KS) & 1u;
+      if (i >= KS && !(ok = mbar_wait(&ctrl->empty[s], ph ^ 1u, abort))) break;
+      uint8_t *st = sStage + s * C::DQ_STAGE;
+      const int kv = i * 128;
+      mbar_arrive_expect_tx_leader(&ctrl->full[s], C::DQ_STAGE_BYTES, leader);
+      for (int ch = 0; ch < C::NDCH; ++ch) {
+        tma_load_3d_leader(st + O_K + ch * (128 * C::DCH * 2), &tm_k, &ctrl->full[s], ch * C::DCH, kv, bh, leader);
+        tma_load_3d_leader(st + O_V + ch * (128 * C::DCH * 2), &tm_v, &ctrl->full[s], ch * C::DCH, kv, bh, leader);
+      }
+      if (C::FAC)
+        for (int ch = 0; ch < C::NFCH; ++ch)
+          tma_load_3d_leader(st + O_FK + ch * (128 * C::FCH * 2), &tm_fk, &ctrl->full[s], ch * C::FCH, kv, fslice,
+                             leader);
+      for (int ch = 0; ch < C::NGCH; ++ch)
+        tma_load_3d_leader(st + O_GK + ch * (128 * C::GCH * 2), &tm_gk, &ctrl->full[s], ch * C::GCH, kv, fslice,
+                           leader);
+    }
+    if (!ok) {
+      mbar_wait_for(&ctrl->fixed_full, 0, 100000000ull);
+      for (int s = 0; s < KS; ++s) {
+        mbar_wait_for(&ctrl->full[s], 0, 100000000ull);
+        mbar_wait_for(&ctrl->full[s], 1, 100000000ull);
+      }
+      if (leader) atomicOr(args.flags, kFlagTimeout);
+    }
+  } else if (warp == C::MMA_WARP) {
+    // ---------------------------------------------------------- MMA issuer
+    const uint32_t tm_u = __shfl_sync(0xffffffffu, tmem, 0);
+    bool ok = __all_sync(0xffffffffu, mbar_wait(&ctrl->fixed_full, 0, abort));  // warp-uniform for elect.sync
+    tc_fence_after();
+    const uint64_t aQ = kdesc<C::DCH>(smem_u32(sQ));
+    const uint64_t aDO = kdesc<C::DCH>(smem_u32(sDO));
+    const uint64_t aFQ = kdesc<C::FCH>(smem_u32(sFQ));
+    for (int i = 0; i < nk && ok; ++i) {
+      const int s = i % KS;
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&ctrl->full[s], uint32_t(i / KS) & 1u, abort)))) break;
+      tc_fence_after();
+      const uint32_t st = smem_u32(sStage + s * C::DQ_STAGE);
+      {  // S = Q K^T (+ phi_q' phi_k'^T), dP = dO V^T
+        uint64_t bk = kdesc<C::DCH>(st + O_K), bv = kdesc<C::DCH>(st + O_V);
+        asm volatile("" : "+l"(bk), "+l"(bv));
+#pragma unroll
+        for (int kk = 0; kk < DP / 16; ++kk)
+          mma_ss_elect(tm_u + C::DQ_S, aQ + kstep<C::DCH, 128>(kk), bk + kstep<C::DCH, 128>(kk), C::IDESC_DQ_S,
+                       kk > 0 ? 1u : 0u);
+        if constexpr (C::FAC) {
+          uint64_t bfk = kdesc<C::FCH>(st + O_FK);
+          asm volatile("" : "+l"(bfk));
+#pragma unroll
+          for (int kk = 0; kk < C::FCH * C::NFCH / 16; ++kk) {
+            if (MODE == kBiasTf32)
+              mma_ss_elect_tf32(tm_u + C::DQ_S, aFQ + kstep<C::FCH, 128>(kk), bfk + kstep<C::FCH, 128>(kk),
+                                C::IDESC_DQ_F, 1u);
+            else
+              mma_ss_elect(tm_u + C::DQ_S, aFQ + kstep<C::FCH, 128>(kk), bfk + kstep<C::FCH, 128>(kk),
+                           C::IDESC_DQ_F, 1u);
+          }
+        }
+#pragma unroll
+        for (int kk = 0; kk < DP / 16; ++kk)
+          mma_ss_elect(tm_u + C::DQ_DP, aDO + kstep<C::DCH, 128>(kk), bv + kstep<C::DCH, 128>(kk), C::IDESC_DQ_S,
+                       kk > 0 ? 1u : 0u);
+      }
+      tc_commit_elect(&ctrl->s_full);
+      __syncwarp();
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&ctrl->p_full, uint32_t(i) & 1u, abort)))) break;
+      tc_fence_after();
+      {  // dQ += dS K, dphi_q += dS phi_k (dS bf16 over the first 64 columns of S)
+        uint64_t bk = mndesc<C::DCH, 128>(st + O_K);
+        asm volatile("" : "+l"(bk));
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts_elect(tm_u + C::DQ_DQ, tm_u + C::DQ_S + uint32_t(kk * 8), bk + mnstep<C::DCH>(kk), C::IDESC_GD,
+                       (i > 0 || kk > 0) ? 1u : 0u);
+        if constexpr (RG > 0) {
+          uint64_t bg = mndesc<C::GCH, 128>(st + O_GK);
+          asm volatile("" : "+l"(bg));
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts_elect(tm_u + C::DQ_DF, tm_u + C::DQ_S + uint32_t(kk * 8), bg + mnstep<C::GCH>(kk), C::IDESC_GR,
+                         (i > 0 || kk > 0) ? 1u : 0u);
+        }
+      }
+      tc_commit_elect(&ctrl->empty[s]);
+      __syncwarp();
+    }
+    if (ok) {
+      tc_commit_elect(&ctrl->acc_done);
+      __syncwarp();
+    }
+    if (!ok && leader) atomicOr(args.flags, kFlagTimeout);
+  } else {
+    // ------------------------------------------------ compute (warps 0-3)
+    const int r_loc = warp * 32 + lane;
+    const int row = q0 + r_loc;  // this thread's query
+    const uint32_t lane_base = tmem + (uint32_t(warp * 32) << 16);
+    const float sl2 = args.scale_log2;
+    const float neg_lse2 = -args.lse2[size_t(bh) * args.Npad + row];  // -inf past N: P = 0
+    const float drow = args.delta[size_t(bh) * args.Npad + row];
+    const int lim = args.causal ? min(row + 1, args.N) : args.N;  // keys [0, lim) are visible
+    bool ok = true;
+    for (int i = 0; i < nk; ++i) {
+      ok = mbar_wait(&ctrl->s_full, uint32_t(i) & 1u, abort);
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int key0 = i * 128;
+      const bool edge = key0 + 127 >= lim || key0 + 128 > args.N;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sx[32], dx[32];
+        tmem_ld32(lane_base + C::DQ_S + uint32_t(32 * c), sx);
+        tmem_ld32(lane_base + C::DQ_DP + uint32_t(32 * c), dx);
+        tmem_ld_wait32(sx);
+        tmem_ld_wait32(dx);
+        uint32_t dd[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float g[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int col = 32 * c + 2 * e + u;
+            float p = ex2_approx(fmaf(__uint_as_float(sx[2 * e + u]), sl2, neg_lse2));
+            if (edge && key0 + col >= lim) p = 0.f;
+            g[u] = p * (__uint_as_float(dx[2 * e + u]) - drow);
+          }
+          dd[e] = pack_bf16x2(g[0], g[1]);
+        }
+        tmem_st16(lane_base + C::DQ_S + uint32_t(16 * c), dd);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&ctrl->p_full);
+    }
+    if (ok) ok = mbar_wait(&ctrl->acc_done, 0, abort);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      tc_fence_after();
+      const bool valid = row < args.N;
+      const int d_st = valid ? args.d : 0;
+      uint16_t *dq_row = static_cast<uint16_t *>(args.dQ) + (size_t(bh) * args.N + (valid ? row : 0)) * args.d;
+#pragma unroll 1
+      for (int c0 = 0; c0 < DP; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld16(lane_base + C::DQ_DQ + uint32_t(c0), r);
+        tmem_ld_wait16(r);
+        store_row16_bf16(r, args.scale, dq_row, c0, d_st);
+      }
+      if constexpr (RG > 0) {
+        const int r_st = valid ? args.R : 0;
+        float *df = args.dphi_q + (args.fac_B > 1 ? int64_t(b) * args.phi_bs : 0) +
+                    (args.fac_H > 1 ? int64_t(h) * args.phi_hs : 0) + int64_t(valid ? row : 0) * args.R;
+#pragma unroll 1
+        for (int c0 = 0; c0 < RG; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld16(lane_base + C::DQ_DF + uint32_t(c0), r);
+          tmem_ld_wait16(r);
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            if (c0 + e < r_st) atomicAdd(df + c0 + e, __uint_as_float(r[e]));
+        }
+      }
+    }
+    if (!ok && lane == 0) atomicOr(args.flags, kFlagTimeout);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == C::MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+namespace {
+
+constexpr int kMaxDevicesB = 64;
+
+template <int DP, int RP, int MODE, int RG>
+cudaError_t launch_bwd_one(const BwdMaps &m, const BwdArgs &a, cudaStream_t stream) {
+  using C = BwdCfg<DP, RP, MODE, RG>;
+  if constexpr (C::KV_KS < 1 || C::DQ_KS < 1) {
+    return cudaErrorInvalidConfiguration;
+  } else {
+    auto kv = attn_bwd_dkdv_sm100<DP, RP, MODE, RG>;
+    auto dq = attn_bwd_dq_sm100<DP, RP, MODE, RG>;
+    static std::atomic<int> ready[kMaxDevicesB];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevicesB) return cudaErrorInvalidDevice;
+    if (!ready[dev].load(std::memory_order_acquire)) {
+      if ((e = cudaFuncSetAttribute(kv, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::KV_SMEM))) != cudaSuccess)
+        return e;
+      if ((e = cudaFuncSetAttribute(dq, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::DQ_SMEM))) != cudaSuccess)
+        return e;
+      ready[dev].store(1, std::memory_order_release);
+    }
+    const unsigned grid = unsigned((long long)a.n_kv * a.B * a.H);
+    kv<<<grid, C::THREADS, C::KV_SMEM, stream>>>(m.k, m.v, m.fk, m.q_blk, m.do_blk, m.fq_blk, m.gq_blk, a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    dq<<<grid, C::THREADS, C::DQ_SMEM, stream>>>(m.q, m.dO, m.fq, m.k, m.v, m.fk, m.gk, a);
+    return cudaGetLastError();
+  }
+}
+
+template <int DP, int RP, int MODE, int RG>
+constexpr int bwd_block_rows() {
+  return BwdCfg<DP, RP, MODE, RG>::BQ;
+}
+
+}  // namespace
+
+#define FB_BWD_MODE(DPv)                                                            \
+  if (p.mode == kBiasNone) return FB_BWD_ACTION(DPv, 0, kBiasNone, 0);              \
+  if (p.mode == kBiasTf32) {                                                        \
+    if (p.RP == 8) return FB_BWD_ACTION(DPv, 8, kBiasTf32, 16);                     \
+    if (p.RP == 16) return FB_BWD_ACTION(DPv, 16, kBiasTf32, 16);                   \
+  }                                                                                 \
+  if (p.mode == kBiasMma) {                                                         \
+    if (p.RP == 16) return FB_BWD_ACTION(DPv, 16, kBiasMma, 16);                    \
+    if (p.RP == 32) return FB_BWD_ACTION(DPv, 32, kBiasMma, 32);                    \
+    if (p.RP == 64) return FB_BWD_ACTION(DPv, 64, kBiasMma, 64);                    \
+    if (p.RP == 128) return FB_BWD_ACTION(DPv, 128, kBiasMma, 128);                 \
+  }
+
+#define FB_BWD_ALL                                                                  \
+  if (p.DP == 16) { FB_BWD_MODE(16) }                                               \
+  if (p.DP == 32) { FB_BWD_MODE(32) }                                               \
+  if (p.DP == 64) { FB_BWD_MODE(64) }                                               \
+  if (p.DP == 128) { FB_BWD_MODE(128) }
+
+int bwd_query_block_rows(const BwdPlan &p) {
+#define FB_BWD_ACTION(DPv, RPv, MODEv, RGv) bwd_block_rows<DPv, RPv, MODEv, RGv>()
+  FB_BWD_ALL
+#undef FB_BWD_ACTION
+  return 0;
+}
+
+cudaError_t bwd_launch(const BwdPlan &p, const BwdMaps &maps, const BwdArgs &a, cudaStream_t stream) {
+#define FB_BWD_ACTION(DPv, RPv, MODEv, RGv) launch_bwd_one<DPv, RPv, MODEv, RGv>(maps, a, stream)
+  FB_BWD_ALL
+#undef FB_BWD_ACTION
+  return cudaErrorInvalidConfiguration;
+}
+
+}  // namespace fb

@@ -319,6 +319,87 @@ cudaError_t launch_prep_factors(int mode, int B, int H, int N, int R, int RP, co
   return cudaGetLastError();
 }
 
+// Backward rows: lse2 = LSE log2(e) and delta = rowsum(dO * O) (fp32 sum of
+// the bf16 products), one warp per row; rows N .. Npad-1 get +inf and 0, so
+// the kernels' padded queries carry P = 0 without a bounds test.
+__global__ void __launch_bounds__(256) bwd_rows_kernel(long long rows, int N, int Npad, int d,
+                                                       const __nv_bfloat16 *__restrict__ O,
+                                                       const __nv_bfloat16 *__restrict__ dO,
+                                                       const float *__restrict__ LSE, float *__restrict__ lse2,
+                                                       float *__restrict__ delta) {
+  const int lane = threadIdx.x & 31;
+  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long w = blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5); w < rows; w += warps) {
+    const long long bh = w / Npad;
+    const int n = int(w - bh * Npad);
+    float acc = 0.f;
+    if (n < N) {
+      const size_t base = (size_t(bh) * N + n) * d;
+      for (int c = lane * 4; c < d; c += 128) {  // d % 8 == 0: 4-element pieces stay in the row
+        const uint2 a = *reinterpret_cast<const uint2 *>(O + base + c);
+        const uint2 g = *reinterpret_cast<const uint2 *>(dO + base + c);
+        const uint32_t av[2] = {a.x, a.y}, gv[2] = {g.x, g.y};
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          acc = fmaf(__uint_as_float(av[e] << 16), __uint_as_float(gv[e] << 16), acc);
+          acc = fmaf(__uint_as_float(av[e] & 0xFFFF0000u), __uint_as_float(gv[e] & 0xFFFF0000u), acc);
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) {
+      lse2[w] = n < N ? LSE[size_t(bh) * N + n] * 1.4426950408889634f : INFINITY;
+      delta[w] = acc;
+    }
+  }
+}
+
+// bf16 copies of the factors for the gradient products, [FB, N, RG] with
+// zero padding, and the factor gradients zeroed (the backward kernels add
+// into them).
+__global__ void prep_grad_factors_kernel(int N, int R, int RG, int fac_H, const float *__restrict__ pq,
+                                         const float *__restrict__ pk, long long bs, long long hs,
+                                         __nv_bfloat16 *__restrict__ gq, __nv_bfloat16 *__restrict__ gk,
+                                         float *__restrict__ dpq, float *__restrict__ dpk, long long total) {
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int r = int(idx % RG);
+    const long long rest = idx / RG;
+    const long long n = rest % N;
+    const long long f = rest / N;
+    const long long fb = f / fac_H, fh = f - (f / fac_H) * fac_H;
+    float vq = 0.f, vk = 0.f;
+    if (r < R) {
+      const long long src = fb * bs + fh * hs + n * R + r;
+      vq = pq[src];
+      vk = pk[src];
+      dpq[src] = 0.f;
+      dpk[src] = 0.f;
+    }
+    gq[idx] = __float2bfloat16_rn(vq);
+    gk[idx] = __float2bfloat16_rn(vk);
+  }
+}
+
+cudaError_t launch_bwd_rows(int BH, int N, int Npad, int d, const void *O, const void *dO, const float *LSE,
+                            float *lse2, float *delta, cudaStream_t s) {
+  const long long rows = (long long)BH * Npad;
+  bwd_rows_kernel<<<grid_for(rows * 32, 256), 256, 0, s>>>(rows, N, Npad, d, static_cast<const __nv_bfloat16 *>(O),
+                                                           static_cast<const __nv_bfloat16 *>(dO), LSE, lse2, delta);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prep_grad_factors(int N, int R, int RG, const float *phi_q, const float *phi_k, int64_t bs,
+                                     int64_t hs, int fac_B, int fac_H, void *gq, void *gk, float *dphi_q,
+                                     float *dphi_k, cudaStream_t s) {
+  const long long total = (long long)fac_B * fac_H * N * RG;
+  prep_grad_factors_kernel<<<grid_for(total, 256), 256, 0, s>>>(
+      N, R, RG, fac_H, phi_q, phi_k, bs, hs, static_cast<__nv_bfloat16 *>(gq), static_cast<__nv_bfloat16 *>(gk),
+      dphi_q, dphi_k, total);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_wait_selftest(int limit_ms, int *flags, cudaStream_t s) {
   wait_selftest_kernel<<<1, 32, 0, s>>>((unsigned long long)limit_ms * 1000000ull, flags);
   return cudaGetLastError();

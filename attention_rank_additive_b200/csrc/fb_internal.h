@@ -78,6 +78,47 @@ cudaError_t launch_prep_mul_bias(int B, int H, int N, int d, int R, int RP, cons
                                  const float *phi_q, const float *phi_k, int64_t bs, int64_t hs, void *q1, void *k1,
                                  void *fq, void *fk, int *flags, cudaStream_t s);
 
+// Backward (gradients of O for dO).
+struct BwdArgs {
+  int B, H, N, d, R;
+  int n_kv;                // 128-row tiles along N
+  int Npad;                // n_kv * 128: row stride of lse2 / delta
+  float scale, scale_log2;
+  int causal;
+  const float *lse2;       // [BH, Npad] LSE * log2(e); +inf past N
+  const float *delta;      // [BH, Npad] rowsum(dO * O); 0 past N
+  void *dQ, *dK, *dV;      // bf16 [BH, N, d]
+  float *dphi_q, *dphi_k;  // fp32, laid out like phi_q / phi_k (zeroed first, accumulated)
+  int64_t phi_bs, phi_hs;  // element strides of the factor tensors
+  int fac_B, fac_H;        // factor slices: B or 1, H or 1
+  int *flags;
+};
+
+struct BwdPlan {
+  int DP;    // padded head dim
+  int RP;    // S-side factor width (as FwdPlan)
+  int mode;  // kBiasNone, kBiasMma or kBiasTf32
+  int RG;    // bf16 gradient factor width: pad_rank(R), 16 for R <= 4, 0 for R = 0
+};
+
+struct BwdMaps {
+  CUtensorMap q, k, v, dO;      // bf16 [BH, N, d], box (min(DP,64), 128, 1)
+  CUtensorMap q_blk, do_blk;    // the same with box rows = the dK/dV kernel's query block
+  CUtensorMap fq, fk, fq_blk;   // S-side factors (as FwdMaps), box rows 128 / query block
+  CUtensorMap gq_blk, gk;       // bf16 gradient factors [FB, N, RG], box rows query block / 128
+};
+
+// Rows of the dK/dV kernel's query block for a plan (0: unsupported).
+int bwd_query_block_rows(const BwdPlan &p);
+cudaError_t bwd_launch(const BwdPlan &p, const BwdMaps &maps, const BwdArgs &a, cudaStream_t stream);
+// lse2 = LSE * log2(e) and delta = rowsum(dO * O) per row, padded to Npad.
+cudaError_t launch_bwd_rows(int BH, int N, int Npad, int d, const void *O, const void *dO, const float *LSE,
+                            float *lse2, float *delta, cudaStream_t s);
+// bf16 copies of the factors [FB, N, RG] (zero-padded) and zeroed factor gradients.
+cudaError_t launch_prep_grad_factors(int N, int R, int RG, const float *phi_q, const float *phi_k, int64_t bs,
+                                     int64_t hs, int fac_B, int fac_H, void *gq, void *gk, float *dphi_q,
+                                     float *dphi_k, cudaStream_t s);
+
 // Per-device flag word (allocated once per device as a module global).
 int *device_flags();
 

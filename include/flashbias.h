@@ -203,6 +203,49 @@ int fb_attn_neural_fwd(int dt, int B, int H, int N, int d,
                        void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Backward of fb_attn_fwd: the gradients of O for an upstream gradient dO.
+ * FlashBias trains with a factorised bias by concatenating the factors to the
+ * queries and keys (rebuttal, reply to Reviewer UJUf, Q2, and its training
+ * speedup in Q1 (3); reply to Reviewer Bp2x, Q3), so the factor gradients are
+ * the extra columns of the concatenated query and key gradients:
+ *
+ *   P = softmax(scale Q K^T + phi_q phi_k^T [+ causal]),  dP = dO V^T,
+ *   dS = P o (dP - rowsum(dO o O)),
+ *   dQ = scale dS K, dK = scale dS^T Q, dV = P^T dO,
+ *   dphi_q = dS phi_k, dphi_k = dS^T phi_q.
+ *
+ *  dt          FB_BF16 only.
+ *  Q..phi_k    the forward's inputs, same layouts and strides.
+ *  O, LSE      the forward's outputs for these inputs (O bf16 [B,H,N,d],
+ *              LSE fp32 [B,H,N], natural log).
+ *  dO          bf16 [B,H,N,d] device.
+ *  dQ, dK, dV  bf16 [B,H,N,d] device outputs, 16-byte aligned.
+ *  dphi_q/k    fp32 device outputs laid out like phi_q / phi_k (the same
+ *              strides; a broadcast factor, stride 0, gets the gradient
+ *              summed over the batches or heads sharing it). Overwritten:
+ *              the call zeroes them, then accumulates. Unused when R = 0.
+ *  workspace   fb_attn_bwd_workspace_bytes(B, H, N, R, phi_bstride,
+ *              phi_hstride) bytes, 256-byte aligned (never 0).
+ * Arithmetic: S and P are recomputed as the forward computes them; the
+ * products with dO, Q, K and the factors run on the tensor cores in bf16 with
+ * fp32 accumulation. Launches: the factor preparation and the bf16 factor
+ * copies (R > 0), the per-row terms, then two tcgen05 kernels (dK, dV,
+ * dphi_k per key tile; dQ, dphi_q per query tile). Argument errors return
+ * before any launch; other errors as fb_attn_fwd.
+ */
+size_t fb_attn_bwd_workspace_bytes(int B, int H, int N, int R,
+                                   int64_t phi_bstride, int64_t phi_hstride);
+
+int fb_attn_bwd(int dt, int B, int H, int N, int d,
+                const void *Q, const void *K, const void *V,
+                int R, const float *phi_q, const float *phi_k,
+                int64_t phi_bstride, int64_t phi_hstride,
+                float scale, int causal,
+                const void *O, const float *LSE, const void *dO,
+                void *dQ, void *dK, void *dV, float *dphi_q, float *dphi_k,
+                void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Truncated SVD of H dense biases on the GPU, for biases known only at call
  * time (the SVD decomposition of the rebuttal, reply to Reviewer xU4x, Q6,
  * done per call; the rebuttal calls this inefficient for dynamic biases,

@@ -315,3 +315,44 @@ def test_neural_workspace_and_argument_errors():
     assert n(d=20) == fb.FB_ERR_UNSUPPORTED
     assert n(workspace=0) == fb.FB_ERR_WORKSPACE
     assert n(workspace_bytes=need - 1) == fb.FB_ERR_WORKSPACE
+
+
+def test_backward_workspace_and_argument_errors():
+    """fb_attn_bwd: the workspace covers the forward's factor tiles, the bf16
+    factor copies and two fp32 rows per (b, h, padded query); every argument
+    error returns before a launch."""
+    al = lambda x: (x + 255) // 256 * 256
+    B, H, N, R = 2, 3, 200, 8
+    Npad = 256
+    fwd = fb.fb_attn_workspace_bytes(B, H, N, R, H * N * R, N * R)
+    assert fb.fb_attn_bwd_workspace_bytes(B, H, N, R, H * N * R, N * R) == \
+        fwd + 2 * al(B * H * N * 16 * 2) + 2 * al(B * H * Npad * 4)
+    # broadcast factors: one factor slice
+    assert fb.fb_attn_bwd_workspace_bytes(B, H, N, R, 0, 0) == \
+        fb.fb_attn_workspace_bytes(B, H, N, R, 0, 0) + 2 * al(N * 16 * 2) + 2 * al(B * H * Npad * 4)
+    assert fb.fb_attn_bwd_workspace_bytes(B, H, N, 0, 0, 0) == 2 * al(B * H * Npad * 4)
+    assert fb.fb_attn_bwd_workspace_bytes(B, H, N, 129, 0, 0) == 0
+    assert fb.fb_attn_bwd_workspace_bytes(0, H, N, R, 0, 0) == 0
+    need = fb.fb_attn_bwd_workspace_bytes(1, 2, 128, R, 2 * 128 * R, 128 * R)
+    run = dict(dt=fb.FB_BF16, B=1, H=2, N=128, d=64, Q=FAKE, K=FAKE, V=FAKE, R=R, phi_q=FAKE, phi_k=FAKE,
+               phi_bstride=2 * 128 * R, phi_hstride=128 * R, scale=0.125, causal=1, O=FAKE, LSE=FAKE, dO=FAKE,
+               dQ=FAKE, dK=FAKE, dV=FAKE, dphi_q=FAKE, dphi_k=FAKE, workspace=FAKE, workspace_bytes=need,
+               stream=None)
+
+    def b(**kw):
+        a = dict(run)
+        a.update(kw)
+        return fb.fb_attn_bwd(**a)
+
+    assert b(dt=fb.FB_F32) == fb.FB_ERR_UNSUPPORTED
+    assert b(R=129) == fb.FB_ERR_UNSUPPORTED
+    assert b(d=20) == fb.FB_ERR_UNSUPPORTED
+    assert b(dO=0) == fb.FB_ERR_INVALID_ARG
+    assert b(dphi_k=0) == fb.FB_ERR_INVALID_ARG
+    assert b(dphi_q=FAKE + 2) == fb.FB_ERR_INVALID_ARG
+    assert b(dK=FAKE + 8) == fb.FB_ERR_INVALID_ARG
+    assert b(phi_hstride=-1) == fb.FB_ERR_INVALID_ARG
+    assert b(scale=float("nan")) == fb.FB_ERR_INVALID_ARG
+    assert b(workspace=0) == fb.FB_ERR_WORKSPACE
+    assert b(workspace_bytes=need - 1) == fb.FB_ERR_WORKSPACE
+    assert b(workspace=FAKE + 16) == fb.FB_ERR_WORKSPACE

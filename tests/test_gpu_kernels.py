@@ -363,3 +363,80 @@ def test_neural_bias_matches_oracle(B, H, N, d, F, R, causal):
     for b in range(B):
         for h in range(H):
             compare(og[b, h], lg[b, h], ro[b, h], rl[b, h], "bf16", f"neural F{F} R{R} ({b},{h})")
+
+
+# ---------------------------------------------------------------- backward
+
+def _grad_close(g, ref, what):
+    """Gradient tolerance: the forward's bf16 bound on O (max 2e-2, mean 2e-3
+    for values of order one) applied to the gradient scaled by its largest
+    reference magnitude, floored at 1e-3 for gradients that vanish exactly
+    (a single visible key makes dS zero; the kernel then returns rounding
+    noise of D = rowsum(dO * O) from the bf16 O)."""
+    g = np.asarray(g, np.float64)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite gradient"
+    m = max(float(np.abs(ref).max()) if ref.size else 0.0, 1e-3)
+    err = np.abs(g - ref) / m
+    assert err.max() <= 2e-2, f"{what}: max rel {err.max():.3e}"
+    assert err.mean() <= 2e-3, f"{what}: mean rel {err.mean():.3e}"
+    return float(err.max()), float(err.mean())
+
+
+BWD_SWEEP = [
+    # B, H, N, d, R, causal, factor layout
+    (1, 2, 200, 64, 64, True, "bhnr"),
+    (1, 1, 1, 64, 8, True, "bhnr"),
+    (2, 1, 257, 128, 2, True, "bhnr"),
+    (1, 2, 300, 128, 128, False, "hnr"),
+    (1, 1, 384, 32, 1, True, "bhnr"),
+    (1, 2, 130, 16, 8, False, "nr"),
+    (1, 2, 255, 24, 32, True, "bhnr"),
+    (1, 1, 513, 40, 4, False, "bhnr"),
+    (1, 2, 700, 64, 0, True, "bhnr"),
+    (1, 1, 400, 96, 100, False, "bhnr"),
+]
+
+
+@pytest.mark.parametrize("B,H,N,d,R,causal,layout", BWD_SWEEP)
+def test_backward_matches_oracle(B, H, N, d, R, causal, layout):
+    seed = 900 + N + d + R
+    q, k, v = si.qkv(B, H, N, d, seed, "bf16")
+    g = si.round_to_bf16(si.normal((B, H, N, d), seed + 3))
+    scale = 1.0 / math.sqrt(d)
+    pq = pk = None
+    if R > 0:
+        shape = {"nr": (N, R), "hnr": (H, N, R), "bhnr": (B, H, N, R)}[layout]
+        pq, pk = si.random_factors(shape, math.sqrt(1.0 / R), seed + 7)
+    tq, tk, tv, tg = (dev(x, "bf16") for x in (q, k, v, g))
+    tpq = None if pq is None else dev(pq, "f32")
+    tpk = None if pk is None else dev(pk, "f32")
+    o, lse = fb.attn(tq, tk, tv, tpq, tpk, scale=scale, causal=causal)
+    dq, dk, dv, dpq, dpk = fb.attn_bwd(tq, tk, tv, tpq, tpk, o, lse, tg, scale=scale, causal=causal)
+    torch.cuda.synchronize()
+    _no_device_error()
+
+    def fac(x, b, h):
+        if x is None:
+            return np.zeros((N, 0))
+        return {"nr": lambda: x, "hnr": lambda: x[h], "bhnr": lambda: x[b, h]}[layout]()
+
+    ref_pq = None if pq is None else np.zeros(pq.shape)
+    ref_pk = None if pk is None else np.zeros(pk.shape)
+    got = {n: host(t) for n, t in (("dq", dq), ("dk", dk), ("dv", dv))}
+    for b in range(B):
+        for h in range(H):
+            r = oracle.attention_lowrank_bwd_head(q[b, h], k[b, h], v[b, h], fac(pq, b, h), fac(pk, b, h),
+                                                  g[b, h], scale, causal)
+            for n in ("dq", "dk", "dv"):
+                _grad_close(got[n][b, h], r[n], f"{n} ({b},{h}) B{B} H{H} N{N} d{d} R{R} c{causal}")
+            if R > 0:
+                for acc, key in ((ref_pq, "dphi_q"), (ref_pk, "dphi_k")):
+                    if layout == "nr":
+                        acc += r[key]
+                    elif layout == "hnr":
+                        acc[h] += r[key]
+                    else:
+                        acc[b, h] += r[key]
+    if R > 0:
+        _grad_close(host(dpq), ref_pq, f"dphi_q B{B} H{H} N{N} d{d} R{R} {layout}")
+        _grad_close(host(dpk), ref_pk, f"dphi_k B{B} H{H} N{N} d{d} R{R} {layout}")
