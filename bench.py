@@ -47,7 +47,7 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--config", type=int, default=1, choices=[0, 1, 2, 3, 4, 5, 6])
+    ap.add_argument("--config", type=int, default=1, choices=[0, 1, 2, 3, 4, 5, 6, 7])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-bias comparison leg")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline leg")
@@ -57,6 +57,8 @@ def parse_args(argv=None):
 def workload(cfg_idx: int) -> dict:
     c = dict(si.CONFIGS[cfg_idx])
     c["flops"] = flops(c["B"], c["H"], c["N"], c["d"], c["R"], c["causal"], c["bias"] == "mulcos")
+    if c.get("bwd"):
+        c["flops"] = bwd_flops(c["B"], c["H"], c["N"], c["d"], c["R"], c["causal"])
     if c["bias"] == "neural":  # plus the two linear layers, per (batch, head)
         c["flops"] += 2.0 * 2.0 * c["B"] * c["H"] * c["N"] * c["F"] * c["R"]
     return c
@@ -71,11 +73,21 @@ def flops(B, H, N, d, R, causal, multiplicative=False) -> float:
     return f / 2.0 if causal else f
 
 
+def bwd_flops(B, H, N, d, R, causal) -> float:
+    """Counted FLOPs of the backward per head: the five products of the
+    concatenated form, 2 N^2 (d + R) each for S, dQ' = dS K' and dK' =
+    dS^T Q', 2 N^2 d each for dP and dV (the dQ kernel's recomputation of S
+    and dP is not counted); halved when causal."""
+    f = float(B) * H * 2.0 * N * N * (5.0 * d + 3.0 * R)
+    return f / 2.0 if causal else f
+
+
 def config_json(c: dict, l2: str) -> dict:
     return {"workload": f"{c['name']} (B={c['B']},H={c['H']},N={c['N']},d={c['d']},R={c['R']},"
                         f"{'causal' if c['causal'] else 'no mask'},{c['bias']} bias)",
             "B": c["B"], "H": c["H"], "N": c["N"], "d": c["d"], "R": c["R"], "causal": c["causal"],
             "bias": c["bias"], "dtype": c["dtype"], "l2": l2,
+            "pass": "backward (dQ, dK, dV, dphi_q, dphi_k for a given dO)" if c.get("bwd") else "forward",
             "factors": ("static (the exact Sandwich/ALiBi decomposition depends on N, H only), generated once "
                         "before timing; prepared (scaled, fp16/paired) and consumed every step"
                         if c["bias"] in ("sandwich", "alibi") else
@@ -296,6 +308,36 @@ class GpuWorkload:
         # reweighting launch instead, the neural case its linear-layer launch in addition
         self.launches_per_step = (3 if self.neural else
                                   (2 if self.mul or (Rk > 0 and c["dtype"] == "bf16") else 1))
+        self.bwd = bool(c.get("bwd"))
+        if self.bwd:  # factor preparation, bf16 factor copies, per-row terms, two gradient kernels
+            self.launches_per_step = 5 if Rk > 0 else 3
+
+    def setup_bwd(self):
+        """Forward outputs O, LSE for the backward workload (once, untimed),
+        the seeded upstream gradient dO, and the gradient buffers."""
+        torch, fb, c = self.torch, self.fb, self.c
+        B, H, N, d = c["B"], c["H"], c["N"], c["d"]
+        self.attn()
+        self.host_o = self.O.cpu().pin_memory()
+        self.host_lse = self.LSE.cpu().pin_memory()
+        g = si.upstream_grad(B, H, N, d, si.DO_SEED_BASE + c["index"])
+        self.host_do = torch.from_numpy(g).to(torch.bfloat16).pin_memory()
+        self.dO = self.host_do.to(self.device)
+        self.dQ, self.dK, self.dV = (torch.empty_like(self.Q) for _ in range(3))
+        self.dpq = torch.empty_like(self.pq) if self.R else None
+        self.dpk = torch.empty_like(self.pk) if self.R else None
+        self.bws_bytes = fb.fb_attn_bwd_workspace_bytes(B, H, N, self.R, self.bs, self.hs)
+        self.bws = torch.empty(self.bws_bytes, device=self.device, dtype=torch.uint8)
+
+    def run_bwd(self):
+        fb, c = self.fb, self.c
+        st = fb.fb_attn_bwd(fb.FB_BF16, c["B"], c["H"], c["N"], c["d"], self.Q.data_ptr(), self.K.data_ptr(),
+                            self.V.data_ptr(), self.R, self.pq.data_ptr() if self.R else 0,
+                            self.pk.data_ptr() if self.R else 0, self.bs, self.hs, self.scale, int(c["causal"]),
+                            self.O.data_ptr(), self.LSE.data_ptr(), self.dO.data_ptr(), self.dQ.data_ptr(),
+                            self.dK.data_ptr(), self.dV.data_ptr(), self.dpq.data_ptr() if self.R else 0,
+                            self.dpk.data_ptr() if self.R else 0, self.bws.data_ptr(), self.bws_bytes, self.stream)
+        assert st == fb.FB_OK, fb.fb_status_str(st)
 
     def _dense_bias(self):
         """The same bias materialised as [B, H, N, N] bf16 (the comparison path's input)."""
@@ -335,7 +377,7 @@ class GpuWorkload:
     def prepare(self):
         """The factor preparation launch (bf16 path with a bias); fb_attn_fwd's first half."""
         fb, c = self.fb, self.c
-        if c["dtype"] != "bf16" or self.R == 0 or self.mul or self.neural:
+        if c["dtype"] != "bf16" or self.R == 0 or self.mul or self.neural or getattr(self, "bwd_active", False):
             return
         st = fb.fb_attn_prepare_factors(c["B"], c["H"], c["N"], self.R, self.pq.data_ptr(), self.pk.data_ptr(),
                                         self.bs, self.hs, self.scale, self.ws.data_ptr(), self.ws_bytes, self.stream)
@@ -344,6 +386,9 @@ class GpuWorkload:
     def run(self):
         """The fused kernel alone (bf16), or the whole fp32 call."""
         fb, c = self.fb, self.c
+        if getattr(self, "bwd_active", False):  # the whole backward call (its preparation included)
+            self.run_bwd()
+            return
         if self.neural:  # linear layers + preparation + fused kernel (one C-ABI call)
             xq, xk, wq, wk = self.nx
             st = fb.fb_attn_neural_fwd(fb.FB_BF16, c["B"], c["H"], c["N"], c["d"], self.Q.data_ptr(),
@@ -438,12 +483,15 @@ def run_ours(args, rank: int, world: int, local: int):
     fb.lib()
     # (no dense counterpart for the multiplicative bias: the comparison kernel adds its bias)
     w = GpuWorkload(c, device, with_dense=not args.no_dense and c["dtype"] == "bf16"
-                    and c["bias"] not in ("mulcos", "neural"))
+                    and c["bias"] not in ("mulcos", "neural") and not c.get("bwd"))
     stream = torch.cuda.current_stream(device)
 
     attn_ms = []
 
     w.gen_factors()  # static factors: once, outside the timed steps
+    if w.bwd:
+        w.setup_bwd()
+        w.bwd_active = True
 
     def step():
         w.prepare()
@@ -488,6 +536,23 @@ def run_ours(args, rank: int, world: int, local: int):
         host_o.copy_(w.O, non_blocking=True)
         host_l.copy_(w.LSE, non_blocking=True)
 
+    if w.bwd:  # inputs Q, K, V, O, LSE, dO up; dQ, dK, dV (and the factor gradients) down
+        host_g = [torch.empty(w.Q.shape, dtype=w.Q.dtype, pin_memory=True) for _ in range(3)]
+        host_gf = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (w.dpq, w.dpk) if t is not None]
+
+        def e2e_step():
+            w.Q.copy_(w.host_q, non_blocking=True)
+            w.K.copy_(w.host_k, non_blocking=True)
+            w.V.copy_(w.host_v, non_blocking=True)
+            w.O.copy_(w.host_o, non_blocking=True)
+            w.LSE.copy_(w.host_lse, non_blocking=True)
+            w.dO.copy_(w.host_do, non_blocking=True)
+            w.run_bwd()
+            for hb, t in zip(host_g, (w.dQ, w.dK, w.dV)):
+                hb.copy_(t, non_blocking=True)
+            for hb, t in zip(host_gf, [t for t in (w.dpq, w.dpk) if t is not None]):
+                hb.copy_(t, non_blocking=True)
+
     for _ in range(3):
         e2e_step()
     e2e_steps = max(5, min(args.steps, 50))
@@ -496,6 +561,9 @@ def run_ours(args, rank: int, world: int, local: int):
     barrier(world)
     h2d = 3 * w.Q.numel() * w.Q.element_size()
     d2h = w.O.numel() * w.O.element_size() + w.LSE.numel() * 4
+    if w.bwd:
+        h2d = 5 * w.Q.numel() * w.Q.element_size() + w.LSE.numel() * 4
+        d2h = 3 * w.Q.numel() * w.Q.element_size() + sum(t.numel() * 4 for t in (w.dpq, w.dpk) if t is not None)
 
     dense = None
     if w.dense is not None:
@@ -522,7 +590,7 @@ def run_ours(args, rank: int, world: int, local: int):
     peak_tf = sustained_tf if capped else burst_tf
     peak_kind = f"{peak_src} bf16 {'sustained (run power-capped)' if capped else 'burst'}"
     achieved = c["flops"] / (kern_ms * 1e-3) / 1e12
-    traffic = profiled_traffic(args.config)
+    traffic = None if w.bwd else profiled_traffic(args.config)
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
@@ -531,7 +599,9 @@ def run_ours(args, rank: int, world: int, local: int):
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": round(achieved / peak_tf, 4), "traffic": traffic,
                      "kernel": ("prep_mul_bias + attn_fwd_sm100" if w.mul else
-                                ("neural_factor + prep + attn_fwd_sm100" if w.neural else "attn_fwd_sm100")),
+                                ("neural_factor + prep + attn_fwd_sm100" if w.neural else
+                                 ("bwd preparation (3) + attn_bwd_dkdv_sm100 + attn_bwd_dq_sm100" if w.bwd
+                                  else "attn_fwd_sm100"))),
                      "peak_kind": peak_kind,
                      "kernel_ms": round(kern_ms, 5)},
         "e2e": {"value": round(c["flops"] * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
@@ -560,6 +630,19 @@ def oracle_sample(c: dict, step: int, rows_per_head: int):
     import oracle
     B, H, N, d, R = c["B"], c["H"], c["N"], c["d"], c["R"]
     b, h = (step // H) % B, step % H
+    if c.get("bwd"):
+        # the causal prefix of n tokens of one head is a complete causal
+        # problem of its own: every gradient of it, by the oracle's backward
+        n = min(N, rows_per_head)
+        q, k, v = (x[:n] for x in _head_inputs(c, b, h))
+        phi = oracle.sandwich_factors(n, R)
+        g = si.upstream_grad(B, H, N, d, si.DO_SEED_BASE + c["index"])[b, h, :n].astype(np.float64)
+        scale = 1.0 / math.sqrt(d)
+
+        def run_bwd():
+            oracle.attention_lowrank_bwd_head(q, k, v, phi, phi, g, scale, c["causal"])
+
+        return run_bwd, bwd_flops(1, 1, n, d, R, c["causal"]), f"causal prefix of {n} tokens of head (b={b}, h={h})"
     rng = si.generator(7000 + step)
     rows = np.sort(rng.choice(N, size=min(rows_per_head, N), replace=False)).astype(np.int64)
     q, k, v = _head_inputs(c, b, h)

@@ -279,7 +279,7 @@ def neural_factors(x_q, x_k, w_q, w_k):
     return np.einsum("bnf,hfr->bhnr", xq, wq), np.einsum("bnf,hfr->bhnr", xk, wk)
 
 
-def attention_lowrank_bwd_head(q, k, v, phi_q, phi_k, do, scale: float, causal: bool):
+def attention_lowrank_bwd_head(q, k, v, phi_q, phi_k, do, scale: float, causal: bool, rows=None):
     """Gradients of one head of O = softmax(scale q k^T + phi_q phi_k^T [causal]) v
     for an upstream gradient dO, in fp64 (the chain rule through the softmax,
     whole rows at once; library matmuls).
@@ -292,10 +292,25 @@ def attention_lowrank_bwd_head(q, k, v, phi_q, phi_k, do, scale: float, causal: 
         dV = P^T dO,  dP = dO v^T,  dS = P * (dP - rowsum(P * dP))
         dq = scale dS k,  dk = scale dS^T q,  dphi_q = dS phi_k,  dphi_k = dS^T phi_q.
     q, k, v, do [N, d]; phi_q, phi_k [N, R]. Returns a dict with dq, dk, dv,
-    dphi_q, dphi_k and the intermediate rowsum(P * dP) as ``delta``."""
+    dphi_q, dphi_k and the intermediate rowsum(P * dP) as ``delta``. With
+    ``rows`` (query indices) only the row-wise results dq, dphi_q and delta
+    of those queries are computed (a query row of dS needs only its own
+    score row)."""
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
     pq, pk = _f64(phi_q), _f64(phi_k)
     N = q.shape[0]
+    if rows is not None:
+        rows = np.asarray(rows, dtype=np.int64)
+        s = float(scale) * (q[rows] @ k.T) + pq[rows] @ pk.T
+        if causal:
+            s = np.where(np.arange(N)[None, :] <= rows[:, None], s, -np.inf)
+        m = np.max(s, axis=1, keepdims=True)
+        e = np.exp(s - m)
+        p = e / np.sum(e, axis=1, keepdims=True)
+        dp = do[rows] @ v.T
+        delta = np.sum(p * dp, axis=1, keepdims=True)
+        ds = p * (dp - delta)
+        return {"dq": float(scale) * (ds @ k), "dphi_q": ds @ pk, "delta": delta[:, 0]}
     s = float(scale) * (q @ k.T) + pq @ pk.T
     if causal:
         s = np.where(np.arange(N)[None, :] <= np.arange(N)[:, None], s, -np.inf)

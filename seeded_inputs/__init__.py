@@ -41,11 +41,15 @@ CONFIGS = [
     # pair-bias shape: a widening case, not a headline
     dict(index=6, name="af3_neural_F64_R32_N1536_d24", dtype="bf16", B=1, H=16, N=1536, d=24, R=32,
          causal=False, bias="neural", F=64),
+    # the backward (training) pass on the GPT-2 Sandwich shape: a widening case, not a headline
+    dict(index=7, name="gpt2_sandwich_bwd_N2048", dtype="bf16", B=8, H=12, N=2048, d=64, R=64,
+         causal=True, bias="sandwich", bwd=True),
 ]
 
 QKV_SEED_BASE = 1000
 FACTOR_SEED_BASE = 2000
 RBF_SEED_BASE = 3000
+DO_SEED_BASE = 4000
 
 
 def generator(seed: int) -> np.random.Generator:
@@ -211,3 +215,9 @@ def bf16_tensor(x: np.ndarray, device):
 def alibi_slope(h: int, H: int) -> float:
     """Slope of head h (0-based) of H in the ALiBi workload: 2^(-8(h+1)/H)."""
     return 2.0 ** (-8.0 * (h + 1) / H)
+
+
+def upstream_grad(B: int, H: int, N: int, d: int, seed: int) -> np.ndarray:
+    """dO ~ N(0, 1) rounded to bf16 values, fp32 [B, H, N, d] (the gradient a
+    loss hands to the attention output in the backward workload)."""
+    return round_to_bf16(normal((B, H, N, d), seed))

@@ -9,7 +9,7 @@ import pytest
 import oracle
 from oracle import HeadBias
 import seeded_inputs as si
-from gpu_util import compare, dev, host
+from gpu_util import compare, dev, grad_close, host
 
 pytestmark = pytest.mark.gpu
 
@@ -197,3 +197,39 @@ def test_config6_neural_full_size():
     rows = si.sample_rows(N, 40, 6)
     _check_rows(o, l, q, k, v, [(0, 0), (0, 7), (0, 15)], rows, lambda b, h: HeadBias.lowrank(pq[b, h], pk[b, h]),
                 scale, False, "bf16", "c6")
+
+
+def test_config7_backward_full_size():
+    """The backward workload (bench.py --config 7: GPT-2 Sandwich shape) at
+    full size through fb_attn_bwd. Every gradient of two whole heads against
+    the oracle; dphi_q (the Sandwich factor is shared by all 96 heads, so its
+    gradient sums over them) on sampled rows through the oracle's
+    row-restricted backward of every head; dphi_k by the zero column sums that
+    rows of dS summing to zero imply."""
+    c = si.CONFIGS[7]
+    B, H, N, d, R = c["B"], c["H"], c["N"], c["d"], c["R"]
+    q, k, v = si.qkv(B, H, N, d, si.QKV_SEED_BASE + 7, "bf16")
+    g = si.upstream_grad(B, H, N, d, si.DO_SEED_BASE + 7)
+    scale = 1.0 / math.sqrt(d)
+    Q, K, V, G = (dev(x, "bf16") for x in (q, k, v, g))
+    phi = fb.factors_sandwich(N, R)
+    o, l = fb.attn(Q, K, V, phi, phi, scale=scale, causal=True)
+    dq, dk, dv, dpq, dpk = fb.attn_bwd(Q, K, V, phi, phi, o, l, G, scale=scale, causal=True)
+    torch.cuda.synchronize()
+    assert fb.fb_check_device_error(_stream()) == fb.FB_OK
+    ph = oracle.sandwich_factors(N, R)
+    got = {"dq": host(dq), "dk": host(dk), "dv": host(dv)}
+    for (b, h) in [(0, 0), (B - 1, H - 1)]:
+        r = oracle.attention_lowrank_bwd_head(q[b, h], k[b, h], v[b, h], ph, ph, g[b, h], scale, True)
+        for n in ("dq", "dk", "dv"):
+            grad_close(got[n][b, h], r[n], f"c7 {n} ({b},{h})")
+    rows = si.sample_rows(N, 12, 7)
+    ref = np.zeros((len(rows), R))
+    for b in range(B):
+        for h in range(H):
+            ref += oracle.attention_lowrank_bwd_head(q[b, h], k[b, h], v[b, h], ph, ph, g[b, h], scale, True,
+                                                     rows=rows)["dphi_q"]
+    grad_close(host(dpq)[rows], ref, "c7 dphi_q rows")
+    gk = host(dpk)
+    assert np.all(np.isfinite(gk))
+    assert np.abs(gk.sum(axis=0)).max() <= 2e-2 * np.abs(gk).max() * math.sqrt(N), "c7 dphi_k column sums"

@@ -10,7 +10,7 @@ import pytest
 import oracle
 from oracle import HeadBias
 import seeded_inputs as si
-from gpu_util import compare, dev, host
+from gpu_util import compare, dev, grad_close, host
 
 pytestmark = pytest.mark.gpu
 
@@ -367,21 +367,6 @@ def test_neural_bias_matches_oracle(B, H, N, d, F, R, causal):
 
 # ---------------------------------------------------------------- backward
 
-def _grad_close(g, ref, what):
-    """Gradient tolerance: the forward's bf16 bound on O (max 2e-2, mean 2e-3
-    for values of order one) applied to the gradient scaled by its largest
-    reference magnitude, floored at 1e-3 for gradients that vanish exactly
-    (a single visible key makes dS zero; the kernel then returns rounding
-    noise of D = rowsum(dO * O) from the bf16 O)."""
-    g = np.asarray(g, np.float64)
-    assert np.all(np.isfinite(g)), f"{what}: non-finite gradient"
-    m = max(float(np.abs(ref).max()) if ref.size else 0.0, 1e-3)
-    err = np.abs(g - ref) / m
-    assert err.max() <= 2e-2, f"{what}: max rel {err.max():.3e}"
-    assert err.mean() <= 2e-3, f"{what}: mean rel {err.mean():.3e}"
-    return float(err.max()), float(err.mean())
-
-
 BWD_SWEEP = [
     # B, H, N, d, R, causal, factor layout
     (1, 2, 200, 64, 64, True, "bhnr"),
@@ -428,7 +413,7 @@ def test_backward_matches_oracle(B, H, N, d, R, causal, layout):
             r = oracle.attention_lowrank_bwd_head(q[b, h], k[b, h], v[b, h], fac(pq, b, h), fac(pk, b, h),
                                                   g[b, h], scale, causal)
             for n in ("dq", "dk", "dv"):
-                _grad_close(got[n][b, h], r[n], f"{n} ({b},{h}) B{B} H{H} N{N} d{d} R{R} c{causal}")
+                grad_close(got[n][b, h], r[n], f"{n} ({b},{h}) B{B} H{H} N{N} d{d} R{R} c{causal}")
             if R > 0:
                 for acc, key in ((ref_pq, "dphi_q"), (ref_pk, "dphi_k")):
                     if layout == "nr":
@@ -438,5 +423,5 @@ def test_backward_matches_oracle(B, H, N, d, R, causal, layout):
                     else:
                         acc[b, h] += r[key]
     if R > 0:
-        _grad_close(host(dpq), ref_pq, f"dphi_q B{B} H{H} N{N} d{d} R{R} {layout}")
-        _grad_close(host(dpk), ref_pk, f"dphi_k B{B} H{H} N{N} d{d} R{R} {layout}")
+        grad_close(host(dpq), ref_pq, f"dphi_q B{B} H{H} N{N} d{d} R{R} {layout}")
+        grad_close(host(dpk), ref_pk, f"dphi_k B{B} H{H} N{N} d{d} R{R} {layout}")

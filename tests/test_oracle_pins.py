@@ -408,3 +408,18 @@ def test_backward_invariants(causal):
     np.testing.assert_allclose(out["delta"], np.sum(o * g, axis=1), atol=1e-12)
     if causal:  # the first query sees only key 0: its dS row is zero
         np.testing.assert_allclose(out["dq"][0], 0.0, atol=1e-15)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_row_subset_matches_whole_head(causal):
+    """The row-restricted backward (dq, dphi_q, delta of chosen queries) is the
+    same computation on fewer score rows: it must agree with the whole head."""
+    N, d, R = 70, 8, 3
+    q, k, v = (_rand((N, d), s) for s in (61, 62, 63))
+    pq, pk = _rand((N, R), 64), _rand((N, R), 65)
+    g = _rand((N, d), 66)
+    full = oracle.attention_lowrank_bwd_head(q, k, v, pq, pk, g, 0.4, causal)
+    rows = np.array([0, 5, 33, 69])
+    part = oracle.attention_lowrank_bwd_head(q, k, v, pq, pk, g, 0.4, causal, rows=rows)
+    for key in ("dq", "dphi_q", "delta"):
+        np.testing.assert_allclose(part[key], full[key][rows], rtol=0, atol=1e-13)
