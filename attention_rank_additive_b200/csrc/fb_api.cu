@@ -569,8 +569,8 @@ int fb_attn_bwd(int dt, int B, int H, int N, int d, const void *Q, const void *K
   plan.mode = R == 0 ? kBiasNone : (R <= 4 ? kBiasTf32 : kBiasMma);
   plan.RP = plan.mode == kBiasMma ? pad_rank(R) : (plan.mode == kBiasTf32 ? tf32_cols(R) : 0);
   plan.RG = L.RG;
-  const int BQ = bwd_query_block_rows(plan);
-  if (BQ == 0) return FB_ERR_UNSUPPORTED;
+  const int BQ = bwd_query_block_rows(plan), BK = bwd_key_block_rows(plan);
+  if (BQ == 0 || BK == 0) return FB_ERR_UNSUPPORTED;
   int *flags = device_flags();
   if (!flags) return FB_ERR_CUDA;
 
@@ -599,15 +599,17 @@ int fb_attn_bwd(int dt, int B, int H, int N, int d, const void *Q, const void *K
   const int DP = plan.DP;
   if (!encode_rows_bf16(&maps.q, Q, BH, N, d, DP, 128) || !encode_rows_bf16(&maps.k, K, BH, N, d, DP, 128) ||
       !encode_rows_bf16(&maps.v, V, BH, N, d, DP, 128) || !encode_rows_bf16(&maps.dO, dO, BH, N, d, DP, 128) ||
-      !encode_rows_bf16(&maps.q_blk, Q, BH, N, d, DP, BQ) || !encode_rows_bf16(&maps.do_blk, dO, BH, N, d, DP, BQ))
+      !encode_rows_bf16(&maps.q_blk, Q, BH, N, d, DP, BQ) || !encode_rows_bf16(&maps.do_blk, dO, BH, N, d, DP, BQ) ||
+      !encode_rows_bf16(&maps.k_blk, K, BH, N, d, DP, BK) || !encode_rows_bf16(&maps.v_blk, V, BH, N, d, DP, BK))
     return FB_ERR_CUDA;
   if (R > 0) {
     void *wq = wsb + L.f.q_off, *wk = wsb + L.f.k_off;
     if (!encode_fac(&maps.fq, plan.mode, wq, FB, N, plan.RP, 128) ||
         !encode_fac(&maps.fk, plan.mode, wk, FB, N, plan.RP, 128) ||
         !encode_fac(&maps.fq_blk, plan.mode, wq, FB, N, plan.RP, BQ) ||
+        !encode_fac(&maps.fk_blk, plan.mode, wk, FB, N, plan.RP, BK) ||
         !encode_rows_bf16(&maps.gq_blk, wsb + L.gq_off, FB, N, L.RG, L.RG, BQ) ||
-        !encode_rows_bf16(&maps.gk, wsb + L.gk_off, FB, N, L.RG, L.RG, 128))
+        !encode_rows_bf16(&maps.gk_blk, wsb + L.gk_off, FB, N, L.RG, L.RG, BK))
       return FB_ERR_CUDA;
   }
   BwdArgs a;

@@ -17,20 +17,24 @@
 //
 // Two kernels, neither with atomics on the bf16 outputs:
 //   attn_bwd_dkdv_sm100  one CTA per (b, h, 128-key tile). The key tile K|phi_k
-//       and V stay in shared memory; query blocks of BQ rows (128, or 64 at
+//       and V stay in shared memory; query blocks of BQ rows (64, or 32 at
 //       head dim 128 so that TMEM holds everything) stream through a ring.
 //       Per block: S^T = K Q^T (+ phi_k' phi_q'^T), dP^T = V dO^T; the CUDA
 //       cores turn them into P^T and dS^T (bf16, written back over S^T and
 //       dP^T in TMEM); then dV += P^T dO, dK += dS^T Q, dphi_k += dS^T phi_q
 //       with the A operand read from TMEM and dO, Q, phi_q as MN-major B.
-//   attn_bwd_dq_sm100    one CTA per (b, h, 128-query tile): S = Q K^T (+ ...),
-//       dP = dO V^T, dS over S in TMEM, dQ += dS K, dphi_q += dS phi_k.
+//   attn_bwd_dq_sm100    one CTA per (b, h, 128-query tile), key blocks of 64:
+//       S = Q K^T (+ ...), dP = dO V^T, dS over S in TMEM, dQ += dS K,
+//       dphi_q += dS phi_k.
+// In both, two compute warpgroups take alternate blocks, each with its own
+// S and dP buffers in TMEM (ping-pong): while one turns its scores into P and
+// dS, the tensor core runs the other's products.
 // The factor gradients of a broadcast factor (stride 0) sum over the heads
 // and batches sharing it, so they are accumulated with fp32 reductions into
 // a buffer zeroed by the preparation step.
 //
-// CTA: warps 0-3 compute (one thread per TMEM lane = tile row), warp 4 TMA
-// producer, warp 5 TMEM allocator and MMA issuer. Every wait is bounded (the
+// CTA: warps 0-7 compute (two warpgroups, one thread per TMEM lane = tile
+// row in each), warp 8 TMA producer, warp 9 TMEM allocator and MMA issuer. Every wait is bounded (the
 // abort flag and the device flag word report a timeout).
 #include <algorithm>
 #include <atomic>
@@ -82,9 +86,14 @@ __host__ __device__ constexpr uint32_t mnstep(int kk) {
 
 template <int DP, int RP, int MODE, int RG>
 struct BwdCfg {
-  // Streamed block of the dK/dV kernel: 128 queries, or 64 at head dim 128
-  // (TMEM: S^T and dP^T BQ columns each, dV and dK DP each, dphi_k RG).
-  static constexpr int BQ = DP == 128 ? 64 : 128;
+  // Two compute warpgroups take alternate row blocks (ping-pong): each has
+  // its own S and dP buffers in TMEM, so the tensor core computes one
+  // block's scores while the CUDA cores turn the other's into P and dS.
+  // dK/dV kernel: streamed query blocks of BQ rows (32 at head dim 128 so
+  // that TMEM holds both buffers and the dV, dK, dphi_k accumulators).
+  static constexpr int BQ = DP == 128 ? 32 : 64;
+  // dQ kernel: streamed key blocks of BK rows.
+  static constexpr int BK = 64;
   static constexpr int DCH = DP > 64 ? 64 : DP;
   static constexpr int NDCH = DP / DCH;
   static constexpr bool FAC = MODE == kBiasMma || MODE == kBiasTf32;
@@ -97,40 +106,42 @@ struct BwdCfg {
   static constexpr int GCH = RG > 64 ? 64 : (RG > 0 ? RG : 16);
   static constexpr int NGCH = RG > 0 ? RG / GCH : 0;
   static constexpr uint32_t align1k(uint32_t x) { return (x + 1023u) & ~1023u; }
-  // dK/dV kernel
-  static constexpr uint32_t KV_FIXED = 2u * 128u * DP * 2u + (FAC ? 128u * RP * FESZ : 0u);
-  static constexpr uint32_t KV_STAGE =
-      align1k(2u * BQ * DP * 2u + (FAC ? BQ * RP * FESZ : 0u) + BQ * RG * 2u + 2u * BQ * 4u);
   static constexpr uint32_t CTRL = 1024;
   static constexpr uint32_t SLACK = 1024;
+  static constexpr int MAX_STAGES = 4;
+  // dK/dV kernel: fixed K, V, phi_k' tiles; per stage Q, dO, phi_q', phi_q (bf16), LSE2, D
+  static constexpr uint32_t KV_FIXED = 2u * 128u * DP * 2u + (FAC ? 128u * RP * FESZ : 0u);
+  static constexpr uint32_t KV_STAGE_BYTES =
+      2u * BQ * DP * 2u + (FAC ? BQ * RP * FESZ : 0u) + BQ * RG * 2u + 2u * BQ * 4u;
+  static constexpr uint32_t KV_STAGE = align1k(KV_STAGE_BYTES);
   static constexpr int KV_KS_FIT =
       kSmemLimitB > KV_FIXED + CTRL + SLACK ? int((kSmemLimitB - KV_FIXED - CTRL - SLACK) / KV_STAGE) : 0;
-  static constexpr int KV_KS = KV_KS_FIT > 2 ? 2 : KV_KS_FIT;
+  static constexpr int KV_KS = KV_KS_FIT > MAX_STAGES ? MAX_STAGES : KV_KS_FIT;
   static constexpr uint32_t KV_SMEM = KV_FIXED + uint32_t(KV_KS) * KV_STAGE + CTRL + SLACK;
-  // dQ kernel
+  // dQ kernel: fixed Q, dO, phi_q' tiles; per stage K, V, phi_k', phi_k (bf16)
   static constexpr uint32_t DQ_FIXED = 2u * 128u * DP * 2u + (FAC ? 128u * RP * FESZ : 0u);
-  static constexpr uint32_t DQ_STAGE_BYTES = 2u * 128u * DP * 2u + (FAC ? 128u * RP * FESZ : 0u) + 128u * RG * 2u;
+  static constexpr uint32_t DQ_STAGE_BYTES = 2u * BK * DP * 2u + (FAC ? BK * RP * FESZ : 0u) + BK * RG * 2u;
   static constexpr uint32_t DQ_STAGE = align1k(DQ_STAGE_BYTES);
   static constexpr int DQ_KS_FIT =
       kSmemLimitB > DQ_FIXED + CTRL + SLACK ? int((kSmemLimitB - DQ_FIXED - CTRL - SLACK) / DQ_STAGE) : 0;
-  static constexpr int DQ_KS = DQ_KS_FIT > 2 ? 2 : DQ_KS_FIT;
+  static constexpr int DQ_KS = DQ_KS_FIT > MAX_STAGES ? MAX_STAGES : DQ_KS_FIT;
   static constexpr uint32_t DQ_SMEM = DQ_FIXED + uint32_t(DQ_KS) * DQ_STAGE + CTRL + SLACK;
-  static constexpr int THREADS = 192;
-  static constexpr int PRODUCER_WARP = 4;
-  static constexpr int MMA_WARP = 5;
+  static constexpr int THREADS = 320;  // 2 compute warpgroups, producer warp, MMA warp
+  static constexpr int PRODUCER_WARP = 8;
+  static constexpr int MMA_WARP = 9;
   static constexpr uint32_t TMEM_COLS = 512;
-  // TMEM columns, dK/dV kernel
-  static constexpr uint32_t KV_S = 0, KV_DP = BQ, KV_DV = 2 * BQ, KV_DK = 2 * BQ + DP, KV_DF = 2 * BQ + 2 * DP;
+  // TMEM columns, dK/dV kernel: buffer t holds S^T at t 2BQ and dP^T at t 2BQ + BQ
+  static constexpr uint32_t KV_DV = 4 * BQ, KV_DK = 4 * BQ + DP, KV_DF = 4 * BQ + 2 * DP;
   static_assert(KV_DF + RG <= TMEM_COLS, "dK/dV TMEM layout");
-  // TMEM columns, dQ kernel
-  static constexpr uint32_t DQ_S = 0, DQ_DP = 128, DQ_DQ = 256, DQ_DF = 256 + DP;
+  // TMEM columns, dQ kernel: buffer t holds S at t 2BK and dP at t 2BK + BK
+  static constexpr uint32_t DQ_DQ = 4 * BK, DQ_DF = 4 * BK + DP;
   static_assert(DQ_DF + RG <= TMEM_COLS, "dQ TMEM layout");
   static constexpr uint32_t IDESC_KV_S = make_idesc_f16(true, true, 128, BQ, false);
   static constexpr uint32_t IDESC_KV_F =
       MODE == kBiasTf32 ? make_idesc_tf32(128, BQ) : make_idesc_f16(false, false, 128, BQ, false);
-  static constexpr uint32_t IDESC_DQ_S = make_idesc_f16(true, true, 128, 128, false);
+  static constexpr uint32_t IDESC_DQ_S = make_idesc_f16(true, true, 128, BK, false);
   static constexpr uint32_t IDESC_DQ_F =
-      MODE == kBiasTf32 ? make_idesc_tf32(128, 128) : make_idesc_f16(false, false, 128, 128, false);
+      MODE == kBiasTf32 ? make_idesc_tf32(128, BK) : make_idesc_f16(false, false, 128, BK, false);
   static constexpr uint32_t IDESC_GD = make_idesc_f16(true, true, 128, DP, true);
   static constexpr uint32_t IDESC_GR = make_idesc_f16(true, true, 128, RG > 0 ? RG : 16, true);
 };
@@ -139,8 +150,9 @@ namespace {
 
 struct BwdCtrl {
   uint64_t fixed_full;
-  uint64_t full[2], empty[2];
-  uint64_t s_full, p_full, acc_done;
+  uint64_t full[4], empty[4];
+  uint64_t s_full[2], p_full[2];
+  uint64_t acc_done;
   uint32_t tmem_base;
   int abort;
 };
@@ -160,7 +172,7 @@ __device__ __forceinline__ void store_row16_bf16(const uint32_t *r, float mul, u
 
 // ------------------------------------------------------------ dK, dV, dphi_k
 template <int DP, int RP, int MODE, int RG>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     attn_bwd_dkdv_sm100(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         const __grid_constant__ CUtensorMap tm_fk, const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_fq,
@@ -168,18 +180,19 @@ __global__ void __launch_bounds__(192, 1)
   using C = BwdCfg<DP, RP, MODE, RG>;
   constexpr int KS = C::KV_KS;
   constexpr int BQ = C::BQ;
-  static_assert(KS >= 1, "configuration does not fit in shared memory");
+  static_assert(KS >= 2, "configuration does not fit in shared memory");
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t *sK = smem;                                  // 128 x DP bf16
-  uint8_t *sV = sK + 128 * DP * 2;                     // 128 x DP bf16
-  uint8_t *sFK = sV + 128 * DP * 2;                    // 128 x RP (fp16 / fp32)
-  uint8_t *sStage = smem + C::KV_FIXED;                // KS x KV_STAGE
+  uint8_t *sK = smem;                    // 128 x DP bf16
+  uint8_t *sV = sK + 128 * DP * 2;       // 128 x DP bf16
+  uint8_t *sFK = sV + 128 * DP * 2;      // 128 x RP (fp16 / fp32)
+  uint8_t *sStage = smem + C::KV_FIXED;  // KS x KV_STAGE
   BwdCtrl *ctrl = reinterpret_cast<BwdCtrl *>(sStage + KS * C::KV_STAGE);
   // offsets inside a stage
   constexpr uint32_t O_Q = 0, O_DO = BQ * DP * 2, O_FQ = 2 * BQ * DP * 2;
   constexpr uint32_t O_GQ = O_FQ + (C::FAC ? BQ * RP * C::FESZ : 0);
   constexpr uint32_t O_L = O_GQ + BQ * RG * 2, O_D = O_L + BQ * 4;
+  static_assert(O_D + BQ * 4 == C::KV_STAGE_BYTES, "stage layout");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int BH = args.B * args.H;
@@ -188,8 +201,8 @@ __global__ void __launch_bounds__(192, 1)
   const int b = bh / args.H, h = bh % args.H;
   const int k0 = kb * 128;
   const int fslice = (args.fac_B > 1 ? b : 0) * args.fac_H + (args.fac_H > 1 ? h : 0);
-  const int n_blk = (args.N + BQ - 1) / BQ;
   const int j0 = args.causal ? k0 / BQ : 0;  // query blocks before the diagonal see none of these keys
+  const int nb = (args.N + BQ - 1) / BQ - j0;  // >= 1
 
   if (threadIdx.x == 0) {
     mbar_init(&ctrl->fixed_full, 1);
@@ -197,8 +210,10 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&ctrl->full[s], 1);
       mbar_init(&ctrl->empty[s], 1);
     }
-    mbar_init(&ctrl->s_full, 1);
-    mbar_init(&ctrl->p_full, 128);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&ctrl->s_full[t], 1);
+      mbar_init(&ctrl->p_full[t], 128);
+    }
     mbar_init(&ctrl->acc_done, 1);
     ctrl->abort = 0;
     fence_mbar_init();
@@ -237,14 +252,12 @@ __global__ void __launch_bounds__(192, 1)
         tma_load_3d_leader(sFK + ch * (128 * C::FCH * 2), &tm_fk, &ctrl->fixed_full, ch * C::FCH, k0, fslice,
                            leader);
     bool ok = true;
-    int it = 0;
-    for (int j = j0; j < n_blk; ++j, ++it) {
-      const int s = it % KS;
-      const uint32_t ph = uint32_t(it / KS) & 1u;
-      if (it >= KS && !(ok = mbar_wait(&ctrl->empty[s], ph ^ 1u, abort))) break;
+    for (int u = 0; u < nb; ++u) {
+      const int s = u % KS;
+      if (u >= KS && !(ok = mbar_wait(&ctrl->empty[s], (uint32_t(u / KS) & 1u) ^ 1u, abort))) break;
       uint8_t *st = sStage + s * C::KV_STAGE;
-      const int q0 = j * BQ;
-      mbar_arrive_expect_tx_leader(&ctrl->full[s], O_D + BQ * 4, leader);
+      const int q0 = (j0 + u) * BQ;
+      mbar_arrive_expect_tx_leader(&ctrl->full[s], C::KV_STAGE_BYTES, leader);
       for (int ch = 0; ch < C::NDCH; ++ch) {
         tma_load_3d_leader(st + O_Q + ch * (BQ * C::DCH * 2), &tm_q, &ctrl->full[s], ch * C::DCH, q0, bh, leader);
         tma_load_3d_leader(st + O_DO + ch * (BQ * C::DCH * 2), &tm_do, &ctrl->full[s], ch * C::DCH, q0, bh, leader);
@@ -271,71 +284,77 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == C::MMA_WARP) {
     // ---------------------------------------------------------- MMA issuer
+    // Order: S(0), S(1), G(0), S(2), G(1), S(3), ... where S(u) computes the
+    // scores of block u into buffer u & 1 and G(u) the gradient products of
+    // block u from that buffer; S(u + 2) follows G(u) (tcgen05 MMAs of one
+    // thread run in order), so it overwrites P and dS only after their use.
     const uint32_t tm_u = __shfl_sync(0xffffffffu, tmem, 0);
     bool ok = __all_sync(0xffffffffu, mbar_wait(&ctrl->fixed_full, 0, abort));  // warp-uniform for elect.sync
     tc_fence_after();
     const uint64_t dK = kdesc<C::DCH>(smem_u32(sK));
     const uint64_t dV = kdesc<C::DCH>(smem_u32(sV));
     const uint64_t dFK = kdesc<C::FCH>(smem_u32(sFK));
-    int it = 0;
-    for (int j = j0; j < n_blk && ok; ++j, ++it) {
-      const int s = it % KS;
-      const uint32_t ph = uint32_t(it / KS) & 1u;
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&ctrl->full[s], ph, abort)))) break;
+    auto issue_s = [&](int u) -> bool {
+      const int s = u % KS;
+      if (!__all_sync(0xffffffffu, mbar_wait(&ctrl->full[s], uint32_t(u / KS) & 1u, abort))) return false;
       tc_fence_after();
       const uint32_t st = smem_u32(sStage + s * C::KV_STAGE);
-      // S^T = K Q^T (+ phi_k' phi_q'^T), dP^T = V dO^T
-      {
-        uint64_t dq = kdesc<C::DCH>(st + O_Q), ddo = kdesc<C::DCH>(st + O_DO);
-        asm volatile("" : "+l"(dq), "+l"(ddo));
+      const uint32_t s_col = tm_u + uint32_t((u & 1) * 2 * BQ);
+      uint64_t dq = kdesc<C::DCH>(st + O_Q), ddo = kdesc<C::DCH>(st + O_DO);
+      asm volatile("" : "+l"(dq), "+l"(ddo));
 #pragma unroll
-        for (int kk = 0; kk < DP / 16; ++kk)
-          mma_ss_elect(tm_u + C::KV_S, dK + kstep<C::DCH, 128>(kk), dq + kstep<C::DCH, BQ>(kk), C::IDESC_KV_S,
-                       kk > 0 ? 1u : 0u);
-        if constexpr (C::FAC) {
-          uint64_t dfq = kdesc<C::FCH>(st + O_FQ);
-          asm volatile("" : "+l"(dfq));
+      for (int kk = 0; kk < DP / 16; ++kk)  // S^T = K Q^T
+        mma_ss_elect(s_col, dK + kstep<C::DCH, 128>(kk), dq + kstep<C::DCH, BQ>(kk), C::IDESC_KV_S, kk > 0 ? 1u : 0u);
+      if constexpr (C::FAC) {  // S^T += phi_k' phi_q'^T
+        uint64_t dfq = kdesc<C::FCH>(st + O_FQ);
+        asm volatile("" : "+l"(dfq));
 #pragma unroll
-          for (int kk = 0; kk < C::FCH * C::NFCH / 16; ++kk) {
-            if (MODE == kBiasTf32)
-              mma_ss_elect_tf32(tm_u + C::KV_S, dFK + kstep<C::FCH, 128>(kk), dfq + kstep<C::FCH, BQ>(kk),
-                                C::IDESC_KV_F, 1u);
-            else
-              mma_ss_elect(tm_u + C::KV_S, dFK + kstep<C::FCH, 128>(kk), dfq + kstep<C::FCH, BQ>(kk),
-                           C::IDESC_KV_F, 1u);
-          }
+        for (int kk = 0; kk < C::FCH * C::NFCH / 16; ++kk) {
+          if (MODE == kBiasTf32)
+            mma_ss_elect_tf32(s_col, dFK + kstep<C::FCH, 128>(kk), dfq + kstep<C::FCH, BQ>(kk), C::IDESC_KV_F, 1u);
+          else
+            mma_ss_elect(s_col, dFK + kstep<C::FCH, 128>(kk), dfq + kstep<C::FCH, BQ>(kk), C::IDESC_KV_F, 1u);
         }
-#pragma unroll
-        for (int kk = 0; kk < DP / 16; ++kk)
-          mma_ss_elect(tm_u + C::KV_DP, dV + kstep<C::DCH, 128>(kk), ddo + kstep<C::DCH, BQ>(kk), C::IDESC_KV_S,
-                       kk > 0 ? 1u : 0u);
       }
-      tc_commit_elect(&ctrl->s_full);
+#pragma unroll
+      for (int kk = 0; kk < DP / 16; ++kk)  // dP^T = V dO^T
+        mma_ss_elect(s_col + BQ, dV + kstep<C::DCH, 128>(kk), ddo + kstep<C::DCH, BQ>(kk), C::IDESC_KV_S,
+                     kk > 0 ? 1u : 0u);
+      tc_commit_elect(&ctrl->s_full[u & 1]);
       __syncwarp();
-      // P^T and dS^T are in TMEM (bf16 over the first BQ/2 columns of S^T and dP^T)
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&ctrl->p_full, uint32_t(it) & 1u, abort)))) break;
+      return true;
+    };
+    auto issue_g = [&](int u) -> bool {
+      if (!__all_sync(0xffffffffu, mbar_wait(&ctrl->p_full[u & 1], uint32_t(u >> 1) & 1u, abort))) return false;
       tc_fence_after();
-      {
-        uint64_t bdo = mndesc<C::DCH, BQ>(st + O_DO), bq = mndesc<C::DCH, BQ>(st + O_Q);
-        asm volatile("" : "+l"(bdo), "+l"(bq));
+      const int s = u % KS;
+      const uint32_t st = smem_u32(sStage + s * C::KV_STAGE);
+      const uint32_t p_col = tm_u + uint32_t((u & 1) * 2 * BQ);  // P^T bf16 over S^T; dS^T over dP^T
+      uint64_t bdo = mndesc<C::DCH, BQ>(st + O_DO), bq = mndesc<C::DCH, BQ>(st + O_Q);
+      asm volatile("" : "+l"(bdo), "+l"(bq));
 #pragma unroll
-        for (int kk = 0; kk < BQ / 16; ++kk) {
-          const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-          mma_ts_elect(tm_u + C::KV_DV, tm_u + C::KV_S + uint32_t(kk * 8), bdo + mnstep<C::DCH>(kk), C::IDESC_GD, acc);
-          mma_ts_elect(tm_u + C::KV_DK, tm_u + C::KV_DP + uint32_t(kk * 8), bq + mnstep<C::DCH>(kk), C::IDESC_GD,
-                       acc);
-        }
-        if constexpr (RG > 0) {
-          uint64_t bg = mndesc<C::GCH, BQ>(st + O_GQ);
-          asm volatile("" : "+l"(bg));
+      for (int kk = 0; kk < BQ / 16; ++kk) {
+        const uint32_t acc = (u > 0 || kk > 0) ? 1u : 0u;
+        mma_ts_elect(tm_u + C::KV_DV, p_col + uint32_t(kk * 8), bdo + mnstep<C::DCH>(kk), C::IDESC_GD, acc);
+        mma_ts_elect(tm_u + C::KV_DK, p_col + BQ + uint32_t(kk * 8), bq + mnstep<C::DCH>(kk), C::IDESC_GD, acc);
+      }
+      if constexpr (RG > 0) {
+        uint64_t bg = mndesc<C::GCH, BQ>(st + O_GQ);
+        asm volatile("" : "+l"(bg));
 #pragma unroll
-          for (int kk = 0; kk < BQ / 16; ++kk)
-            mma_ts_elect(tm_u + C::KV_DF, tm_u + C::KV_DP + uint32_t(kk * 8), bg + mnstep<C::GCH>(kk), C::IDESC_GR,
-                         (it > 0 || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < BQ / 16; ++kk)
+          mma_ts_elect(tm_u + C::KV_DF, p_col + BQ + uint32_t(kk * 8), bg + mnstep<C::GCH>(kk), C::IDESC_GR,
+                       (u > 0 || kk > 0) ? 1u : 0u);
       }
       tc_commit_elect(&ctrl->empty[s]);
       __syncwarp();
+      return true;
+    };
+    if (ok) ok = issue_s(0);
+    if (ok && nb > 1) ok = issue_s(1);
+    for (int u = 0; u < nb && ok; ++u) {
+      ok = issue_g(u);
+      if (ok && u + 2 < nb) ok = issue_s(u + 2);
     }
     if (ok) {
       tc_commit_elect(&ctrl->acc_done);
@@ -343,17 +362,19 @@ __global__ void __launch_bounds__(192, 1)
     }
     if (!ok && leader) atomicOr(args.flags, kFlagTimeout);
   } else {
-    // ------------------------------------------------ compute (warps 0-3)
-    const int r_loc = warp * 32 + lane;
+    // ------------------------------- compute: warpgroup t takes blocks u = t mod 2
+    const int t = warp >> 2, quarter = warp & 3;
+    const int r_loc = quarter * 32 + lane;
     const int krow = k0 + r_loc;  // this thread's key
-    const uint32_t lane_base = tmem + (uint32_t(warp * 32) << 16);
+    const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
+    const uint32_t s_tm = lane_base + uint32_t(t * 2 * BQ), dp_tm = s_tm + BQ;
     const float sl2 = args.scale_log2;
     bool ok = true;
-    int it = 0;
-    for (int j = j0; j < n_blk; ++j, ++it) {
-      const int s = it % KS;
+    for (int u = t; u < nb; u += 2) {
+      const int s = u % KS;
       // the whole warp leaves together: the TMEM accesses below are warp-collective
-      ok = mbar_wait(&ctrl->full[s], uint32_t(it / KS) & 1u, abort) && mbar_wait(&ctrl->s_full, uint32_t(it) & 1u, abort);
+      ok = mbar_wait(&ctrl->full[s], uint32_t(u / KS) & 1u, abort) &&
+           mbar_wait(&ctrl->s_full[t], uint32_t(u >> 1) & 1u, abort);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
@@ -362,13 +383,13 @@ __global__ void __launch_bounds__(192, 1)
       const uint8_t *st = sStage + s * C::KV_STAGE;
       const float *sL = reinterpret_cast<const float *>(st + O_L);
       const float *sD = reinterpret_cast<const float *>(st + O_D);
-      const int q0 = j * BQ;
+      const int q0 = (j0 + u) * BQ;
       const bool diag = args.causal && q0 < k0 + 127;  // some query of the block precedes some key
-#pragma unroll 1
+#pragma unroll
       for (int c = 0; c < BQ / 32; ++c) {
         uint32_t sx[32], dx[32];
-        tmem_ld32(lane_base + C::KV_S + uint32_t(32 * c), sx);
-        tmem_ld32(lane_base + C::KV_DP + uint32_t(32 * c), dx);
+        tmem_ld32(s_tm + uint32_t(32 * c), sx);
+        tmem_ld32(dp_tm + uint32_t(32 * c), dx);
         tmem_ld_wait32(sx);
         tmem_ld_wait32(dx);
         uint32_t pp[16], dd[16];
@@ -390,44 +411,46 @@ __global__ void __launch_bounds__(192, 1)
           dd[2 * e4] = pack_bf16x2(g[0], g[1]);
           dd[2 * e4 + 1] = pack_bf16x2(g[2], g[3]);
         }
-        tmem_st16(lane_base + C::KV_S + uint32_t(16 * c), pp);
-        tmem_st16(lane_base + C::KV_DP + uint32_t(16 * c), dd);
+        tmem_st16(s_tm + uint32_t(16 * c), pp);
+        tmem_st16(dp_tm + uint32_t(16 * c), dd);
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&ctrl->p_full);
+      mbar_arrive(&ctrl->p_full[t]);
     }
     if (ok) ok = mbar_wait(&ctrl->acc_done, 0, abort);
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
+      // epilogue: warpgroup 0 writes dV and dphi_k, warpgroup 1 dK. TMEM loads
+      // are warp-collective: every lane loads, rows past N store nothing.
       tc_fence_after();
-      // TMEM loads are warp-collective: every lane loads, rows past N store nothing
       const bool valid = krow < args.N;
       const int d_st = valid ? args.d : 0;
-      uint16_t *dv_row = static_cast<uint16_t *>(args.dV) + (size_t(bh) * args.N + (valid ? krow : 0)) * args.d;
-      uint16_t *dk_row = static_cast<uint16_t *>(args.dK) + (size_t(bh) * args.N + (valid ? krow : 0)) * args.d;
+      const size_t row_off = (size_t(bh) * args.N + (valid ? krow : 0)) * args.d;
+      uint16_t *dst = static_cast<uint16_t *>(t == 0 ? args.dV : args.dK) + row_off;
+      const uint32_t acc_tm = lane_base + (t == 0 ? C::KV_DV : C::KV_DK);
+      const float mul = t == 0 ? 1.f : args.scale;
 #pragma unroll 1
       for (int c0 = 0; c0 < DP; c0 += 16) {
         uint32_t r[16];
-        tmem_ld16(lane_base + C::KV_DV + uint32_t(c0), r);
+        tmem_ld16(acc_tm + uint32_t(c0), r);
         tmem_ld_wait16(r);
-        store_row16_bf16(r, 1.f, dv_row, c0, d_st);
-        tmem_ld16(lane_base + C::KV_DK + uint32_t(c0), r);
-        tmem_ld_wait16(r);
-        store_row16_bf16(r, args.scale, dk_row, c0, d_st);
+        store_row16_bf16(r, mul, dst, c0, d_st);
       }
       if constexpr (RG > 0) {
-        const int r_st = valid ? args.R : 0;
-        float *df = args.dphi_k + (args.fac_B > 1 ? int64_t(b) * args.phi_bs : 0) +
-                    (args.fac_H > 1 ? int64_t(h) * args.phi_hs : 0) + int64_t(valid ? krow : 0) * args.R;
+        if (t == 0) {
+          const int r_st = valid ? args.R : 0;
+          float *df = args.dphi_k + (args.fac_B > 1 ? int64_t(b) * args.phi_bs : 0) +
+                      (args.fac_H > 1 ? int64_t(h) * args.phi_hs : 0) + int64_t(valid ? krow : 0) * args.R;
 #pragma unroll 1
-        for (int c0 = 0; c0 < RG; c0 += 16) {
-          uint32_t r[16];
-          tmem_ld16(lane_base + C::KV_DF + uint32_t(c0), r);
-          tmem_ld_wait16(r);
+          for (int c0 = 0; c0 < RG; c0 += 16) {
+            uint32_t r[16];
+            tmem_ld16(lane_base + C::KV_DF + uint32_t(c0), r);
+            tmem_ld_wait16(r);
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            if (c0 + e < r_st) atomicAdd(df + c0 + e, __uint_as_float(r[e]));
+            for (int e = 0; e < 16; ++e)
+              if (c0 + e < r_st) atomicAdd(df + c0 + e, __uint_as_float(r[e]));
+          }
         }
       }
     }
@@ -444,14 +467,15 @@ __global__ void __launch_bounds__(192, 1)
 
 // ------------------------------------------------------------------ dQ, dphi_q
 template <int DP, int RP, int MODE, int RG>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     attn_bwd_dq_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                       const __grid_constant__ CUtensorMap tm_fq, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_fk,
                       const __grid_constant__ CUtensorMap tm_gk, const BwdArgs args) {
   using C = BwdCfg<DP, RP, MODE, RG>;
   constexpr int KS = C::DQ_KS;
-  static_assert(KS >= 1, "configuration does not fit in shared memory");
+  constexpr int BK = C::BK;
+  static_assert(KS >= 2, "configuration does not fit in shared memory");
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sQ = smem;                    // 128 x DP bf16
@@ -459,8 +483,9 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t *sFQ = sDO + 128 * DP * 2;     // 128 x RP (fp16 / fp32)
   uint8_t *sStage = smem + C::DQ_FIXED;  // KS x DQ_STAGE
   BwdCtrl *ctrl = reinterpret_cast<BwdCtrl *>(sStage + KS * C::DQ_STAGE);
-  constexpr uint32_t O_K = 0, O_V = 128 * DP * 2, O_FK = 2 * 128 * DP * 2;
-  constexpr uint32_t O_GK = O_FK + (C::FAC ? 128 * RP * C::FESZ : 0);
+  constexpr uint32_t O_K = 0, O_V = BK * DP * 2, O_FK = 2 * BK * DP * 2;
+  constexpr uint32_t O_GK = O_FK + (C::FAC ? BK * RP * C::FESZ : 0);
+  static_assert(O_GK + BK * RG * 2 == C::DQ_STAGE_BYTES, "stage layout");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int BH = args.B * args.H;
@@ -469,7 +494,9 @@ __global__ void __launch_bounds__(192, 1)
   const int b = bh / args.H, h = bh % args.H;
   const int q0 = qb * 128;
   const int fslice = (args.fac_B > 1 ? b : 0) * args.fac_H + (args.fac_H > 1 ? h : 0);
-  const int nk = args.causal ? qb + 1 : args.n_kv;  // key tiles this query tile sees
+  // key blocks this query tile sees: keys [0, min(q0 + 128, N)) when causal
+  const int key_end = args.causal ? min(q0 + 128, args.N) : args.N;
+  const int nb = (key_end + BK - 1) / BK;
 
   if (threadIdx.x == 0) {
     mbar_init(&ctrl->fixed_full, 1);
@@ -477,8 +504,10 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&ctrl->full[s], 1);
       mbar_init(&ctrl->empty[s], 1);
     }
-    mbar_init(&ctrl->s_full, 1);
-    mbar_init(&ctrl->p_full, 128);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&ctrl->s_full[t], 1);
+      mbar_init(&ctrl->p_full[t], 128);
+    }
     mbar_init(&ctrl->acc_done, 1);
     ctrl->abort = 0;
     fence_mbar_init();
@@ -517,23 +546,22 @@ __global__ void __launch_bounds__(192, 1)
         tma_load_3d_leader(sFQ + ch * (128 * C::FCH * 2), &tm_fq, &ctrl->fixed_full, ch * C::FCH, q0, fslice,
                            leader);
     bool ok = true;
-    for (int i = 0; i < nk; ++i) {
-      const int s = i % KS;
-      const uint32_t ph = uint32_t(i / KS) & 1u;
-      if (i >= KS && !(ok = mbar_wait(&ctrl->empty[s], ph ^ 1u, abort))) break;
+    for (int u = 0; u < nb; ++u) {
+      const int s = u % KS;
+      if (u >= KS && !(ok = mbar_wait(&ctrl->empty[s], (uint32_t(u / KS) & 1u) ^ 1u, abort))) break;
       uint8_t *st = sStage + s * C::DQ_STAGE;
-      const int kv = i * 128;
+      const int kv = u * BK;
       mbar_arrive_expect_tx_leader(&ctrl->full[s], C::DQ_STAGE_BYTES, leader);
       for (int ch = 0; ch < C::NDCH; ++ch) {
-        tma_load_3d_leader(st + O_K + ch * (128 * C::DCH * 2), &tm_k, &ctrl->full[s], ch * C::DCH, kv, bh, leader);
-        tma_load_3d_leader(st + O_V + ch * (128 * C::DCH * 2), &tm_v, &ctrl->full[s], ch * C::DCH, kv, bh, leader);
+        tma_load_3d_leader(st + O_K + ch * (BK * C::DCH * 2), &tm_k, &ctrl->full[s], ch * C::DCH, kv, bh, leader);
+        tma_load_3d_leader(st + O_V + ch * (BK * C::DCH * 2), &tm_v, &ctrl->full[s], ch * C::DCH, kv, bh, leader);
       }
       if (C::FAC)
         for (int ch = 0; ch < C::NFCH; ++ch)
-          tma_load_3d_leader(st + O_FK + ch * (128 * C::FCH * 2), &tm_fk, &ctrl->full[s], ch * C::FCH, kv, fslice,
+          tma_load_3d_leader(st + O_FK + ch * (BK * C::FCH * 2), &tm_fk, &ctrl->full[s], ch * C::FCH, kv, fslice,
                              leader);
       for (int ch = 0; ch < C::NGCH; ++ch)
-        tma_load_3d_leader(st + O_GK + ch * (128 * C::GCH * 2), &tm_gk, &ctrl->full[s], ch * C::GCH, kv, fslice,
+        tma_load_3d_leader(st + O_GK + ch * (BK * C::GCH * 2), &tm_gk, &ctrl->full[s], ch * C::GCH, kv, fslice,
                            leader);
     }
     if (!ok) {
@@ -546,64 +574,72 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == C::MMA_WARP) {
     // ---------------------------------------------------------- MMA issuer
+    // S(0), S(1), G(0), S(2), G(1), ... as in the dK/dV kernel.
     const uint32_t tm_u = __shfl_sync(0xffffffffu, tmem, 0);
-    bool ok = __all_sync(0xffffffffu, mbar_wait(&ctrl->fixed_full, 0, abort));  // warp-uniform for elect.sync
+    bool ok = __all_sync(0xffffffffu, mbar_wait(&ctrl->fixed_full, 0, abort));
     tc_fence_after();
     const uint64_t aQ = kdesc<C::DCH>(smem_u32(sQ));
     const uint64_t aDO = kdesc<C::DCH>(smem_u32(sDO));
     const uint64_t aFQ = kdesc<C::FCH>(smem_u32(sFQ));
-    for (int i = 0; i < nk && ok; ++i) {
-      const int s = i % KS;
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&ctrl->full[s], uint32_t(i / KS) & 1u, abort)))) break;
+    auto issue_s = [&](int u) -> bool {
+      const int s = u % KS;
+      if (!__all_sync(0xffffffffu, mbar_wait(&ctrl->full[s], uint32_t(u / KS) & 1u, abort))) return false;
       tc_fence_after();
       const uint32_t st = smem_u32(sStage + s * C::DQ_STAGE);
-      {  // S = Q K^T (+ phi_q' phi_k'^T), dP = dO V^T
-        uint64_t bk = kdesc<C::DCH>(st + O_K), bv = kdesc<C::DCH>(st + O_V);
-        asm volatile("" : "+l"(bk), "+l"(bv));
+      const uint32_t s_col = tm_u + uint32_t((u & 1) * 2 * BK);
+      uint64_t bk = kdesc<C::DCH>(st + O_K), bv = kdesc<C::DCH>(st + O_V);
+      asm volatile("" : "+l"(bk), "+l"(bv));
 #pragma unroll
-        for (int kk = 0; kk < DP / 16; ++kk)
-          mma_ss_elect(tm_u + C::DQ_S, aQ + kstep<C::DCH, 128>(kk), bk + kstep<C::DCH, 128>(kk), C::IDESC_DQ_S,
-                       kk > 0 ? 1u : 0u);
-        if constexpr (C::FAC) {
-          uint64_t bfk = kdesc<C::FCH>(st + O_FK);
-          asm volatile("" : "+l"(bfk));
+      for (int kk = 0; kk < DP / 16; ++kk)  // S = Q K^T
+        mma_ss_elect(s_col, aQ + kstep<C::DCH, 128>(kk), bk + kstep<C::DCH, BK>(kk), C::IDESC_DQ_S, kk > 0 ? 1u : 0u);
+      if constexpr (C::FAC) {  // S += phi_q' phi_k'^T
+        uint64_t bfk = kdesc<C::FCH>(st + O_FK);
+        asm volatile("" : "+l"(bfk));
 #pragma unroll
-          for (int kk = 0; kk < C::FCH * C::NFCH / 16; ++kk) {
-            if (MODE == kBiasTf32)
-              mma_ss_elect_tf32(tm_u + C::DQ_S, aFQ + kstep<C::FCH, 128>(kk), bfk + kstep<C::FCH, 128>(kk),
-                                C::IDESC_DQ_F, 1u);
-            else
-              mma_ss_elect(tm_u + C::DQ_S, aFQ + kstep<C::FCH, 128>(kk), bfk + kstep<C::FCH, 128>(kk),
-                           C::IDESC_DQ_F, 1u);
-          }
+        for (int kk = 0; kk < C::FCH * C::NFCH / 16; ++kk) {
+          if (MODE == kBiasTf32)
+            mma_ss_elect_tf32(s_col, aFQ + kstep<C::FCH, 128>(kk), bfk + kstep<C::FCH, BK>(kk), C::IDESC_DQ_F, 1u);
+          else
+            mma_ss_elect(s_col, aFQ + kstep<C::FCH, 128>(kk), bfk + kstep<C::FCH, BK>(kk), C::IDESC_DQ_F, 1u);
         }
-#pragma unroll
-        for (int kk = 0; kk < DP / 16; ++kk)
-          mma_ss_elect(tm_u + C::DQ_DP, aDO + kstep<C::DCH, 128>(kk), bv + kstep<C::DCH, 128>(kk), C::IDESC_DQ_S,
-                       kk > 0 ? 1u : 0u);
       }
-      tc_commit_elect(&ctrl->s_full);
+#pragma unroll
+      for (int kk = 0; kk < DP / 16; ++kk)  // dP = dO V^T
+        mma_ss_elect(s_col + BK, aDO + kstep<C::DCH, 128>(kk), bv + kstep<C::DCH, BK>(kk), C::IDESC_DQ_S,
+                     kk > 0 ? 1u : 0u);
+      tc_commit_elect(&ctrl->s_full[u & 1]);
       __syncwarp();
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&ctrl->p_full, uint32_t(i) & 1u, abort)))) break;
+      return true;
+    };
+    auto issue_g = [&](int u) -> bool {
+      if (!__all_sync(0xffffffffu, mbar_wait(&ctrl->p_full[u & 1], uint32_t(u >> 1) & 1u, abort))) return false;
       tc_fence_after();
-      {  // dQ += dS K, dphi_q += dS phi_k (dS bf16 over the first 64 columns of S)
-        uint64_t bk = mndesc<C::DCH, 128>(st + O_K);
-        asm volatile("" : "+l"(bk));
+      const int s = u % KS;
+      const uint32_t st = smem_u32(sStage + s * C::DQ_STAGE);
+      const uint32_t ds_col = tm_u + uint32_t((u & 1) * 2 * BK);  // dS bf16 over S
+      uint64_t bk = mndesc<C::DCH, BK>(st + O_K);
+      asm volatile("" : "+l"(bk));
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts_elect(tm_u + C::DQ_DQ, tm_u + C::DQ_S + uint32_t(kk * 8), bk + mnstep<C::DCH>(kk), C::IDESC_GD,
-                       (i > 0 || kk > 0) ? 1u : 0u);
-        if constexpr (RG > 0) {
-          uint64_t bg = mndesc<C::GCH, 128>(st + O_GK);
-          asm volatile("" : "+l"(bg));
+      for (int kk = 0; kk < BK / 16; ++kk)  // dQ += dS K
+        mma_ts_elect(tm_u + C::DQ_DQ, ds_col + uint32_t(kk * 8), bk + mnstep<C::DCH>(kk), C::IDESC_GD,
+                     (u > 0 || kk > 0) ? 1u : 0u);
+      if constexpr (RG > 0) {  // dphi_q += dS phi_k
+        uint64_t bg = mndesc<C::GCH, BK>(st + O_GK);
+        asm volatile("" : "+l"(bg));
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts_elect(tm_u + C::DQ_DF, tm_u + C::DQ_S + uint32_t(kk * 8), bg + mnstep<C::GCH>(kk), C::IDESC_GR,
-                         (i > 0 || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < BK / 16; ++kk)
+          mma_ts_elect(tm_u + C::DQ_DF, ds_col + uint32_t(kk * 8), bg + mnstep<C::GCH>(kk), C::IDESC_GR,
+                       (u > 0 || kk > 0) ? 1u : 0u);
       }
       tc_commit_elect(&ctrl->empty[s]);
       __syncwarp();
+      return true;
+    };
+    if (ok) ok = issue_s(0);
+    if (ok && nb > 1) ok = issue_s(1);
+    for (int u = 0; u < nb && ok; ++u) {
+      ok = issue_g(u);
+      if (ok && u + 2 < nb) ok = issue_s(u + 2);
     }
     if (ok) {
       tc_commit_elect(&ctrl->acc_done);
@@ -611,29 +647,31 @@ __global__ void __launch_bounds__(192, 1)
     }
     if (!ok && leader) atomicOr(args.flags, kFlagTimeout);
   } else {
-    // ------------------------------------------------ compute (warps 0-3)
-    const int r_loc = warp * 32 + lane;
+    // ------------------------------- compute: warpgroup t takes blocks u = t mod 2
+    const int t = warp >> 2, quarter = warp & 3;
+    const int r_loc = quarter * 32 + lane;
     const int row = q0 + r_loc;  // this thread's query
-    const uint32_t lane_base = tmem + (uint32_t(warp * 32) << 16);
+    const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
+    const uint32_t s_tm = lane_base + uint32_t(t * 2 * BK), dp_tm = s_tm + BK;
     const float sl2 = args.scale_log2;
     const float neg_lse2 = -args.lse2[size_t(bh) * args.Npad + row];  // -inf past N: P = 0
     const float drow = args.delta[size_t(bh) * args.Npad + row];
     const int lim = args.causal ? min(row + 1, args.N) : args.N;  // keys [0, lim) are visible
     bool ok = true;
-    for (int i = 0; i < nk; ++i) {
-      ok = mbar_wait(&ctrl->s_full, uint32_t(i) & 1u, abort);
+    for (int u = t; u < nb; u += 2) {
+      ok = mbar_wait(&ctrl->s_full[t], uint32_t(u >> 1) & 1u, abort);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const int key0 = i * 128;
-      const bool edge = key0 + 127 >= lim || key0 + 128 > args.N;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      const int key0 = u * BK;
+      const bool edge = key0 + BK > lim;
+#pragma unroll
+      for (int c = 0; c < BK / 32; ++c) {
         uint32_t sx[32], dx[32];
-        tmem_ld32(lane_base + C::DQ_S + uint32_t(32 * c), sx);
-        tmem_ld32(lane_base + C::DQ_DP + uint32_t(32 * c), dx);
+        tmem_ld32(s_tm + uint32_t(32 * c), sx);
+        tmem_ld32(dp_tm + uint32_t(32 * c), dx);
         tmem_ld_wait32(sx);
         tmem_ld_wait32(dx);
         uint32_t dd[16];
@@ -641,46 +679,51 @@ __global__ void __launch_bounds__(192, 1)
         for (int e = 0; e < 16; ++e) {
           float g[2];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int col = 32 * c + 2 * e + u;
-            float p = ex2_approx(fmaf(__uint_as_float(sx[2 * e + u]), sl2, neg_lse2));
+          for (int v2 = 0; v2 < 2; ++v2) {
+            const int col = 32 * c + 2 * e + v2;
+            float p = ex2_approx(fmaf(__uint_as_float(sx[2 * e + v2]), sl2, neg_lse2));
             if (edge && key0 + col >= lim) p = 0.f;
-            g[u] = p * (__uint_as_float(dx[2 * e + u]) - drow);
+            g[v2] = p * (__uint_as_float(dx[2 * e + v2]) - drow);
           }
           dd[e] = pack_bf16x2(g[0], g[1]);
         }
-        tmem_st16(lane_base + C::DQ_S + uint32_t(16 * c), dd);
+        tmem_st16(s_tm + uint32_t(16 * c), dd);
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&ctrl->p_full);
+      mbar_arrive(&ctrl->p_full[t]);
     }
     if (ok) ok = mbar_wait(&ctrl->acc_done, 0, abort);
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
+      // epilogue: warpgroup 0 writes dQ, warpgroup 1 dphi_q
       tc_fence_after();
       const bool valid = row < args.N;
-      const int d_st = valid ? args.d : 0;
-      uint16_t *dq_row = static_cast<uint16_t *>(args.dQ) + (size_t(bh) * args.N + (valid ? row : 0)) * args.d;
+      if (t == 0) {
+        const int d_st = valid ? args.d : 0;
+        uint16_t *dq_row = static_cast<uint16_t *>(args.dQ) + (size_t(bh) * args.N + (valid ? row : 0)) * args.d;
 #pragma unroll 1
-      for (int c0 = 0; c0 < DP; c0 += 16) {
-        uint32_t r[16];
-        tmem_ld16(lane_base + C::DQ_DQ + uint32_t(c0), r);
-        tmem_ld_wait16(r);
-        store_row16_bf16(r, args.scale, dq_row, c0, d_st);
+        for (int c0 = 0; c0 < DP; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld16(lane_base + C::DQ_DQ + uint32_t(c0), r);
+          tmem_ld_wait16(r);
+          store_row16_bf16(r, args.scale, dq_row, c0, d_st);
+        }
       }
       if constexpr (RG > 0) {
-        const int r_st = valid ? args.R : 0;
-        float *df = args.dphi_q + (args.fac_B > 1 ? int64_t(b) * args.phi_bs : 0) +
-                    (args.fac_H > 1 ? int64_t(h) * args.phi_hs : 0) + int64_t(valid ? row : 0) * args.R;
+        if (t == 1) {
+          const int r_st = valid ? args.R : 0;
+          float *df = args.dphi_q + (args.fac_B > 1 ? int64_t(b) * args.phi_bs : 0) +
+                      (args.fac_H > 1 ? int64_t(h) * args.phi_hs : 0) + int64_t(valid ? row : 0) * args.R;
 #pragma unroll 1
-        for (int c0 = 0; c0 < RG; c0 += 16) {
-          uint32_t r[16];
-          tmem_ld16(lane_base + C::DQ_DF + uint32_t(c0), r);
-          tmem_ld_wait16(r);
+          for (int c0 = 0; c0 < RG; c0 += 16) {
+            uint32_t r[16];
+            tmem_ld16(lane_base + C::DQ_DF + uint32_t(c0), r);
+            tmem_ld_wait16(r);
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            if (c0 + e < r_st) atomicAdd(df + c0 + e, __uint_as_float(r[e]));
+            for (int e = 0; e < 16; ++e)
+              if (c0 + e < r_st) atomicAdd(df + c0 + e, __uint_as_float(r[e]));
+          }
         }
       }
     }
@@ -694,6 +737,7 @@ __global__ void __launch_bounds__(192, 1)
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
+
 
 namespace {
 
@@ -722,7 +766,7 @@ cudaError_t launch_bwd_one(const BwdMaps &m, const BwdArgs &a, cudaStream_t stre
     const unsigned grid = unsigned((long long)a.n_kv * a.B * a.H);
     kv<<<grid, C::THREADS, C::KV_SMEM, stream>>>(m.k, m.v, m.fk, m.q_blk, m.do_blk, m.fq_blk, m.gq_blk, a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    dq<<<grid, C::THREADS, C::DQ_SMEM, stream>>>(m.q, m.dO, m.fq, m.k, m.v, m.fk, m.gk, a);
+    dq<<<grid, C::THREADS, C::DQ_SMEM, stream>>>(m.q, m.dO, m.fq, m.k_blk, m.v_blk, m.fk_blk, m.gk_blk, a);
     return cudaGetLastError();
   }
 }
@@ -730,6 +774,10 @@ cudaError_t launch_bwd_one(const BwdMaps &m, const BwdArgs &a, cudaStream_t stre
 template <int DP, int RP, int MODE, int RG>
 constexpr int bwd_block_rows() {
   return BwdCfg<DP, RP, MODE, RG>::BQ;
+}
+template <int DP, int RP, int MODE, int RG>
+constexpr int bwd_key_block_rows() {
+  return BwdCfg<DP, RP, MODE, RG>::BK;
 }
 
 }  // namespace
@@ -755,6 +803,13 @@ constexpr int bwd_block_rows() {
 
 int bwd_query_block_rows(const BwdPlan &p) {
 #define FB_BWD_ACTION(DPv, RPv, MODEv, RGv) bwd_block_rows<DPv, RPv, MODEv, RGv>()
+  FB_BWD_ALL
+#undef FB_BWD_ACTION
+  return 0;
+}
+
+int bwd_key_block_rows(const BwdPlan &p) {
+#define FB_BWD_ACTION(DPv, RPv, MODEv, RGv) bwd_key_block_rows<DPv, RPv, MODEv, RGv>()
   FB_BWD_ALL
 #undef FB_BWD_ACTION
   return 0;

@@ -320,38 +320,39 @@ cudaError_t launch_prep_factors(int mode, int B, int H, int N, int R, int RP, co
 }
 
 // Backward rows: lse2 = LSE log2(e) and delta = rowsum(dO * O) (fp32 sum of
-// the bf16 products), one warp per row; rows N .. Npad-1 get +inf and 0, so
-// the kernels' padded queries carry P = 0 without a bounds test.
+// the bf16 products). Eight threads per row, 16 bytes of O and dO each per
+// step (d % 8 == 0); rows N .. Npad-1 get +inf and 0, so the kernels' padded
+// queries carry P = 0 without a bounds test.
 __global__ void __launch_bounds__(256) bwd_rows_kernel(long long rows, int N, int Npad, int d,
                                                        const __nv_bfloat16 *__restrict__ O,
                                                        const __nv_bfloat16 *__restrict__ dO,
                                                        const float *__restrict__ LSE, float *__restrict__ lse2,
                                                        float *__restrict__ delta) {
-  const int lane = threadIdx.x & 31;
-  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
-  for (long long w = blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5); w < rows; w += warps) {
-    const long long bh = w / Npad;
-    const int n = int(w - bh * Npad);
-    float acc = 0.f;
-    if (n < N) {
-      const size_t base = (size_t(bh) * N + n) * d;
-      for (int c = lane * 4; c < d; c += 128) {  // d % 8 == 0: 4-element pieces stay in the row
-        const uint2 a = *reinterpret_cast<const uint2 *>(O + base + c);
-        const uint2 g = *reinterpret_cast<const uint2 *>(dO + base + c);
-        const uint32_t av[2] = {a.x, a.y}, gv[2] = {g.x, g.y};
+  const long long w = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 3;  // row
+  const int sub = threadIdx.x & 7;
+  if (w >= rows) return;  // whole 8-thread groups leave together
+  const long long bh = w / Npad;
+  const int n = int(w - bh * Npad);
+  float acc = 0.f;
+  if (n < N) {
+    const size_t base = (size_t(bh) * N + n) * d;
+    for (int c = sub * 8; c < d; c += 64) {
+      const uint4 a = *reinterpret_cast<const uint4 *>(O + base + c);
+      const uint4 g = *reinterpret_cast<const uint4 *>(dO + base + c);
+      const uint32_t av[4] = {a.x, a.y, a.z, a.w}, gv[4] = {g.x, g.y, g.z, g.w};
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          acc = fmaf(__uint_as_float(av[e] << 16), __uint_as_float(gv[e] << 16), acc);
-          acc = fmaf(__uint_as_float(av[e] & 0xFFFF0000u), __uint_as_float(gv[e] & 0xFFFF0000u), acc);
-        }
+      for (int e = 0; e < 4; ++e) {
+        acc = fmaf(__uint_as_float(av[e] << 16), __uint_as_float(gv[e] << 16), acc);
+        acc = fmaf(__uint_as_float(av[e] & 0xFFFF0000u), __uint_as_float(gv[e] & 0xFFFF0000u), acc);
       }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) {
-      lse2[w] = n < N ? LSE[size_t(bh) * N + n] * 1.4426950408889634f : INFINITY;
-      delta[w] = acc;
-    }
+  }
+  acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+  acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+  acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+  if (sub == 0) {
+    lse2[w] = n < N ? LSE[size_t(bh) * N + n] * 1.4426950408889634f : INFINITY;
+    delta[w] = acc;
   }
 }
 
@@ -384,9 +385,11 @@ __global__ void prep_grad_factors_kernel(int N, int R, int RG, int fac_H, const 
 
 cudaError_t launch_bwd_rows(int BH, int N, int Npad, int d, const void *O, const void *dO, const float *LSE,
                             float *lse2, float *delta, cudaStream_t s) {
-  const long long rows = (long long)BH * Npad;
-  bwd_rows_kernel<<<grid_for(rows * 32, 256), 256, 0, s>>>(rows, N, Npad, d, static_cast<const __nv_bfloat16 *>(O),
-                                                           static_cast<const __nv_bfloat16 *>(dO), LSE, lse2, delta);
+  const long long rows = (long long)BH * Npad;  // a multiple of 128: full warps
+  const long long blocks = (rows * 8 + 255) / 256;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  bwd_rows_kernel<<<unsigned(blocks), 256, 0, s>>>(rows, N, Npad, d, static_cast<const __nv_bfloat16 *>(O),
+                                                   static_cast<const __nv_bfloat16 *>(dO), LSE, lse2, delta);
   return cudaGetLastError();
 }
 

@@ -102,14 +102,18 @@ struct BwdPlan {
 };
 
 struct BwdMaps {
-  CUtensorMap q, k, v, dO;      // bf16 [BH, N, d], box (min(DP,64), 128, 1)
-  CUtensorMap q_blk, do_blk;    // the same with box rows = the dK/dV kernel's query block
-  CUtensorMap fq, fk, fq_blk;   // S-side factors (as FwdMaps), box rows 128 / query block
-  CUtensorMap gq_blk, gk;       // bf16 gradient factors [FB, N, RG], box rows query block / 128
+  CUtensorMap q, dO, fq;                         // dQ kernel, fixed tiles: box rows 128
+  CUtensorMap k, v, fk;                          // dK/dV kernel, fixed tiles: box rows 128
+  CUtensorMap q_blk, do_blk, fq_blk, gq_blk;     // dK/dV kernel, streamed query blocks
+  CUtensorMap k_blk, v_blk, fk_blk, gk_blk;      // dQ kernel, streamed key blocks
+  // Q, K, V, dO: bf16 [BH, N, d], box (min(DP,64), rows, 1); fq/fk: the forward's
+  // factor tiles; gq/gk: bf16 gradient factors [FB, N, RG].
 };
 
-// Rows of the dK/dV kernel's query block for a plan (0: unsupported).
+// Rows of the dK/dV kernel's query block and of the dQ kernel's key block
+// for a plan (0: unsupported).
 int bwd_query_block_rows(const BwdPlan &p);
+int bwd_key_block_rows(const BwdPlan &p);
 cudaError_t bwd_launch(const BwdPlan &p, const BwdMaps &maps, const BwdArgs &a, cudaStream_t stream);
 // lse2 = LSE * log2(e) and delta = rowsum(dO * O) per row, padded to Npad.
 cudaError_t launch_bwd_rows(int BH, int N, int Npad, int d, const void *O, const void *dO, const float *LSE,
