@@ -230,13 +230,14 @@ def fb_attn_bwd(dt, B, H, N, d, Q, K, V, R, phi_q, phi_k, phi_bstride, phi_hstri
                              LSE, dO, dQ, dK, dV, dphi_q, dphi_k, workspace, workspace_bytes, stream)
 
 
-def attn_bwd(q, k, v, phi_q, phi_k, o, lse, do, scale=None, causal=False, workspace=None):
+def attn_bwd(q, k, v, phi_q, phi_k, o, lse, do, scale=None, causal=False, workspace=None, factor_grads=True):
     """Gradients of attn's O for an upstream gradient do (fb_attn_bwd).
 
     q, k, v, o, do: bf16 CUDA [B, H, N, d] contiguous; lse: fp32 [B, H, N]
     from the forward; phi_q, phi_k as for attn (or None). Returns
     (dq, dk, dv, dphi_q, dphi_k): bf16 [B, H, N, d] and fp32 gradients shaped
-    like phi_q, phi_k (None without factors)."""
+    like phi_q, phi_k (None without factors, or with factor_grads=False for
+    fixed factors, whose gradient products are then skipped)."""
     import torch
     for t in (q, k, v, o, do):
         assert t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()
@@ -250,8 +251,9 @@ def attn_bwd(q, k, v, phi_q, phi_k, o, lse, do, scale=None, causal=False, worksp
         R = phi_q.shape[-1]
         bs, hs = _factor_strides(phi_q, B, H, N, R)
         pq, pk = phi_q.data_ptr(), phi_k.data_ptr()
-        dpq, dpk = torch.empty_like(phi_q), torch.empty_like(phi_k)
-        gq, gk = dpq.data_ptr(), dpk.data_ptr()
+        if factor_grads:
+            dpq, dpk = torch.empty_like(phi_q), torch.empty_like(phi_k)
+            gq, gk = dpq.data_ptr(), dpk.data_ptr()
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     nb = fb_attn_bwd_workspace_bytes(B, H, N, R, bs, hs)
     if workspace is None:

@@ -496,8 +496,9 @@ int fb_factors_alibi(int H, int N, float *phi_q, float *phi_k, void *stream) {
 namespace {
 struct BwdLayout {
   WsLayout f;  // the S-side factor tiles (as the forward's workspace)
-  size_t gq_off, gk_off, l_off, d_off, total;
+  size_t gq_off, gk_off, l_off, d_off, pq_off, pk_off, total;
   int RG, Npad;
+  bool shared_slices;  // some factor slice serves several heads: per-head partial gradients
 };
 size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 BwdLayout bwd_layout(int B, int H, int N, int R, int64_t bs, int64_t hs) {
@@ -512,7 +513,11 @@ BwdLayout bwd_layout(int B, int H, int N, int R, int64_t bs, int64_t hs) {
   w.gk_off = w.gq_off + g;
   w.l_off = w.gk_off + g;
   w.d_off = w.l_off + rows;
-  w.total = w.d_off + rows;
+  w.shared_slices = R > 0 && fb < size_t(B) * H;
+  const size_t part = w.shared_slices ? al256(size_t(B) * H * size_t(N) * size_t(R) * 4) : 0;
+  w.pq_off = w.d_off + rows;
+  w.pk_off = w.pq_off + part;
+  w.total = w.pk_off + part;
   return w;
 }
 bool encode_rows_bf16(CUtensorMap *m, const void *ptr, int slices, int N, int cols, int width, int rows) {
@@ -550,8 +555,10 @@ int fb_attn_bwd(int dt, int B, int H, int N, int d, const void *Q, const void *K
   if (!Q || !K || !V || !O || !LSE || !dO || !dQ || !dK || !dV) return FB_ERR_INVALID_ARG;
   if (dt != FB_BF16) return FB_ERR_UNSUPPORTED;
   if (R < 0 || R > 128) return FB_ERR_UNSUPPORTED;
-  if (R > 0 && (!phi_q || !phi_k || !dphi_q || !dphi_k || phi_bstride < 0 || phi_hstride < 0))
-    return FB_ERR_INVALID_ARG;
+  // factor gradients: both or neither (neither: fixed factors, their products skipped)
+  const bool want_dphi = dphi_q != nullptr && dphi_k != nullptr;
+  if (R > 0 && (!phi_q || !phi_k || phi_bstride < 0 || phi_hstride < 0)) return FB_ERR_INVALID_ARG;
+  if (R > 0 && !want_dphi && (dphi_q || dphi_k)) return FB_ERR_INVALID_ARG;
   if (R > 0 && (((reinterpret_cast<uintptr_t>(phi_q) | reinterpret_cast<uintptr_t>(phi_k) |
                   reinterpret_cast<uintptr_t>(dphi_q) | reinterpret_cast<uintptr_t>(dphi_k)) &
                  3u) != 0))
@@ -568,7 +575,7 @@ int fb_attn_bwd(int dt, int B, int H, int N, int d, const void *Q, const void *K
   plan.DP = pad_dim(d);
   plan.mode = R == 0 ? kBiasNone : (R <= 4 ? kBiasTf32 : kBiasMma);
   plan.RP = plan.mode == kBiasMma ? pad_rank(R) : (plan.mode == kBiasTf32 ? tf32_cols(R) : 0);
-  plan.RG = L.RG;
+  plan.RG = want_dphi ? L.RG : 0;
   const int BQ = bwd_query_block_rows(plan), BK = bwd_key_block_rows(plan);
   if (BQ == 0 || BK == 0) return FB_ERR_UNSUPPORTED;
   int *flags = device_flags();
@@ -584,8 +591,8 @@ int fb_attn_bwd(int dt, int B, int H, int N, int d, const void *Q, const void *K
                                            workspace_bytes, stream);
     if (rc != FB_OK) return rc;
     // 2. bf16 factor copies for the gradient products; zeroed factor gradients
-    if (launch_prep_grad_factors(N, R, L.RG, phi_q, phi_k, phi_bstride, phi_hstride, fac_B, fac_H, wsb + L.gq_off,
-                                 wsb + L.gk_off, dphi_q, dphi_k, st) != cudaSuccess)
+    if (want_dphi && launch_prep_grad_factors(N, R, L.RG, phi_q, phi_k, phi_bstride, phi_hstride, fac_B, fac_H,
+                                              wsb + L.gq_off, wsb + L.gk_off, st) != cudaSuccess)
       return FB_ERR_CUDA;
   }
   // 3. per-row LSE in log2 units and rowsum(dO * O)
@@ -607,9 +614,10 @@ int fb_attn_bwd(int dt, int B, int H, int N, int d, const void *Q, const void *K
     if (!encode_fac(&maps.fq, plan.mode, wq, FB, N, plan.RP, 128) ||
         !encode_fac(&maps.fk, plan.mode, wk, FB, N, plan.RP, 128) ||
         !encode_fac(&maps.fq_blk, plan.mode, wq, FB, N, plan.RP, BQ) ||
-        !encode_fac(&maps.fk_blk, plan.mode, wk, FB, N, plan.RP, BK) ||
-        !encode_rows_bf16(&maps.gq_blk, wsb + L.gq_off, FB, N, L.RG, L.RG, BQ) ||
-        !encode_rows_bf16(&maps.gk_blk, wsb + L.gk_off, FB, N, L.RG, L.RG, BK))
+        !encode_fac(&maps.fk_blk, plan.mode, wk, FB, N, plan.RP, BK))
+      return FB_ERR_CUDA;
+    if (want_dphi && (!encode_rows_bf16(&maps.gq_blk, wsb + L.gq_off, FB, N, L.RG, L.RG, BQ) ||
+                      !encode_rows_bf16(&maps.gk_blk, wsb + L.gk_off, FB, N, L.RG, L.RG, BK)))
       return FB_ERR_CUDA;
   }
   BwdArgs a;
@@ -624,10 +632,19 @@ int fb_attn_bwd(int dt, int B, int H, int N, int d, const void *Q, const void *K
   a.delta = delta;
   a.dQ = dQ, a.dK = dK, a.dV = dV;
   a.dphi_q = dphi_q, a.dphi_k = dphi_k;
+  a.dphi_direct = L.shared_slices ? 0 : 1;
+  a.dphi_q_part = L.shared_slices ? reinterpret_cast<float *>(wsb + L.pq_off) : nullptr;
+  a.dphi_k_part = L.shared_slices ? reinterpret_cast<float *>(wsb + L.pk_off) : nullptr;
   a.phi_bs = phi_bstride, a.phi_hs = phi_hstride;
   a.fac_B = fac_B, a.fac_H = fac_H;
   a.flags = flags;
-  return bwd_launch(plan, maps, a, st) == cudaSuccess ? FB_OK : FB_ERR_CUDA;
+  if (bwd_launch(plan, maps, a, st) != cudaSuccess) return FB_ERR_CUDA;
+  // 5. factor slices shared by several heads: sum the per-head rows
+  if (want_dphi && L.shared_slices &&
+      launch_reduce_factor_grads(B, H, N, R, fac_B, fac_H, phi_bstride, phi_hstride, a.dphi_q_part, a.dphi_k_part,
+                                 dphi_q, dphi_k, st) != cudaSuccess)
+    return FB_ERR_CUDA;
+  return FB_OK;
 }
 
 int fb_check_device_error(void *stream) {

@@ -30,8 +30,9 @@
 // S and dP buffers in TMEM (ping-pong): while one turns its scores into P and
 // dS, the tensor core runs the other's products.
 // The factor gradients of a broadcast factor (stride 0) sum over the heads
-// and batches sharing it, so they are accumulated with fp32 reductions into
-// a buffer zeroed by the preparation step.
+// and batches sharing it: each head writes its rows to per-head partials and
+// a reduction over the sharing heads follows; a per-head factor gets its rows
+// written directly. No atomics anywhere.
 //
 // CTA: warps 0-7 compute (two warpgroups, one thread per TMEM lane = tile
 // row in each), warp 8 TMA producer, warp 9 TMEM allocator and MMA issuer. Every wait is bounded (the
@@ -166,6 +167,43 @@ __device__ __forceinline__ void store_row16_bf16(const uint32_t *r, float mul, u
   for (int e = 0; e < 8; ++e) w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * mul, __uint_as_float(r[2 * e + 1]) * mul);
   if (c0 + 8 <= d) *reinterpret_cast<uint4 *>(row + c0) = make_uint4(w[0], w[1], w[2], w[3]);
   if (c0 + 16 <= d) *reinterpret_cast<uint4 *>(row + c0 + 8) = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
+// The factor-gradient row of head (b, h) and row n: in the caller's tensor
+// when every head has its own factor slice (each row is then written by
+// exactly one CTA), else in the per-head partial rows [BH, N, R] that a
+// reduction over the heads sharing a slice sums afterwards. No atomics.
+__device__ __forceinline__ float *factor_grad_row(const BwdArgs &a, float *dphi, float *part, int b, int h, int bh,
+                                                  int n) {
+  if (a.dphi_direct)
+    return dphi + (a.fac_B > 1 ? int64_t(b) * a.phi_bs : 0) + (a.fac_H > 1 ? int64_t(h) * a.phi_hs : 0) +
+           int64_t(n) * a.R;
+  return part + (int64_t(bh) * a.N + n) * a.R;
+}
+
+// The first `valid` of the RG fp32 columns of this thread's TMEM lane to a
+// global row (16-byte stores when the row allows them). TMEM loads are
+// warp-collective: every lane loads, lanes with valid = 0 store nothing.
+template <int RG>
+__device__ __forceinline__ void store_factor_grad_row(uint32_t taddr, float *row, int valid) {
+  const bool vec = (valid & 3) == 0 && (reinterpret_cast<uintptr_t>(row) & 15u) == 0;
+#pragma unroll 1
+  for (int c0 = 0; c0 < RG; c0 += 16) {
+    uint32_t r[16];
+    tmem_ld16(taddr + uint32_t(c0), r);
+    tmem_ld_wait16(r);
+    if (vec) {
+#pragma unroll
+      for (int e = 0; e < 16; e += 4)
+        if (c0 + e < valid)
+          *reinterpret_cast<float4 *>(row + c0 + e) = make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
+                                                                  __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
+    } else {
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        if (c0 + e < valid) row[c0 + e] = __uint_as_float(r[e]);
+    }
+  }
 }
 
 }  // namespace
@@ -440,17 +478,9 @@ __global__ void __launch_bounds__(320, 1)
       if constexpr (RG > 0) {
         if (t == 0) {
           const int r_st = valid ? args.R : 0;
-          float *df = args.dphi_k + (args.fac_B > 1 ? int64_t(b) * args.phi_bs : 0) +
-                      (args.fac_H > 1 ? int64_t(h) * args.phi_hs : 0) + int64_t(valid ? krow : 0) * args.R;
-#pragma unroll 1
-          for (int c0 = 0; c0 < RG; c0 += 16) {
-            uint32_t r[16];
-            tmem_ld16(lane_base + C::KV_DF + uint32_t(c0), r);
-            tmem_ld_wait16(r);
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-              if (c0 + e < r_st) atomicAdd(df + c0 + e, __uint_as_float(r[e]));
-          }
+          store_factor_grad_row<RG>(lane_base + C::KV_DF, factor_grad_row(args, args.dphi_k, args.dphi_k_part, b, h,
+                                                                           bh, valid ? krow : 0),
+                                    r_st);
         }
       }
     }
@@ -713,17 +743,9 @@ __global__ void __launch_bounds__(320, 1)
       if constexpr (RG > 0) {
         if (t == 1) {
           const int r_st = valid ? args.R : 0;
-          float *df = args.dphi_q + (args.fac_B > 1 ? int64_t(b) * args.phi_bs : 0) +
-                      (args.fac_H > 1 ? int64_t(h) * args.phi_hs : 0) + int64_t(valid ? row : 0) * args.R;
-#pragma unroll 1
-          for (int c0 = 0; c0 < RG; c0 += 16) {
-            uint32_t r[16];
-            tmem_ld16(lane_base + C::DQ_DF + uint32_t(c0), r);
-            tmem_ld_wait16(r);
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-              if (c0 + e < r_st) atomicAdd(df + c0 + e, __uint_as_float(r[e]));
-          }
+          store_factor_grad_row<RG>(lane_base + C::DQ_DF, factor_grad_row(args, args.dphi_q, args.dphi_q_part, b, h,
+                                                                           bh, valid ? row : 0),
+                                    r_st);
         }
       }
     }
@@ -782,17 +804,18 @@ constexpr int bwd_key_block_rows() {
 
 }  // namespace
 
+// RG = 0: the factors are fixed (no factor gradients requested)
 #define FB_BWD_MODE(DPv)                                                            \
   if (p.mode == kBiasNone) return FB_BWD_ACTION(DPv, 0, kBiasNone, 0);              \
   if (p.mode == kBiasTf32) {                                                        \
-    if (p.RP == 8) return FB_BWD_ACTION(DPv, 8, kBiasTf32, 16);                     \
-    if (p.RP == 16) return FB_BWD_ACTION(DPv, 16, kBiasTf32, 16);                   \
+    if (p.RP == 8) return p.RG ? FB_BWD_ACTION(DPv, 8, kBiasTf32, 16) : FB_BWD_ACTION(DPv, 8, kBiasTf32, 0);    \
+    if (p.RP == 16) return p.RG ? FB_BWD_ACTION(DPv, 16, kBiasTf32, 16) : FB_BWD_ACTION(DPv, 16, kBiasTf32, 0); \
   }                                                                                 \
   if (p.mode == kBiasMma) {                                                         \
-    if (p.RP == 16) return FB_BWD_ACTION(DPv, 16, kBiasMma, 16);                    \
-    if (p.RP == 32) return FB_BWD_ACTION(DPv, 32, kBiasMma, 32);                    \
-    if (p.RP == 64) return FB_BWD_ACTION(DPv, 64, kBiasMma, 64);                    \
-    if (p.RP == 128) return FB_BWD_ACTION(DPv, 128, kBiasMma, 128);                 \
+    if (p.RP == 16) return p.RG ? FB_BWD_ACTION(DPv, 16, kBiasMma, 16) : FB_BWD_ACTION(DPv, 16, kBiasMma, 0);   \
+    if (p.RP == 32) return p.RG ? FB_BWD_ACTION(DPv, 32, kBiasMma, 32) : FB_BWD_ACTION(DPv, 32, kBiasMma, 0);   \
+    if (p.RP == 64) return p.RG ? FB_BWD_ACTION(DPv, 64, kBiasMma, 64) : FB_BWD_ACTION(DPv, 64, kBiasMma, 0);   \
+    if (p.RP == 128) return p.RG ? FB_BWD_ACTION(DPv, 128, kBiasMma, 128) : FB_BWD_ACTION(DPv, 128, kBiasMma, 0); \
   }
 
 #define FB_BWD_ALL                                                                  \

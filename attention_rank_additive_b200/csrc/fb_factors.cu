@@ -357,12 +357,11 @@ __global__ void __launch_bounds__(256) bwd_rows_kernel(long long rows, int N, in
 }
 
 // bf16 copies of the factors for the gradient products, [FB, N, RG] with
-// zero padding, and the factor gradients zeroed (the backward kernels add
-// into them).
+// zero padding.
 __global__ void prep_grad_factors_kernel(int N, int R, int RG, int fac_H, const float *__restrict__ pq,
                                          const float *__restrict__ pk, long long bs, long long hs,
                                          __nv_bfloat16 *__restrict__ gq, __nv_bfloat16 *__restrict__ gk,
-                                         float *__restrict__ dpq, float *__restrict__ dpk, long long total) {
+                                         long long total) {
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
        idx += (long long)gridDim.x * blockDim.x) {
     const int r = int(idx % RG);
@@ -375,8 +374,6 @@ __global__ void prep_grad_factors_kernel(int N, int R, int RG, int fac_H, const 
       const long long src = fb * bs + fh * hs + n * R + r;
       vq = pq[src];
       vk = pk[src];
-      dpq[src] = 0.f;
-      dpk[src] = 0.f;
     }
     gq[idx] = __float2bfloat16_rn(vq);
     gk[idx] = __float2bfloat16_rn(vk);
@@ -394,12 +391,46 @@ cudaError_t launch_bwd_rows(int BH, int N, int Npad, int d, const void *O, const
 }
 
 cudaError_t launch_prep_grad_factors(int N, int R, int RG, const float *phi_q, const float *phi_k, int64_t bs,
-                                     int64_t hs, int fac_B, int fac_H, void *gq, void *gk, float *dphi_q,
-                                     float *dphi_k, cudaStream_t s) {
+                                     int64_t hs, int fac_B, int fac_H, void *gq, void *gk, cudaStream_t s) {
   const long long total = (long long)fac_B * fac_H * N * RG;
   prep_grad_factors_kernel<<<grid_for(total, 256), 256, 0, s>>>(
       N, R, RG, fac_H, phi_q, phi_k, bs, hs, static_cast<__nv_bfloat16 *>(gq), static_cast<__nv_bfloat16 *>(gk),
-      dphi_q, dphi_k, total);
+      total);
+  return cudaGetLastError();
+}
+
+// dphi[fb, fh, n, r] = sum over the heads (b, h) that share slice (fb, fh)
+// of part[b H + h, n, r]: one thread per output element, fp32 in head order.
+__global__ void reduce_factor_grads_kernel(int B, int H, int N, int R, int fac_B, int fac_H, long long bs,
+                                           long long hs, const float *__restrict__ pq, const float *__restrict__ pk,
+                                           float *__restrict__ dq, float *__restrict__ dk, long long total) {
+  const long long NR = (long long)N * R;
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const long long f = idx / NR, e = idx - f * NR;
+    const int fb = int(f / fac_H), fh = int(f - (f / fac_H) * fac_H);
+    const int b0 = fac_B > 1 ? fb : 0, b1 = fac_B > 1 ? fb + 1 : B;
+    const int h0 = fac_H > 1 ? fh : 0, h1 = fac_H > 1 ? fh + 1 : H;
+    float aq = 0.f, ak = 0.f;
+    for (int b = b0; b < b1; ++b)
+      for (int h = h0; h < h1; ++h) {
+        const long long o = ((long long)b * H + h) * NR + e;
+        aq += pq[o];
+        ak += pk[o];
+      }
+    const long long n = e / R, r = e - (e / R) * R;
+    const long long dst = fb * bs + fh * hs + n * R + r;
+    dq[dst] = aq;
+    dk[dst] = ak;
+  }
+}
+
+cudaError_t launch_reduce_factor_grads(int B, int H, int N, int R, int fac_B, int fac_H, int64_t bs, int64_t hs,
+                                       const float *part_q, const float *part_k, float *dphi_q, float *dphi_k,
+                                       cudaStream_t s) {
+  const long long total = (long long)fac_B * fac_H * N * R;
+  reduce_factor_grads_kernel<<<grid_for(total, 256), 256, 0, s>>>(B, H, N, R, fac_B, fac_H, bs, hs, part_q, part_k,
+                                                                  dphi_q, dphi_k, total);
   return cudaGetLastError();
 }
 

@@ -88,7 +88,9 @@ struct BwdArgs {
   const float *lse2;       // [BH, Npad] LSE * log2(e); +inf past N
   const float *delta;      // [BH, Npad] rowsum(dO * O); 0 past N
   void *dQ, *dK, *dV;      // bf16 [BH, N, d]
-  float *dphi_q, *dphi_k;  // fp32, laid out like phi_q / phi_k (zeroed first, accumulated)
+  float *dphi_q, *dphi_k;  // fp32, laid out like phi_q / phi_k
+  float *dphi_q_part, *dphi_k_part;  // per-head partial rows [BH, N, R] (shared factor slices)
+  int dphi_direct;         // 1: every head has its own factor slice, rows go straight to dphi
   int64_t phi_bs, phi_hs;  // element strides of the factor tensors
   int fac_B, fac_H;        // factor slices: B or 1, H or 1
   int *flags;
@@ -118,10 +120,14 @@ cudaError_t bwd_launch(const BwdPlan &p, const BwdMaps &maps, const BwdArgs &a, 
 // lse2 = LSE * log2(e) and delta = rowsum(dO * O) per row, padded to Npad.
 cudaError_t launch_bwd_rows(int BH, int N, int Npad, int d, const void *O, const void *dO, const float *LSE,
                             float *lse2, float *delta, cudaStream_t s);
-// bf16 copies of the factors [FB, N, RG] (zero-padded) and zeroed factor gradients.
+// bf16 copies of the factors [FB, N, RG] (zero-padded).
 cudaError_t launch_prep_grad_factors(int N, int R, int RG, const float *phi_q, const float *phi_k, int64_t bs,
-                                     int64_t hs, int fac_B, int fac_H, void *gq, void *gk, float *dphi_q,
-                                     float *dphi_k, cudaStream_t s);
+                                     int64_t hs, int fac_B, int fac_H, void *gq, void *gk, cudaStream_t s);
+// Factor gradients of shared slices: dphi[f] = sum over the heads of slice f of
+// the per-head partial rows [B*H, N, R].
+cudaError_t launch_reduce_factor_grads(int B, int H, int N, int R, int fac_B, int fac_H, int64_t bs, int64_t hs,
+                                       const float *part_q, const float *part_k, float *dphi_q, float *dphi_k,
+                                       cudaStream_t s);
 
 // Per-device flag word (allocated once per device as a module global).
 int *device_flags();

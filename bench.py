@@ -73,12 +73,13 @@ def flops(B, H, N, d, R, causal, multiplicative=False) -> float:
     return f / 2.0 if causal else f
 
 
-def bwd_flops(B, H, N, d, R, causal) -> float:
+def bwd_flops(B, H, N, d, R, causal, factor_grads=True) -> float:
     """Counted FLOPs of the backward per head: the five products of the
     concatenated form, 2 N^2 (d + R) each for S, dQ' = dS K' and dK' =
     dS^T Q', 2 N^2 d each for dP and dV (the dQ kernel's recomputation of S
-    and dP is not counted); halved when causal."""
-    f = float(B) * H * 2.0 * N * N * (5.0 * d + 3.0 * R)
+    and dP is not counted); without factor gradients dQ and dK are 2 N^2 d
+    each; halved when causal."""
+    f = float(B) * H * 2.0 * N * N * ((5.0 * d + 3.0 * R) if factor_grads else (5.0 * d + R))
     return f / 2.0 if causal else f
 
 
@@ -309,8 +310,10 @@ class GpuWorkload:
         self.launches_per_step = (3 if self.neural else
                                   (2 if self.mul or (Rk > 0 and c["dtype"] == "bf16") else 1))
         self.bwd = bool(c.get("bwd"))
-        if self.bwd:  # factor preparation, bf16 factor copies, per-row terms, two gradient kernels
-            self.launches_per_step = 5 if Rk > 0 else 3
+        if self.bwd:  # factor preparation, bf16 factor copies, per-row terms, two gradient kernels, and
+            # the reduction of per-head factor gradients when a factor slice serves several heads
+            shared = Rk > 0 and (self.bs == 0 and B > 1 or self.hs == 0 and H > 1)
+            self.launches_per_step = (5 + (1 if shared else 0)) if Rk > 0 else 3
 
     def setup_bwd(self):
         """Forward outputs O, LSE for the backward workload (once, untimed),
@@ -329,14 +332,15 @@ class GpuWorkload:
         self.bws_bytes = fb.fb_attn_bwd_workspace_bytes(B, H, N, self.R, self.bs, self.hs)
         self.bws = torch.empty(self.bws_bytes, device=self.device, dtype=torch.uint8)
 
-    def run_bwd(self):
+    def run_bwd(self, factor_grads=True):
         fb, c = self.fb, self.c
+        fg = factor_grads and self.R > 0
         st = fb.fb_attn_bwd(fb.FB_BF16, c["B"], c["H"], c["N"], c["d"], self.Q.data_ptr(), self.K.data_ptr(),
                             self.V.data_ptr(), self.R, self.pq.data_ptr() if self.R else 0,
                             self.pk.data_ptr() if self.R else 0, self.bs, self.hs, self.scale, int(c["causal"]),
                             self.O.data_ptr(), self.LSE.data_ptr(), self.dO.data_ptr(), self.dQ.data_ptr(),
-                            self.dK.data_ptr(), self.dV.data_ptr(), self.dpq.data_ptr() if self.R else 0,
-                            self.dpk.data_ptr() if self.R else 0, self.bws.data_ptr(), self.bws_bytes, self.stream)
+                            self.dK.data_ptr(), self.dV.data_ptr(), self.dpq.data_ptr() if fg else 0,
+                            self.dpk.data_ptr() if fg else 0, self.bws.data_ptr(), self.bws_bytes, self.stream)
         assert st == fb.FB_OK, fb.fb_status_str(st)
 
     def _dense_bias(self):
@@ -600,7 +604,8 @@ def run_ours(args, rank: int, world: int, local: int):
                      "frac": round(achieved / peak_tf, 4), "traffic": traffic,
                      "kernel": ("prep_mul_bias + attn_fwd_sm100" if w.mul else
                                 ("neural_factor + prep + attn_fwd_sm100" if w.neural else
-                                 ("bwd preparation (3) + attn_bwd_dkdv_sm100 + attn_bwd_dq_sm100" if w.bwd
+                                 ("bwd preparation (3) + attn_bwd_dkdv_sm100 + attn_bwd_dq_sm100 + factor-gradient "
+                                  "reduction" if w.bwd
                                   else "attn_fwd_sm100"))),
                      "peak_kind": peak_kind,
                      "kernel_ms": round(kern_ms, 5)},
@@ -609,6 +614,19 @@ def run_ours(args, rank: int, world: int, local: int):
         "gpu_launches": w.launches_per_step * args.steps,
         "dense_bias": dense,
     }
+    if w.bwd and w.R > 0:
+        # the same backward with fixed factors (the exact Sandwich factors are not
+        # trained): no factor gradients, FLOPs counted without their products
+        for _ in range(3):
+            w.run_bwd(factor_grads=False)
+        f_steps = max(5, min(args.steps, 100))
+        barrier(world)
+        f_ms = reduce_max(statistics.mean(time_steps(torch, lambda: w.run_bwd(factor_grads=False), w.flush_l2,
+                                                     f_steps, stream)), world, device)
+        barrier(world)
+        f_flops = bwd_flops(c["B"], c["H"], c["N"], c["d"], c["R"], c["causal"], factor_grads=False)
+        out["bwd_fixed_factors"] = {"ms": round(f_ms, 5), "tflops": round(f_flops / (f_ms * 1e-3) / 1e12, 2),
+                                    "launches_per_step": 4}
     if hasattr(w, "svd_err"):
         out["svd_rank_error_energy_per_head"] = w.svd_err
         out["svd_device"] = svd_device_leg(torch, fb, w, c, stream)

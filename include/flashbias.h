@@ -222,16 +222,21 @@ int fb_attn_neural_fwd(int dt, int B, int H, int N, int d,
  *  dQ, dK, dV  bf16 [B,H,N,d] device outputs, 16-byte aligned.
  *  dphi_q/k    fp32 device outputs laid out like phi_q / phi_k (the same
  *              strides; a broadcast factor, stride 0, gets the gradient
- *              summed over the batches or heads sharing it). Overwritten:
- *              the call zeroes them, then accumulates. Unused when R = 0.
+ *              summed over the batches or heads sharing it). Overwritten
+ *              (no accumulation into the caller's values). Both NULL: the factors
+ *              are fixed (e.g. the exact Sandwich or ALiBi factors) and their
+ *              gradient products are skipped; one NULL is an argument error.
+ *              Unused when R = 0. They must not alias any input.
  *  workspace   fb_attn_bwd_workspace_bytes(B, H, N, R, phi_bstride,
  *              phi_hstride) bytes, 256-byte aligned (never 0).
  * Arithmetic: S and P are recomputed as the forward computes them; the
  * products with dO, Q, K and the factors run on the tensor cores in bf16 with
  * fp32 accumulation. Launches: the factor preparation and the bf16 factor
  * copies (R > 0), the per-row terms, then two tcgen05 kernels (dK, dV,
- * dphi_k per key tile; dQ, dphi_q per query tile). Argument errors return
- * before any launch; other errors as fb_attn_fwd.
+ * dphi_k per key tile; dQ, dphi_q per query tile), and for a factor shared
+ * by several heads one reduction of the per-head factor gradients (kept in
+ * the workspace). Argument errors return before any launch; other errors as
+ * fb_attn_fwd.
  */
 size_t fb_attn_bwd_workspace_bytes(int B, int H, int N, int R,
                                    int64_t phi_bstride, int64_t phi_hstride);

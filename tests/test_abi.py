@@ -327,9 +327,10 @@ def test_backward_workspace_and_argument_errors():
     fwd = fb.fb_attn_workspace_bytes(B, H, N, R, H * N * R, N * R)
     assert fb.fb_attn_bwd_workspace_bytes(B, H, N, R, H * N * R, N * R) == \
         fwd + 2 * al(B * H * N * 16 * 2) + 2 * al(B * H * Npad * 4)
-    # broadcast factors: one factor slice
+    # broadcast factors: one factor slice, plus per-head partial factor gradients
     assert fb.fb_attn_bwd_workspace_bytes(B, H, N, R, 0, 0) == \
-        fb.fb_attn_workspace_bytes(B, H, N, R, 0, 0) + 2 * al(N * 16 * 2) + 2 * al(B * H * Npad * 4)
+        fb.fb_attn_workspace_bytes(B, H, N, R, 0, 0) + 2 * al(N * 16 * 2) + 2 * al(B * H * Npad * 4) + \
+        2 * al(B * H * N * R * 4)
     assert fb.fb_attn_bwd_workspace_bytes(B, H, N, 0, 0, 0) == 2 * al(B * H * Npad * 4)
     assert fb.fb_attn_bwd_workspace_bytes(B, H, N, 129, 0, 0) == 0
     assert fb.fb_attn_bwd_workspace_bytes(0, H, N, R, 0, 0) == 0
@@ -348,7 +349,7 @@ def test_backward_workspace_and_argument_errors():
     assert b(R=129) == fb.FB_ERR_UNSUPPORTED
     assert b(d=20) == fb.FB_ERR_UNSUPPORTED
     assert b(dO=0) == fb.FB_ERR_INVALID_ARG
-    assert b(dphi_k=0) == fb.FB_ERR_INVALID_ARG
+    assert b(dphi_k=0) == fb.FB_ERR_INVALID_ARG  # one factor gradient without the other
     assert b(dphi_q=FAKE + 2) == fb.FB_ERR_INVALID_ARG
     assert b(dK=FAKE + 8) == fb.FB_ERR_INVALID_ARG
     assert b(phi_hstride=-1) == fb.FB_ERR_INVALID_ARG

@@ -425,3 +425,29 @@ def test_backward_matches_oracle(B, H, N, d, R, causal, layout):
     if R > 0:
         grad_close(host(dpq), ref_pq, f"dphi_q B{B} H{H} N{N} d{d} R{R} {layout}")
         grad_close(host(dpk), ref_pk, f"dphi_k B{B} H{H} N{N} d{d} R{R} {layout}")
+
+
+@pytest.mark.parametrize("B,H,N,d,R,causal", [(1, 2, 200, 64, 64, True), (1, 1, 257, 128, 2, False),
+                                               (1, 2, 300, 32, 100, True)])
+def test_backward_fixed_factors_matches_oracle(B, H, N, d, R, causal):
+    """Fixed factors (no factor gradients requested): dQ, dK, dV still match."""
+    seed = 1900 + N + R
+    q, k, v = si.qkv(B, H, N, d, seed, "bf16")
+    g = si.round_to_bf16(si.normal((B, H, N, d), seed + 3))
+    pq, pk = si.random_factors((B, H, N, R), math.sqrt(1.0 / R), seed + 7)
+    scale = 1.0 / math.sqrt(d)
+    tq, tk, tv, tg = (dev(x, "bf16") for x in (q, k, v, g))
+    tpq, tpk = dev(pq, "f32"), dev(pk, "f32")
+    o, lse = fb.attn(tq, tk, tv, tpq, tpk, scale=scale, causal=causal)
+    dq, dk, dv, dpq, dpk = fb.attn_bwd(tq, tk, tv, tpq, tpk, o, lse, tg, scale=scale, causal=causal,
+                                       factor_grads=False)
+    torch.cuda.synchronize()
+    _no_device_error()
+    assert dpq is None and dpk is None
+    got = {n: host(t) for n, t in (("dq", dq), ("dk", dk), ("dv", dv))}
+    for b in range(B):
+        for h in range(H):
+            r = oracle.attention_lowrank_bwd_head(q[b, h], k[b, h], v[b, h], pq[b, h], pk[b, h], g[b, h], scale,
+                                                  causal)
+            for n in ("dq", "dk", "dv"):
+                grad_close(got[n][b, h], r[n], f"{n} ({b},{h}) fixed factors N{N} d{d} R{R}")
