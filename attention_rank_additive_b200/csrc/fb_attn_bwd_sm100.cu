@@ -15,7 +15,7 @@
 // forward's P; the gradient products run in bf16 with fp32 accumulation, the
 // factors entering them as bf16 copies.
 //
-// Two kernels, neither with atomics on the bf16 outputs:
+// Two kernels, no atomics:
 //   attn_bwd_dkdv_sm100  one CTA per (b, h, 128-key tile). The key tile K|phi_k
 //       and V stay in shared memory; query blocks of BQ rows (64, or 32 at
 //       head dim 128 so that TMEM holds everything) stream through a ring.
@@ -35,8 +35,9 @@
 // written directly. No atomics anywhere.
 //
 // CTA: warps 0-7 compute (two warpgroups, one thread per TMEM lane = tile
-// row in each), warp 8 TMA producer, warp 9 TMEM allocator and MMA issuer. Every wait is bounded (the
-// abort flag and the device flag word report a timeout).
+// row in each), warp 8 TMA producer, warp 9 TMEM allocator and MMA issuer.
+// Every wait is bounded (the abort flag and the device flag word report a
+// timeout).
 #include <algorithm>
 #include <atomic>
 
