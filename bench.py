@@ -723,9 +723,10 @@ def cpu_baseline(c: dict, budget_s: float):
         total_fl += fl
         parts.append(desc)
         step += 1
+    what = ("causal prefixes of 256 tokens (every gradient, fp64 oracle backward, counted FLOPs of the prefix)"
+            if c.get("bwd") else "256 sampled query rows (fp64 oracle, counted FLOPs of those rows)")
     return {"value": total_fl / total_s / 1e12, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{step} heads x 256 sampled query rows (fp64 oracle, counted FLOPs of those rows), "
-                      f"{total_s:.1f} s"}
+            "sample": f"{step} heads x {what}, {total_s:.1f} s"}
 
 
 def run_reference(args, rank: int, world: int):
@@ -752,7 +753,10 @@ def run_reference(args, rank: int, world: int):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded; see seeded_inputs)",
         "config": config_json(c, "n/a (host)"),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-                         "sample": f"per step {rows} sampled query rows of one head (rotating over heads)"},
+                         "sample": (f"per step every gradient of the causal prefix of {rows} tokens of one head "
+                                    "(rotating over heads; the oracle backward on a complete sub-problem)"
+                                    if c.get("bwd") else
+                                    f"per step {rows} sampled query rows of one head (rotating over heads)")},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
