@@ -40,6 +40,8 @@ METRIC = "biased-attn fwd TFLOP/s & ms at 1 B200 (% of bf16 TC peak) vs dense-bi
 UNIT = "TFLOP/s"
 L2_FLUSH_BYTES = 256 << 20
 KERNEL_SOURCES = ("attention_rank_additive_b200/csrc/fb_attn_sm100.cu", "attention_rank_additive_b200/csrc/fb_ptx.cuh")
+BWD_KERNEL_SOURCES = ("attention_rank_additive_b200/csrc/fb_attn_bwd_sm100.cu",
+                      "attention_rank_additive_b200/csrc/fb_ptx.cuh")
 
 
 def parse_args(argv=None):
@@ -197,24 +199,27 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- profiles
 
-def kernel_source_sha() -> str:
+def kernel_source_sha(sources=KERNEL_SOURCES) -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in sources:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
 def profiled_traffic(cfg_idx: int):
-    """dram bytes per launch of the fused kernel from the committed ncu summary,
-    if it was taken on the current kernel source and this workload; else None."""
-    path = os.path.join(ROOT, "profiles", f"attn_fwd_sm100_{si.CONFIGS[cfg_idx]['name']}.md")
+    """dram bytes per launch of the fused kernel (per call of the two gradient
+    kernels for the backward) from the committed ncu summary, if it was taken
+    on the current kernel source and this workload; else None."""
+    c = si.CONFIGS[cfg_idx]
+    bwd = bool(c.get("bwd"))
+    path = os.path.join(ROOT, "profiles", f"attn_{'bwd' if bwd else 'fwd'}_sm100_{c['name']}.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
     sha = re.search(r"kernel_source_sha:\s*([0-9a-f]+)", text)
     val = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    if not sha or not val or sha.group(1) != kernel_source_sha():
+    if not sha or not val or sha.group(1) != kernel_source_sha(BWD_KERNEL_SOURCES if bwd else KERNEL_SOURCES):
         return None
     return float(val.group(1))
 
@@ -594,7 +599,7 @@ def run_ours(args, rank: int, world: int, local: int):
     peak_tf = sustained_tf if capped else burst_tf
     peak_kind = f"{peak_src} bf16 {'sustained (run power-capped)' if capped else 'burst'}"
     achieved = c["flops"] / (kern_ms * 1e-3) / 1e12
-    traffic = None if w.bwd else profiled_traffic(args.config)
+    traffic = profiled_traffic(args.config)
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
