@@ -595,10 +595,10 @@ int fb_attn_bwd(int dt, int B, int H, int N, int d, const void *Q, const void *K
                                               wsb + L.gq_off, wsb + L.gk_off, st) != cudaSuccess)
       return FB_ERR_CUDA;
   }
-  // 3. per-row LSE in log2 units and rowsum(dO * O)
-  float *lse2 = reinterpret_cast<float *>(wsb + L.l_off);
+  // 3. per-row -LSE in log2 units and rowsum(dO * O)
+  float *nlse2 = reinterpret_cast<float *>(wsb + L.l_off);
   float *delta = reinterpret_cast<float *>(wsb + L.d_off);
-  if (launch_bwd_rows(BH, N, L.Npad, d, O, dO, LSE, lse2, delta, st) != cudaSuccess) return FB_ERR_CUDA;
+  if (launch_bwd_rows(BH, N, L.Npad, d, O, dO, LSE, nlse2, delta, st) != cudaSuccess) return FB_ERR_CUDA;
 
   // 4. the two gradient kernels
   BwdMaps maps;
@@ -628,7 +628,7 @@ int fb_attn_bwd(int dt, int B, int H, int N, int d, const void *Q, const void *K
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.causal = causal ? 1 : 0;
-  a.lse2 = lse2;
+  a.nlse2 = nlse2;
   a.delta = delta;
   a.dQ = dQ, a.dK = dK, a.dV = dV;
   a.dphi_q = dphi_q, a.dphi_k = dphi_k;

@@ -61,6 +61,13 @@ __device__ __forceinline__ void bulk_load_leader(void *dst, const void *src, uin
       : "memory");
 }
 
+// Packed f32x2 multiply (one instruction for two lanes' worth of products).
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
 // K-major tile of ROWS rows x (NCH * CH) 16-bit units stored as NCH swizzled
 // chunks of CH units: descriptor of the base and offset (>> 4) of K-step kk
 // (32 bytes of a row).
@@ -309,7 +316,7 @@ __global__ void __launch_bounds__(320, 1)
         tma_load_3d_leader(st + O_GQ + ch * (BQ * C::GCH * 2), &tm_gq, &ctrl->full[s], ch * C::GCH, q0, fslice,
                            leader);
       const size_t roff = size_t(bh) * args.Npad + q0;
-      bulk_load_leader(st + O_L, args.lse2 + roff, BQ * 4, &ctrl->full[s], leader);
+      bulk_load_leader(st + O_L, args.nlse2 + roff, BQ * 4, &ctrl->full[s], leader);
       bulk_load_leader(st + O_D, args.delta + roff, BQ * 4, &ctrl->full[s], leader);
     }
     if (!ok) {
@@ -408,6 +415,7 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
     const uint32_t s_tm = lane_base + uint32_t(t * 2 * BQ), dp_tm = s_tm + BQ;
     const float sl2 = args.scale_log2;
+    const uint64_t sl2x2 = f2_pack(sl2, sl2);
     bool ok = true;
     for (int u = t; u < nb; u += 2) {
       const int s = u % KS;
@@ -434,21 +442,28 @@ __global__ void __launch_bounds__(320, 1)
         uint32_t pp[16], dd[16];
 #pragma unroll
         for (int e4 = 0; e4 < 8; ++e4) {
+          // sL holds -LSE log2(e): x = S scale log2(e) - LSE log2(e), two columns per instruction
           const float4 l4 = *reinterpret_cast<const float4 *>(sL + 32 * c + 4 * e4);
           const float4 d4 = *reinterpret_cast<const float4 *>(sD + 32 * c + 4 * e4);
-          const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
-          float p[4], g[4];
+          const uint64_t l2[2] = {f2_pack(l4.x, l4.y), f2_pack(l4.z, l4.w)};
+          const uint64_t d2[2] = {f2_pack(d4.x, d4.y), f2_pack(d4.z, d4.w)};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int col = 32 * c + 4 * e4 + e;
-            p[e] = ex2_approx(fmaf(__uint_as_float(sx[4 * e4 + e]), sl2, -lv[e]));
-            if (diag && q0 + col < krow) p[e] = 0.f;
-            g[e] = p[e] * (__uint_as_float(dx[4 * e4 + e]) - dv[e]);
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int i = 4 * e4 + 2 * h2;
+            float a0, a1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sx[i]), __uint_as_float(sx[i + 1])), sl2x2, l2[h2]), a0, a1);
+            float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
+            if (diag) {
+              const int col = 32 * c + i;
+              if (q0 + col < krow) p0 = 0.f;
+              if (q0 + col + 1 < krow) p1 = 0.f;
+            }
+            const uint64_t p2 = f2_pack(p0, p1);
+            float g0, g1;
+            f2_unpack(f2_mul(p2, f2_sub(f2_pack(__uint_as_float(dx[i]), __uint_as_float(dx[i + 1])), d2[h2])), g0, g1);
+            pp[2 * e4 + h2] = pack_bf16x2(p0, p1);
+            dd[2 * e4 + h2] = pack_bf16x2(g0, g1);
           }
-          pp[2 * e4] = pack_bf16x2(p[0], p[1]);
-          pp[2 * e4 + 1] = pack_bf16x2(p[2], p[3]);
-          dd[2 * e4] = pack_bf16x2(g[0], g[1]);
-          dd[2 * e4 + 1] = pack_bf16x2(g[2], g[3]);
         }
         tmem_st16(s_tm + uint32_t(16 * c), pp);
         tmem_st16(dp_tm + uint32_t(16 * c), dd);
@@ -685,8 +700,9 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
     const uint32_t s_tm = lane_base + uint32_t(t * 2 * BK), dp_tm = s_tm + BK;
     const float sl2 = args.scale_log2;
-    const float neg_lse2 = -args.lse2[size_t(bh) * args.Npad + row];  // -inf past N: P = 0
+    const float neg_lse2 = args.nlse2[size_t(bh) * args.Npad + row];  // -inf past N: P = 0
     const float drow = args.delta[size_t(bh) * args.Npad + row];
+    const uint64_t sl2x2 = f2_pack(sl2, sl2), nl2 = f2_pack(neg_lse2, neg_lse2), d2 = f2_pack(drow, drow);
     const int lim = args.causal ? min(row + 1, args.N) : args.N;  // keys [0, lim) are visible
     bool ok = true;
     for (int u = t; u < nb; u += 2) {
@@ -707,16 +723,19 @@ __global__ void __launch_bounds__(320, 1)
         tmem_ld_wait32(dx);
         uint32_t dd[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float g[2];
-#pragma unroll
-          for (int v2 = 0; v2 < 2; ++v2) {
-            const int col = 32 * c + 2 * e + v2;
-            float p = ex2_approx(fmaf(__uint_as_float(sx[2 * e + v2]), sl2, neg_lse2));
-            if (edge && key0 + col >= lim) p = 0.f;
-            g[v2] = p * (__uint_as_float(dx[2 * e + v2]) - drow);
+        for (int e = 0; e < 16; ++e) {  // two keys per packed f32x2 instruction
+          float a0, a1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sx[2 * e]), __uint_as_float(sx[2 * e + 1])), sl2x2, nl2), a0, a1);
+          float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
+          if (edge) {
+            const int col = 32 * c + 2 * e;
+            if (key0 + col >= lim) p0 = 0.f;
+            if (key0 + col + 1 >= lim) p1 = 0.f;
           }
-          dd[e] = pack_bf16x2(g[0], g[1]);
+          float g0, g1;
+          f2_unpack(f2_mul(f2_pack(p0, p1), f2_sub(f2_pack(__uint_as_float(dx[2 * e]), __uint_as_float(dx[2 * e + 1])), d2)),
+                    g0, g1);
+          dd[e] = pack_bf16x2(g0, g1);
         }
         tmem_st16(s_tm + uint32_t(16 * c), dd);
       }

@@ -319,14 +319,14 @@ cudaError_t launch_prep_factors(int mode, int B, int H, int N, int R, int RP, co
   return cudaGetLastError();
 }
 
-// Backward rows: lse2 = LSE log2(e) and delta = rowsum(dO * O) (fp32 sum of
+// Backward rows: nlse2 = -LSE log2(e) and delta = rowsum(dO * O) (fp32 sum of
 // the bf16 products). Eight threads per row, 16 bytes of O and dO each per
-// step (d % 8 == 0); rows N .. Npad-1 get +inf and 0, so the kernels' padded
+// step (d % 8 == 0); rows N .. Npad-1 get -inf and 0, so the kernels' padded
 // queries carry P = 0 without a bounds test.
 __global__ void __launch_bounds__(256) bwd_rows_kernel(long long rows, int N, int Npad, int d,
                                                        const __nv_bfloat16 *__restrict__ O,
                                                        const __nv_bfloat16 *__restrict__ dO,
-                                                       const float *__restrict__ LSE, float *__restrict__ lse2,
+                                                       const float *__restrict__ LSE, float *__restrict__ nlse2,
                                                        float *__restrict__ delta) {
   const long long w = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 3;  // row
   const int sub = threadIdx.x & 7;
@@ -351,7 +351,7 @@ __global__ void __launch_bounds__(256) bwd_rows_kernel(long long rows, int N, in
   acc += __shfl_xor_sync(0xffffffffu, acc, 2);
   acc += __shfl_xor_sync(0xffffffffu, acc, 1);
   if (sub == 0) {
-    lse2[w] = n < N ? LSE[size_t(bh) * N + n] * 1.4426950408889634f : INFINITY;
+    nlse2[w] = n < N ? -LSE[size_t(bh) * N + n] * 1.4426950408889634f : -INFINITY;
     delta[w] = acc;
   }
 }
@@ -381,12 +381,12 @@ __global__ void prep_grad_factors_kernel(int N, int R, int RG, int fac_H, const 
 }
 
 cudaError_t launch_bwd_rows(int BH, int N, int Npad, int d, const void *O, const void *dO, const float *LSE,
-                            float *lse2, float *delta, cudaStream_t s) {
+                            float *nlse2, float *delta, cudaStream_t s) {
   const long long rows = (long long)BH * Npad;  // a multiple of 128: full warps
   const long long blocks = (rows * 8 + 255) / 256;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
   bwd_rows_kernel<<<unsigned(blocks), 256, 0, s>>>(rows, N, Npad, d, static_cast<const __nv_bfloat16 *>(O),
-                                                   static_cast<const __nv_bfloat16 *>(dO), LSE, lse2, delta);
+                                                   static_cast<const __nv_bfloat16 *>(dO), LSE, nlse2, delta);
   return cudaGetLastError();
 }
 

@@ -85,7 +85,7 @@ struct BwdArgs {
   int Npad;                // n_kv * 128: row stride of lse2 / delta
   float scale, scale_log2;
   int causal;
-  const float *lse2;       // [BH, Npad] LSE * log2(e); +inf past N
+  const float *nlse2;      // [BH, Npad] -LSE * log2(e); -inf past N
   const float *delta;      // [BH, Npad] rowsum(dO * O); 0 past N
   void *dQ, *dK, *dV;      // bf16 [BH, N, d]
   float *dphi_q, *dphi_k;  // fp32, laid out like phi_q / phi_k
@@ -117,9 +117,9 @@ struct BwdMaps {
 int bwd_query_block_rows(const BwdPlan &p);
 int bwd_key_block_rows(const BwdPlan &p);
 cudaError_t bwd_launch(const BwdPlan &p, const BwdMaps &maps, const BwdArgs &a, cudaStream_t stream);
-// lse2 = LSE * log2(e) and delta = rowsum(dO * O) per row, padded to Npad.
+// nlse2 = -LSE * log2(e) and delta = rowsum(dO * O) per row, padded to Npad.
 cudaError_t launch_bwd_rows(int BH, int N, int Npad, int d, const void *O, const void *dO, const float *LSE,
-                            float *lse2, float *delta, cudaStream_t s);
+                            float *nlse2, float *delta, cudaStream_t s);
 // bf16 copies of the factors [FB, N, RG] (zero-padded).
 cudaError_t launch_prep_grad_factors(int N, int R, int RG, const float *phi_q, const float *phi_k, int64_t bs,
                                      int64_t hs, int fac_B, int fac_H, void *gq, void *gk, cudaStream_t s);
