@@ -379,6 +379,10 @@ BWD_SWEEP = [
     (1, 1, 513, 40, 4, False, "bhnr"),
     (1, 2, 700, 64, 0, True, "bhnr"),
     (1, 1, 400, 96, 100, False, "bhnr"),
+    (2, 3, 129, 8, 4, True, "hnr"),      # d = 8 (head dim 16 padded), ragged by one row, head-shared factors
+    (1, 1, 640, 128, 16, True, "bhnr"),  # head dim 128 with 32-row query blocks, several diagonal blocks
+    (3, 2, 96, 64, 64, False, "nr"),     # one factor slice for all six heads, N below one tile
+    (1, 1, 1024, 32, 0, False, "bhnr"),  # plain attention, many blocks
 ]
 
 
