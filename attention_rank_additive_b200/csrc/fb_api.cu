@@ -585,22 +585,10 @@ int fb_attn_bwd(int dt, int B, int H, int N, int d, const void *Q, const void *K
   const int fac_B = phi_bstride == 0 ? 1 : B, fac_H = phi_hstride == 0 ? 1 : H;
   const int FB = fac_B * fac_H;
   const int BH = B * H;
-  // 1. the forward's factor tiles (S is recomputed as the forward computed it)
-  if (R > 0) {
-    const int rc = fb_attn_prepare_factors(B, H, N, R, phi_q, phi_k, phi_bstride, phi_hstride, scale, workspace,
-                                           workspace_bytes, stream);
-    if (rc != FB_OK) return rc;
-    // 2. bf16 factor copies for the gradient products; zeroed factor gradients
-    if (want_dphi && launch_prep_grad_factors(N, R, L.RG, phi_q, phi_k, phi_bstride, phi_hstride, fac_B, fac_H,
-                                              wsb + L.gq_off, wsb + L.gk_off, st) != cudaSuccess)
-      return FB_ERR_CUDA;
-  }
-  // 3. per-row -LSE in log2 units and rowsum(dO * O)
   float *nlse2 = reinterpret_cast<float *>(wsb + L.l_off);
   float *delta = reinterpret_cast<float *>(wsb + L.d_off);
-  if (launch_bwd_rows(BH, N, L.Npad, d, O, dO, LSE, nlse2, delta, st) != cudaSuccess) return FB_ERR_CUDA;
 
-  // 4. the two gradient kernels
+  // tensor maps first: a failure here returns before anything is launched
   BwdMaps maps;
   std::memset(&maps, 0, sizeof(maps));
   const int DP = plan.DP;
@@ -620,6 +608,21 @@ int fb_attn_bwd(int dt, int B, int H, int N, int d, const void *Q, const void *K
                       !encode_rows_bf16(&maps.gk_blk, wsb + L.gk_off, FB, N, L.RG, L.RG, BK)))
       return FB_ERR_CUDA;
   }
+
+  // 1. the forward's factor tiles (S is recomputed as the forward computed it)
+  if (R > 0) {
+    const int rc = fb_attn_prepare_factors(B, H, N, R, phi_q, phi_k, phi_bstride, phi_hstride, scale, workspace,
+                                           workspace_bytes, stream);
+    if (rc != FB_OK) return rc;
+    // 2. bf16 factor copies for the gradient products
+    if (want_dphi && launch_prep_grad_factors(N, R, L.RG, phi_q, phi_k, phi_bstride, phi_hstride, fac_B, fac_H,
+                                              wsb + L.gq_off, wsb + L.gk_off, st) != cudaSuccess)
+      return FB_ERR_CUDA;
+  }
+  // 3. per-row -LSE in log2 units and rowsum(dO * O)
+  if (launch_bwd_rows(BH, N, L.Npad, d, O, dO, LSE, nlse2, delta, st) != cudaSuccess) return FB_ERR_CUDA;
+
+  // 4. the two gradient kernels
   BwdArgs a;
   std::memset(&a, 0, sizeof(a));
   a.B = B, a.H = H, a.N = N, a.d = d, a.R = R;
