@@ -42,7 +42,7 @@ extern "C" {
 typedef enum {
   FB_OK = 0,
   FB_ERR_INVALID_ARG = 1, /* null pointer, bad shape, bad stride, bad scale   */
-  FB_ERR_UNSUPPORTED = 2, /* valid but outside what this build implements     */
+  FB_ERR_UNSUPPORTED = 2, /* valid but outside what the library implements   */
   FB_ERR_RANGE = 3,       /* a factor value does not fit the kernel's type    */
   FB_ERR_WORKSPACE = 4,   /* workspace missing, too small or misaligned       */
   FB_ERR_CUDA = 5,        /* CUDA runtime/driver call or launch failed        */
