@@ -328,3 +328,30 @@ def attention_lowrank_bwd_head(q, k, v, phi_q, phi_k, do, scale: float, causal: 
         "dphi_k": ds.T @ pq,
         "delta": delta[:, 0],
     }
+
+
+def neural_bwd(x_q, x_k, w_q, w_k, q, k, v, do, scale: float, causal: bool):
+    """Gradients of the neural-decomposition attention (rebuttal, reply to
+    Reviewer xU4x, Q4: phi_q[b, h] = x_q[b] w_q[h], phi_k[b, h] = x_k[b] w_k[h])
+    for an upstream gradient do, in fp64: the factor gradients of every head
+    from ``attention_lowrank_bwd_head``, then the chain rule through the linear
+    layers, dw[h] = sum_b x[b]^T dphi[b, h] and dx[b] = sum_h dphi[b, h] w[h]^T.
+    x [B, N, F], w [H, F, R], q, k, v, do [B, H, N, d]. Returns a dict with
+    dq, dk, dv [B, H, N, d], dx_q, dx_k [B, N, F] and dw_q, dw_k [H, F, R]."""
+    xq, xk, wq, wk = _f64(x_q), _f64(x_k), _f64(w_q), _f64(w_k)
+    B, H, N, d = np.shape(q)
+    pq, pk = neural_factors(xq, xk, wq, wk)
+    out = {n: np.zeros((B, H, N, d)) for n in ("dq", "dk", "dv")}
+    dpq = np.zeros(pq.shape)
+    dpk = np.zeros(pk.shape)
+    for b in range(B):
+        for h in range(H):
+            r = attention_lowrank_bwd_head(q[b, h], k[b, h], v[b, h], pq[b, h], pk[b, h], do[b, h], scale, causal)
+            for n in ("dq", "dk", "dv"):
+                out[n][b, h] = r[n]
+            dpq[b, h], dpk[b, h] = r["dphi_q"], r["dphi_k"]
+    out["dw_q"] = np.einsum("bnf,bhnr->hfr", xq, dpq)
+    out["dw_k"] = np.einsum("bnf,bhnr->hfr", xk, dpk)
+    out["dx_q"] = np.einsum("bhnr,hfr->bnf", dpq, wq)
+    out["dx_k"] = np.einsum("bhnr,hfr->bnf", dpk, wk)
+    return out

@@ -423,3 +423,39 @@ def test_backward_row_subset_matches_whole_head(causal):
     part = oracle.attention_lowrank_bwd_head(q, k, v, pq, pk, g, 0.4, causal, rows=rows)
     for key in ("dq", "dphi_q", "delta"):
         np.testing.assert_allclose(part[key], full[key][rows], rtol=0, atol=1e-13)
+
+
+def test_neural_backward_matches_finite_differences():
+    """Gradients of the linear layers of the neural decomposition against a
+    central difference of the forward definition (the factors as library
+    matmuls of the features and weights, attention by the C oracle)."""
+    B, H, N, d, F, R = 1, 2, 5, 3, 3, 2
+    xq, xk = _rand((B, N, F), 71, 0.7), _rand((B, N, F), 72, 0.7)
+    wq, wk = _rand((H, F, R), 73, 0.7), _rand((H, F, R), 74, 0.7)
+    q, k, v = (_rand((B, H, N, d), s) for s in (75, 76, 77))
+    g = _rand((B, H, N, d), 78)
+    scale = 0.6
+
+    def loss():
+        pq, pk = np.einsum("bnf,hfr->bhnr", xq, wq), np.einsum("bnf,hfr->bhnr", xk, wk)
+        tot = 0.0
+        for b in range(B):
+            for h in range(H):
+                o, _ = oracle.attention_head(q[b, h], k[b, h], v[b, h], HeadBias.lowrank(pq[b, h], pk[b, h]),
+                                             scale, True)
+                tot += float(np.sum(o * g[b, h]))
+        return tot
+
+    out = oracle.neural_bwd(xq, xk, wq, wk, q, k, v, g, scale, True)
+    step = 1e-6
+    for name, x in (("dx_q", xq), ("dx_k", xk), ("dw_q", wq), ("dw_k", wk)):
+        fd = np.empty_like(x)
+        for idx in np.ndindex(x.shape):
+            x0 = x[idx]
+            x[idx] = x0 + step
+            up = loss()
+            x[idx] = x0 - step
+            dn = loss()
+            x[idx] = x0
+            fd[idx] = (up - dn) / (2 * step)
+        np.testing.assert_allclose(out[name], fd, rtol=0, atol=5e-8, err_msg=name)
