@@ -42,7 +42,7 @@ EXPORTED = (
     "fb_selftest_wait_timeout", "fb_attn_fwd_noalloc", "fb_attn_prepare_factors", "fb_attn_fwd_prepared",
     "fb_attn_mul_bias_workspace_bytes", "fb_attn_mul_bias_fwd", "fb_svd_device_workspace_bytes",
     "fb_svd_factors_device", "fb_attn_neural_workspace_bytes", "fb_attn_neural_fwd", "fb_attn_bwd_workspace_bytes",
-    "fb_attn_bwd",
+    "fb_attn_bwd", "fb_attn_neural_bwd_workspace_bytes", "fb_attn_neural_bwd",
 )
 
 
@@ -98,6 +98,11 @@ def lib() -> ctypes.CDLL:
         L.fb_attn_bwd.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, i32, vp, vp, i64, i64, f32, i32, vp, vp, vp,
                                   vp, vp, vp, vp, vp, vp, sz, vp]
         L.fb_attn_bwd.restype = i32
+        L.fb_attn_neural_bwd_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
+        L.fb_attn_neural_bwd_workspace_bytes.restype = sz
+        L.fb_attn_neural_bwd.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, i32, i32, vp, vp, vp, vp, f32, i32, vp,
+                                         vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.fb_attn_neural_bwd.restype = i32
         L.fb_attn_dense_bias_fwd.argtypes = [i32, i32, i32, i32, i32, vp, vp, vp, vp, i64, i64, f32, i32, vp, vp, vp]
         L.fb_attn_dense_bias_fwd.restype = i32
         L.fb_factors_sandwich.argtypes, L.fb_factors_sandwich.restype = [i32, i32, vp, vp, vp], i32
@@ -262,6 +267,43 @@ def attn_bwd(q, k, v, phi_q, phi_k, o, lse, do, scale=None, causal=False, worksp
                        int(bool(causal)), o.data_ptr(), lse.data_ptr(), do.data_ptr(), dq.data_ptr(), dk.data_ptr(),
                        dv.data_ptr(), gq, gk, workspace.data_ptr(), nb, _stream(q.device)), "fb_attn_bwd")
     return dq, dk, dv, dpq, dpk
+
+
+def fb_attn_neural_bwd_workspace_bytes(B, H, N, F, R) -> int:
+    return lib().fb_attn_neural_bwd_workspace_bytes(B, H, N, F, R)
+
+
+def fb_attn_neural_bwd(dt, B, H, N, d, Q, K, V, F, R, X_q, X_k, W_q, W_k, scale, causal, O, LSE, dO, dQ, dK, dV,
+                       dX_q, dX_k, dW_q, dW_k, workspace, workspace_bytes, stream) -> int:
+    return lib().fb_attn_neural_bwd(dt, B, H, N, d, Q, K, V, F, R, X_q, X_k, W_q, W_k, scale, causal, O, LSE, dO, dQ,
+                                    dK, dV, dX_q, dX_k, dW_q, dW_k, workspace, workspace_bytes, stream)
+
+
+def attn_neural_bwd(q, k, v, x_q, x_k, w_q, w_k, o, lse, do, scale=None, causal=False, feature_grads=True):
+    """Gradients of attn_neural's O for an upstream gradient do
+    (fb_attn_neural_bwd). Returns (dq, dk, dv, dx_q, dx_k, dw_q, dw_k); dx
+    are None with feature_grads=False."""
+    import torch
+    for t in (q, k, v, o, do):
+        assert t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous()
+    for t in (x_q, x_k, w_q, w_k):
+        assert t.is_cuda and t.dtype == torch.float32 and t.is_contiguous()
+    B, H, N, d = q.shape
+    F, R = w_q.shape[1], w_q.shape[2]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dwq, dwk = torch.empty_like(w_q), torch.empty_like(w_k)
+    dxq = torch.empty_like(x_q) if feature_grads else None
+    dxk = torch.empty_like(x_k) if feature_grads else None
+    nb = fb_attn_neural_bwd_workspace_bytes(B, H, N, F, R)
+    ws = torch.empty(max(nb, 1), device=q.device, dtype=torch.uint8)
+    _check(fb_attn_neural_bwd(FB_BF16, B, H, N, d, q.data_ptr(), k.data_ptr(), v.data_ptr(), F, R, x_q.data_ptr(),
+                              x_k.data_ptr(), w_q.data_ptr(), w_k.data_ptr(), scale, int(bool(causal)), o.data_ptr(),
+                              lse.data_ptr(), do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                              dxq.data_ptr() if dxq is not None else 0, dxk.data_ptr() if dxk is not None else 0,
+                              dwq.data_ptr(), dwk.data_ptr(), ws.data_ptr(), nb, _stream(q.device)),
+           "fb_attn_neural_bwd")
+    return dq, dk, dv, dxq, dxk, dwq, dwk
 
 
 def fb_attn_fwd_noalloc(dt, B, H, N, d, Q, K, V, R, phi_q, phi_k, phi_bstride, phi_hstride, scale, causal, O, LSE,

@@ -414,6 +414,55 @@ int fb_attn_neural_fwd(int dt, int B, int H, int N, int d, const void *Q, const 
                      m.prep_bytes, stream);
 }
 
+size_t fb_attn_neural_bwd_workspace_bytes(int B, int H, int N, int F, int R) {
+  if (B < 1 || H < 1 || N < 1 || !neural_ok(F, R)) return 0;
+  const size_t phi = align256(size_t(B) * H * N * R * 4);
+  const int64_t hs = int64_t(N) * R, bs = int64_t(H) * hs;
+  const size_t bwd = fb_attn_bwd_workspace_bytes(B, H, N, R, bs, hs);
+  return bwd == 0 ? 0 : 4 * phi + bwd;
+}
+
+int fb_attn_neural_bwd(int dt, int B, int H, int N, int d, const void *Q, const void *K, const void *V, int F,
+                       int R, const float *X_q, const float *X_k, const float *W_q, const float *W_k, float scale,
+                       int causal, const void *O, const float *LSE, const void *dO, void *dQ, void *dK, void *dV,
+                       float *dX_q, float *dX_k, float *dW_q, float *dW_k, void *workspace, size_t workspace_bytes,
+                       void *stream) {
+  if (!Q || !K || !V || !O || !LSE || !dO || !dQ || !dK || !dV || !X_q || !X_k || !W_q || !W_k || !dW_q || !dW_k)
+    return FB_ERR_INVALID_ARG;
+  if ((dX_q == nullptr) != (dX_k == nullptr)) return FB_ERR_INVALID_ARG;  // both or neither
+  if (dt != FB_BF16) return FB_ERR_UNSUPPORTED;
+  if (!neural_ok(F, R)) return FB_ERR_UNSUPPORTED;
+  if (!valid_scale(scale)) return FB_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE) || !aligned16(dO) ||
+      !aligned16(dQ) || !aligned16(dK) || !aligned16(dV))
+    return FB_ERR_INVALID_ARG;
+  if (((reinterpret_cast<uintptr_t>(X_q) | reinterpret_cast<uintptr_t>(X_k) | reinterpret_cast<uintptr_t>(W_q) |
+        reinterpret_cast<uintptr_t>(W_k) | reinterpret_cast<uintptr_t>(dW_q) | reinterpret_cast<uintptr_t>(dW_k) |
+        reinterpret_cast<uintptr_t>(dX_q) | reinterpret_cast<uintptr_t>(dX_k)) & 3u) != 0)
+    return FB_ERR_INVALID_ARG;
+  if (!valid_shape_bf16(B, H, N, d)) return FB_ERR_UNSUPPORTED;
+  const size_t need = fb_attn_neural_bwd_workspace_bytes(B, H, N, F, R);
+  if (need == 0) return FB_ERR_UNSUPPORTED;
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return FB_ERR_WORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  const size_t phi = align256(size_t(B) * H * N * R * 4);
+  float *pq = reinterpret_cast<float *>(ws), *pk = reinterpret_cast<float *>(ws + phi);
+  float *dpq = reinterpret_cast<float *>(ws + 2 * phi), *dpk = reinterpret_cast<float *>(ws + 3 * phi);
+  // the factors again (as the forward made them), the attention backward with
+  // per-head factors, then the chain rule through the linear layers
+  if (launch_neural_factors(B, H, N, F, R, X_q, X_k, W_q, W_k, pq, pk, st) != cudaSuccess) return FB_ERR_CUDA;
+  const int64_t hs = int64_t(N) * R, bs = int64_t(H) * hs;
+  const int rc = fb_attn_bwd(FB_BF16, B, H, N, d, Q, K, V, R, pq, pk, bs, hs, scale, causal, O, LSE, dO, dQ, dK, dV,
+                             dpq, dpk, ws + 4 * phi, need - 4 * phi, stream);
+  if (rc != FB_OK) return rc;
+  return launch_neural_grads(B, H, N, F, R, X_q, X_k, W_q, W_k, dpq, dpk, dW_q, dW_k, dX_q, dX_k, st) ==
+                 cudaSuccess
+             ? FB_OK
+             : FB_ERR_CUDA;
+}
+
 int fb_attn_dense_bias_fwd(int dt, int B, int H, int N, int d, const void *Q, const void *K, const void *V,
                            const void *Bias, int64_t bias_bstride, int64_t bias_hstride, float scale, int causal,
                            void *O, float *LSE, void *stream) {

@@ -434,6 +434,60 @@ cudaError_t launch_reduce_factor_grads(int B, int H, int N, int R, int fac_B, in
   return cudaGetLastError();
 }
 
+// Gradients of the neural decomposition's linear layers from the factor
+// gradients dphi [B, H, N, R]: dW[h, f, r] = sum_b sum_n X[b, n, f] dphi[b, h, n, r]
+// (one thread per weight; the warp's lanes run along r, so the dphi loads
+// coalesce and the X load is a broadcast) and dX[b, n, f] = sum_h sum_r
+// dphi[b, h, n, r] W[h, f, r] (one thread per feature). fp32, fixed order.
+__global__ void neural_grad_w_kernel(int B, int H, int N, int F, int R, const float *__restrict__ X,
+                                     const float *__restrict__ dphi, float *__restrict__ dW, long long total) {
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int r = int(idx % R);
+    const int f = int((idx / R) % F);
+    const int h = int(idx / ((long long)R * F));
+    float acc = 0.f;
+    for (int b = 0; b < B; ++b) {
+      const float *xb = X + (long long)b * N * F + f;
+      const float *gb = dphi + ((long long)b * H + h) * N * R + r;
+      for (int n = 0; n < N; ++n) acc = fmaf(xb[(long long)n * F], gb[(long long)n * R], acc);
+    }
+    dW[idx] = acc;
+  }
+}
+
+__global__ void neural_grad_x_kernel(int B, int H, int N, int F, int R, const float *__restrict__ W,
+                                     const float *__restrict__ dphi, float *__restrict__ dX, long long total) {
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int f = int(idx % F);
+    const long long bn = idx / F;
+    const int n = int(bn % N);
+    const int b = int(bn / N);
+    float acc = 0.f;
+    for (int h = 0; h < H; ++h) {
+      const float *g = dphi + (((long long)b * H + h) * N + n) * R;
+      const float *w = W + ((long long)h * F + f) * R;
+      for (int r = 0; r < R; ++r) acc = fmaf(g[r], w[r], acc);
+    }
+    dX[idx] = acc;
+  }
+}
+
+cudaError_t launch_neural_grads(int B, int H, int N, int F, int R, const float *Xq, const float *Xk,
+                                const float *Wq, const float *Wk, const float *dpq, const float *dpk, float *dWq,
+                                float *dWk, float *dXq, float *dXk, cudaStream_t s) {
+  const long long nw = (long long)H * F * R;
+  neural_grad_w_kernel<<<grid_for(nw, 128), 128, 0, s>>>(B, H, N, F, R, Xq, dpq, dWq, nw);
+  neural_grad_w_kernel<<<grid_for(nw, 128), 128, 0, s>>>(B, H, N, F, R, Xk, dpk, dWk, nw);
+  if (dXq != nullptr && dXk != nullptr) {
+    const long long nx = (long long)B * N * F;
+    neural_grad_x_kernel<<<grid_for(nx, 256), 256, 0, s>>>(B, H, N, F, R, Wq, dpq, dXq, nx);
+    neural_grad_x_kernel<<<grid_for(nx, 256), 256, 0, s>>>(B, H, N, F, R, Wk, dpk, dXk, nx);
+  }
+  return cudaGetLastError();
+}
+
 cudaError_t launch_wait_selftest(int limit_ms, int *flags, cudaStream_t s) {
   wait_selftest_kernel<<<1, 32, 0, s>>>((unsigned long long)limit_ms * 1000000ull, flags);
   return cudaGetLastError();

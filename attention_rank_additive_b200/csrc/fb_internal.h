@@ -74,6 +74,11 @@ cudaError_t launch_wait_selftest(int limit_ms, int *flags, cudaStream_t s);
 // Neural decomposition: phi_q[b, h] = X_q[b] W_q[h], phi_k[b, h] = X_k[b] W_k[h] (fp32).
 cudaError_t launch_neural_factors(int B, int H, int N, int F, int R, const float *Xq, const float *Xk,
                                   const float *Wq, const float *Wk, float *pq, float *pk, cudaStream_t s);
+// Gradients of the neural decomposition's linear layers: dW [H, F, R] from X and
+// dphi [B, H, N, R]; dX [B, N, F] from W and dphi (skipped when dXq or dXk is null).
+cudaError_t launch_neural_grads(int B, int H, int N, int F, int R, const float *Xq, const float *Xk,
+                                const float *Wq, const float *Wk, const float *dpq, const float *dpk, float *dWq,
+                                float *dWk, float *dXq, float *dXk, cudaStream_t s);
 cudaError_t launch_prep_mul_bias(int B, int H, int N, int d, int R, int RP, const void *Q, const void *K,
                                  const float *phi_q, const float *phi_k, int64_t bs, int64_t hs, void *q1, void *k1,
                                  void *fq, void *fk, int *flags, cudaStream_t s);

@@ -251,6 +251,37 @@ int fb_attn_bwd(int dt, int B, int H, int N, int d,
                 void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Backward of fb_attn_neural_fwd: the gradients of O for an upstream
+ * gradient dO, down to the features and the weights of the two linear
+ * layers of the neural decomposition (rebuttal, reply to Reviewer xU4x, Q4):
+ *
+ *   dphi_q, dphi_k     as fb_attn_bwd, per (b, h)
+ *   dW_q[h] = sum_b X_q[b]^T dphi_q[b, h],  dX_q[b] = sum_h dphi_q[b, h] W_q[h]^T
+ *   (and the same for k)
+ *
+ *  Q..W_k      the forward's inputs; O, LSE its outputs; dO bf16 [B,H,N,d].
+ *  dQ, dK, dV  bf16 [B,H,N,d] device outputs, 16-byte aligned.
+ *  dW_q, dW_k  fp32 [H, F, R] device outputs.
+ *  dX_q, dX_k  fp32 [B, N, F] device outputs, or both NULL (fixed features).
+ *  workspace   fb_attn_neural_bwd_workspace_bytes(B, H, N, F, R) bytes,
+ *              256-byte aligned.
+ * The factors are recomputed as the forward made them; the attention part is
+ * fb_attn_bwd's; the linear-layer gradients run in fp32 on the CUDA cores.
+ * Limits, arguments and errors as fb_attn_neural_fwd and fb_attn_bwd.
+ */
+size_t fb_attn_neural_bwd_workspace_bytes(int B, int H, int N, int F, int R);
+
+int fb_attn_neural_bwd(int dt, int B, int H, int N, int d,
+                       const void *Q, const void *K, const void *V,
+                       int F, int R, const float *X_q, const float *X_k,
+                       const float *W_q, const float *W_k,
+                       float scale, int causal,
+                       const void *O, const float *LSE, const void *dO,
+                       void *dQ, void *dK, void *dV,
+                       float *dX_q, float *dX_k, float *dW_q, float *dW_k,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Truncated SVD of H dense biases on the GPU, for biases known only at call
  * time (the SVD decomposition of the rebuttal, reply to Reviewer xU4x, Q6,
  * done per call; the rebuttal calls this inefficient for dynamic biases,

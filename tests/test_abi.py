@@ -357,3 +357,36 @@ def test_backward_workspace_and_argument_errors():
     assert b(workspace=0) == fb.FB_ERR_WORKSPACE
     assert b(workspace_bytes=need - 1) == fb.FB_ERR_WORKSPACE
     assert b(workspace=FAKE + 16) == fb.FB_ERR_WORKSPACE
+
+
+def test_neural_backward_workspace_and_argument_errors():
+    """fb_attn_neural_bwd: the workspace holds the factors, their gradients and
+    fb_attn_bwd's own (per-head factor slices); argument errors return before a
+    launch."""
+    al = lambda x: (x + 255) // 256 * 256
+    B, H, N, F, R = 2, 3, 100, 16, 8
+    phi = al(B * H * N * R * 4)
+    assert fb.fb_attn_neural_bwd_workspace_bytes(B, H, N, F, R) == \
+        4 * phi + fb.fb_attn_bwd_workspace_bytes(B, H, N, R, H * N * R, N * R)
+    assert fb.fb_attn_neural_bwd_workspace_bytes(B, H, N, 128, 128) == 0  # F R > 8192
+    need = fb.fb_attn_neural_bwd_workspace_bytes(1, 2, 128, F, R)
+    run = dict(dt=fb.FB_BF16, B=1, H=2, N=128, d=64, Q=FAKE, K=FAKE, V=FAKE, F=F, R=R, X_q=FAKE, X_k=FAKE,
+               W_q=FAKE, W_k=FAKE, scale=0.125, causal=1, O=FAKE, LSE=FAKE, dO=FAKE, dQ=FAKE, dK=FAKE, dV=FAKE,
+               dX_q=FAKE, dX_k=FAKE, dW_q=FAKE, dW_k=FAKE, workspace=FAKE, workspace_bytes=need, stream=None)
+
+    def n(**kw):
+        a = dict(run)
+        a.update(kw)
+        return fb.fb_attn_neural_bwd(**a)
+
+    assert n(dt=fb.FB_F32) == fb.FB_ERR_UNSUPPORTED
+    assert n(F=0) == fb.FB_ERR_UNSUPPORTED
+    assert n(R=129) == fb.FB_ERR_UNSUPPORTED
+    assert n(dW_k=0) == fb.FB_ERR_INVALID_ARG
+    assert n(dX_q=0) == fb.FB_ERR_INVALID_ARG  # one feature gradient without the other
+    assert n(W_q=FAKE + 2) == fb.FB_ERR_INVALID_ARG
+    assert n(dV=FAKE + 8) == fb.FB_ERR_INVALID_ARG
+    assert n(scale=0.0) == fb.FB_ERR_INVALID_ARG
+    assert n(d=20) == fb.FB_ERR_UNSUPPORTED
+    assert n(workspace=0) == fb.FB_ERR_WORKSPACE
+    assert n(workspace_bytes=need - 1) == fb.FB_ERR_WORKSPACE

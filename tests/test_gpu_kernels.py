@@ -455,3 +455,24 @@ def test_backward_fixed_factors_matches_oracle(B, H, N, d, R, causal):
                                                   causal)
             for n in ("dq", "dk", "dv"):
                 grad_close(got[n][b, h], r[n], f"{n} ({b},{h}) fixed factors N{N} d{d} R{R}")
+
+
+@pytest.mark.parametrize("B,H,N,d,F,R,causal", [(2, 3, 200, 64, 16, 8, True), (1, 2, 130, 24, 64, 32, False)])
+def test_neural_backward_matches_oracle(B, H, N, d, F, R, causal):
+    """The neural decomposition's backward (fb_attn_neural_bwd) down to the
+    linear layers' features and weights."""
+    seed = 2900 + N + F
+    q, k, v = si.qkv(B, H, N, d, seed, "bf16")
+    g = si.round_to_bf16(si.normal((B, H, N, d), seed + 3))
+    xq, xk, wq, wk = si.neural_inputs(B, H, N, F, R, seed + 5)
+    scale = 1.0 / math.sqrt(d)
+    tq, tk, tv, tg = (dev(x, "bf16") for x in (q, k, v, g))
+    txq, txk, twq, twk = (dev(x, "f32") for x in (xq, xk, wq, wk))
+    o, lse = fb.attn_neural(tq, tk, tv, txq, txk, twq, twk, scale=scale, causal=causal)
+    dq, dk, dv, dxq, dxk, dwq, dwk = fb.attn_neural_bwd(tq, tk, tv, txq, txk, twq, twk, o, lse, tg, scale=scale,
+                                                        causal=causal)
+    torch.cuda.synchronize()
+    _no_device_error()
+    ref = oracle.neural_bwd(xq, xk, wq, wk, q, k, v, g, scale, causal)
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv), ("dx_q", dxq), ("dx_k", dxk), ("dw_q", dwq), ("dw_k", dwk)):
+        grad_close(host(t), ref[name], f"{name} B{B} H{H} N{N} d{d} F{F} R{R} c{causal}")
