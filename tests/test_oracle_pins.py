@@ -459,3 +459,49 @@ def test_neural_backward_matches_finite_differences():
             x[idx] = x0
             fd[idx] = (up - dn) / (2 * step)
         np.testing.assert_allclose(out[name], fd, rtol=0, atol=5e-8, err_msg=name)
+
+
+def test_backward_single_key_closed_form():
+    """One key: P = 1 whatever the scores, so dV = dO and every score
+    gradient (dq, dk, dphi_q, dphi_k) is exactly zero."""
+    q, k, v = (_rand((1, 4), s) for s in (81, 82, 83))
+    pq, pk = _rand((1, 2), 84), _rand((1, 2), 85)
+    g = _rand((1, 4), 86)
+    out = oracle.attention_lowrank_bwd_head(q, k, v, pq, pk, g, 0.5, True)
+    np.testing.assert_array_equal(out["dv"], g)
+    for name in ("dq", "dk", "dphi_q", "dphi_k"):
+        np.testing.assert_array_equal(out[name], 0.0)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_uniform_attention_by_loops(causal):
+    """q = 0 and a zero bias give uniform attention over the visible keys,
+    P_ij = 1 / n_i. The gradients then follow from the definition alone,
+    written here as plain loops: dv_j = sum_i dO_i / n_i, and with
+    dP_ij = dO_i . v_j, dS_ij = (dP_ij - mean_j dP_ij) / n_i,
+    dq_i = scale sum_j dS_ij k_j, dk_j = scale sum_i dS_ij q_i = 0."""
+    N, d, R = 7, 3, 2
+    q = np.zeros((N, d))
+    k, v = _rand((N, d), 91), _rand((N, d), 92)
+    pq, pk = np.zeros((N, R)), _rand((N, R), 93)
+    g = _rand((N, d), 94)
+    scale = 0.8
+    out = oracle.attention_lowrank_bwd_head(q, k, v, pq, pk, g, scale, causal)
+    dv = np.zeros((N, d))
+    dq = np.zeros((N, d))
+    dphi_q = np.zeros((N, R))
+    for i in range(N):
+        vis = list(range(i + 1)) if causal else list(range(N))
+        n = len(vis)
+        dp = [float(np.dot(g[i], v[j])) for j in vis]
+        mean = sum(dp) / n
+        for t, j in enumerate(vis):
+            dv[j] += g[i] / n
+            ds = (dp[t] - mean) / n
+            dq[i] += scale * ds * k[j]
+            dphi_q[i] += ds * pk[j]
+    np.testing.assert_allclose(out["dv"], dv, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(out["dq"], dq, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(out["dphi_q"], dphi_q, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(out["dk"], 0.0, atol=1e-15)
+    np.testing.assert_allclose(out["dphi_k"], 0.0, atol=1e-15)
