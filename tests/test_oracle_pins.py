@@ -505,3 +505,40 @@ def test_backward_uniform_attention_by_loops(causal):
     np.testing.assert_allclose(out["dphi_q"], dphi_q, rtol=0, atol=1e-13)
     np.testing.assert_allclose(out["dk"], 0.0, atol=1e-15)
     np.testing.assert_allclose(out["dphi_k"], 0.0, atol=1e-15)
+
+
+@pytest.mark.parametrize("mistake", ["dk_without_scale", "delta_dropped", "factor_grads_swapped", "dv_untransposed"])
+def test_backward_pin_catches_planted_mistakes(mistake, monkeypatch):
+    """Each plausible slip in the backward (a dropped scale, the rowsum term
+    left out, the two factor gradients exchanged, P instead of P^T for dV),
+    planted in the oracle on the CPU, fails the finite-difference pin."""
+    true_bwd = oracle.attention_lowrank_bwd_head
+
+    def planted(q, k, v, pq, pk, do, scale, causal, rows=None):
+        r = true_bwd(q, k, v, pq, pk, do, scale, causal)
+        if mistake == "dk_without_scale":
+            r["dk"] = r["dk"] / scale
+        elif mistake == "delta_dropped":
+            N = np.shape(q)[0]
+            s = scale * (np.asarray(q) @ np.asarray(k).T) + np.asarray(pq) @ np.asarray(pk).T
+            if causal:
+                s = np.where(np.arange(N)[None, :] <= np.arange(N)[:, None], s, -np.inf)
+            p = np.exp(s - s.max(axis=1, keepdims=True))
+            p /= p.sum(axis=1, keepdims=True)
+            ds = p * (np.asarray(do) @ np.asarray(v).T)  # the - rowsum(P dP) term left out
+            r["dq"] = scale * ds @ np.asarray(k)
+        elif mistake == "factor_grads_swapped":
+            r["dphi_q"], r["dphi_k"] = r["dphi_k"], r["dphi_q"]
+        else:
+            N = np.shape(q)[0]
+            s = scale * (np.asarray(q) @ np.asarray(k).T) + np.asarray(pq) @ np.asarray(pk).T
+            if causal:
+                s = np.where(np.arange(N)[None, :] <= np.arange(N)[:, None], s, -np.inf)
+            p = np.exp(s - s.max(axis=1, keepdims=True))
+            p /= p.sum(axis=1, keepdims=True)
+            r["dv"] = p @ np.asarray(do)
+        return r
+
+    monkeypatch.setattr(oracle, "attention_lowrank_bwd_head", planted)
+    with pytest.raises(AssertionError):
+        test_backward_matches_finite_differences(True)
