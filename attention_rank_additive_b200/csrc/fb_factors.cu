@@ -1,5 +1,7 @@
 // fb_factors.cu -- exact factor generators (Sandwich, ALiBi), the factor
-// preparation step that feeds the tensor-core kernel, and the wait self-test.
+// preparation step that feeds the tensor-core kernels, the multiplicative-bias
+// reweighting, the neural decomposition's linear layers and their gradients,
+// the small row and reduction steps of the backward, and the wait self-test.
 #include <atomic>
 #include <cmath>
 
