@@ -18,7 +18,7 @@ import os
 
 __all__ = [
     "FB_OK", "FB_ERR_INVALID_ARG", "FB_ERR_UNSUPPORTED", "FB_ERR_RANGE", "FB_ERR_WORKSPACE", "FB_ERR_CUDA",
-    "FB_ERR_TIMEOUT", "FB_F32", "FB_BF16", "FlashBiasError", "lib", "lib_path", "EXPORTED",
+    "FB_ERR_TIMEOUT", "FB_F32", "FB_BF16", "FB_F16", "FlashBiasError", "lib", "lib_path", "EXPORTED",
     "fb_status_str", "fb_version", "fb_attn_workspace_bytes", "fb_attn_fwd", "fb_attn_dense_bias_fwd",
     "fb_factors_sandwich", "fb_factors_alibi", "fb_svd_factors_host", "fb_check_device_error",
     "fb_selftest_wait_timeout", "fb_attn_fwd_noalloc", "fb_attn_prepare_factors", "fb_attn_fwd_prepared",
@@ -30,7 +30,7 @@ __all__ = [
 ]
 
 FB_OK, FB_ERR_INVALID_ARG, FB_ERR_UNSUPPORTED, FB_ERR_RANGE, FB_ERR_WORKSPACE, FB_ERR_CUDA, FB_ERR_TIMEOUT = range(7)
-FB_F32, FB_BF16 = 0, 1
+FB_F32, FB_BF16, FB_F16 = 0, 1, 2
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(_HERE, "libflashbias.so")

@@ -75,6 +75,16 @@ bool encode_qkv(CUtensorMap *m, const void *ptr, int BH, int N, int d, int DP) {
   return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, ptr, dims, strides, box, swizzle_for(ch * 2));
 }
 
+// O: bf16 [BH, N, d] with a box of (min(DP, 32), 32, 1), the epilogue's
+// per-warp TMA store (columns and rows past the tensor are not written).
+bool encode_o(CUtensorMap *m, void *ptr, int BH, int N, int d, int DP) {
+  const int e = DP < 32 ? DP : 32;
+  const uint64_t dims[3] = {uint64_t(d), uint64_t(N), uint64_t(BH)};
+  const uint64_t strides[2] = {uint64_t(d) * 2, uint64_t(N) * d * 2};
+  const uint32_t box[3] = {uint32_t(e), 32u, 1u};
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, ptr, dims, strides, box, swizzle_for(e * 2));
+}
+
 int *flags_for_current_device() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
@@ -88,7 +98,7 @@ int *flags_for_current_device() {
 }
 
 struct WsLayout {
-  size_t q_off, k_off, total;
+  size_t q_off, k_off, sched_off, total;
 };
 
 // Rank <= 4 factors go to the tensor cores as tf32 hi/lo parts: q' = [qh, qh, ql],
@@ -96,7 +106,7 @@ struct WsLayout {
 int tf32_cols(int R) { return R <= 2 ? 8 : 16; }
 
 WsLayout workspace_layout(int B, int H, int N, int R, int64_t bs, int64_t hs) {
-  WsLayout w{0, 0, 0};
+  WsLayout w{0, 0, 0, 0};
   if (R <= 0) return w;
   const size_t fb = size_t(bs == 0 ? 1 : B) * size_t(hs == 0 ? 1 : H);
   // rank <= 4: fp32 hi/lo split factors, 8 or 16 columns; else fp16 padded to 16..128
@@ -104,7 +114,10 @@ WsLayout workspace_layout(int B, int H, int N, int R, int64_t bs, int64_t hs) {
   const size_t per_al = (per + 255) & ~size_t(255);
   w.q_off = 0;
   w.k_off = per_al;
-  w.total = 2 * per_al;
+  // the fused kernel's work counter (two words; zeroed by the preparation
+  // step, reset by the kernel itself at the end of every launch)
+  w.sched_off = 2 * per_al;
+  w.total = 2 * per_al + 256;
   return w;
 }
 
@@ -116,6 +129,13 @@ bool valid_shape_bf16(int B, int H, int N, int d) {
 }
 
 bool valid_scale(float s) { return std::isfinite(s) && s > 0.f; }
+
+// FB_ERR_INVALID_ARG for an empty batch, head count or sequence, else
+// FB_ERR_UNSUPPORTED for a shape the tensor-core kernels do not take, else FB_OK.
+int shape_status_bf16(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1) return FB_ERR_INVALID_ARG;
+  return valid_shape_bf16(B, H, N, d) ? FB_OK : FB_ERR_UNSUPPORTED;
+}
 
 // Pick query tiles per CTA: two (the K/V tiles serve 256 rows) when there are
 // enough CTAs to fill the GPU at one CTA per SM and the ring keeps >= 2 stages.
@@ -155,6 +175,27 @@ int sm_count() {
 
 int *device_flags() { return flags_for_current_device(); }
 
+// Every argument check of fb_attn_fwd except the workspace, in its order.
+int fwd_arg_status(int dt, int B, int H, int N, int d, const void *Q, const void *K, const void *V, int R,
+                   const float *phi_q, const float *phi_k, int64_t phi_bstride, int64_t phi_hstride, float scale,
+                   const void *O, const float *LSE) {
+  if (!Q || !K || !V || !O || !LSE) return FB_ERR_INVALID_ARG;
+  if (R < 0 || R > 128) return FB_ERR_UNSUPPORTED;
+  if (R > 0 && (!phi_q || !phi_k || phi_bstride < 0 || phi_hstride < 0)) return FB_ERR_INVALID_ARG;
+  if (!valid_scale(scale)) return FB_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE)) return FB_ERR_INVALID_ARG;
+  if (R > 0 && (((reinterpret_cast<uintptr_t>(phi_q) | reinterpret_cast<uintptr_t>(phi_k)) & 3u) != 0))
+    return FB_ERR_INVALID_ARG;
+  if (dt == FB_F32) {
+    if (B < 1 || H < 1 || N < 1) return FB_ERR_INVALID_ARG;
+    if (d < 4 || d > 128 || d % 4 != 0 || (N + 31) / 32 > (1 << 30) || (long long)B * H > 65535)
+      return FB_ERR_UNSUPPORTED;
+    return FB_OK;
+  }
+  if (dt != FB_BF16) return FB_ERR_UNSUPPORTED;
+  return shape_status_bf16(B, H, N, d);
+}
+
 }  // namespace fb
 
 using namespace fb;
@@ -183,7 +224,8 @@ size_t fb_attn_workspace_bytes(int B, int H, int N, int R, int64_t phi_bstride, 
 
 int fb_attn_prepare_factors(int B, int H, int N, int R, const float *phi_q, const float *phi_k, int64_t phi_bstride,
                             int64_t phi_hstride, float scale, void *workspace, size_t workspace_bytes, void *stream) {
-  if (R < 0 || R > 128 || B < 1 || H < 1 || N < 1) return FB_ERR_UNSUPPORTED;
+  if (B < 1 || H < 1 || N < 1) return FB_ERR_INVALID_ARG;
+  if (R < 0 || R > 128) return FB_ERR_UNSUPPORTED;
   if (R == 0) return FB_OK;
   if (!phi_q || !phi_k || phi_bstride < 0 || phi_hstride < 0) return FB_ERR_INVALID_ARG;
   if (((reinterpret_cast<uintptr_t>(phi_q) | reinterpret_cast<uintptr_t>(phi_k)) & 3u) != 0) return FB_ERR_INVALID_ARG;
@@ -200,6 +242,7 @@ int fb_attn_prepare_factors(int B, int H, int N, int R, const float *phi_q, cons
   uint8_t *wsb = static_cast<uint8_t *>(workspace);
   const cudaError_t e = launch_prep_factors(mode, B, H, N, R, RP, phi_q, phi_k, phi_bstride, phi_hstride, fac_B,
                                             fac_H, scale, wsb + ws.q_off, wsb + ws.k_off, flags,
+                                            reinterpret_cast<unsigned int *>(wsb + ws.sched_off),
                                             static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FB_OK : FB_ERR_CUDA;
 }
@@ -214,7 +257,7 @@ int fb_attn_fwd_prepared(int dt, int B, int H, int N, int d, const void *Q, cons
   if (R > 0 && (phi_bstride < 0 || phi_hstride < 0)) return FB_ERR_INVALID_ARG;
   if (!valid_scale(scale)) return FB_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE)) return FB_ERR_INVALID_ARG;
-  if (!valid_shape_bf16(B, H, N, d)) return FB_ERR_UNSUPPORTED;
+  if (const int sh = shape_status_bf16(B, H, N, d)) return sh;
 
   const WsLayout ws = workspace_layout(B, H, N, R, phi_bstride, phi_hstride);
   if (ws.total > 0) {
@@ -235,7 +278,7 @@ int fb_attn_fwd_prepared(int dt, int B, int H, int N, int d, const void *Q, cons
   std::memset(&maps, 0, sizeof(maps));
   const int BH = B * H;
   if (!encode_qkv(&maps.q, Q, BH, N, d, DP) || !encode_qkv(&maps.k, K, BH, N, d, DP) ||
-      !encode_qkv(&maps.v, V, BH, N, d, DP))
+      !encode_qkv(&maps.v, V, BH, N, d, DP) || !encode_o(&maps.o, O, BH, N, d, DP))
     return FB_ERR_CUDA;
   const uint8_t *wsb = static_cast<const uint8_t *>(workspace);
   void *wq = ws.total ? const_cast<uint8_t *>(wsb) + ws.q_off : nullptr;
@@ -270,25 +313,21 @@ int fb_attn_fwd_prepared(int dt, int B, int H, int N, int d, const void *Q, cons
   a.fac_B = fac_B, a.fac_H = fac_H;
   a.bias_B = 1, a.bias_H = 1;
   a.flags = flags;
+  a.sched = ws.total ? reinterpret_cast<unsigned int *>(const_cast<uint8_t *>(wsb) + ws.sched_off) : nullptr;
   const cudaError_t e = sm100_launch(plan, maps, a, st);
   return e == cudaSuccess ? FB_OK : FB_ERR_CUDA;
 }
+
 
 int fb_attn_fwd(int dt, int B, int H, int N, int d, const void *Q, const void *K, const void *V, int R,
                 const float *phi_q, const float *phi_k, int64_t phi_bstride, int64_t phi_hstride, float scale,
                 int causal, void *O, float *LSE, void *workspace, size_t workspace_bytes, void *stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (!Q || !K || !V || !O || !LSE) return FB_ERR_INVALID_ARG;
-  if (R < 0 || R > 128) return FB_ERR_UNSUPPORTED;
-  if (R > 0 && (!phi_q || !phi_k || phi_bstride < 0 || phi_hstride < 0)) return FB_ERR_INVALID_ARG;
-  if (!valid_scale(scale)) return FB_ERR_INVALID_ARG;
-  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE)) return FB_ERR_INVALID_ARG;
-  if (R > 0 && (((reinterpret_cast<uintptr_t>(phi_q) | reinterpret_cast<uintptr_t>(phi_k)) & 3u) != 0))
-    return FB_ERR_INVALID_ARG;
+  if (const int a = fwd_arg_status(dt, B, H, N, d, Q, K, V, R, phi_q, phi_k, phi_bstride, phi_hstride, scale, O,
+                                   LSE))
+    return a;
 
   if (dt == FB_F32) {
-    if (B < 1 || H < 1 || N < 1 || d < 4 || d > 128 || d % 4 != 0 || (N + 31) / 32 > (1 << 30) || B * H > 65535)
-      return FB_ERR_UNSUPPORTED;
     int *flags = device_flags();
     if (!flags) return FB_ERR_CUDA;
     cudaError_t e = f32_launch(B, H, N, d, static_cast<const float *>(Q), static_cast<const float *>(K),
@@ -296,8 +335,6 @@ int fb_attn_fwd(int dt, int B, int H, int N, int d, const void *Q, const void *K
                                scale, causal, static_cast<float *>(O), LSE, st);
     return e == cudaSuccess ? FB_OK : FB_ERR_CUDA;
   }
-  if (dt != FB_BF16) return FB_ERR_UNSUPPORTED;
-  if (!valid_shape_bf16(B, H, N, d)) return FB_ERR_UNSUPPORTED;
   const WsLayout ws = workspace_layout(B, H, N, R, phi_bstride, phi_hstride);
   if (ws.total > 0) {
     if (!workspace || workspace_bytes < ws.total) return FB_ERR_WORKSPACE;
@@ -347,7 +384,7 @@ int fb_attn_mul_bias_fwd(int dt, int B, int H, int N, int d, const void *Q, cons
   if (!valid_scale(scale)) return FB_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE)) return FB_ERR_INVALID_ARG;
   if (((reinterpret_cast<uintptr_t>(phi_q) | reinterpret_cast<uintptr_t>(phi_k)) & 3u) != 0) return FB_ERR_INVALID_ARG;
-  if (!valid_shape_bf16(B, H, N, d)) return FB_ERR_UNSUPPORTED;
+  if (const int sh = shape_status_bf16(B, H, N, d)) return sh;
   const MulLayout m = mul_layout(B, H, N, d, R);
   if (!workspace || workspace_bytes < m.total || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return FB_ERR_WORKSPACE;
@@ -359,8 +396,9 @@ int fb_attn_mul_bias_fwd(int dt, int B, int H, int N, int d, const void *Q, cons
   const int RP = m.Rf > 0 ? pad_rank(m.Rf) : 0;
   void *fq = m.Rf > 0 ? ws + m.fac_off + fl.q_off : nullptr;
   void *fk = m.Rf > 0 ? ws + m.fac_off + fl.k_off : nullptr;
+  unsigned int *sched = m.Rf > 0 ? reinterpret_cast<unsigned int *>(ws + m.fac_off + fl.sched_off) : nullptr;
   if (launch_prep_mul_bias(B, H, N, d, R, RP, Q, K, phi_q, phi_k, phi_bstride, phi_hstride, ws + m.q1_off,
-                           ws + m.k1_off, fq, fk, flags, st) != cudaSuccess)
+                           ws + m.k1_off, fq, fk, flags, sched, st) != cudaSuccess)
     return FB_ERR_CUDA;
   return fb_attn_fwd_prepared(FB_BF16, B, H, N, d, ws + m.q1_off, ws + m.k1_off, V, m.Rf, bs, hs, scale, causal, O, LSE,
                               m.Rf > 0 ? ws + m.fac_off : nullptr, m.fac_bytes, stream);
@@ -400,7 +438,7 @@ int fb_attn_neural_fwd(int dt, int B, int H, int N, int d, const void *Q, const 
   if (((reinterpret_cast<uintptr_t>(X_q) | reinterpret_cast<uintptr_t>(X_k) | reinterpret_cast<uintptr_t>(W_q) |
         reinterpret_cast<uintptr_t>(W_k)) & 3u) != 0)
     return FB_ERR_INVALID_ARG;
-  if (!valid_shape_bf16(B, H, N, d)) return FB_ERR_UNSUPPORTED;
+  if (const int sh = shape_status_bf16(B, H, N, d)) return sh;
   const NeuralLayout m = neural_layout(B, H, N, R);
   if (!workspace || workspace_bytes < m.total || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return FB_ERR_WORKSPACE;
@@ -440,7 +478,7 @@ int fb_attn_neural_bwd(int dt, int B, int H, int N, int d, const void *Q, const 
         reinterpret_cast<uintptr_t>(W_k) | reinterpret_cast<uintptr_t>(dW_q) | reinterpret_cast<uintptr_t>(dW_k) |
         reinterpret_cast<uintptr_t>(dX_q) | reinterpret_cast<uintptr_t>(dX_k)) & 3u) != 0)
     return FB_ERR_INVALID_ARG;
-  if (!valid_shape_bf16(B, H, N, d)) return FB_ERR_UNSUPPORTED;
+  if (const int sh = shape_status_bf16(B, H, N, d)) return sh;
   const size_t need = fb_attn_neural_bwd_workspace_bytes(B, H, N, F, R);
   if (need == 0) return FB_ERR_UNSUPPORTED;
   if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
@@ -473,7 +511,8 @@ int fb_attn_dense_bias_fwd(int dt, int B, int H, int N, int d, const void *Q, co
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE) || !aligned16(Bias))
     return FB_ERR_INVALID_ARG;
   if (dt == FB_F32) {
-    if (B < 1 || H < 1 || N < 1 || d < 4 || d > 128 || d % 4 != 0 || B * H > 65535) return FB_ERR_UNSUPPORTED;
+    if (B < 1 || H < 1 || N < 1) return FB_ERR_INVALID_ARG;
+    if (d < 4 || d > 128 || d % 4 != 0 || (long long)B * H > 65535) return FB_ERR_UNSUPPORTED;
     if (!device_flags()) return FB_ERR_CUDA;
     cudaError_t e = f32_launch(B, H, N, d, static_cast<const float *>(Q), static_cast<const float *>(K),
                                static_cast<const float *>(V), 0, nullptr, nullptr, 0, 0,
@@ -482,7 +521,7 @@ int fb_attn_dense_bias_fwd(int dt, int B, int H, int N, int d, const void *Q, co
     return e == cudaSuccess ? FB_OK : FB_ERR_CUDA;
   }
   if (dt != FB_BF16) return FB_ERR_UNSUPPORTED;
-  if (!valid_shape_bf16(B, H, N, d)) return FB_ERR_UNSUPPORTED;
+  if (const int sh = shape_status_bf16(B, H, N, d)) return sh;
   if (N % 8 != 0 || bias_bstride % 8 != 0 || bias_hstride % 8 != 0) return FB_ERR_UNSUPPORTED;
   const int DP = pad_dim(d);
   // The dense path keeps a two-deep ring: one query tile per CTA when two do not leave room for it.
@@ -503,7 +542,7 @@ int fb_attn_dense_bias_fwd(int dt, int B, int H, int N, int d, const void *Q, co
   std::memset(&maps, 0, sizeof(maps));
   const int BH = B * H;
   if (!encode_qkv(&maps.q, Q, BH, N, d, DP) || !encode_qkv(&maps.k, K, BH, N, d, DP) ||
-      !encode_qkv(&maps.v, V, BH, N, d, DP))
+      !encode_qkv(&maps.v, V, BH, N, d, DP) || !encode_o(&maps.o, O, BH, N, d, DP))
     return FB_ERR_CUDA;
   const int bias_B = bias_bstride == 0 ? 1 : B, bias_H = bias_hstride == 0 ? 1 : H;
   {
@@ -616,7 +655,7 @@ int fb_attn_bwd(int dt, int B, int H, int N, int d, const void *Q, const void *K
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) || !aligned16(dQ) ||
       !aligned16(dK) || !aligned16(dV) || !aligned16(LSE))
     return FB_ERR_INVALID_ARG;
-  if (!valid_shape_bf16(B, H, N, d)) return FB_ERR_UNSUPPORTED;
+  if (const int sh = shape_status_bf16(B, H, N, d)) return sh;
   const BwdLayout L = bwd_layout(B, H, N, R, phi_bstride, phi_hstride);
   if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return FB_ERR_WORKSPACE;

@@ -93,13 +93,24 @@ struct Sm100Cfg {
                                     ? int((kSmemLimit - FIXED - CTRL - ALIGN_SLACK) / STAGE)
                                     : 0;
   static constexpr int KS = KS_FIT > 3 ? 3 : KS_FIT;
-  static constexpr uint32_t SMEM = FIXED + uint32_t(KS) * STAGE + CTRL + ALIGN_SLACK;
   // QT softmax warpgroups + one warpgroup holding the producer warp, the MMA
   // warp and two idle warps. Registers are moved from that warpgroup to the
   // softmax warpgroups with setmaxnreg: the launch allocation is
   // THREADS * LAUNCH_REGS and the shares below add up to exactly that.
   static constexpr int THREADS = NSWG * 128 + 128;
   static constexpr bool SMALL = QT == 1 && !KSPLIT;  // two CTAs per SM
+  // Epilogue: O leaves through shared memory and TMA stores, EPI_E columns of
+  // a warp's 32 rows at a time (one staging slot per softmax warp), when the
+  // slots fit beside the rings (for a two-per-SM plan: within half an SM);
+  // otherwise each thread stores its own row.
+  static constexpr int EPI_E = DP < 32 ? DP : 32;
+  static constexpr uint32_t STG_WARP = 32u * uint32_t(EPI_E) * 2u;
+  static constexpr uint32_t STG = uint32_t(NSWG) * 4u * STG_WARP;
+  static constexpr uint32_t SMEM_BASE = FIXED + uint32_t(KS) * STAGE + CTRL + ALIGN_SLACK;
+  static constexpr uint32_t kPairLimit = 228u * 1024u / 2u - 1024u;
+  static constexpr bool TMA_EPI = (SMALL && SMEM_BASE <= kPairLimit) ? (SMEM_BASE + STG <= kPairLimit)
+                                                                      : (SMEM_BASE + STG <= kSmemLimit);
+  static constexpr uint32_t SMEM = SMEM_BASE + (TMA_EPI ? STG : 0u);
   static constexpr int MIN_BLOCKS = SMALL ? 2 : 1;
   static constexpr int LAUNCH_REGS = SMALL ? 128 : 168;
   static constexpr int REG_SOFTMAX = SMALL ? 192 : 216;
@@ -122,6 +133,8 @@ struct Sm100Cfg {
   // MMA issuer warps (one per query tile or key half with separate P, else
   // one), each of which releases every K/V stage once per key step.
   static constexpr int RELEASERS = SEP_P ? NSWG : 1;
+  // Warps that read the work-item ring: the MMA issuers and the softmax warps.
+  static constexpr int ITEM_READERS = RELEASERS + 4 * NSWG;
   static constexpr uint32_t IDESC_QK = make_idesc_f16(true, true, 128, 128, false);
   static constexpr uint32_t IDESC_F =
       MODE == kBiasTf32 ? make_idesc_tf32(128, 128) : make_idesc_f16(false, false, 128, 128, false);
@@ -138,6 +151,8 @@ struct SmemCtrl {
   uint64_t s_full[2], p_full[2];
   uint64_t aux_full[2][3], aux_empty[2][3];
   uint64_t pair[4];  // key split: the two halves of a 32-row quarter exchange (m, l)
+  uint64_t item_full[4], item_empty[4];  // the work-item ring (producer -> every other role)
+  int item[4];
   uint32_t tmem_base;
   int abort;
 };
@@ -183,6 +198,33 @@ __device__ __forceinline__ float row_max(const uint32_t *x) {
     for (int e = 0; e < 8; ++e) mp[e] = fmaxf(mp[e], __uint_as_float(x[NC - 8 + e]));
   }
   return fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
+}
+
+// One chunk of the epilogue: a warp's 32 rows x E bf16 columns (thread =
+// row; pk holds its E/2 packed pairs) go into the warp's staging slot, laid
+// out in the TMA swizzle of an E*2-byte row (64 B: 16-byte chunk j of row r
+// at j ^ ((r >> 1) & 3); 32 B: at j ^ ((r >> 2) & 1)), so that the
+// row-per-thread writes are free of bank conflicts; lane 0 then issues one
+// tiled store of the slot at (col, row0, bh). The slot is rewritten only
+// after its previous store has read it.
+template <int E>
+__device__ __forceinline__ void stage_and_store_o(uint8_t *slot, const uint32_t *pk, int lane, const CUtensorMap *map,
+                                                  int col, int row0, int bh) {
+  static_assert(E == 16 || E == 32, "staging chunk");
+  if (lane == 0) bulk_wait_group_read0();
+  __syncwarp();
+#pragma unroll
+  for (int j = 0; j < E / 8; ++j) {
+    const int pj = E == 32 ? (j ^ ((lane >> 1) & 3)) : (j ^ ((lane >> 2) & 1));
+    *reinterpret_cast<uint4 *>(slot + lane * (E * 2) + pj * 16) =
+        make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_3d(map, slot, col, row0, bh);
+    bulk_commit_group();
+  }
 }
 
 // One schedulable work item: a group of QT query tiles of one (b, h) head.
@@ -231,12 +273,51 @@ __device__ __forceinline__ int item_of_pass(int p, int n_items) {
   return k < n_items ? k : -1;
 }
 
+// The p-th work item of this CTA. With a work counter (sched), CTA c starts
+// with item c (items are numbered heaviest first and the grid is never larger
+// than the item count) and then takes the items after the first gridDim.x in
+// order, each when it gets to it, so that the CTAs finish together whatever
+// their item mix and speed; without a counter, the fixed passes above. Items
+// are claimed by the producer's lane 0 only.
+__device__ __forceinline__ int claim_item(int p, int n_items, unsigned int *sched) {
+  if (sched == nullptr) return item_of_pass(p, n_items);
+  if (p == 0) return int(blockIdx.x);
+  const unsigned int k = gridDim.x + atomicAdd(sched, 1u);
+  return k < unsigned(n_items) ? int(k) : -1;
+}
+
+// After its last claim, each CTA counts itself out on sched[1]; the last one
+// resets both words, so the counter starts at zero for the next launch in
+// stream order (the factor preparation zeroes it before the first).
+__device__ __forceinline__ void release_sched(unsigned int *sched) {
+  if (sched == nullptr) return;
+  __threadfence();
+  if (atomicAdd(sched + 1, 1u) == gridDim.x - 1) {
+    sched[0] = 0u;
+    sched[1] = 0u;
+    __threadfence();
+  }
+}
+
+// Work-item ring: the producer publishes the item of pass p (or -1: no more)
+// in slot p % 4; every reading warp waits for it, reads it and frees the slot.
+__device__ __forceinline__ int read_item(uint64_t *full, uint64_t *empty, const int *items, int p,
+                                         volatile int *abort, bool &ok) {
+  const int slot = p & 3;
+  ok = mbar_wait(&full[slot], uint32_t(p >> 2) & 1u, abort);
+  if (!ok) return -1;
+  const int k = *reinterpret_cast<const volatile int *>(&items[slot]);
+  __syncwarp();
+  if ((threadIdx.x & 31u) == 0) mbar_arrive(&empty[slot]);
+  return k;
+}
+
 template <int DP, int RP, int MODE, int QT>
 __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<DP, RP, MODE, QT>::MIN_BLOCKS)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_fq,
                    const __grid_constant__ CUtensorMap tm_fk, const __grid_constant__ CUtensorMap tm_bias,
-                   const FwdArgs args) {
+                   const __grid_constant__ CUtensorMap tm_o, const FwdArgs args) {
   using C = Sm100Cfg<DP, RP, MODE, QT>;
   constexpr int KS = C::KS;
   static_assert(KS >= 1, "configuration does not fit in shared memory");
@@ -249,7 +330,15 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
   uint8_t *sFK = sK + KS * C::KV_TILE;   // KS x FK_TILE
   uint8_t *sV = sFK + KS * C::FK_TILE;   // KS x KV_TILE
   uint8_t *sAux = sV + KS * C::KV_TILE;  // QT x KS x AUX_TILE
-  SmemCtrl *ctrl = reinterpret_cast<SmemCtrl *>(sAux + QT * KS * C::AUX_TILE);
+  constexpr uint32_t STG_OFF = QT * (C::Q_TILE + C::FQ_TILE) + KS * (2 * C::KV_TILE + C::FK_TILE + QT * C::AUX_TILE);
+  uint8_t *sStg = smem + STG_OFF;  // NSWG x 4 x STG_WARP (TMA_EPI), 1024-aligned
+  SmemCtrl *ctrl = reinterpret_cast<SmemCtrl *>(sStg + (C::TMA_EPI ? C::STG : 0u));
+  // The epilogue's staging slot of softmax warp wi, recomputed from the
+  // shared-memory base where it is needed rather than kept live in a register.
+  auto stg_slot = [&](int wi) {
+    const uintptr_t base = (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023);
+    return reinterpret_cast<uint8_t *>(base) + STG_OFF + uint32_t(wi) * C::STG_WARP;
+  };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -287,6 +376,10 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
       }
       for (int q = 0; q < 4; ++q) mbar_init(&ctrl->pair[q], 64);
     }
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(&ctrl->item_full[q], 1);
+      mbar_init(&ctrl->item_empty[q], C::ITEM_READERS);
+    }
     ctrl->abort = 0;
     fence_mbar_init();
   }
@@ -323,11 +416,16 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
     }
     bool ok = true;
     int g = 0, it = 0, la[2] = {0, 0};
-    for (int p = 0; ok; ++p) {
-      if (p * int(gridDim.x) >= n_items) break;
-      const int k = item_of_pass(p, n_items);
-      if (k < 0) continue;
-      const WorkItem w = make_item<QT>(k, args);
+    // The item of pass 0 is claimed and published before the loop; each pass
+    // p claims and publishes the item of pass p + 1 once its own loads are
+    // issued, the last published item being -1.
+    int cur = __shfl_sync(0xffffffffu, leader ? claim_item(0, n_items, args.sched) : 0, 0);
+    if (leader) {
+      ctrl->item[0] = cur;
+      mbar_arrive(&ctrl->item_full[0]);
+    }
+    for (int p = 0; ok && cur >= 0; ++p) {
+      const WorkItem w = make_item<QT>(cur, args);
       // Q and phi_q of the item, once the previous item's last S MMAs are done.
       if (it > 0 && !(ok = mbar_wait(&ctrl->q_empty, uint32_t(it - 1) & 1u, abort))) break;
       uint32_t qbytes = 0;
@@ -379,8 +477,33 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
           tma_load_3d_leader(sV + s * C::KV_TILE + ch * (128 * C::DCH * 2), &tm_v, &ctrl->v_full[s], ch * C::DCH,
                              kv, w.bh, leader);
       }
+      if (!ok) break;
+      // All of this item's loads are issued: claim and publish the item of
+      // pass p + 1 now, close to when the CTA will get to it. Slot (p + 1) % 4
+      // last held pass p - 3, which every reader has freed by now (the
+      // issuers are past the last S of pass p - 1).
+      const int q1 = p + 1;
+      if (q1 >= 4 && !(ok = mbar_wait(&ctrl->item_empty[q1 & 3], uint32_t((q1 >> 2) - 1) & 1u, abort))) break;
+      const int nxt = __shfl_sync(0xffffffffu, leader ? claim_item(q1, n_items, args.sched) : 0, 0);
+      if (leader) {
+        ctrl->item[q1 & 3] = nxt;
+        mbar_arrive(&ctrl->item_full[q1 & 3]);
+        // its Q and phi_q tiles go to L2 now, so their load at the item
+        // change waits for L2, not HBM
+        if (nxt >= 0) {
+          const WorkItem w2 = make_item<QT>(nxt, args);
+          for (int t = 0; t < QT; ++t) {
+            if (w2.nk[t] == 0) continue;
+            for (int ch = 0; ch < C::NDCH; ++ch) tma_prefetch_l2_3d(&tm_q, ch * C::DCH, w2.q0[t], w2.bh);
+            if (C::FAC_MMA)
+              for (int ch = 0; ch < C::NRCH; ++ch) tma_prefetch_l2_3d(&tm_fq, ch * C::RCH, w2.q0[t], w2.fb_slice);
+          }
+        }
+      }
       ++it;
+      cur = nxt;
     }
+    if (leader) release_sched(args.sched);  // this CTA claims nothing more
     if (!ok) {
       // Aborted: let the copies already issued land before the CTA exits.
       for (int s = 0; s < KS; ++s) {
@@ -457,9 +580,8 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
       const int hh = warp - C::MMA_WARP;
       int L = 0;
       for (int p = 0; ok; ++p) {
-        if (p * int(gridDim.x) >= n_items) break;
-        const int k = item_of_pass(p, n_items);
-        if (k < 0) continue;
+        const int k = read_item(ctrl->item_full, ctrl->item_empty, ctrl->item, p, abort, ok);
+        if (k < 0) break;
         const WorkItem w = make_item<QT>(k, args);
         const int n = w.n_steps;
         if (hh == 0) {
@@ -525,18 +647,13 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
       const int t = warp - C::MMA_WARP;
       int L = 0;
       for (int p = 0; ok; ++p) {
-        if (p * int(gridDim.x) >= n_items) break;
-        const int k = item_of_pass(p, n_items);
-        if (k < 0) continue;
+        const int k = read_item(ctrl->item_full, ctrl->item_empty, ctrl->item, p, abort, ok);
+        if (k < 0) break;
         const WorkItem w = make_item<QT>(k, args);
         const int nk_t = pick(w.nk, t), first_t = pick(w.first, t);
         if (!(ok = mbar_wait(&ctrl->q_full, uint32_t(it) & 1u, abort))) break;
         tc_fence_after();
-        bool q_released = false;
-        if (nk_t == 0) {
-          tc_commit_elect(&ctrl->q_empty);
-          q_released = true;
-        }
+        if (nk_t == 0) tc_commit_elect(&ctrl->q_empty);  // this tile reads no Q in this item
         for (int i = 0; i < w.n_steps && ok; ++i) {
           const int gi = g + i;
           const int s = gi % KS;
@@ -567,10 +684,7 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
             tc_commit_elect(&ctrl->s_full[t]);
             tc_commit_elect(&ctrl->k_empty[s1]);
           }
-          if (i + 1 == w.n_steps && !q_released) {
-            tc_commit_elect(&ctrl->q_empty);  // last S of this item issued
-            q_released = true;
-          }
+          if (i + 1 == w.n_steps && nk_t > 0) tc_commit_elect(&ctrl->q_empty);  // last S of this item issued
           if (!(ok = mbar_wait(&ctrl->v_full[s], ph, abort))) break;
           if (!(ok = mbar_wait(&ctrl->p_full[t], uint32_t(L) & 1u, abort))) break;
           // the first PV of an item overwrites O_t: its epilogue must have read it
@@ -597,9 +711,8 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
       // of one thread run in order).
       int L[2] = {0, 0};
       for (int p = 0; ok; ++p) {
-        if (p * int(gridDim.x) >= n_items) break;
-        const int k = item_of_pass(p, n_items);
-        if (k < 0) continue;
+        const int k = read_item(ctrl->item_full, ctrl->item_empty, ctrl->item, p, abort, ok);
+        if (k < 0) break;
         const WorkItem w = make_item<QT>(k, args);
         auto act = [&](int t, int i) { return t < QT && i >= w.first[t] && i < w.n_steps; };
         if (!(ok = mbar_wait(&ctrl->q_full, uint32_t(it) & 1u, abort))) break;
@@ -698,9 +811,8 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
       bool ok = true;
       int L = 0, it = 0;
       for (int p = 0; ok; ++p) {
-        if (p * int(gridDim.x) >= n_items) break;
-        const int k = item_of_pass(p, n_items);
-        if (k < 0) continue;
+        const int k = read_item(ctrl->item_full, ctrl->item_empty, ctrl->item, p, abort, ok);
+        if (k < 0) break;
         const WorkItem w = make_item<QT>(k, args);
         const int q0 = w.q0[0], n = w.n_steps;
         const int row = q0 + r_loc;
@@ -826,6 +938,37 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
         const float l_tot = w0 * l0 + w1 * l1;
         const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
         const float c0s = w0 * inv_l, c1s = w1 * inv_l;
+        if constexpr (C::TMA_EPI) {
+          // this half stores O columns 64h .. 64h+63 of the warp's rows in two
+          // staged chunks; both O accumulators are handed back after the last read
+          const bool rows_live = q0 + 32 * wq < N;  // warp-uniform
+          uint8_t *slot = stg_slot(warp);
+#pragma unroll
+          for (int cc = 0; cc < 64; cc += 32) {
+            const int col0 = 64 * h + cc;
+            uint32_t r0[32], r1[32];
+            tmem_ld32(o0_tm + col0, r0);
+            tmem_ld32(o1_tm + col0, r1);
+            tmem_ld_wait32(r0);
+            tmem_ld_wait32(r1);
+            if (cc == 32) {
+              tc_fence_before();
+              mbar_arrive(&ctrl->o_free[0]);  // both O accumulators have been read
+            }
+            if (rows_live && col0 < args.d) {  // chunks past the head dim hold padding only
+              uint32_t pkd[16];
+#pragma unroll
+              for (int e = 0; e < 16; ++e)
+                pkd[e] = pack_bf16x2(fmaf(__uint_as_float(r0[2 * e]), c0s, __uint_as_float(r1[2 * e]) * c1s),
+                                     fmaf(__uint_as_float(r0[2 * e + 1]), c0s, __uint_as_float(r1[2 * e + 1]) * c1s));
+              stage_and_store_o<32>(slot, pkd, lane, &tm_o, col0, q0 + 32 * wq, w.bh);
+            }
+          }
+          if (h == 0 && row < N)
+            args.LSE[size_t(w.bh) * N + row] = l_tot > 0.f ? (M + __log2f(l_tot)) * kLn2 : -INFINITY;
+          ++it;
+          continue;
+        }
         __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(args.O) + (size_t(w.bh) * N + row) * args.d;
 #pragma unroll
         for (int cc = 0; cc < 64; cc += 16) {  // this half writes O columns 64h .. 64h+63
@@ -874,9 +1017,8 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
       bool ok = true;
       int L = 0, it = 0;
       for (int p = 0; ok; ++p) {
-        if (p * int(gridDim.x) >= n_items) break;
-        const int k = item_of_pass(p, n_items);
-        if (k < 0) continue;
+        const int k = read_item(ctrl->item_full, ctrl->item_empty, ctrl->item, p, abort, ok);
+        if (k < 0) break;
         const WorkItem w = make_item<QT>(k, args);
         const int q0_t = pick(w.q0, t), nk_t = pick(w.nk, t), first_t = pick(w.first, t);
         const int row = q0_t + r_loc;
@@ -1022,6 +1164,48 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
         // ---------------------------------------------------------- epilogue
         if (!(ok = mbar_wait(&ctrl->o_final[t], uint32_t(it) & 1u, abort))) break;
         tc_fence_after();
+        if constexpr (C::TMA_EPI) {
+          // O leaves in chunks of EPI_E columns through this warp's staging
+          // slot; O_t is handed back to the MMA warp as soon as its last chunk
+          // is in registers, and the TMA stores complete on their own.
+          if (nk_t > 0) {
+            const uint32_t tid = tid_x_fresh();
+            const int e_lane = int(tid & 31u), e_warp = int(tid >> 5);
+            const int row0 = q0_t + 32 * (e_warp & 3);  // first row of this warp's TMEM lane quarter
+            const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
+            const bool rows_live = row0 < N;  // warp-uniform
+            uint8_t *slot = stg_slot(e_warp);
+#pragma unroll
+            for (int c0 = 0; c0 < DP; c0 += C::EPI_E) {
+              uint32_t r[C::EPI_E];
+              if constexpr (C::EPI_E == 32) {
+                tmem_ld32(o_tm + c0, r);
+                tmem_ld_wait32(r);
+              } else {
+                tmem_ld16(o_tm + c0, r);
+                tmem_ld_wait16(r);
+              }
+              if (c0 + C::EPI_E == DP) {
+                tc_fence_before();
+                mbar_arrive(&ctrl->o_free[t]);  // O_t has been read
+              }
+              if (rows_live && c0 < args.d) {  // chunks past the head dim hold padding only
+                uint32_t pkd[C::EPI_E / 2];
+#pragma unroll
+                for (int e = 0; e < C::EPI_E / 2; ++e)
+                  pkd[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l, __uint_as_float(r[2 * e + 1]) * inv_l);
+                stage_and_store_o<C::EPI_E>(slot, pkd, e_lane, &tm_o, c0, row0, w.bh);
+              }
+            }
+            if (row0 + e_lane < N)
+              args.LSE[size_t(w.bh) * N + row0 + e_lane] = l_sum > 0.f ? (m_use + __log2f(l_sum)) * kLn2 : -INFINITY;
+          } else {
+            tc_fence_before();
+            mbar_arrive(&ctrl->o_free[t]);
+          }
+          ++it;
+          continue;
+        }
         if (nk_t > 0) {
           const float inv_l = l_sum > 0.f ? 1.f / l_sum : 0.f;
           __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(args.O) + (size_t(w.bh) * N + row) * args.d;
@@ -1056,6 +1240,10 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
     }
   }
 
+  if constexpr (C::TMA_EPI) {
+    // the staging slots must outlive the stores that read them
+    if (warp < C::PRODUCER_WARP && lane == 0) bulk_wait_group0();
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == C::MMA_WARP) {
@@ -1115,7 +1303,7 @@ static cudaError_t launch_one(const FwdMaps &m, const FwdArgs &a, cudaStream_t s
     // walking its share of the work items.
     const long long items = (long long)a.n_cta_q * a.B * a.H;
     const long long ctas = std::min<long long>(items, cap);
-    kern<<<dim3(unsigned(ctas)), C::THREADS, C::SMEM, stream>>>(m.q, m.k, m.v, m.fq, m.fk, m.bias, a);
+    kern<<<dim3(unsigned(ctas)), C::THREADS, C::SMEM, stream>>>(m.q, m.k, m.v, m.fq, m.fk, m.bias, m.o, a);
     return cudaGetLastError();
   }
 }

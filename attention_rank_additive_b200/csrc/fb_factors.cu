@@ -55,7 +55,9 @@ __global__ void alibi_kernel(int H, int N, float *__restrict__ phi_q, float *__r
 // Values beyond the fp16 range are saturated and raise kFlagRange.
 __global__ void prep_mma_kernel(int N, int R, int RP, int fac_H, const float *__restrict__ pq,
                                 const float *__restrict__ pk, long long bs, long long hs, float inv_scale,
-                                __half *__restrict__ oq, __half *__restrict__ ok, int *flags, long long total) {
+                                __half *__restrict__ oq, __half *__restrict__ ok, int *flags, long long total,
+                                unsigned int *sched) {
+  if (sched != nullptr && blockIdx.x == 0 && threadIdx.x == 0) sched[0] = sched[1] = 0u;  // the work counter
   bool overflow = false;
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
        idx += (long long)gridDim.x * blockDim.x) {
@@ -91,7 +93,9 @@ __device__ __forceinline__ float tf32_hi(float x) { return __uint_as_float(__flo
 
 __global__ void prep_tf32_kernel(int N, int R, int KT, int fac_H, const float *__restrict__ pq,
                                  const float *__restrict__ pk, long long bs, long long hs, float inv_scale,
-                                 float *__restrict__ oq, float *__restrict__ ok, long long total) {
+                                 float *__restrict__ oq, float *__restrict__ ok, long long total,
+                                 unsigned int *sched) {
+  if (sched != nullptr && blockIdx.x == 0 && threadIdx.x == 0) sched[0] = sched[1] = 0u;  // the work counter
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
        idx += (long long)gridDim.x * blockDim.x) {
     const long long n = idx % N;
@@ -136,7 +140,8 @@ __global__ void prep_mul_bias_kernel(int H, int N, int d, int R, int RP, const _
                                      const float *__restrict__ pk, long long bs, long long hs,
                                      __nv_bfloat16 *__restrict__ q1, __nv_bfloat16 *__restrict__ k1,
                                      __half *__restrict__ fq, __half *__restrict__ fk, int *flags, int width,
-                                     long long total) {
+                                     long long total, unsigned int *sched) {
+  if (sched != nullptr && blockIdx.x == 0 && threadIdx.x == 0) sched[0] = sched[1] = 0u;  // the work counter
   bool overflow = false;
   const int used = d * (R - 1);
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
@@ -257,13 +262,13 @@ static int grid_for(long long total, int block);
 
 cudaError_t launch_prep_mul_bias(int B, int H, int N, int d, int R, int RP, const void *Q, const void *K,
                                  const float *phi_q, const float *phi_k, int64_t bs, int64_t hs, void *q1, void *k1,
-                                 void *fq, void *fk, int *flags, cudaStream_t s) {
+                                 void *fq, void *fk, int *flags, unsigned int *sched, cudaStream_t s) {
   const int width = (d > RP - d * (R - 1) ? d : RP - d * (R - 1)) / 8;  // groups of 8 columns
   const long long total = (long long)B * H * N * width;
   prep_mul_bias_kernel<<<grid_for(total, 256), 256, 0, s>>>(
       H, N, d, R, RP, static_cast<const __nv_bfloat16 *>(Q), static_cast<const __nv_bfloat16 *>(K), phi_q, phi_k,
       bs, hs, static_cast<__nv_bfloat16 *>(q1), static_cast<__nv_bfloat16 *>(k1), static_cast<__half *>(fq),
-      static_cast<__half *>(fk), flags, width, total);
+      static_cast<__half *>(fk), flags, width, total, sched);
   return cudaGetLastError();
 }
 
@@ -304,19 +309,19 @@ cudaError_t launch_alibi(int H, int N, float *phi_q, float *phi_k, cudaStream_t 
 
 cudaError_t launch_prep_factors(int mode, int B, int H, int N, int R, int RP, const float *phi_q, const float *phi_k,
                                 int64_t bs, int64_t hs, int fac_B, int fac_H, float scale, void *out_q, void *out_k,
-                                int *flags, cudaStream_t s) {
+                                int *flags, unsigned int *sched, cudaStream_t s) {
   (void)B;
   (void)H;
   if (mode == kBiasMma) {
     const long long total = (long long)fac_B * fac_H * N * RP;
     prep_mma_kernel<<<grid_for(total, 256), 256, 0, s>>>(N, R, RP, fac_H, phi_q, phi_k, bs, hs, 1.0f / scale,
                                                          static_cast<__half *>(out_q), static_cast<__half *>(out_k),
-                                                         flags, total);
+                                                         flags, total, sched);
   } else {
     const long long total = (long long)fac_B * fac_H * N;
     prep_tf32_kernel<<<grid_for(total, 256), 256, 0, s>>>(N, R, RP, fac_H, phi_q, phi_k, bs, hs, 1.0f / scale,
                                                           static_cast<float *>(out_q), static_cast<float *>(out_k),
-                                                          total);
+                                                          total, sched);
   }
   return cudaGetLastError();
 }

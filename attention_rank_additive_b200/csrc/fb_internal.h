@@ -34,6 +34,7 @@ struct FwdArgs {
   int fac_B, fac_H;       // factor slices: B or 1, H or 1 (1 = broadcast)
   int bias_B, bias_H;     // dense bias slices, same convention
   int *flags;             // device flag word
+  unsigned int *sched;    // work counter [2] (zero at launch), or null: a fixed item order
 };
 
 // Launch description chosen by the host for one call.
@@ -48,6 +49,7 @@ struct FwdMaps {
   CUtensorMap q, k, v;  // bf16 [BH, N, d] with box (min(DP,64), 128, 1)
   CUtensorMap fq, fk;   // factors: fp16 [FB, N, RP] (mma) or fp32 [FB, N, RP] (tf32)
   CUtensorMap bias;     // dense bias bf16 [B', H', N, N] with box (64, 128, 1, 1)
+  CUtensorMap o;        // O bf16 [BH, N, d] with box (min(DP,32), 32, 1): the epilogue's TMA stores
 };
 
 // Shared-memory bytes the kernel needs for a plan, or 0 if it does not fit.
@@ -65,9 +67,10 @@ cudaError_t f32_launch(int B, int H, int N, int d, const float *Q, const float *
 cudaError_t launch_sandwich(int N, int C, float *phi_q, float *phi_k, cudaStream_t s);
 cudaError_t launch_alibi(int H, int N, float *phi_q, float *phi_k, cudaStream_t s);
 // kBiasMma: fp16 [FB, N, RP], phi_q / scale. kBiasTf32: fp32 [FB, N, RP] hi/lo split, phi_q / scale.
+// Also zeroes the fused kernel's work counter sched[2] when sched is not null.
 cudaError_t launch_prep_factors(int mode, int B, int H, int N, int R, int RP, const float *phi_q, const float *phi_k,
                                 int64_t bs, int64_t hs, int fac_B, int fac_H, float scale, void *out_q, void *out_k,
-                                int *flags, cudaStream_t s);
+                                int *flags, unsigned int *sched, cudaStream_t s);
 cudaError_t launch_wait_selftest(int limit_ms, int *flags, cudaStream_t s);
 // Multiplicative bias: q1 = q phi_q,0 and k1 = k phi_k,0 (bf16 [BH, N, d]);
 // fp16 factor rows [BH, N, RP] with the terms r >= 1.
@@ -81,7 +84,7 @@ cudaError_t launch_neural_grads(int B, int H, int N, int F, int R, const float *
                                 float *dWk, float *dXq, float *dXk, cudaStream_t s);
 cudaError_t launch_prep_mul_bias(int B, int H, int N, int d, int R, int RP, const void *Q, const void *K,
                                  const float *phi_q, const float *phi_k, int64_t bs, int64_t hs, void *q1, void *k1,
-                                 void *fq, void *fk, int *flags, cudaStream_t s);
+                                 void *fq, void *fk, int *flags, unsigned int *sched, cudaStream_t s);
 
 // Backward (gradients of O for dO).
 struct BwdArgs {
@@ -136,5 +139,11 @@ cudaError_t launch_reduce_factor_grads(int B, int H, int N, int R, int fac_B, in
 
 // Per-device flag word (allocated once per device as a module global).
 int *device_flags();
+
+// fb_attn_fwd's argument checks other than the workspace (FB_OK or the status
+// fb_attn_fwd returns), for entry points that must report the same errors.
+int fwd_arg_status(int dt, int B, int H, int N, int d, const void *Q, const void *K, const void *V, int R,
+                   const float *phi_q, const float *phi_k, int64_t phi_bstride, int64_t phi_hstride, float scale,
+                   const void *O, const float *LSE);
 
 }  // namespace fb

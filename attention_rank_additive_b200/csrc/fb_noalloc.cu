@@ -53,9 +53,14 @@ void *scratch_for_current_device() {
 extern "C" int fb_attn_fwd_noalloc(int dt, int B, int H, int N, int d, const void *Q, const void *K, const void *V,
                                    int R, const float *phi_q, const float *phi_k, int64_t phi_bstride,
                                    int64_t phi_hstride, float scale, int causal, void *O, float *LSE, void *stream) {
+  // fb_attn_fwd's own argument checks come first, so that both entry points
+  // report the same status for the same bad argument; the size limit of the
+  // fixed array is checked after them.
+  if (const int a = fb::fwd_arg_status(dt, B, H, N, d, Q, K, V, R, phi_q, phi_k, phi_bstride, phi_hstride, scale, O,
+                                       LSE))
+    return a;
   size_t need = 0;
   if (dt == FB_BF16) {
-    if (B < 1 || H < 1 || N < 1 || R < 0 || R > 128) return FB_ERR_UNSUPPORTED;
     need = fb_attn_workspace_bytes(B, H, N, R, phi_bstride, phi_hstride);
     if (need > fb::kNoAllocScratchBytes) return FB_ERR_WORKSPACE;  // beyond the fixed scratch
   }

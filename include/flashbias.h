@@ -26,8 +26,11 @@
  *  - Kernel-side conditions (a pipeline wait that ran out, a factor that
  *    overflowed fp16) set a library-wide device flag that
  *    fb_check_device_error() reads back; the kernels never trap.
+ *  - Entry points declared to return int return an fb_status value.
  *  - No C++ exception crosses this interface. Entry points may be called
- *    from several host threads.
+ *    from several host threads, except that fb_attn_fwd_noalloc calls that
+ *    can overlap on one device must be serialised by the caller (they share
+ *    one scratch array; see there).
  */
 #ifndef FLASHBIAS_H_
 #define FLASHBIAS_H_
@@ -41,15 +44,19 @@ extern "C" {
 
 typedef enum {
   FB_OK = 0,
-  FB_ERR_INVALID_ARG = 1, /* null pointer, bad shape, bad stride, bad scale   */
-  FB_ERR_UNSUPPORTED = 2, /* valid but outside what the library implements   */
+  FB_ERR_INVALID_ARG = 1, /* null or misaligned pointer, empty shape (a size
+                             below 1), bad stride, bad scale                 */
+  FB_ERR_UNSUPPORTED = 2, /* valid but outside what the library implements
+                             (a head dim, rank, dtype or size it does not take) */
   FB_ERR_RANGE = 3,       /* a factor value does not fit the kernel's type    */
   FB_ERR_WORKSPACE = 4,   /* workspace missing, too small or misaligned       */
   FB_ERR_CUDA = 5,        /* CUDA runtime/driver call or launch failed        */
   FB_ERR_TIMEOUT = 6      /* a kernel's bounded pipeline wait ran out         */
 } fb_status;
 
-typedef enum { FB_F32 = 0, FB_BF16 = 1 } fb_dtype;
+/* Element type of Q, K, V, O (and of a dense bias). fp16 inputs are not
+ * implemented: every entry point returns FB_ERR_UNSUPPORTED for FB_F16. */
+typedef enum { FB_F32 = 0, FB_BF16 = 1, FB_F16 = 2 } fb_dtype;
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *fb_status_str(int status);
@@ -60,8 +67,12 @@ int fb_version(void);
 /*
  * Workspace for fb_attn_fwd with the bf16 path: the factor tensors after the
  * preparation step (scaled, converted and padded so the tensor cores can read
- * them). Depends on which factor dimensions are broadcast (stride 0).
- * Returns 0 when R == 0. The fp32 path needs no workspace.
+ * them), followed by a 256-byte block holding the fused kernel's work counter
+ * (the preparation step zeroes it and every fused launch leaves it at zero;
+ * the counter lets the CTAs take work items in order as they become free).
+ * Depends on which factor dimensions are broadcast (stride 0).
+ * Returns 0 when R == 0 (the kernel then deals out its work items in a fixed
+ * order). The fp32 path needs no workspace.
  */
 size_t fb_attn_workspace_bytes(int B, int H, int N, int R,
                                int64_t phi_bstride, int64_t phi_hstride);

@@ -44,14 +44,16 @@ def test_status_strings_and_version():
 
 
 def test_workspace_bytes():
+    # Every nonzero size ends in the fused kernel's 256-byte work-counter block.
+    C = 256
     assert fb.fb_attn_workspace_bytes(8, 12, 2048, 0, 0, 0) == 0
     # broadcast Sandwich factors: one [N, 64] fp16 slice per side
-    assert fb.fb_attn_workspace_bytes(8, 12, 2048, 64, 0, 0) == 2 * 2048 * 64 * 2
+    assert fb.fb_attn_workspace_bytes(8, 12, 2048, 64, 0, 0) == 2 * 2048 * 64 * 2 + C
     # rank 8 pads to 16 columns; per-head factors
-    assert fb.fb_attn_workspace_bytes(4, 8, 4096, 8, 0, 4096 * 8) == 2 * 8 * 4096 * 16 * 2
+    assert fb.fb_attn_workspace_bytes(4, 8, 4096, 8, 0, 4096 * 8) == 2 * 8 * 4096 * 16 * 2 + C
     # rank <= 4: fp32 hi/lo split factors, 3R columns padded to 8 (R <= 2) or 16
-    assert fb.fb_attn_workspace_bytes(4, 16, 8192, 2, 0, 8192 * 2) == 2 * 16 * 8192 * 8 * 4
-    assert fb.fb_attn_workspace_bytes(1, 1, 17, 3, 0, 0) == 2 * 1280  # 17 rows x 64 B, rounded to 256 B
+    assert fb.fb_attn_workspace_bytes(4, 16, 8192, 2, 0, 8192 * 2) == 2 * 16 * 8192 * 8 * 4 + C
+    assert fb.fb_attn_workspace_bytes(1, 1, 17, 3, 0, 0) == 2 * 1280 + C  # 17 rows x 64 B, rounded to 256 B
     assert fb.fb_attn_workspace_bytes(1, 1, 16, 129, 0, 0) == 0  # out of range -> 0
 
 
@@ -63,6 +65,26 @@ def _fwd(**kw):
              phi_hstride=0, scale=0.125, causal=0, O=FAKE, LSE=FAKE, workspace=0, workspace_bytes=0, stream=None)
     a.update(kw)
     return fb.fb_attn_fwd(**a)
+
+
+def test_noalloc_reports_fb_attn_fwd_argument_errors_first():
+    """fb_attn_fwd_noalloc runs fb_attn_fwd's argument checks before its own
+    size limit, so a bad argument gets the same status from both, even for a
+    problem whose prepared factors would not fit its fixed array."""
+    def na(**kw):
+        a = dict(dt=fb.FB_BF16, B=4, H=16, N=8192, d=64, Q=FAKE, K=FAKE, V=FAKE, R=64, phi_q=FAKE, phi_k=FAKE,
+                 phi_bstride=16 * 8192 * 64, phi_hstride=8192 * 64, scale=0.125, causal=1, O=FAKE, LSE=FAKE,
+                 stream=None)
+        a.update(kw)
+        return fb.fb_attn_fwd_noalloc(**a)
+
+    for bad in (dict(Q=0), dict(O=FAKE + 4), dict(scale=0.0), dict(phi_hstride=-1), dict(d=12), dict(N=0),
+                dict(dt=fb.FB_F16), dict(R=200)):
+        full = dict(B=4, H=16, N=8192, d=64, R=64, phi_q=FAKE, phi_k=FAKE, phi_bstride=16 * 8192 * 64,
+                    phi_hstride=8192 * 64, causal=1)
+        full.update(bad)
+        assert na(**bad) == _fwd(**full) != fb.FB_OK, bad
+    assert na() == fb.FB_ERR_WORKSPACE  # valid, but beyond the 8 MiB array
 
 
 def test_forward_rejects_bad_arguments_before_launch():
@@ -78,9 +100,10 @@ def test_forward_rejects_bad_arguments_before_launch():
     assert _fwd(R=8, phi_q=FAKE, phi_k=FAKE, phi_bstride=-1) == fb.FB_ERR_INVALID_ARG
     assert _fwd(d=12) == fb.FB_ERR_UNSUPPORTED
     assert _fwd(d=136) == fb.FB_ERR_UNSUPPORTED
-    assert _fwd(N=0) == fb.FB_ERR_UNSUPPORTED
-    assert _fwd(B=0) == fb.FB_ERR_UNSUPPORTED
+    assert _fwd(N=0) == fb.FB_ERR_INVALID_ARG
+    assert _fwd(B=0) == fb.FB_ERR_INVALID_ARG
     assert _fwd(dt=7) == fb.FB_ERR_UNSUPPORTED
+    assert _fwd(dt=fb.FB_F16) == fb.FB_ERR_UNSUPPORTED  # fp16 inputs are not implemented
     assert _fwd(dt=fb.FB_F32, d=6) == fb.FB_ERR_UNSUPPORTED
     # workspace missing / too small / misaligned
     assert _fwd(R=8, phi_q=FAKE, phi_k=FAKE) == fb.FB_ERR_WORKSPACE
@@ -195,7 +218,7 @@ def test_prepared_entry_points_reject_bad_arguments_before_launch():
 
     assert p(R=0, phi_q=0, phi_k=0, workspace=0, workspace_bytes=0) == fb.FB_OK  # nothing to prepare
     assert p(R=129) == fb.FB_ERR_UNSUPPORTED
-    assert p(N=0) == fb.FB_ERR_UNSUPPORTED
+    assert p(N=0) == fb.FB_ERR_INVALID_ARG
     assert p(phi_q=0) == fb.FB_ERR_INVALID_ARG
     assert p(phi_k=FAKE + 2) == fb.FB_ERR_INVALID_ARG
     assert p(phi_hstride=-1) == fb.FB_ERR_INVALID_ARG
