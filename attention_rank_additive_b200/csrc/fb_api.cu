@@ -75,10 +75,11 @@ bool encode_qkv(CUtensorMap *m, const void *ptr, int BH, int N, int d, int DP) {
   return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, ptr, dims, strides, box, swizzle_for(ch * 2));
 }
 
-// O: bf16 [BH, N, d] with a box of (min(DP, 32), 32, 1), the epilogue's
-// per-warp TMA store (columns and rows past the tensor are not written).
-bool encode_o(CUtensorMap *m, void *ptr, int BH, int N, int d, int DP) {
-  const int e = DP < 32 ? DP : 32;
+// O: bf16 [BH, N, d] with a box of (e, 32, 1), e the plan's epilogue chunk
+// width: the per-warp TMA store (columns and rows past the tensor are not
+// written).
+bool encode_o(CUtensorMap *m, void *ptr, int BH, int N, int d, int e) {
+  if (e != 16 && e != 32 && e != 64) return false;
   const uint64_t dims[3] = {uint64_t(d), uint64_t(N), uint64_t(BH)};
   const uint64_t strides[2] = {uint64_t(d) * 2, uint64_t(N) * d * 2};
   const uint32_t box[3] = {uint32_t(e), 32u, 1u};
@@ -278,7 +279,7 @@ int fb_attn_fwd_prepared(int dt, int B, int H, int N, int d, const void *Q, cons
   std::memset(&maps, 0, sizeof(maps));
   const int BH = B * H;
   if (!encode_qkv(&maps.q, Q, BH, N, d, DP) || !encode_qkv(&maps.k, K, BH, N, d, DP) ||
-      !encode_qkv(&maps.v, V, BH, N, d, DP) || !encode_o(&maps.o, O, BH, N, d, DP))
+      !encode_qkv(&maps.v, V, BH, N, d, DP) || !encode_o(&maps.o, O, BH, N, d, sm100_epi_cols(plan)))
     return FB_ERR_CUDA;
   const uint8_t *wsb = static_cast<const uint8_t *>(workspace);
   void *wq = ws.total ? const_cast<uint8_t *>(wsb) + ws.q_off : nullptr;
@@ -542,7 +543,7 @@ int fb_attn_dense_bias_fwd(int dt, int B, int H, int N, int d, const void *Q, co
   std::memset(&maps, 0, sizeof(maps));
   const int BH = B * H;
   if (!encode_qkv(&maps.q, Q, BH, N, d, DP) || !encode_qkv(&maps.k, K, BH, N, d, DP) ||
-      !encode_qkv(&maps.v, V, BH, N, d, DP) || !encode_o(&maps.o, O, BH, N, d, DP))
+      !encode_qkv(&maps.v, V, BH, N, d, DP) || !encode_o(&maps.o, O, BH, N, d, sm100_epi_cols(plan)))
     return FB_ERR_CUDA;
   const int bias_B = bias_bstride == 0 ? 1 : B, bias_H = bias_hstride == 0 ? 1 : H;
   {

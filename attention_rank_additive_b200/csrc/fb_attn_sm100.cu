@@ -50,6 +50,10 @@
 
 namespace fb {
 
+#ifndef FB_KS_MAX
+#define FB_KS_MAX 2
+#endif
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when the max grows by > 2^8
@@ -92,7 +96,8 @@ struct Sm100Cfg {
   static constexpr int KS_FIT = (kSmemLimit > FIXED + CTRL + ALIGN_SLACK)
                                     ? int((kSmemLimit - FIXED - CTRL - ALIGN_SLACK) / STAGE)
                                     : 0;
-  static constexpr int KS = KS_FIT > 3 ? 3 : KS_FIT;
+  static constexpr int KS_MAX = FB_KS_MAX;
+  static constexpr int KS = KS_FIT > KS_MAX ? KS_MAX : KS_FIT;
   // QT softmax warpgroups + one warpgroup holding the producer warp, the MMA
   // warp and two idle warps. Registers are moved from that warpgroup to the
   // softmax warpgroups with setmaxnreg: the launch allocation is
@@ -103,13 +108,18 @@ struct Sm100Cfg {
   // a warp's 32 rows at a time (one staging slot per softmax warp), when the
   // slots fit beside the rings (for a two-per-SM plan: within half an SM);
   // otherwise each thread stores its own row.
-  static constexpr int EPI_E = DP < 32 ? DP : 32;
-  static constexpr uint32_t STG_WARP = 32u * uint32_t(EPI_E) * 2u;
-  static constexpr uint32_t STG = uint32_t(NSWG) * 4u * STG_WARP;
   static constexpr uint32_t SMEM_BASE = FIXED + uint32_t(KS) * STAGE + CTRL + ALIGN_SLACK;
   static constexpr uint32_t kPairLimit = 228u * 1024u / 2u - 1024u;
-  static constexpr bool TMA_EPI = (SMALL && SMEM_BASE <= kPairLimit) ? (SMEM_BASE + STG <= kPairLimit)
-                                                                      : (SMEM_BASE + STG <= kSmemLimit);
+  static constexpr uint32_t SMEM_CAP = (SMALL && SMEM_BASE <= kPairLimit) ? kPairLimit : kSmemLimit;
+  // a whole 64-column row chunk per warp where it fits (one store per warp
+  // for head dims up to 64), else 32 columns (the key split always uses 32)
+  static constexpr int EPI_E_WIDE = DP < 64 ? DP : 64;
+  static constexpr bool WIDE_FITS =
+      !KSPLIT && SMEM_BASE + uint32_t(NSWG) * 4u * 32u * uint32_t(EPI_E_WIDE) * 2u <= SMEM_CAP;
+  static constexpr int EPI_E = WIDE_FITS ? EPI_E_WIDE : (DP < 32 ? DP : 32);
+  static constexpr uint32_t STG_WARP = 32u * uint32_t(EPI_E) * 2u;
+  static constexpr uint32_t STG = uint32_t(NSWG) * 4u * STG_WARP;
+  static constexpr bool TMA_EPI = SMEM_BASE + STG <= SMEM_CAP;
   static constexpr uint32_t SMEM = SMEM_BASE + (TMA_EPI ? STG : 0u);
   static constexpr int MIN_BLOCKS = SMALL ? 2 : 1;
   static constexpr int LAUNCH_REGS = SMALL ? 128 : 168;
@@ -202,20 +212,20 @@ __device__ __forceinline__ float row_max(const uint32_t *x) {
 
 // One chunk of the epilogue: a warp's 32 rows x E bf16 columns (thread =
 // row; pk holds its E/2 packed pairs) go into the warp's staging slot, laid
-// out in the TMA swizzle of an E*2-byte row (64 B: 16-byte chunk j of row r
-// at j ^ ((r >> 1) & 3); 32 B: at j ^ ((r >> 2) & 1)), so that the
+// out in the TMA swizzle of an E*2-byte row (128 B: 16-byte chunk j of row r
+// at j ^ (r & 7); 64 B: at j ^ ((r >> 1) & 3); 32 B: at j ^ ((r >> 2) & 1)), so that the
 // row-per-thread writes are free of bank conflicts; lane 0 then issues one
 // tiled store of the slot at (col, row0, bh). The slot is rewritten only
 // after its previous store has read it.
 template <int E>
 __device__ __forceinline__ void stage_and_store_o(uint8_t *slot, const uint32_t *pk, int lane, const CUtensorMap *map,
                                                   int col, int row0, int bh) {
-  static_assert(E == 16 || E == 32, "staging chunk");
+  static_assert(E == 16 || E == 32 || E == 64, "staging chunk");
   if (lane == 0) bulk_wait_group_read0();
   __syncwarp();
 #pragma unroll
   for (int j = 0; j < E / 8; ++j) {
-    const int pj = E == 32 ? (j ^ ((lane >> 1) & 3)) : (j ^ ((lane >> 2) & 1));
+    const int pj = E == 64 ? (j ^ (lane & 7)) : (E == 32 ? (j ^ ((lane >> 1) & 3)) : (j ^ ((lane >> 2) & 1)));
     *reinterpret_cast<uint4 *>(slot + lane * (E * 2) + pj * 16) =
         make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
   }
@@ -1178,7 +1188,12 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
 #pragma unroll
             for (int c0 = 0; c0 < DP; c0 += C::EPI_E) {
               uint32_t r[C::EPI_E];
-              if constexpr (C::EPI_E == 32) {
+              if constexpr (C::EPI_E == 64) {
+                tmem_ld32(o_tm + c0, r);
+                tmem_ld32(o_tm + c0 + 32, r + 32);
+                tmem_ld_wait32(r);
+                tmem_ld_wait32(r + 32);
+              } else if constexpr (C::EPI_E == 32) {
                 tmem_ld32(o_tm + c0, r);
                 tmem_ld_wait32(r);
               } else {
@@ -1314,6 +1329,12 @@ static constexpr size_t smem_of() {
   return C::KS >= 1 ? size_t(C::SMEM) : 0;
 }
 
+template <int DP, int RP, int MODE, int QT>
+static constexpr int epi_cols_of() {
+  using C = Sm100Cfg<DP, RP, MODE, QT>;
+  return C::EPI_E;
+}
+
 #define FB_DISPATCH_QT(DPv, RPv, MODEv)                                          \
   if (p.QT == 1) return FB_ACTION(DPv, RPv, MODEv, 1);                           \
   if (p.QT == 2) return FB_ACTION(DPv, RPv, MODEv, 2);
@@ -1340,6 +1361,13 @@ static constexpr size_t smem_of() {
 
 size_t sm100_smem_bytes(const FwdPlan &p) {
 #define FB_ACTION(DPv, RPv, MODEv, QTv) smem_of<DPv, RPv, MODEv, QTv>()
+  FB_DISPATCH_ALL
+#undef FB_ACTION
+  return 0;
+}
+
+int sm100_epi_cols(const FwdPlan &p) {
+#define FB_ACTION(DPv, RPv, MODEv, QTv) epi_cols_of<DPv, RPv, MODEv, QTv>()
   FB_DISPATCH_ALL
 #undef FB_ACTION
   return 0;

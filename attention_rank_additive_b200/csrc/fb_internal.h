@@ -54,6 +54,8 @@ struct FwdMaps {
 
 // Shared-memory bytes the kernel needs for a plan, or 0 if it does not fit.
 size_t sm100_smem_bytes(const FwdPlan &p);
+// Columns of O per epilogue TMA store (the O tensor map's box width) for a plan.
+int sm100_epi_cols(const FwdPlan &p);
 // Launches the tcgen05 kernel; returns a cudaError_t.
 cudaError_t sm100_launch(const FwdPlan &p, const FwdMaps &maps, const FwdArgs &a, cudaStream_t stream);
 

@@ -2,11 +2,14 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
 
-One step is one pass of the whole hot path over one batch of the workload:
-exact factor generation (device), factor preparation and the fused tcgen05
-attention kernel. The default workload is the GPT-2-small-shaped causal
-attention with the Sandwich bias (B=8, H=12, N=2048, d=64, exact rank 64);
---config selects another of the five workloads (0..4) for measurement.
+One step is one pass of the hot path over one batch of the workload: the
+factor preparation and the fused tcgen05 attention kernel. The exact
+Sandwich/ALiBi factors depend only on N and H, so they are generated once on
+the device before timing. The default workload is the GPT-2-small-shaped
+causal attention with the Sandwich bias (B=8, H=12, N=2048, d=64, exact rank
+64); --config selects another workload (0..7) for measurement. The default
+single-GPU run also times the fused and the dense-bias kernels of the four
+bf16 workloads (1..4) on their own and reports them under "per_config".
 
 Prints one JSON line (rank 0). Under torchrun every rank runs its own batch
 (independent problems, weak scaling, no data-path collective); timing is on
@@ -53,6 +56,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-bias comparison leg")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline leg")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the per-workload leg (fused and dense kernels of workloads 1..4)")
     return ap.parse_args(argv)
 
 
@@ -466,6 +471,72 @@ def svd_device_leg(torch, fb, w, c, stream):
             "host_settings": "fb_svd_factors_host, oversample 64, power_iters 1, fp64"}
 
 
+# ------------------------------------------------------------ per workload
+
+PER_CONFIG_STEPS = {1: 100, 2: 30, 3: 60, 4: 200}
+MUFU_EXP2_PER_CLK_PER_SM = 16  # B200 special-function unit rate for exp2
+
+
+def exp2_elements(c: dict) -> float:
+    """Scores that need an exponential: B H N^2, halved when causal (as counted FLOPs)."""
+    e = float(c["B"]) * c["H"] * c["N"] * c["N"]
+    return e / 2.0 if c["causal"] else e
+
+
+def per_config_leg(torch, fb, device, stream):
+    """The fused kernel alone and the dense-bias kernel alone on each bf16
+    workload (1..4), L2 flushed between launches, CUDA events on the launching
+    stream, clocks sampled during the fused timing: the roofline fraction
+    against the peak the clock record calls for, the exp2 (special-function
+    unit) floor, and the dense kernel's bias stream against the HBM peak."""
+    burst_tf, sustained_tf, peak_hbm, peak_src = measured_peaks()
+    out = {}
+    for ci in (1, 2, 3, 4):
+        c = workload(ci)
+        w = GpuWorkload(c, device, with_dense=True)
+        w.gen_factors()
+        for _ in range(3):
+            w.attn()
+        torch.cuda.synchronize()
+        st = fb.fb_check_device_error(stream.cuda_stream)
+        assert st == fb.FB_OK, fb.fb_status_str(st)
+        w.prepare()
+        steps = PER_CONFIG_STEPS[ci]
+        with ClockSampler(device.index or 0) as clk:
+            ms = time_steps(torch, w.run, w.flush_l2, steps, stream)
+        clk_sum = clk.summary()
+        kms = statistics.median(ms)
+        capped = bool(clk_sum) and "sw_power_cap" in clk_sum.get("reasons", [])
+        peak_tf = sustained_tf if capped else burst_tf
+        achieved = c["flops"] / (kms * 1e-3) / 1e12
+        sm_max_hz = 1e6 * (clk_sum["sm_max_mhz"] if clk_sum else 1965.0)
+        floor_ms = exp2_elements(c) / (MUFU_EXP2_PER_CLK_PER_SM * 148 * sm_max_hz) * 1e3
+        entry = {"workload": config_json(c, "")["workload"], "steps": steps, "kernel_ms": round(kms, 5),
+                 "kernel_ms_mean": round(statistics.mean(ms), 5), "tflops": round(achieved, 2),
+                 "peak": peak_tf, "peak_kind": f"{peak_src} bf16 {'sustained (power-capped)' if capped else 'burst'}",
+                 "frac": round(achieved / peak_tf, 4), "traffic": profiled_traffic(ci),
+                 "exp2_floor_ms": round(floor_ms, 5), "exp2_floor_frac": round(floor_ms / kms, 4),
+                 "clocks": clk_sum}
+        if w.dense is not None:
+            for _ in range(3):
+                w.dense_attn()
+            d_ms = statistics.median(time_steps(torch, w.dense_attn, w.flush_l2, max(10, steps // 2), stream))
+            n_kv = (c["N"] + 127) // 128
+            tiles = c["B"] * c["H"] * (n_kv * (n_kv + 1) // 2 if c["causal"] else n_kv * n_kv)
+            bias_bytes = tiles * 128 * 128 * 2
+            entry["dense"] = {"ms": round(d_ms, 5), "bias_bytes_read": bias_bytes,
+                              "bias_gbs": round(bias_bytes / (d_ms * 1e-3) / 1e9, 1),
+                              "hbm_frac": round(bias_bytes / (d_ms * 1e-3) / 1e9 / peak_hbm, 4),
+                              "fused_speedup": round(d_ms / kms, 3)}
+        st = fb.fb_check_device_error(stream.cuda_stream)
+        assert st == fb.FB_OK, fb.fb_status_str(st)
+        out[f"c{ci}"] = entry
+        del w
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    return out
+
+
 # ------------------------------------------------------------------ timing
 
 def time_steps(torch, fn, before, steps: int, stream):
@@ -639,6 +710,10 @@ def run_ours(args, rank: int, world: int, local: int):
         # every rank sampled its own GPU; rank 0 reports its own
         pass
     out["clocks"] = clk_sum
+    if world == 1 and args.config == 1 and not args.no_per_config:
+        del w
+        torch.cuda.empty_cache()
+        out["per_config"] = per_config_leg(torch, fb, device, stream)
     if rank == 0 and not args.no_cpu:
         out["cpu_baseline"] = cpu_baseline(c, budget_s=12.0)
     return out
