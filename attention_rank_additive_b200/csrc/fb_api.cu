@@ -406,19 +406,11 @@ int fb_attn_mul_bias_fwd(int dt, int B, int H, int N, int d, const void *Q, cons
 }
 
 namespace {
-struct NeuralLayout {
-  size_t q_off, k_off, prep_off, prep_bytes, total;
-};
-NeuralLayout neural_layout(int B, int H, int N, int R) {
-  NeuralLayout m{};
-  const size_t phi = align256(size_t(B) * H * N * R * 4);
-  m.q_off = 0;
-  m.k_off = phi;
-  m.prep_off = 2 * phi;
+// The forward's workspace is the prepared per-head factors (as fb_attn_fwd's
+// with strides bs = H N R, hs = N R): the linear layers write them directly.
+WsLayout neural_layout(int B, int H, int N, int R) {
   const int64_t hs = int64_t(N) * R, bs = int64_t(H) * hs;
-  m.prep_bytes = workspace_layout(B, H, N, R, bs, hs).total;
-  m.total = m.prep_off + m.prep_bytes;
-  return m;
+  return workspace_layout(B, H, N, R, bs, hs);
 }
 bool neural_ok(int F, int R) { return F >= 1 && F <= 256 && R >= 1 && R <= 128 && F * R <= 8192; }
 }  // namespace
@@ -440,17 +432,21 @@ int fb_attn_neural_fwd(int dt, int B, int H, int N, int d, const void *Q, const 
         reinterpret_cast<uintptr_t>(W_k)) & 3u) != 0)
     return FB_ERR_INVALID_ARG;
   if (const int sh = shape_status_bf16(B, H, N, d)) return sh;
-  const NeuralLayout m = neural_layout(B, H, N, R);
+  const WsLayout m = neural_layout(B, H, N, R);
   if (!workspace || workspace_bytes < m.total || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return FB_ERR_WORKSPACE;
+  int *flags = device_flags();
+  if (!flags) return FB_ERR_CUDA;
   uint8_t *ws = static_cast<uint8_t *>(workspace);
-  float *pq = reinterpret_cast<float *>(ws + m.q_off), *pk = reinterpret_cast<float *>(ws + m.k_off);
-  if (launch_neural_factors(B, H, N, F, R, X_q, X_k, W_q, W_k, pq, pk, static_cast<cudaStream_t>(stream)) !=
-      cudaSuccess)
+  // one launch makes the factors in the layout the fused kernel reads, the
+  // fused kernel follows in stream order
+  const bool tf32 = R <= 4;
+  if (launch_neural_prep(B, H, N, F, R, tf32 ? tf32_cols(R) : pad_rank(R), tf32 ? 1 : 0, X_q, X_k, W_q, W_k, scale,
+                         ws + m.q_off, ws + m.k_off, flags, reinterpret_cast<unsigned int *>(ws + m.sched_off),
+                         static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return FB_ERR_CUDA;
   const int64_t hs = int64_t(N) * R, bs = int64_t(H) * hs;
-  return fb_attn_fwd(FB_BF16, B, H, N, d, Q, K, V, R, pq, pk, bs, hs, scale, causal, O, LSE, ws + m.prep_off,
-                     m.prep_bytes, stream);
+  return fb_attn_fwd_prepared(FB_BF16, B, H, N, d, Q, K, V, R, bs, hs, scale, causal, O, LSE, ws, m.total, stream);
 }
 
 size_t fb_attn_neural_bwd_workspace_bytes(int B, int H, int N, int F, int R) {

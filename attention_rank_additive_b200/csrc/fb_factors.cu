@@ -238,6 +238,114 @@ __global__ void __launch_bounds__(256) neural_factor_kernel(int H, int N, int F,
   }
 }
 
+// The neural decomposition made straight into the fused kernel's factor
+// layout, in one launch (the linear layers and the preparation step fused):
+// phi_q = X_q[b] W_q[h], phi_k = X_k[b] W_k[h] in fp32 (each sum in the order
+// f = 0, 1, ..., as neural_factor_kernel), then as the preparation step makes
+// them: fp16 [B*H, N, RP] with phi_q / scale (R > 4), or the tf32 hi/lo split
+// rows of KT = RP columns (R <= 4). One CTA per (b, h) and 64 rows, the head's
+// weights in shared memory; also zeroes the fused kernel's work counter.
+__global__ void __launch_bounds__(256) neural_prep_kernel(int H, int N, int F, int R, int RP, int tf32,
+                                                          const float *__restrict__ Xq,
+                                                          const float *__restrict__ Xk,
+                                                          const float *__restrict__ Wq,
+                                                          const float *__restrict__ Wk, float inv_scale,
+                                                          void *__restrict__ out_q, void *__restrict__ out_k,
+                                                          int *flags, unsigned int *sched) {
+  if (sched != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) sched[0] = sched[1] = 0u;
+  extern __shared__ float wsm[];  // [2][F][R]
+  const int bh = blockIdx.y, b = bh / H, h = bh - (bh / H) * H;
+  for (int e = threadIdx.x; e < F * R; e += blockDim.x) {
+    wsm[e] = Wq[(long long)h * F * R + e];
+    wsm[F * R + e] = Wk[(long long)h * F * R + e];
+  }
+  __syncthreads();
+  const long long n0 = (long long)blockIdx.x * 64;
+  bool overflow = false;
+  if (!tf32) {
+    __half *oq = static_cast<__half *>(out_q), *ok = static_cast<__half *>(out_k);
+    for (int e = threadIdx.x; e < 64 * RP; e += blockDim.x) {
+      const int rr = e / RP, r = e - rr * RP;
+      const long long n = n0 + rr;
+      if (n >= N) break;
+      float sq = 0.f, sk = 0.f;
+      if (r < R) {
+        const float *xq = Xq + ((long long)b * N + n) * F;
+        const float *xk = Xk + ((long long)b * N + n) * F;
+        for (int f = 0; f < F; ++f) {
+          sq = fmaf(xq[f], wsm[f * R + r], sq);
+          sk = fmaf(xk[f], wsm[F * R + f * R + r], sk);
+        }
+      }
+      float vq = sq * inv_scale, vk = sk;
+      if (fabsf(vq) > 65504.f) { vq = copysignf(65504.f, vq); overflow = true; }
+      if (fabsf(vk) > 65504.f) { vk = copysignf(65504.f, vk); overflow = true; }
+      if (!(vq == vq) || !(vk == vk)) overflow = true;
+      const long long o = ((long long)bh * N + n) * RP + r;
+      oq[o] = __float2half_rn(vq);
+      ok[o] = __float2half_rn(vk);
+    }
+  } else {
+    float *oq = static_cast<float *>(out_q), *ok = static_cast<float *>(out_k);
+    for (int rr = threadIdx.x; rr < 64; rr += blockDim.x) {
+      const long long n = n0 + rr;
+      if (n >= N) break;
+      const float *xq = Xq + ((long long)b * N + n) * F;
+      const float *xk = Xk + ((long long)b * N + n) * F;
+      float q[16], k[16];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) q[c] = k[c] = 0.f;
+      for (int r = 0; r < R; ++r) {
+        float sq = 0.f, sk = 0.f;
+        for (int f = 0; f < F; ++f) {
+          sq = fmaf(xq[f], wsm[f * R + r], sq);
+          sk = fmaf(xk[f], wsm[F * R + f * R + r], sk);
+        }
+        const float x = sq * inv_scale, y = sk;
+        const float xh = tf32_hi(x), yh = tf32_hi(y);
+        q[r] = xh;
+        q[R + r] = xh;
+        q[2 * R + r] = x - xh;
+        k[r] = yh;
+        k[R + r] = y - yh;
+        k[2 * R + r] = yh;
+      }
+      float4 *dq = reinterpret_cast<float4 *>(oq + ((long long)bh * N + n) * RP);
+      float4 *dk = reinterpret_cast<float4 *>(ok + ((long long)bh * N + n) * RP);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        if (4 * v < RP) {
+          dq[v] = make_float4(q[4 * v], q[4 * v + 1], q[4 * v + 2], q[4 * v + 3]);
+          dk[v] = make_float4(k[4 * v], k[4 * v + 1], k[4 * v + 2], k[4 * v + 3]);
+        }
+      }
+    }
+  }
+  if (overflow) atomicOr(flags, kFlagRange);
+}
+
+cudaError_t launch_neural_prep(int B, int H, int N, int F, int R, int RP, int tf32, const float *Xq, const float *Xk,
+                               const float *Wq, const float *Wk, float scale, void *out_q, void *out_k, int *flags,
+                               unsigned int *sched, cudaStream_t s) {
+  const size_t smem = size_t(2) * F * R * sizeof(float);
+  if (smem > 48 * 1024) {  // the opt-in above the default, once per device (64 KB covers F R <= 8192)
+    static std::atomic<int> done[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!done[dev].load(std::memory_order_acquire)) {
+      e = cudaFuncSetAttribute(neural_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+      if (e != cudaSuccess) return e;
+      done[dev].store(1, std::memory_order_release);
+    }
+  }
+  const dim3 grid((N + 63) / 64, B * H);
+  neural_prep_kernel<<<grid, 256, smem, s>>>(H, N, F, R, RP, tf32, Xq, Xk, Wq, Wk, 1.0f / scale, out_q, out_k,
+                                              flags, sched);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_neural_factors(int B, int H, int N, int F, int R, const float *Xq, const float *Xk,
                                   const float *Wq, const float *Wk, float *pq, float *pk, cudaStream_t s) {
   const size_t smem = size_t(2) * F * R * sizeof(float);

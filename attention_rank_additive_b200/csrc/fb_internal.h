@@ -79,6 +79,12 @@ cudaError_t launch_wait_selftest(int limit_ms, int *flags, cudaStream_t s);
 // Neural decomposition: phi_q[b, h] = X_q[b] W_q[h], phi_k[b, h] = X_k[b] W_k[h] (fp32).
 cudaError_t launch_neural_factors(int B, int H, int N, int F, int R, const float *Xq, const float *Xk,
                                   const float *Wq, const float *Wk, float *pq, float *pk, cudaStream_t s);
+// The same factors made straight into the fused kernel's prepared layout (fp16
+// [B*H, N, RP] with phi_q / scale, or tf32 hi/lo rows of RP columns when tf32),
+// zeroing the work counter: the linear layers and the preparation in one launch.
+cudaError_t launch_neural_prep(int B, int H, int N, int F, int R, int RP, int tf32, const float *Xq, const float *Xk,
+                               const float *Wq, const float *Wk, float scale, void *out_q, void *out_k, int *flags,
+                               unsigned int *sched, cudaStream_t s);
 // Gradients of the neural decomposition's linear layers: dW [H, F, R] from X and
 // dphi [B, H, N, R]; dX [B, N, F] from W and dphi (skipped when dXq or dXk is null).
 cudaError_t launch_neural_grads(int B, int H, int N, int F, int R, const float *Xq, const float *Xk,

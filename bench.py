@@ -229,6 +229,13 @@ def profiled_traffic(cfg_idx: int):
     return float(val.group(1))
 
 
+def fp32_fma_peak_tflops(clk_sum) -> float:
+    """fp32 FMA peak of the GPU from its unit counts and clock: 148 SMs x 128
+    FMA lanes per clock x 2 FLOP, at the maximum SM clock the run reported."""
+    mhz = clk_sum["sm_max_mhz"] if clk_sum else 1965.0
+    return 148 * 128 * 2 * mhz * 1e6 / 1e12
+
+
 def measured_peaks():
     """(bf16 burst TF/s, bf16 sustained TF/s, HBM GB/s, 'measured' | 'fallback')."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -316,8 +323,8 @@ class GpuWorkload:
         if with_dense and c["dtype"] == "bf16":
             self.dense = self._dense_bias()
         # fused kernel, plus the preparation launch (bf16 with a bias); the multiplicative case has its
-        # reweighting launch instead, the neural case its linear-layer launch in addition
-        self.launches_per_step = (3 if self.neural else
+        # reweighting launch instead, the neural case its linear layers (which write the prepared factors)
+        self.launches_per_step = (2 if self.neural else
                                   (2 if self.mul or (Rk > 0 and c["dtype"] == "bf16") else 1))
         self.bwd = bool(c.get("bwd"))
         if self.bwd:  # factor preparation, bf16 factor copies, per-row terms, two gradient kernels, and
@@ -403,7 +410,7 @@ class GpuWorkload:
         if getattr(self, "bwd_active", False):  # the whole backward call (its preparation included)
             self.run_bwd()
             return
-        if self.neural:  # linear layers + preparation + fused kernel (one C-ABI call)
+        if self.neural:  # linear layers writing the prepared factors + fused kernel (one C-ABI call)
             xq, xk, wq, wk = self.nx
             st = fb.fb_attn_neural_fwd(fb.FB_BF16, c["B"], c["H"], c["N"], c["d"], self.Q.data_ptr(),
                                        self.K.data_ptr(), self.V.data_ptr(), c["F"], self.R, xq.data_ptr(),
@@ -669,6 +676,10 @@ def run_ours(args, rank: int, world: int, local: int):
     capped = bool(clk_sum) and "sw_power_cap" in clk_sum.get("reasons", [])
     peak_tf = sustained_tf if capped else burst_tf
     peak_kind = f"{peak_src} bf16 {'sustained (run power-capped)' if capped else 'burst'}"
+    bound = "tensor"
+    if c["dtype"] == "f32":  # the fp32 path runs on the CUDA cores' FMA pipe
+        bound, peak_tf = "alu", fp32_fma_peak_tflops(clk_sum)
+        peak_kind = "derived: 148 SMs x 128 fp32 FMA/clk x 2 FLOP x max SM clock"
     achieved = c["flops"] / (kern_ms * 1e-3) / 1e12
     traffic = profiled_traffic(args.config)
     out = {
@@ -676,10 +687,10 @@ def run_ours(args, rank: int, world: int, local: int):
         "warmup": max(3, args.warmup), "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": c["dtype"], "data": "synthetic (seeded; see seeded_inputs)",
         "config": config_json(c, "flushed: 256 MiB memset between timed steps (untimed)"),
-        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak_tf, "unit": "TFLOP/s",
+        "roofline": {"bound": bound, "achieved": round(achieved, 2), "peak": round(peak_tf, 1), "unit": "TFLOP/s",
                      "frac": round(achieved / peak_tf, 4), "traffic": traffic,
                      "kernel": ("prep_mul_bias + attn_fwd_sm100" if w.mul else
-                                ("neural_factor + prep + attn_fwd_sm100" if w.neural else
+                                ("neural_prep + attn_fwd_sm100" if w.neural else
                                  ("bwd preparation (3) + attn_bwd_dkdv_sm100 + attn_bwd_dq_sm100 + factor-gradient "
                                   "reduction" if w.bwd
                                   else "attn_fwd_sm100"))),

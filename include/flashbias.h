@@ -199,9 +199,12 @@ int fb_attn_mul_bias_fwd(int dt, int B, int H, int N, int d,
  *  W_q, W_k    [H, F, R] fp32 device weights of the two linear layers.
  *              1 <= F <= 256, 1 <= R <= 128, F R <= 8192.
  *  workspace   fb_attn_neural_workspace_bytes(B, H, N, F, R) bytes, 256-byte
- *              aligned: the fp32 factors and their prepared form.
- *  Other arguments and errors as fb_attn_fwd (dt = FB_BF16 only). The linear
- *  layers run in fp32 in one launch, then fb_attn_fwd's two launches.
+ *              aligned: the factors in the form the fused kernel reads (as
+ *              fb_attn_prepare_factors writes them for per-head factors) and
+ *              the work counter.
+ *  Other arguments and errors as fb_attn_fwd (dt = FB_BF16 only). Two
+ *  launches: the linear layers run in fp32 and write the prepared factors
+ *  directly (the preparation step fused into them), then the fused kernel.
  */
 size_t fb_attn_neural_workspace_bytes(int B, int H, int N, int F, int R);
 

@@ -279,7 +279,7 @@ def neural_factors(x_q, x_k, w_q, w_k):
     return np.einsum("bnf,hfr->bhnr", xq, wq), np.einsum("bnf,hfr->bhnr", xk, wk)
 
 
-def attention_lowrank_bwd_head(q, k, v, phi_q, phi_k, do, scale: float, causal: bool, rows=None):
+def attention_lowrank_bwd_head(q, k, v, phi_q, phi_k, do, scale: float, causal: bool, rows=None, key_rows=None):
     """Gradients of one head of O = softmax(scale q k^T + phi_q phi_k^T [causal]) v
     for an upstream gradient dO, in fp64 (the chain rule through the softmax,
     whole rows at once; library matmuls).
@@ -295,10 +295,26 @@ def attention_lowrank_bwd_head(q, k, v, phi_q, phi_k, do, scale: float, causal: 
     dphi_q, dphi_k and the intermediate rowsum(P * dP) as ``delta``. With
     ``rows`` (query indices) only the row-wise results dq, dphi_q and delta
     of those queries are computed (a query row of dS needs only its own
-    score row)."""
+    score row). With ``key_rows`` (key indices) only the key-wise results dk,
+    dv and dphi_k of those keys are computed: a key column of dS needs every
+    row's softmax normaliser and rowsum(P * dP), taken here as rowsum(dO * O)
+    (equal, since O = P v), and only the dP columns of those keys."""
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
     pq, pk = _f64(phi_q), _f64(phi_k)
     N = q.shape[0]
+    if key_rows is not None:
+        kr = np.asarray(key_rows, dtype=np.int64)
+        s = float(scale) * (q @ k.T) + pq @ pk.T
+        if causal:
+            s = np.where(np.arange(N)[None, :] <= np.arange(N)[:, None], s, -np.inf)
+        m = np.max(s, axis=1, keepdims=True)
+        e = np.exp(s - m)
+        lsum = np.sum(e, axis=1, keepdims=True)
+        o = (e @ v) / lsum
+        delta = np.sum(do * o, axis=1, keepdims=True)
+        p_cols = e[:, kr] / lsum
+        ds_cols = p_cols * (do @ v[kr].T - delta)
+        return {"dk": float(scale) * (ds_cols.T @ q), "dv": p_cols.T @ do, "dphi_k": ds_cols.T @ pq}
     if rows is not None:
         rows = np.asarray(rows, dtype=np.int64)
         s = float(scale) * (q[rows] @ k.T) + pq[rows] @ pk.T

@@ -313,10 +313,11 @@ def test_svd_device_workspace_and_argument_errors():
 
 
 def test_neural_workspace_and_argument_errors():
-    al = lambda x: (x + 255) // 256 * 256
     B, H, N, F, R = 2, 4, 100, 16, 8
+    # the linear layers write the prepared per-head factors directly: the
+    # workspace is fb_attn_fwd's for per-head factors, nothing more
     prep = fb.fb_attn_workspace_bytes(B, H, N, R, H * N * R, N * R)
-    assert fb.fb_attn_neural_workspace_bytes(B, H, N, F, R) == 2 * al(B * H * N * R * 4) + prep
+    assert fb.fb_attn_neural_workspace_bytes(B, H, N, F, R) == prep
     assert fb.fb_attn_neural_workspace_bytes(B, H, N, 128, 128) == 0  # F R > 8192
     need = fb.fb_attn_neural_workspace_bytes(1, 2, 128, F, R)
     run = dict(dt=fb.FB_BF16, B=1, H=2, N=128, d=64, Q=FAKE, K=FAKE, V=FAKE, F=F, R=R, X_q=FAKE, X_k=FAKE,

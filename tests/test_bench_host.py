@@ -54,3 +54,14 @@ def test_reference_arm_json_line(cfg):
     assert out["e2e"]["h2d_bytes_per_step"] == 0 and out["e2e"]["d2h_bytes_per_step"] == 0
     assert out["cpu_baseline"]["kind"] == "oracle" and out["cpu_baseline"]["value"] == out["value"]
     json.dumps(out)
+
+
+def test_fp32_peak_and_exp2_counts():
+    """The fp32 path's roofline peak (148 SMs x 128 FMA lanes x 2 FLOP per
+    clock) and the exp2 counts behind the special-function-unit floor."""
+    assert abs(bench.fp32_fma_peak_tflops({"sm_max_mhz": 1965.0}) - 74.45) < 0.01
+    assert abs(bench.fp32_fma_peak_tflops(None) - 74.45) < 0.01
+    c1 = bench.workload(1)  # causal: half of B H N^2
+    assert bench.exp2_elements(c1) == 8 * 12 * 2048 * 2048 / 2
+    c3 = bench.workload(3)  # no mask: all of them
+    assert bench.exp2_elements(c3) == 4 * 8 * 4096 * 4096

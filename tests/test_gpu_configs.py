@@ -1,7 +1,9 @@
 """GPU parity on the five benchmark workloads at their full sizes, in the
 launch configuration the benchmark uses. The oracle evaluates sampled query
 rows of sampled heads one by one (always the first and last row)."""
+import concurrent.futures
 import math
+import os
 
 import numpy as np
 import pytest
@@ -204,8 +206,9 @@ def test_config7_backward_full_size():
     full size through fb_attn_bwd. Every gradient of two whole heads against
     the oracle; dphi_q (the Sandwich factor is shared by all 96 heads, so its
     gradient sums over them) on sampled rows through the oracle's
-    row-restricted backward of every head; dphi_k by the zero column sums that
-    rows of dS summing to zero imply."""
+    row-restricted backward of every head, and dphi_k on sampled rows through
+    its key-restricted backward of every head; also the zero column sums of
+    dphi_k that rows of dS summing to zero imply."""
     c = si.CONFIGS[7]
     B, H, N, d, R = c["B"], c["H"], c["N"], c["d"], c["R"]
     q, k, v = si.qkv(B, H, N, d, si.QKV_SEED_BASE + 7, "bf16")
@@ -230,6 +233,16 @@ def test_config7_backward_full_size():
             ref += oracle.attention_lowrank_bwd_head(q[b, h], k[b, h], v[b, h], ph, ph, g[b, h], scale, True,
                                                      rows=rows)["dphi_q"]
     grad_close(host(dpq)[rows], ref, "c7 dphi_q rows")
+    keys = si.sample_rows(N, 12, 17)
+
+    def key_part(bh):  # one head's contribution (its whole score matrix, in fp64)
+        b, h = divmod(bh, H)
+        return oracle.attention_lowrank_bwd_head(q[b, h], k[b, h], v[b, h], ph, ph, g[b, h], scale, True,
+                                                 key_rows=keys)["dphi_k"]
+
+    with concurrent.futures.ThreadPoolExecutor(max_workers=os.cpu_count() or 4) as pool:
+        refk = sum(pool.map(key_part, range(B * H)))
+    grad_close(host(dpk)[keys], refk, "c7 dphi_k rows")
     gk = host(dpk)
     assert np.all(np.isfinite(gk))
     assert np.abs(gk.sum(axis=0)).max() <= 2e-2 * np.abs(gk).max() * math.sqrt(N), "c7 dphi_k column sums"

@@ -413,7 +413,9 @@ def test_backward_invariants(causal):
 @pytest.mark.parametrize("causal", [False, True])
 def test_backward_row_subset_matches_whole_head(causal):
     """The row-restricted backward (dq, dphi_q, delta of chosen queries) is the
-    same computation on fewer score rows: it must agree with the whole head."""
+    same computation on fewer score rows, and the key-restricted one (dk, dv,
+    dphi_k of chosen keys) takes rowsum(P dP) as rowsum(dO O): both must agree
+    with the whole head."""
     N, d, R = 70, 8, 3
     q, k, v = (_rand((N, d), s) for s in (61, 62, 63))
     pq, pk = _rand((N, R), 64), _rand((N, R), 65)
@@ -423,6 +425,11 @@ def test_backward_row_subset_matches_whole_head(causal):
     part = oracle.attention_lowrank_bwd_head(q, k, v, pq, pk, g, 0.4, causal, rows=rows)
     for key in ("dq", "dphi_q", "delta"):
         np.testing.assert_allclose(part[key], full[key][rows], rtol=0, atol=1e-13)
+    # the key-row form (its rowsum term through rowsum(dO * O)) against the whole head
+    keys = np.array([0, 4, 33, 69])
+    kpart = oracle.attention_lowrank_bwd_head(q, k, v, pq, pk, g, 0.4, causal, key_rows=keys)
+    for key in ("dk", "dv", "dphi_k"):
+        np.testing.assert_allclose(kpart[key], full[key][keys], rtol=0, atol=1e-12)
 
 
 def test_neural_backward_matches_finite_differences():
