@@ -308,6 +308,7 @@ int fb_attn_fwd_prepared(int dt, int B, int H, int N, int d, const void *Q, cons
   a.n_kv = (N + 127) / 128;
   a.n_cta_q = (a.n_kv + plan.QT - 1) / plan.QT;
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.scale = scale;
   a.causal = causal ? 1 : 0;
   a.O = O;
   a.LSE = LSE;
@@ -558,6 +559,7 @@ int fb_attn_dense_bias_fwd(int dt, int B, int H, int N, int d, const void *Q, co
   a.n_kv = (N + 127) / 128;
   a.n_cta_q = (a.n_kv + plan.QT - 1) / plan.QT;
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.scale = scale;
   a.causal = causal ? 1 : 0;
   a.O = O;
   a.LSE = LSE;
@@ -715,6 +717,7 @@ int fb_attn_bwd(int dt, int B, int H, int N, int d, const void *Q, const void *K
   a.Npad = L.Npad;
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.scale = scale;
   a.causal = causal ? 1 : 0;
   a.nlse2 = nlse2;
   a.delta = delta;

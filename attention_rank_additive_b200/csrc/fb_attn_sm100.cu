@@ -237,6 +237,30 @@ __device__ __forceinline__ void stage_and_store_o(uint8_t *slot, const uint32_t 
   }
 }
 
+// Dense-bias comparison path: x[c] = scale * x[c] + bias[c] (natural-log
+// units; the softmax then multiplies by log2 e) for 64 columns of this
+// thread's row, the bias read from its 128-byte-swizzled bf16 tile in shared
+// memory (16-byte chunk j of row r at j ^ (r & 7)). A bf16 pair becomes an
+// fp32 pair by a shift and a mask, then one packed fma per pair.
+__device__ __forceinline__ void add_dense_bias(uint32_t *x, const uint8_t *tile, int r_loc, float scale) {
+  const uint64_t sc2 = f2_pack(scale, scale);
+#pragma unroll
+  for (int ck = 0; ck < 8; ++ck) {
+    const uint4 u = *reinterpret_cast<const uint4 *>(tile + r_loc * 128 + ((ck ^ (r_loc & 7)) * 16));
+    const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int c = ck * 8 + 2 * e;
+      const uint64_t b2 = f2_pack(__uint_as_float(wv[e] << 16), __uint_as_float(wv[e] & 0xFFFF0000u));
+      const uint64_t r2 = f2_fma(f2_pack(__uint_as_float(x[c]), __uint_as_float(x[c + 1])), sc2, b2);
+      float lo, hi;
+      f2_unpack(r2, lo, hi);
+      x[c] = __float_as_uint(lo);
+      x[c + 1] = __float_as_uint(hi);
+    }
+  }
+}
+
 // One schedulable work item: a group of QT query tiles of one (b, h) head.
 struct WorkItem {
   int bh, b, h, fb_slice;
@@ -840,23 +864,11 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
           tmem_ld_wait32(x + 32);
           tc_fence_before();
           mbar_arrive(&ctrl->s_free[0]);  // S is in registers: the tensor core may overwrite it
-          float mul = sl2;  // logit = raw * mul
+          float mul = sl2;  // log2-domain logit = x * mul
           if (MODE == kBiasDense) {
-            const uint8_t *tile = sAux + s * C::AUX_TILE + h * 16384;
-#pragma unroll
-            for (int ck = 0; ck < 8; ++ck) {
-              const uint4 u = *reinterpret_cast<const uint4 *>(tile + r_loc * 128 + ((ck ^ (r_loc & 7)) * 16));
-              const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int c = ck * 8 + 2 * e;
-                x[c] = __float_as_uint(fmaf(__uint_as_float(wv[e] << 16), kLog2e, __uint_as_float(x[c]) * sl2));
-                x[c + 1] = __float_as_uint(
-                    fmaf(__uint_as_float(wv[e] & 0xFFFF0000u), kLog2e, __uint_as_float(x[c + 1]) * sl2));
-              }
-            }
+            add_dense_bias(x, sAux + s * C::AUX_TILE + h * 16384, r_loc, args.scale);
             mbar_arrive(&ctrl->aux_empty[0][s]);
-            mul = 1.f;
+            mul = kLog2e;
           }
           // Causal diagonal tile and the ragged last key tile.
           const int key0 = (n - 1 - i) * 128 + 64 * h;  // first key of this half
@@ -1056,27 +1068,13 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
             tc_fence_before();
             mbar_arrive(&ctrl->s_free[t]);
           }
-          float mul = sl2;  // logit = raw * mul
+          float mul = sl2;  // log2-domain logit = x * mul
           if (MODE == kBiasDense) {
             const uint8_t *tile = sAux + (t * KS + s) * C::AUX_TILE;
-  #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-  #pragma unroll
-              for (int ck = 0; ck < 8; ++ck) {
-                const uint4 u =
-                    *reinterpret_cast<const uint4 *>(tile + hh * 16384 + r_loc * 128 + ((ck ^ (r_loc & 7)) * 16));
-                const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
-  #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const int c = hh * 64 + ck * 8 + 2 * e;
-                  x[c] = __float_as_uint(fmaf(__uint_as_float(wv[e] << 16), kLog2e, __uint_as_float(x[c]) * sl2));
-                  x[c + 1] = __float_as_uint(
-                      fmaf(__uint_as_float(wv[e] & 0xFFFF0000u), kLog2e, __uint_as_float(x[c + 1]) * sl2));
-                }
-              }
-            }
+            add_dense_bias(x, tile, r_loc, args.scale);
+            add_dense_bias(x + 64, tile + 16384, r_loc, args.scale);
             mbar_arrive(&ctrl->aux_empty[t][s]);
-            mul = 1.f;
+            mul = kLog2e;
           }
           // Causal diagonal tile and the ragged last key tile.
           const int key0 = (w.n_steps - 1 - i) * 128;

@@ -240,109 +240,161 @@ __global__ void __launch_bounds__(256) neural_factor_kernel(int H, int N, int F,
 
 // The neural decomposition made straight into the fused kernel's factor
 // layout, in one launch (the linear layers and the preparation step fused):
-// phi_q = X_q[b] W_q[h], phi_k = X_k[b] W_k[h] in fp32 (each sum in the order
-// f = 0, 1, ..., as neural_factor_kernel), then as the preparation step makes
-// them: fp16 [B*H, N, RP] with phi_q / scale (R > 4), or the tf32 hi/lo split
-// rows of KT = RP columns (R <= 4). One CTA per (b, h) and 64 rows, the head's
-// weights in shared memory; also zeroes the fused kernel's work counter.
-__global__ void __launch_bounds__(256) neural_prep_kernel(int H, int N, int F, int R, int RP, int tf32,
-                                                          const float *__restrict__ Xq,
-                                                          const float *__restrict__ Xk,
-                                                          const float *__restrict__ Wq,
-                                                          const float *__restrict__ Wk, float inv_scale,
-                                                          void *__restrict__ out_q, void *__restrict__ out_k,
-                                                          int *flags, unsigned int *sched) {
-  if (sched != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) sched[0] = sched[1] = 0u;
-  extern __shared__ float wsm[];  // [2][F][R]
+// phi_q = X_q[b] W_q[h], phi_k = X_k[b] W_k[h] in fp32, each sum in the order
+// f = 0, 1, ..., F-1 (as neural_factor_kernel), then as the preparation step
+// makes them: fp16 [B*H, N, RP] with phi_q / scale (R > 4), or the tf32 hi/lo
+// split rows of KT = RP columns (R <= 4). Also zeroes the fused kernel's work
+// counter.
+//
+// R > 4: a 64-row x TW-column tile of phi per CTA (TW = 32, or 16 when
+// RP = 16), X and W staged in shared memory 32 features at a time (X
+// transposed), each thread a 4 x 4 block of both products.
+template <int TW>
+__global__ void __launch_bounds__(64 * TW / 16) neural_prep_mma_kernel(
+    int H, int N, int F, int R, int RP, const float *__restrict__ Xq, const float *__restrict__ Xk,
+    const float *__restrict__ Wq, const float *__restrict__ Wk, float inv_scale, __half *__restrict__ oq,
+    __half *__restrict__ ok, int *flags, unsigned int *sched) {
+  constexpr int NT = 64 * TW / 16;  // threads
+  constexpr int FC = 32;            // features per stage
+  __shared__ __align__(16) float xs[2][FC][68];   // [side][f][row], rows padded against bank conflicts
+  __shared__ __align__(16) float ws[2][FC][TW];   // [side][f][col]
+  if (sched != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0)
+    sched[0] = sched[1] = 0u;
   const int bh = blockIdx.y, b = bh / H, h = bh - (bh / H) * H;
-  for (int e = threadIdx.x; e < F * R; e += blockDim.x) {
-    wsm[e] = Wq[(long long)h * F * R + e];
-    wsm[F * R + e] = Wk[(long long)h * F * R + e];
-  }
-  __syncthreads();
   const long long n0 = (long long)blockIdx.x * 64;
-  bool overflow = false;
-  if (!tf32) {
-    __half *oq = static_cast<__half *>(out_q), *ok = static_cast<__half *>(out_k);
-    for (int e = threadIdx.x; e < 64 * RP; e += blockDim.x) {
-      const int rr = e / RP, r = e - rr * RP;
+  const int c0 = blockIdx.z * TW;
+  const int tr = threadIdx.x % 16, tc = threadIdx.x / 16;  // rows 4 tr .. 4 tr + 3, cols 4 tc .. 4 tc + 3
+  float aq[4][4], ak[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) aq[i][j] = ak[i][j] = 0.f;
+  for (int f0 = 0; f0 < F; f0 += FC) {
+    const int fc = min(FC, F - f0);
+    for (int e = threadIdx.x; e < 64 * FC; e += NT) {
+      const int rr = e / FC, f = e - rr * FC;  // consecutive threads: consecutive features of one row
       const long long n = n0 + rr;
-      if (n >= N) break;
-      float sq = 0.f, sk = 0.f;
-      if (r < R) {
-        const float *xq = Xq + ((long long)b * N + n) * F;
-        const float *xk = Xk + ((long long)b * N + n) * F;
-        for (int f = 0; f < F; ++f) {
-          sq = fmaf(xq[f], wsm[f * R + r], sq);
-          sk = fmaf(xk[f], wsm[F * R + f * R + r], sk);
-        }
+      float vq = 0.f, vk = 0.f;
+      if (n < N && f < fc) {
+        vq = Xq[((long long)b * N + n) * F + f0 + f];
+        vk = Xk[((long long)b * N + n) * F + f0 + f];
       }
-      float vq = sq * inv_scale, vk = sk;
+      xs[0][f][rr] = vq;
+      xs[1][f][rr] = vk;
+    }
+    for (int e = threadIdx.x; e < FC * TW; e += NT) {
+      const int f = e / TW, c = e - f * TW;
+      const int r = c0 + c;
+      float vq = 0.f, vk = 0.f;
+      if (f < fc && r < R) {
+        vq = Wq[((long long)h * F + f0 + f) * R + r];
+        vk = Wk[((long long)h * F + f0 + f) * R + r];
+      }
+      ws[0][f][c] = vq;
+      ws[1][f][c] = vk;
+    }
+    __syncthreads();
+    for (int f = 0; f < fc; ++f) {
+      const float4 xq4 = *reinterpret_cast<const float4 *>(&xs[0][f][4 * tr]);
+      const float4 xk4 = *reinterpret_cast<const float4 *>(&xs[1][f][4 * tr]);
+      const float4 wq4 = *reinterpret_cast<const float4 *>(&ws[0][f][4 * tc]);
+      const float4 wk4 = *reinterpret_cast<const float4 *>(&ws[1][f][4 * tc]);
+      const float xq[4] = {xq4.x, xq4.y, xq4.z, xq4.w}, xk[4] = {xk4.x, xk4.y, xk4.z, xk4.w};
+      const float wq[4] = {wq4.x, wq4.y, wq4.z, wq4.w}, wk[4] = {wk4.x, wk4.y, wk4.z, wk4.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          aq[i][j] = fmaf(xq[i], wq[j], aq[i][j]);
+          ak[i][j] = fmaf(xk[i], wk[j], ak[i][j]);
+        }
+    }
+    __syncthreads();
+  }
+  bool overflow = false;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const long long n = n0 + 4 * tr + i;
+    if (n >= N) break;
+    __half hq[4], hk[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float vq = aq[i][j] * inv_scale, vk = ak[i][j];
       if (fabsf(vq) > 65504.f) { vq = copysignf(65504.f, vq); overflow = true; }
       if (fabsf(vk) > 65504.f) { vk = copysignf(65504.f, vk); overflow = true; }
       if (!(vq == vq) || !(vk == vk)) overflow = true;
-      const long long o = ((long long)bh * N + n) * RP + r;
-      oq[o] = __float2half_rn(vq);
-      ok[o] = __float2half_rn(vk);
+      hq[j] = __float2half_rn(vq);
+      hk[j] = __float2half_rn(vk);
     }
-  } else {
-    float *oq = static_cast<float *>(out_q), *ok = static_cast<float *>(out_k);
-    for (int rr = threadIdx.x; rr < 64; rr += blockDim.x) {
-      const long long n = n0 + rr;
-      if (n >= N) break;
-      const float *xq = Xq + ((long long)b * N + n) * F;
-      const float *xk = Xk + ((long long)b * N + n) * F;
-      float q[16], k[16];
-#pragma unroll
-      for (int c = 0; c < 16; ++c) q[c] = k[c] = 0.f;
-      for (int r = 0; r < R; ++r) {
-        float sq = 0.f, sk = 0.f;
-        for (int f = 0; f < F; ++f) {
-          sq = fmaf(xq[f], wsm[f * R + r], sq);
-          sk = fmaf(xk[f], wsm[F * R + f * R + r], sk);
-        }
-        const float x = sq * inv_scale, y = sk;
-        const float xh = tf32_hi(x), yh = tf32_hi(y);
-        q[r] = xh;
-        q[R + r] = xh;
-        q[2 * R + r] = x - xh;
-        k[r] = yh;
-        k[R + r] = y - yh;
-        k[2 * R + r] = yh;
-      }
-      float4 *dq = reinterpret_cast<float4 *>(oq + ((long long)bh * N + n) * RP);
-      float4 *dk = reinterpret_cast<float4 *>(ok + ((long long)bh * N + n) * RP);
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        if (4 * v < RP) {
-          dq[v] = make_float4(q[4 * v], q[4 * v + 1], q[4 * v + 2], q[4 * v + 3]);
-          dk[v] = make_float4(k[4 * v], k[4 * v + 1], k[4 * v + 2], k[4 * v + 3]);
-        }
-      }
-    }
+    const long long o = ((long long)bh * N + n) * RP + c0 + 4 * tc;  // 8-byte aligned: RP, c0, 4 tc multiples of 4
+    *reinterpret_cast<uint2 *>(oq + o) = *reinterpret_cast<const uint2 *>(hq);
+    *reinterpret_cast<uint2 *>(ok + o) = *reinterpret_cast<const uint2 *>(hk);
   }
   if (overflow) atomicOr(flags, kFlagRange);
+}
+
+// R <= 4: one thread per row, the few products as plain loops, then the tf32
+// hi/lo split of the preparation step.
+__global__ void __launch_bounds__(128) neural_prep_tf32_kernel(int H, int N, int F, int R, int KT,
+                                                               const float *__restrict__ Xq,
+                                                               const float *__restrict__ Xk,
+                                                               const float *__restrict__ Wq,
+                                                               const float *__restrict__ Wk, float inv_scale,
+                                                               float *__restrict__ oq, float *__restrict__ ok,
+                                                               unsigned int *sched) {
+  if (sched != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) sched[0] = sched[1] = 0u;
+  const int bh = blockIdx.y, b = bh / H, h = bh - (bh / H) * H;
+  const long long n = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= N) return;
+  const float *xq = Xq + ((long long)b * N + n) * F;
+  const float *xk = Xk + ((long long)b * N + n) * F;
+  float q[16], k[16];
+#pragma unroll
+  for (int c = 0; c < 16; ++c) q[c] = k[c] = 0.f;
+  for (int r = 0; r < R; ++r) {
+    float sq = 0.f, sk = 0.f;
+    for (int f = 0; f < F; ++f) {
+      sq = fmaf(xq[f], Wq[((long long)h * F + f) * R + r], sq);
+      sk = fmaf(xk[f], Wk[((long long)h * F + f) * R + r], sk);
+    }
+    const float x = sq * inv_scale, y = sk;
+    const float xh = tf32_hi(x), yh = tf32_hi(y);
+    q[r] = xh;
+    q[R + r] = xh;
+    q[2 * R + r] = x - xh;
+    k[r] = yh;
+    k[R + r] = y - yh;
+    k[2 * R + r] = yh;
+  }
+  float4 *dq = reinterpret_cast<float4 *>(oq + ((long long)bh * N + n) * KT);
+  float4 *dk = reinterpret_cast<float4 *>(ok + ((long long)bh * N + n) * KT);
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    if (4 * v < KT) {
+      dq[v] = make_float4(q[4 * v], q[4 * v + 1], q[4 * v + 2], q[4 * v + 3]);
+      dk[v] = make_float4(k[4 * v], k[4 * v + 1], k[4 * v + 2], k[4 * v + 3]);
+    }
+  }
 }
 
 cudaError_t launch_neural_prep(int B, int H, int N, int F, int R, int RP, int tf32, const float *Xq, const float *Xk,
                                const float *Wq, const float *Wk, float scale, void *out_q, void *out_k, int *flags,
                                unsigned int *sched, cudaStream_t s) {
-  const size_t smem = size_t(2) * F * R * sizeof(float);
-  if (smem > 48 * 1024) {  // the opt-in above the default, once per device (64 KB covers F R <= 8192)
-    static std::atomic<int> done[64];
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!done[dev].load(std::memory_order_acquire)) {
-      e = cudaFuncSetAttribute(neural_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-      if (e != cudaSuccess) return e;
-      done[dev].store(1, std::memory_order_release);
-    }
+  if (tf32) {
+    const dim3 grid((N + 127) / 128, B * H);
+    neural_prep_tf32_kernel<<<grid, 128, 0, s>>>(H, N, F, R, RP, Xq, Xk, Wq, Wk, 1.0f / scale,
+                                                 static_cast<float *>(out_q), static_cast<float *>(out_k), sched);
+  } else if (RP == 16) {
+    const dim3 grid((N + 63) / 64, B * H, 1);
+    neural_prep_mma_kernel<16><<<grid, 64, 0, s>>>(H, N, F, R, RP, Xq, Xk, Wq, Wk, 1.0f / scale,
+                                                   static_cast<__half *>(out_q), static_cast<__half *>(out_k), flags,
+                                                   sched);
+  } else {
+    const dim3 grid((N + 63) / 64, B * H, RP / 32);
+    neural_prep_mma_kernel<32><<<grid, 128, 0, s>>>(H, N, F, R, RP, Xq, Xk, Wq, Wk, 1.0f / scale,
+                                                    static_cast<__half *>(out_q), static_cast<__half *>(out_k), flags,
+                                                    sched);
   }
-  const dim3 grid((N + 63) / 64, B * H);
-  neural_prep_kernel<<<grid, 256, smem, s>>>(H, N, F, R, RP, tf32, Xq, Xk, Wq, Wk, 1.0f / scale, out_q, out_k,
-                                              flags, sched);
   return cudaGetLastError();
 }
 

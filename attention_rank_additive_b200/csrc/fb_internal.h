@@ -28,6 +28,7 @@ struct FwdArgs {
   int n_kv;          // number of 128-key tiles
   int n_cta_q;       // number of CTA row groups along N
   float scale_log2;  // scale * log2(e)
+  float scale;       // the score scale itself (the dense path adds its bias to scale * QK^T)
   int causal;
   void *O;
   float *LSE;
