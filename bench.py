@@ -56,13 +56,21 @@ def parse_args(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-bias comparison leg")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline leg")
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's B (a smaller case, e.g. to profile)")
+    ap.add_argument("--heads", type=int, default=0, help="override the workload's H (a smaller case, e.g. to profile)")
     ap.add_argument("--no-per-config", action="store_true",
                     help="skip the per-workload leg (fused and dense kernels of workloads 1..4)")
     return ap.parse_args(argv)
 
 
-def workload(cfg_idx: int) -> dict:
+def workload(cfg_idx: int, batch: int = 0, heads: int = 0) -> dict:
+    """The seeded workload cfg_idx, optionally with fewer batches or heads (a
+    smaller case of the same kernel, for profiling); counted FLOPs follow."""
     c = dict(si.CONFIGS[cfg_idx])
+    if batch > 0:
+        c["B"] = batch
+    if heads > 0:
+        c["H"] = heads
     c["flops"] = flops(c["B"], c["H"], c["N"], c["d"], c["R"], c["causal"], c["bias"] == "mulcos")
     if c.get("bwd"):
         c["flops"] = bwd_flops(c["B"], c["H"], c["N"], c["d"], c["R"], c["causal"])
@@ -564,7 +572,7 @@ def run_ours(args, rank: int, world: int, local: int):
     import torch
 
     import attention_rank_additive_b200 as fb
-    c = workload(args.config)
+    c = workload(args.config, args.batch, args.heads)
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     fb.lib()
