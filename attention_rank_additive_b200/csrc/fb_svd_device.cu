@@ -26,6 +26,41 @@ namespace {
 
 constexpr int kMaxL = 32;
 
+// Stage columns c0 .. c0+W-1 of the l rows of a [l][N] fp32 matrix into
+// shared memory (row pitch W), zero outside the matrix. Each of the NT
+// threads owns whole 16-byte pieces and issues all of its loads before its
+// stores, so a chunk costs one memory latency, not one per element. Needs
+// NT * 4 * K == kMaxL * W for some K.
+template <int W, int NT>
+__device__ __forceinline__ void stage_rows(float (*xs)[W], const float *__restrict__ A, int l, int N, long long c0,
+                                           long long c_end) {
+  constexpr int PIECES = kMaxL * W / 4;  // 16-byte pieces of a full kMaxL x W tile
+  constexpr int K = PIECES / NT;
+  static_assert(K * NT == PIECES, "staging split");
+  const bool vec = (N & 3) == 0 && (reinterpret_cast<uintptr_t>(A) & 15u) == 0;
+  float4 v[K];
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    const int piece = k * NT + int(threadIdx.x);
+    const int j = piece / (W / 4), t = (piece - j * (W / 4)) * 4;
+    const long long c = c0 + t;
+    if (j < l && vec && c + 3 < c_end) {
+      v[k] = *reinterpret_cast<const float4 *>(A + (long long)j * N + c);
+    } else {
+      float e[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) e[q] = (j < l && c + q < c_end) ? A[(long long)j * N + c + q] : 0.f;
+      v[k] = make_float4(e[0], e[1], e[2], e[3]);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < K; ++k) {
+    const int piece = k * NT + int(threadIdx.x);
+    const int j = piece / (W / 4), t = (piece - j * (W / 4)) * 4;
+    *reinterpret_cast<float4 *>(&xs[j][t]) = v[k];
+  }
+}
+
 // ------------------------------------------------------------------ kernels
 
 // Counter-based Gaussian: splitmix64 at state seed + c * gamma (Steele, Lea
@@ -49,83 +84,158 @@ __global__ void gauss_kernel(int H, int N, int l, uint64_t seed, float *__restri
   }
 }
 
-// Y[h] = B[h] X[h]: B [N, N] row-major, X and Y [l][N]. One warp per row of
-// B (16 rows per CTA); X is staged in shared memory 256 columns at a time.
-__global__ void __launch_bounds__(512) bx_kernel(int N, int l, const float *__restrict__ B,
+// Y[h] = B[h] X[h]: B [N, N] row-major, X and Y [l][N]. A CTA of 8 warps
+// takes 32 rows of B, each warp 4 of them; X is staged in shared memory 256
+// columns at a time and each lane works on 4 consecutive columns, so one
+// 16-byte shared load of X feeds 16 FMAs (4 rows x 4 columns) and each row's
+// 16-byte loads of B are coalesced across the warp. The per-lane partial
+// sums are reduced across the warp at the end.
+constexpr int kBxRows = 4;  // rows per warp
+__global__ void __launch_bounds__(256) bx_kernel(int N, int l, const float *__restrict__ B,
                                                  const float *__restrict__ X, float *__restrict__ Y) {
-  __shared__ float xs[kMaxL][256];
+  __shared__ __align__(16) float xs[kMaxL][256];
   const int h = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long i = (long long)blockIdx.x * 16 + warp;
+  const long long i0 = (long long)blockIdx.x * (8 * kBxRows) + warp * kBxRows;
   const float *Bh = B + (long long)h * N * N;
   const float *Xh = X + (long long)h * l * N;
-  float acc[kMaxL];
+  // rows of B start on 16-byte boundaries: 16-byte loads
+  const bool vec = (N & 3) == 0 && (reinterpret_cast<uintptr_t>(B) & 15u) == 0;
+  float acc[kBxRows][kMaxL];
 #pragma unroll
-  for (int j = 0; j < kMaxL; ++j) acc[j] = 0.f;
+  for (int r = 0; r < kBxRows; ++r)
+#pragma unroll
+    for (int j = 0; j < kMaxL; ++j) acc[r][j] = 0.f;
   for (int c0 = 0; c0 < N; c0 += 256) {
-    for (int e = threadIdx.x; e < l * 256; e += blockDim.x) {
-      const int j = e / 256, t = e - j * 256;
-      xs[j][t] = c0 + t < N ? Xh[(long long)j * N + c0 + t] : 0.f;
+    // this chunk's B values first (they stream from HBM while X is staged)
+    float bv2[2][kBxRows][4];
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const int t = 128 * m + 4 * lane;  // this lane's 4 columns of the chunk
+#pragma unroll
+      for (int r = 0; r < kBxRows; ++r) {
+        const long long i = i0 + r;
+        const long long c = c0 + t;
+        if (i < N && vec && c + 3 < N) {
+          const float4 b4 = *reinterpret_cast<const float4 *>(Bh + i * N + c);
+          bv2[m][r][0] = b4.x, bv2[m][r][1] = b4.y, bv2[m][r][2] = b4.z, bv2[m][r][3] = b4.w;
+        } else {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) bv2[m][r][q] = (i < N && c + q < N) ? Bh[i * N + c + q] : 0.f;
+        }
+      }
     }
+    stage_rows<256, 256>(xs, Xh, l, N, c0, N);
     __syncthreads();
-    if (i < N) {
 #pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const int t = lane + 32 * m;
-        const float bv = c0 + t < N ? Bh[i * N + c0 + t] : 0.f;
+    for (int m = 0; m < 2; ++m) {
+      const int t = 128 * m + 4 * lane;  // this lane's 4 columns of the chunk
+      const float(&bv)[kBxRows][4] = bv2[m];
 #pragma unroll
-        for (int j = 0; j < kMaxL; ++j)
-          if (j < l) acc[j] = fmaf(bv, xs[j][t], acc[j]);
+      for (int j = 0; j < kMaxL; ++j) {
+        if (j < l) {
+          const float4 x4 = *reinterpret_cast<const float4 *>(&xs[j][t]);
+#pragma unroll
+          for (int r = 0; r < kBxRows; ++r) {
+            float a = acc[r][j];
+            a = fmaf(bv[r][0], x4.x, a);
+            a = fmaf(bv[r][1], x4.y, a);
+            a = fmaf(bv[r][2], x4.z, a);
+            a = fmaf(bv[r][3], x4.w, a);
+            acc[r][j] = a;
+          }
+        }
       }
     }
     __syncthreads();
   }
-  if (i < N) {
+#pragma unroll
+  for (int r = 0; r < kBxRows; ++r) {
+    const long long i = i0 + r;
 #pragma unroll
     for (int j = 0; j < kMaxL; ++j) {
       if (j >= l) break;
-      float v = acc[j];
+      float v = acc[r][j];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0) Y[(long long)h * l * N + (long long)j * N + i] = v;
+      if (lane == 0 && i < N) Y[(long long)h * l * N + (long long)j * N + i] = v;
     }
   }
 }
 
 // Z[h] += B[h]^T X[h] over one slice of 512 rows of B (Z zeroed beforehand):
-// one thread per column of B (128 per CTA), X staged in shared memory 64 rows
-// at a time; grid (column blocks, H, row slices), partial sums added with
-// atomics.
-__global__ void __launch_bounds__(128) btx_kernel(int N, int l, const float *__restrict__ B,
+// each thread takes 4 consecutive columns of B (256 threads, 1024 columns per
+// CTA) and walks the slice 4 rows at a time, X staged in shared memory 64 rows
+// at a time, so that one 16-byte broadcast load of X (4 rows of one column of
+// X) feeds 16 FMAs; grid (column blocks, H, row slices), partial sums added
+// with atomics.
+__global__ void __launch_bounds__(256) btx_kernel(int N, int l, const float *__restrict__ B,
                                                   const float *__restrict__ X, float *__restrict__ Z) {
-  __shared__ float xs[kMaxL][64];
+  __shared__ __align__(16) float xs[kMaxL][64];
   const int h = blockIdx.y;
-  const long long c = (long long)blockIdx.x * 128 + threadIdx.x;
+  const long long c = ((long long)blockIdx.x * 256 + threadIdx.x) * 4;  // first of this thread's 4 columns
   const float *Bh = B + (long long)h * N * N;
   const float *Xh = X + (long long)h * l * N;
-  float acc[kMaxL];
+  const bool vec = (N & 3) == 0 && (reinterpret_cast<uintptr_t>(B) & 15u) == 0;
+  float acc[4][kMaxL];
 #pragma unroll
-  for (int j = 0; j < kMaxL; ++j) acc[j] = 0.f;
+  for (int q = 0; q < 4; ++q)
+#pragma unroll
+    for (int j = 0; j < kMaxL; ++j) acc[q][j] = 0.f;
   const int i_end = min(N, int(blockIdx.z + 1) * 512);
   for (int i0 = int(blockIdx.z) * 512; i0 < i_end; i0 += 64) {
-    for (int e = threadIdx.x; e < l * 64; e += blockDim.x) {
-      const int j = e / 64, r = e - j * 64;
-      xs[j][r] = i0 + r < N ? Xh[(long long)j * N + i0 + r] : 0.f;
-    }
+    stage_rows<64, 256>(xs, Xh, l, N, i0, i_end);
     __syncthreads();
     if (c < N) {
       const int rmax = min(64, i_end - i0);
-      for (int r = 0; r < rmax; ++r) {
-        const float bv = Bh[(long long)(i0 + r) * N + c];
+      // B values of 4 rows x this thread's 4 columns; the next group's are
+      // loaded before the current group's FMAs
+      auto load4 = [&](int r, float (&bv)[4][4]) {
 #pragma unroll
-        for (int j = 0; j < kMaxL; ++j)
-          if (j < l) acc[j] = fmaf(bv, xs[j][r], acc[j]);
+        for (int u = 0; u < 4; ++u) {
+          const long long i = i0 + r + u;
+          if (r + u < rmax && vec && c + 3 < N) {
+            const float4 b4 = *reinterpret_cast<const float4 *>(Bh + i * N + c);
+            bv[u][0] = b4.x, bv[u][1] = b4.y, bv[u][2] = b4.z, bv[u][3] = b4.w;
+          } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) bv[u][q] = (r + u < rmax && c + q < N) ? Bh[i * N + c + q] : 0.f;
+          }
+        }
+      };
+      float nb[4][4];
+      load4(0, nb);
+      for (int r = 0; r < rmax; r += 4) {
+        float bv[4][4];  // [row][column]
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) bv[u][q] = nb[u][q];
+        if (r + 4 < rmax) load4(r + 4, nb);
+#pragma unroll
+        for (int j = 0; j < kMaxL; ++j) {
+          if (j < l) {
+            const float4 x4 = *reinterpret_cast<const float4 *>(&xs[j][r]);  // rows r .. r+3 (zero past the slice)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              float a = acc[q][j];
+              a = fmaf(bv[0][q], x4.x, a);
+              a = fmaf(bv[1][q], x4.y, a);
+              a = fmaf(bv[2][q], x4.z, a);
+              a = fmaf(bv[3][q], x4.w, a);
+              acc[q][j] = a;
+            }
+          }
+        }
       }
     }
     __syncthreads();
   }
-  if (c < N) {
-    for (int j = 0; j < l; ++j) atomicAdd(&Z[(long long)h * l * N + (long long)j * N + c], acc[j]);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+#pragma unroll
+    for (int j = 0; j < kMaxL; ++j)  // compile-time indices keep acc in registers
+      if (j < l && c + q < N) atomicAdd(&Z[(long long)h * l * N + (long long)j * N + c + q], acc[q][j]);
   }
 }
 
@@ -134,7 +244,7 @@ __global__ void __launch_bounds__(128) btx_kernel(int N, int l, const float *__r
 // (row chunks, H); one thread per (a, b) pair with a <= b.
 __global__ void __launch_bounds__(512) gram_kernel(int N, int l, const float *__restrict__ A,
                                                    double *__restrict__ G) {
-  __shared__ float as[kMaxL][256];
+  __shared__ float as[kMaxL][257];  // padded: threads of one warp read different rows at the same t
   const int h = blockIdx.y;
   const long long i0 = (long long)blockIdx.x * 256;
   const float *Ah = A + (long long)h * l * N;
@@ -165,11 +275,12 @@ __global__ void __launch_bounds__(512) gram_kernel(int N, int l, const float *__
 // lane j solves column j of the inverse.
 __global__ void chol_kernel(int H, int N, int l, double shift_coef, const double *__restrict__ G,
                             double *__restrict__ T) {
-  __shared__ double Rm[kMaxL][kMaxL];
+  __shared__ double Rm[kMaxL][kMaxL], Ti[kMaxL][kMaxL], g[kMaxL * kMaxL];
   __shared__ bool dead[kMaxL];
   const int h = blockIdx.x, lane = threadIdx.x;
   if (h >= H) return;
-  const double *g = G + (long long)h * l * l;
+  for (int e = lane; e < l * l; e += 32) g[e] = G[(long long)h * l * l + e];  // the Gram matrix, once
+  __syncwarp();
   double *t = T + (long long)h * l * l;
   double tr = 0.0;
   for (int a = 0; a < l; ++a) tr += g[a * l + a];
@@ -200,13 +311,14 @@ __global__ void chol_kernel(int H, int N, int l, double shift_coef, const double
   if (j < l) {
     for (int i = l - 1; i >= 0; --i) {
       if (i > j || dead[i]) {
-        t[i * l + j] = 0.0;
+        Ti[i][j] = 0.0;
         continue;
       }
       double v = (i == j) ? 1.0 : 0.0;
-      for (int k = i + 1; k <= j; ++k) v -= Rm[i][k] * t[k * l + j];
-      t[i * l + j] = v / Rm[i][i];
+      for (int k = i + 1; k <= j; ++k) v -= Rm[i][k] * Ti[k][j];
+      Ti[i][j] = v / Rm[i][i];
     }
+    for (int i = 0; i < l; ++i) t[i * l + j] = Ti[i][j];
   }
   (void)N;
 }
@@ -214,11 +326,13 @@ __global__ void chol_kernel(int H, int N, int l, double shift_coef, const double
 // Out[h] = A[h] T[h] (A, Out [l][N], T [l][l] fp64); one thread per row.
 __global__ void apply_kernel(int N, int l, const float *__restrict__ A, const double *__restrict__ T,
                              float *__restrict__ Out) {
+  __shared__ double t[kMaxL * kMaxL];
   const int h = blockIdx.y;
+  for (int e = threadIdx.x; e < l * l; e += blockDim.x) t[e] = T[(long long)h * l * l + e];
+  __syncthreads();
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= N) return;
   const float *Ah = A + (long long)h * l * N;
-  const double *t = T + (long long)h * l * l;
   double a[kMaxL];
 #pragma unroll
   for (int k = 0; k < kMaxL; ++k) a[k] = k < l ? double(Ah[(long long)k * N + i]) : 0.0;
@@ -231,61 +345,92 @@ __global__ void apply_kernel(int N, int l, const float *__restrict__ A, const do
   }
 }
 
-// Symmetric eigen-decomposition of M = Z^T Z (fp64 cyclic Jacobi), then the
+// Symmetric eigen-decomposition of M = Z^T Z (fp64 Jacobi), then the
 // coefficient matrices of the balanced factors: Cq = W_R diag(sqrt sigma),
 // Ck = W_R diag(1 / sqrt sigma), sigma^2 the R largest eigenvalues;
-// sig2[h] = sum of those sigma^2. One warp per head: every lane forms the
-// rotation, lane k updates entry k of the two columns, rows and V columns.
+// sig2[h] = sum of those sigma^2. One warp per head, parallel ordering: the
+// matrix is padded to an even size n and each sweep is n - 1 rounds of the
+// round-robin pairing (index 0 fixed, the others rotating), whose n / 2
+// pairs are disjoint, so their rotations commute: all angles are taken from
+// the current matrix, then every column pair is rotated (lane k: row k),
+// then every row pair (lane k: column k), and the eigenvector columns.
 __global__ void eig_kernel(int H, int l, int R, const double *__restrict__ Mg, double *__restrict__ Cq,
                            double *__restrict__ Ck, double *__restrict__ sig2) {
-  __shared__ double A[kMaxL][kMaxL], V[kMaxL][kMaxL];
+  // rows padded by one entry: lane k walking row k of A or V then hits its own bank
+  __shared__ double A[kMaxL][kMaxL + 1], V[kMaxL][kMaxL + 1];
+  __shared__ double cs_s[kMaxL / 2], sn_s[kMaxL / 2];
+  __shared__ int pp_s[kMaxL / 2], qq_s[kMaxL / 2];
   __shared__ int order[kMaxL];
   const int h = blockIdx.x, k = threadIdx.x;
   if (h >= H) return;
-  for (int i = 0; i < l; ++i) {
-    if (k < l) {
-      A[i][k] = Mg[(long long)h * l * l + i * l + k];
+  const int n = (l + 1) & ~1;  // padded size (the pad row and column stay zero)
+  for (int i = 0; i < n; ++i) {
+    if (k < n) {
+      A[i][k] = (i < l && k < l) ? Mg[(long long)h * l * l + i * l + k] : 0.0;
       V[i][k] = i == k ? 1.0 : 0.0;
     }
   }
   __syncwarp();
-  for (int sweep = 0; sweep < 60; ++sweep) {
-    double off = 0.0, diag = 0.0;
-    if (k < l) {
-      diag = A[k][k] * A[k][k];
-      for (int j = k + 1; j < l; ++j) off += A[k][j] * A[k][j];
-    }
+  // A rotation is skipped when |a_pq| is at rounding level next to the
+  // largest diagonal entry (the leading eigenpairs, the only ones used, are
+  // then converged); the iteration stops after a sweep without one.
+  for (int sweep = 0; sweep < 40; ++sweep) {
+    bool rotated = false;
+    double dmax = k < n ? fabs(A[k][k]) : 0.0;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      off += __shfl_xor_sync(0xffffffffu, off, o);
-      diag += __shfl_xor_sync(0xffffffffu, diag, o);
-    }
-    if (off <= 1e-26 * diag || off == 0.0) break;
-    for (int p = 0; p < l - 1; ++p) {
-      for (int q = p + 1; q < l; ++q) {
+    for (int o = 16; o > 0; o >>= 1) dmax = fmax(dmax, __shfl_xor_sync(0xffffffffu, dmax, o));
+    const double tol = 1e-15 * dmax;
+    for (int round = 0; round < n - 1; ++round) {
+      // pair m of this round: positions m and n-1-m of the sequence
+      // [0, (round + 0) .. (round + n - 2) mod (n - 1) + 1]
+      if (k < n / 2) {
+        auto member = [&](int pos) { return pos == 0 ? 0 : ((pos - 1 + round) % (n - 1)) + 1; };
+        int p = member(k), q = member(n - 1 - k);
+        if (p > q) {
+          const int t = p;
+          p = q;
+          q = t;
+        }
         const double apq = A[p][q];
-        if (fabs(apq) < 1e-300) continue;
-        const double theta = (A[q][q] - A[p][p]) / (2.0 * apq);
-        const double tt = (theta >= 0 ? 1.0 : -1.0) / (fabs(theta) + sqrt(theta * theta + 1.0));
-        const double cs = 1.0 / sqrt(tt * tt + 1.0), sn = tt * cs;
-        __syncwarp();
-        if (k < l) {  // columns p, q
-          const double akp = A[k][p], akq = A[k][q];
-          A[k][p] = cs * akp - sn * akq;
-          A[k][q] = sn * akp + cs * akq;
+        double c = 1.0, sn = 0.0;
+        if (fabs(apq) >= 1e-300 && fabs(apq) > tol) {
+          rotated = true;
+          const double theta = (A[q][q] - A[p][p]) / (2.0 * apq);
+          const double tt = (theta >= 0 ? 1.0 : -1.0) / (fabs(theta) + sqrt(theta * theta + 1.0));
+          c = 1.0 / sqrt(tt * tt + 1.0);
+          sn = tt * c;
         }
-        __syncwarp();
-        if (k < l) {  // rows p, q
-          const double apk = A[p][k], aqk = A[q][k];
-          A[p][k] = cs * apk - sn * aqk;
-          A[q][k] = sn * apk + cs * aqk;
-          const double vkp = V[k][p], vkq = V[k][q];
-          V[k][p] = cs * vkp - sn * vkq;
-          V[k][q] = sn * vkp + cs * vkq;
-        }
-        __syncwarp();
+        pp_s[k] = p;
+        qq_s[k] = q;
+        cs_s[k] = c;
+        sn_s[k] = sn;
       }
+      __syncwarp();
+      if (k < n) {  // columns p, q of row k; eigenvector columns of row k
+        for (int m = 0; m < n / 2; ++m) {
+          const int p = pp_s[m], q = qq_s[m];
+          const double c = cs_s[m], sn = sn_s[m];
+          const double akp = A[k][p], akq = A[k][q];
+          A[k][p] = c * akp - sn * akq;
+          A[k][q] = sn * akp + c * akq;
+          const double vkp = V[k][p], vkq = V[k][q];
+          V[k][p] = c * vkp - sn * vkq;
+          V[k][q] = sn * vkp + c * vkq;
+        }
+      }
+      __syncwarp();
+      if (k < n) {  // rows p, q of column k
+        for (int m = 0; m < n / 2; ++m) {
+          const int p = pp_s[m], q = qq_s[m];
+          const double c = cs_s[m], sn = sn_s[m];
+          const double apk = A[p][k], aqk = A[q][k];
+          A[p][k] = c * apk - sn * aqk;
+          A[q][k] = sn * apk + c * aqk;
+        }
+      }
+      __syncwarp();
     }
+    if (!__any_sync(0xffffffffu, rotated)) break;
   }
   // the R largest eigenvalues, in decreasing order (lane 0 picks them)
   if (k == 0) {
@@ -454,7 +599,8 @@ extern "C" int fb_svd_factors_device(int H, int N, int R, int oversample, int po
   double *sums = sig2 + H;
   double *out = sums + 2 * H;
 
-  const dim3 rows16((N + 15) / 16, H), cols128((N + 127) / 128, H, (N + 511) / 512), rows256((N + 255) / 256, H);
+  const dim3 rows16((N + 15) / 16, H), rows32((N + 31) / 32, H), cols1024((N + 1023) / 1024, H, (N + 511) / 512),
+      rows256((N + 255) / 256, H);
   const double u = 1.1102230246251565e-16;  // 2^-53: unit roundoff of the fp64 Gram matrices
   const double shift_coef = 11.0 * (double(N) * l + double(l) * (l + 1)) * u;
   const int hb = (H + 31) / 32;
@@ -477,17 +623,17 @@ extern "C" int fb_svd_factors_device(int H, int N, int R, int oversample, int po
   };
   const long long ng = (long long)H * l * N;
   gauss_kernel<<<int(std::min<long long>((ng + 255) / 256, 148 * 16)), 256, 0, st>>>(H, N, l, seed, P1);
-  bx_kernel<<<rows16, 512, 0, st>>>(N, l, bias, P1, P0);  // Y = B Omega
+  bx_kernel<<<rows32, 256, 0, st>>>(N, l, bias, P1, P0);  // Y = B Omega
   orth(P0, P1, P2);                                         // Q in P2
   for (int it = 0; it < power_iters; ++it) {
     cudaMemsetAsync(P0, 0, size_t(H) * l * N * sizeof(float), st);
-    btx_kernel<<<cols128, 128, 0, st>>>(N, l, bias, P2, P0);  // Z = B^T Q
+    btx_kernel<<<cols1024, 256, 0, st>>>(N, l, bias, P2, P0);  // Z = B^T Q
     orth(P0, P2, P1);                                         // Z orthonormal in P1
-    bx_kernel<<<rows16, 512, 0, st>>>(N, l, bias, P1, P0);   // Y = B Z
+    bx_kernel<<<rows32, 256, 0, st>>>(N, l, bias, P1, P0);   // Y = B Z
     orth(P0, P1, P2);                                         // Q in P2
   }
   cudaMemsetAsync(P0, 0, size_t(H) * l * N * sizeof(float), st);
-  btx_kernel<<<cols128, 128, 0, st>>>(N, l, bias, P2, P0);  // M = B^T Q
+  btx_kernel<<<cols1024, 256, 0, st>>>(N, l, bias, P2, P0);  // M = B^T Q
   gram(P0);                                                 // M^T M
   eig_kernel<<<H, 32, 0, st>>>(H, l, R, G, Cq, Ck, sig2);
   rows_kernel<<<rows256, 256, 0, st>>>(N, l, R, P2, Cq, phi_q);
