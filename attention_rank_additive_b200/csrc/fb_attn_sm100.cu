@@ -426,6 +426,10 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
   tc_fence_after();
   const uint32_t tmem = ctrl->tmem_base;
   volatile int *abort = &ctrl->abort;
+  // The set-up above touches no global memory; what the previous kernel in
+  // the stream writes (the prepared factors, the work counter) is read only
+  // after it has completed.
+  griddep_wait();
 
   // Barrier phases run on per-role counters that continue across work items:
   // g counts key steps (K/V ring), it counts items (Q, O), L_t counts the
@@ -1316,7 +1320,21 @@ static cudaError_t launch_one(const FwdMaps &m, const FwdArgs &a, cudaStream_t s
     // walking its share of the work items.
     const long long items = (long long)a.n_cta_q * a.B * a.H;
     const long long ctas = std::min<long long>(items, cap);
-    kern<<<dim3(unsigned(ctas)), C::THREADS, C::SMEM, stream>>>(m.q, m.k, m.v, m.fq, m.fk, m.bias, m.o, a);
+    // Programmatic stream serialization: the CTAs may start their set-up
+    // while the preparation kernel before them finishes (they wait for it
+    // before reading anything it writes).
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(ctas));
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, m.q, m.k, m.v, m.fq, m.fk, m.bias, m.o, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
 }

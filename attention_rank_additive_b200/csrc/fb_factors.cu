@@ -59,6 +59,7 @@ __global__ void prep_mma_kernel(int N, int R, int RP, int fac_H, const float *__
                                 unsigned int *sched) {
   if (sched != nullptr && blockIdx.x == 0 && threadIdx.x == 0) sched[0] = sched[1] = 0u;  // the work counter
   bool overflow = false;
+  griddep_launch_dependents();  // the fused kernel may start its set-up now
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
        idx += (long long)gridDim.x * blockDim.x) {
     const int r = int(idx % RP);
@@ -96,6 +97,7 @@ __global__ void prep_tf32_kernel(int N, int R, int KT, int fac_H, const float *_
                                  float *__restrict__ oq, float *__restrict__ ok, long long total,
                                  unsigned int *sched) {
   if (sched != nullptr && blockIdx.x == 0 && threadIdx.x == 0) sched[0] = sched[1] = 0u;  // the work counter
+  griddep_launch_dependents();  // the fused kernel may start its set-up now
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
        idx += (long long)gridDim.x * blockDim.x) {
     const long long n = idx % N;
@@ -142,6 +144,7 @@ __global__ void prep_mul_bias_kernel(int H, int N, int d, int R, int RP, const _
                                      __half *__restrict__ fq, __half *__restrict__ fk, int *flags, int width,
                                      long long total, unsigned int *sched) {
   if (sched != nullptr && blockIdx.x == 0 && threadIdx.x == 0) sched[0] = sched[1] = 0u;  // the work counter
+  griddep_launch_dependents();  // the fused kernel may start its set-up now
   bool overflow = false;
   const int used = d * (R - 1);
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
@@ -260,6 +263,7 @@ __global__ void __launch_bounds__(64 * TW / 16) neural_prep_mma_kernel(
   __shared__ __align__(16) float ws[2][FC][TW];   // [side][f][col]
   if (sched != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0)
     sched[0] = sched[1] = 0u;
+  griddep_launch_dependents();  // the fused kernel may start its set-up now
   const int bh = blockIdx.y, b = bh / H, h = bh - (bh / H) * H;
   const long long n0 = (long long)blockIdx.x * 64;
   const int c0 = blockIdx.z * TW;
@@ -343,6 +347,7 @@ __global__ void __launch_bounds__(128) neural_prep_tf32_kernel(int H, int N, int
                                                                float *__restrict__ oq, float *__restrict__ ok,
                                                                unsigned int *sched) {
   if (sched != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) sched[0] = sched[1] = 0u;
+  griddep_launch_dependents();  // the fused kernel may start its set-up now
   const int bh = blockIdx.y, b = bh / H, h = bh - (bh / H) * H;
   const long long n = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (n >= N) return;
