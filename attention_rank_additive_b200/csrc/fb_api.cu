@@ -583,7 +583,9 @@ int fb_factors_alibi(int H, int N, float *phi_q, float *phi_k, void *stream) {
 namespace {
 struct BwdLayout {
   WsLayout f;  // the S-side factor tiles (as the forward's workspace)
-  size_t gq_off, gk_off, l_off, d_off, pq_off, pk_off, total;
+  // acc_off: the fused kernel's fp32 dq' accumulator [BH, Npad, up to 128]; the
+  // two-kernel path keeps its per-head dphi_q rows there instead (pq_off).
+  size_t gq_off, gk_off, l_off, d_off, acc_off, pq_off, pk_off, total;
   int RG, Npad;
   bool shared_slices;  // some factor slice serves several heads: per-head partial gradients
 };
@@ -602,8 +604,10 @@ BwdLayout bwd_layout(int B, int H, int N, int R, int64_t bs, int64_t hs) {
   w.d_off = w.l_off + rows;
   w.shared_slices = R > 0 && fb < size_t(B) * H;
   const size_t part = w.shared_slices ? al256(size_t(B) * H * size_t(N) * size_t(R) * 4) : 0;
-  w.pq_off = w.d_off + rows;
-  w.pk_off = w.pq_off + part;
+  const size_t acc = al256(size_t(B) * H * size_t(w.Npad) * 128 * 4);  // >= part (R <= 128, N <= Npad)
+  w.acc_off = w.d_off + rows;
+  w.pq_off = w.acc_off;
+  w.pk_off = w.acc_off + acc;
   w.total = w.pk_off + part;
   return w;
 }
@@ -692,7 +696,18 @@ int fb_attn_bwd(int dt, int B, int H, int N, int d, const void *Q, const void *K
         !encode_fac(&maps.fk_blk, plan.mode, wk, FB, N, plan.RP, BK))
       return FB_ERR_CUDA;
     if (want_dphi && (!encode_rows_bf16(&maps.gq_blk, wsb + L.gq_off, FB, N, L.RG, L.RG, BQ) ||
-                      !encode_rows_bf16(&maps.gk_blk, wsb + L.gk_off, FB, N, L.RG, L.RG, BK)))
+                      !encode_rows_bf16(&maps.gk_blk, wsb + L.gk_off, FB, N, L.RG, L.RG, BK) ||
+                      !encode_rows_bf16(&maps.gk, wsb + L.gk_off, FB, N, L.RG, L.RG, 128)))
+      return FB_ERR_CUDA;
+  }
+  const bool fused = bwd_fused(plan);
+  const int dqw = 64 + plan.RG;  // fused: accumulator columns (dQ | dphi_q)
+  float *acc = reinterpret_cast<float *>(wsb + L.acc_off);
+  if (fused) {
+    const uint64_t dims[3] = {uint64_t(dqw), uint64_t(L.Npad), uint64_t(BH)};
+    const uint64_t strides[2] = {uint64_t(dqw) * 4, uint64_t(L.Npad) * dqw * 4};
+    const uint32_t box[3] = {uint32_t(dqw), dqw == 128 ? 16u : 32u, 1u};  // the kernel's staging pieces
+    if (!encode(&maps.acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, acc, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE))
       return FB_ERR_CUDA;
   }
 
@@ -707,9 +722,11 @@ int fb_attn_bwd(int dt, int B, int H, int N, int d, const void *Q, const void *K
       return FB_ERR_CUDA;
   }
   // 3. per-row -LSE in log2 units and rowsum(dO * O)
-  if (launch_bwd_rows(BH, N, L.Npad, d, O, dO, LSE, nlse2, delta, st) != cudaSuccess) return FB_ERR_CUDA;
+  //    (and, fused, the zeroed accumulator)
+  if (launch_bwd_rows(BH, N, L.Npad, d, O, dO, LSE, nlse2, delta, fused ? acc : nullptr, dqw, st) != cudaSuccess)
+    return FB_ERR_CUDA;
 
-  // 4. the two gradient kernels
+  // 4. the gradient kernels: the fused kernel, or the dK/dV and dQ kernels
   BwdArgs a;
   std::memset(&a, 0, sizeof(a));
   a.B = B, a.H = H, a.N = N, a.d = d, a.R = R;
@@ -728,13 +745,23 @@ int fb_attn_bwd(int dt, int B, int H, int N, int d, const void *Q, const void *K
   a.dphi_k_part = L.shared_slices ? reinterpret_cast<float *>(wsb + L.pk_off) : nullptr;
   a.phi_bs = phi_bstride, a.phi_hs = phi_hstride;
   a.fac_B = fac_B, a.fac_H = fac_H;
+  a.dqacc = fused ? acc : nullptr;
   a.flags = flags;
   if (bwd_launch(plan, maps, a, st) != cudaSuccess) return FB_ERR_CUDA;
-  // 5. factor slices shared by several heads: sum the per-head rows
-  if (want_dphi && L.shared_slices &&
-      launch_reduce_factor_grads(B, H, N, R, fac_B, fac_H, phi_bstride, phi_hstride, a.dphi_q_part, a.dphi_k_part,
-                                 dphi_q, dphi_k, st) != cudaSuccess)
+  // 5. fused: dQ (and per-head dphi_q) from the accumulator
+  if (fused && launch_bwd_dq_convert(B, H, N, L.Npad, d, want_dphi ? R : 0, dqw, scale, acc, dQ,
+                                     want_dphi && !L.shared_slices ? dphi_q : nullptr, phi_bstride, phi_hstride,
+                                     fac_B, fac_H, st) != cudaSuccess)
     return FB_ERR_CUDA;
+  // 6. factor slices shared by several heads: sum the per-head rows
+  if (want_dphi && L.shared_slices) {
+    const cudaError_t e =
+        fused ? launch_reduce_factor_grads(B, H, N, R, fac_B, fac_H, phi_bstride, phi_hstride, acc,
+                                           int64_t(L.Npad) * dqw, dqw, 64, a.dphi_k_part, dphi_q, dphi_k, st)
+              : launch_reduce_factor_grads(B, H, N, R, fac_B, fac_H, phi_bstride, phi_hstride, a.dphi_q_part,
+                                           int64_t(N) * R, R, 0, a.dphi_k_part, dphi_q, dphi_k, st);
+    if (e != cudaSuccess) return FB_ERR_CUDA;
+  }
   return FB_OK;
 }
 

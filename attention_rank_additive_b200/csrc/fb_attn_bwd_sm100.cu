@@ -781,14 +781,495 @@ __global__ void __launch_bounds__(320, 1)
 }
 
 
+// ------------------------------------------ fused: dK, dV, dphi_k and dQ, dphi_q
+// At head dim 64 with gradient factor width 0 or 64, one kernel does the
+// whole backward of a 128-key tile: besides dV, dK and dphi_k (as above),
+// each query block contributes dq' = dS [K | phi_k] for its BQ queries. The
+// compute warps also write dS^T (bf16) to shared memory, one MMA computes
+// dq'^T = [K | phi_k]^T dS^T into TMEM (128 lanes: the concatenated columns;
+// BQ TMEM columns: the queries), and a fourth warpgroup reads it out and adds
+// it into an fp32 accumulator [BH, Npad, 64 + RG] with TMA reduce-adds
+// (performed at L2). The per-row pass zeroes the accumulator beforehand; a
+// conversion pass turns it into dQ (bf16, times the scale) and dphi_q. This
+// replaces the dQ kernel and with it the second evaluation of S, dP and
+// the exponentials.
+template <int RP, int MODE, int RG>
+struct FusedCfg {
+  using B = BwdCfg<64, RP, MODE, RG>;
+  static_assert(RG == 0 || RG == 64, "fused backward: gradient factor width 0 or 64");
+  static constexpr int BQ = 64;
+  static constexpr int DQW = 64 + RG;                // accumulator columns (dQ | dphi_q)
+  static constexpr uint32_t TILE = 128u * 64u * 2u;  // one 128-row x 64-column bf16 tile
+  static constexpr uint32_t align1k(uint32_t x) { return (x + 1023u) & ~1023u; }
+  // fixed tiles: K, then phi_k (bf16, RG = 64), V, phi_k' (S side). [K | phi_k]
+  // read as one MN-major A operand of 128 rows: its second 64-row chunk is the
+  // tile after K (phi_k, or V when RG = 0, whose products are not read).
+  static constexpr uint32_t O_K = 0, O_GK = TILE, O_V = O_GK + (RG ? TILE : 0u), O_FK = O_V + TILE;
+  static constexpr uint32_t FIXED = O_FK + (B::FAC ? 128u * RP * B::FESZ : 0u);
+  static constexpr uint32_t O_DS = align1k(FIXED);    // dS^T [128 keys][64 queries] bf16, one per warpgroup
+  // dq' leaves in pieces of QR queries through two staging tiles [QR][DQW]
+  // fp32 (8 KB each), so that one is written while the other is being read
+  // by its TMA reduce.
+  static constexpr int QR = DQW == 128 ? 16 : 32;
+  static constexpr uint32_t O_DQS = O_DS + 2 * TILE;
+  static constexpr uint32_t DQS_ONE = uint32_t(QR) * DQW * 4u, DQS = 2 * DQS_ONE;
+  static constexpr uint32_t O_ST = align1k(O_DQS + DQS);
+  static constexpr uint32_t STAGE_BYTES = B::KV_STAGE_BYTES, STAGE = B::KV_STAGE;
+  static constexpr uint32_t CTRL = 1024, SLACK = 1024;
+  static constexpr int KS_FIT = kSmemLimitB > O_ST + CTRL + SLACK ? int((kSmemLimitB - O_ST - CTRL - SLACK) / STAGE) : 0;
+  static constexpr int KS = KS_FIT > 4 ? 4 : KS_FIT;
+  static constexpr uint32_t SMEM = O_ST + uint32_t(KS) * STAGE + CTRL + SLACK;
+  // warpgroups: 0, 1 compute; 2 the producer warp (8), the MMA warp (9), the
+  // warp issuing the dq' MMAs (10: its waits for the readout then hold up
+  // nothing else) and an idle warp; 3 the dq' readout. Registers move to the
+  // compute warpgroups (shares chosen so that no role spills).
+  static constexpr int THREADS = 512;
+  static constexpr int PRODUCER_WARP = 8, MMA_WARP = 9, DQ_MMA_WARP = 10, DQ_WARP0 = 12;
+  static constexpr uint32_t LAUNCH_REGS = 128, REG_COMPUTE = 176, REG_OTHER = 72, REG_DQ = 88;
+  static_assert(2 * 128 * REG_COMPUTE + 128 * REG_OTHER + 128 * REG_DQ == THREADS * LAUNCH_REGS, "register split");
+  // TMEM columns: buffer t (S^T at t 2BQ, dP^T at t 2BQ + BQ), dV, dK, dphi_k,
+  // then dq'^T, twice where the columns allow (the MMA of block u then waits
+  // for the readout of block u - 2 instead of u - 1)
+  static constexpr uint32_t C_DV = 4 * BQ, C_DK = C_DV + 64, C_DF = C_DK + 64, C_DQ = C_DF + RG;
+  static constexpr int NDQ = C_DQ + 2 * BQ <= 512 ? 2 : 1;
+  static_assert(C_DQ + NDQ * BQ <= 512, "fused TMEM layout");
+  static constexpr uint32_t IDESC_DQ = make_idesc_bf16_mn(128, BQ);
+};
+
+struct FusedCtrl {
+  uint64_t fixed_full;
+  uint64_t full[4], empty[4];
+  uint64_t s_full[2], p_full[2];
+  uint64_t ds_free[2];             // the dq' MMA has read warpgroup t's dS^T tile
+  uint64_t dq_full[2], dq_free[2];  // dq'^T buffer b in TMEM: written by the MMA / read by the readout
+  uint64_t acc_done;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(FusedCtrl) <= 1024, "control block too large");
+
+template <int RP, int MODE, int RG>
+__global__ void __launch_bounds__(512, 1)
+    attn_bwd_fused_sm100(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                         const __grid_constant__ CUtensorMap tm_fk, const __grid_constant__ CUtensorMap tm_gk,
+                         const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                         const __grid_constant__ CUtensorMap tm_fq, const __grid_constant__ CUtensorMap tm_gq,
+                         const __grid_constant__ CUtensorMap tm_acc, const BwdArgs args) {
+  using F = FusedCfg<RP, MODE, RG>;
+  using C = typename F::B;
+  constexpr int KS = F::KS;
+  constexpr int BQ = F::BQ;
+  constexpr int DP = 64;
+  static_assert(KS >= 3, "configuration does not fit in shared memory");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sK = smem + F::O_K, *sGK = smem + F::O_GK, *sV = smem + F::O_V, *sFK = smem + F::O_FK;
+  uint8_t *sDS = smem + F::O_DS;
+  float *sDQ = reinterpret_cast<float *>(smem + F::O_DQS);
+  uint8_t *sStage = smem + F::O_ST;
+  FusedCtrl *ctrl = reinterpret_cast<FusedCtrl *>(sStage + KS * F::STAGE);
+  constexpr uint32_t O_Q = 0, O_DO = BQ * DP * 2, O_FQ = 2 * BQ * DP * 2;
+  constexpr uint32_t O_GQ = O_FQ + (C::FAC ? BQ * RP * C::FESZ : 0);
+  constexpr uint32_t O_L = O_GQ + BQ * RG * 2, O_D = O_L + BQ * 4;
+  static_assert(O_D + BQ * 4 == F::STAGE_BYTES, "stage layout");
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int BH = args.B * args.H;
+  const int kb = int(blockIdx.x) / BH;  // key tile; the heaviest causal tiles come first
+  const int bh = int(blockIdx.x) % BH;
+  const int b = bh / args.H, h = bh % args.H;
+  const int k0 = kb * 128;
+  const int fslice = (args.fac_B > 1 ? b : 0) * args.fac_H + (args.fac_H > 1 ? h : 0);
+  const int j0 = args.causal ? k0 / BQ : 0;
+  const int nb = (args.N + BQ - 1) / BQ - j0;  // >= 1
+
+  if (threadIdx.x == 0) {
+    mbar_init(&ctrl->fixed_full, 1);
+    for (int s = 0; s < KS; ++s) {
+      mbar_init(&ctrl->full[s], 1);
+      mbar_init(&ctrl->empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&ctrl->s_full[t], 1);
+      mbar_init(&ctrl->p_full[t], 128);
+      mbar_init(&ctrl->ds_free[t], 1);
+    }
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(&ctrl->dq_full[q], 1);
+      mbar_init(&ctrl->dq_free[q], 128);
+    }
+    mbar_init(&ctrl->acc_done, 1);
+    ctrl->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == F::MMA_WARP) {
+    tmem_alloc(&ctrl->tmem_base, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctrl->tmem_base;
+  volatile int *abort = &ctrl->abort;
+  const uint32_t leader = lane == 0 ? 1u : 0u;
+
+  if (warp >= F::PRODUCER_WARP && warp < F::DQ_WARP0) {
+    setmaxnreg_dec<F::REG_OTHER>();
+    if (warp == F::PRODUCER_WARP) {
+      // ---------------------------------------------------------- producer
+      if (leader) {
+        tma_prefetch_map(&tm_k);
+        tma_prefetch_map(&tm_v);
+        tma_prefetch_map(&tm_q);
+        tma_prefetch_map(&tm_do);
+        if (C::FAC) {
+          tma_prefetch_map(&tm_fk);
+          tma_prefetch_map(&tm_fq);
+        }
+        if (RG > 0) {
+          tma_prefetch_map(&tm_gk);
+          tma_prefetch_map(&tm_gq);
+        }
+      }
+      mbar_arrive_expect_tx_leader(&ctrl->fixed_full, F::FIXED, leader);
+      tma_load_3d_leader(sK, &tm_k, &ctrl->fixed_full, 0, k0, bh, leader);
+      tma_load_3d_leader(sV, &tm_v, &ctrl->fixed_full, 0, k0, bh, leader);
+      if (RG > 0) tma_load_3d_leader(sGK, &tm_gk, &ctrl->fixed_full, 0, k0, fslice, leader);
+      if (C::FAC)
+        for (int ch = 0; ch < C::NFCH; ++ch)
+          tma_load_3d_leader(sFK + ch * (128 * C::FCH * 2), &tm_fk, &ctrl->fixed_full, ch * C::FCH, k0, fslice,
+                             leader);
+      bool ok = true;
+      for (int u = 0; u < nb; ++u) {
+        const int s = u % KS;
+        if (u >= KS && !(ok = mbar_wait(&ctrl->empty[s], (uint32_t(u / KS) & 1u) ^ 1u, abort))) break;
+        uint8_t *st = sStage + s * F::STAGE;
+        const int q0 = (j0 + u) * BQ;
+        mbar_arrive_expect_tx_leader(&ctrl->full[s], F::STAGE_BYTES, leader);
+        tma_load_3d_leader(st + O_Q, &tm_q, &ctrl->full[s], 0, q0, bh, leader);
+        tma_load_3d_leader(st + O_DO, &tm_do, &ctrl->full[s], 0, q0, bh, leader);
+        if (C::FAC)
+          for (int ch = 0; ch < C::NFCH; ++ch)
+            tma_load_3d_leader(st + O_FQ + ch * (BQ * C::FCH * 2), &tm_fq, &ctrl->full[s], ch * C::FCH, q0, fslice,
+                               leader);
+        if (RG > 0) tma_load_3d_leader(st + O_GQ, &tm_gq, &ctrl->full[s], 0, q0, fslice, leader);
+        const size_t roff = size_t(bh) * args.Npad + q0;
+        bulk_load_leader(st + O_L, args.nlse2 + roff, BQ * 4, &ctrl->full[s], leader);
+        bulk_load_leader(st + O_D, args.delta + roff, BQ * 4, &ctrl->full[s], leader);
+      }
+      if (!ok) {
+        mbar_wait_for(&ctrl->fixed_full, 0, 100000000ull);
+        for (int s = 0; s < KS; ++s) {
+          mbar_wait_for(&ctrl->full[s], 0, 100000000ull);
+          mbar_wait_for(&ctrl->full[s], 1, 100000000ull);
+        }
+        if (leader) atomicOr(args.flags, kFlagTimeout);
+      }
+    } else if (warp == F::MMA_WARP) {
+      // -------------------------------------------------------- MMA issuer
+      // S(0), S(1), then per block u: G(u), S(u + 2), where G(u) is the
+      // key-side gradient products (from TMEM P^T, dS^T).
+      const uint32_t tm_u = __shfl_sync(0xffffffffu, tmem, 0);
+      bool ok = __all_sync(0xffffffffu, mbar_wait(&ctrl->fixed_full, 0, abort));
+      tc_fence_after();
+      const uint64_t dK = kdesc<64>(smem_u32(sK));
+      const uint64_t dV = kdesc<64>(smem_u32(sV));
+      const uint64_t dFK = kdesc<C::FCH>(smem_u32(sFK));
+      auto issue_s = [&](int u) -> bool {
+        const int s = u % KS;
+        if (!__all_sync(0xffffffffu, mbar_wait(&ctrl->full[s], uint32_t(u / KS) & 1u, abort))) return false;
+        tc_fence_after();
+        const uint32_t st = smem_u32(sStage + s * F::STAGE);
+        const uint32_t s_col = tm_u + uint32_t((u & 1) * 2 * BQ);
+        uint64_t dq = kdesc<64>(st + O_Q), ddo = kdesc<64>(st + O_DO);
+        asm volatile("" : "+l"(dq), "+l"(ddo));
+#pragma unroll
+        for (int kk = 0; kk < DP / 16; ++kk)  // S^T = K Q^T
+          mma_ss_elect(s_col, dK + kstep<64, 128>(kk), dq + kstep<64, BQ>(kk), C::IDESC_KV_S, kk > 0 ? 1u : 0u);
+        if constexpr (C::FAC) {  // S^T += phi_k' phi_q'^T
+          uint64_t dfq = kdesc<C::FCH>(st + O_FQ);
+          asm volatile("" : "+l"(dfq));
+#pragma unroll
+          for (int kk = 0; kk < C::FCH * C::NFCH / 16; ++kk) {
+            if (MODE == kBiasTf32)
+              mma_ss_elect_tf32(s_col, dFK + kstep<C::FCH, 128>(kk), dfq + kstep<C::FCH, BQ>(kk), C::IDESC_KV_F, 1u);
+            else
+              mma_ss_elect(s_col, dFK + kstep<C::FCH, 128>(kk), dfq + kstep<C::FCH, BQ>(kk), C::IDESC_KV_F, 1u);
+          }
+        }
+#pragma unroll
+        for (int kk = 0; kk < DP / 16; ++kk)  // dP^T = V dO^T
+          mma_ss_elect(s_col + BQ, dV + kstep<64, 128>(kk), ddo + kstep<64, BQ>(kk), C::IDESC_KV_S, kk > 0 ? 1u : 0u);
+        tc_commit_elect(&ctrl->s_full[u & 1]);
+        __syncwarp();
+        return true;
+      };
+      auto issue_g = [&](int u) -> bool {
+        if (!__all_sync(0xffffffffu, mbar_wait(&ctrl->p_full[u & 1], uint32_t(u >> 1) & 1u, abort))) return false;
+        tc_fence_after();
+        const int s = u % KS;
+        const uint32_t st = smem_u32(sStage + s * F::STAGE);
+        const uint32_t p_col = tm_u + uint32_t((u & 1) * 2 * BQ);  // P^T bf16 over S^T; dS^T over dP^T
+        uint64_t bdo = mndesc<64, BQ>(st + O_DO), bq = mndesc<64, BQ>(st + O_Q);
+        asm volatile("" : "+l"(bdo), "+l"(bq));
+#pragma unroll
+        for (int kk = 0; kk < BQ / 16; ++kk) {
+          const uint32_t acc = (u > 0 || kk > 0) ? 1u : 0u;
+          mma_ts_elect(tm_u + F::C_DV, p_col + uint32_t(kk * 8), bdo + mnstep<64>(kk), C::IDESC_GD, acc);
+          mma_ts_elect(tm_u + F::C_DK, p_col + BQ + uint32_t(kk * 8), bq + mnstep<64>(kk), C::IDESC_GD, acc);
+        }
+        if constexpr (RG > 0) {
+          uint64_t bg = mndesc<64, BQ>(st + O_GQ);
+          asm volatile("" : "+l"(bg));
+#pragma unroll
+          for (int kk = 0; kk < BQ / 16; ++kk)
+            mma_ts_elect(tm_u + F::C_DF, p_col + BQ + uint32_t(kk * 8), bg + mnstep<64>(kk), C::IDESC_GR,
+                         (u > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit_elect(&ctrl->empty[s]);
+        __syncwarp();
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      if (ok && nb > 1) ok = issue_s(1);
+      for (int u = 0; u < nb && ok; ++u) {
+        ok = issue_g(u);
+        if (ok && u + 2 < nb) ok = issue_s(u + 2);
+      }
+      if (ok) {
+        tc_commit_elect(&ctrl->acc_done);
+        __syncwarp();
+      }
+      if (!ok && leader) atomicOr(args.flags, kFlagTimeout);
+    } else if (warp == F::DQ_MMA_WARP) {
+      // ------------------------------------------------ dq' MMA issuer
+      // Q(u): dq'^T = [K | phi_k]^T dS^T over the 128 keys, into TMEM buffer
+      // u mod NDQ once the readout has emptied it, as soon as block u's
+      // dS^T is in shared memory.
+      const uint32_t tm_u = __shfl_sync(0xffffffffu, tmem, 0);
+      bool ok = __all_sync(0xffffffffu, mbar_wait(&ctrl->fixed_full, 0, abort));
+      const uint64_t aKT = mndesc<64, 128>(smem_u32(sK));  // [K | phi_k]^T, 128 rows
+      for (int u = 0; u < nb && ok; ++u) {
+        const int bq = u % F::NDQ;
+        ok = __all_sync(0xffffffffu, mbar_wait(&ctrl->p_full[u & 1], uint32_t(u >> 1) & 1u, abort) &&
+                                         (u < F::NDQ || mbar_wait(&ctrl->dq_free[bq],
+                                                                  uint32_t(u / F::NDQ - 1) & 1u, abort)));
+        if (!ok) break;
+        tc_fence_after();
+        uint64_t bds = mndesc<64, 128>(smem_u32(sDS + (u & 1) * F::TILE));
+        asm volatile("" : "+l"(bds));
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          mma_ss_elect(tm_u + F::C_DQ + uint32_t(bq * BQ), aKT + mnstep<64>(kk), bds + mnstep<64>(kk), F::IDESC_DQ,
+                       kk > 0 ? 1u : 0u);
+        tc_commit_elect(&ctrl->dq_full[bq]);
+        tc_commit_elect(&ctrl->ds_free[u & 1]);
+        __syncwarp();
+      }
+      if (!ok && leader) atomicOr(args.flags, kFlagTimeout);
+    }
+  } else if (warp >= F::DQ_WARP0) {
+    setmaxnreg_dec<F::REG_DQ>();
+    // ------------------------------------------------------ dq' readout
+    // Each thread holds one accumulator column (TMEM lane) for the block's
+    // queries and hands TMEM back at once; the block leaves in pieces of QR
+    // queries through the two staging tiles, one thread adding each piece
+    // into the accumulator with a TMA reduce.
+    const int qw = warp & 3;
+    const int col = qw * 32 + lane;
+    const uint32_t lane_base = tmem + (uint32_t(qw * 32) << 16);
+    const bool has_col = col < F::DQW;
+    const bool issuer = warp == F::DQ_WARP0 && lane == 0;
+    constexpr int QR = F::QR;
+    bool ok = true;
+    int pc = 0;  // pieces issued
+    for (int u = 0; u < nb; ++u) {
+      const int bq = u % F::NDQ;
+      ok = named_bar_and(2, 128, mbar_wait(&ctrl->dq_full[bq], uint32_t(u / F::NDQ) & 1u, abort));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t v[64];
+      tmem_ld32(lane_base + F::C_DQ + uint32_t(bq * BQ), v);
+      tmem_ld32(lane_base + F::C_DQ + uint32_t(bq * BQ) + 32, v + 32);
+      tmem_ld_wait32(v);
+      tmem_ld_wait32(v + 32);
+      tc_fence_before();
+      mbar_arrive(&ctrl->dq_free[bq]);
+      const int q0 = (j0 + u) * BQ;
+#pragma unroll
+      for (int piece = 0; piece < BQ / QR; ++piece, ++pc) {
+        float *stg = sDQ + (pc & 1) * (QR * F::DQW);
+        if (issuer) bulk_wait_group_read1();  // the reduce that last read this tile is done reading
+        named_bar_sync(1, 128);
+        if (has_col) {
+#pragma unroll
+          for (int i = 0; i < QR; ++i) stg[i * F::DQW + col] = __uint_as_float(v[QR * piece + i]);
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (issuer) {
+          tma_reduce_add_3d(&tm_acc, stg, 0, q0 + QR * piece, bh);
+          bulk_commit_group();
+        }
+      }
+    }
+    if (issuer) bulk_wait_group0();
+    if (!ok && lane == 0) atomicOr(args.flags, kFlagTimeout);
+  } else {
+    setmaxnreg_inc<F::REG_COMPUTE>();
+    // ------------------------------- compute: warpgroup t takes blocks u = t mod 2
+    const int t = warp >> 2, quarter = warp & 3;
+    const int r_loc = quarter * 32 + lane;
+    const int krow = k0 + r_loc;  // this thread's key
+    const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
+    const uint32_t s_tm = lane_base + uint32_t(t * 2 * BQ), dp_tm = s_tm + BQ;
+    // this thread's row of the dS^T tile (128-byte rows, 16-byte chunks swizzled by row)
+    const uint32_t ds_row = smem_u32(sDS + t * F::TILE) + uint32_t(r_loc) * 128u;
+    const uint32_t sw = uint32_t(r_loc) & 7u;
+    const float sl2 = args.scale_log2;
+    const uint64_t sl2x2 = f2_pack(sl2, sl2);
+    bool ok = true;
+    for (int u = t; u < nb; u += 2) {
+      const int s = u % KS;
+      ok = mbar_wait(&ctrl->full[s], uint32_t(u / KS) & 1u, abort) &&
+           mbar_wait(&ctrl->s_full[t], uint32_t(u >> 1) & 1u, abort) &&
+           (u < 2 || mbar_wait(&ctrl->ds_free[t], uint32_t((u >> 1) - 1) & 1u, abort));
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint8_t *st = sStage + s * F::STAGE;
+      const float *sL = reinterpret_cast<const float *>(st + O_L);
+      const float *sD = reinterpret_cast<const float *>(st + O_D);
+      const int q0 = (j0 + u) * BQ;
+      const bool diag = args.causal && q0 < k0 + 127;
+#pragma unroll
+      for (int c = 0; c < BQ / 32; ++c) {
+        uint32_t sx[32], dx[32];
+        tmem_ld32(s_tm + uint32_t(32 * c), sx);
+        tmem_ld32(dp_tm + uint32_t(32 * c), dx);
+        tmem_ld_wait32(sx);
+        tmem_ld_wait32(dx);
+        uint32_t pp[16], dd[16];
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 l4 = *reinterpret_cast<const float4 *>(sL + 32 * c + 4 * e4);
+          const float4 d4 = *reinterpret_cast<const float4 *>(sD + 32 * c + 4 * e4);
+          const uint64_t l2[2] = {f2_pack(l4.x, l4.y), f2_pack(l4.z, l4.w)};
+          const uint64_t d2[2] = {f2_pack(d4.x, d4.y), f2_pack(d4.z, d4.w)};
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int i = 4 * e4 + 2 * h2;
+            float a0, a1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sx[i]), __uint_as_float(sx[i + 1])), sl2x2, l2[h2]), a0, a1);
+            float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
+            if (diag) {
+              const int cq = 32 * c + i;
+              if (q0 + cq < krow) p0 = 0.f;
+              if (q0 + cq + 1 < krow) p1 = 0.f;
+            }
+            const uint64_t p2 = f2_pack(p0, p1);
+            float g0, g1;
+            f2_unpack(f2_mul(p2, f2_sub(f2_pack(__uint_as_float(dx[i]), __uint_as_float(dx[i + 1])), d2[h2])), g0, g1);
+            pp[2 * e4 + h2] = pack_bf16x2(p0, p1);
+            dd[2 * e4 + h2] = pack_bf16x2(g0, g1);
+          }
+        }
+        tmem_st16(s_tm + uint32_t(16 * c), pp);
+        tmem_st16(dp_tm + uint32_t(16 * c), dd);
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj)
+          st_shared_v4(ds_row + (((uint32_t(4 * c + jj)) ^ sw) << 4), dd[4 * jj], dd[4 * jj + 1], dd[4 * jj + 2],
+                       dd[4 * jj + 3]);
+      }
+      tmem_st_wait();
+      fence_proxy_async_smem();  // dS^T in shared memory, for the dq' MMA
+      tc_fence_before();
+      mbar_arrive(&ctrl->p_full[t]);
+    }
+    if (ok) ok = mbar_wait(&ctrl->acc_done, 0, abort);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      // epilogue: warpgroup 0 writes dV and dphi_k, warpgroup 1 dK
+      tc_fence_after();
+      const bool valid = krow < args.N;
+      const int d_st = valid ? args.d : 0;
+      const size_t row_off = (size_t(bh) * args.N + (valid ? krow : 0)) * args.d;
+      uint16_t *dst = static_cast<uint16_t *>(t == 0 ? args.dV : args.dK) + row_off;
+      const uint32_t acc_tm = lane_base + (t == 0 ? F::C_DV : F::C_DK);
+      const float mul = t == 0 ? 1.f : args.scale;
+#pragma unroll 1
+      for (int c0 = 0; c0 < DP; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld16(acc_tm + uint32_t(c0), r);
+        tmem_ld_wait16(r);
+        store_row16_bf16(r, mul, dst, c0, d_st);
+      }
+      if constexpr (RG > 0) {
+        if (t == 0) {
+          const int r_st = valid ? args.R : 0;
+          store_factor_grad_row<RG>(lane_base + F::C_DF, factor_grad_row(args, args.dphi_k, args.dphi_k_part, b, h,
+                                                                          bh, valid ? krow : 0),
+                                    r_st);
+        }
+      }
+    }
+    if (!ok && lane == 0) atomicOr(args.flags, kFlagTimeout);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == F::MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+
 namespace {
 
 constexpr int kMaxDevicesB = 64;
 
+// The fused kernel serves head dim 64 with gradient factor width 0 or 64.
+template <int DP, int RP, int MODE, int RG>
+constexpr bool fused_ok() {
+  if constexpr (DP == 64 && (RG == 0 || RG == 64))
+    return FusedCfg<RP, MODE, RG>::KS >= 3;
+  else
+    return false;
+}
+
+template <int RP, int MODE, int RG>
+cudaError_t launch_bwd_fused(const BwdMaps &m, const BwdArgs &a, cudaStream_t stream) {
+  using F = FusedCfg<RP, MODE, RG>;
+  auto kern = attn_bwd_fused_sm100<RP, MODE, RG>;
+  static std::atomic<int> ready[kMaxDevicesB];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevicesB) return cudaErrorInvalidDevice;
+  if (!ready[dev].load(std::memory_order_acquire)) {
+    // setmaxnreg.inc waits until the block's pool has the registers, so the
+    // launch allocation must be exactly what the split assumes.
+    cudaFuncAttributes fa;
+    if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return e;
+    if (fa.numRegs != int(F::LAUNCH_REGS)) return cudaErrorInvalidConfiguration;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(F::SMEM))) != cudaSuccess)
+      return e;
+    ready[dev].store(1, std::memory_order_release);
+  }
+  const unsigned grid = unsigned((long long)a.n_kv * a.B * a.H);
+  kern<<<grid, F::THREADS, F::SMEM, stream>>>(m.k, m.v, m.fk, m.gk, m.q_blk, m.do_blk, m.fq_blk, m.gq_blk, m.acc, a);
+  return cudaGetLastError();
+}
+
 template <int DP, int RP, int MODE, int RG>
 cudaError_t launch_bwd_one(const BwdMaps &m, const BwdArgs &a, cudaStream_t stream) {
   using C = BwdCfg<DP, RP, MODE, RG>;
-  if constexpr (C::KV_KS < 1 || C::DQ_KS < 1) {
+  if constexpr (fused_ok<DP, RP, MODE, RG>()) {
+    return launch_bwd_fused<RP, MODE, RG>(m, a, stream);
+  } else if constexpr (C::KV_KS < 1 || C::DQ_KS < 1) {
     return cudaErrorInvalidConfiguration;
   } else {
     auto kv = attn_bwd_dkdv_sm100<DP, RP, MODE, RG>;
@@ -849,6 +1330,13 @@ int bwd_query_block_rows(const BwdPlan &p) {
   FB_BWD_ALL
 #undef FB_BWD_ACTION
   return 0;
+}
+
+bool bwd_fused(const BwdPlan &p) {
+#define FB_BWD_ACTION(DPv, RPv, MODEv, RGv) fused_ok<DPv, RPv, MODEv, RGv>()
+  FB_BWD_ALL
+#undef FB_BWD_ACTION
+  return false;
 }
 
 int bwd_key_block_rows(const BwdPlan &p) {

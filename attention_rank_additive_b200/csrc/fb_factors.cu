@@ -499,10 +499,15 @@ __global__ void __launch_bounds__(256) bwd_rows_kernel(long long rows, int N, in
                                                        const __nv_bfloat16 *__restrict__ O,
                                                        const __nv_bfloat16 *__restrict__ dO,
                                                        const float *__restrict__ LSE, float *__restrict__ nlse2,
-                                                       float *__restrict__ delta) {
+                                                       float *__restrict__ delta, float *__restrict__ dq_acc,
+                                                       int dqw) {
   const long long w = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 3;  // row
   const int sub = threadIdx.x & 7;
   if (w >= rows) return;  // whole 8-thread groups leave together
+  if (dq_acc) {
+    float4 *dst = reinterpret_cast<float4 *>(dq_acc + w * dqw);
+    for (int c = sub; c < dqw / 4; c += 8) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   const long long bh = w / Npad;
   const int n = int(w - bh * Npad);
   float acc = 0.f;
@@ -553,12 +558,65 @@ __global__ void prep_grad_factors_kernel(int N, int R, int RG, int fac_H, const 
 }
 
 cudaError_t launch_bwd_rows(int BH, int N, int Npad, int d, const void *O, const void *dO, const float *LSE,
-                            float *nlse2, float *delta, cudaStream_t s) {
+                            float *nlse2, float *delta, float *acc, int dqw, cudaStream_t s) {
   const long long rows = (long long)BH * Npad;  // a multiple of 128: full warps
   const long long blocks = (rows * 8 + 255) / 256;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
   bwd_rows_kernel<<<unsigned(blocks), 256, 0, s>>>(rows, N, Npad, d, static_cast<const __nv_bfloat16 *>(O),
-                                                   static_cast<const __nv_bfloat16 *>(dO), LSE, nlse2, delta);
+                                                   static_cast<const __nv_bfloat16 *>(dO), LSE, nlse2, delta, acc,
+                                                   dqw);
+  return cudaGetLastError();
+}
+
+// The fused backward's accumulator [BH, Npad, dqw] (fp32; columns [0, 64):
+// dQ / scale, columns [64, 64 + R): dphi_q of the head) to dQ (bf16, times the
+// scale) and, where every head has its own factor slice, to dphi_q. One
+// 8-thread group per row; a thread takes 8 consecutive columns.
+__global__ void __launch_bounds__(256) bwd_dq_convert_kernel(long long rows, int H, int N, int Npad, int d, int R,
+                                                             int dqw, float scale, const float *__restrict__ acc,
+                                                             __nv_bfloat16 *__restrict__ dQ,
+                                                             float *__restrict__ dphi_q, long long bs, long long hs,
+                                                             int fac_B, int fac_H) {
+  const long long w = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 3;  // row (bh, n), n < N
+  const int sub = threadIdx.x & 7;
+  if (w >= rows) return;
+  const long long bh = w / N;
+  const int n = int(w - bh * N);
+  const float *src = acc + (bh * Npad + n) * dqw;
+  const int c0 = sub * 8;
+  if (c0 < d) {
+    const float4 a = *reinterpret_cast<const float4 *>(src + c0);
+    const float4 b = *reinterpret_cast<const float4 *>(src + c0 + 4);
+    const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    __nv_bfloat16 *dst = dQ + w * d + c0;
+    if (c0 + 8 <= d && (d & 7) == 0) {
+      uint32_t p[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const __nv_bfloat162 t = __floats2bfloat162_rn(v[2 * e] * scale, v[2 * e + 1] * scale);
+        p[e] = *reinterpret_cast<const uint32_t *>(&t);
+      }
+      *reinterpret_cast<uint4 *>(dst) = make_uint4(p[0], p[1], p[2], p[3]);
+    } else {
+      for (int e = 0; e < 8 && c0 + e < d; ++e) dst[e] = __float2bfloat16_rn(v[e] * scale);
+    }
+  }
+  if (dphi_q) {
+    const int b = int(bh / H), h = int(bh - (bh / H) * H);
+    float *row = dphi_q + (fac_B > 1 ? b * bs : 0) + (fac_H > 1 ? h * hs : 0) + (long long)n * R;
+    for (int r = sub; r < R; r += 8) row[r] = src[64 + r];
+  }
+}
+
+cudaError_t launch_bwd_dq_convert(int B, int H, int N, int Npad, int d, int R, int dqw, float scale,
+                                  const float *acc, void *dQ, float *dphi_q, int64_t bs, int64_t hs, int fac_B,
+                                  int fac_H, cudaStream_t s) {
+  const long long rows = (long long)B * H * N;
+  const long long blocks = (rows * 8 + 255) / 256;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  bwd_dq_convert_kernel<<<unsigned(blocks), 256, 0, s>>>(rows, H, N, Npad, d, R, dqw, scale, acc,
+                                                         static_cast<__nv_bfloat16 *>(dQ), dphi_q, bs, hs, fac_B,
+                                                         fac_H);
   return cudaGetLastError();
 }
 
@@ -573,9 +631,12 @@ cudaError_t launch_prep_grad_factors(int N, int R, int RG, const float *phi_q, c
 
 // dphi[fb, fh, n, r] = sum over the heads (b, h) that share slice (fb, fh)
 // of part[b H + h, n, r]: one thread per output element, fp32 in head order.
+// The q-side rows may sit in a wider buffer: row n of head bh at
+// pq + bh q_head + n q_row + q_off.
 __global__ void reduce_factor_grads_kernel(int B, int H, int N, int R, int fac_B, int fac_H, long long bs,
-                                           long long hs, const float *__restrict__ pq, const float *__restrict__ pk,
-                                           float *__restrict__ dq, float *__restrict__ dk, long long total) {
+                                           long long hs, const float *__restrict__ pq, long long q_head, int q_row,
+                                           int q_off, const float *__restrict__ pk, float *__restrict__ dq,
+                                           float *__restrict__ dk, long long total) {
   const long long NR = (long long)N * R;
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
        idx += (long long)gridDim.x * blockDim.x) {
@@ -583,14 +644,15 @@ __global__ void reduce_factor_grads_kernel(int B, int H, int N, int R, int fac_B
     const int fb = int(f / fac_H), fh = int(f - (f / fac_H) * fac_H);
     const int b0 = fac_B > 1 ? fb : 0, b1 = fac_B > 1 ? fb + 1 : B;
     const int h0 = fac_H > 1 ? fh : 0, h1 = fac_H > 1 ? fh + 1 : H;
+    const long long n = e / R, r = e - (e / R) * R;
+    const long long oq = n * q_row + q_off + r;
     float aq = 0.f, ak = 0.f;
     for (int b = b0; b < b1; ++b)
       for (int h = h0; h < h1; ++h) {
-        const long long o = ((long long)b * H + h) * NR + e;
-        aq += pq[o];
-        ak += pk[o];
+        const long long hb = (long long)b * H + h;
+        aq += pq[hb * q_head + oq];
+        ak += pk[hb * NR + e];
       }
-    const long long n = e / R, r = e - (e / R) * R;
     const long long dst = fb * bs + fh * hs + n * R + r;
     dq[dst] = aq;
     dk[dst] = ak;
@@ -598,11 +660,11 @@ __global__ void reduce_factor_grads_kernel(int B, int H, int N, int R, int fac_B
 }
 
 cudaError_t launch_reduce_factor_grads(int B, int H, int N, int R, int fac_B, int fac_H, int64_t bs, int64_t hs,
-                                       const float *part_q, const float *part_k, float *dphi_q, float *dphi_k,
-                                       cudaStream_t s) {
+                                       const float *part_q, int64_t q_head, int q_row, int q_off, const float *part_k,
+                                       float *dphi_q, float *dphi_k, cudaStream_t s) {
   const long long total = (long long)fac_B * fac_H * N * R;
-  reduce_factor_grads_kernel<<<grid_for(total, 256), 256, 0, s>>>(B, H, N, R, fac_B, fac_H, bs, hs, part_q, part_k,
-                                                                  dphi_q, dphi_k, total);
+  reduce_factor_grads_kernel<<<grid_for(total, 256), 256, 0, s>>>(B, H, N, R, fac_B, fac_H, bs, hs, part_q, q_head,
+                                                                  q_row, q_off, part_k, dphi_q, dphi_k, total);
   return cudaGetLastError();
 }
 

@@ -110,6 +110,7 @@ struct BwdArgs {
   int dphi_direct;         // 1: every head has its own factor slice, rows go straight to dphi
   int64_t phi_bs, phi_hs;  // element strides of the factor tensors
   int fac_B, fac_H;        // factor slices: B or 1, H or 1
+  float *dqacc;            // fused kernel: fp32 [BH, Npad, 64 + RG] accumulator of dq' = dS [K | phi_k]
   int *flags;
 };
 
@@ -125,6 +126,8 @@ struct BwdMaps {
   CUtensorMap k, v, fk;                          // dK/dV kernel, fixed tiles: box rows 128
   CUtensorMap q_blk, do_blk, fq_blk, gq_blk;     // dK/dV kernel, streamed query blocks
   CUtensorMap k_blk, v_blk, fk_blk, gk_blk;      // dQ kernel, streamed key blocks
+  CUtensorMap gk;                                // fused kernel: fixed bf16 gradient factor tile, box rows 128
+  CUtensorMap acc;                               // fused kernel: fp32 dq' accumulator, box (64 + RG, 16 or 32, 1)
   // Q, K, V, dO: bf16 [BH, N, d], box (min(DP,64), rows, 1); fq/fk: the forward's
   // factor tiles; gq/gk: bf16 gradient factors [FB, N, RG].
 };
@@ -133,18 +136,29 @@ struct BwdMaps {
 // for a plan (0: unsupported).
 int bwd_query_block_rows(const BwdPlan &p);
 int bwd_key_block_rows(const BwdPlan &p);
+// Whether the plan runs as the single fused kernel (dq' accumulated in the
+// workspace, then converted) instead of the dK/dV and dQ kernels.
+bool bwd_fused(const BwdPlan &p);
+// dQ = scale acc[:, :d] (bf16) and, where every head has its own factor slice,
+// dphi_q = acc[:, 64:64+R], from the fused kernel's accumulator.
+cudaError_t launch_bwd_dq_convert(int B, int H, int N, int Npad, int d, int R, int dqw, float scale,
+                                  const float *acc, void *dQ, float *dphi_q, int64_t bs, int64_t hs, int fac_B,
+                                  int fac_H, cudaStream_t s);
 cudaError_t bwd_launch(const BwdPlan &p, const BwdMaps &maps, const BwdArgs &a, cudaStream_t stream);
 // nlse2 = -LSE * log2(e) and delta = rowsum(dO * O) per row, padded to Npad.
+// With acc != nullptr, also zeroes the fused kernel's accumulator rows [BH, Npad, dqw].
 cudaError_t launch_bwd_rows(int BH, int N, int Npad, int d, const void *O, const void *dO, const float *LSE,
-                            float *nlse2, float *delta, cudaStream_t s);
+                            float *nlse2, float *delta, float *acc, int dqw, cudaStream_t s);
 // bf16 copies of the factors [FB, N, RG] (zero-padded).
 cudaError_t launch_prep_grad_factors(int N, int R, int RG, const float *phi_q, const float *phi_k, int64_t bs,
                                      int64_t hs, int fac_B, int fac_H, void *gq, void *gk, cudaStream_t s);
 // Factor gradients of shared slices: dphi[f] = sum over the heads of slice f of
-// the per-head partial rows [B*H, N, R].
+// the per-head partial rows: [B*H, N, R] for k; for q, row n of head bh at
+// part_q + bh q_head + n q_row + q_off (the partial rows, or the fused
+// kernel's accumulator).
 cudaError_t launch_reduce_factor_grads(int B, int H, int N, int R, int fac_B, int fac_H, int64_t bs, int64_t hs,
-                                       const float *part_q, const float *part_k, float *dphi_q, float *dphi_k,
-                                       cudaStream_t s);
+                                       const float *part_q, int64_t q_head, int q_row, int q_off, const float *part_k,
+                                       float *dphi_q, float *dphi_k, cudaStream_t s);
 
 // Per-device flag word (allocated once per device as a module global).
 int *device_flags();

@@ -246,11 +246,17 @@ int fb_attn_neural_fwd(int dt, int B, int H, int N, int d,
  * Arithmetic: S and P are recomputed as the forward computes them; the
  * products with dO, Q, K and the factors run on the tensor cores in bf16 with
  * fp32 accumulation. Launches: the factor preparation and the bf16 factor
- * copies (R > 0), the per-row terms, then two tcgen05 kernels (dK, dV,
- * dphi_k per key tile; dQ, dphi_q per query tile), and for a factor shared
- * by several heads one reduction of the per-head factor gradients (kept in
- * the workspace). Argument errors return before any launch; other errors as
- * fb_attn_fwd.
+ * copies (R > 0), the per-row terms, then the gradient kernels, and for a
+ * factor shared by several heads one reduction of the per-head factor
+ * gradients (kept in the workspace). The gradient kernels: for head dims 33
+ * to 64 with fixed factors (or R = 0) or with 33 <= R <= 64, one tcgen05
+ * kernel per key tile that also adds each query block's dS [K | phi_k] into
+ * an fp32 accumulator in the workspace (TMA reduce-adds at L2), then a
+ * conversion to dQ and dphi_q; the order of those fp32 additions varies
+ * between runs, so dQ and dphi_q may differ in the last bits from run to run.
+ * Otherwise two tcgen05 kernels (dK, dV, dphi_k per key tile; dQ, dphi_q per
+ * query tile), bitwise reproducible. Argument errors return before any
+ * launch; other errors as fb_attn_fwd.
  */
 size_t fb_attn_bwd_workspace_bytes(int B, int H, int N, int R,
                                    int64_t phi_bstride, int64_t phi_hstride);
