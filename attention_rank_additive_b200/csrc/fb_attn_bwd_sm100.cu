@@ -912,6 +912,10 @@ __global__ void __launch_bounds__(512, 1)
   const uint32_t tmem = ctrl->tmem_base;
   volatile int *abort = &ctrl->abort;
   const uint32_t leader = lane == 0 ? 1u : 0u;
+  // The set-up above reads no global memory; the per-row terms and the zeroed
+  // accumulator of the kernel before are read only once it has completed.
+  griddep_launch_dependents();
+  griddep_wait();
 
   if (warp >= F::PRODUCER_WARP && warp < F::DQ_WARP0) {
     setmaxnreg_dec<F::REG_OTHER>();
@@ -1113,7 +1117,9 @@ __global__ void __launch_bounds__(512, 1)
         }
       }
     }
-    if (issuer) bulk_wait_group0();
+    // the staging tiles must outlive the reads of the last reduces; the adds
+    // themselves complete with the kernel
+    if (issuer) bulk_wait_group_read0();
     if (!ok && lane == 0) atomicOr(args.flags, kFlagTimeout);
   } else {
     setmaxnreg_inc<F::REG_COMPUTE>();
@@ -1191,7 +1197,8 @@ __global__ void __launch_bounds__(512, 1)
     if (ok) ok = mbar_wait(&ctrl->acc_done, 0, abort);
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
-      // epilogue: warpgroup 0 writes dV and dphi_k, warpgroup 1 dK
+      // epilogue: warpgroup 0 writes dV, warpgroup 1 dK, each half of dphi_k's
+      // columns; all TMEM loads are issued before one wait
       tc_fence_after();
       const bool valid = krow < args.N;
       const int d_st = valid ? args.d : 0;
@@ -1199,19 +1206,32 @@ __global__ void __launch_bounds__(512, 1)
       uint16_t *dst = static_cast<uint16_t *>(t == 0 ? args.dV : args.dK) + row_off;
       const uint32_t acc_tm = lane_base + (t == 0 ? F::C_DV : F::C_DK);
       const float mul = t == 0 ? 1.f : args.scale;
-#pragma unroll 1
-      for (int c0 = 0; c0 < DP; c0 += 16) {
-        uint32_t r[16];
-        tmem_ld16(acc_tm + uint32_t(c0), r);
-        tmem_ld_wait16(r);
-        store_row16_bf16(r, mul, dst, c0, d_st);
-      }
+      uint32_t r[64], g[RG > 0 ? 32 : 1];
+      tmem_ld32(acc_tm, r);
+      tmem_ld32(acc_tm + 32, r + 32);
+      if constexpr (RG > 0) tmem_ld32(lane_base + F::C_DF + uint32_t(32 * t), g);
+      tmem_ld_wait32(r);
+      tmem_ld_wait32(r + 32);
+      if constexpr (RG > 0) tmem_ld_wait32(g);
+#pragma unroll
+      for (int c0 = 0; c0 < DP; c0 += 16) store_row16_bf16(r + c0, mul, dst, c0, d_st);
       if constexpr (RG > 0) {
-        if (t == 0) {
-          const int r_st = valid ? args.R : 0;
-          store_factor_grad_row<RG>(lane_base + F::C_DF, factor_grad_row(args, args.dphi_k, args.dphi_k_part, b, h,
-                                                                          bh, valid ? krow : 0),
-                                    r_st);
+        // columns [32 t, 32 t + 32) of this key's dphi_k row, those below R
+        float *frow =
+            factor_grad_row(args, args.dphi_k, args.dphi_k_part, b, h, bh, valid ? krow : 0) + 32 * t;
+        const int n_st = valid ? min(32, max(0, args.R - 32 * t)) : 0;
+        const bool vec = (n_st & 3) == 0 && (reinterpret_cast<uintptr_t>(frow) & 15u) == 0;
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          if (vec) {
+            if (e < n_st)
+              *reinterpret_cast<float4 *>(frow + e) = make_float4(__uint_as_float(g[e]), __uint_as_float(g[e + 1]),
+                                                                   __uint_as_float(g[e + 2]), __uint_as_float(g[e + 3]));
+          } else {
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+              if (e + x < n_st) frow[e + x] = __uint_as_float(g[e + x]);
+          }
         }
       }
     }
@@ -1260,8 +1280,8 @@ cudaError_t launch_bwd_fused(const BwdMaps &m, const BwdArgs &a, cudaStream_t st
     ready[dev].store(1, std::memory_order_release);
   }
   const unsigned grid = unsigned((long long)a.n_kv * a.B * a.H);
-  kern<<<grid, F::THREADS, F::SMEM, stream>>>(m.k, m.v, m.fk, m.gk, m.q_blk, m.do_blk, m.fq_blk, m.gq_blk, m.acc, a);
-  return cudaGetLastError();
+  return launch_programmatic(kern, dim3(grid), dim3(F::THREADS), F::SMEM, stream, m.k, m.v, m.fk, m.gk, m.q_blk,
+                             m.do_blk, m.fq_blk, m.gq_blk, m.acc, a);
 }
 
 template <int DP, int RP, int MODE, int RG>

@@ -501,6 +501,7 @@ __global__ void __launch_bounds__(256) bwd_rows_kernel(long long rows, int N, in
                                                        const float *__restrict__ LSE, float *__restrict__ nlse2,
                                                        float *__restrict__ delta, float *__restrict__ dq_acc,
                                                        int dqw) {
+  griddep_launch_dependents();  // the gradient kernel may start its set-up now
   const long long w = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 3;  // row
   const int sub = threadIdx.x & 7;
   if (w >= rows) return;  // whole 8-thread groups leave together
@@ -577,6 +578,8 @@ __global__ void __launch_bounds__(256) bwd_dq_convert_kernel(long long rows, int
                                                              __nv_bfloat16 *__restrict__ dQ,
                                                              float *__restrict__ dphi_q, long long bs, long long hs,
                                                              int fac_B, int fac_H) {
+  griddep_launch_dependents();
+  griddep_wait();  // the fused kernel's accumulator is complete
   const long long w = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 3;  // row (bh, n), n < N
   const int sub = threadIdx.x & 7;
   if (w >= rows) return;
@@ -614,10 +617,9 @@ cudaError_t launch_bwd_dq_convert(int B, int H, int N, int Npad, int d, int R, i
   const long long rows = (long long)B * H * N;
   const long long blocks = (rows * 8 + 255) / 256;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-  bwd_dq_convert_kernel<<<unsigned(blocks), 256, 0, s>>>(rows, H, N, Npad, d, R, dqw, scale, acc,
-                                                         static_cast<__nv_bfloat16 *>(dQ), dphi_q, bs, hs, fac_B,
-                                                         fac_H);
-  return cudaGetLastError();
+  return launch_programmatic(bwd_dq_convert_kernel, dim3(unsigned(blocks)), dim3(256), 0, s, rows, H, N, Npad, d, R,
+                             dqw, scale, acc, static_cast<__nv_bfloat16 *>(dQ), dphi_q, (long long)bs,
+                             (long long)hs, fac_B, fac_H);
 }
 
 cudaError_t launch_prep_grad_factors(int N, int R, int RG, const float *phi_q, const float *phi_k, int64_t bs,
@@ -637,6 +639,7 @@ __global__ void reduce_factor_grads_kernel(int B, int H, int N, int R, int fac_B
                                            long long hs, const float *__restrict__ pq, long long q_head, int q_row,
                                            int q_off, const float *__restrict__ pk, float *__restrict__ dq,
                                            float *__restrict__ dk, long long total) {
+  griddep_wait();  // the gradient kernels' partial rows are complete
   const long long NR = (long long)N * R;
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
        idx += (long long)gridDim.x * blockDim.x) {
@@ -663,9 +666,9 @@ cudaError_t launch_reduce_factor_grads(int B, int H, int N, int R, int fac_B, in
                                        const float *part_q, int64_t q_head, int q_row, int q_off, const float *part_k,
                                        float *dphi_q, float *dphi_k, cudaStream_t s) {
   const long long total = (long long)fac_B * fac_H * N * R;
-  reduce_factor_grads_kernel<<<grid_for(total, 256), 256, 0, s>>>(B, H, N, R, fac_B, fac_H, bs, hs, part_q, q_head,
-                                                                  q_row, q_off, part_k, dphi_q, dphi_k, total);
-  return cudaGetLastError();
+  return launch_programmatic(reduce_factor_grads_kernel, dim3(grid_for(total, 256)), dim3(256), 0, s, B, H, N, R,
+                             fac_B, fac_H, (long long)bs, (long long)hs, part_q, (long long)q_head, q_row, q_off,
+                             part_k, dphi_q, dphi_k, total);
 }
 
 // Gradients of the neural decomposition's linear layers from the factor

@@ -160,6 +160,26 @@ cudaError_t launch_reduce_factor_grads(int B, int H, int N, int R, int fac_B, in
                                        const float *part_q, int64_t q_head, int q_row, int q_off, const float *part_k,
                                        float *dphi_q, float *dphi_k, cudaStream_t s);
 
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel in the stream finishes, and must call griddep_wait()
+// before it reads anything that kernel writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_programmatic(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                                Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 // Per-device flag word (allocated once per device as a module global).
 int *device_flags();
 
