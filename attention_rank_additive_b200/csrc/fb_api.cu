@@ -585,7 +585,7 @@ struct BwdLayout {
   WsLayout f;  // the S-side factor tiles (as the forward's workspace)
   // acc_off: the fused kernel's fp32 dq' accumulator [BH, Npad, up to 128]; the
   // two-kernel path keeps its per-head dphi_q rows there instead (pq_off).
-  size_t gq_off, gk_off, l_off, d_off, acc_off, pq_off, pk_off, total;
+  size_t gq_off, gk_off, l_off, d_off, acc_off, pq_off, pk_off, sched_off, total;
   int RG, Npad;
   bool shared_slices;  // some factor slice serves several heads: per-head partial gradients
 };
@@ -608,7 +608,8 @@ BwdLayout bwd_layout(int B, int H, int N, int R, int64_t bs, int64_t hs) {
   w.acc_off = w.d_off + rows;
   w.pq_off = w.acc_off;
   w.pk_off = w.acc_off + acc;
-  w.total = w.pk_off + part;
+  w.sched_off = w.pk_off + part;  // the fused kernel's work counter
+  w.total = w.sched_off + 256;
   return w;
 }
 bool encode_rows_bf16(CUtensorMap *m, const void *ptr, int slices, int N, int cols, int width, int rows) {
@@ -723,7 +724,9 @@ int fb_attn_bwd(int dt, int B, int H, int N, int d, const void *Q, const void *K
   }
   // 3. per-row -LSE in log2 units and rowsum(dO * O)
   //    (and, fused, the zeroed accumulator)
-  if (launch_bwd_rows(BH, N, L.Npad, d, O, dO, LSE, nlse2, delta, fused ? acc : nullptr, dqw, st) != cudaSuccess)
+  unsigned int *sched = reinterpret_cast<unsigned int *>(wsb + L.sched_off);
+  if (launch_bwd_rows(BH, N, L.Npad, d, O, dO, LSE, nlse2, delta, fused ? acc : nullptr, dqw,
+                      fused ? sched : nullptr, st) != cudaSuccess)
     return FB_ERR_CUDA;
 
   // 4. the gradient kernels: the fused kernel, or the dK/dV and dQ kernels
@@ -746,6 +749,7 @@ int fb_attn_bwd(int dt, int B, int H, int N, int d, const void *Q, const void *K
   a.phi_bs = phi_bstride, a.phi_hs = phi_hstride;
   a.fac_B = fac_B, a.fac_H = fac_H;
   a.dqacc = fused ? acc : nullptr;
+  a.sched = fused ? sched : nullptr;
   a.flags = flags;
   if (bwd_launch(plan, maps, a, st) != cudaSuccess) return FB_ERR_CUDA;
   // 5. fused: dQ (and per-head dphi_q) from the accumulator

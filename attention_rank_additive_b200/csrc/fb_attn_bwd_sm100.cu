@@ -837,17 +837,66 @@ struct FusedCfg {
 };
 
 struct FusedCtrl {
-  uint64_t fixed_full;
+  uint64_t fixed_full, fixed_empty;  // the item's fixed tiles: loaded / read by its last S and dq' MMAs
   uint64_t full[4], empty[4];
   uint64_t s_full[2], p_full[2];
-  uint64_t ds_free[2];             // the dq' MMA has read warpgroup t's dS^T tile
+  uint64_t ds_free[2];              // the dq' MMA has read warpgroup t's dS^T tile
   uint64_t dq_full[2], dq_free[2];  // dq'^T buffer b in TMEM: written by the MMA / read by the readout
-  uint64_t acc_done;
+  uint64_t acc_done, acc_empty;     // the item's dV, dK, dphi_k: complete / read out of TMEM
+  uint64_t item_full[4], item_empty[4];  // the work-item ring (producer -> every other warp)
+  int item[4];
   uint32_t tmem_base;
   int abort;
 };
 static_assert(sizeof(FusedCtrl) <= 1024, "control block too large");
 
+// Warps that read each published work item: the MMA warp, the dq' MMA warp,
+// the four readout warps and the eight compute warps (lane 0 of each frees
+// the ring slot).
+constexpr int kFusedItemReaders = 1 + 1 + 4 + 8;
+
+// A work item (key tile, head) of the fused kernel; items are numbered
+// heaviest causal key tile first.
+struct FusedItem {
+  int kb, bh, b, h, k0, fslice, j0, nb;
+};
+__device__ __forceinline__ FusedItem fused_item(int k, const BwdArgs &a) {
+  FusedItem w;
+  const int BH = a.B * a.H;
+  w.kb = k / BH;
+  w.bh = k - w.kb * BH;
+  w.b = w.bh / a.H;
+  w.h = w.bh - w.b * a.H;
+  w.k0 = w.kb * 128;
+  w.fslice = (a.fac_B > 1 ? w.b : 0) * a.fac_H + (a.fac_H > 1 ? w.h : 0);
+  w.j0 = a.causal ? w.k0 / 64 : 0;  // query blocks before the diagonal see none of these keys
+  w.nb = (a.N + 63) / 64 - w.j0;    // >= 1
+  return w;
+}
+
+// The item of the CTA's pass p: its own index first, then the next unclaimed
+// one from the counter (zeroed by the per-row pass before the launch).
+__device__ __forceinline__ int fused_claim(int p, int n_items, unsigned int *sched) {
+  if (p == 0) return int(blockIdx.x);
+  const unsigned int k = gridDim.x + atomicAdd(sched, 1u);
+  return k < unsigned(n_items) ? int(k) : -1;
+}
+
+// Ring read by one warp: wait for pass p's item, read it, free the slot.
+__device__ __forceinline__ int fused_read_item(FusedCtrl *ctrl, int p, volatile int *abort, bool &ok) {
+  const int slot = p & 3;
+  ok = mbar_wait(&ctrl->item_full[slot], uint32_t(p >> 2) & 1u, abort);
+  if (!ok) return -1;
+  const int k = *reinterpret_cast<const volatile int *>(&ctrl->item[slot]);
+  __syncwarp();
+  if ((threadIdx.x & 31u) == 0) mbar_arrive(&ctrl->item_empty[slot]);
+  return k;
+}
+
+// Persistent: one CTA per SM walks work items (key tile, head). Every
+// barrier phase runs on counters that continue across items: g counts query
+// blocks (stage ring, score buffers, dq' buffers), p counts items (fixed
+// tiles, accumulators).
 template <int RP, int MODE, int RG>
 __global__ void __launch_bounds__(512, 1)
     attn_bwd_fused_sm100(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -874,17 +923,11 @@ __global__ void __launch_bounds__(512, 1)
   static_assert(O_D + BQ * 4 == F::STAGE_BYTES, "stage layout");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int BH = args.B * args.H;
-  const int kb = int(blockIdx.x) / BH;  // key tile; the heaviest causal tiles come first
-  const int bh = int(blockIdx.x) % BH;
-  const int b = bh / args.H, h = bh % args.H;
-  const int k0 = kb * 128;
-  const int fslice = (args.fac_B > 1 ? b : 0) * args.fac_H + (args.fac_H > 1 ? h : 0);
-  const int j0 = args.causal ? k0 / BQ : 0;
-  const int nb = (args.N + BQ - 1) / BQ - j0;  // >= 1
+  const int n_items = args.n_kv * args.B * args.H;
 
   if (threadIdx.x == 0) {
     mbar_init(&ctrl->fixed_full, 1);
+    mbar_init(&ctrl->fixed_empty, 2);
     for (int s = 0; s < KS; ++s) {
       mbar_init(&ctrl->full[s], 1);
       mbar_init(&ctrl->empty[s], 1);
@@ -893,12 +936,15 @@ __global__ void __launch_bounds__(512, 1)
       mbar_init(&ctrl->s_full[t], 1);
       mbar_init(&ctrl->p_full[t], 128);
       mbar_init(&ctrl->ds_free[t], 1);
-    }
-    for (int q = 0; q < 2; ++q) {
-      mbar_init(&ctrl->dq_full[q], 1);
-      mbar_init(&ctrl->dq_free[q], 128);
+      mbar_init(&ctrl->dq_full[t], 1);
+      mbar_init(&ctrl->dq_free[t], 128);
     }
     mbar_init(&ctrl->acc_done, 1);
+    mbar_init(&ctrl->acc_empty, 256);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&ctrl->item_full[i], 1);
+      mbar_init(&ctrl->item_empty[i], kFusedItemReaders);
+    }
     ctrl->abort = 0;
     fence_mbar_init();
   }
@@ -912,8 +958,9 @@ __global__ void __launch_bounds__(512, 1)
   const uint32_t tmem = ctrl->tmem_base;
   volatile int *abort = &ctrl->abort;
   const uint32_t leader = lane == 0 ? 1u : 0u;
-  // The set-up above reads no global memory; the per-row terms and the zeroed
-  // accumulator of the kernel before are read only once it has completed.
+  // The set-up above reads no global memory; the per-row terms, the zeroed
+  // accumulator and work counter of the kernel before are read only once it
+  // has completed.
   griddep_launch_dependents();
   griddep_wait();
 
@@ -921,6 +968,10 @@ __global__ void __launch_bounds__(512, 1)
     setmaxnreg_dec<F::REG_OTHER>();
     if (warp == F::PRODUCER_WARP) {
       // ---------------------------------------------------------- producer
+      // Per item: the first KS query blocks' stages (they free up during the
+      // previous item's last blocks), the fixed tiles once the previous item's
+      // last S and dq' MMAs have read them, then the remaining stages. The
+      // next item is claimed and published after the item's loads.
       if (leader) {
         tma_prefetch_map(&tm_k);
         tma_prefetch_map(&tm_v);
@@ -935,34 +986,63 @@ __global__ void __launch_bounds__(512, 1)
           tma_prefetch_map(&tm_gq);
         }
       }
-      mbar_arrive_expect_tx_leader(&ctrl->fixed_full, F::FIXED, leader);
-      tma_load_3d_leader(sK, &tm_k, &ctrl->fixed_full, 0, k0, bh, leader);
-      tma_load_3d_leader(sV, &tm_v, &ctrl->fixed_full, 0, k0, bh, leader);
-      if (RG > 0) tma_load_3d_leader(sGK, &tm_gk, &ctrl->fixed_full, 0, k0, fslice, leader);
-      if (C::FAC)
-        for (int ch = 0; ch < C::NFCH; ++ch)
-          tma_load_3d_leader(sFK + ch * (128 * C::FCH * 2), &tm_fk, &ctrl->fixed_full, ch * C::FCH, k0, fslice,
-                             leader);
       bool ok = true;
-      for (int u = 0; u < nb; ++u) {
-        const int s = u % KS;
-        if (u >= KS && !(ok = mbar_wait(&ctrl->empty[s], (uint32_t(u / KS) & 1u) ^ 1u, abort))) break;
-        uint8_t *st = sStage + s * F::STAGE;
-        const int q0 = (j0 + u) * BQ;
-        mbar_arrive_expect_tx_leader(&ctrl->full[s], F::STAGE_BYTES, leader);
-        tma_load_3d_leader(st + O_Q, &tm_q, &ctrl->full[s], 0, q0, bh, leader);
-        tma_load_3d_leader(st + O_DO, &tm_do, &ctrl->full[s], 0, q0, bh, leader);
+      int cur = __shfl_sync(0xffffffffu, leader ? fused_claim(0, n_items, args.sched) : 0, 0);
+      if (leader) {
+        ctrl->item[0] = cur;
+        mbar_arrive(&ctrl->item_full[0]);
+      }
+      int g = 0;
+      for (int p = 0; ok && cur >= 0; ++p) {
+        const FusedItem w = fused_item(cur, args);
+        auto load_stage = [&](int u) -> bool {
+          const int gg = g + u;
+          const int s = gg % KS;
+          if (gg >= KS && !mbar_wait(&ctrl->empty[s], (uint32_t(gg / KS) & 1u) ^ 1u, abort)) return false;
+          uint8_t *st = sStage + s * F::STAGE;
+          const int q0 = (w.j0 + u) * BQ;
+          mbar_arrive_expect_tx_leader(&ctrl->full[s], F::STAGE_BYTES, leader);
+          tma_load_3d_leader(st + O_Q, &tm_q, &ctrl->full[s], 0, q0, w.bh, leader);
+          tma_load_3d_leader(st + O_DO, &tm_do, &ctrl->full[s], 0, q0, w.bh, leader);
+          if (C::FAC)
+            for (int ch = 0; ch < C::NFCH; ++ch)
+              tma_load_3d_leader(st + O_FQ + ch * (BQ * C::FCH * 2), &tm_fq, &ctrl->full[s], ch * C::FCH, q0,
+                                 w.fslice, leader);
+          if (RG > 0) tma_load_3d_leader(st + O_GQ, &tm_gq, &ctrl->full[s], 0, q0, w.fslice, leader);
+          const size_t roff = size_t(w.bh) * args.Npad + q0;
+          bulk_load_leader(st + O_L, args.nlse2 + roff, BQ * 4, &ctrl->full[s], leader);
+          bulk_load_leader(st + O_D, args.delta + roff, BQ * 4, &ctrl->full[s], leader);
+          return true;
+        };
+        const int early = w.nb < KS ? w.nb : KS;
+        for (int u = 0; u < early && ok; ++u) ok = load_stage(u);
+        if (!ok) break;
+        if (p > 0 && !(ok = mbar_wait(&ctrl->fixed_empty, uint32_t(p - 1) & 1u, abort))) break;
+        mbar_arrive_expect_tx_leader(&ctrl->fixed_full, F::FIXED, leader);
+        tma_load_3d_leader(sK, &tm_k, &ctrl->fixed_full, 0, w.k0, w.bh, leader);
+        tma_load_3d_leader(sV, &tm_v, &ctrl->fixed_full, 0, w.k0, w.bh, leader);
+        if (RG > 0) tma_load_3d_leader(sGK, &tm_gk, &ctrl->fixed_full, 0, w.k0, w.fslice, leader);
         if (C::FAC)
           for (int ch = 0; ch < C::NFCH; ++ch)
-            tma_load_3d_leader(st + O_FQ + ch * (BQ * C::FCH * 2), &tm_fq, &ctrl->full[s], ch * C::FCH, q0, fslice,
+            tma_load_3d_leader(sFK + ch * (128 * C::FCH * 2), &tm_fk, &ctrl->fixed_full, ch * C::FCH, w.k0, w.fslice,
                                leader);
-        if (RG > 0) tma_load_3d_leader(st + O_GQ, &tm_gq, &ctrl->full[s], 0, q0, fslice, leader);
-        const size_t roff = size_t(bh) * args.Npad + q0;
-        bulk_load_leader(st + O_L, args.nlse2 + roff, BQ * 4, &ctrl->full[s], leader);
-        bulk_load_leader(st + O_D, args.delta + roff, BQ * 4, &ctrl->full[s], leader);
+        for (int u = early; u < w.nb && ok; ++u) ok = load_stage(u);
+        if (!ok) break;
+        g += w.nb;
+        // the next item, published once its ring slot is free
+        const int nxt = __shfl_sync(0xffffffffu, leader ? fused_claim(p + 1, n_items, args.sched) : 0, 0);
+        const int slot = (p + 1) & 3;
+        if (p + 1 >= 4 && !(ok = mbar_wait(&ctrl->item_empty[slot], uint32_t((p + 1) / 4 - 1) & 1u, abort))) break;
+        if (leader) {
+          ctrl->item[slot] = nxt;
+          mbar_arrive(&ctrl->item_full[slot]);
+        }
+        cur = nxt;
       }
       if (!ok) {
+        // Aborted: let the copies already issued land before the CTA exits.
         mbar_wait_for(&ctrl->fixed_full, 0, 100000000ull);
+        mbar_wait_for(&ctrl->fixed_full, 1, 100000000ull);
         for (int s = 0; s < KS; ++s) {
           mbar_wait_for(&ctrl->full[s], 0, 100000000ull);
           mbar_wait_for(&ctrl->full[s], 1, 100000000ull);
@@ -971,20 +1051,21 @@ __global__ void __launch_bounds__(512, 1)
       }
     } else if (warp == F::MMA_WARP) {
       // -------------------------------------------------------- MMA issuer
-      // S(0), S(1), then per block u: G(u), S(u + 2), where G(u) is the
-      // key-side gradient products (from TMEM P^T, dS^T).
+      // Per item: S(0), S(1), then per block u: G(u), S(u + 2), where G(u) is
+      // the key-side gradient products (from TMEM P^T, dS^T); the first G of
+      // an item waits for the previous item's accumulators to be read out.
       const uint32_t tm_u = __shfl_sync(0xffffffffu, tmem, 0);
-      bool ok = __all_sync(0xffffffffu, mbar_wait(&ctrl->fixed_full, 0, abort));
-      tc_fence_after();
       const uint64_t dK = kdesc<64>(smem_u32(sK));
       const uint64_t dV = kdesc<64>(smem_u32(sV));
       const uint64_t dFK = kdesc<C::FCH>(smem_u32(sFK));
-      auto issue_s = [&](int u) -> bool {
-        const int s = u % KS;
-        if (!__all_sync(0xffffffffu, mbar_wait(&ctrl->full[s], uint32_t(u / KS) & 1u, abort))) return false;
+      bool ok = true;
+      int g = 0;
+      auto issue_s = [&](int gg, int u, int j0) -> bool {
+        const int s = gg % KS;
+        if (!__all_sync(0xffffffffu, mbar_wait(&ctrl->full[s], uint32_t(gg / KS) & 1u, abort))) return false;
         tc_fence_after();
         const uint32_t st = smem_u32(sStage + s * F::STAGE);
-        const uint32_t s_col = tm_u + uint32_t((u & 1) * 2 * BQ);
+        const uint32_t s_col = tm_u + uint32_t((gg & 1) * 2 * BQ);
         uint64_t dq = kdesc<64>(st + O_Q), ddo = kdesc<64>(st + O_DO);
         asm volatile("" : "+l"(dq), "+l"(ddo));
 #pragma unroll
@@ -1004,16 +1085,16 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
         for (int kk = 0; kk < DP / 16; ++kk)  // dP^T = V dO^T
           mma_ss_elect(s_col + BQ, dV + kstep<64, 128>(kk), ddo + kstep<64, BQ>(kk), C::IDESC_KV_S, kk > 0 ? 1u : 0u);
-        tc_commit_elect(&ctrl->s_full[u & 1]);
+        tc_commit_elect(&ctrl->s_full[gg & 1]);
         __syncwarp();
         return true;
       };
-      auto issue_g = [&](int u) -> bool {
-        if (!__all_sync(0xffffffffu, mbar_wait(&ctrl->p_full[u & 1], uint32_t(u >> 1) & 1u, abort))) return false;
+      auto issue_g = [&](int gg, int u) -> bool {
+        if (!__all_sync(0xffffffffu, mbar_wait(&ctrl->p_full[gg & 1], uint32_t(gg >> 1) & 1u, abort))) return false;
         tc_fence_after();
-        const int s = u % KS;
+        const int s = gg % KS;
         const uint32_t st = smem_u32(sStage + s * F::STAGE);
-        const uint32_t p_col = tm_u + uint32_t((u & 1) * 2 * BQ);  // P^T bf16 over S^T; dS^T over dP^T
+        const uint32_t p_col = tm_u + uint32_t((gg & 1) * 2 * BQ);  // P^T bf16 over S^T; dS^T over dP^T
         uint64_t bdo = mndesc<64, BQ>(st + O_DO), bq = mndesc<64, BQ>(st + O_Q);
         asm volatile("" : "+l"(bdo), "+l"(bq));
 #pragma unroll
@@ -1034,40 +1115,67 @@ __global__ void __launch_bounds__(512, 1)
         __syncwarp();
         return true;
       };
-      if (ok) ok = issue_s(0);
-      if (ok && nb > 1) ok = issue_s(1);
-      for (int u = 0; u < nb && ok; ++u) {
-        ok = issue_g(u);
-        if (ok && u + 2 < nb) ok = issue_s(u + 2);
-      }
-      if (ok) {
+      for (int p = 0; ok; ++p) {
+        const int k = fused_read_item(ctrl, p, abort, ok);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok || k < 0) break;
+        const FusedItem w = fused_item(k, args);
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&ctrl->fixed_full, uint32_t(p) & 1u, abort)))) break;
+        tc_fence_after();
+        ok = issue_s(g, 0, w.j0);
+        if (ok && w.nb > 1) ok = issue_s(g + 1, 1, w.j0);
+        if (ok && w.nb <= 2) tc_commit_elect(&ctrl->fixed_empty);  // the item's last S is issued
+        for (int u = 0; u < w.nb && ok; ++u) {
+          if (u == 0 && p > 0 &&
+              !(ok = __all_sync(0xffffffffu, mbar_wait(&ctrl->acc_empty, uint32_t(p - 1) & 1u, abort))))
+            break;
+          ok = issue_g(g + u, u);
+          if (ok && u + 2 < w.nb) {
+            ok = issue_s(g + u + 2, u + 2, w.j0);
+            if (ok && u + 2 == w.nb - 1) tc_commit_elect(&ctrl->fixed_empty);
+          }
+        }
+        if (!ok) break;
         tc_commit_elect(&ctrl->acc_done);
         __syncwarp();
+        g += w.nb;
       }
       if (!ok && leader) atomicOr(args.flags, kFlagTimeout);
     } else if (warp == F::DQ_MMA_WARP) {
       // ------------------------------------------------ dq' MMA issuer
-      // Q(u): dq'^T = [K | phi_k]^T dS^T over the 128 keys, into TMEM buffer
-      // u mod NDQ once the readout has emptied it, as soon as block u's
-      // dS^T is in shared memory.
+      // Q(g): dq'^T = [K | phi_k]^T dS^T over the item's 128 keys, into TMEM
+      // buffer g mod NDQ once the readout has emptied it, as soon as block g's
+      // dS^T is in shared memory. After the item's last Q the fixed tiles are
+      // free (together with the MMA warp's commit after the last S).
       const uint32_t tm_u = __shfl_sync(0xffffffffu, tmem, 0);
-      bool ok = __all_sync(0xffffffffu, mbar_wait(&ctrl->fixed_full, 0, abort));
       const uint64_t aKT = mndesc<64, 128>(smem_u32(sK));  // [K | phi_k]^T, 128 rows
-      for (int u = 0; u < nb && ok; ++u) {
-        const int bq = u % F::NDQ;
-        ok = __all_sync(0xffffffffu, mbar_wait(&ctrl->p_full[u & 1], uint32_t(u >> 1) & 1u, abort) &&
-                                         (u < F::NDQ || mbar_wait(&ctrl->dq_free[bq],
-                                                                  uint32_t(u / F::NDQ - 1) & 1u, abort)));
-        if (!ok) break;
-        tc_fence_after();
-        uint64_t bds = mndesc<64, 128>(smem_u32(sDS + (u & 1) * F::TILE));
-        asm volatile("" : "+l"(bds));
+      bool ok = true;
+      int g = 0;
+      for (int p = 0; ok; ++p) {
+        const int k = fused_read_item(ctrl, p, abort, ok);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok || k < 0) break;
+        const FusedItem w = fused_item(k, args);
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&ctrl->fixed_full, uint32_t(p) & 1u, abort)))) break;
+        for (int u = 0; u < w.nb && ok; ++u, ++g) {
+          const int bq = g % F::NDQ;
+          ok = __all_sync(0xffffffffu, mbar_wait(&ctrl->p_full[g & 1], uint32_t(g >> 1) & 1u, abort) &&
+                                           (g < F::NDQ || mbar_wait(&ctrl->dq_free[bq],
+                                                                    uint32_t(g / F::NDQ - 1) & 1u, abort)));
+          if (!ok) break;
+          tc_fence_after();
+          uint64_t bds = mndesc<64, 128>(smem_u32(sDS + (g & 1) * F::TILE));
+          asm volatile("" : "+l"(bds));
 #pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk)
-          mma_ss_elect(tm_u + F::C_DQ + uint32_t(bq * BQ), aKT + mnstep<64>(kk), bds + mnstep<64>(kk), F::IDESC_DQ,
-                       kk > 0 ? 1u : 0u);
-        tc_commit_elect(&ctrl->dq_full[bq]);
-        tc_commit_elect(&ctrl->ds_free[u & 1]);
+          for (int kk = 0; kk < 128 / 16; ++kk)
+            mma_ss_elect(tm_u + F::C_DQ + uint32_t(bq * BQ), aKT + mnstep<64>(kk), bds + mnstep<64>(kk), F::IDESC_DQ,
+                         kk > 0 ? 1u : 0u);
+          tc_commit_elect(&ctrl->dq_full[bq]);
+          tc_commit_elect(&ctrl->ds_free[g & 1]);
+          __syncwarp();
+        }
+        if (!ok) break;
+        tc_commit_elect(&ctrl->fixed_empty);
         __syncwarp();
       }
       if (!ok && leader) atomicOr(args.flags, kFlagTimeout);
@@ -1087,33 +1195,40 @@ __global__ void __launch_bounds__(512, 1)
     constexpr int QR = F::QR;
     bool ok = true;
     int pc = 0;  // pieces issued
-    for (int u = 0; u < nb; ++u) {
-      const int bq = u % F::NDQ;
-      ok = named_bar_and(2, 128, mbar_wait(&ctrl->dq_full[bq], uint32_t(u / F::NDQ) & 1u, abort));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t v[64];
-      tmem_ld32(lane_base + F::C_DQ + uint32_t(bq * BQ), v);
-      tmem_ld32(lane_base + F::C_DQ + uint32_t(bq * BQ) + 32, v + 32);
-      tmem_ld_wait32(v);
-      tmem_ld_wait32(v + 32);
-      tc_fence_before();
-      mbar_arrive(&ctrl->dq_free[bq]);
-      const int q0 = (j0 + u) * BQ;
+    int g = 0;
+    for (int p = 0; ok; ++p) {
+      const int k = fused_read_item(ctrl, p, abort, ok);
+      ok = named_bar_and(2, 128, ok);
+      if (!ok || k < 0) break;
+      const FusedItem w = fused_item(k, args);
+      for (int u = 0; u < w.nb; ++u, ++g) {
+        const int bq = g % F::NDQ;
+        ok = named_bar_and(2, 128, mbar_wait(&ctrl->dq_full[bq], uint32_t(g / F::NDQ) & 1u, abort));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t v[64];
+        tmem_ld32(lane_base + F::C_DQ + uint32_t(bq * BQ), v);
+        tmem_ld32(lane_base + F::C_DQ + uint32_t(bq * BQ) + 32, v + 32);
+        tmem_ld_wait32(v);
+        tmem_ld_wait32(v + 32);
+        tc_fence_before();
+        mbar_arrive(&ctrl->dq_free[bq]);
+        const int q0 = (w.j0 + u) * BQ;
 #pragma unroll
-      for (int piece = 0; piece < BQ / QR; ++piece, ++pc) {
-        float *stg = sDQ + (pc & 1) * (QR * F::DQW);
-        if (issuer) bulk_wait_group_read1();  // the reduce that last read this tile is done reading
-        named_bar_sync(1, 128);
-        if (has_col) {
+        for (int piece = 0; piece < BQ / QR; ++piece, ++pc) {
+          float *stg = sDQ + (pc & 1) * (QR * F::DQW);
+          if (issuer) bulk_wait_group_read1();  // the reduce that last read this tile is done reading
+          named_bar_sync(1, 128);
+          if (has_col) {
 #pragma unroll
-          for (int i = 0; i < QR; ++i) stg[i * F::DQW + col] = __uint_as_float(v[QR * piece + i]);
-        }
-        fence_proxy_async_smem();
-        named_bar_sync(1, 128);
-        if (issuer) {
-          tma_reduce_add_3d(&tm_acc, stg, 0, q0 + QR * piece, bh);
-          bulk_commit_group();
+            for (int i = 0; i < QR; ++i) stg[i * F::DQW + col] = __uint_as_float(v[QR * piece + i]);
+          }
+          fence_proxy_async_smem();
+          named_bar_sync(1, 128);
+          if (issuer) {
+            tma_reduce_add_3d(&tm_acc, stg, 0, q0 + QR * piece, w.bh);
+            bulk_commit_group();
+          }
         }
       }
     }
@@ -1123,10 +1238,9 @@ __global__ void __launch_bounds__(512, 1)
     if (!ok && lane == 0) atomicOr(args.flags, kFlagTimeout);
   } else {
     setmaxnreg_inc<F::REG_COMPUTE>();
-    // ------------------------------- compute: warpgroup t takes blocks u = t mod 2
+    // ------------------------------- compute: warpgroup t takes blocks g = t mod 2
     const int t = warp >> 2, quarter = warp & 3;
     const int r_loc = quarter * 32 + lane;
-    const int krow = k0 + r_loc;  // this thread's key
     const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
     const uint32_t s_tm = lane_base + uint32_t(t * 2 * BQ), dp_tm = s_tm + BQ;
     // this thread's row of the dS^T tile (128-byte rows, 16-byte chunks swizzled by row)
@@ -1135,102 +1249,114 @@ __global__ void __launch_bounds__(512, 1)
     const float sl2 = args.scale_log2;
     const uint64_t sl2x2 = f2_pack(sl2, sl2);
     bool ok = true;
-    for (int u = t; u < nb; u += 2) {
-      const int s = u % KS;
-      ok = mbar_wait(&ctrl->full[s], uint32_t(u / KS) & 1u, abort) &&
-           mbar_wait(&ctrl->s_full[t], uint32_t(u >> 1) & 1u, abort) &&
-           (u < 2 || mbar_wait(&ctrl->ds_free[t], uint32_t((u >> 1) - 1) & 1u, abort));
-      if (!__all_sync(0xffffffffu, ok)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const uint8_t *st = sStage + s * F::STAGE;
-      const float *sL = reinterpret_cast<const float *>(st + O_L);
-      const float *sD = reinterpret_cast<const float *>(st + O_D);
-      const int q0 = (j0 + u) * BQ;
-      const bool diag = args.causal && q0 < k0 + 127;
-#pragma unroll
-      for (int c = 0; c < BQ / 32; ++c) {
-        uint32_t sx[32], dx[32];
-        tmem_ld32(s_tm + uint32_t(32 * c), sx);
-        tmem_ld32(dp_tm + uint32_t(32 * c), dx);
-        tmem_ld_wait32(sx);
-        tmem_ld_wait32(dx);
-        uint32_t pp[16], dd[16];
-#pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) {
-          const float4 l4 = *reinterpret_cast<const float4 *>(sL + 32 * c + 4 * e4);
-          const float4 d4 = *reinterpret_cast<const float4 *>(sD + 32 * c + 4 * e4);
-          const uint64_t l2[2] = {f2_pack(l4.x, l4.y), f2_pack(l4.z, l4.w)};
-          const uint64_t d2[2] = {f2_pack(d4.x, d4.y), f2_pack(d4.z, d4.w)};
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const int i = 4 * e4 + 2 * h2;
-            float a0, a1;
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(sx[i]), __uint_as_float(sx[i + 1])), sl2x2, l2[h2]), a0, a1);
-            float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
-            if (diag) {
-              const int cq = 32 * c + i;
-              if (q0 + cq < krow) p0 = 0.f;
-              if (q0 + cq + 1 < krow) p1 = 0.f;
-            }
-            const uint64_t p2 = f2_pack(p0, p1);
-            float g0, g1;
-            f2_unpack(f2_mul(p2, f2_sub(f2_pack(__uint_as_float(dx[i]), __uint_as_float(dx[i + 1])), d2[h2])), g0, g1);
-            pp[2 * e4 + h2] = pack_bf16x2(p0, p1);
-            dd[2 * e4 + h2] = pack_bf16x2(g0, g1);
-          }
+    int g0 = 0;  // the item's first block
+    for (int p = 0; ok; ++p) {
+      const int k = fused_read_item(ctrl, p, abort, ok);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok || k < 0) break;
+      const FusedItem w = fused_item(k, args);
+      const int krow = w.k0 + r_loc;  // this thread's key
+      for (int g = g0 + ((g0 & 1) != t ? 1 : 0); g < g0 + w.nb; g += 2) {
+        const int u = g - g0;
+        const int s = g % KS;
+        ok = mbar_wait(&ctrl->full[s], uint32_t(g / KS) & 1u, abort) &&
+             mbar_wait(&ctrl->s_full[t], uint32_t(g >> 1) & 1u, abort) &&
+             (g < 2 || mbar_wait(&ctrl->ds_free[t], uint32_t((g >> 1) - 1) & 1u, abort));
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
         }
-        tmem_st16(s_tm + uint32_t(16 * c), pp);
-        tmem_st16(dp_tm + uint32_t(16 * c), dd);
+        tc_fence_after();
+        const uint8_t *st = sStage + s * F::STAGE;
+        const float *sL = reinterpret_cast<const float *>(st + O_L);
+        const float *sD = reinterpret_cast<const float *>(st + O_D);
+        const int q0 = (w.j0 + u) * BQ;
+        const bool diag = args.causal && q0 < w.k0 + 127;
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj)
-          st_shared_v4(ds_row + (((uint32_t(4 * c + jj)) ^ sw) << 4), dd[4 * jj], dd[4 * jj + 1], dd[4 * jj + 2],
-                       dd[4 * jj + 3]);
+        for (int c = 0; c < BQ / 32; ++c) {
+          uint32_t sx[32], dx[32];
+          tmem_ld32(s_tm + uint32_t(32 * c), sx);
+          tmem_ld32(dp_tm + uint32_t(32 * c), dx);
+          tmem_ld_wait32(sx);
+          tmem_ld_wait32(dx);
+          uint32_t pp[16], dd[16];
+#pragma unroll
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 l4 = *reinterpret_cast<const float4 *>(sL + 32 * c + 4 * e4);
+            const float4 d4 = *reinterpret_cast<const float4 *>(sD + 32 * c + 4 * e4);
+            const uint64_t l2[2] = {f2_pack(l4.x, l4.y), f2_pack(l4.z, l4.w)};
+            const uint64_t d2[2] = {f2_pack(d4.x, d4.y), f2_pack(d4.z, d4.w)};
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int i = 4 * e4 + 2 * h2;
+              float a0, a1;
+              f2_unpack(f2_fma(f2_pack(__uint_as_float(sx[i]), __uint_as_float(sx[i + 1])), sl2x2, l2[h2]), a0, a1);
+              float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
+              if (diag) {
+                const int cq = 32 * c + i;
+                if (q0 + cq < krow) p0 = 0.f;
+                if (q0 + cq + 1 < krow) p1 = 0.f;
+              }
+              const uint64_t p2 = f2_pack(p0, p1);
+              float g0f, g1f;
+              f2_unpack(f2_mul(p2, f2_sub(f2_pack(__uint_as_float(dx[i]), __uint_as_float(dx[i + 1])), d2[h2])),
+                        g0f, g1f);
+              pp[2 * e4 + h2] = pack_bf16x2(p0, p1);
+              dd[2 * e4 + h2] = pack_bf16x2(g0f, g1f);
+            }
+          }
+          tmem_st16(s_tm + uint32_t(16 * c), pp);
+          tmem_st16(dp_tm + uint32_t(16 * c), dd);
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj)
+            st_shared_v4(ds_row + (((uint32_t(4 * c + jj)) ^ sw) << 4), dd[4 * jj], dd[4 * jj + 1], dd[4 * jj + 2],
+                         dd[4 * jj + 3]);
+        }
+        tmem_st_wait();
+        fence_proxy_async_smem();  // dS^T in shared memory, for the dq' MMA
+        tc_fence_before();
+        mbar_arrive(&ctrl->p_full[t]);
       }
-      tmem_st_wait();
-      fence_proxy_async_smem();  // dS^T in shared memory, for the dq' MMA
-      tc_fence_before();
-      mbar_arrive(&ctrl->p_full[t]);
-    }
-    if (ok) ok = mbar_wait(&ctrl->acc_done, 0, abort);
-    ok = __all_sync(0xffffffffu, ok);
-    if (ok) {
-      // epilogue: warpgroup 0 writes dV, warpgroup 1 dK, each half of dphi_k's
-      // columns; all TMEM loads are issued before one wait
+      if (!ok) break;
+      g0 += w.nb;
+      // epilogue of the item: warpgroup 0 writes dV, warpgroup 1 dK, each half
+      // of dphi_k's columns; the accumulators are handed back once loaded
+      ok = __all_sync(0xffffffffu, mbar_wait(&ctrl->acc_done, uint32_t(p) & 1u, abort));
+      if (!ok) break;
       tc_fence_after();
       const bool valid = krow < args.N;
       const int d_st = valid ? args.d : 0;
-      const size_t row_off = (size_t(bh) * args.N + (valid ? krow : 0)) * args.d;
+      const size_t row_off = (size_t(w.bh) * args.N + (valid ? krow : 0)) * args.d;
       uint16_t *dst = static_cast<uint16_t *>(t == 0 ? args.dV : args.dK) + row_off;
       const uint32_t acc_tm = lane_base + (t == 0 ? F::C_DV : F::C_DK);
       const float mul = t == 0 ? 1.f : args.scale;
-      uint32_t r[64], g[RG > 0 ? 32 : 1];
+      uint32_t r[64], gr[RG > 0 ? 32 : 1];
       tmem_ld32(acc_tm, r);
       tmem_ld32(acc_tm + 32, r + 32);
-      if constexpr (RG > 0) tmem_ld32(lane_base + F::C_DF + uint32_t(32 * t), g);
+      if constexpr (RG > 0) tmem_ld32(lane_base + F::C_DF + uint32_t(32 * t), gr);
       tmem_ld_wait32(r);
       tmem_ld_wait32(r + 32);
-      if constexpr (RG > 0) tmem_ld_wait32(g);
+      if constexpr (RG > 0) tmem_ld_wait32(gr);
+      tc_fence_before();
+      mbar_arrive(&ctrl->acc_empty);
 #pragma unroll
       for (int c0 = 0; c0 < DP; c0 += 16) store_row16_bf16(r + c0, mul, dst, c0, d_st);
       if constexpr (RG > 0) {
         // columns [32 t, 32 t + 32) of this key's dphi_k row, those below R
         float *frow =
-            factor_grad_row(args, args.dphi_k, args.dphi_k_part, b, h, bh, valid ? krow : 0) + 32 * t;
+            factor_grad_row(args, args.dphi_k, args.dphi_k_part, w.b, w.h, w.bh, valid ? krow : 0) + 32 * t;
         const int n_st = valid ? min(32, max(0, args.R - 32 * t)) : 0;
         const bool vec = (n_st & 3) == 0 && (reinterpret_cast<uintptr_t>(frow) & 15u) == 0;
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
           if (vec) {
             if (e < n_st)
-              *reinterpret_cast<float4 *>(frow + e) = make_float4(__uint_as_float(g[e]), __uint_as_float(g[e + 1]),
-                                                                   __uint_as_float(g[e + 2]), __uint_as_float(g[e + 3]));
+              *reinterpret_cast<float4 *>(frow + e) = make_float4(
+                  __uint_as_float(gr[e]), __uint_as_float(gr[e + 1]), __uint_as_float(gr[e + 2]), __uint_as_float(gr[e + 3]));
           } else {
 #pragma unroll
             for (int x = 0; x < 4; ++x)
-              if (e + x < n_st) frow[e + x] = __uint_as_float(g[e + x]);
+              if (e + x < n_st) frow[e + x] = __uint_as_float(gr[e + x]);
           }
         }
       }
@@ -1245,7 +1371,6 @@ __global__ void __launch_bounds__(512, 1)
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
-
 
 namespace {
 
@@ -1279,7 +1404,12 @@ cudaError_t launch_bwd_fused(const BwdMaps &m, const BwdArgs &a, cudaStream_t st
       return e;
     ready[dev].store(1, std::memory_order_release);
   }
-  const unsigned grid = unsigned((long long)a.n_kv * a.B * a.H);
+  // persistent: one CTA per SM (the TMEM allocation and the shared memory
+  // admit one), never more than there are work items
+  int sms = 0;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const long long items = (long long)a.n_kv * a.B * a.H;
+  const unsigned grid = unsigned(std::min<long long>(items, sms));
   return launch_programmatic(kern, dim3(grid), dim3(F::THREADS), F::SMEM, stream, m.k, m.v, m.fk, m.gk, m.q_blk,
                              m.do_blk, m.fq_blk, m.gq_blk, m.acc, a);
 }

@@ -500,8 +500,9 @@ __global__ void __launch_bounds__(256) bwd_rows_kernel(long long rows, int N, in
                                                        const __nv_bfloat16 *__restrict__ dO,
                                                        const float *__restrict__ LSE, float *__restrict__ nlse2,
                                                        float *__restrict__ delta, float *__restrict__ dq_acc,
-                                                       int dqw) {
+                                                       int dqw, unsigned int *__restrict__ sched) {
   griddep_launch_dependents();  // the gradient kernel may start its set-up now
+  if (sched && blockIdx.x == 0 && threadIdx.x == 0) *sched = 0u;
   const long long w = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 3;  // row
   const int sub = threadIdx.x & 7;
   if (w >= rows) return;  // whole 8-thread groups leave together
@@ -559,13 +560,13 @@ __global__ void prep_grad_factors_kernel(int N, int R, int RG, int fac_H, const 
 }
 
 cudaError_t launch_bwd_rows(int BH, int N, int Npad, int d, const void *O, const void *dO, const float *LSE,
-                            float *nlse2, float *delta, float *acc, int dqw, cudaStream_t s) {
+                            float *nlse2, float *delta, float *acc, int dqw, unsigned int *sched, cudaStream_t s) {
   const long long rows = (long long)BH * Npad;  // a multiple of 128: full warps
   const long long blocks = (rows * 8 + 255) / 256;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
   bwd_rows_kernel<<<unsigned(blocks), 256, 0, s>>>(rows, N, Npad, d, static_cast<const __nv_bfloat16 *>(O),
                                                    static_cast<const __nv_bfloat16 *>(dO), LSE, nlse2, delta, acc,
-                                                   dqw);
+                                                   dqw, sched);
   return cudaGetLastError();
 }
 

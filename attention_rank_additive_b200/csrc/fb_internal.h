@@ -111,6 +111,7 @@ struct BwdArgs {
   int64_t phi_bs, phi_hs;  // element strides of the factor tensors
   int fac_B, fac_H;        // factor slices: B or 1, H or 1
   float *dqacc;            // fused kernel: fp32 [BH, Npad, 64 + RG] accumulator of dq' = dS [K | phi_k]
+  unsigned int *sched;     // fused kernel: work counter (zeroed by the per-row pass)
   int *flags;
 };
 
@@ -146,9 +147,10 @@ cudaError_t launch_bwd_dq_convert(int B, int H, int N, int Npad, int d, int R, i
                                   int fac_H, cudaStream_t s);
 cudaError_t bwd_launch(const BwdPlan &p, const BwdMaps &maps, const BwdArgs &a, cudaStream_t stream);
 // nlse2 = -LSE * log2(e) and delta = rowsum(dO * O) per row, padded to Npad.
-// With acc != nullptr, also zeroes the fused kernel's accumulator rows [BH, Npad, dqw].
+// With acc != nullptr, also zeroes the fused kernel's accumulator rows [BH, Npad, dqw]
+// and its work counter *sched.
 cudaError_t launch_bwd_rows(int BH, int N, int Npad, int d, const void *O, const void *dO, const float *LSE,
-                            float *nlse2, float *delta, float *acc, int dqw, cudaStream_t s);
+                            float *nlse2, float *delta, float *acc, int dqw, unsigned int *sched, cudaStream_t s);
 // bf16 copies of the factors [FB, N, RG] (zero-padded).
 cudaError_t launch_prep_grad_factors(int N, int R, int RG, const float *phi_q, const float *phi_k, int64_t bs,
                                      int64_t hs, int fac_B, int fac_H, void *gq, void *gk, cudaStream_t s);

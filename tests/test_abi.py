@@ -345,20 +345,21 @@ def test_backward_workspace_and_argument_errors():
     """fb_attn_bwd: the workspace covers the forward's factor tiles, the bf16
     factor copies, two fp32 rows per (b, h, padded query) and a 128-column
     fp32 accumulator row per (b, h, padded query) (the fused kernel's dq', or
-    the two-kernel path's per-head dphi_q rows); every argument error returns
-    before a launch."""
+    the two-kernel path's per-head dphi_q rows) and the fused kernel's work
+    counter; every argument error returns before a launch."""
     al = lambda x: (x + 255) // 256 * 256
     B, H, N, R = 2, 3, 200, 8
     Npad = 256
     acc = al(B * H * Npad * 128 * 4)
     fwd = fb.fb_attn_workspace_bytes(B, H, N, R, H * N * R, N * R)
+    sched = 256  # the fused kernel's work counter
     assert fb.fb_attn_bwd_workspace_bytes(B, H, N, R, H * N * R, N * R) == \
-        fwd + 2 * al(B * H * N * 16 * 2) + 2 * al(B * H * Npad * 4) + acc
+        fwd + 2 * al(B * H * N * 16 * 2) + 2 * al(B * H * Npad * 4) + acc + sched
     # broadcast factors: one factor slice, plus per-head partial dphi_k rows
     assert fb.fb_attn_bwd_workspace_bytes(B, H, N, R, 0, 0) == \
         fb.fb_attn_workspace_bytes(B, H, N, R, 0, 0) + 2 * al(N * 16 * 2) + 2 * al(B * H * Npad * 4) + \
-        acc + al(B * H * N * R * 4)
-    assert fb.fb_attn_bwd_workspace_bytes(B, H, N, 0, 0, 0) == 2 * al(B * H * Npad * 4) + acc
+        acc + al(B * H * N * R * 4) + sched
+    assert fb.fb_attn_bwd_workspace_bytes(B, H, N, 0, 0, 0) == 2 * al(B * H * Npad * 4) + acc + sched
     assert fb.fb_attn_bwd_workspace_bytes(B, H, N, 129, 0, 0) == 0
     assert fb.fb_attn_bwd_workspace_bytes(0, H, N, R, 0, 0) == 0
     need = fb.fb_attn_bwd_workspace_bytes(1, 2, 128, R, 2 * 128 * R, 128 * R)
