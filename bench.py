@@ -221,9 +221,9 @@ def kernel_source_sha(sources=KERNEL_SOURCES) -> str:
 
 
 def profiled_traffic(cfg_idx: int):
-    """dram bytes per launch of the fused kernel (per call of the two gradient
-    kernels for the backward) from the committed ncu summary, if it was taken
-    on the current kernel source and this workload; else None."""
+    """dram bytes per launch of the fused kernel (of the fused backward kernel
+    for the backward) from the committed ncu summary, if it was taken on the
+    current kernel source and this workload; else None."""
     c = si.CONFIGS[cfg_idx]
     bwd = bool(c.get("bwd"))
     path = os.path.join(ROOT, "profiles", f"attn_{'bwd' if bwd else 'fwd'}_sm100_{c['name']}.md")
@@ -335,8 +335,9 @@ class GpuWorkload:
         self.launches_per_step = (2 if self.neural else
                                   (2 if self.mul or (Rk > 0 and c["dtype"] == "bf16") else 1))
         self.bwd = bool(c.get("bwd"))
-        if self.bwd:  # factor preparation, bf16 factor copies, per-row terms, two gradient kernels, and
-            # the reduction of per-head factor gradients when a factor slice serves several heads
+        if self.bwd:  # factor preparation, bf16 factor copies, per-row terms, the gradient kernels (the
+            # fused kernel and its dQ conversion at head dim 64; else the dK/dV and dQ kernels), and the
+            # reduction of per-head factor gradients when a factor slice serves several heads
             shared = Rk > 0 and (self.bs == 0 and B > 1 or self.hs == 0 and H > 1)
             self.launches_per_step = (5 + (1 if shared else 0)) if Rk > 0 else 3
 
@@ -699,8 +700,10 @@ def run_ours(args, rank: int, world: int, local: int):
                      "frac": round(achieved / peak_tf, 4), "traffic": traffic,
                      "kernel": ("prep_mul_bias + attn_fwd_sm100" if w.mul else
                                 ("neural_prep + attn_fwd_sm100" if w.neural else
-                                 ("bwd preparation (3) + attn_bwd_dkdv_sm100 + attn_bwd_dq_sm100 + factor-gradient "
-                                  "reduction" if w.bwd
+                                 ("bwd preparation (3) + attn_bwd_fused_sm100 + dQ conversion + factor-gradient "
+                                  "reduction" if w.bwd and c["d"] > 32 and c["d"] <= 64
+                                  else "bwd preparation (3) + attn_bwd_dkdv_sm100 + attn_bwd_dq_sm100 + "
+                                       "factor-gradient reduction" if w.bwd
                                   else "attn_fwd_sm100"))),
                      "peak_kind": peak_kind,
                      "kernel_ms": round(kern_ms, 5)},
