@@ -484,48 +484,86 @@ __global__ void rows_kernel(int N, int l, int R, const float *__restrict__ A, co
   }
 }
 
-// sums[h] += (||B - phi_q phi_k^T||_F^2, ||B||_F^2), fp64; one warp per row,
-// phi_k staged 256 rows at a time.
-__global__ void __launch_bounds__(512) err_kernel(int N, int R, const float *__restrict__ B,
+// sums[h] += (||B - phi_q phi_k^T||_F^2, ||B||_F^2). A CTA takes 32 rows and
+// 256 * CPT columns of B: each thread keeps its CPT columns of phi_k in
+// registers and walks the rows (phi_q rows from shared memory, broadcast
+// 16-byte loads), 4 rows' loads of B in flight at a time. The squares of a
+// thread's CPT columns are summed in fp32 (at most 4 terms), everything
+// above in fp64.
+constexpr int kErrRows = 32;
+template <int RT, int CPT>
+__global__ void __launch_bounds__(256) err_kernel(int N, int R, const float *__restrict__ B,
                                                   const float *__restrict__ pq, const float *__restrict__ pk,
                                                   double *__restrict__ sums) {
-  __shared__ float ks[kMaxL][257];
-  const int h = blockIdx.y;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long i = (long long)blockIdx.x * 16 + warp;
+  __shared__ __align__(16) float qs[kErrRows][RT];
+  const int h = blockIdx.z;
+  const long long i0 = (long long)blockIdx.y * kErrRows;
+  const long long c = ((long long)blockIdx.x * 256 + threadIdx.x) * CPT;  // this thread's first column
   const float *Bh = B + (long long)h * N * N;
-  float q[kMaxL];
+  for (int e = threadIdx.x; e < kErrRows * RT; e += 256) {
+    const int rr = e / RT, r = e - rr * RT;
+    const long long i = i0 + rr;
+    qs[rr][r] = (i < N && r < R) ? pq[((long long)h * N + i) * R + r] : 0.f;
+  }
+  float k[CPT][RT];
 #pragma unroll
-  for (int r = 0; r < kMaxL; ++r) q[r] = (i < N && r < R) ? pq[((long long)h * N + i) * R + r] : 0.f;
+  for (int q = 0; q < CPT; ++q)
+#pragma unroll
+    for (int r = 0; r < RT; ++r) k[q][r] = (c + q < N && r < R) ? pk[((long long)h * N + c + q) * R + r] : 0.f;
+  __syncthreads();
+  const bool vec = (N % CPT) == 0 && (reinterpret_cast<uintptr_t>(B) % (CPT * 4)) == 0 && c + CPT <= N;
   double e2 = 0.0, f2 = 0.0;
-  for (int c0 = 0; c0 < N; c0 += 256) {
-    for (int e = threadIdx.x; e < 256 * R; e += blockDim.x) {
-      const int t = e / R, r = e - t * R;
-      ks[r][t] = c0 + t < N ? pk[((long long)h * N + c0 + t) * R + r] : 0.f;
-    }
-    __syncthreads();
-    if (i < N) {
-      for (int m = 0; m < 8; ++m) {
-        const int t = lane + 32 * m;
-        if (c0 + t >= N) break;
-        float pred = 0.f;
+  for (int rb = 0; rb < kErrRows; rb += 4) {
+    float bv[4][CPT];
 #pragma unroll
-        for (int r = 0; r < kMaxL; ++r)
-          if (r < R) pred = fmaf(q[r], ks[r][t], pred);
-        const float bv = Bh[i * N + c0 + t];
-        const double dv = double(bv) - double(pred);
-        e2 += dv * dv;
-        f2 += double(bv) * double(bv);
+    for (int u = 0; u < 4; ++u) {
+      const long long i = i0 + rb + u;
+      if (i < N && vec) {
+        if constexpr (CPT == 4) {
+          const float4 b4 = *reinterpret_cast<const float4 *>(Bh + i * N + c);
+          bv[u][0] = b4.x, bv[u][1] = b4.y, bv[u][2] = b4.z, bv[u][3] = b4.w;
+        } else {
+          const float2 b2 = *reinterpret_cast<const float2 *>(Bh + i * N + c);
+          bv[u][0] = b2.x, bv[u][1] = b2.y;
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < CPT; ++q) bv[u][q] = (i < N && c + q < N) ? Bh[i * N + c + q] : 0.f;
       }
     }
-    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      float pred[CPT];
+#pragma unroll
+      for (int q = 0; q < CPT; ++q) pred[q] = 0.f;
+#pragma unroll
+      for (int r = 0; r < RT; r += 4) {
+        const float4 q4 = *reinterpret_cast<const float4 *>(&qs[rb + u][r]);
+#pragma unroll
+        for (int q = 0; q < CPT; ++q) {
+          pred[q] = fmaf(q4.x, k[q][r], pred[q]);
+          pred[q] = fmaf(q4.y, k[q][r + 1], pred[q]);
+          pred[q] = fmaf(q4.z, k[q][r + 2], pred[q]);
+          pred[q] = fmaf(q4.w, k[q][r + 3], pred[q]);
+        }
+      }
+      float ee = 0.f, ff = 0.f;  // rows or columns past N hold zeros
+#pragma unroll
+      for (int q = 0; q < CPT; ++q) {
+        const float dv = bv[u][q] - pred[q];
+        ee = fmaf(dv, dv, ee);
+        ff = fmaf(bv[u][q], bv[u][q], ff);
+      }
+      e2 += double(ee);
+      f2 += double(ff);
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     e2 += __shfl_xor_sync(0xffffffffu, e2, o);
     f2 += __shfl_xor_sync(0xffffffffu, f2, o);
   }
-  if (lane == 0 && i < N) {
+  if ((threadIdx.x & 31u) == 0) {
     atomicAdd(&sums[2 * h], e2);
     atomicAdd(&sums[2 * h + 1], f2);
   }
@@ -599,7 +637,7 @@ extern "C" int fb_svd_factors_device(int H, int N, int R, int oversample, int po
   double *sums = sig2 + H;
   double *out = sums + 2 * H;
 
-  const dim3 rows16((N + 15) / 16, H), rows32((N + 31) / 32, H), cols1024((N + 1023) / 1024, H, (N + 511) / 512),
+  const dim3 rows32((N + 31) / 32, H), cols1024((N + 1023) / 1024, H, (N + 511) / 512),
       rows256((N + 255) / 256, H);
   const double u = 1.1102230246251565e-16;  // 2^-53: unit roundoff of the fp64 Gram matrices
   const double shift_coef = 11.0 * (double(N) * l + double(l) * (l + 1)) * u;
@@ -640,7 +678,13 @@ extern "C" int fb_svd_factors_device(int H, int N, int R, int oversample, int po
   rows_kernel<<<rows256, 256, 0, st>>>(N, l, R, P0, Ck, phi_k);
   if (err_energy) {
     if (cudaMemsetAsync(sums, 0, size_t(2) * H * sizeof(double), st) != cudaSuccess) return FB_ERR_CUDA;
-    err_kernel<<<rows16, 512, 0, st>>>(N, R, bias, phi_q, phi_k, sums);
+    const int rows_err = (N + kErrRows - 1) / kErrRows;
+    if (R <= 8)
+      err_kernel<8, 4><<<dim3((N + 1023) / 1024, rows_err, H), 256, 0, st>>>(N, R, bias, phi_q, phi_k, sums);
+    else if (R <= 16)
+      err_kernel<16, 4><<<dim3((N + 1023) / 1024, rows_err, H), 256, 0, st>>>(N, R, bias, phi_q, phi_k, sums);
+    else
+      err_kernel<32, 2><<<dim3((N + 511) / 512, rows_err, H), 256, 0, st>>>(N, R, bias, phi_q, phi_k, sums);
     finish_kernel<<<hb, 32, 0, st>>>(H, sums, sig2, out);
     if (cudaMemcpyAsync(err_energy, out, size_t(2) * H * sizeof(double), cudaMemcpyDeviceToDevice, st) !=
         cudaSuccess)
