@@ -85,14 +85,25 @@ __global__ void gauss_kernel(int H, int N, int l, uint64_t seed, float *__restri
 }
 
 // Y[h] = B[h] X[h]: B [N, N] row-major, X and Y [l][N]. A CTA of 8 warps
-// takes 32 rows of B, each warp 4 of them; X is staged in shared memory 256
-// columns at a time and each lane works on 4 consecutive columns, so one
-// 16-byte shared load of X feeds 16 FMAs (4 rows x 4 columns) and each row's
-// 16-byte loads of B are coalesced across the warp. The per-lane partial
-// sums are reduced across the warp at the end.
-constexpr int kBxRows = 4;  // rows per warp
-__global__ void __launch_bounds__(256) bx_kernel(int N, int l, const float *__restrict__ B,
-                                                 const float *__restrict__ X, float *__restrict__ Y) {
+// takes 8 kBxRows rows of B, each warp kBxRows of them; X is staged in shared
+// memory 256 columns at a time and each lane works on 4 consecutive columns,
+// so one 16-byte shared load of X feeds 4 kBxRows FMAs and each row's 16-byte
+// loads of B are coalesced across the warp. The per-lane partial sums are
+// reduced across the warp at the end.
+// Rows of B per warp (B X) and columns of B per thread (B^T X): 2 each keeps
+// a thread under 128 registers, so that two CTAs share an SM (4 each: one
+// CTA of 8 warps per SM, about 4 % slower over the whole SVD).
+#ifndef FB_SVD_BX_ROWS
+#define FB_SVD_BX_ROWS 2
+#endif
+#ifndef FB_SVD_BTX_COLS
+#define FB_SVD_BTX_COLS 2
+#endif
+constexpr int kBxRows = FB_SVD_BX_ROWS;  // rows per warp
+constexpr int kBtxCols = FB_SVD_BTX_COLS;  // columns per thread
+__global__ void __launch_bounds__(256, kBxRows <= 2 ? 2 : 1) bx_kernel(int N, int l, const float *__restrict__ B,
+                                                                      const float *__restrict__ X,
+                                                                      float *__restrict__ Y) {
   __shared__ __align__(16) float xs[kMaxL][256];
   const int h = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -164,22 +175,24 @@ __global__ void __launch_bounds__(256) bx_kernel(int N, int l, const float *__re
 }
 
 // Z[h] += B[h]^T X[h] over one slice of 512 rows of B (Z zeroed beforehand):
-// each thread takes 4 consecutive columns of B (256 threads, 1024 columns per
-// CTA) and walks the slice 4 rows at a time, X staged in shared memory 64 rows
-// at a time, so that one 16-byte broadcast load of X (4 rows of one column of
-// X) feeds 16 FMAs; grid (column blocks, H, row slices), partial sums added
-// with atomics.
-__global__ void __launch_bounds__(256) btx_kernel(int N, int l, const float *__restrict__ B,
-                                                  const float *__restrict__ X, float *__restrict__ Z) {
+// each thread takes kBtxCols consecutive columns of B (256 threads per CTA)
+// and walks the slice 4 rows at a time, X staged in shared memory 64 rows at
+// a time, so that one 16-byte broadcast load of X (4 rows of one column of X)
+// feeds 4 kBtxCols FMAs; grid (column blocks, H, row slices), partial sums
+// added with atomics.
+__global__ void __launch_bounds__(256, kBtxCols <= 2 ? 2 : 1) btx_kernel(int N, int l, const float *__restrict__ B,
+                                                                         const float *__restrict__ X,
+                                                                         float *__restrict__ Z) {
+  constexpr int CQ = kBtxCols;
   __shared__ __align__(16) float xs[kMaxL][64];
   const int h = blockIdx.y;
-  const long long c = ((long long)blockIdx.x * 256 + threadIdx.x) * 4;  // first of this thread's 4 columns
+  const long long c = ((long long)blockIdx.x * 256 + threadIdx.x) * CQ;  // first of this thread's CQ columns
   const float *Bh = B + (long long)h * N * N;
   const float *Xh = X + (long long)h * l * N;
-  const bool vec = (N & 3) == 0 && (reinterpret_cast<uintptr_t>(B) & 15u) == 0;
-  float acc[4][kMaxL];
+  const bool vec = (N % CQ) == 0 && (reinterpret_cast<uintptr_t>(B) % (4 * CQ)) == 0;
+  float acc[CQ][kMaxL];
 #pragma unroll
-  for (int q = 0; q < 4; ++q)
+  for (int q = 0; q < CQ; ++q)
 #pragma unroll
     for (int j = 0; j < kMaxL; ++j) acc[q][j] = 0.f;
   const int i_end = min(N, int(blockIdx.z + 1) * 512);
@@ -190,34 +203,39 @@ __global__ void __launch_bounds__(256) btx_kernel(int N, int l, const float *__r
       const int rmax = min(64, i_end - i0);
       // B values of 4 rows x this thread's 4 columns; the next group's are
       // loaded before the current group's FMAs
-      auto load4 = [&](int r, float (&bv)[4][4]) {
+      auto load4 = [&](int r, float (&bv)[4][CQ]) {
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const long long i = i0 + r + u;
-          if (r + u < rmax && vec && c + 3 < N) {
-            const float4 b4 = *reinterpret_cast<const float4 *>(Bh + i * N + c);
-            bv[u][0] = b4.x, bv[u][1] = b4.y, bv[u][2] = b4.z, bv[u][3] = b4.w;
+          if (r + u < rmax && vec && c + CQ - 1 < N) {
+            if constexpr (CQ == 4) {
+              const float4 b4 = *reinterpret_cast<const float4 *>(Bh + i * N + c);
+              bv[u][0] = b4.x, bv[u][1] = b4.y, bv[u][2] = b4.z, bv[u][3] = b4.w;
+            } else {
+              const float2 b2 = *reinterpret_cast<const float2 *>(Bh + i * N + c);
+              bv[u][0] = b2.x, bv[u][1] = b2.y;
+            }
           } else {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) bv[u][q] = (r + u < rmax && c + q < N) ? Bh[i * N + c + q] : 0.f;
+            for (int q = 0; q < CQ; ++q) bv[u][q] = (r + u < rmax && c + q < N) ? Bh[i * N + c + q] : 0.f;
           }
         }
       };
-      float nb[4][4];
+      float nb[4][CQ];
       load4(0, nb);
       for (int r = 0; r < rmax; r += 4) {
-        float bv[4][4];  // [row][column]
+        float bv[4][CQ];  // [row][column]
 #pragma unroll
         for (int u = 0; u < 4; ++u)
 #pragma unroll
-          for (int q = 0; q < 4; ++q) bv[u][q] = nb[u][q];
+          for (int q = 0; q < CQ; ++q) bv[u][q] = nb[u][q];
         if (r + 4 < rmax) load4(r + 4, nb);
 #pragma unroll
         for (int j = 0; j < kMaxL; ++j) {
           if (j < l) {
             const float4 x4 = *reinterpret_cast<const float4 *>(&xs[j][r]);  // rows r .. r+3 (zero past the slice)
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < CQ; ++q) {
               float a = acc[q][j];
               a = fmaf(bv[0][q], x4.x, a);
               a = fmaf(bv[1][q], x4.y, a);
@@ -232,7 +250,7 @@ __global__ void __launch_bounds__(256) btx_kernel(int N, int l, const float *__r
     __syncthreads();
   }
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
+  for (int q = 0; q < CQ; ++q) {
 #pragma unroll
     for (int j = 0; j < kMaxL; ++j)  // compile-time indices keep acc in registers
       if (j < l && c + q < N) atomicAdd(&Z[(long long)h * l * N + (long long)j * N + c + q], acc[q][j]);
@@ -261,8 +279,12 @@ __global__ void __launch_bounds__(512) gram_kernel(int N, int l, const float *__
       ++a;
     }
     const int b = a + rem;
-    double s = 0.0;
-    for (int t = 0; t < 256; ++t) s += double(as[a][t]) * double(as[b][t]);
+    double s4[4] = {0.0, 0.0, 0.0, 0.0};  // independent chains
+    for (int t = 0; t < 256; t += 4) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) s4[u] += double(as[a][t + u]) * double(as[b][t + u]);
+    }
+    const double s = (s4[0] + s4[1]) + (s4[2] + s4[3]);
     atomicAdd(&G[(long long)h * l * l + a * l + b], s);
     if (a != b) atomicAdd(&G[(long long)h * l * l + b * l + a], s);
   }
@@ -271,54 +293,71 @@ __global__ void __launch_bounds__(512) gram_kernel(int N, int l, const float *__
 // T[h] = R^{-1} with R^T R = G + shift I (R upper triangular, Cholesky in
 // fp64), so that A T has orthonormal columns. A pivot that is not positive
 // (a column dependent on the previous ones) zeroes that column of T.
-// One warp per head: lane i updates entry i of the current row of R, and
-// lane j solves column j of the inverse.
-__global__ void chol_kernel(int H, int N, int l, double shift_coef, const double *__restrict__ G,
-                            double *__restrict__ T) {
-  __shared__ double Rm[kMaxL][kMaxL], Ti[kMaxL][kMaxL], g[kMaxL * kMaxL];
-  __shared__ bool dead[kMaxL];
+// One warp per head, all in registers: lane i holds row i of the (trailing)
+// matrix and, after step j, R[j][i]; each step broadcasts row j of R with
+// shuffles and updates the trailing rows (right-looking). Then lane j
+// back-substitutes column j of the inverse.
+__device__ __forceinline__ double shfl_d(double v, int src) { return __shfl_sync(0xffffffffu, v, src); }
+__global__ void __launch_bounds__(32) chol_kernel(int H, int N, int l, double shift_coef,
+                                                  const double *__restrict__ G, double *__restrict__ T) {
   const int h = blockIdx.x, lane = threadIdx.x;
   if (h >= H) return;
-  for (int e = lane; e < l * l; e += 32) g[e] = G[(long long)h * l * l + e];  // the Gram matrix, once
-  __syncwarp();
-  double *t = T + (long long)h * l * l;
-  double tr = 0.0;
-  for (int a = 0; a < l; ++a) tr += g[a * l + a];
+  const double *g = G + (long long)h * l * l;
+  double a[kMaxL];  // row `lane` of G + shift I, then of the trailing matrix
+#pragma unroll
+  for (int k = 0; k < kMaxL; ++k) a[k] = (lane < l && k < l) ? g[lane * l + k] : 0.0;
+  double diag = 0.0;
+#pragma unroll
+  for (int k = 0; k < kMaxL; ++k)
+    if (k == lane) diag = a[k];
+  double tr = diag;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) tr += __shfl_xor_sync(0xffffffffu, tr, o);
   const double shift = shift_coef * tr;
-  for (int i = 0; i < l; ++i) Rm[i][lane] = 0.0;
-  __syncwarp();
-  for (int j = 0; j < l; ++j) {
-    double dj = g[j * l + j] + shift;
-    for (int k = 0; k < j; ++k) dj -= Rm[k][j] * Rm[k][j];
-    const bool dj_dead = !(dj > 1e-300 && dj > 1e-14 * (g[j * l + j] + shift));
-    const double rjj = dj_dead ? 0.0 : sqrt(dj);
-    const int i = lane;  // row j of R, entry i > j
-    double v = 0.0;
-    if (i > j && i < l) {
-      v = g[j * l + i];
-      for (int k = 0; k < j; ++k) v -= Rm[k][j] * Rm[k][i];
-    }
-    __syncwarp();
-    if (lane == 0) {
-      dead[j] = dj_dead;
-      Rm[j][j] = rjj;
-    }
-    if (i > j && i < l) Rm[j][i] = dj_dead ? 0.0 : v / rjj;
-    __syncwarp();
-  }
-  // inverse of the upper triangular Rm: lane j back-substitutes column j
-  const int j = lane;
-  if (j < l) {
-    for (int i = l - 1; i >= 0; --i) {
-      if (i > j || dead[i]) {
-        Ti[i][j] = 0.0;
-        continue;
+  const double gdiag = diag + shift;  // this row's pivot before elimination
+#pragma unroll
+  for (int k = 0; k < kMaxL; ++k)
+    if (k == lane) a[k] += shift;
+  double r[kMaxL];  // r[j] = R[j][lane]
+  uint32_t dead = 0u;  // bit j: pivot j not positive (the same in every lane)
+#pragma unroll
+  for (int j = 0; j < kMaxL; ++j) {
+    r[j] = 0.0;
+    if (j < l) {
+      const double ajj = shfl_d(a[j], j);
+      const double gjj = shfl_d(gdiag, j);
+      const bool dj_dead = !(ajj > 1e-300 && ajj > 1e-14 * gjj);
+      if (dj_dead) dead |= 1u << j;
+      const double rjj = dj_dead ? 0.0 : sqrt(ajj);
+      // lane i > j holds A[i][j] = A[j][i]
+      const double rji = lane == j ? rjj : ((lane > j && lane < l && !dj_dead) ? a[j] / rjj : 0.0);
+      r[j] = rji;
+#pragma unroll
+      for (int k = j + 1; k < kMaxL; ++k) {
+        const double rjk = shfl_d(rji, k);
+        if (lane > j) a[k] -= rji * rjk;
       }
-      double v = (i == j) ? 1.0 : 0.0;
-      for (int k = i + 1; k <= j; ++k) v -= Rm[i][k] * Ti[k][j];
-      Ti[i][j] = v / Rm[i][i];
     }
-    for (int i = 0; i < l; ++i) t[i * l + j] = Ti[i][j];
+  }
+  // inverse of R: lane j back-substitutes column j (t[i] = T[i][lane])
+  double t[kMaxL];
+#pragma unroll
+  for (int i = 0; i < kMaxL; ++i) t[i] = 0.0;
+#pragma unroll
+  for (int i = kMaxL - 1; i >= 0; --i) {
+    if (i < l) {
+      const double rii = shfl_d(r[i], i);
+      double v = (i == lane) ? 1.0 : 0.0;
+#pragma unroll
+      for (int k = i + 1; k < kMaxL; ++k) v -= shfl_d(r[i], k) * t[k];  // R[i][k], zero past l
+      t[i] = (i <= lane && !((dead >> i) & 1u)) ? v / rii : 0.0;
+    }
+  }
+  if (lane < l) {
+    double *out = T + (long long)h * l * l;
+#pragma unroll
+    for (int i = 0; i < kMaxL; ++i)
+      if (i < l) out[i * l + lane] = t[i];
   }
   (void)N;
 }
@@ -637,7 +676,8 @@ extern "C" int fb_svd_factors_device(int H, int N, int R, int oversample, int po
   double *sums = sig2 + H;
   double *out = sums + 2 * H;
 
-  const dim3 rows32((N + 31) / 32, H), cols1024((N + 1023) / 1024, H, (N + 511) / 512),
+  const dim3 rows32((N + 8 * kBxRows - 1) / (8 * kBxRows), H),
+      cols1024((N + 256 * kBtxCols - 1) / (256 * kBtxCols), H, (N + 511) / 512),
       rows256((N + 255) / 256, H);
   const double u = 1.1102230246251565e-16;  // 2^-53: unit roundoff of the fp64 Gram matrices
   const double shift_coef = 11.0 * (double(N) * l + double(l) * (l + 1)) * u;
