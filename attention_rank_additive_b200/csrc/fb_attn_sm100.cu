@@ -267,13 +267,33 @@ struct WorkItem {
   int q0[2], nk[2], first[2], n_steps;
 };
 
-template <int QT>
+template <int QT, bool GROUPED>
 __device__ __forceinline__ WorkItem make_item(int k, const FwdArgs &a) {
-  // Heaviest query groups first (causal work grows with the query index).
+  // Items in groups of head_group heads, and within a group heaviest query
+  // groups first (causal work grows with the query index): the CTAs at work
+  // then share few heads, whose K and V stay in L2 while every query group of
+  // the head reads them. One group (the plain heaviest-first order) when all
+  // heads' K and V fit in L2 anyway. Only the head-dim-128 kernels carry the
+  // grouped form (GROUPED): at the smaller head dims all heads' K and V fit
+  // for the sequence lengths at hand, and the extra code cost the d = 16
+  // kernel 3 % through register allocation.
   const int BH = a.B * a.H;
   WorkItem w;
-  w.bh = k % BH;
-  const int qg = a.n_cta_q - 1 - k / BH;
+  const int G = GROUPED ? a.head_group : BH;
+  int qg;
+  if (!GROUPED || G >= BH) {
+    w.bh = k % BH;
+    qg = a.n_cta_q - 1 - k / BH;
+  } else {
+    const int per_group = G * a.n_cta_q;
+    const int n_groups = (BH + G - 1) / G;
+    const int grp = min(k / per_group, n_groups - 1);
+    const int first = grp * G;
+    const int gh = min(G, BH - first);  // heads in this group
+    const int i = k - grp * per_group;
+    w.bh = first + i % gh;
+    qg = a.n_cta_q - 1 - i / gh;
+  }
   w.b = w.bh / a.H;
   w.h = w.bh - w.b * a.H;
   w.fb_slice = (a.fac_B > 1 ? w.b : 0) * a.fac_H + (a.fac_H > 1 ? w.h : 0);
@@ -463,7 +483,7 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
       mbar_arrive(&ctrl->item_full[0]);
     }
     for (int p = 0; ok && cur >= 0; ++p) {
-      const WorkItem w = make_item<QT>(cur, args);
+      const WorkItem w = make_item<QT, (DP == 128)>(cur, args);
       // Q and phi_q of the item, once the previous item's last S MMAs are done.
       if (it > 0 && !(ok = mbar_wait(&ctrl->q_empty, uint32_t(it - 1) & 1u, abort))) break;
       uint32_t qbytes = 0;
@@ -529,7 +549,7 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
         // its Q and phi_q tiles go to L2 now, so their load at the item
         // change waits for L2, not HBM
         if (nxt >= 0) {
-          const WorkItem w2 = make_item<QT>(nxt, args);
+          const WorkItem w2 = make_item<QT, (DP == 128)>(nxt, args);
           for (int t = 0; t < QT; ++t) {
             if (w2.nk[t] == 0) continue;
             for (int ch = 0; ch < C::NDCH; ++ch) tma_prefetch_l2_3d(&tm_q, ch * C::DCH, w2.q0[t], w2.bh);
@@ -620,7 +640,7 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
       for (int p = 0; ok; ++p) {
         const int k = read_item(ctrl->item_full, ctrl->item_empty, ctrl->item, p, abort, ok);
         if (k < 0) break;
-        const WorkItem w = make_item<QT>(k, args);
+        const WorkItem w = make_item<QT, (DP == 128)>(k, args);
         const int n = w.n_steps;
         if (hh == 0) {
           if (!(ok = mbar_wait(&ctrl->q_full, uint32_t(it) & 1u, abort))) break;
@@ -687,7 +707,7 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
       for (int p = 0; ok; ++p) {
         const int k = read_item(ctrl->item_full, ctrl->item_empty, ctrl->item, p, abort, ok);
         if (k < 0) break;
-        const WorkItem w = make_item<QT>(k, args);
+        const WorkItem w = make_item<QT, (DP == 128)>(k, args);
         const int nk_t = pick(w.nk, t), first_t = pick(w.first, t);
         if (!(ok = mbar_wait(&ctrl->q_full, uint32_t(it) & 1u, abort))) break;
         tc_fence_after();
@@ -751,7 +771,7 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
       for (int p = 0; ok; ++p) {
         const int k = read_item(ctrl->item_full, ctrl->item_empty, ctrl->item, p, abort, ok);
         if (k < 0) break;
-        const WorkItem w = make_item<QT>(k, args);
+        const WorkItem w = make_item<QT, (DP == 128)>(k, args);
         auto act = [&](int t, int i) { return t < QT && i >= w.first[t] && i < w.n_steps; };
         if (!(ok = mbar_wait(&ctrl->q_full, uint32_t(it) & 1u, abort))) break;
         tc_fence_after();
@@ -851,7 +871,7 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
       for (int p = 0; ok; ++p) {
         const int k = read_item(ctrl->item_full, ctrl->item_empty, ctrl->item, p, abort, ok);
         if (k < 0) break;
-        const WorkItem w = make_item<QT>(k, args);
+        const WorkItem w = make_item<QT, (DP == 128)>(k, args);
         const int q0 = w.q0[0], n = w.n_steps;
         const int row = q0 + r_loc;
         float m_use = -INFINITY, l_sum = 0.f;
@@ -1045,7 +1065,7 @@ __global__ void __launch_bounds__(Sm100Cfg<DP, RP, MODE, QT>::THREADS, Sm100Cfg<
       for (int p = 0; ok; ++p) {
         const int k = read_item(ctrl->item_full, ctrl->item_empty, ctrl->item, p, abort, ok);
         if (k < 0) break;
-        const WorkItem w = make_item<QT>(k, args);
+        const WorkItem w = make_item<QT, (DP == 128)>(k, args);
         const int q0_t = pick(w.q0, t), nk_t = pick(w.nk, t), first_t = pick(w.first, t);
         const int row = q0_t + r_loc;
         float m_use = -INFINITY, l_sum = 0.f;

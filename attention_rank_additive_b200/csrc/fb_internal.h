@@ -36,6 +36,7 @@ struct FwdArgs {
   int bias_B, bias_H;     // dense bias slices, same convention
   int *flags;             // device flag word
   unsigned int *sched;    // work counter [2] (zero at launch), or null: a fixed item order
+  int head_group;         // work items are numbered in groups of this many heads (B*H: one group)
 };
 
 // Launch description chosen by the host for one call.
