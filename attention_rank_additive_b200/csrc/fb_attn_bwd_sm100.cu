@@ -15,7 +15,10 @@
 // forward's P; the gradient products run in bf16 with fp32 accumulation, the
 // factors entering them as bf16 copies.
 //
-// Two kernels, no atomics:
+// At head dim 64 (fixed factors, or 33 <= R <= 64) one persistent kernel,
+// attn_bwd_fused_sm100 (below), computes every gradient of a 128-key tile and
+// adds each query block's dQ and dphi_q into an fp32 accumulator with TMA
+// reduce-adds. Otherwise two kernels, no atomics:
 //   attn_bwd_dkdv_sm100  one CTA per (b, h, 128-key tile). The key tile K|phi_k
 //       and V stay in shared memory; query blocks of BQ rows (64, or 32 at
 //       head dim 128 so that TMEM holds everything) stream through a ring.
@@ -26,18 +29,18 @@
 //   attn_bwd_dq_sm100    one CTA per (b, h, 128-query tile), key blocks of 64:
 //       S = Q K^T (+ ...), dP = dO V^T, dS over S in TMEM, dQ += dS K,
 //       dphi_q += dS phi_k.
-// In both, two compute warpgroups take alternate blocks, each with its own
-// S and dP buffers in TMEM (ping-pong): while one turns its scores into P and
-// dS, the tensor core runs the other's products.
+// In all of them, two compute warpgroups take alternate blocks, each with its
+// own S and dP buffers in TMEM (ping-pong): while one turns its scores into P
+// and dS, the tensor core runs the other's products.
 // The factor gradients of a broadcast factor (stride 0) sum over the heads
 // and batches sharing it: each head writes its rows to per-head partials and
 // a reduction over the sharing heads follows; a per-head factor gets its rows
-// written directly. No atomics anywhere.
+// written directly.
 //
-// CTA: warps 0-7 compute (two warpgroups, one thread per TMEM lane = tile
-// row in each), warp 8 TMA producer, warp 9 TMEM allocator and MMA issuer.
-// Every wait is bounded (the abort flag and the device flag word report a
-// timeout).
+// Two-kernel CTA: warps 0-7 compute (two warpgroups, one thread per TMEM lane
+// = tile row in each), warp 8 TMA producer, warp 9 TMEM allocator and MMA
+// issuer. Every wait is bounded (the abort flag and the device flag word
+// report a timeout).
 #include <algorithm>
 #include <atomic>
 
