@@ -273,29 +273,45 @@ __global__ void __launch_bounds__(64 * TW / 16) neural_prep_mma_kernel(
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) aq[i][j] = ak[i][j] = 0.f;
+  // each thread's share of a stage: all of its loads are issued before its
+  // shared-memory stores, so a stage costs one memory latency, not one per
+  // element
+  constexpr int XK = 64 * FC / NT, WK = FC * TW / NT;
+  static_assert(XK * NT == 64 * FC && WK * NT == FC * TW, "staging split");
   for (int f0 = 0; f0 < F; f0 += FC) {
     const int fc = min(FC, F - f0);
-    for (int e = threadIdx.x; e < 64 * FC; e += NT) {
+    float xv[2][XK], wv[2][WK];
+#pragma unroll
+    for (int u = 0; u < XK; ++u) {
+      const int e = int(threadIdx.x) + u * NT;
       const int rr = e / FC, f = e - rr * FC;  // consecutive threads: consecutive features of one row
       const long long n = n0 + rr;
-      float vq = 0.f, vk = 0.f;
-      if (n < N && f < fc) {
-        vq = Xq[((long long)b * N + n) * F + f0 + f];
-        vk = Xk[((long long)b * N + n) * F + f0 + f];
-      }
-      xs[0][f][rr] = vq;
-      xs[1][f][rr] = vk;
+      const bool in = n < N && f < fc;
+      xv[0][u] = in ? Xq[((long long)b * N + n) * F + f0 + f] : 0.f;
+      xv[1][u] = in ? Xk[((long long)b * N + n) * F + f0 + f] : 0.f;
     }
-    for (int e = threadIdx.x; e < FC * TW; e += NT) {
+#pragma unroll
+    for (int u = 0; u < WK; ++u) {
+      const int e = int(threadIdx.x) + u * NT;
       const int f = e / TW, c = e - f * TW;
       const int r = c0 + c;
-      float vq = 0.f, vk = 0.f;
-      if (f < fc && r < R) {
-        vq = Wq[((long long)h * F + f0 + f) * R + r];
-        vk = Wk[((long long)h * F + f0 + f) * R + r];
-      }
-      ws[0][f][c] = vq;
-      ws[1][f][c] = vk;
+      const bool in = f < fc && r < R;
+      wv[0][u] = in ? Wq[((long long)h * F + f0 + f) * R + r] : 0.f;
+      wv[1][u] = in ? Wk[((long long)h * F + f0 + f) * R + r] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < XK; ++u) {
+      const int e = int(threadIdx.x) + u * NT;
+      const int rr = e / FC, f = e - rr * FC;
+      xs[0][f][rr] = xv[0][u];
+      xs[1][f][rr] = xv[1][u];
+    }
+#pragma unroll
+    for (int u = 0; u < WK; ++u) {
+      const int e = int(threadIdx.x) + u * NT;
+      const int f = e / TW, c = e - f * TW;
+      ws[0][f][c] = wv[0][u];
+      ws[1][f][c] = wv[1][u];
     }
     __syncthreads();
     for (int f = 0; f < fc; ++f) {
